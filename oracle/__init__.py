@@ -1,0 +1,230 @@
+"""Float64 CPU oracle for online log-domain Sinkhorn -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product path (the CUDA library in
+``log_domain_sinkhorn_online_b200``) never does, and this package imports
+nothing from it.
+
+The arithmetic lives in ``sinkhorn_oracle.c`` (plain C, float64, OpenMP over
+rows); this module compiles it with gcc on first use and wraps each entry
+point with ctypes + numpy. Every function states what it computes and the
+page it follows; see the C file's header for the readings taken where the
+pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sinkhorn_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+SCALE_NONE, SCALE_MEAN, SCALE_MAX_COST, SCALE_VALUE = 0, 1, 2, 3
+_SCALE_NAMES = {"none": SCALE_NONE, "mean": SCALE_MEAN, "max_cost": SCALE_MAX_COST}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (gcc -O2, no fast-math, OpenMP) into oracle/_build."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64, I32, D = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+            lib.orc_num_threads.restype = I32
+            lib.orc_inv_scale_cost.argtypes = [P, P, I64, I64, I32, I32, D]
+            lib.orc_inv_scale_cost.restype = D
+            lib.orc_f_step.argtypes = [P, P, P, P, I64, I64, I32, D, D, P, I64, P]
+            lib.orc_g_step.argtypes = [P, P, P, P, I64, I64, I32, D, D, P, I64, P]
+            lib.orc_marginal_residual.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D,
+                                                  P, P, P, P]
+            lib.orc_sinkhorn.argtypes = [P, P, P, P, I64, I64, I32, D, D, I32, D, P, P, P]
+            lib.orc_sinkhorn.restype = I32
+            lib.orc_sinkhorn_anneal.argtypes = [P, P, P, P, I64, I64, I32, D, D, D, D, I32,
+                                                P, P, P]
+            lib.orc_sinkhorn_anneal.restype = I32
+            lib.orc_materialize_rows.argtypes = [P, P, P, P, I64, I64, I32, D, D, P, I64, P]
+            lib.orc_dense_plan.argtypes = [P, P, P, P, I64, I64, I32, D, D, P]
+            lib.orc_min_row.argtypes = [P, P, P, P, P, I64, I64, I32, D, D, I64, P, P, P, P]
+            lib.orc_min_row.restype = I64
+            _lib = lib
+    return _lib
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _pts(x, y):
+    x, y = _f32(x), _f32(y)
+    if x.ndim == 1:
+        x = x[:, None]
+    if y.ndim == 1:
+        y = y[:, None]
+    assert x.shape[1] == y.shape[1]
+    return x, y, x.shape[0], y.shape[0], x.shape[1]
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses."""
+    return int(_load().orc_num_threads())
+
+
+def inv_scale_cost(x, y, scale="none", value=None) -> float:
+    """c such that the cost used is C_ij = c * ||x_i - y_j||^2.
+
+    "none" -> 1; "mean" -> 1 / mean over all n*m pairs (brute force);
+    "max_cost" -> 1 / max over all pairs; a number v -> 1 / v. The parent
+    problem's c is resolved once and reused for every row subset (moscot
+    PR #846, section "Fix").
+    """
+    x, y, n, m, d = _pts(x, y)
+    if isinstance(scale, str):
+        mode, val = _SCALE_NAMES[scale], 0.0
+    else:
+        mode, val = SCALE_VALUE, float(scale if value is None else value)
+    return float(_load().orc_inv_scale_cost(_ptr(x), _ptr(y), n, m, d, mode, val))
+
+
+def f_step(x, y, a, g, c, eps, rows=None):
+    """f_i = eps ln a_i - eps LSE_j((g_j - C_ij)/eps) (FlashSinkhorn 2, section 2.1).
+
+    rows: optional int64 indices; then only those rows are returned.
+    """
+    x, y, n, m, d = _pts(x, y)
+    a, g = _f64(a), _f64(g)
+    if rows is None:
+        out = np.empty(n)
+        _load().orc_f_step(_ptr(x), _ptr(y), _ptr(a), _ptr(g), n, m, d, c, eps, None, 0,
+                           _ptr(out))
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        out = np.empty(rows.shape[0])
+        _load().orc_f_step(_ptr(x), _ptr(y), _ptr(a), _ptr(g), n, m, d, c, eps, _ptr(rows),
+                           rows.shape[0], _ptr(out))
+    return out
+
+
+def g_step(x, y, b, f, c, eps, cols=None):
+    """g_j = eps ln b_j - eps LSE_i((f_i - C_ij)/eps) (FlashSinkhorn 2, section 2.1)."""
+    x, y, n, m, d = _pts(x, y)
+    b, f = _f64(b), _f64(f)
+    if cols is None:
+        out = np.empty(m)
+        _load().orc_g_step(_ptr(x), _ptr(y), _ptr(b), _ptr(f), n, m, d, c, eps, None, 0,
+                           _ptr(out))
+    else:
+        cols = np.ascontiguousarray(cols, dtype=np.int64)
+        out = np.empty(cols.shape[0])
+        _load().orc_g_step(_ptr(x), _ptr(y), _ptr(b), _ptr(f), n, m, d, c, eps, _ptr(cols),
+                           cols.shape[0], _ptr(out))
+    return out
+
+
+def sinkhorn(x, y, a, b, c, eps, n_iters, tol=0.0, f0=None, g0=None):
+    """Alternating f/g updates from f=g=0 (or f0/g0).
+
+    Returns (f, g, iterations, row_residual_of_returned_state). With tol > 0
+    it stops after the first iteration whose ||T1 - a||_1 <= tol.
+    """
+    x, y, n, m, d = _pts(x, y)
+    a, b = _f64(a), _f64(b)
+    f = np.zeros(n) if f0 is None else _f64(f0).copy()
+    g = np.zeros(m) if g0 is None else _f64(g0).copy()
+    r = ctypes.c_double(0.0)
+    it = _load().orc_sinkhorn(_ptr(x), _ptr(y), _ptr(a), _ptr(b), n, m, d, c, eps,
+                              int(n_iters), float(tol), _ptr(f), _ptr(g), ctypes.byref(r))
+    return f, g, int(it), float(r.value)
+
+
+def sinkhorn_anneal(x, y, a, b, c, eps_target, eps_init=1.0, decay=0.7, iters_per_stage=20,
+                    f0=None, g0=None):
+    """eps-annealing: stage k at max(eps_target, eps_init*decay**k), carried potentials.
+
+    Returns (f, g, stages, row_residual).
+    """
+    x, y, n, m, d = _pts(x, y)
+    a, b = _f64(a), _f64(b)
+    f = np.zeros(n) if f0 is None else _f64(f0).copy()
+    g = np.zeros(m) if g0 is None else _f64(g0).copy()
+    r = ctypes.c_double(0.0)
+    k = _load().orc_sinkhorn_anneal(_ptr(x), _ptr(y), _ptr(a), _ptr(b), n, m, d, c,
+                                    float(eps_target), float(eps_init), float(decay),
+                                    int(iters_per_stage), _ptr(f), _ptr(g), ctypes.byref(r))
+    return f, g, int(k), float(r.value)
+
+
+def marginal_residual(x, y, a, b, f, g, c, eps, return_sums=False):
+    """(||T1 - a||_1, ||T^T 1 - b||_1) with T_ij = exp((f_i+g_j-C_ij)/eps)."""
+    x, y, n, m, d = _pts(x, y)
+    a, b, f, g = _f64(a), _f64(b), _f64(f), _f64(g)
+    r, q = ctypes.c_double(), ctypes.c_double()
+    rs, cs = (np.empty(n), np.empty(m)) if return_sums else (None, None)
+    _load().orc_marginal_residual(_ptr(x), _ptr(y), _ptr(a), _ptr(b), _ptr(f), _ptr(g), n, m,
+                                  d, c, eps, ctypes.byref(r), ctypes.byref(q), _ptr(rs),
+                                  _ptr(cs))
+    if return_sums:
+        return float(r.value), float(q.value), rs, cs
+    return float(r.value), float(q.value)
+
+
+def materialize_rows(x, y, f, g, c, eps, row_idx):
+    """T[row_idx, :] with T_ij = exp((f_i + g_j - C_ij)/eps) (moscot PR #846, "Fix")."""
+    x, y, n, m, d = _pts(x, y)
+    f, g = _f64(f), _f64(g)
+    row_idx = np.ascontiguousarray(row_idx, dtype=np.int64)
+    out = np.empty((row_idx.shape[0], m))
+    _load().orc_materialize_rows(_ptr(x), _ptr(y), _ptr(f), _ptr(g), n, m, d, c, eps,
+                                 _ptr(row_idx), row_idx.shape[0], _ptr(out))
+    return out
+
+
+def dense_plan(x, y, f, g, c, eps):
+    """The full n x m plan (small inputs only)."""
+    x, y, n, m, d = _pts(x, y)
+    f, g = _f64(f), _f64(g)
+    T = np.empty((n, m))
+    _load().orc_dense_plan(_ptr(x), _ptr(y), _ptr(f), _ptr(g), n, m, d, c, eps, _ptr(T))
+    return T
+
+
+def min_row(x, y, a, f, g, c, eps, block_rows=0):
+    """Exact min_row threshold (moscot PR #846, "Behavioural changes").
+
+    Returns dict(thr, argmin, counts[n], nnz, n_massless).
+    """
+    x, y, n, m, d = _pts(x, y)
+    a, f, g = _f64(a), _f64(f), _f64(g)
+    thr, arg, nnz = ctypes.c_double(), ctypes.c_int64(), ctypes.c_int64()
+    counts = np.empty(n, dtype=np.int64)
+    nm = _load().orc_min_row(_ptr(x), _ptr(y), _ptr(a), _ptr(f), _ptr(g), n, m, d, c, eps,
+                             int(block_rows), ctypes.byref(thr), ctypes.byref(arg),
+                             _ptr(counts), ctypes.byref(nnz))
+    return dict(thr=float(thr.value), argmin=int(arg.value), counts=counts,
+                nnz=int(nnz.value), n_massless=int(nm))

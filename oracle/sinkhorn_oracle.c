@@ -1,0 +1,344 @@
+/*
+ * sinkhorn_oracle.c -- TEST INFRASTRUCTURE, not part of the product path.
+ *
+ * A plain, slow, float64 CPU statement of what the GPU library computes:
+ * online log-domain Sinkhorn between two point clouds under squared-Euclidean
+ * cost, the transport-plan row formula, the marginal residuals and the exact
+ * min_row threshold. Only the test suite, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load this library. It shares no code,
+ * header, table or constant with the CUDA sources.
+ *
+ * Sources (the pages this follows):
+ *  - moscot PR #846, "materialize transport-matrix rows instead of pushing
+ *    indicator columns", section "Fix": the entropic plan entry
+ *    T_ij = exp((f_i + g_j - C_ij) / eps) with C from the point-cloud cost, and
+ *    the rule that the parent's resolved inv_scale_cost / eps are captured
+ *    (never re-derived from a subset).
+ *  - same page, section "Behavioural changes": min_row keeps the largest
+ *    threshold that leaves every row non-empty, min_i max_j T_ij; rows that
+ *    carry no mass keep nothing and do not take part in the threshold.
+ *  - "FlashSinkhorn 2: Block-Sparse Entropic Optimal Transport", section 2.1:
+ *    log-domain Sinkhorn alternates source and target dual-potential updates,
+ *    each a log-sum-exp reduction; the cost is computed on the fly.
+ *  - same paper, section D.3: accurate evaluation builds the cost from
+ *    coordinate differences in FP64 (this file always does).
+ *  - POT PR #868, test list: a log-sum-exp over an all -inf row is -inf.
+ *
+ * Readings where the pages are silent (each one is listed with the design):
+ *  - No a(x)b factor in the plan (plan = exp((f+g-C)/eps)), so the updates are
+ *      f_i = eps*ln(a_i) - eps*LSE_j((g_j - C_ij)/eps)
+ *      g_j = eps*ln(b_j) - eps*LSE_i((f_i - C_ij)/eps),
+ *    f first, from f = g = 0 unless a warm start is given.
+ *  - The stopping residual is ||T 1 - a||_1 of the state after a full
+ *    iteration, checked after every iteration when tol > 0.
+ *  - scale "mean"/"max" are the unweighted mean / max over all n*m pairs of
+ *    the squared distance; eps is absolute, on the scaled cost.
+ *  - A massless row (a_i == 0) has f_i = -inf.
+ *
+ * Parallelism: OpenMP over rows (or columns), each row reduced serially in
+ * index order, so results do not depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* squared Euclidean distance from coordinate differences, in float64 */
+static double sqdist(const float *p, const float *q, int d) {
+    double s = 0.0;
+    for (int k = 0; k < d; ++k) {
+        double t = (double)p[k] - (double)q[k];
+        s += t * t;
+    }
+    return s;
+}
+
+/* C_ij as used by the method: inv_scale_cost * ||x_i - y_j||^2 */
+static double cost(const float *x, const float *y, int64_t i, int64_t j, int d, double c) {
+    return c * sqdist(x + i * (int64_t)d, y + j * (int64_t)d, d);
+}
+
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------- scale --
+ * mode 0: no scaling (c = 1); 1: c = 1/mean_ij ||x_i-y_j||^2 (brute force over
+ * all pairs); 2: c = 1/max_ij ||x_i-y_j||^2; 3: c = 1/value.               */
+double orc_inv_scale_cost(const float *x, const float *y, int64_t n, int64_t m, int d,
+                          int mode, double value) {
+    if (mode == 0) return 1.0;
+    if (mode == 3) return 1.0 / value;
+    double *acc = (double *)calloc((size_t)n, sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double s = 0.0, mx = 0.0;
+        for (int64_t j = 0; j < m; ++j) {
+            double cij = cost(x, y, i, j, d, 1.0);
+            s += cij;
+            if (cij > mx) mx = cij;
+        }
+        acc[i] = (mode == 1) ? s : mx;
+    }
+    double r = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        if (mode == 1) r += acc[i];
+        else if (acc[i] > r) r = acc[i];
+    }
+    free(acc);
+    if (mode == 1) r /= ((double)n * (double)m);
+    return 1.0 / r;
+}
+
+/* ------------------------------------------------------------------ LSE --
+ * log(sum_k exp(v_k)) with the max shift; all -inf gives -inf.             */
+static double lse(const double *v, int64_t len) {
+    double mx = -INFINITY;
+    for (int64_t k = 0; k < len; ++k)
+        if (v[k] > mx) mx = v[k];
+    if (mx == -INFINITY) return -INFINITY;
+    double s = 0.0;
+    for (int64_t k = 0; k < len; ++k) s += exp(v[k] - mx);
+    return mx + log(s);
+}
+
+/* ----------------------------------------------------------- half-steps --
+ * f-update (FlashSinkhorn 2, section 2.1; source potential first):
+ *   f_i = eps*ln a_i - eps*LSE_j((g_j - C_ij)/eps),   f_i = -inf if a_i == 0.
+ * rows: only the listed rows are updated when rows != NULL (used to check a
+ * sample of a large problem one row at a time).                            */
+void orc_f_step(const float *x, const float *y, const double *a, const double *g,
+                int64_t n, int64_t m, int d, double c, double eps,
+                const int64_t *rows, int64_t nrows, double *f_out) {
+    int64_t cnt = rows ? nrows : n;
+    #pragma omp parallel
+    {
+        double *v = (double *)malloc((size_t)(m > 0 ? m : 1) * sizeof(double));
+        #pragma omp for schedule(static)
+        for (int64_t r = 0; r < cnt; ++r) {
+            int64_t i = rows ? rows[r] : r;
+            double out;
+            if (a[i] == 0.0) {
+                out = -INFINITY;
+            } else {
+                for (int64_t j = 0; j < m; ++j) v[j] = (g[j] - cost(x, y, i, j, d, c)) / eps;
+                out = eps * log(a[i]) - eps * lse(v, m);
+            }
+            f_out[rows ? r : i] = out;
+        }
+        free(v);
+    }
+}
+
+/* g-update, the same reduction over the other index:
+ *   g_j = eps*ln b_j - eps*LSE_i((f_i - C_ij)/eps),   g_j = -inf if b_j == 0. */
+void orc_g_step(const float *x, const float *y, const double *b, const double *f,
+                int64_t n, int64_t m, int d, double c, double eps,
+                const int64_t *cols, int64_t ncols, double *g_out) {
+    int64_t cnt = cols ? ncols : m;
+    #pragma omp parallel
+    {
+        double *v = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+        #pragma omp for schedule(static)
+        for (int64_t r = 0; r < cnt; ++r) {
+            int64_t j = cols ? cols[r] : r;
+            double out;
+            if (b[j] == 0.0) {
+                out = -INFINITY;
+            } else {
+                for (int64_t i = 0; i < n; ++i) v[i] = (f[i] - cost(x, y, i, j, d, c)) / eps;
+                out = eps * log(b[j]) - eps * lse(v, n);
+            }
+            g_out[cols ? r : j] = out;
+        }
+        free(v);
+    }
+}
+
+/* ----------------------------------------------------------- plan entry --
+ * T_ij = exp((f_i + g_j - C_ij)/eps)  (moscot PR #846, "Fix", entropic rows). */
+static double plan_entry(const float *x, const float *y, const double *f, const double *g,
+                         int64_t i, int64_t j, int d, double c, double eps) {
+    if (f[i] == -INFINITY || g[j] == -INFINITY) return 0.0;
+    return exp((f[i] + g[j] - cost(x, y, i, j, d, c)) / eps);
+}
+
+/* ------------------------------------------------------------- residual --
+ * row_l1 = sum_i |sum_j T_ij - a_i|, col_l1 = sum_j |sum_i T_ij - b_j|;
+ * row_sums/col_sums (optional) receive the marginals of T.                  */
+void orc_marginal_residual(const float *x, const float *y, const double *a, const double *b,
+                           const double *f, const double *g, int64_t n, int64_t m, int d,
+                           double c, double eps, double *row_l1, double *col_l1,
+                           double *row_sums, double *col_sums) {
+    double *rs = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    double *cs = (double *)malloc((size_t)(m > 0 ? m : 1) * sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double s = 0.0;
+        for (int64_t j = 0; j < m; ++j) s += plan_entry(x, y, f, g, i, j, d, c, eps);
+        rs[i] = s;
+    }
+    #pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < m; ++j) {
+        double s = 0.0;
+        for (int64_t i = 0; i < n; ++i) s += plan_entry(x, y, f, g, i, j, d, c, eps);
+        cs[j] = s;
+    }
+    double r = 0.0, q = 0.0;
+    for (int64_t i = 0; i < n; ++i) r += fabs(rs[i] - a[i]);
+    for (int64_t j = 0; j < m; ++j) q += fabs(cs[j] - b[j]);
+    if (row_l1) *row_l1 = r;
+    if (col_l1) *col_l1 = q;
+    if (row_sums) memcpy(row_sums, rs, (size_t)n * sizeof(double));
+    if (col_sums) memcpy(col_sums, cs, (size_t)m * sizeof(double));
+    free(rs);
+    free(cs);
+}
+
+/* row residual only (the stopping test), ||T 1 - a||_1 */
+static double row_residual(const float *x, const float *y, const double *a, const double *f,
+                           const double *g, int64_t n, int64_t m, int d, double c, double eps) {
+    double *rs = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double s = 0.0;
+        for (int64_t j = 0; j < m; ++j) s += plan_entry(x, y, f, g, i, j, d, c, eps);
+        rs[i] = fabs(s - a[i]);
+    }
+    double r = 0.0;
+    for (int64_t i = 0; i < n; ++i) r += rs[i];
+    free(rs);
+    return r;
+}
+
+/* ------------------------------------------------------------ iterations --
+ * One iteration = f-update then g-update (FlashSinkhorn 2, section 2.1).
+ * f, g: in (warm start; zeros for a cold start) and out.
+ * n_iters is the cap; tol > 0 stops after the first iteration whose state has
+ * ||T 1 - a||_1 <= tol. Returns the number of iterations done; *resid gets the
+ * row residual of the returned state (always computed).                    */
+int orc_sinkhorn(const float *x, const float *y, const double *a, const double *b,
+                 int64_t n, int64_t m, int d, double c, double eps, int n_iters, double tol,
+                 double *f, double *g, double *resid) {
+    int it = 0;
+    double r = NAN;
+    for (it = 1; it <= n_iters; ++it) {
+        orc_f_step(x, y, a, g, n, m, d, c, eps, NULL, 0, f);
+        orc_g_step(x, y, b, f, n, m, d, c, eps, NULL, 0, g);
+        if (tol > 0.0) {
+            r = row_residual(x, y, a, f, g, n, m, d, c, eps);
+            if (r <= tol) break;
+        }
+    }
+    if (it > n_iters) it = n_iters;
+    if (tol <= 0.0 || isnan(r)) r = row_residual(x, y, a, f, g, n, m, d, c, eps);
+    if (resid) *resid = r;
+    return it;
+}
+
+/* eps-annealing driver (FlashSinkhorn 2, sections 3.1 and C.3 anneal eps and
+ * continue at the target eps; the schedule itself is this build's reading):
+ * stage k runs iters_per_stage iterations at eps_k = max(eps_target,
+ * eps_init * decay^k), potentials carried over unchanged; the last stage is
+ * the first one whose eps_k equals eps_target. Returns the number of stages;
+ * *resid is the row residual at the end.                                   */
+int orc_sinkhorn_anneal(const float *x, const float *y, const double *a, const double *b,
+                        int64_t n, int64_t m, int d, double c, double eps_target,
+                        double eps_init, double decay, int iters_per_stage,
+                        double *f, double *g, double *resid) {
+    int k = 0;
+    for (;; ++k) {
+        double ek = eps_init * pow(decay, (double)k);
+        if (ek < eps_target) ek = eps_target;
+        double r = 0.0;
+        orc_sinkhorn(x, y, a, b, n, m, d, c, ek, iters_per_stage, 0.0, f, g, &r);
+        if (ek == eps_target) {
+            if (resid) *resid = r;
+            break;
+        }
+    }
+    return k + 1;
+}
+
+/* --------------------------------------------------------- materializer --
+ * out[r*m + j] = T_{row_idx[r], j}  (moscot PR #846, "Fix": rows built from
+ * the potentials and the captured inv_scale_cost/eps, O(k*m) memory).      */
+void orc_materialize_rows(const float *x, const float *y, const double *f, const double *g,
+                          int64_t n, int64_t m, int d, double c, double eps,
+                          const int64_t *row_idx, int64_t k, double *out) {
+    (void)n;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < k; ++r) {
+        int64_t i = row_idx[r];
+        for (int64_t j = 0; j < m; ++j)
+            out[r * m + j] = plan_entry(x, y, f, g, i, j, d, c, eps);
+    }
+}
+
+/* the full n x m plan, entry by entry (used only on small inputs) */
+void orc_dense_plan(const float *x, const float *y, const double *f, const double *g,
+                    int64_t n, int64_t m, int d, double c, double eps, double *T) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < m; ++j)
+            T[i * m + j] = plan_entry(x, y, f, g, i, j, d, c, eps);
+}
+
+/* --------------------------------------------------------------- min_row --
+ * moscot PR #846, "Behavioural changes": thr = min over rows carrying mass of
+ * max_j T_ij; entries with T_ij >= thr are kept; massless rows (a_i == 0) keep
+ * nothing and are excluded from the min. The rows are visited in blocks of
+ * block_rows, which must not change any result. counts (optional, [n]) gets
+ * the kept entries per row. Returns the number of massless rows; *thr_out is
+ * +inf when every row is massless; *argmin_out is the row attaining thr
+ * (smallest index on ties).                                                 */
+int64_t orc_min_row(const float *x, const float *y, const double *a, const double *f,
+                    const double *g, int64_t n, int64_t m, int d, double c, double eps,
+                    int64_t block_rows, double *thr_out, int64_t *argmin_out,
+                    int64_t *counts, int64_t *nnz_out) {
+    double *rowmax = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    if (block_rows <= 0) block_rows = n > 0 ? n : 1;
+    for (int64_t r0 = 0; r0 < n; r0 += block_rows) {
+        int64_t r1 = r0 + block_rows < n ? r0 + block_rows : n;
+        #pragma omp parallel for schedule(static)
+        for (int64_t i = r0; i < r1; ++i) {
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < m; ++j) {
+                double t = plan_entry(x, y, f, g, i, j, d, c, eps);
+                if (t > mx) mx = t;
+            }
+            rowmax[i] = mx;
+        }
+    }
+    double thr = INFINITY;
+    int64_t arg = -1, massless = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        if (a[i] == 0.0) { ++massless; continue; }
+        if (rowmax[i] < thr) { thr = rowmax[i]; arg = i; }
+    }
+    int64_t nnz = 0;
+    for (int64_t r0 = 0; r0 < n; r0 += block_rows) {
+        int64_t r1 = r0 + block_rows < n ? r0 + block_rows : n;
+        #pragma omp parallel for schedule(static) reduction(+ : nnz)
+        for (int64_t i = r0; i < r1; ++i) {
+            int64_t cnt = 0;
+            if (a[i] != 0.0)
+                for (int64_t j = 0; j < m; ++j)
+                    if (plan_entry(x, y, f, g, i, j, d, c, eps) >= thr) ++cnt;
+            if (counts) counts[i] = cnt;
+            nnz += cnt;
+        }
+    }
+    free(rowmax);
+    if (thr_out) *thr_out = thr;
+    if (argmin_out) *argmin_out = arg;
+    if (nnz_out) *nnz_out = nnz;
+    return massless;
+}
