@@ -1,0 +1,330 @@
+"""Benchmark of the online log-domain Sinkhorn hot path on B200.
+
+One step = the whole path on the 8000 x 8000, d = 3 Gaussian-mixture workload
+(scale "mean", eps 0.01): the solve to ||T1 - a||_1 <= 1e-3 (cap 2000, fused
+f/g half-steps with the in-loop residual), the float64-assembled marginal
+residual at the returned potentials, the exact min_row threshold and per-row
+counts in row blocks of 1024, and the materialisation of every row in blocks of
+1024. Inputs are resident in HBM before the timed region; L2 is flushed before
+every step. The metric counts Sinkhorn pair-updates (n*m per half-step) per
+second; the row passes are inside the timed step but add no units.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload w2]
+
+Under torchrun (N > 1) every rank solves its own replica (no collective on the
+data path); rank 0 prints the JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Sinkhorn pair-updates/s (n·m per half-step) and % of ex2/MUFU roofline"
+UNIT = "pair-updates/s"
+# MUFU ex2 peak: 148 SMs x 16 ex2 per clock per SM x 1.965 GHz (max SM clock)
+SMS, EX2_PER_CLK = 148, 16
+# DRAM traffic of one half-step launch from the committed ncu capture (bytes), or None
+HALFSTEP_TRAFFIC = None
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="w2", choices=["w1", "w2", "w3", "w4", "w5"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _workload(name):
+    from log_domain_sinkhorn_online_b200 import workloads
+    return workloads.ALL[name]()
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.path = index, None, None
+
+    def start(self):
+        import tempfile
+        self.path = tempfile.mktemp(suffix=".csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows if len(r) >= 9 for k in range(4)
+                          if r[5 + k].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _dist_init(n_gpus):
+    import torch
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, None
+    import datetime
+    import torch.distributed as dist
+    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    return rank, world, dist
+
+
+def _max_over_ranks(v, dist):
+    import torch
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def _solve_kwargs(w):
+    kw = dict(eps=w.eps, scale=w.scale, n_iters=w.n_iters, tol=w.tol)
+    if w.anneal:
+        kw.update(eps_init=w.anneal["eps_init"], eps_decay=w.anneal["decay"],
+                  iters_per_stage=w.anneal["iters_per_stage"])
+    return kw
+
+
+class Step:
+    """The whole hot path on one workload, device-resident buffers reused across steps."""
+
+    def __init__(self, ot, w, dev):
+        import torch
+        self.ot, self.w, self.dev = ot, w, dev
+        self.x, self.y, self.a, self.b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev)
+                                          for v in (w.x, w.y, w.a, w.b))
+        self.f = torch.empty(w.n, dtype=torch.float32, device=dev)
+        self.g = torch.empty(w.m, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(w.n, dtype=torch.int64, device=dev)
+        self.block = w.block_rows if w.block_rows else 1024
+        rows = w.rows if w.rows is not None else (np.arange(w.n, dtype=np.int64) if w.block_rows else None)
+        self.rows = None if rows is None else torch.from_numpy(rows).to(dev)
+        self.out = None if rows is None else torch.empty((min(self.block, len(rows)), w.m),
+                                                         dtype=torch.float32, device=dev)
+
+    def __call__(self, timing=False):
+        w = self.w
+        plan = self.ot.sinkhorn(self.x, self.y, self.a, self.b, f=self.f, g=self.g, timing=timing,
+                                **_solve_kwargs(w))
+        launches = plan.info.kernel_launches
+        plan.marginal_residual()
+        launches += 6
+        mr = plan.sparsify_min_row(block_rows=w.block_rows, counts=self.counts)
+        nb = -(-w.n // (w.block_rows or w.n))
+        launches += 1 + 2 * nb + 2
+        if self.rows is not None:
+            for r0 in range(0, self.rows.numel(), self.block):
+                r = self.rows[r0:r0 + self.block]
+                plan.materialize_rows(r, out=self.out[:r.numel()])
+                launches += 2
+        info = plan.info
+        plan.close()
+        return info, mr, launches
+
+
+def _flush_l2(buf):
+    buf.zero_()
+
+
+def _cpu_baseline(w, target_s=10.0):
+    """The float64 oracle (as it stands) on a bounded row sample of the f-half-step."""
+    import oracle
+    oracle.build()
+    c = 1.0  # the arithmetic per pair does not depend on the scale value
+    g = np.zeros(w.m)
+    probe = min(w.n, 64)
+    t0 = time.perf_counter()
+    oracle.f_step(w.x, w.y, w.a, g, c, w.eps, rows=np.arange(probe))
+    rate = probe * w.m / max(time.perf_counter() - t0, 1e-6)
+    rows = int(max(probe, min(w.n, rate * target_s / w.m)))
+    idx = np.linspace(0, w.n - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.f_step(w.x, w.y, w.a, g, c, w.eps, rows=idx)
+    dt = time.perf_counter() - t0
+    return {"value": rows * w.m / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"one f-half-step on {rows} of {w.n} rows x all {w.m} columns "
+                      f"(float64 C, OpenMP), {dt:.1f} s"}
+
+
+def _config(w, world, info=None):
+    cfg = {"workload": w.name, "n": w.n, "m": w.m, "d": w.d, "eps": w.eps, "scale": w.scale,
+           "tol": w.tol, "cap": w.n_iters, "block_rows": w.block_rows,
+           "l2": "flushed (512 MiB write) before every step",
+           "parallelism": "replicas" if world > 1 else "single-gpu"}
+    if w.anneal:
+        cfg["anneal"] = w.anneal
+    if info is not None:
+        cfg["iterations"] = int(info.iterations)
+        cfg["half_steps"] = int(info.half_steps)
+        cfg["col_splits"] = int(info.col_splits)
+    return cfg
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: bounded row samples of one half-step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = _workload(args.workload)
+    times, units = [], 0
+    for it in range(args.warmup + args.steps):
+        cb = _cpu_baseline(w, target_s=8.0)
+        if it >= args.warmup:
+            times.append(cb)
+    value = statistics.mean(t["value"] for t in times)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": _config(w, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": times[0]["cores"], "kind": "oracle",
+                             "sample": times[0]["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import log_domain_sinkhorn_online_b200 as ot
+    rank, world, dist = _dist_init(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = _workload(args.workload)
+    step = Step(ot, w, dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region
+    clocks = Clocks(torch.cuda.current_device())
+    _barrier(dist)
+    clocks.start()
+    total_ms, loop_ms, half_steps, launches, info = 0.0, 0.0, 0, 0, None
+    for _ in range(args.steps):
+        _flush_l2(flush)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        info, mr, nl = step(timing=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total_ms += e0.elapsed_time(e1)
+        loop_ms += info.loop_ms
+        half_steps += info.half_steps
+        launches += nl
+    clk = clocks.stop()
+    _barrier(dist)
+    total_ms = _max_over_ranks(total_ms, dist)
+    units = float(w.n) * float(w.m) * half_steps / args.steps  # pair-updates per step (this rank)
+    value = units * world / (total_ms / args.steps / 1e3)
+
+    # ---- end to end through the public API: pinned host inputs in, results out
+    host = [torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for v in (w.x, w.y, w.a, w.b)]
+    outs = [torch.empty(w.n, dtype=torch.float32).pin_memory(), torch.empty(w.m, dtype=torch.float32).pin_memory(),
+            torch.empty(w.n, dtype=torch.int64).pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    e2e_ms, e2e_units = 0.0, 0.0
+    _barrier(dist)
+    for _ in range(args.steps):
+        _flush_l2(flush)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for dst, src in zip((step.x, step.y, step.a, step.b), host):
+            dst.copy_(src, non_blocking=True)
+        inf, _, _ = step()
+        outs[0].copy_(step.f, non_blocking=True)
+        outs[1].copy_(step.g, non_blocking=True)
+        outs[2].copy_(step.counts, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+        e2e_units += float(w.n) * float(w.m) * inf.half_steps
+    e2e_ms = _max_over_ranks(e2e_ms, dist)
+    e2e_value = e2e_units * world / (e2e_ms / 1e3)
+
+    if rank == 0:
+        peaks, kind = _peaks()
+        sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+        peak_tex2 = SMS * EX2_PER_CLK * sm_max * 1e6 / 1e12
+        per_launch_ms = loop_ms / max(half_steps, 1)
+        achieved = float(w.n) * float(w.m) / (per_launch_ms / 1e3) / 1e12
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded point clouds; recipe in log_domain_sinkhorn_online_b200/workloads.py)",
+                "config": _config(w, world, info),
+                "roofline": {"bound": "alu", "kernel": "hs_lowd_kernel (fused f/g half-step)" if w.d <= 3
+                             else "hs_generic_kernel (fused f/g half-step)",
+                             "achieved": achieved, "peak": peak_tex2, "unit": "Tex2/s",
+                             "frac": achieved / peak_tex2, "traffic": HALFSTEP_TRAFFIC,
+                             "per_launch_us": per_launch_ms * 1e3,
+                             "peak_note": f"148 SMs x 16 MUFU ex2/clk x {sm_max:.0f} MHz ({kind} sm_max)"},
+                "clocks": clk,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = _cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+/*
+ * ot_sinkhorn.h -- C ABI of the B200 (sm_100a) online log-domain Sinkhorn library.
+ *
+ * Entropic optimal transport between two point clouds x[n,d], y[m,d] with
+ * weights a[n], b[m] under the squared-Euclidean cost
+ *     C_ij = inv_scale_cost * ||x_i - y_j||^2,
+ * solved by alternating log-domain updates of the dual potentials f[n], g[m]
+ * ("FlashSinkhorn 2: Block-Sparse Entropic Optimal Transport", section 2.1:
+ * source and target potentials are updated in turn, each update a streaming
+ * log-sum-exp over on-the-fly costs, O((n+m)d) working memory, the n x m
+ * matrix never stored):
+ *     f_i <- eps*ln a_i - eps*LSE_j((g_j - C_ij)/eps)
+ *     g_j <- eps*ln b_j - eps*LSE_i((f_i - C_ij)/eps)
+ * and the transport plan they define (moscot PR #846, "materialize
+ * transport-matrix rows instead of pushing indicator columns", section Fix):
+ *     T_ij = exp((f_i + g_j - C_ij)/eps).
+ *
+ * Conventions for every entry point:
+ *  - Arrays named as device arrays are CUDA device pointers on the current
+ *    device, owned by the caller; the library never frees them and keeps no
+ *    reference to them beyond the lifetime of a plan that was given them.
+ *  - Floating-point inputs are float32, contiguous, row-major ([n,d]: point i
+ *    at x + i*d). Indices and counts are int64.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Work is ordered after everything already queued on it, and the
+ *    results are complete on it when the call returns, unless stated otherwise.
+ *  - Every call returns an int status (OT_OK = 0, warnings > 0, errors < 0),
+ *    never aborts and never prints. ot_last_error_string() describes the last
+ *    non-OK status of the calling thread.
+ *  - No CPU fallback exists: without a usable sm_100 device every call that
+ *    computes returns OT_ERR_CUDA.
+ */
+#ifndef OT_SINKHORN_H
+#define OT_SINKHORN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OT_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define OT_API __attribute__((visibility("default")))
+#else
+#define OT_API
+#endif
+
+/* ----------------------------------------------------------- status codes */
+#define OT_OK 0
+#define OT_WARN_MASSLESS_ROWS 1   /* results valid; some a_i == 0 (moscot PR #846,
+                                     "Behavioural changes": such rows keep no
+                                     entries and do not take part in min_row) */
+#define OT_ERR_INVALID_ARG (-1)   /* bad pointer/size/eps/weights/row index */
+#define OT_ERR_OVERFLOW (-2)      /* a size product exceeds what the kernels index */
+#define OT_ERR_CUDA (-3)          /* a CUDA runtime call failed (no device, bad stream) */
+#define OT_ERR_OOM (-4)           /* workspace allocation failed */
+#define OT_ERR_NONFINITE (-5)     /* a NaN/inf input, or a potential left the finite range */
+#define OT_ERR_UNSUPPORTED (-6)   /* a valid request this build does not implement */
+
+/* ------------------------------------------------------------ cost scale
+ * The cost is scaled once, on the whole problem, and that resolved factor is
+ * captured by the plan and reused by every later call on any row subset
+ * (moscot PR #846, section Fix: re-deriving it from a subset gave 15% value
+ * error). eps is absolute and applies to the scaled cost.                 */
+typedef enum ot_scale {
+    OT_SCALE_NONE = 0,      /* inv_scale_cost = 1 */
+    OT_SCALE_MEAN = 1,      /* 1 / (mean over all n*m pairs of ||x_i - y_j||^2) */
+    OT_SCALE_MAX_COST = 2,  /* 1 / (max over all n*m pairs of ||x_i - y_j||^2) */
+    OT_SCALE_VALUE = 3      /* 1 / opt->scale_value */
+} ot_scale;
+
+/* ---------------------------------------------------------------- options
+ * Fill with ot_options_default() and change fields; NULL means defaults.   */
+typedef struct ot_options {
+    int32_t warm_start;       /* 0: start from f = g = 0; 1: f, g hold the start */
+    int32_t check_every;      /* iterations between host reads of the stop flag
+                                 (also the CUDA-graph chunk length); default 16 */
+    int32_t use_graphs;       /* 1 (default): replay the iteration loop as CUDA
+                                 graphs; 0: plain launches */
+    int32_t iters_per_stage;  /* annealing: iterations per eps stage (default 20) */
+    double scale_value;       /* divisor for OT_SCALE_VALUE */
+    double eps_init;          /* > 0 enables eps-annealing: stage k runs at
+                                 max(eps, eps_init * eps_decay^k); the last stage
+                                 is the first at eps (FlashSinkhorn 2, sections
+                                 3.1 and C.3 anneal eps and continue at the
+                                 target). 0 (default): no annealing */
+    double eps_decay;         /* in (0, 1); default 0.7 */
+    int32_t timing;           /* 1: time the iteration loop with CUDA events on the
+                                 internal stream (ot_info.loop_ms); default 0 */
+    int32_t reserved0;
+} ot_options;
+
+/* -------------------------------------------------------- solve report   */
+typedef struct ot_info {
+    int32_t iterations;        /* iterations of the returned state (all stages) */
+    int32_t converged;         /* 1 if the tol test stopped the loop */
+    int32_t stages;            /* eps stages run (1 without annealing) */
+    int32_t col_splits;        /* launch shape of the f half-step: column splits */
+    double residual;           /* ||T 1 - a||_1 of the returned state, measured in
+                                  the loop from the next f-update (float32 LSE) */
+    double inv_scale_cost;     /* resolved scale factor, captured by the plan */
+    double eps;                /* resolved (final) eps, captured by the plan */
+    int64_t n_massless_rows;   /* number of a_i == 0 */
+    int64_t n_massless_cols;   /* number of b_j == 0 */
+    int64_t half_steps;        /* half-step launches that did work (2 per iteration,
+                                  plus the f-update that measures the final residual) */
+    int64_t kernel_launches;   /* kernels this call launched (graph nodes included) */
+    double loop_ms;            /* device time of the iteration loop, from CUDA events
+                                  around each chunk (opt->timing), else 0 */
+} ot_info;
+
+/* Opaque plan: the pages' "row materializer built once", which captures the
+ * resolved eps and inv_scale_cost (moscot PR #846, section Fix). It borrows
+ * x, y, a, b, f, g (read again by every later call, so they must stay alive
+ * and unchanged) and owns its device workspace.                            */
+typedef struct ot_plan ot_plan;
+
+/* ABI version (OT_ABI_VERSION of the build). */
+OT_API int ot_version(void);
+
+/* Human-readable description of the calling thread's last non-OK status. */
+OT_API const char *ot_last_error_string(void);
+
+/* Default options (warm_start 0, check_every 16, use_graphs 1,
+ * iters_per_stage 20, scale_value 1, eps_init 0, eps_decay 0.7, timing 0). */
+OT_API void ot_options_default(ot_options *opt);
+
+/* ------------------------------------------------- ot_sinkhorn_pointcloud
+ * Solves the problem above on one GPU.
+ *  x [n,d], y [m,d], a [n], b [m]: device, float32. Weights must be finite and
+ *      >= 0 with positive sums; they are not renormalised. 1 <= d <= 64.
+ *  eps > 0: entropic regularisation on the scaled cost (the final eps when
+ *      annealing).
+ *  scale_cost: see ot_scale.
+ *  n_iters >= 0: iteration cap (one iteration = f-update then g-update; the
+ *      f-update comes first, from f = g = 0 unless opt->warm_start).
+ *      n_iters == 0 runs nothing and builds a plan at the given f, g (which
+ *      must then be a warm start), e.g. to materialise rows of a known plan.
+ *  tol: if > 0, stop after the first iteration whose ||T 1 - a||_1 <= tol;
+ *      if <= 0, run exactly n_iters iterations. Missing tol is not an error.
+ *  f [n], g [m]: device float32 outputs (and inputs for a warm start). A
+ *      massless row/column gets -inf.
+ *  plan_out: if non-NULL, receives a plan to pass to the calls below; free it
+ *      with ot_plan_destroy. If NULL, the workspace is freed before returning.
+ *  info: if non-NULL, receives the report.
+ * Returns OT_OK, OT_WARN_MASSLESS_ROWS, or an error (then *plan_out = NULL and
+ * f, g are unspecified). Synchronises `stream` (it reads scalars back). */
+OT_API int ot_sinkhorn_pointcloud(const float *x, const float *y, const float *a, const float *b,
+                           int64_t n, int64_t m, int32_t d, float eps, ot_scale scale_cost,
+                           int32_t n_iters, float tol, float *f, float *g, void *stream,
+                           const ot_options *opt, ot_plan **plan_out, ot_info *info);
+
+/* ---------------------------------------------------- ot_marginal_residual
+ * row_l1 = sum_i |sum_j T_ij - a_i|, col_l1 = sum_j |sum_i T_ij - b_j| at the
+ * plan's current f, g (FlashSinkhorn 2, sections 3.1 and C.4: the residual is
+ * evaluated at the returned potentials; section D.3: the exponent is built in
+ * float64 from the coordinates). Each T_ij: float64 exponent, float32 exp.
+ * Deterministic (fixed reduction order). row_l1/col_l1: host pointers, either
+ * may be NULL. Synchronises `stream`. */
+OT_API int ot_marginal_residual(const ot_plan *plan, double *row_l1, double *col_l1, void *stream);
+
+/* ------------------------------------------------------ ot_materialize_rows
+ * out[r*m + j] = T_{row_idx[r], j} for r < k, j < m (moscot PR #846, section
+ * Fix: entropic rows exp((f_i + g_j - C_ij)/eps) with the captured scale and
+ * eps; O(k*m) memory). row_idx [k]: device int64, each in [0, n) (repeats
+ * allowed); out [k,m]: device float32, row-major. The exponent is assembled
+ * in float64; the value is rounded to float32. A row index out of range makes
+ * the call return OT_ERR_INVALID_ARG (checked on the device, no fault); the
+ * rows with valid indices are still written. Synchronises `stream`. */
+OT_API int ot_materialize_rows(const ot_plan *plan, const int64_t *row_idx, int64_t k, float *out,
+                        void *stream);
+
+/* ------------------------------------------------------ ot_sparsify_min_row
+ * The exact min_row threshold (moscot PR #846, "Behavioural changes"):
+ *     thr = min over rows with a_i > 0 of max_j T_ij,
+ * with every T_ij computed by the same float path as ot_materialize_rows, so
+ * that keeping T_ij >= thr leaves every massful row non-empty. Massless rows
+ * (a_i == 0) keep nothing and take no part. block_rows (> 0, or 0 = all rows)
+ * only sets how many rows one launch covers; it never changes a result.
+ *  thr_out: host float (+inf if every row is massless).
+ *  row_counts: device int64 [n] or NULL: kept entries per row.
+ *  nnz_out, n_massless_out, argmin_out: host int64 or NULL (argmin_out: the
+ *      row attaining thr, smallest index on ties; -1 if none).
+ * Returns OT_WARN_MASSLESS_ROWS if any row is massless. Synchronises `stream`. */
+OT_API int ot_sparsify_min_row(const ot_plan *plan, int64_t block_rows, float *thr_out,
+                        int64_t *row_counts, int64_t *nnz_out, int64_t *n_massless_out,
+                        int64_t *argmin_out, void *stream);
+
+/* Frees the plan's workspace (NULL is a no-op). Does not touch borrowed arrays. */
+OT_API void ot_plan_destroy(ot_plan *plan);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* OT_SINKHORN_H */

@@ -1,0 +1,115 @@
+"""Online log-domain Sinkhorn for point clouds on NVIDIA B200 (sm_100a).
+
+Entropic OT between x[n,d] and y[m,d] under squared-Euclidean cost, computed
+by hand-written CUDA kernels behind the C ABI of ``include/ot_sinkhorn.h``
+("FlashSinkhorn 2: Block-Sparse Entropic Optimal Transport", section 2.1, for
+the streaming log-sum-exp half-steps; moscot PR #846, section Fix, for the
+plan rows and the captured scale). PyTorch only supplies device memory and
+streams here: every step runs in the library's kernels.
+
+    import torch, log_domain_sinkhorn_online_b200 as ot
+    plan = ot.sinkhorn(x, y, a, b, eps=0.01, scale="mean", n_iters=2000, tol=1e-3)
+    rows = plan.materialize_rows(torch.arange(16, device="cuda"))
+    thr, counts, nnz = plan.sparsify_min_row(block_rows=1024)
+"""
+from __future__ import annotations
+
+from . import _binding as B
+from ._binding import OTError  # noqa: F401
+
+_SCALES = {"none": B.OT_SCALE_NONE, "mean": B.OT_SCALE_MEAN, "max_cost": B.OT_SCALE_MAX_COST}
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(t, dtype, name):
+    import torch
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+class Plan:
+    """A solved problem: potentials f, g and the captured eps / scale (owns the C plan)."""
+
+    def __init__(self, handle, x, y, a, b, f, g, info, status):
+        self._h = handle
+        self._keep = (x, y, a, b)
+        self.f, self.g, self.info, self.status = f, g, info, status
+
+    def close(self):
+        if self._h:
+            B.ot_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def handle(self):
+        return self._h
+
+    def marginal_residual(self, stream=None):
+        _, r, c = B.ot_marginal_residual(self._h, _stream(stream))
+        return r, c
+
+    def materialize_rows(self, row_idx, out=None, stream=None):
+        import torch
+        row_idx = _dev(row_idx, torch.int64, "row_idx")
+        k = row_idx.numel()
+        if out is None:
+            out = torch.empty((k, self.g.numel()), dtype=torch.float32, device=row_idx.device)
+        _dev(out, torch.float32, "out")
+        B.ot_materialize_rows(self._h, row_idx.data_ptr(), k, out.data_ptr(), _stream(stream))
+        return out
+
+    def sparsify_min_row(self, block_rows=0, counts=None, stream=None):
+        """Returns dict(thr, counts, nnz, n_massless, argmin, status)."""
+        import torch
+        if counts is None:
+            counts = torch.empty(self.f.numel(), dtype=torch.int64, device=self.f.device)
+        _dev(counts, torch.int64, "counts")
+        st, thr, nnz, nm, arg = B.ot_sparsify_min_row(self._h, int(block_rows), counts.data_ptr(),
+                                                      _stream(stream))
+        return dict(thr=thr, counts=counts, nnz=nnz, n_massless=nm, argmin=arg, status=st)
+
+
+def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None, warm_start=False,
+             check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,
+             timing=False, stream=None) -> Plan:
+    """Solves on the GPU; x [n,d], y [m,d], a [n], b [m] float32 CUDA tensors."""
+    import torch
+    x, y = _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y")
+    a, b = _dev(a, torch.float32, "a"), _dev(b, torch.float32, "b")
+    n, d = x.shape
+    m = y.shape[0]
+    f = torch.empty(n, dtype=torch.float32, device=x.device) if f is None else _dev(f, torch.float32, "f")
+    g = torch.empty(m, dtype=torch.float32, device=x.device) if g is None else _dev(g, torch.float32, "g")
+    opt = B.ot_options_default()
+    opt.warm_start = int(warm_start)
+    opt.check_every = int(check_every)
+    opt.use_graphs = int(use_graphs)
+    opt.eps_init = float(eps_init)
+    opt.eps_decay = float(eps_decay)
+    opt.iters_per_stage = int(iters_per_stage)
+    opt.timing = int(timing)
+    if isinstance(scale, str):
+        sc = _SCALES[scale]
+    else:
+        sc = B.OT_SCALE_VALUE
+        opt.scale_value = float(scale)
+    st, h, info = B.ot_sinkhorn_pointcloud(x.data_ptr(), y.data_ptr(), a.data_ptr(), b.data_ptr(),
+                                           n, m, d, float(eps), sc, int(n_iters), float(tol),
+                                           f.data_ptr(), g.data_ptr(), _stream(stream), opt)
+    return Plan(h, x, y, a, b, f, g, info, st)

@@ -1,0 +1,147 @@
+"""ctypes binding of ``include/ot_sinkhorn.h`` -- argument marshalling only.
+
+Each function has the name of the C entry point it calls and takes raw device
+pointers (ints), sizes and a stream handle (int, 0 = legacy default stream).
+No arithmetic of the method happens here. Loading fails loudly when the
+compiled library is missing: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libot_sinkhorn.so")
+_lock = threading.Lock()
+_lib = None
+
+OT_OK = 0
+OT_WARN_MASSLESS_ROWS = 1
+OT_ERR_INVALID_ARG = -1
+OT_ERR_OVERFLOW = -2
+OT_ERR_CUDA = -3
+OT_ERR_OOM = -4
+OT_ERR_NONFINITE = -5
+OT_ERR_UNSUPPORTED = -6
+
+OT_SCALE_NONE, OT_SCALE_MEAN, OT_SCALE_MAX_COST, OT_SCALE_VALUE = 0, 1, 2, 3
+
+# every symbol the header declares (checked by the CPU test suite)
+EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sinkhorn_pointcloud",
+            "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy")
+
+
+class OtOptions(ctypes.Structure):
+    _fields_ = [("warm_start", ctypes.c_int32), ("check_every", ctypes.c_int32),
+                ("use_graphs", ctypes.c_int32), ("iters_per_stage", ctypes.c_int32),
+                ("scale_value", ctypes.c_double), ("eps_init", ctypes.c_double),
+                ("eps_decay", ctypes.c_double), ("timing", ctypes.c_int32),
+                ("reserved0", ctypes.c_int32)]
+
+
+class OtInfo(ctypes.Structure):
+    _fields_ = [("iterations", ctypes.c_int32), ("converged", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("col_splits", ctypes.c_int32),
+                ("residual", ctypes.c_double), ("inv_scale_cost", ctypes.c_double),
+                ("eps", ctypes.c_double), ("n_massless_rows", ctypes.c_int64),
+                ("n_massless_cols", ctypes.c_int64), ("half_steps", ctypes.c_int64),
+                ("kernel_launches", ctypes.c_int64), ("loop_ms", ctypes.c_double)]
+
+
+class OTError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"status {status}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m log_domain_sinkhorn_online_b200.build` (there is no CPU fallback)")
+            L = ctypes.CDLL(_LIB_PATH)
+            P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+            L.ot_version.restype = ctypes.c_int
+            L.ot_last_error_string.restype = ctypes.c_char_p
+            L.ot_options_default.argtypes = [ctypes.POINTER(OtOptions)]
+            L.ot_options_default.restype = None
+            L.ot_sinkhorn_pointcloud.argtypes = [P, P, P, P, I64, I64, I32, ctypes.c_float, ctypes.c_int,
+                                                 I32, ctypes.c_float, P, P, P,
+                                                 ctypes.POINTER(OtOptions), ctypes.POINTER(P),
+                                                 ctypes.POINTER(OtInfo)]
+            L.ot_sinkhorn_pointcloud.restype = ctypes.c_int
+            L.ot_marginal_residual.argtypes = [P, ctypes.POINTER(D), ctypes.POINTER(D), P]
+            L.ot_marginal_residual.restype = ctypes.c_int
+            L.ot_materialize_rows.argtypes = [P, P, I64, P, P]
+            L.ot_materialize_rows.restype = ctypes.c_int
+            L.ot_sparsify_min_row.argtypes = [P, I64, ctypes.POINTER(ctypes.c_float), P,
+                                              ctypes.POINTER(I64), ctypes.POINTER(I64),
+                                              ctypes.POINTER(I64), P]
+            L.ot_sparsify_min_row.restype = ctypes.c_int
+            L.ot_plan_destroy.argtypes = [P]
+            L.ot_plan_destroy.restype = None
+            _lib = L
+    return _lib
+
+
+def _check(status: int) -> int:
+    if status < 0:
+        raise OTError(status, ot_last_error_string())
+    return status
+
+
+def ot_version() -> int:
+    return int(lib().ot_version())
+
+
+def ot_last_error_string() -> str:
+    return lib().ot_last_error_string().decode()
+
+
+def ot_options_default() -> OtOptions:
+    o = OtOptions()
+    lib().ot_options_default(ctypes.byref(o))
+    return o
+
+
+def ot_sinkhorn_pointcloud(x, y, a, b, n, m, d, eps, scale_cost, n_iters, tol, f, g, stream,
+                           opt: OtOptions | None = None, want_plan: bool = True):
+    """Returns (status, plan handle or None, OtInfo); raises OTError on errors."""
+    plan = ctypes.c_void_p()
+    info = OtInfo()
+    st = lib().ot_sinkhorn_pointcloud(x, y, a, b, n, m, d, eps, int(scale_cost), n_iters, tol, f, g,
+                                      stream, ctypes.byref(opt) if opt is not None else None,
+                                      ctypes.byref(plan) if want_plan else None,
+                                      ctypes.byref(info))
+    _check(st)
+    return st, (plan.value if want_plan else None), info
+
+
+def ot_marginal_residual(plan, stream):
+    """Returns (status, row_l1, col_l1)."""
+    r, c = ctypes.c_double(), ctypes.c_double()
+    st = _check(lib().ot_marginal_residual(plan, ctypes.byref(r), ctypes.byref(c), stream))
+    return st, r.value, c.value
+
+
+def ot_materialize_rows(plan, row_idx, k, out, stream) -> int:
+    return _check(lib().ot_materialize_rows(plan, row_idx, k, out, stream))
+
+
+def ot_sparsify_min_row(plan, block_rows, row_counts, stream):
+    """Returns (status, thr, nnz, n_massless, argmin); row_counts: device int64 [n] or 0."""
+    thr = ctypes.c_float()
+    nnz, nm, arg = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    st = _check(lib().ot_sparsify_min_row(plan, block_rows, ctypes.byref(thr), row_counts or None,
+                                          ctypes.byref(nnz), ctypes.byref(nm), ctypes.byref(arg),
+                                          stream))
+    return st, thr.value, nnz.value, nm.value, arg.value
+
+
+def ot_plan_destroy(plan) -> None:
+    if plan:
+        lib().ot_plan_destroy(plan)

@@ -1,0 +1,707 @@
+// api.cu -- host runtime behind the C ABI declared in include/ot_sinkhorn.h.
+//
+// Argument checks, one-time scale resolution (captured by the plan, moscot PR
+// #846 "materialize transport-matrix rows instead of pushing indicator
+// columns", section Fix), workspace sizing, launch shapes, and the iteration
+// driver: the f/g half-step pair is replayed as a CUDA graph in chunks of
+// check_every iterations on an internal stream; the host reads back only
+// scalars (the device stop flag, the in-loop residual, the iteration count).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "ot_sinkhorn.h"
+#include "runtime.h"
+
+using namespace ot;
+
+namespace {
+
+thread_local char g_err[512] = "no error";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+#define OT_CU(call)                                                                      \
+    do {                                                                                 \
+        cudaError_t e_ = (call);                                                         \
+        if (e_ != cudaSuccess)                                                           \
+            return fail(e_ == cudaErrorMemoryAllocation ? OT_ERR_OOM : OT_ERR_CUDA,       \
+                        "%s failed: %s", #call, cudaGetErrorString(e_));                 \
+    } while (0)
+
+int64_t round_up(int64_t v, int64_t q) { return (v + q - 1) / q * q; }
+
+// small device-side scalars of a plan
+struct DevScalars {
+    int flags[4];                 // x, y, a, b: bit0 non-finite, bit1 negative
+    unsigned long long zeros[2];  // zero weights in a, b
+    unsigned max_bits;            // max-cost pass result (float bits)
+    int bad;                      // row kernels: an index out of range
+    float thr;
+    int pad;
+    int64_t argmin, n_massless, nnz;
+    double r_sum[2];
+    double sums[4][kMaxD];        // sum x, sum x^2, sum y, sum y^2 (per coordinate)
+    double wsum[4];               // sum a, -, sum b, -
+};
+
+// pinned host mirror for read-backs
+struct HostScalars {
+    DevScalars s;
+    State st;
+    double o[kMaxD];
+};
+
+struct Side {          // one cloud's half of the problem
+    int64_t cnt, pad;  // points, padded to kColPad
+    float *rowtab;     // [pad][dp]
+    float *coltab;     // layout per kind
+    int tiles, splits, grid;
+    int64_t cps;       // columns per split of the OTHER side's table
+};
+
+}  // namespace
+
+struct ot_plan {
+    int device = 0;
+    const float *x = nullptr, *y = nullptr, *a = nullptr, *b = nullptr;
+    float *f = nullptr, *g = nullptr;
+    int64_t n = 0, m = 0;
+    int d = 0, kind = 0, dim = 0, dp = 0;
+    double eps = 0.0, c = 1.0;
+    int64_t n_massless_rows = 0, n_massless_cols = 0;
+    // workspace (one allocation, carved)
+    char *ws = nullptr;
+    Params *prm = nullptr;
+    State *st = nullptr;
+    double *o = nullptr;
+    DevScalars *ds = nullptr;
+    double *part1 = nullptr, *part2 = nullptr;  // coordinate-stat partials
+    float *fspare = nullptr;
+    float2 *part = nullptr;
+    unsigned *tile_cnt = nullptr;
+    double *tile_resid = nullptr;
+    Side sx{}, sy{};
+    // lazily allocated for the row kernels
+    char *ws_rows = nullptr;
+    double *dcol = nullptr, *rpart = nullptr;
+    float *rowmax = nullptr;
+    int64_t *counts = nullptr;
+    HostScalars *hs = nullptr;  // pinned
+    cudaStream_t s_int = nullptr;
+    cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+    cudaGraphExec_t graph[2] = {nullptr, nullptr};  // chunk graphs by start parity
+    int graph_len = 0;
+    int sm_count = 0;
+    // accounting and optional loop timing (events around each chunk)
+    int64_t launches = 0;
+    bool timing = false;
+    std::vector<cudaEvent_t> tev;
+    size_t tev_used = 0;
+};
+
+namespace {
+
+void plan_free(ot_plan *p) {
+    if (!p) return;
+    for (auto &gx : p->graph)
+        if (gx) cudaGraphExecDestroy(gx);
+    for (auto ev : p->tev) cudaEventDestroy(ev);
+    if (p->ws) cudaFree(p->ws);
+    if (p->ws_rows) cudaFree(p->ws_rows);
+    if (p->hs) cudaFreeHost(p->hs);
+    if (p->ev_in) cudaEventDestroy(p->ev_in);
+    if (p->ev_out) cudaEventDestroy(p->ev_out);
+    if (p->s_int) cudaStreamDestroy(p->s_int);
+    delete p;
+}
+
+// Carves aligned sub-buffers out of one allocation (first pass: sizing only).
+struct Carver {
+    char *base;
+    size_t off = 0;
+    template <typename T>
+    T *take(int64_t count) {
+        off = (size_t)round_up((int64_t)off, 256);
+        T *ptr = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += (size_t)count * sizeof(T);
+        return ptr;
+    }
+};
+
+// Column splits for one half-step: rows -> tiles of `tile`; the column table of
+// `cols_pad` columns is cut into `splits` spans (multiples of kColPad). Picks
+// the split count whose critical path (waves x columns per split) is shortest
+// for `cap` resident blocks, preferring fewer splits on ties.
+void choose_splits(int64_t rows, int64_t cols_pad, int tile, int cap, Side &sd) {
+    const int64_t tiles = (rows + tile - 1) / tile;
+    double best = 1e300;
+    int best_s = 1;
+    int64_t best_cps = cols_pad;
+    const int64_t max_s = std::min<int64_t>(cols_pad / kColPad, 4096);
+    for (int64_t s = 1; s <= max_s; ++s) {
+        const int64_t cps = round_up((cols_pad + s - 1) / s, kColPad);
+        const int64_t s_eff = (cols_pad + cps - 1) / cps;
+        if (s_eff != s) continue;
+        const int64_t items = tiles * s_eff;
+        const int64_t waves = (items + cap - 1) / cap;
+        // per-item fixed cost ~ 64 columns of work (row loads, partial writes, combine)
+        const double t = (double)waves * (double)(cps + 64);
+        if (t < best * 0.995) {
+            best = t;
+            best_s = (int)s_eff;
+            best_cps = cps;
+        }
+    }
+    sd.tiles = (int)tiles;
+    sd.splits = best_s;
+    sd.cps = best_cps;
+    sd.grid = (int)std::min<int64_t>(tiles * best_s, cap);
+}
+
+}  // namespace
+
+namespace {
+
+// Reads the solver state back (synchronises the internal stream).
+int read_state(ot_plan *p) {
+    OT_CU(cudaMemcpyAsync(&p->hs->st, p->st, sizeof(State), cudaMemcpyDeviceToHost, p->s_int));
+    OT_CU(cudaStreamSynchronize(p->s_int));
+    return OT_OK;
+}
+
+int read_scalars(ot_plan *p) {
+    OT_CU(cudaMemcpyAsync(&p->hs->s, p->ds, sizeof(DevScalars), cudaMemcpyDeviceToHost, p->s_int));
+    OT_CU(cudaStreamSynchronize(p->s_int));
+    return OT_OK;
+}
+
+HalfStep make_step(const ot_plan *p, int side, int parity) {
+    HalfStep A{};
+    const bool f = side == 0;
+    const Side &rows = f ? p->sx : p->sy;
+    const Side &cols = f ? p->sy : p->sx;
+    float *fb[2] = {p->f, p->fspare};
+    A.coltab = reinterpret_cast<const float4 *>(cols.coltab);
+    A.rowtab = rows.rowtab;
+    A.rows = rows.cnt;
+    A.cols_pad = cols.pad;
+    A.cols_per_split = rows.cps;
+    A.splits = rows.splits;
+    A.tiles = rows.tiles;
+    A.dp = p->dp;
+    A.side = side;
+    A.part = p->part;
+    A.tile_cnt = p->tile_cnt;
+    A.tile_resid = p->tile_resid;
+    A.w = f ? p->a : p->b;
+    A.pot_old = f ? fb[parity] : p->g;
+    A.pot_new = f ? fb[parity ^ 1] : p->g;
+    A.next_col = rows.coltab;  // this side's column table feeds the other half-step
+    if (p->kind == 0) {
+        A.nxt_a = 8; A.nxt_l = 1; A.nxt_b = 6;
+    } else {
+        A.nxt_a = 2 * (p->dp + 4); A.nxt_l = p->dp + 4; A.nxt_b = p->dp;
+    }
+    A.prm = p->prm;
+    A.st = p->st;
+    return A;
+}
+
+// Records a timing event on the internal stream (no-op unless timing).
+cudaError_t mark(ot_plan *p) {
+    if (!p->timing) return cudaSuccess;
+    if (p->tev_used == p->tev.size()) {
+        cudaEvent_t ev;
+        cudaError_t e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) return e;
+        p->tev.push_back(ev);
+    }
+    return cudaEventRecord(p->tev[p->tev_used++], p->s_int);
+}
+
+cudaError_t launch_iteration(const ot_plan *p, int parity) {
+    cudaError_t e = launch_halfstep(p->kind, p->dim, make_step(p, 0, parity), p->sx.grid, p->s_int);
+    if (e != cudaSuccess) return e;
+    return launch_halfstep(p->kind, p->dim, make_step(p, 1, parity), p->sy.grid, p->s_int);
+}
+
+// Runs `iters` iterations starting at global parity `parity0`, in chunks of
+// graph_len (replayed graphs when enabled). With `check`, the stop flag is
+// read after every chunk. Returns OT status.
+int run_iterations(ot_plan *p, int parity0, int iters, bool check, bool use_graphs) {
+    int i = 0;
+    while (i < iters) {
+        const int len = std::min(p->graph_len, iters - i);
+        const int par = (parity0 + i) & 1;
+        OT_CU(mark(p));
+        if (use_graphs && len == p->graph_len) {
+            if (!p->graph[par]) {
+                cudaGraph_t gr = nullptr;
+                OT_CU(cudaStreamBeginCapture(p->s_int, cudaStreamCaptureModeThreadLocal));
+                cudaError_t le = cudaSuccess;
+                for (int k = 0; k < len && le == cudaSuccess; ++k)
+                    le = launch_iteration(p, (par + k) & 1);
+                cudaError_t ce = cudaStreamEndCapture(p->s_int, &gr);
+                if (le != cudaSuccess || ce != cudaSuccess) {
+                    if (gr) cudaGraphDestroy(gr);
+                    return fail(OT_ERR_CUDA, "graph capture failed: %s",
+                                cudaGetErrorString(le != cudaSuccess ? le : ce));
+                }
+                cudaError_t ie = cudaGraphInstantiate(&p->graph[par], gr, 0);
+                cudaGraphDestroy(gr);
+                if (ie != cudaSuccess)
+                    return fail(OT_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(ie));
+            }
+            OT_CU(cudaGraphLaunch(p->graph[par], p->s_int));
+        } else {
+            for (int k = 0; k < len; ++k) OT_CU(launch_iteration(p, (par + k) & 1));
+        }
+        OT_CU(mark(p));
+        p->launches += 2 * len;
+        i += len;
+        if (check) {
+            int rc = read_state(p);
+            if (rc != OT_OK) return rc;
+            if (p->hs->st.stop) break;
+        }
+    }
+    return OT_OK;
+}
+
+int check_device(int *dev, int *sms) {
+    OT_CU(cudaGetDevice(dev));
+    cudaDeviceProp prop;
+    OT_CU(cudaGetDeviceProperties(&prop, *dev));
+    if (prop.major != 10)
+        return fail(OT_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a", *dev,
+                    prop.major, prop.minor);
+    *sms = prop.multiProcessorCount;
+    return OT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ot_version(void) { return OT_ABI_VERSION; }
+
+const char *ot_last_error_string(void) { return g_err; }
+
+void ot_options_default(ot_options *opt) {
+    if (!opt) return;
+    std::memset(opt, 0, sizeof *opt);
+    opt->warm_start = 0;
+    opt->check_every = 16;
+    opt->use_graphs = 1;
+    opt->iters_per_stage = 20;
+    opt->scale_value = 1.0;
+    opt->eps_init = 0.0;
+    opt->eps_decay = 0.7;
+    opt->timing = 0;
+}
+
+void ot_plan_destroy(ot_plan *plan) { plan_free(plan); }
+
+}  // extern "C"
+
+namespace {
+
+// Allocates the plan's solve workspace and chooses launch shapes.
+int plan_setup(ot_plan *p) {
+    p->kind = p->d <= 3 ? 0 : 1;
+    if (p->kind == 0) {
+        p->dim = p->d;
+        p->dp = 4;
+    } else {
+        p->dim = p->d <= 8 ? 8 : p->d <= 16 ? 16 : p->d <= 32 ? 32 : 64;
+        p->dp = p->dim;
+    }
+    const int tile = p->kind == 0 ? kHsTile : kGnTile;
+    const int64_t colw = p->kind == 0 ? 4 : p->dp + 4;
+    p->sx.cnt = p->n;
+    p->sy.cnt = p->m;
+    p->sx.pad = round_up(p->n, kColPad);
+    p->sy.pad = round_up(p->m, kColPad);
+    const int bps = halfstep_blocks_per_sm(p->kind, p->dim);
+    if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
+    const int cap = bps * p->sm_count;
+    choose_splits(p->n, p->sy.pad, tile, cap, p->sx);
+    choose_splits(p->m, p->sx.pad, tile, cap, p->sy);
+    const int64_t part_cnt = std::max((int64_t)p->sx.splits * p->sx.tiles,
+                                      (int64_t)p->sy.splits * p->sy.tiles) * tile;
+    const int64_t tiles = std::max(p->sx.tiles, p->sy.tiles);
+
+    for (int pass = 0; pass < 2; ++pass) {
+        Carver cv{pass ? p->ws : nullptr};
+        p->prm = cv.take<Params>(1);
+        p->st = cv.take<State>(1);
+        p->o = cv.take<double>(kMaxD);
+        p->ds = cv.take<DevScalars>(1);
+        p->part1 = cv.take<double>((int64_t)kMaxD * 1024);
+        p->part2 = cv.take<double>((int64_t)kMaxD * 1024);
+        p->fspare = cv.take<float>(p->n);
+        p->sx.rowtab = cv.take<float>(p->sx.pad * p->dp);
+        p->sy.rowtab = cv.take<float>(p->sy.pad * p->dp);
+        p->sx.coltab = cv.take<float>(p->sx.pad * colw);
+        p->sy.coltab = cv.take<float>(p->sy.pad * colw);
+        p->part = cv.take<float2>(part_cnt);
+        p->tile_cnt = cv.take<unsigned>(tiles);
+        p->tile_resid = cv.take<double>(tiles);
+        if (pass == 0) OT_CU(cudaMalloc(&p->ws, cv.off));
+    }
+    OT_CU(cudaMemsetAsync(p->tile_cnt, 0, sizeof(unsigned) * tiles, p->s_int));
+    OT_CU(cudaMemsetAsync(p->st, 0, sizeof(State), p->s_int));
+    OT_CU(cudaMemsetAsync(p->ds, 0, sizeof(DevScalars), p->s_int));
+    return OT_OK;
+}
+
+// Input statistics, validation and the captured scale.
+int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
+    DevScalars *ds = p->ds;
+    OT_CU(launch_coord_stats(p->x, p->n, p->d, p->part1, p->part2, ds->sums[0], ds->sums[1],
+                             &ds->flags[0], nullptr, p->s_int));
+    OT_CU(launch_coord_stats(p->y, p->m, p->d, p->part1, p->part2, ds->sums[2], ds->sums[3],
+                             &ds->flags[1], nullptr, p->s_int));
+    OT_CU(launch_coord_stats(p->a, p->n, 1, p->part1, p->part2, &ds->wsum[0], &ds->wsum[1],
+                             &ds->flags[2], &ds->zeros[0], p->s_int));
+    OT_CU(launch_coord_stats(p->b, p->m, 1, p->part1, p->part2, &ds->wsum[2], &ds->wsum[3],
+                             &ds->flags[3], &ds->zeros[1], p->s_int));
+    p->launches += 8;
+    int rc = read_scalars(p);
+    if (rc != OT_OK) return rc;
+    const DevScalars &h = p->hs->s;
+    if ((h.flags[0] | h.flags[1]) & 1) return fail(OT_ERR_NONFINITE, "x or y holds a NaN or inf");
+    if ((h.flags[2] | h.flags[3]) & 1) return fail(OT_ERR_NONFINITE, "a or b holds a NaN or inf");
+    if ((h.flags[2] | h.flags[3]) & 2) return fail(OT_ERR_INVALID_ARG, "negative weight in a or b");
+    if (!(h.wsum[0] > 0.0) || !(h.wsum[2] > 0.0))
+        return fail(OT_ERR_INVALID_ARG, "a and b must have positive sums");
+    p->n_massless_rows = (int64_t)h.zeros[0];
+    p->n_massless_cols = (int64_t)h.zeros[1];
+    double dot = 0.0, sxx = 0.0, syy = 0.0;
+    for (int k = 0; k < p->d; ++k) {
+        const double mx = h.sums[0][k] / (double)p->n, my = h.sums[2][k] / (double)p->m;
+        p->hs->o[k] = 0.5 * (mx + my);
+        dot += mx * my;
+        sxx += h.sums[1][k];
+        syy += h.sums[3][k];
+    }
+    for (int k = p->d; k < kMaxD; ++k) p->hs->o[k] = 0.0;
+    OT_CU(cudaMemcpyAsync(p->o, p->hs->o, sizeof(double) * kMaxD, cudaMemcpyHostToDevice, p->s_int));
+    double c = 1.0;
+    if (scale == OT_SCALE_MEAN) {
+        const double mean = sxx / (double)p->n + syy / (double)p->m - 2.0 * dot;
+        c = 1.0 / mean;
+    } else if (scale == OT_SCALE_MAX_COST) {
+        OT_CU(launch_max_cost(p->x, p->y, p->n, p->m, p->d, &ds->max_bits, p->s_int));
+        p->launches += 1;
+        rc = read_scalars(p);
+        if (rc != OT_OK) return rc;
+        float mx;
+        std::memcpy(&mx, &p->hs->s.max_bits, sizeof mx);
+        c = 1.0 / (double)mx;
+    } else if (scale == OT_SCALE_VALUE) {
+        c = 1.0 / scale_value;
+    }
+    if (!std::isfinite(c) || !(c > 0.0))
+        return fail(OT_ERR_INVALID_ARG, "cost scale is zero or not finite (all points equal?)");
+    p->c = c;
+    // the stream must not leave before the pinned o[] has been copied
+    OT_CU(cudaStreamSynchronize(p->s_int));
+    return OT_OK;
+}
+
+int validate(const float *x, const float *y, const float *a, const float *b, int64_t n,
+             int64_t m, int32_t d, float eps, ot_scale scale, int32_t n_iters, float *f,
+             float *g, const ot_options &o) {
+    if (!x || !y || !a || !b || !f || !g) return fail(OT_ERR_INVALID_ARG, "null array pointer");
+    if (n < 1 || m < 1) return fail(OT_ERR_INVALID_ARG, "n and m must be >= 1 (n=%lld m=%lld)",
+                                    (long long)n, (long long)m);
+    if (n > INT32_MAX || m > INT32_MAX)
+        return fail(OT_ERR_OVERFLOW, "n and m must be < 2^31 (n=%lld m=%lld)", (long long)n,
+                    (long long)m);
+    if (d < 1 || d > kMaxD) return fail(d < 1 ? OT_ERR_INVALID_ARG : OT_ERR_UNSUPPORTED,
+                                        "d=%d outside 1..%d", d, kMaxD);
+    if (!(eps > 0.0f) || !std::isfinite(eps)) return fail(OT_ERR_INVALID_ARG, "eps must be > 0 and finite");
+    if (scale < OT_SCALE_NONE || scale > OT_SCALE_VALUE) return fail(OT_ERR_INVALID_ARG, "bad scale_cost");
+    if (scale == OT_SCALE_VALUE && !(o.scale_value > 0.0 && std::isfinite(o.scale_value)))
+        return fail(OT_ERR_INVALID_ARG, "scale_value must be > 0 and finite");
+    if (n_iters < 0) return fail(OT_ERR_INVALID_ARG, "n_iters must be >= 0");
+    if (n_iters == 0 && !o.warm_start)
+        return fail(OT_ERR_INVALID_ARG, "n_iters == 0 needs warm_start (a plan at given f, g)");
+    if (o.check_every < 1) return fail(OT_ERR_INVALID_ARG, "check_every must be >= 1");
+    if (o.eps_init > 0.0) {
+        if (!(o.eps_decay > 0.0 && o.eps_decay < 1.0)) return fail(OT_ERR_INVALID_ARG, "eps_decay must be in (0,1)");
+        if (o.iters_per_stage < 1) return fail(OT_ERR_INVALID_ARG, "iters_per_stage must be >= 1");
+    }
+    return OT_OK;
+}
+
+}  // namespace
+
+extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const float *a,
+                                      const float *b, int64_t n, int64_t m, int32_t d, float eps,
+                                      ot_scale scale_cost, int32_t n_iters, float tol, float *f,
+                                      float *g, void *stream, const ot_options *opt,
+                                      ot_plan **plan_out, ot_info *info) {
+    if (plan_out) *plan_out = nullptr;
+    ot_options o;
+    ot_options_default(&o);
+    if (opt) o = *opt;
+    int rc = validate(x, y, a, b, n, m, d, eps, scale_cost, n_iters, f, g, o);
+    if (rc != OT_OK) return rc;
+    ot_plan *p = new (std::nothrow) ot_plan();
+    if (!p) return fail(OT_ERR_OOM, "host allocation failed");
+    struct Guard {
+        ot_plan *p;
+        bool keep = false;
+        ~Guard() {
+            if (!keep) plan_free(p);
+        }
+    } guard{p};
+    rc = check_device(&p->device, &p->sm_count);
+    if (rc != OT_OK) return rc;
+    p->x = x; p->y = y; p->a = a; p->b = b; p->f = f; p->g = g;
+    p->n = n; p->m = m; p->d = d;
+    cudaStream_t us = (cudaStream_t)stream;
+    OT_CU(cudaStreamCreateWithFlags(&p->s_int, cudaStreamNonBlocking));
+    OT_CU(cudaEventCreateWithFlags(&p->ev_in, cudaEventDisableTiming));
+    OT_CU(cudaEventCreateWithFlags(&p->ev_out, cudaEventDisableTiming));
+    OT_CU(cudaMallocHost(&p->hs, sizeof(HostScalars)));
+    OT_CU(cudaEventRecord(p->ev_in, us));
+    OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
+    if ((rc = plan_setup(p)) != OT_OK) return rc;
+    if ((rc = resolve_scale(p, scale_cost, o.scale_value)) != OT_OK) return rc;
+    if (!o.warm_start) {
+        OT_CU(cudaMemsetAsync(f, 0, sizeof(float) * n, p->s_int));
+        OT_CU(cudaMemsetAsync(g, 0, sizeof(float) * m, p->s_int));
+    }
+    p->graph_len = std::max(2, (o.check_every + 1) / 2 * 2);
+    p->timing = o.timing != 0;
+
+    // eps stages: FlashSinkhorn 2 (sections 3.1, C.3) anneals eps and continues
+    // at the target; here stage k runs at max(eps, eps_init * decay^k)
+    std::vector<double> stage_eps;
+    if (o.eps_init > 0.0) {
+        for (int k = 0;; ++k) {
+            const double ek = std::max((double)eps, o.eps_init * std::pow(o.eps_decay, (double)k));
+            stage_eps.push_back(ek);
+            if (ek == (double)eps || k > 100000) break;
+        }
+    } else {
+        stage_eps.push_back((double)eps);
+    }
+    float *fb[2] = {p->f, p->fspare};
+    const int layout = p->kind == 0 ? 0 : 1;
+    int t = 0, converged = 0;
+    int64_t half_steps = 0;
+    double resid = NAN;
+    for (size_t si = 0; si < stage_eps.size(); ++si) {
+        const bool last = si + 1 == stage_eps.size();
+        const double tol_s = (last && tol > 0.0f) ? (double)tol : 0.0;
+        const int iters = last ? n_iters : o.iters_per_stage;
+        OT_CU(launch_set_params(p->prm, stage_eps[si], p->c, tol_s, p->s_int));
+        OT_CU(launch_reset_state(p->st, p->s_int));
+        OT_CU(launch_tables(x, fb[t & 1], n, p->sx.pad, d, p->dp, p->o, p->prm, p->sx.rowtab,
+                            p->sx.coltab, layout, p->s_int));
+        OT_CU(launch_tables(y, g, m, p->sy.pad, d, p->dp, p->o, p->prm, p->sy.rowtab,
+                            p->sy.coltab, layout, p->s_int));
+        p->launches += 4;
+        if ((rc = run_iterations(p, t & 1, iters, tol_s > 0.0, o.use_graphs != 0)) != OT_OK) return rc;
+        if ((rc = read_state(p)) != OT_OK) return rc;
+        const int done = p->hs->st.stop ? p->hs->st.conv_iter : iters;
+        t += done;
+        half_steps += 2 * (int64_t)done + (p->hs->st.stop ? 1 : 0);
+        if (last) {
+            if (p->hs->st.stop) {
+                converged = 1;
+                resid = p->hs->st.resid[0];
+            } else if (iters > 0) {
+                // one more f-update measures ||T1 - a||_1 of the final state
+                OT_CU(mark(p));
+                OT_CU(launch_halfstep(p->kind, p->dim, make_step(p, 0, t & 1), p->sx.grid, p->s_int));
+                OT_CU(mark(p));
+                p->launches += 1;
+                half_steps += 1;
+                if ((rc = read_state(p)) != OT_OK) return rc;
+                resid = p->hs->st.resid[0];
+                converged = p->hs->st.stop;
+            }
+        }
+    }
+    if (t & 1) OT_CU(cudaMemcpyAsync(p->f, p->fspare, sizeof(float) * n, cudaMemcpyDeviceToDevice, p->s_int));
+    if ((rc = read_state(p)) != OT_OK) return rc;
+    if (p->hs->st.nonfinite)
+        return fail(OT_ERR_NONFINITE, "a potential left the finite range (eps too small for float32?)");
+    p->eps = stage_eps.back();
+    double loop_ms = 0.0;
+    for (size_t e = 0; e + 1 < p->tev_used; e += 2) {
+        float ms = 0.0f;
+        OT_CU(cudaEventElapsedTime(&ms, p->tev[e], p->tev[e + 1]));
+        loop_ms += ms;
+    }
+    OT_CU(cudaEventRecord(p->ev_out, p->s_int));
+    OT_CU(cudaStreamWaitEvent(us, p->ev_out, 0));
+    if (info) {
+        info->iterations = t;
+        info->converged = converged;
+        info->stages = (int32_t)stage_eps.size();
+        info->col_splits = p->sx.splits;
+        info->residual = resid;
+        info->inv_scale_cost = p->c;
+        info->eps = p->eps;
+        info->n_massless_rows = p->n_massless_rows;
+        info->n_massless_cols = p->n_massless_cols;
+        info->half_steps = half_steps;
+        info->kernel_launches = p->launches;
+        info->loop_ms = loop_ms;
+    }
+    if (plan_out) {
+        *plan_out = p;
+        guard.keep = true;
+    }
+    if (p->n_massless_rows > 0) {
+        fail(OT_WARN_MASSLESS_ROWS, "%lld rows carry no mass", (long long)p->n_massless_rows);
+        return OT_WARN_MASSLESS_ROWS;
+    }
+    return OT_OK;
+}
+
+namespace {
+
+int plan_check(const ot_plan *p) {
+    if (!p) return fail(OT_ERR_INVALID_ARG, "null plan");
+    int dev = -1;
+    OT_CU(cudaGetDevice(&dev));
+    if (dev != p->device) return fail(OT_ERR_INVALID_ARG, "plan belongs to device %d, current is %d", p->device, dev);
+    return OT_OK;
+}
+
+// Workspace of the row kernels, allocated on first use and kept by the plan.
+int ensure_rows_ws(ot_plan *p) {
+    if (p->ws_rows) return OT_OK;
+    const int64_t big = std::max(p->n, p->m);
+    for (int pass = 0; pass < 2; ++pass) {
+        Carver cv{pass ? p->ws_rows : nullptr};
+        p->dcol = cv.take<double>(big * (p->d + 1));
+        p->rpart = cv.take<double>(rowpass_blocks(big));
+        p->rowmax = cv.take<float>(p->n);
+        p->counts = cv.take<int64_t>(p->n);
+        if (pass == 0) OT_CU(cudaMalloc(&p->ws_rows, cv.off));
+    }
+    return OT_OK;
+}
+
+int sync_read(ot_plan *p, cudaStream_t s) {
+    OT_CU(cudaMemcpyAsync(&p->hs->s, p->ds, sizeof(DevScalars), cudaMemcpyDeviceToHost, s));
+    OT_CU(cudaStreamSynchronize(s));
+    return OT_OK;
+}
+
+}  // namespace
+
+extern "C" int ot_materialize_rows(const ot_plan *cplan, const int64_t *row_idx, int64_t k,
+                                   float *out, void *stream) {
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if (k < 0) return fail(OT_ERR_INVALID_ARG, "k must be >= 0");
+    if (k == 0) return OT_OK;
+    if (!row_idx || !out) return fail(OT_ERR_INVALID_ARG, "null row_idx or out");
+    if (k > INT64_MAX / p->m) return fail(OT_ERR_OVERFLOW, "k*m overflows int64");
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    OT_CU(cudaMemsetAsync(&p->ds->bad, 0, sizeof(int), s));
+    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    MatArgs M{};
+    M.x = p->x; M.f = p->f; M.dcol = p->dcol; M.o = p->o; M.prm = p->prm;
+    M.row_idx = row_idx; M.k = k; M.n = p->n; M.m = p->m; M.d = p->d;
+    M.vec = (p->m % 4 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
+    M.out = out;
+    M.bad = &p->ds->bad;
+    OT_CU(launch_materialize(M, s));
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    if (p->hs->s.bad) return fail(OT_ERR_INVALID_ARG, "a row index is outside [0, n)");
+    return OT_OK;
+}
+
+extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, float *thr_out,
+                                   int64_t *row_counts, int64_t *nnz_out,
+                                   int64_t *n_massless_out, int64_t *argmin_out, void *stream) {
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if (block_rows < 0) return fail(OT_ERR_INVALID_ARG, "block_rows must be >= 0");
+    if (block_rows == 0 || block_rows > p->n) block_rows = p->n;
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    RowPassArgs R{};
+    R.pts = p->x; R.pot = p->f; R.w = p->a; R.dcol = p->dcol; R.o = p->o; R.prm = p->prm;
+    R.cols = p->m; R.d = p->d; R.rowmax = p->rowmax;
+    R.counts = row_counts ? row_counts : p->counts;
+    // pass A: max_j T_ij of every row, block by block
+    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
+        R.row_begin = r0;
+        R.row_end = std::min(p->n, r0 + block_rows);
+        OT_CU(launch_rowpass(0, R, s));
+    }
+    OT_CU(launch_min_row_reduce(p->rowmax, p->a, p->n, &p->ds->thr, &p->ds->argmin,
+                                &p->ds->n_massless, s));
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    const float thr = p->hs->s.thr;
+    const int64_t argmin = p->hs->s.argmin, nm = p->hs->s.n_massless;
+    // pass B: entries kept per row (T_ij >= thr, same float path)
+    R.thr = thr;
+    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
+        R.row_begin = r0;
+        R.row_end = std::min(p->n, r0 + block_rows);
+        OT_CU(launch_rowpass(1, R, s));
+    }
+    OT_CU(launch_sum_i64(R.counts, p->n, &p->ds->nnz, s));
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    if (thr_out) *thr_out = thr;
+    if (nnz_out) *nnz_out = p->hs->s.nnz;
+    if (n_massless_out) *n_massless_out = nm;
+    if (argmin_out) *argmin_out = argmin;
+    if (nm > 0) {
+        fail(OT_WARN_MASSLESS_ROWS, "%lld rows carry no mass", (long long)nm);
+        return OT_WARN_MASSLESS_ROWS;
+    }
+    return OT_OK;
+}
+
+extern "C" int ot_marginal_residual(const ot_plan *cplan, double *row_l1, double *col_l1,
+                                    void *stream) {
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    RowPassArgs R{};
+    R.o = p->o; R.prm = p->prm; R.d = p->d; R.dcol = p->dcol; R.part = p->rpart;
+    // rows: sum_j T_ij against a_i
+    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    R.pts = p->x; R.pot = p->f; R.w = p->a; R.cols = p->m; R.row_begin = 0; R.row_end = p->n;
+    OT_CU(launch_rowpass(2, R, s));
+    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->n), &p->ds->r_sum[0], s));
+    // columns: the same pass with the clouds' roles swapped
+    OT_CU(launch_dcol(p->x, p->f, p->n, p->d, p->o, p->prm, p->dcol, s));
+    R.pts = p->y; R.pot = p->g; R.w = p->b; R.cols = p->n; R.row_begin = 0; R.row_end = p->m;
+    OT_CU(launch_rowpass(2, R, s));
+    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->m), &p->ds->r_sum[1], s));
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    if (row_l1) *row_l1 = p->hs->s.r_sum[0];
+    if (col_l1) *col_l1 = p->hs->s.r_sum[1];
+    return OT_OK;
+}

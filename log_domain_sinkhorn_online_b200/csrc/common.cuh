@@ -1,0 +1,94 @@
+// common.cuh -- device-side helpers and the structs shared by the kernels and
+// the host runtime of the B200 Sinkhorn library (internal; not installed).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ot {
+
+// ------------------------------------------------------------ constants --
+constexpr int kMaxD = 64;            // largest point dimension this build supports
+constexpr double kLog2e = 1.4426950408889634073599246810019;
+constexpr double kLn2 = 0.69314718055994530941723212145818;
+
+// Low-d half-step tiling: 128 threads x 8 rows each = 1024 rows per tile; the
+// column table is streamed through shared memory 256 columns at a time.
+constexpr int kHsThreads = 128;
+constexpr int kHsRows = 8;
+constexpr int kHsTile = kHsThreads * kHsRows;
+constexpr int kHsChunk = 256;
+
+// Generic-d half-step tiling: 128 threads x 2 rows, 64-column chunks.
+constexpr int kGnThreads = 128;
+constexpr int kGnRows = 2;
+constexpr int kGnTile = kGnThreads * kGnRows;
+constexpr int kGnChunk = 64;
+
+// every column table is padded (G = -inf) to a multiple of this many columns;
+// column splits are multiples of it too, so no inner loop has a tail
+constexpr int kColPad = 8;
+
+// A lazily refreshed running maximum may lag the true one by this much (base-2
+// units): every summed term is then at most 2^8, far from float overflow.
+constexpr float kLazyMax = 8.0f;
+constexpr float kNegBig = -1.0e30f;  // finite "no column seen yet" maximum
+
+// -------------------------------------------------------- device structs --
+// Per-stage scalars, resident on the device so one captured graph serves all
+// annealing stages.
+struct Params {
+    double eps;       // entropic regularisation (scaled cost units)
+    double kappa;     // log2(e) / eps
+    double c;         // inv_scale_cost
+    double tol;       // stopping tolerance on ||T1 - a||_1 (<= 0: none)
+};
+
+// Solver state written by the kernels' last-finishing blocks.
+struct State {
+    int stop;           // set when the tol test passed: later half-steps return at once
+    int nonfinite;      // a massful row produced a non-finite potential
+    int bad_index;      // a row index outside [0, n) was given to a row kernel
+    int iter_done;      // completed iterations in the current stage
+    int conv_iter;      // iteration count at which tol was met (-1: not yet)
+    int pad0;
+    double resid[2];    // last in-loop marginal residual of each side (0: rows, 1: cols)
+    unsigned tiles_done[2];
+    unsigned pad1[2];
+};
+
+// Arguments of one half-step launch (the same kernel serves f and g: rows are
+// the side being updated, columns the other side).
+struct HalfStep {
+    const float4 *coltab;      // column table (layout depends on the kernel)
+    const float *rowtab;       // row coordinates minus the shift, [rows_pad][dp]
+    int64_t rows;              // rows updated (n for the f side, m for g)
+    int64_t cols_pad;          // padded column count (multiple of kColPad)
+    int64_t cols_per_split;    // multiple of kColPad (the last chunk of a split may be partial)
+    int splits;                // column splits S
+    int tiles;                 // row tiles
+    int dp;                    // row-table stride in floats
+    int side;                  // 0: f-update (runs the stop test), 1: g-update
+    float2 *part;              // [splits][tiles*tile] (running max, sum) partials
+    unsigned *tile_cnt;        // [tiles] splits finished, reset by the last one
+    double *tile_resid;        // [tiles] residual partial of each tile
+    const float *w;            // weights of the updated side (a or b)
+    const float *pot_old;      // potential before the update
+    float *pot_new;            // potential after the update
+    float *next_col;           // column table of the other half-step (float view)
+    int64_t nxt_a, nxt_l, nxt_b;  // column i's G' sits at (i>>1)*nxt_a + (i&1)*nxt_l + nxt_b
+    const Params *prm;
+    State *st;
+};
+
+// ------------------------------------------------------ device helpers --
+__device__ __forceinline__ float ex2_approx(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ int ld_volatile(const int *p) {
+    return *reinterpret_cast<const volatile int *>(p);
+}
+
+}  // namespace ot

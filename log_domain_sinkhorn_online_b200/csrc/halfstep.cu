@@ -1,0 +1,355 @@
+// halfstep.cu -- fused log-domain Sinkhorn half-step for sm_100a.
+//
+// One launch performs f_i <- eps ln a_i - eps LSE_j((g_j - C_ij)/eps) for every
+// row i (or the g-update with the roles of the clouds swapped), following
+// "FlashSinkhorn 2: Block-Sparse Entropic Optimal Transport", section 2.1: the
+// update is a streaming log-sum-exp over column tiles whose costs are generated
+// on the fly, so the n x m matrix never exists.
+//
+// Cost tile generator. In base-2 units, with kappa = log2(e)/eps, the shift o
+// (midpoint of the two clouds' means) and x' = x - o, y' = y - o:
+//   kappa (g_j - C_ij) = G_j + 2 c kappa x'_i . y'_j + R_i,
+//   G_j = kappa (g_j - c |y'_j|^2)   (column table, refreshed by the other half-step),
+//   R_i = -c kappa |x'_i|^2           (row constant, added once per row in float64).
+// For d <= 3 the per-pair work is d packed-f32x2 FMAs (two columns per
+// instruction), one subtraction of the running maximum, one MUFU ex2 and one
+// add: the kernel is bound by the ex2 rate, not by memory.
+//
+// Split-column combine. Each work item is (row tile, column split). It writes
+// (running max, sum) per row; the last split of a tile to finish (atomic
+// ticket, no waiting) merges them in float64 in split order, writes the new
+// potential, the other half-step's column-table entry, and this row's term of
+// the marginal residual ||T 1 - a||_1 at the state before the update:
+//   sum_j T_ij(old) = 2^(kappa f_old_i + L_i),  L_i = log2 sum_j 2^(kappa (g_j - C_ij)).
+// The last tile to finish sums the residual partials in tile order (no float
+// atomics, so the result is deterministic) and runs the stop test.
+#include "common.cuh"
+
+namespace ot {
+
+// Merge the column splits of one row tile; run by the block that finishes a
+// tile last. Returns nothing; all threads of the block must call it.
+template <int THREADS, int TILE>
+__device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_flag) {
+    const int tid = threadIdx.x;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        unsigned prev = atomicAdd(&A.tile_cnt[tile], 1u);
+        *s_flag = (prev == (unsigned)(A.splits - 1));
+    }
+    __syncthreads();
+    if (!*s_flag) return;
+    __threadfence();
+
+    const double eps = A.prm->eps, kappa = A.prm->kappa, c = A.prm->c, tol = A.prm->tol;
+    const int64_t stride = (int64_t)A.tiles * TILE;
+    double rsum = 0.0;
+    bool bad = false;
+#pragma unroll 1
+    for (int k = 0; k < TILE / THREADS; ++k) {
+        const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
+        if (row >= A.rows) continue;
+        float M = kNegBig;
+        for (int s = 0; s < A.splits; ++s) M = fmaxf(M, __ldcg(&A.part[s * stride + row]).x);
+        double S = 0.0;
+        for (int s = 0; s < A.splits; ++s) {
+            float2 p = __ldcg(&A.part[s * stride + row]);
+            if (p.y > 0.0f) S += (double)p.y * exp2((double)p.x - (double)M);
+        }
+        const float *xr = A.rowtab + row * (int64_t)A.dp;
+        double nrm = 0.0;
+        for (int q = 0; q < A.dp; ++q) nrm += (double)xr[q] * (double)xr[q];
+        const double wi = (double)A.w[row];
+        double pot = 0.0, term = 0.0;
+        if (wi == 0.0) {
+            pot = -INFINITY;  // massless row: empty row of the plan
+        } else if (!(S > 0.0)) {
+            pot = INFINITY;   // every column is massless: no finite potential
+            bad = true;
+        } else {
+            const double L = (double)M + log2(S) - kappa * c * nrm;
+            pot = eps * log(wi) - L / kappa;
+            const double old = (double)A.pot_old[row];
+            term = fabs(exp2(kappa * old + L) - wi);
+        }
+        const float pf = (float)pot;
+        if (wi != 0.0 && !isfinite(pf)) bad = true;
+        A.pot_new[row] = pf;
+        A.next_col[(row >> 1) * A.nxt_a + (row & 1) * A.nxt_l + A.nxt_b] =
+            (wi == 0.0) ? -INFINITY : (float)(kappa * ((double)pf - c * nrm));
+        rsum += term;
+    }
+    if (bad) atomicExch(&A.st->nonfinite, 1);
+    if (tid == 0) A.tile_cnt[tile] = 0;
+
+    // deterministic block sum of the residual terms
+    for (int off = 16; off > 0; off >>= 1) rsum += __shfl_xor_sync(0xffffffffu, rsum, off);
+    if ((tid & 31) == 0) s_red[tid >> 5] = rsum;
+    __syncthreads();
+    if (tid == 0) {
+        double t = 0.0;
+        for (int w = 0; w < THREADS / 32; ++w) t += s_red[w];
+        A.tile_resid[tile] = t;
+        __threadfence();
+        unsigned prev = atomicAdd(&A.st->tiles_done[A.side], 1u);
+        *s_flag = (prev == (unsigned)(A.tiles - 1));
+    }
+    __syncthreads();
+    if (!*s_flag) return;
+    __threadfence();
+    if (tid < 32) {
+        double v = 0.0;
+        for (int t = tid; t < A.tiles; t += 32) v += __ldcg(&A.tile_resid[t]);
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (tid == 0) {
+            State *st = A.st;
+            st->resid[A.side] = v;
+            st->tiles_done[A.side] = 0;
+            if (A.side == 0) {
+                if (tol > 0.0 && st->iter_done >= 1 && v <= tol) {
+                    st->stop = 1;
+                    st->conv_iter = st->iter_done;
+                }
+            } else {
+                st->iter_done += 1;
+            }
+            __threadfence();
+        }
+    }
+}
+
+// ------------------------------------------------------------ d <= 3 path
+// Column table: for the column pair (2p, 2p+1), two float4
+//   [Y0_2p, Y0_2p+1, Y1_2p, Y1_2p+1]  [Y2_2p, Y2_2p+1, G_2p, G_2p+1]
+// with Y = 2 c kappa y' (zero past d) and G as above; padding columns have
+// Y = 0, G = -inf and add nothing. So column c's data starts at float4 c (c
+// even) and a chunk of 256 columns is 256 float4 (4 KB of shared memory).
+// Rows: thread t of a tile owns rows t + 128 k, k < 8.
+template <int D>
+__global__ void __launch_bounds__(kHsThreads, 3) hs_lowd_kernel(HalfStep A) {
+    __shared__ __align__(16) float4 sm[2][kHsChunk];
+    __shared__ double s_red[kHsThreads / 32];
+    __shared__ int s_flag;
+    if (ld_volatile(&A.st->stop)) return;
+    const int tid = threadIdx.x;
+    const int64_t n_items = (int64_t)A.tiles * A.splits;
+    const float4 *rt4 = reinterpret_cast<const float4 *>(A.rowtab);
+
+    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int tile = (int)(item / A.splits);
+        const int split = (int)(item % A.splits);
+
+        float2 xd[kHsRows][3];
+        float m[kHsRows], tot[kHsRows];
+        float2 nm[kHsRows], acc[kHsRows];
+#pragma unroll
+        for (int k = 0; k < kHsRows; ++k) {
+            const int64_t row = (int64_t)tile * kHsTile + k * kHsThreads + tid;
+            const float4 p = row < A.rows ? rt4[row] : make_float4(0.f, 0.f, 0.f, 0.f);
+            xd[k][0] = make_float2(p.x, p.x);
+            xd[k][1] = make_float2(p.y, p.y);
+            xd[k][2] = make_float2(p.z, p.z);
+            m[k] = kNegBig;
+            nm[k] = make_float2(-kNegBig, -kNegBig);
+            acc[k] = make_float2(0.f, 0.f);
+            tot[k] = 0.f;
+        }
+
+        const int64_t c0 = (int64_t)split * A.cols_per_split;
+        const int64_t span = min(c0 + A.cols_per_split, A.cols_pad) - c0;  // multiple of 8
+        const int nch = (int)((span + kHsChunk - 1) / kHsChunk);
+        const float4 *src = A.coltab + c0;
+        const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 p0 = tid < span ? src[tid] : zero4;
+        float4 p1 = tid + kHsThreads < span ? src[tid + kHsThreads] : zero4;
+
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+            float4 *buf = sm[ch & 1];
+            buf[tid] = p0;
+            buf[tid + kHsThreads] = p1;
+            __syncthreads();
+            const int64_t nb = (int64_t)(ch + 1) * kHsChunk;
+            if (ch + 1 < nch) {
+                p0 = nb + tid < span ? src[nb + tid] : zero4;
+                p1 = nb + kHsThreads + tid < span ? src[nb + kHsThreads + tid] : zero4;
+            }
+            const int ncols = (int)min((int64_t)kHsChunk, span - (int64_t)ch * kHsChunk);
+#pragma unroll 1
+            for (int q = 0; q < ncols; q += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = buf[q + u];
+#pragma unroll
+                for (int k = 0; k < kHsRows; ++k) {
+                    float2 t[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float4 lo = v[2 * p], hi = v[2 * p + 1];
+                        float2 tt = __ffma2_rn(make_float2(lo.x, lo.y), xd[k][0],
+                                               make_float2(hi.z, hi.w));
+                        if (D >= 2) tt = __ffma2_rn(make_float2(lo.z, lo.w), xd[k][1], tt);
+                        if (D >= 3) tt = __ffma2_rn(make_float2(hi.x, hi.y), xd[k][2], tt);
+                        t[p] = tt;
+                    }
+                    const float cm = fmaxf(fmaxf(fmaxf(t[0].x, t[0].y), fmaxf(t[1].x, t[1].y)),
+                                           fmaxf(fmaxf(t[2].x, t[2].y), fmaxf(t[3].x, t[3].y)));
+                    if (cm > m[k] + kLazyMax) {  // rare: refresh the running maximum
+                        const float sc = ex2_approx(m[k] - cm);
+                        acc[k] = __fmul2_rn(acc[k], make_float2(sc, sc));
+                        tot[k] *= sc;
+                        m[k] = cm;
+                        nm[k] = make_float2(-cm, -cm);
+                    }
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 u = __fadd2_rn(t[p], nm[k]);
+                        acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u.x), ex2_approx(u.y)));
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kHsRows; ++k) {
+                tot[k] += acc[k].x + acc[k].y;
+                acc[k] = make_float2(0.f, 0.f);
+            }
+        }
+
+        const int64_t stride = (int64_t)A.tiles * kHsTile;
+#pragma unroll
+        for (int k = 0; k < kHsRows; ++k) {
+            const int64_t row = (int64_t)tile * kHsTile + k * kHsThreads + tid;
+            if (row < A.rows) A.part[split * stride + row] = make_float2(m[k], tot[k]);
+        }
+        finish_tile<kHsThreads, kHsTile>(A, tile, s_red, &s_flag);
+        __syncthreads();
+    }
+}
+
+// --------------------------------------------------------- generic-d path
+// For 3 < d <= 64 (CUDA-core FMA path). Column table: per column DP + 4
+// floats, [Y_0 .. Y_{DP-1}, G, 0, 0, 0] (Y = 2 c kappa y', zero past d). Row
+// table: [rows][DP] floats x' (zero past d). Thread t owns rows t and t + 128
+// of the tile; the dot products run as packed f32x2 FMAs over coordinate pairs.
+template <int DP>
+__global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
+    constexpr int ST = DP + 4;
+    constexpr int CH4 = kGnChunk * ST / 4;  // float4 per chunk
+    __shared__ __align__(16) float4 sm[2][CH4];
+    __shared__ double s_red[kGnThreads / 32];
+    __shared__ int s_flag;
+    if (ld_volatile(&A.st->stop)) return;
+    const int tid = threadIdx.x;
+    const int64_t n_items = (int64_t)A.tiles * A.splits;
+
+    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int tile = (int)(item / A.splits);
+        const int split = (int)(item % A.splits);
+
+        float2 xp[kGnRows][DP / 2];
+        float m[kGnRows], tot[kGnRows];
+        float2 acc[kGnRows];
+#pragma unroll
+        for (int k = 0; k < kGnRows; ++k) {
+            const int64_t row = (int64_t)tile * kGnTile + k * kGnThreads + tid;
+            const float2 *src = reinterpret_cast<const float2 *>(A.rowtab + row * (int64_t)DP);
+#pragma unroll
+            for (int q = 0; q < DP / 2; ++q) xp[k][q] = row < A.rows ? src[q] : make_float2(0.f, 0.f);
+            m[k] = kNegBig;
+            acc[k] = make_float2(0.f, 0.f);
+            tot[k] = 0.f;
+        }
+
+        const int64_t c0 = (int64_t)split * A.cols_per_split;
+        const int64_t span = min(c0 + A.cols_per_split, A.cols_pad) - c0;  // multiple of 8
+        const int nch = (int)((span + kGnChunk - 1) / kGnChunk);
+        const float4 *src = A.coltab + c0 * (ST / 4);
+
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+            float4 *buf = sm[ch & 1];
+            const int ncols = (int)min((int64_t)kGnChunk, span - (int64_t)ch * kGnChunk);
+            for (int u = tid; u < ncols * (ST / 4); u += kGnThreads) buf[u] = src[(int64_t)ch * CH4 + u];
+            __syncthreads();
+            const float *bf = reinterpret_cast<const float *>(buf);
+#pragma unroll 1
+            for (int j = 0; j < ncols; j += 4) {
+#pragma unroll
+                for (int k = 0; k < kGnRows; ++k) {
+                    float t[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 *col = reinterpret_cast<const float4 *>(bf + (j + u) * ST);
+                        float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int q = 0; q < DP / 4; ++q) {
+                            const float4 yv = col[q];
+                            s = __ffma2_rn(xp[k][2 * q], make_float2(yv.x, yv.y), s);
+                            s = __ffma2_rn(xp[k][2 * q + 1], make_float2(yv.z, yv.w), s);
+                        }
+                        t[u] = bf[(j + u) * ST + DP] + (s.x + s.y);
+                    }
+                    const float cm = fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3]));
+                    if (cm > m[k] + kLazyMax) {
+                        const float sc = ex2_approx(m[k] - cm);
+                        acc[k] = __fmul2_rn(acc[k], make_float2(sc, sc));
+                        tot[k] *= sc;
+                        m[k] = cm;
+                    }
+                    const float2 nm = make_float2(-m[k], -m[k]);
+                    const float2 u0 = __fadd2_rn(make_float2(t[0], t[1]), nm);
+                    const float2 u1 = __fadd2_rn(make_float2(t[2], t[3]), nm);
+                    acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
+                    acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u1.x), ex2_approx(u1.y)));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kGnRows; ++k) {
+                tot[k] += acc[k].x + acc[k].y;
+                acc[k] = make_float2(0.f, 0.f);
+            }
+            __syncthreads();
+        }
+
+        const int64_t stride = (int64_t)A.tiles * kGnTile;
+#pragma unroll
+        for (int k = 0; k < kGnRows; ++k) {
+            const int64_t row = (int64_t)tile * kGnTile + k * kGnThreads + tid;
+            if (row < A.rows) A.part[split * stride + row] = make_float2(m[k], tot[k]);
+        }
+        finish_tile<kGnThreads, kGnTile>(A, tile, s_red, &s_flag);
+        __syncthreads();
+    }
+}
+
+// ----------------------------------------------------------------- launchers
+// kind 0: low-d (dim = d in 1..3); kind 1: generic (dim = DP in {8,16,32,64}).
+static const void *halfstep_fn(int kind, int dim) {
+    if (kind == 0) {
+        if (dim == 1) return (const void *)hs_lowd_kernel<1>;
+        if (dim == 2) return (const void *)hs_lowd_kernel<2>;
+        return (const void *)hs_lowd_kernel<3>;
+    }
+    if (dim == 8) return (const void *)hs_generic_kernel<8>;
+    if (dim == 16) return (const void *)hs_generic_kernel<16>;
+    if (dim == 32) return (const void *)hs_generic_kernel<32>;
+    return (const void *)hs_generic_kernel<64>;
+}
+
+int halfstep_blocks_per_sm(int kind, int dim) {
+    int nb = 0;
+    const int threads = kind == 0 ? kHsThreads : kGnThreads;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, halfstep_fn(kind, dim), threads, 0) !=
+        cudaSuccess)
+        return 0;
+    return nb;
+}
+
+cudaError_t launch_halfstep(int kind, int dim, const HalfStep &A, int grid, cudaStream_t s) {
+    const int threads = kind == 0 ? kHsThreads : kGnThreads;
+    void *args[] = {(void *)&A};
+    return cudaLaunchKernel(halfstep_fn(kind, dim), dim3(grid), dim3(threads), args, 0, s);
+}
+
+}  // namespace ot

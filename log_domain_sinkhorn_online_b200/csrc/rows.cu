@@ -1,0 +1,354 @@
+// rows.cu -- plan entries: row materializer, exact min_row, marginal residual.
+//
+// Every entry of the plan is T_ij = exp((f_i + g_j - C_ij)/eps) (moscot PR
+// #846, "materialize transport-matrix rows instead of pushing indicator
+// columns", section Fix), produced by ONE device function, plan_entry(), so the
+// min_row threshold and the values it is compared with come from the same
+// float path ("Behavioural changes": the old threshold and values came from two
+// paths and could empty a row).
+//
+// Precision. In base 2 with kappa = log2(e)/eps and the shifted coordinates
+// x' = x - o, y' = y - o held in float64:
+//   e2_ij = A_i + B_j + sum_q P_iq y'_jq,
+//   A_i = kappa (f_i - c |x'_i|^2), B_j = kappa (g_j - c |y'_j|^2), P_i = 2 c kappa x'_i,
+// all in float64 (FlashSinkhorn 2, section D.3: accurate evaluation is done in
+// FP64). Then e2 = k + r with k = rint(e2), |r| <= 1/2; T = 2^r (MUFU ex2 on
+// the float r, relative error ~2^-22) scaled by 2^k through the exponent
+// field, with a two-step scaling into the subnormal range. A massless side
+// (potential -inf) gives e2 = -inf and T = 0.
+#include "runtime.h"
+
+namespace ot {
+
+__device__ __forceinline__ float exp2_split(double e2) {
+    if (!(e2 > -152.0)) return 0.0f;          // below half the smallest subnormal
+    if (e2 >= 128.0) return INFINITY;
+    const int k = __double2int_rn(e2);
+    const float p = ex2_approx((float)(e2 - (double)k));  // in [2^-1/2, 2^1/2]
+    if (k >= -125) return __int_as_float(__float_as_int(p) + (k << 23));
+    return p * __int_as_float((k + 64 + 127) << 23) * 5.42101086242752217e-20f;  // * 2^-64
+}
+
+// the one float path for a plan entry: row data (A, P[d]), column data (y'[d], B)
+template <int D>
+__device__ __forceinline__ float plan_entry(double A, const double *P, const double *col, int d) {
+    const int dd = D > 0 ? D : d;
+    double s = A + col[dd];
+#pragma unroll
+    for (int q = 0; q < (D > 0 ? D : 1); ++q) {
+        if (D > 0) s = fma(P[q], col[q], s);
+    }
+    if (D == 0)
+        for (int q = 0; q < dd; ++q) s = fma(P[q], col[q], s);
+    return exp2_split(s);
+}
+
+// Column table in float64: dcol[j*(d+1) + q] = y'_jq (q < d), dcol[j*(d+1) + d] = B_j.
+__global__ void build_dcol_kernel(const float *__restrict__ p, const float *__restrict__ pot,
+                                  int64_t cnt, int d, const double *__restrict__ o,
+                                  const Params *__restrict__ prm, double *dcol) {
+    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= cnt) return;
+    const double kappa = prm->kappa, c = prm->c;
+    double nrm = 0.0;
+    for (int q = 0; q < d; ++q) {
+        const double v = (double)p[j * d + q] - o[q];
+        dcol[j * (d + 1) + q] = v;
+        nrm += v * v;
+    }
+    const float pv = pot[j];
+    dcol[j * (d + 1) + d] = (pv == -INFINITY) ? -INFINITY : kappa * ((double)pv - c * nrm);
+}
+
+// Row data of one row into shared memory: A and P (d values).
+__device__ __forceinline__ void load_row(const float *pts, const float *pot, int64_t i, int d,
+                                         const double *o, double kappa, double c, double *A,
+                                         double *P) {
+    double nrm = 0.0;
+    for (int q = 0; q < d; ++q) {
+        const double v = (double)pts[i * d + q] - o[q];
+        P[q] = 2.0 * c * kappa * v;
+        nrm += v * v;
+    }
+    const float pv = pot[i];
+    *A = (pv == -INFINITY) ? -INFINITY : kappa * ((double)pv - c * nrm);
+}
+
+// ------------------------------------------------------------ materializer
+// Block: 256 threads x 4 consecutive columns (1024 columns) x 16 rows of the
+// row list. Each thread keeps its 4 columns' float64 data in registers (d <= 3)
+// and streams 16 rows of float4 evict-first stores, coalesced per warp.
+constexpr int kMtThreads = 256, kMtRows = 16;
+
+
+template <int D>
+__global__ void __launch_bounds__(kMtThreads) materialize_kernel(MatArgs M) {
+    __shared__ double sA[kMtRows], sP[kMtRows][D > 0 ? D : kMaxD];
+    __shared__ int sValid[kMtRows];
+    const int tid = threadIdx.x;
+    const int64_t r0 = (int64_t)blockIdx.y * kMtRows;
+    const int d = D > 0 ? D : M.d;
+    if (tid < kMtRows) {
+        const int64_t r = r0 + tid;
+        int ok = 0;
+        if (r < M.k) {
+            const int64_t i = M.row_idx[r];
+            if (i >= 0 && i < M.n) {
+                ok = 1;
+                load_row(M.x, M.f, i, d, M.o, M.prm->kappa, M.prm->c, &sA[tid], sP[tid]);
+            } else {
+                atomicExch(M.bad, 1);
+            }
+        }
+        sValid[tid] = ok;
+    }
+    __syncthreads();
+    const int64_t j0 = ((int64_t)blockIdx.x * kMtThreads + tid) * 4;
+    if (j0 >= M.m) return;
+    const int ncol = (int)min((int64_t)4, M.m - j0);
+    constexpr int DS = (D > 0 ? D : 1) + 1;
+    double cd[4][DS];
+    if (D > 0) {
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int q = 0; q < DS; ++q)
+                cd[u][q] = u < ncol ? M.dcol[(j0 + u) * DS + q] : -INFINITY;
+    }
+    for (int rr = 0; rr < kMtRows; ++rr) {
+        if (!sValid[rr]) continue;
+        const int64_t r = r0 + rr;
+        float t[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (D > 0)
+                t[u] = u < ncol ? plan_entry<D>(sA[rr], sP[rr], cd[u], d) : 0.0f;
+            else
+                t[u] = u < ncol ? plan_entry<0>(sA[rr], sP[rr], M.dcol + (j0 + u) * (d + 1), d)
+                                : 0.0f;
+        }
+        float *dst = M.out + r * M.m + j0;
+        if (M.vec && ncol == 4) {
+            __stcs(reinterpret_cast<float4 *>(dst), make_float4(t[0], t[1], t[2], t[3]));
+        } else {
+            for (int u = 0; u < ncol; ++u) __stcs(dst + u, t[u]);
+        }
+    }
+}
+
+// ------------------------------------------------------- row-complete passes
+// A block owns 8 rows and visits every column, so each row's reduction stays
+// in one block and is done in a fixed order (deterministic):
+//   OP_MAX:   rowmax[i] = max_j T_ij                       (min_row, pass A)
+//   OP_COUNT: counts[i] = #{j : T_ij >= thr} if w_i > 0    (min_row, pass B)
+//   OP_SUM:   part[block] = sum over its rows of |sum_j T_ij - w_i|  (residual)
+// "Rows" may be either cloud: the column residual runs the same pass with the
+// roles of (x, f, a) and (y, g, b) swapped, since T is symmetric in them.
+enum { OP_MAX = 0, OP_COUNT = 1, OP_SUM = 2 };
+constexpr int kRpThreads = 256, kRpRows = 8;
+
+
+template <int D, int OP>
+__global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
+    __shared__ double sA[kRpRows], sP[kRpRows][D > 0 ? D : kMaxD];
+    __shared__ double sRed[kRpThreads / 32][kRpRows];
+    const int tid = threadIdx.x;
+    const int64_t r0 = R.row_begin + (int64_t)blockIdx.x * kRpRows;
+    const int d = D > 0 ? D : R.d;
+    if (tid < kRpRows) {
+        const int64_t i = r0 + tid;
+        if (i < R.row_end)
+            load_row(R.pts, R.pot, i, d, R.o, R.prm->kappa, R.prm->c, &sA[tid], sP[tid]);
+        else
+            sA[tid] = -INFINITY;
+    }
+    __syncthreads();
+    double acc[kRpRows];
+#pragma unroll
+    for (int r = 0; r < kRpRows; ++r) acc[r] = OP == OP_MAX ? -1.0 : 0.0;
+    constexpr int DS = (D > 0 ? D : 1) + 1;
+    for (int64_t j = tid; j < R.cols; j += kRpThreads) {
+        double cd[DS];
+        const double *col = R.dcol + j * (d + 1);
+        if (D > 0) {
+#pragma unroll
+            for (int q = 0; q < DS; ++q) cd[q] = col[q];
+        }
+#pragma unroll
+        for (int r = 0; r < kRpRows; ++r) {
+            const float t = D > 0 ? plan_entry<D>(sA[r], sP[r], cd, d)
+                                  : plan_entry<0>(sA[r], sP[r], col, d);
+            if (OP == OP_MAX) acc[r] = fmax(acc[r], (double)t);
+            if (OP == OP_COUNT) acc[r] += (t >= R.thr) ? 1.0 : 0.0;
+            if (OP == OP_SUM) acc[r] += (double)t;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kRpRows; ++r) {
+        double v = acc[r];
+        for (int off = 16; off > 0; off >>= 1) {
+            const double o2 = __shfl_xor_sync(0xffffffffu, v, off);
+            v = OP == OP_MAX ? fmax(v, o2) : v + o2;
+        }
+        if ((tid & 31) == 0) sRed[tid >> 5][r] = v;
+    }
+    __syncthreads();
+    if (tid < kRpRows) {
+        double v = sRed[0][tid];
+        for (int w = 1; w < kRpThreads / 32; ++w) v = OP == OP_MAX ? fmax(v, sRed[w][tid]) : v + sRed[w][tid];
+        const int64_t i = r0 + tid;
+        if (i < R.row_end) {
+            const float wi = R.w[i];
+            if (OP == OP_MAX) R.rowmax[i] = (float)v;
+            if (OP == OP_COUNT) R.counts[i] = wi > 0.0f ? (int64_t)v : 0;
+            if (OP == OP_SUM) sRed[0][tid] = fabs(v - (double)wi);
+        } else if (OP == OP_SUM) {
+            sRed[0][tid] = 0.0;
+        }
+    }
+    if (OP == OP_SUM) {
+        __syncthreads();
+        if (tid == 0) {
+            double t = 0.0;
+            for (int r = 0; r < kRpRows; ++r) t += sRed[0][r];
+            R.part[blockIdx.x] = t;
+        }
+    }
+}
+
+// ------------------------------------------------------------ reductions
+// min over massful rows of rowmax (smallest index on ties), number of massless
+// rows and (after the count pass) nnz. One block; fixed order per thread, then
+// a fixed tree, so the result does not depend on timing.
+constexpr int kRedThreads = 1024;
+
+__global__ void __launch_bounds__(kRedThreads) min_row_reduce_kernel(const float *rowmax,
+                                                                     const float *w, int64_t n,
+                                                                     float *thr,
+                                                                     int64_t *argmin,
+                                                                     int64_t *n_massless) {
+    __shared__ float sv[kRedThreads];
+    __shared__ int64_t si[kRedThreads], sc[kRedThreads];
+    const int tid = threadIdx.x;
+    float best = INFINITY;
+    int64_t bi = -1, nm = 0;
+    for (int64_t i = tid; i < n; i += kRedThreads) {
+        if (w[i] > 0.0f) {
+            const float v = rowmax[i];
+            if (v < best) {
+                best = v;
+                bi = i;
+            }
+        } else {
+            ++nm;
+        }
+    }
+    sv[tid] = best;
+    si[tid] = bi;
+    sc[tid] = nm;
+    __syncthreads();
+    for (int s = kRedThreads / 2; s > 0; s >>= 1) {
+        if (tid < s) {
+            const float v2 = sv[tid + s];
+            const int64_t i2 = si[tid + s];
+            if (i2 >= 0 && (si[tid] < 0 || v2 < sv[tid] || (v2 == sv[tid] && i2 < si[tid]))) {
+                sv[tid] = v2;
+                si[tid] = i2;
+            }
+            sc[tid] += sc[tid + s];
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        *thr = sv[0];
+        *argmin = si[0];
+        *n_massless = sc[0];
+    }
+}
+
+// out = sum of v[0..cnt) for int64 (exact) or double (fixed order).
+template <typename T>
+__global__ void __launch_bounds__(kRedThreads) sum_kernel(const T *v, int64_t cnt, T *out) {
+    __shared__ T s[kRedThreads];
+    const int tid = threadIdx.x;
+    T acc = 0;
+    for (int64_t i = tid; i < cnt; i += kRedThreads) acc += v[i];
+    s[tid] = acc;
+    __syncthreads();
+    for (int st = kRedThreads / 2; st > 0; st >>= 1) {
+        if (tid < st) s[tid] += s[tid + st];
+        __syncthreads();
+    }
+    if (tid == 0) *out = s[0];
+}
+
+
+// ----------------------------------------------------------------- launchers
+cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, const double *o,
+                        const Params *prm, double *dcol, cudaStream_t s) {
+    if (cnt <= 0) return cudaSuccess;
+    build_dcol_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, s>>>(p, pot, cnt, d, o, prm, dcol);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s) {
+    const int64_t col_blocks = (M.m + kMtThreads * 4 - 1) / (kMtThreads * 4);
+    // at most 65535 row groups per launch: split long row lists
+    const int64_t max_rows = (int64_t)65535 * kMtRows;
+    for (int64_t r = 0; r < M.k; r += max_rows) {
+        MatArgs A = M;
+        A.row_idx = M.row_idx + r;
+        A.out = M.out + r * M.m;
+        A.k = min(max_rows, M.k - r);
+        dim3 grid((unsigned)col_blocks, (unsigned)((A.k + kMtRows - 1) / kMtRows));
+        switch (M.d) {
+            case 1: materialize_kernel<1><<<grid, kMtThreads, 0, s>>>(A); break;
+            case 2: materialize_kernel<2><<<grid, kMtThreads, 0, s>>>(A); break;
+            case 3: materialize_kernel<3><<<grid, kMtThreads, 0, s>>>(A); break;
+            default: materialize_kernel<0><<<grid, kMtThreads, 0, s>>>(A); break;
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <int OP>
+static void rowpass_dispatch(const RowPassArgs &R, unsigned grid, cudaStream_t s) {
+    switch (R.d) {
+        case 1: rowpass_kernel<1, OP><<<grid, kRpThreads, 0, s>>>(R); break;
+        case 2: rowpass_kernel<2, OP><<<grid, kRpThreads, 0, s>>>(R); break;
+        case 3: rowpass_kernel<3, OP><<<grid, kRpThreads, 0, s>>>(R); break;
+        default: rowpass_kernel<0, OP><<<grid, kRpThreads, 0, s>>>(R); break;
+    }
+}
+
+// op: 0 max, 1 count, 2 sum; rows [row_begin, row_end)
+cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s) {
+    const int64_t rows = R.row_end - R.row_begin;
+    if (rows <= 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + kRpRows - 1) / kRpRows);
+    if (op == OP_MAX) rowpass_dispatch<OP_MAX>(R, grid, s);
+    else if (op == OP_COUNT) rowpass_dispatch<OP_COUNT>(R, grid, s);
+    else rowpass_dispatch<OP_SUM>(R, grid, s);
+    return cudaGetLastError();
+}
+
+int64_t rowpass_blocks(int64_t rows) { return (rows + kRpRows - 1) / kRpRows; }
+
+cudaError_t launch_min_row_reduce(const float *rowmax, const float *w, int64_t n, float *thr,
+                                  int64_t *argmin, int64_t *n_massless, cudaStream_t s) {
+    min_row_reduce_kernel<<<1, kRedThreads, 0, s>>>(rowmax, w, n, thr, argmin, n_massless);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sum_i64(const int64_t *v, int64_t cnt, int64_t *out, cudaStream_t s) {
+    sum_kernel<int64_t><<<1, kRedThreads, 0, s>>>(v, cnt, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sum_f64(const double *v, int64_t cnt, double *out, cudaStream_t s) {
+    sum_kernel<double><<<1, kRedThreads, 0, s>>>(v, cnt, out);
+    return cudaGetLastError();
+}
+
+}  // namespace ot

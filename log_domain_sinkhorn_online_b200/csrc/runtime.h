@@ -1,0 +1,55 @@
+// runtime.h -- host-side declarations of the kernel launchers (internal).
+#pragma once
+#include "common.cuh"
+
+namespace ot {
+
+// halfstep.cu
+int halfstep_blocks_per_sm(int kind, int dim);
+cudaError_t launch_halfstep(int kind, int dim, const HalfStep &A, int grid, cudaStream_t s);
+
+// prep.cu
+cudaError_t launch_coord_stats(const float *v, int64_t cnt, int d, double *part, double *part2,
+                               double *out, double *out2, int *flags,
+                               unsigned long long *zero_count, cudaStream_t s);
+cudaError_t launch_max_cost(const float *x, const float *y, int64_t n, int64_t m, int d,
+                            unsigned *out_bits, cudaStream_t s);
+cudaError_t launch_set_params(Params *prm, double eps, double c, double tol, cudaStream_t s);
+cudaError_t launch_reset_state(State *st, cudaStream_t s);
+cudaError_t launch_tables(const float *p, const float *pot, int64_t cnt, int64_t cnt_pad, int d,
+                          int dp, const double *o, const Params *prm, float *rowtab,
+                          float *coltab, int layout, cudaStream_t s);
+
+// rows.cu
+struct MatArgs {
+    const float *x, *f;
+    const double *dcol, *o;
+    const Params *prm;
+    const int64_t *row_idx;
+    int64_t k, n, m;
+    int d, vec;
+    float *out;
+    int *bad;
+};
+struct RowPassArgs {
+    const float *pts, *pot, *w;
+    const double *dcol, *o;
+    const Params *prm;
+    int64_t row_begin, row_end, cols;
+    int d;
+    float thr;
+    float *rowmax;
+    int64_t *counts;
+    double *part;
+};
+cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, const double *o,
+                        const Params *prm, double *dcol, cudaStream_t s);
+cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s);
+cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s);
+int64_t rowpass_blocks(int64_t rows);
+cudaError_t launch_min_row_reduce(const float *rowmax, const float *w, int64_t n, float *thr,
+                                  int64_t *argmin, int64_t *n_massless, cudaStream_t s);
+cudaError_t launch_sum_i64(const int64_t *v, int64_t cnt, int64_t *out, cudaStream_t s);
+cudaError_t launch_sum_f64(const double *v, int64_t cnt, double *out, cudaStream_t s);
+
+}  // namespace ot

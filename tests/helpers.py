@@ -1,0 +1,69 @@
+"""Shared helpers for the GPU parity tests (comparison rules and device transfer).
+
+Tolerances (the readings are listed in the design doc):
+ - potentials: max |f - f_ref| and |g - g_ref| <= 1e-4 * max_ij C_ij (the cost
+   as used, i.e. scaled), -inf at the same (massless) entries;
+ - plan entries at the GPU's potentials: |T - T_ref| <= 1e-5 * T_ref where
+   T_ref >= 1e-30, and T <= 1e-30 where T_ref < 1e-30;
+ - marginal residual at the GPU's potentials: within 1e-5 (absolute; the
+   residual of a unit-mass plan is at most 2);
+ - min_row: thr within 1e-5 relative, the same argmin row, the same kept
+   (i, j) entries except those within 1e-5 relative of thr (counted).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+POT_TOL = 1e-4
+ROW_TOL = 1e-5
+RES_TOL = 1e-5
+TINY = 1e-30
+
+
+def to_dev(w, dev="cuda"):
+    import torch
+    return tuple(torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
+
+
+def max_cost(x, y, c, block=4096):
+    """max_ij c * ||x_i - y_j||^2 in float64 (expansion form, blockwise): only the
+    normaliser of the potential tolerance, so 1e-12 relative is ample."""
+    xd, yd = np.asarray(x, np.float64), np.asarray(y, np.float64)
+    best = 0.0
+    yy = (yd ** 2).sum(1)
+    for i0 in range(0, xd.shape[0], block):
+        xb = xd[i0:i0 + block]
+        dist = (xb ** 2).sum(1)[:, None] + yy[None, :] - 2 * xb @ yd.T
+        best = max(best, float(dist.max()))
+    return c * best
+
+
+def assert_potentials(got, ref, maxc, tol=POT_TOL, what="f"):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    ninf_g, ninf_r = np.isneginf(got), np.isneginf(ref)
+    assert np.array_equal(ninf_g, ninf_r), f"{what}: -inf pattern differs"
+    fin = ~ninf_r
+    assert np.isfinite(got[fin]).all(), f"{what}: non-finite entries"
+    err = np.abs(got[fin] - ref[fin]).max() / maxc if fin.any() else 0.0
+    assert err <= tol, f"{what}: max err {err:.3e} of max C (tol {tol})"
+    return err
+
+
+def assert_entries(T, T_ref, tol=ROW_TOL):
+    T, T_ref = np.asarray(T, np.float64), np.asarray(T_ref, np.float64)
+    big = T_ref >= TINY
+    rel = np.abs(T[big] - T_ref[big]) / T_ref[big]
+    worst = float(rel.max()) if rel.size else 0.0
+    assert worst <= tol, f"plan entries: max rel err {worst:.3e}"
+    assert np.all(T[~big] <= TINY), "entries below 1e-30 in the oracle are not below 1e-30 here"
+    return worst
+
+
+def assert_min_row(got, ref, T_ref_rows=None, rows=None, tol=ROW_TOL):
+    assert got["n_massless"] == ref["n_massless"]
+    if ref["argmin"] < 0:
+        assert got["argmin"] == -1 and np.isinf(got["thr"])
+        return 0
+    assert abs(got["thr"] - ref["thr"]) <= tol * ref["thr"], (got["thr"], ref["thr"])
+    assert got["argmin"] == ref["argmin"]
+    return 0

@@ -1,0 +1,217 @@
+"""GPU parity against the float64 oracle on the same seeded inputs (-m gpu).
+
+Every call goes through the C ABI (via the ctypes binding). Sizes are chosen
+so the oracle finishes in seconds yet the kernels see several row tiles
+(1024 rows), several column splits and ragged tails.
+"""
+import numpy as np
+import pytest
+
+import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ot():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import log_domain_sinkhorn_online_b200 as pkg
+    return pkg
+
+
+@pytest.fixture(scope="module")
+def orc():
+    import oracle
+    oracle.build()
+    return oracle
+
+
+def _solve_both(ot, orc, w, n_iters, tol=0.0, **kw):
+    import torch
+    x, y, a, b = H.to_dev(w)
+    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=n_iters, tol=tol, **kw)
+    torch.cuda.synchronize()
+    c = orc.inv_scale_cost(w.x, w.y, w.scale)
+    assert abs(plan.info.inv_scale_cost - c) <= 2e-7 * c
+    f_ref, g_ref, it_ref, r_ref = orc.sinkhorn(w.x, w.y, w.a, w.b, c, w.eps, n_iters, tol)
+    return plan, c, f_ref, g_ref, it_ref, r_ref
+
+
+def _pots(plan):
+    return plan.f.double().cpu().numpy(), plan.g.double().cpu().numpy()
+
+
+def _cloud(seed, n, m, d, scale="none", eps=0.05):
+    from log_domain_sinkhorn_online_b200.workloads import Workload
+    rng = np.random.default_rng(seed)
+    x = rng.random((n, d)).astype(np.float32)
+    y = (rng.random((m, d)) * 0.8 + 0.15).astype(np.float32)
+    a = (rng.random(n) + 0.5)
+    b = (rng.random(m) + 0.5)
+    return Workload("cloud", x, y, (a / a.sum()).astype(np.float32), (b / b.sum()).astype(np.float32),
+                    eps=eps, scale=scale, n_iters=30)
+
+
+# --------------------------------------------------------------- trajectories
+@pytest.mark.parametrize("d", [1, 2, 3])
+@pytest.mark.parametrize("scale", ["none", "mean", "max_cost"])
+def test_lowd_trajectory_ragged(ot, orc, d, scale):
+    w = _cloud(10 + d, 2085, 1379, d, scale=scale, eps=0.02)
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 25)
+    maxc = H.max_cost(w.x, w.y, c)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+    assert plan.info.iterations == 25
+
+
+@pytest.mark.parametrize("d", [4, 5, 16, 33, 50, 64])
+def test_generic_d_trajectory(ot, orc, d):
+    w = _cloud(30 + d, 611, 530, d, scale="mean", eps=0.05)
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 15)
+    maxc = H.max_cost(w.x, w.y, c)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+
+
+def test_w1_full_workload(ot, orc):
+    """512 x 512 uniform in 2-D, eps 0.05, exactly 200 iterations, all rows, min_row."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w1()
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, w.n_iters)
+    maxc = H.max_cost(w.x, w.y, c)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+    T = plan.materialize_rows(torch.arange(w.n, device="cuda")).double().cpu().numpy()
+    T_ref = orc.dense_plan(w.x, w.y, f, g, c, w.eps)
+    H.assert_entries(T, T_ref)
+    mr = plan.sparsify_min_row()
+    ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)
+    H.assert_min_row(mr, ref)
+    kept = T >= mr["thr"]
+    kept_ref = T_ref >= ref["thr"]
+    band = np.abs(T_ref - ref["thr"]) <= 1e-5 * ref["thr"]
+    assert np.array_equal(kept[~band], kept_ref[~band])
+    assert (kept.sum(1) >= 1).all()
+    assert mr["nnz"] == int(kept.sum())
+    r = plan.marginal_residual()
+    r_ref = orc.marginal_residual(w.x, w.y, w.a, w.b, f, g, c, w.eps)
+    assert abs(r[0] - r_ref[0]) <= H.RES_TOL and abs(r[1] - r_ref[1]) <= H.RES_TOL
+
+
+def test_tol_stopping_counts(ot, orc):
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w2(n=1500, m=1400)
+    plan, c, f_ref, g_ref, it_ref, r_ref = _solve_both(ot, orc, w, 2000, tol=w.tol)
+    maxc = H.max_cost(w.x, w.y, c)
+    assert plan.info.converged == 1 and it_ref < 2000
+    if plan.info.iterations != it_ref:
+        # the residual crossed tol within rounding: rerun both with the oracle's count
+        assert abs(plan.info.iterations - it_ref) <= 2
+        plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, it_ref)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+    assert abs(plan.info.residual - r_ref) <= 1e-3 * max(r_ref, w.tol)
+
+
+def test_massless_rows_and_columns(ot, orc):
+    w = _cloud(5, 1500, 1100, 3, eps=0.03)
+    w.a[[0, 7, 1024, 1499]] = 0.0
+    w.b[[3, 1099]] = 0.0
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 20)
+    assert plan.status == 1 and plan.info.n_massless_rows == 4 and plan.info.n_massless_cols == 2
+    maxc = H.max_cost(w.x, w.y, c)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+    mr = plan.sparsify_min_row(block_rows=333)
+    ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)
+    H.assert_min_row(mr, ref)
+    counts = mr["counts"].cpu().numpy()
+    assert (counts[[0, 7, 1024, 1499]] == 0).all() and (np.delete(counts, [0, 7, 1024, 1499]) >= 1).all()
+
+
+@pytest.mark.parametrize("n,m", [(1, 1), (1, 37), (37, 1), (8, 8), (9, 1031), (1031, 9)])
+def test_tiny_and_degenerate_sizes(ot, orc, n, m):
+    w = _cloud(n * 7 + m, n, m, 3, eps=0.1)
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 10)
+    maxc = max(H.max_cost(w.x, w.y, c), 1e-6)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+
+
+def test_no_graphs_same_result(ot, orc):
+    import torch
+    w = _cloud(77, 1200, 900, 3, eps=0.02)
+    x, y, a, b = H.to_dev(w)
+    p1 = ot.sinkhorn(x, y, a, b, eps=w.eps, n_iters=37, use_graphs=True, check_every=8)
+    p2 = ot.sinkhorn(x, y, a, b, eps=w.eps, n_iters=37, use_graphs=False)
+    torch.cuda.synchronize()
+    assert torch.equal(p1.f, p2.f) and torch.equal(p1.g, p2.g)  # deterministic kernels
+
+
+def test_rows_and_residual_at_gpu_potentials(ot, orc):
+    import torch
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w2(n=3001, m=2777)
+    x, y, a, b = H.to_dev(w)
+    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=60)
+    f, g = _pots(plan)
+    c = plan.info.inv_scale_cost
+    rows = np.array([0, 1, 1023, 1024, 2047, 3000, 5, 5], dtype=np.int64)
+    T = plan.materialize_rows(torch.from_numpy(rows).cuda()).double().cpu().numpy()
+    H.assert_entries(T, orc.materialize_rows(w.x, w.y, f, g, c, w.eps, rows))
+    r = plan.marginal_residual()
+    r_ref = orc.marginal_residual(w.x, w.y, w.a, w.b, f, g, c, w.eps)
+    assert abs(r[0] - r_ref[0]) <= H.RES_TOL and abs(r[1] - r_ref[1]) <= H.RES_TOL
+    ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)
+    outs = [plan.sparsify_min_row(block_rows=br) for br in (1, 64, 1024, 0)]
+    for o in outs:
+        H.assert_min_row(o, ref)
+        assert o["thr"] == outs[0]["thr"] and o["nnz"] == outs[0]["nnz"]
+        assert torch.equal(o["counts"], outs[0]["counts"])
+
+
+def test_bad_row_index_is_reported(ot):
+    import torch
+    w = _cloud(3, 300, 200, 2)
+    x, y, a, b = H.to_dev(w)
+    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, n_iters=3)
+    with pytest.raises(ot.OTError) as e:
+        plan.materialize_rows(torch.tensor([0, 300], device="cuda"))
+    assert e.value.status == -1
+    out = plan.materialize_rows(torch.tensor([299, 0], device="cuda"))
+    assert torch.isfinite(out).all()
+
+
+def test_nonfinite_input_is_reported(ot):
+    w = _cloud(4, 100, 90, 3)
+    w.x[5, 1] = np.nan
+    x, y, a, b = H.to_dev(w)
+    with pytest.raises(ot.OTError) as e:
+        ot.sinkhorn(x, y, a, b, eps=w.eps, n_iters=3)
+    assert e.value.status == -5
+
+
+def test_annealing_matches_oracle(ot, orc):
+    from log_domain_sinkhorn_online_b200 import workloads
+    import torch
+    w = workloads.w4(n=2000)
+    x, y, a, b = H.to_dev(w)
+    eps_t = 0.002
+    plan = ot.sinkhorn(x, y, a, b, eps=eps_t, n_iters=10, eps_init=1.0, eps_decay=0.7,
+                       iters_per_stage=10)
+    torch.cuda.synchronize()
+    f_ref, g_ref, stages, r_ref = orc.sinkhorn_anneal(w.x, w.y, w.a, w.b, 1.0, eps_t, 1.0, 0.7, 10)
+    assert plan.info.stages == stages
+    maxc = H.max_cost(w.x, w.y, 1.0)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
