@@ -68,6 +68,7 @@ struct Side {          // one cloud's half of the problem
     float *coltab;     // layout per kind
     int tiles, splits, grid;
     int64_t cps;       // columns per split of the OTHER side's table
+    int rpt, tile;     // rows per thread and rows per tile of this side's half-step
 };
 
 }  // namespace
@@ -139,11 +140,13 @@ struct Carver {
     }
 };
 
-// Column splits for one half-step: rows -> tiles of `tile`; the column table of
-// `cols_pad` columns is cut into `splits` spans (multiples of kColPad). Picks
-// the split count whose critical path (waves x columns per split) is shortest
-// for `cap` resident blocks, preferring fewer splits on ties.
-void choose_splits(int64_t rows, int64_t cols_pad, int tile, int cap, Side &sd) {
+// Column splits for one half-step: rows -> tiles of `tile` rows; the column
+// table of `cols_pad` columns is cut into `splits` spans (multiples of
+// kColPad). Cost model in column-equivalents of one thread's work: every wave
+// of `cap` resident blocks costs rpt * (cps + 64 per-item overhead), and the
+// block that finishes a tile merges `splits` partials per row (~8 columns
+// each). Returns the estimate of the best split count, which it stores in sd.
+double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd) {
     const int64_t tiles = (rows + tile - 1) / tile;
     double best = 1e300;
     int best_s = 1;
@@ -155,8 +158,7 @@ void choose_splits(int64_t rows, int64_t cols_pad, int tile, int cap, Side &sd) 
         if (s_eff != s) continue;
         const int64_t items = tiles * s_eff;
         const int64_t waves = (items + cap - 1) / cap;
-        // per-item fixed cost ~ 64 columns of work (row loads, partial writes, combine)
-        const double t = (double)waves * (double)(cps + 64);
+        const double t = (double)waves * rpt * (double)(cps + 64) + 8.0 * rpt * (double)s_eff;
         if (t < best * 0.995) {
             best = t;
             best_s = (int)s_eff;
@@ -167,6 +169,35 @@ void choose_splits(int64_t rows, int64_t cols_pad, int tile, int cap, Side &sd) 
     sd.splits = best_s;
     sd.cps = best_cps;
     sd.grid = (int)std::min<int64_t>(tiles * best_s, cap);
+    sd.rpt = rpt;
+    sd.tile = tile;
+    return best;
+}
+
+// Launch shape of one side's half-step: for d <= 3 also picks the rows per
+// thread (8, 4 or 2) with the smallest estimate.
+int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Side &sd) {
+    if (kind == 1) {
+        const int bps = halfstep_blocks_per_sm(1, dim, kGnRows);
+        if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
+        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd);
+        return OT_OK;
+    }
+    double best = 1e300;
+    for (int rpt : {8, 4, 2}) {
+        const int bps = halfstep_blocks_per_sm(0, dim, rpt);
+        if (bps <= 0) continue;
+        Side tmp = sd;
+        // fewer rows per thread re-read the shared column data more often
+        const double eff = rpt == 2 ? 0.9 : 1.0;
+        const double t = choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp) / eff;
+        if (t < best) {
+            best = t;
+            sd = tmp;
+        }
+    }
+    if (best >= 1e300) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
+    return OT_OK;
 }
 
 }  // namespace
@@ -231,9 +262,11 @@ cudaError_t mark(ot_plan *p) {
 }
 
 cudaError_t launch_iteration(const ot_plan *p, int parity) {
-    cudaError_t e = launch_halfstep(p->kind, p->dim, make_step(p, 0, parity), p->sx.grid, p->s_int);
+    cudaError_t e = launch_halfstep(p->kind, p->dim, p->sx.rpt, make_step(p, 0, parity),
+                                    p->sx.grid, p->s_int);
     if (e != cudaSuccess) return e;
-    return launch_halfstep(p->kind, p->dim, make_step(p, 1, parity), p->sy.grid, p->s_int);
+    return launch_halfstep(p->kind, p->dim, p->sy.rpt, make_step(p, 1, parity), p->sy.grid,
+                           p->s_int);
 }
 
 // Runs `iters` iterations starting at global parity `parity0`, in chunks of
@@ -327,19 +360,16 @@ int plan_setup(ot_plan *p) {
         p->dim = p->d <= 8 ? 8 : p->d <= 16 ? 16 : p->d <= 32 ? 32 : 64;
         p->dp = p->dim;
     }
-    const int tile = p->kind == 0 ? kHsTile : kGnTile;
     const int64_t colw = p->kind == 0 ? 4 : p->dp + 4;
     p->sx.cnt = p->n;
     p->sy.cnt = p->m;
     p->sx.pad = round_up(p->n, kColPad);
     p->sy.pad = round_up(p->m, kColPad);
-    const int bps = halfstep_blocks_per_sm(p->kind, p->dim);
-    if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
-    const int cap = bps * p->sm_count;
-    choose_splits(p->n, p->sy.pad, tile, cap, p->sx);
-    choose_splits(p->m, p->sx.pad, tile, cap, p->sy);
-    const int64_t part_cnt = std::max((int64_t)p->sx.splits * p->sx.tiles,
-                                      (int64_t)p->sy.splits * p->sy.tiles) * tile;
+    int rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx);
+    if (rc != OT_OK) return rc;
+    if ((rc = choose_shape(p->kind, p->dim, p->sm_count, p->m, p->sx.pad, p->sy)) != OT_OK) return rc;
+    const int64_t part_cnt = std::max((int64_t)p->sx.splits * p->sx.tiles * p->sx.tile,
+                                      (int64_t)p->sy.splits * p->sy.tiles * p->sy.tile);
     const int64_t tiles = std::max(p->sx.tiles, p->sy.tiles);
 
     for (int pass = 0; pass < 2; ++pass) {
@@ -529,7 +559,8 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
             } else if (iters > 0) {
                 // one more f-update measures ||T1 - a||_1 of the final state
                 OT_CU(mark(p));
-                OT_CU(launch_halfstep(p->kind, p->dim, make_step(p, 0, t & 1), p->sx.grid, p->s_int));
+                OT_CU(launch_halfstep(p->kind, p->dim, p->sx.rpt, make_step(p, 0, t & 1), p->sx.grid,
+                                      p->s_int));
                 OT_CU(mark(p));
                 p->launches += 1;
                 half_steps += 1;

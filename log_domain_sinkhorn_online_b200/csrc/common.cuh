@@ -11,11 +11,10 @@ constexpr int kMaxD = 64;            // largest point dimension this build suppo
 constexpr double kLog2e = 1.4426950408889634073599246810019;
 constexpr double kLn2 = 0.69314718055994530941723212145818;
 
-// Low-d half-step tiling: 128 threads x 8 rows each = 1024 rows per tile; the
-// column table is streamed through shared memory 256 columns at a time.
+// Low-d half-step tiling: 128 threads x R rows each (R = 2, 4 or 8, chosen per
+// problem); the column table is streamed through shared memory 256 columns at
+// a time.
 constexpr int kHsThreads = 128;
-constexpr int kHsRows = 8;
-constexpr int kHsTile = kHsThreads * kHsRows;
 constexpr int kHsChunk = 256;
 
 // Generic-d half-step tiling: 128 threads x 2 rows, 64-column chunks.

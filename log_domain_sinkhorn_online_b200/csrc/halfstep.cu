@@ -50,12 +50,32 @@ __device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_f
     for (int k = 0; k < TILE / THREADS; ++k) {
         const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
         if (row >= A.rows) continue;
+        // merge the splits' (max, sum) pairs 8 at a time (independent loads in flight)
         float M = kNegBig;
-        for (int s = 0; s < A.splits; ++s) M = fmaxf(M, __ldcg(&A.part[s * stride + row]).x);
         double S = 0.0;
-        for (int s = 0; s < A.splits; ++s) {
-            float2 p = __ldcg(&A.part[s * stride + row]);
-            if (p.y > 0.0f) S += (double)p.y * exp2((double)p.x - (double)M);
+        int s = 0;
+        for (; s + 8 <= A.splits; s += 8) {
+            float2 pp[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pp[u] = __ldcg(&A.part[(s + u) * stride + row]);
+            float bm = pp[0].x;
+#pragma unroll
+            for (int u = 1; u < 8; ++u) bm = fmaxf(bm, pp[u].x);
+            if (bm > M) {
+                S *= (double)ex2_approx(M - bm);
+                M = bm;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (pp[u].y > 0.0f) S += (double)pp[u].y * (double)ex2_approx(pp[u].x - M);
+        }
+        for (; s < A.splits; ++s) {
+            const float2 pp = __ldcg(&A.part[s * stride + row]);
+            if (pp.x > M) {
+                S *= (double)ex2_approx(M - pp.x);
+                M = pp.x;
+            }
+            if (pp.y > 0.0f) S += (double)pp.y * (double)ex2_approx(pp.x - M);
         }
         const float *xr = A.rowtab + row * (int64_t)A.dp;
         double nrm = 0.0;
@@ -125,9 +145,13 @@ __device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_f
 // with Y = 2 c kappa y' (zero past d) and G as above; padding columns have
 // Y = 0, G = -inf and add nothing. So column c's data starts at float4 c (c
 // even) and a chunk of 256 columns is 256 float4 (4 KB of shared memory).
-// Rows: thread t of a tile owns rows t + 128 k, k < 8.
-template <int D>
-__global__ void __launch_bounds__(kHsThreads, 3) hs_lowd_kernel(HalfStep A) {
+// Rows: thread t of a tile owns rows t + 128 k, k < R (R = 2, 4 or 8; the tile
+// is 128 R rows: fewer rows per thread give more tiles, hence fewer column
+// splits to merge, on small problems).
+template <int D, int R>
+__global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : 4) hs_lowd_kernel(HalfStep A) {
+    constexpr int kHsRows = R;
+    constexpr int kHsTile = kHsThreads * R;
     __shared__ __align__(16) float4 sm[2][kHsChunk];
     __shared__ double s_red[kHsThreads / 32];
     __shared__ int s_flag;
@@ -324,32 +348,37 @@ __global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
 }
 
 // ----------------------------------------------------------------- launchers
-// kind 0: low-d (dim = d in 1..3); kind 1: generic (dim = DP in {8,16,32,64}).
-static const void *halfstep_fn(int kind, int dim) {
-    if (kind == 0) {
-        if (dim == 1) return (const void *)hs_lowd_kernel<1>;
-        if (dim == 2) return (const void *)hs_lowd_kernel<2>;
-        return (const void *)hs_lowd_kernel<3>;
-    }
+template <int R>
+static const void *lowd_fn(int dim) {
+    if (dim == 1) return (const void *)hs_lowd_kernel<1, R>;
+    if (dim == 2) return (const void *)hs_lowd_kernel<2, R>;
+    return (const void *)hs_lowd_kernel<3, R>;
+}
+
+// kind 0: low-d (dim = d in 1..3, rpt = rows per thread 2/4/8);
+// kind 1: generic (dim = DP in {8,16,32,64}, rpt ignored).
+static const void *halfstep_fn(int kind, int dim, int rpt) {
+    if (kind == 0) return rpt == 8 ? lowd_fn<8>(dim) : rpt == 4 ? lowd_fn<4>(dim) : lowd_fn<2>(dim);
     if (dim == 8) return (const void *)hs_generic_kernel<8>;
     if (dim == 16) return (const void *)hs_generic_kernel<16>;
     if (dim == 32) return (const void *)hs_generic_kernel<32>;
     return (const void *)hs_generic_kernel<64>;
 }
 
-int halfstep_blocks_per_sm(int kind, int dim) {
+int halfstep_blocks_per_sm(int kind, int dim, int rpt) {
     int nb = 0;
     const int threads = kind == 0 ? kHsThreads : kGnThreads;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, halfstep_fn(kind, dim), threads, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, halfstep_fn(kind, dim, rpt), threads, 0) !=
         cudaSuccess)
         return 0;
     return nb;
 }
 
-cudaError_t launch_halfstep(int kind, int dim, const HalfStep &A, int grid, cudaStream_t s) {
+cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,
+                            cudaStream_t s) {
     const int threads = kind == 0 ? kHsThreads : kGnThreads;
     void *args[] = {(void *)&A};
-    return cudaLaunchKernel(halfstep_fn(kind, dim), dim3(grid), dim3(threads), args, 0, s);
+    return cudaLaunchKernel(halfstep_fn(kind, dim, rpt), dim3(grid), dim3(threads), args, 0, s);
 }
 
 }  // namespace ot

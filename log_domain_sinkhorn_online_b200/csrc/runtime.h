@@ -5,8 +5,9 @@
 namespace ot {
 
 // halfstep.cu
-int halfstep_blocks_per_sm(int kind, int dim);
-cudaError_t launch_halfstep(int kind, int dim, const HalfStep &A, int grid, cudaStream_t s);
+int halfstep_blocks_per_sm(int kind, int dim, int rpt);
+cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,
+                            cudaStream_t s);
 
 // prep.cu
 cudaError_t launch_coord_stats(const float *v, int64_t cnt, int d, double *part, double *part2,
