@@ -188,6 +188,34 @@ OT_API int ot_sparsify_min_row(const ot_plan *plan, int64_t block_rows, float *t
                         int64_t *row_counts, int64_t *nnz_out, int64_t *n_massless_out,
                         int64_t *argmin_out, void *stream);
 
+/* ------------------------------------------- ot_marginal_residual_noalloc
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory when they need a residual -- a process
+ * whose device memory is wholly owned by another allocator (a framework's
+ * caching pool, or a budget fixed at start-up), or a tight loop in which a
+ * cudaMalloc/cudaFree would stall every stream on the device. It returns the
+ * same two sums as ot_marginal_residual, at the given f, g, without a plan and
+ * without allocating anything: its scratch is a fixed array of
+ * OT_NOALLOC_MAX_POINTS/8 + 2 doubles (1 MiB) in the library's device image,
+ * which every device that loads the library keeps until the process exits.
+ *  x [n,d], y [m,d], a [n], b [m], f [n], g [m]: device float32, caller-owned.
+ *  eps > 0 and inv_scale_cost > 0: the resolved values (e.g. ot_info.eps and
+ *      ot_info.inv_scale_cost of the solve), so that C = inv_scale_cost*|x-y|^2.
+ *  row_l1, col_l1: host doubles (either may be NULL).
+ * n or m above OT_NOALLOC_MAX_POINTS returns OT_ERR_UNSUPPORTED with a message.
+ * The first call on a device looks up the scratch's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls on a device share the scratch and each call overwrites
+ * every slot it reads, so nothing carries over from the previous call; but
+ * calls whose GPU work overlaps (e.g. from two host threads on two streams)
+ * race on it. Synchronises `stream`. Calls no allocating routine.           */
+#define OT_NOALLOC_MAX_POINTS (1 << 20)
+OT_API int ot_marginal_residual_noalloc(const float *x, const float *y, const float *a,
+                                        const float *b, const float *f, const float *g,
+                                        int64_t n, int64_t m, int32_t d, double eps,
+                                        double inv_scale_cost, double *row_l1, double *col_l1,
+                                        void *stream);
+
 /* Frees the plan's workspace (NULL is a no-op). Does not touch borrowed arrays. */
 OT_API void ot_plan_destroy(ot_plan *plan);
 

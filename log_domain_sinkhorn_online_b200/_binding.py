@@ -28,7 +28,9 @@ OT_SCALE_NONE, OT_SCALE_MEAN, OT_SCALE_MAX_COST, OT_SCALE_VALUE = 0, 1, 2, 3
 
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sinkhorn_pointcloud",
-            "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy")
+            "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy",
+            "ot_marginal_residual_noalloc")
+OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
 class OtOptions(ctypes.Structure):
@@ -82,6 +84,9 @@ def lib() -> ctypes.CDLL:
                                               ctypes.POINTER(I64), ctypes.POINTER(I64),
                                               ctypes.POINTER(I64), P]
             L.ot_sparsify_min_row.restype = ctypes.c_int
+            L.ot_marginal_residual_noalloc.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D,
+                                                       ctypes.POINTER(D), ctypes.POINTER(D), P]
+            L.ot_marginal_residual_noalloc.restype = ctypes.c_int
             L.ot_plan_destroy.argtypes = [P]
             L.ot_plan_destroy.restype = None
             _lib = L
@@ -140,6 +145,14 @@ def ot_sparsify_min_row(plan, block_rows, row_counts, stream):
                                           ctypes.byref(nnz), ctypes.byref(nm), ctypes.byref(arg),
                                           stream))
     return st, thr.value, nnz.value, nm.value, arg.value
+
+
+def ot_marginal_residual_noalloc(x, y, a, b, f, g, n, m, d, eps, inv_scale_cost, stream):
+    """Returns (status, row_l1, col_l1); allocates nothing (see the header)."""
+    r, c = ctypes.c_double(), ctypes.c_double()
+    st = _check(lib().ot_marginal_residual_noalloc(x, y, a, b, f, g, n, m, d, eps, inv_scale_cost,
+                                                   ctypes.byref(r), ctypes.byref(c), stream))
+    return st, r.value, c.value
 
 
 def ot_plan_destroy(plan) -> None:

@@ -23,13 +23,21 @@ namespace {
 
 thread_local char g_err[512] = "no error";
 
-int fail(int code, const char *fmt, ...) {
+}  // namespace
+
+// Records the calling thread's error text; returns code (shared by every
+// entry point of the library).
+int ot::set_error(int code, const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
     vsnprintf(g_err, sizeof g_err, fmt, ap);
     va_end(ap);
     return code;
 }
+
+namespace {
+
+#define fail ot::set_error
 
 #define OT_CU(call)                                                                      \
     do {                                                                                 \

@@ -4,6 +4,9 @@
 
 namespace ot {
 
+// api.cu: sets the thread's last-error text and returns code
+int set_error(int code, const char *fmt, ...);
+
 // halfstep.cu
 int halfstep_blocks_per_sm(int kind, int dim, int rpt);
 cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,
