@@ -89,6 +89,9 @@ typedef struct ot_options {
     double eps_decay;         /* in (0, 1); default 0.7 */
     int32_t timing;           /* 1: time the iteration loop with CUDA events on the
                                  internal stream (ot_info.loop_ms); default 0 */
+    int32_t col_splits;       /* tuning: column splits of the half-steps (0 = chosen
+                                 from the problem size and the SM count) */
+    int32_t rows_per_thread;  /* tuning, d <= 3: 2, 4 or 8 rows per thread (0 = auto) */
     int32_t reserved0;
 } ot_options;
 

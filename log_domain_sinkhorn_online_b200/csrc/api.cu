@@ -154,7 +154,8 @@ struct Carver {
 // of `cap` resident blocks costs rpt * (cps + 64 per-item overhead), and the
 // block that finishes a tile merges `splits` partials per row (~8 columns
 // each). Returns the estimate of the best split count, which it stores in sd.
-double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd) {
+double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd,
+                     int force_s = 0) {
     const int64_t tiles = (rows + tile - 1) / tile;
     double best = 1e300;
     int best_s = 1;
@@ -163,7 +164,11 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
     for (int64_t s = 1; s <= max_s; ++s) {
         const int64_t cps = round_up((cols_pad + s - 1) / s, kColPad);
         const int64_t s_eff = (cols_pad + cps - 1) / cps;
-        if (s_eff != s) continue;
+        if (force_s > 0) {
+            if (s != std::min<int64_t>(force_s, max_s)) continue;  // the nearest attainable count
+        } else if (s_eff != s) {
+            continue;
+        }
         const int64_t items = tiles * s_eff;
         const int64_t waves = (items + cap - 1) / cap;
         const double t = (double)waves * rpt * (double)(cps + 64) + 8.0 * rpt * (double)s_eff;
@@ -184,21 +189,24 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
 
 // Launch shape of one side's half-step: for d <= 3 also picks the rows per
 // thread (8, 4 or 2) with the smallest estimate.
-int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Side &sd) {
+int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Side &sd,
+                 int force_s, int force_rpt) {
     if (kind == 1) {
         const int bps = halfstep_blocks_per_sm(1, dim, kGnRows);
         if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
-        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd);
+        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd, force_s);
         return OT_OK;
     }
     double best = 1e300;
     for (int rpt : {8, 4, 2}) {
+        if (force_rpt > 0 && rpt != force_rpt) continue;
         const int bps = halfstep_blocks_per_sm(0, dim, rpt);
         if (bps <= 0) continue;
         Side tmp = sd;
         // fewer rows per thread re-read the shared column data more often
         const double eff = rpt == 2 ? 0.9 : 1.0;
-        const double t = choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp) / eff;
+        const double t =
+            choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp, force_s) / eff;
         if (t < best) {
             best = t;
             sd = tmp;
@@ -359,7 +367,7 @@ void ot_plan_destroy(ot_plan *plan) { plan_free(plan); }
 namespace {
 
 // Allocates the plan's solve workspace and chooses launch shapes.
-int plan_setup(ot_plan *p) {
+int plan_setup(ot_plan *p, const ot_options &o) {
     p->kind = p->d <= 3 ? 0 : 1;
     if (p->kind == 0) {
         p->dim = p->d;
@@ -373,9 +381,12 @@ int plan_setup(ot_plan *p) {
     p->sy.cnt = p->m;
     p->sx.pad = round_up(p->n, kColPad);
     p->sy.pad = round_up(p->m, kColPad);
-    int rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx);
+    int rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx, o.col_splits,
+                          o.rows_per_thread);
     if (rc != OT_OK) return rc;
-    if ((rc = choose_shape(p->kind, p->dim, p->sm_count, p->m, p->sx.pad, p->sy)) != OT_OK) return rc;
+    if ((rc = choose_shape(p->kind, p->dim, p->sm_count, p->m, p->sx.pad, p->sy, o.col_splits,
+                           o.rows_per_thread)) != OT_OK)
+        return rc;
     const int64_t part_cnt = std::max((int64_t)p->sx.splits * p->sx.tiles * p->sx.tile,
                                       (int64_t)p->sy.splits * p->sy.tiles * p->sy.tile);
     const int64_t tiles = std::max(p->sx.tiles, p->sy.tiles);
@@ -478,6 +489,10 @@ int validate(const float *x, const float *y, const float *a, const float *b, int
     if (n_iters == 0 && !o.warm_start)
         return fail(OT_ERR_INVALID_ARG, "n_iters == 0 needs warm_start (a plan at given f, g)");
     if (o.check_every < 1) return fail(OT_ERR_INVALID_ARG, "check_every must be >= 1");
+    if (o.col_splits < 0) return fail(OT_ERR_INVALID_ARG, "col_splits must be >= 0");
+    if (o.rows_per_thread != 0 && o.rows_per_thread != 2 && o.rows_per_thread != 4 &&
+        o.rows_per_thread != 8)
+        return fail(OT_ERR_INVALID_ARG, "rows_per_thread must be 0, 2, 4 or 8");
     if (o.eps_init > 0.0) {
         if (!(o.eps_decay > 0.0 && o.eps_decay < 1.0)) return fail(OT_ERR_INVALID_ARG, "eps_decay must be in (0,1)");
         if (o.iters_per_stage < 1) return fail(OT_ERR_INVALID_ARG, "iters_per_stage must be >= 1");
@@ -518,7 +533,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     OT_CU(cudaMallocHost(&p->hs, sizeof(HostScalars)));
     OT_CU(cudaEventRecord(p->ev_in, us));
     OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
-    if ((rc = plan_setup(p)) != OT_OK) return rc;
+    if ((rc = plan_setup(p, o)) != OT_OK) return rc;
     if ((rc = resolve_scale(p, scale_cost, o.scale_value)) != OT_OK) return rc;
     if (!o.warm_start) {
         OT_CU(cudaMemsetAsync(f, 0, sizeof(float) * n, p->s_int));

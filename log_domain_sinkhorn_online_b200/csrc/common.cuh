@@ -86,6 +86,13 @@ __device__ __forceinline__ float ex2_approx(float v) {
     return r;
 }
 
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ int ld_volatile(const int *p) {
     return *reinterpret_cast<const volatile int *>(p);
 }

@@ -44,39 +44,48 @@ __device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_f
 
     const double eps = A.prm->eps, kappa = A.prm->kappa, c = A.prm->c, tol = A.prm->tol;
     const int64_t stride = (int64_t)A.tiles * TILE;
+    constexpr int RPT = TILE / THREADS;       // rows of this thread
+    constexpr int BU = RPT >= 8 ? 2 : 16 / RPT;  // splits per batch: 16 loads in flight
+    // merge the splits' (max, sum) pairs: every load of a batch, for all of this
+    // thread's rows, is independent, so one L2 round trip serves 16 partials
+    float M[RPT];
+    double S[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        M[k] = kNegBig;
+        S[k] = 0.0;
+    }
+    for (int s0 = 0; s0 < A.splits; s0 += BU) {
+        float2 pp[RPT][BU];
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
+#pragma unroll
+            for (int u = 0; u < BU; ++u)
+                pp[k][u] = (s0 + u < A.splits && row < A.rows)
+                               ? __ldcg(&A.part[(s0 + u) * stride + row])
+                               : make_float2(kNegBig, 0.0f);
+        }
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            float bm = pp[k][0].x;
+#pragma unroll
+            for (int u = 1; u < BU; ++u) bm = fmaxf(bm, pp[k][u].x);
+            if (bm > M[k]) {
+                S[k] *= (double)ex2_approx(M[k] - bm);
+                M[k] = bm;
+            }
+#pragma unroll
+            for (int u = 0; u < BU; ++u)
+                if (pp[k][u].y > 0.0f) S[k] += (double)pp[k][u].y * (double)ex2_approx(pp[k][u].x - M[k]);
+        }
+    }
     double rsum = 0.0;
     bool bad = false;
-#pragma unroll 1
-    for (int k = 0; k < TILE / THREADS; ++k) {
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
         const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
         if (row >= A.rows) continue;
-        // merge the splits' (max, sum) pairs 8 at a time (independent loads in flight)
-        float M = kNegBig;
-        double S = 0.0;
-        int s = 0;
-        for (; s + 8 <= A.splits; s += 8) {
-            float2 pp[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) pp[u] = __ldcg(&A.part[(s + u) * stride + row]);
-            float bm = pp[0].x;
-#pragma unroll
-            for (int u = 1; u < 8; ++u) bm = fmaxf(bm, pp[u].x);
-            if (bm > M) {
-                S *= (double)ex2_approx(M - bm);
-                M = bm;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (pp[u].y > 0.0f) S += (double)pp[u].y * (double)ex2_approx(pp[u].x - M);
-        }
-        for (; s < A.splits; ++s) {
-            const float2 pp = __ldcg(&A.part[s * stride + row]);
-            if (pp.x > M) {
-                S *= (double)ex2_approx(M - pp.x);
-                M = pp.x;
-            }
-            if (pp.y > 0.0f) S += (double)pp.y * (double)ex2_approx(pp.x - M);
-        }
         const float *xr = A.rowtab + row * (int64_t)A.dp;
         double nrm = 0.0;
         for (int q = 0; q < A.dp; ++q) nrm += (double)xr[q] * (double)xr[q];
@@ -84,11 +93,11 @@ __device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_f
         double pot = 0.0, term = 0.0;
         if (wi == 0.0) {
             pot = -INFINITY;  // massless row: empty row of the plan
-        } else if (!(S > 0.0)) {
+        } else if (!(S[k] > 0.0)) {
             pot = INFINITY;   // every column is massless: no finite potential
             bad = true;
         } else {
-            const double L = (double)M + log2(S) - kappa * c * nrm;
+            const double L = (double)M[k] + log2(S[k]) - kappa * c * nrm;
             pot = eps * log(wi) - L / kappa;
             const double old = (double)A.pot_old[row];
             term = fabs(exp2(kappa * old + L) - wi);
@@ -149,7 +158,7 @@ __device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_f
 // is 128 R rows: fewer rows per thread give more tiles, hence fewer column
 // splits to merge, on small problems).
 template <int D, int R>
-__global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : 4) hs_lowd_kernel(HalfStep A) {
+__global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lowd_kernel(HalfStep A) {
     constexpr int kHsRows = R;
     constexpr int kHsTile = kHsThreads * R;
     __shared__ __align__(16) float4 sm[2][kHsChunk];
@@ -166,7 +175,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : 4) hs_lowd_kernel(Hal
 
         float2 xd[kHsRows][3];
         float m[kHsRows], tot[kHsRows];
-        float2 nm[kHsRows], acc[kHsRows];
+        float2 nm[kHsRows], acc[kHsRows], acc2[kHsRows];
 #pragma unroll
         for (int k = 0; k < kHsRows; ++k) {
             const int64_t row = (int64_t)tile * kHsTile + k * kHsThreads + tid;
@@ -177,6 +186,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : 4) hs_lowd_kernel(Hal
             m[k] = kNegBig;
             nm[k] = make_float2(-kNegBig, -kNegBig);
             acc[k] = make_float2(0.f, 0.f);
+            acc2[k] = make_float2(0.f, 0.f);
             tot[k] = 0.f;
         }
 
@@ -217,26 +227,29 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : 4) hs_lowd_kernel(Hal
                         if (D >= 3) tt = __ffma2_rn(make_float2(hi.x, hi.y), xd[k][2], tt);
                         t[p] = tt;
                     }
-                    const float cm = fmaxf(fmaxf(fmaxf(t[0].x, t[0].y), fmaxf(t[1].x, t[1].y)),
-                                           fmaxf(fmaxf(t[2].x, t[2].y), fmaxf(t[3].x, t[3].y)));
+                    const float cm = fmax3(fmax3(t[0].x, t[0].y, t[1].x), fmax3(t[1].y, t[2].x, t[2].y),
+                                           fmaxf(t[3].x, t[3].y));
                     if (cm > m[k] + kLazyMax) {  // rare: refresh the running maximum
                         const float sc = ex2_approx(m[k] - cm);
                         acc[k] = __fmul2_rn(acc[k], make_float2(sc, sc));
+                        acc2[k] = __fmul2_rn(acc2[k], make_float2(sc, sc));
                         tot[k] *= sc;
                         m[k] = cm;
                         nm[k] = make_float2(-cm, -cm);
                     }
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const float2 u = __fadd2_rn(t[p], nm[k]);
-                        acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u.x), ex2_approx(u.y)));
-                    }
+                    const float2 u0 = __fadd2_rn(t[0], nm[k]), u1 = __fadd2_rn(t[1], nm[k]);
+                    const float2 u2 = __fadd2_rn(t[2], nm[k]), u3 = __fadd2_rn(t[3], nm[k]);
+                    acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
+                    acc2[k] = __fadd2_rn(acc2[k], make_float2(ex2_approx(u1.x), ex2_approx(u1.y)));
+                    acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u2.x), ex2_approx(u2.y)));
+                    acc2[k] = __fadd2_rn(acc2[k], make_float2(ex2_approx(u3.x), ex2_approx(u3.y)));
                 }
             }
 #pragma unroll
             for (int k = 0; k < kHsRows; ++k) {
-                tot[k] += acc[k].x + acc[k].y;
+                tot[k] += (acc[k].x + acc[k].y) + (acc2[k].x + acc2[k].y);
                 acc[k] = make_float2(0.f, 0.f);
+                acc2[k] = make_float2(0.f, 0.f);
             }
         }
 

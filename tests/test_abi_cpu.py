@@ -45,7 +45,7 @@ def test_version_and_defaults(B):
 
 
 def test_struct_sizes_match_header_layout(B):
-    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 2 * 4
+    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 4 * 4
     assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8
 
 
