@@ -92,7 +92,9 @@ typedef struct ot_options {
     int32_t col_splits;       /* tuning: column splits of the half-steps (0 = chosen
                                  from the problem size and the SM count) */
     int32_t rows_per_thread;  /* tuning, d <= 3: 2, 4 or 8 rows per thread (0 = auto) */
-    int32_t reserved0;
+    int32_t tensor_cores;     /* 16 <= d <= 64: 1 (default) computes x.y on the tcgen05
+                                 tensor cores (bf16 splits, fp32 accumulation); 0 uses
+                                 the CUDA-core FMA kernel */
 } ot_options;
 
 /* -------------------------------------------------------- solve report   */
@@ -127,7 +129,8 @@ OT_API int ot_version(void);
 OT_API const char *ot_last_error_string(void);
 
 /* Default options (warm_start 0, check_every 16, use_graphs 1,
- * iters_per_stage 20, scale_value 1, eps_init 0, eps_decay 0.7, timing 0). */
+ * iters_per_stage 20, scale_value 1, eps_init 0, eps_decay 0.7, timing 0,
+ * col_splits 0, rows_per_thread 0, tensor_cores 1). */
 OT_API void ot_options_default(ot_options *opt);
 
 /* ------------------------------------------------- ot_sinkhorn_pointcloud

@@ -77,6 +77,7 @@ struct Side {          // one cloud's half of the problem
     int tiles, splits, grid;
     int64_t cps;       // columns per split of the OTHER side's table
     int rpt, tile;     // rows per thread and rows per tile of this side's half-step
+    void *arow, *bcol; // tensor-core path: bf16 operand tables [pad][kp] (rows, columns)
 };
 
 }  // namespace
@@ -107,6 +108,8 @@ struct ot_plan {
     float *rowmax = nullptr;
     int64_t *counts = nullptr;
     HostScalars *hs = nullptr;  // pinned
+    int kp = 0;                 // tensor-core path: bf16 K extent of the operand tables
+    CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
     cudaStream_t s_int = nullptr;
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
     cudaGraphExec_t graph[2] = {nullptr, nullptr};  // chunk graphs by start parity
@@ -155,14 +158,14 @@ struct Carver {
 // block that finishes a tile merges `splits` partials per row (~8 columns
 // each). Returns the estimate of the best split count, which it stores in sd.
 double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd,
-                     int force_s = 0) {
+                     int force_s = 0, int gran = kColPad) {
     const int64_t tiles = (rows + tile - 1) / tile;
     double best = 1e300;
     int best_s = 1;
     int64_t best_cps = cols_pad;
-    const int64_t max_s = std::min<int64_t>(cols_pad / kColPad, 4096);
+    const int64_t max_s = std::min<int64_t>(cols_pad / gran, 4096);
     for (int64_t s = 1; s <= max_s; ++s) {
-        const int64_t cps = round_up((cols_pad + s - 1) / s, kColPad);
+        const int64_t cps = round_up((cols_pad + s - 1) / s, gran);
         const int64_t s_eff = (cols_pad + cps - 1) / cps;
         if (force_s > 0) {
             if (s != std::min<int64_t>(force_s, max_s)) continue;  // the nearest attainable count
@@ -191,6 +194,10 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
 // thread (8, 4 or 2) with the smallest estimate.
 int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Side &sd,
                  int force_s, int force_rpt) {
+    if (kind == 2) {  // tensor cores: one 288-thread block per SM, 128-row tiles, 128-column chunks
+        choose_splits(rows, cols_pad, 1, 128, sms, sd, force_s, 128);
+        return OT_OK;
+    }
     if (kind == 1) {
         const int bps = halfstep_blocks_per_sm(1, dim, kGnRows);
         if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
@@ -255,10 +262,15 @@ HalfStep make_step(const ot_plan *p, int side, int parity) {
     A.pot_old = f ? fb[parity] : p->g;
     A.pot_new = f ? fb[parity ^ 1] : p->g;
     A.next_col = rows.coltab;  // this side's column table feeds the other half-step
+    A.nxt_bf16 = 0;
     if (p->kind == 0) {
         A.nxt_a = 8; A.nxt_l = 1; A.nxt_b = 6;
-    } else {
+    } else if (p->kind == 1) {
         A.nxt_a = 2 * (p->dp + 4); A.nxt_l = p->dp + 4; A.nxt_b = p->dp;
+    } else {
+        A.next_col = static_cast<float *>(rows.bcol);
+        A.nxt_bf16 = 1;
+        A.nxt_a = p->kp; A.nxt_l = 0; A.nxt_b = 3 * p->d;
     }
     A.prm = p->prm;
     A.st = p->st;
@@ -277,12 +289,20 @@ cudaError_t mark(ot_plan *p) {
     return cudaEventRecord(p->tev[p->tev_used++], p->s_int);
 }
 
+// One half-step: side 0 updates f (rows x, columns y), side 1 updates g.
+cudaError_t launch_side(const ot_plan *p, int side, int parity) {
+    const Side &sd = side == 0 ? p->sx : p->sy;
+    if (p->kind == 2)
+        return launch_halfstep_tc(p->d, make_step(p, side, parity),
+                                  side == 0 ? &p->tm_arow_x : &p->tm_arow_y,
+                                  side == 0 ? &p->tm_bcol_y : &p->tm_bcol_x, sd.grid, p->s_int);
+    return launch_halfstep(p->kind, p->dim, sd.rpt, make_step(p, side, parity), sd.grid, p->s_int);
+}
+
 cudaError_t launch_iteration(const ot_plan *p, int parity) {
-    cudaError_t e = launch_halfstep(p->kind, p->dim, p->sx.rpt, make_step(p, 0, parity),
-                                    p->sx.grid, p->s_int);
+    cudaError_t e = launch_side(p, 0, parity);
     if (e != cudaSuccess) return e;
-    return launch_halfstep(p->kind, p->dim, p->sy.rpt, make_step(p, 1, parity), p->sy.grid,
-                           p->s_int);
+    return launch_side(p, 1, parity);
 }
 
 // Runs `iters` iterations starting at global parity `parity0`, in chunks of
@@ -358,6 +378,9 @@ void ot_options_default(ot_options *opt) {
     opt->eps_init = 0.0;
     opt->eps_decay = 0.7;
     opt->timing = 0;
+    opt->col_splits = 0;
+    opt->rows_per_thread = 0;
+    opt->tensor_cores = 1;
 }
 
 void ot_plan_destroy(ot_plan *plan) { plan_free(plan); }
@@ -368,19 +391,26 @@ namespace {
 
 // Allocates the plan's solve workspace and chooses launch shapes.
 int plan_setup(ot_plan *p, const ot_options &o) {
-    p->kind = p->d <= 3 ? 0 : 1;
-    if (p->kind == 0) {
+    if (p->d <= 3) {
+        p->kind = 0;
         p->dim = p->d;
         p->dp = 4;
+    } else if (p->d >= 16 && o.tensor_cores) {
+        p->kind = 2;
+        p->dim = p->d;
+        p->dp = (int)round_up(p->d, 4);
+        p->kp = 64 * tc_slabs(p->d);
     } else {
+        p->kind = 1;
         p->dim = p->d <= 8 ? 8 : p->d <= 16 ? 16 : p->d <= 32 ? 32 : 64;
         p->dp = p->dim;
     }
-    const int64_t colw = p->kind == 0 ? 4 : p->dp + 4;
+    const int64_t colw = p->kind == 0 ? 4 : p->kind == 1 ? p->dp + 4 : 0;
+    const int64_t padq = p->kind == 2 ? 128 : kColPad;
     p->sx.cnt = p->n;
     p->sy.cnt = p->m;
-    p->sx.pad = round_up(p->n, kColPad);
-    p->sy.pad = round_up(p->m, kColPad);
+    p->sx.pad = round_up(p->n, padq);
+    p->sy.pad = round_up(p->m, padq);
     int rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx, o.col_splits,
                           o.rows_per_thread);
     if (rc != OT_OK) return rc;
@@ -404,10 +434,22 @@ int plan_setup(ot_plan *p, const ot_options &o) {
         p->sy.rowtab = cv.take<float>(p->sy.pad * p->dp);
         p->sx.coltab = cv.take<float>(p->sx.pad * colw);
         p->sy.coltab = cv.take<float>(p->sy.pad * colw);
+        p->sx.arow = cv.take<uint16_t>(p->sx.pad * p->kp);
+        p->sx.bcol = cv.take<uint16_t>(p->sx.pad * p->kp);
+        p->sy.arow = cv.take<uint16_t>(p->sy.pad * p->kp);
+        p->sy.bcol = cv.take<uint16_t>(p->sy.pad * p->kp);
         p->part = cv.take<float2>(part_cnt);
         p->tile_cnt = cv.take<unsigned>(tiles);
         p->tile_resid = cv.take<double>(tiles);
         if (pass == 0) OT_CU(cudaMalloc(&p->ws, cv.off));
+    }
+    if (p->kind == 2) {
+        OT_CU(tc_setup(p->d));
+        int e = make_operand_map(&p->tm_arow_x, p->sx.arow, p->sx.pad, p->kp);
+        if (!e) e = make_operand_map(&p->tm_bcol_y, p->sy.bcol, p->sy.pad, p->kp);
+        if (!e) e = make_operand_map(&p->tm_arow_y, p->sy.arow, p->sy.pad, p->kp);
+        if (!e) e = make_operand_map(&p->tm_bcol_x, p->sx.bcol, p->sx.pad, p->kp);
+        if (e) return fail(OT_ERR_CUDA, "tensor map encoding failed (%d)", e);
     }
     OT_CU(cudaMemsetAsync(p->tile_cnt, 0, sizeof(unsigned) * tiles, p->s_int));
     OT_CU(cudaMemsetAsync(p->st, 0, sizeof(State), p->s_int));
@@ -555,7 +597,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         stage_eps.push_back((double)eps);
     }
     float *fb[2] = {p->f, p->fspare};
-    const int layout = p->kind == 0 ? 0 : 1;
+    const int layout = p->kind == 0 ? 0 : 1;  // CUDA-core paths' column-table layout
     int t = 0, converged = 0;
     int64_t half_steps = 0;
     double resid = NAN;
@@ -565,10 +607,17 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         const int iters = last ? n_iters : o.iters_per_stage;
         OT_CU(launch_set_params(p->prm, stage_eps[si], p->c, tol_s, p->s_int));
         OT_CU(launch_reset_state(p->st, p->s_int));
-        OT_CU(launch_tables(x, fb[t & 1], n, p->sx.pad, d, p->dp, p->o, p->prm, p->sx.rowtab,
-                            p->sx.coltab, layout, p->s_int));
-        OT_CU(launch_tables(y, g, m, p->sy.pad, d, p->dp, p->o, p->prm, p->sy.rowtab,
-                            p->sy.coltab, layout, p->s_int));
+        if (p->kind == 2) {
+            OT_CU(launch_tc_tables(x, fb[t & 1], n, p->sx.pad, d, p->dp, p->kp, p->o, p->prm,
+                                   p->sx.rowtab, p->sx.arow, p->sx.bcol, p->s_int));
+            OT_CU(launch_tc_tables(y, g, m, p->sy.pad, d, p->dp, p->kp, p->o, p->prm,
+                                   p->sy.rowtab, p->sy.arow, p->sy.bcol, p->s_int));
+        } else {
+            OT_CU(launch_tables(x, fb[t & 1], n, p->sx.pad, d, p->dp, p->o, p->prm, p->sx.rowtab,
+                                p->sx.coltab, layout, p->s_int));
+            OT_CU(launch_tables(y, g, m, p->sy.pad, d, p->dp, p->o, p->prm, p->sy.rowtab,
+                                p->sy.coltab, layout, p->s_int));
+        }
         p->launches += 4;
         if ((rc = run_iterations(p, t & 1, iters, tol_s > 0.0, o.use_graphs != 0)) != OT_OK) return rc;
         if ((rc = read_state(p)) != OT_OK) return rc;
@@ -582,8 +631,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
             } else if (iters > 0) {
                 // one more f-update measures ||T1 - a||_1 of the final state
                 OT_CU(mark(p));
-                OT_CU(launch_halfstep(p->kind, p->dim, p->sx.rpt, make_step(p, 0, t & 1), p->sx.grid,
-                                      p->s_int));
+                OT_CU(launch_side(p, 0, t & 1));
                 OT_CU(mark(p));
                 p->launches += 1;
                 half_steps += 1;
@@ -595,6 +643,8 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     }
     if (t & 1) OT_CU(cudaMemcpyAsync(p->f, p->fspare, sizeof(float) * n, cudaMemcpyDeviceToDevice, p->s_int));
     if ((rc = read_state(p)) != OT_OK) return rc;
+    if (p->hs->st.wait_timeout)
+        return fail(OT_ERR_CUDA, "a tensor-core pipeline wait timed out (results invalid)");
     if (p->hs->st.nonfinite)
         return fail(OT_ERR_NONFINITE, "a potential left the finite range (eps too small for float32?)");
     p->eps = stage_eps.back();

@@ -49,7 +49,7 @@ struct State {
     int bad_index;      // a row index outside [0, n) was given to a row kernel
     int iter_done;      // completed iterations in the current stage
     int conv_iter;      // iteration count at which tol was met (-1: not yet)
-    int pad0;
+    int wait_timeout;   // a bounded wait in a tensor-core kernel gave up (error)
     double resid[2];    // last in-loop marginal residual of each side (0: rows, 1: cols)
     unsigned tiles_done[2];
     unsigned pad1[2];
@@ -75,6 +75,8 @@ struct HalfStep {
     float *pot_new;            // potential after the update
     float *next_col;           // column table of the other half-step (float view)
     int64_t nxt_a, nxt_l, nxt_b;  // column i's G' sits at (i>>1)*nxt_a + (i&1)*nxt_l + nxt_b
+    int nxt_bf16;              // 1: the other table is bf16 and G is stored as three bf16
+                               //    terms at element i*nxt_a + nxt_b (tensor-core path)
     const Params *prm;
     State *st;
 };

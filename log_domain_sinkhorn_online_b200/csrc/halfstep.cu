@@ -23,130 +23,9 @@
 //   sum_j T_ij(old) = 2^(kappa f_old_i + L_i),  L_i = log2 sum_j 2^(kappa (g_j - C_ij)).
 // The last tile to finish sums the residual partials in tile order (no float
 // atomics, so the result is deterministic) and runs the stop test.
-#include "common.cuh"
+#include "finish.cuh"
 
 namespace ot {
-
-// Merge the column splits of one row tile; run by the block that finishes a
-// tile last. Returns nothing; all threads of the block must call it.
-template <int THREADS, int TILE>
-__device__ void finish_tile(const HalfStep &A, int tile, double *s_red, int *s_flag) {
-    const int tid = threadIdx.x;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        unsigned prev = atomicAdd(&A.tile_cnt[tile], 1u);
-        *s_flag = (prev == (unsigned)(A.splits - 1));
-    }
-    __syncthreads();
-    if (!*s_flag) return;
-    __threadfence();
-
-    const double eps = A.prm->eps, kappa = A.prm->kappa, c = A.prm->c, tol = A.prm->tol;
-    const int64_t stride = (int64_t)A.tiles * TILE;
-    constexpr int RPT = TILE / THREADS;       // rows of this thread
-    constexpr int BU = RPT >= 8 ? 2 : 16 / RPT;  // splits per batch: 16 loads in flight
-    // merge the splits' (max, sum) pairs: every load of a batch, for all of this
-    // thread's rows, is independent, so one L2 round trip serves 16 partials
-    float M[RPT];
-    double S[RPT];
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-        M[k] = kNegBig;
-        S[k] = 0.0;
-    }
-    for (int s0 = 0; s0 < A.splits; s0 += BU) {
-        float2 pp[RPT][BU];
-#pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-            const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
-#pragma unroll
-            for (int u = 0; u < BU; ++u)
-                pp[k][u] = (s0 + u < A.splits && row < A.rows)
-                               ? __ldcg(&A.part[(s0 + u) * stride + row])
-                               : make_float2(kNegBig, 0.0f);
-        }
-#pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-            float bm = pp[k][0].x;
-#pragma unroll
-            for (int u = 1; u < BU; ++u) bm = fmaxf(bm, pp[k][u].x);
-            if (bm > M[k]) {
-                S[k] *= (double)ex2_approx(M[k] - bm);
-                M[k] = bm;
-            }
-#pragma unroll
-            for (int u = 0; u < BU; ++u)
-                if (pp[k][u].y > 0.0f) S[k] += (double)pp[k][u].y * (double)ex2_approx(pp[k][u].x - M[k]);
-        }
-    }
-    double rsum = 0.0;
-    bool bad = false;
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-        const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
-        if (row >= A.rows) continue;
-        const float *xr = A.rowtab + row * (int64_t)A.dp;
-        double nrm = 0.0;
-        for (int q = 0; q < A.dp; ++q) nrm += (double)xr[q] * (double)xr[q];
-        const double wi = (double)A.w[row];
-        double pot = 0.0, term = 0.0;
-        if (wi == 0.0) {
-            pot = -INFINITY;  // massless row: empty row of the plan
-        } else if (!(S[k] > 0.0)) {
-            pot = INFINITY;   // every column is massless: no finite potential
-            bad = true;
-        } else {
-            const double L = (double)M[k] + log2(S[k]) - kappa * c * nrm;
-            pot = eps * log(wi) - L / kappa;
-            const double old = (double)A.pot_old[row];
-            term = fabs(exp2(kappa * old + L) - wi);
-        }
-        const float pf = (float)pot;
-        if (wi != 0.0 && !isfinite(pf)) bad = true;
-        A.pot_new[row] = pf;
-        A.next_col[(row >> 1) * A.nxt_a + (row & 1) * A.nxt_l + A.nxt_b] =
-            (wi == 0.0) ? -INFINITY : (float)(kappa * ((double)pf - c * nrm));
-        rsum += term;
-    }
-    if (bad) atomicExch(&A.st->nonfinite, 1);
-    if (tid == 0) A.tile_cnt[tile] = 0;
-
-    // deterministic block sum of the residual terms
-    for (int off = 16; off > 0; off >>= 1) rsum += __shfl_xor_sync(0xffffffffu, rsum, off);
-    if ((tid & 31) == 0) s_red[tid >> 5] = rsum;
-    __syncthreads();
-    if (tid == 0) {
-        double t = 0.0;
-        for (int w = 0; w < THREADS / 32; ++w) t += s_red[w];
-        A.tile_resid[tile] = t;
-        __threadfence();
-        unsigned prev = atomicAdd(&A.st->tiles_done[A.side], 1u);
-        *s_flag = (prev == (unsigned)(A.tiles - 1));
-    }
-    __syncthreads();
-    if (!*s_flag) return;
-    __threadfence();
-    if (tid < 32) {
-        double v = 0.0;
-        for (int t = tid; t < A.tiles; t += 32) v += __ldcg(&A.tile_resid[t]);
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (tid == 0) {
-            State *st = A.st;
-            st->resid[A.side] = v;
-            st->tiles_done[A.side] = 0;
-            if (A.side == 0) {
-                if (tol > 0.0 && st->iter_done >= 1 && v <= tol) {
-                    st->stop = 1;
-                    st->conv_iter = st->iter_done;
-                }
-            } else {
-                st->iter_done += 1;
-            }
-            __threadfence();
-        }
-    }
-}
 
 // ------------------------------------------------------------ d <= 3 path
 // Column table: for the column pair (2p, 2p+1), two float4
@@ -259,7 +138,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lo
             const int64_t row = (int64_t)tile * kHsTile + k * kHsThreads + tid;
             if (row < A.rows) A.part[split * stride + row] = make_float2(m[k], tot[k]);
         }
-        finish_tile<kHsThreads, kHsTile>(A, tile, s_red, &s_flag);
+        finish_tile<kHsThreads, kHsTile, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
     }
 }
@@ -355,7 +234,7 @@ __global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
             const int64_t row = (int64_t)tile * kGnTile + k * kGnThreads + tid;
             if (row < A.rows) A.part[split * stride + row] = make_float2(m[k], tot[k]);
         }
-        finish_tile<kGnThreads, kGnTile>(A, tile, s_red, &s_flag);
+        finish_tile<kGnThreads, kGnTile, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
     }
 }

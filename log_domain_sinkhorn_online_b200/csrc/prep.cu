@@ -129,6 +129,7 @@ __global__ void set_params_kernel(Params *prm, double eps, double c, double tol)
 
 __global__ void reset_state_kernel(State *st) {
     st->stop = 0;
+    st->wait_timeout = 0;
     st->iter_done = 0;
     st->conv_iter = -1;
     st->resid[0] = st->resid[1] = -1.0;

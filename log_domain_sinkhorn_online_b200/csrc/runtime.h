@@ -1,5 +1,7 @@
 // runtime.h -- host-side declarations of the kernel launchers (internal).
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace ot {
@@ -11,6 +13,17 @@ int set_error(int code, const char *fmt, ...);
 int halfstep_blocks_per_sm(int kind, int dim, int rpt);
 cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,
                             cudaStream_t s);
+
+// halfstep_tc.cu (16 <= d <= 64: tensor-core path)
+int tc_ksteps(int d);
+int tc_slabs(int d);
+cudaError_t tc_setup(int d);
+cudaError_t launch_halfstep_tc(int d, const HalfStep &A, const CUtensorMap *tmA,
+                               const CUtensorMap *tmB, int grid, cudaStream_t s);
+cudaError_t launch_tc_tables(const float *p, const float *pot, int64_t cnt, int64_t pad, int d,
+                             int dpf, int kp, const double *o, const Params *prm, float *rowtab,
+                             void *arow, void *bcol, cudaStream_t s);
+int make_operand_map(CUtensorMap *map, void *base, int64_t rows, int kp);
 
 // prep.cu
 cudaError_t launch_coord_stats(const float *v, int64_t cnt, int d, double *part, double *part2,

@@ -67,10 +67,13 @@ def test_lowd_trajectory_ragged(ot, orc, d, scale):
     assert plan.info.iterations == 25
 
 
-@pytest.mark.parametrize("d", [4, 5, 16, 33, 50, 64])
-def test_generic_d_trajectory(ot, orc, d):
+@pytest.mark.parametrize("d,tc", [(4, False), (5, False), (15, False), (16, False), (16, True),
+                                  (17, True), (33, True), (50, False), (50, True), (64, True)])
+def test_generic_d_trajectory(ot, orc, d, tc):
+    """3 < d <= 64: CUDA-core FMA kernel, or for d >= 16 the tcgen05 tensor-core
+    kernel (bf16 splits, fp32 accumulation); ragged sizes over several tiles."""
     w = _cloud(30 + d, 611, 530, d, scale="mean", eps=0.05)
-    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 15)
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 15, tensor_cores=tc)
     maxc = H.max_cost(w.x, w.y, c)
     f, g = _pots(plan)
     H.assert_potentials(f, f_ref, maxc, what="f")
@@ -212,6 +215,22 @@ def test_annealing_matches_oracle(ot, orc):
     f_ref, g_ref, stages, r_ref = orc.sinkhorn_anneal(w.x, w.y, w.a, w.b, 1.0, eps_t, 1.0, 0.7, 10)
     assert plan.info.stages == stages
     maxc = H.max_cost(w.x, w.y, 1.0)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+
+
+@pytest.mark.parametrize("n,m", [(1, 300), (129, 127), (2000, 3001)])
+def test_tensor_core_path_ragged_and_massless(ot, orc, n, m):
+    """tcgen05 path on sizes that are not multiples of the 128-row tile, with a
+    massless row and column, against the oracle's trajectory."""
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w3(n=n, m=m)
+    if n > 1:
+        w.a[n // 2] = 0.0
+    w.b[m // 3] = 0.0
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 12)
+    maxc = H.max_cost(w.x, w.y, c)
     f, g = _pots(plan)
     H.assert_potentials(f, f_ref, maxc, what="f")
     H.assert_potentials(g, g_ref, maxc, what="g")
