@@ -494,7 +494,7 @@ int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
         const double mean = sxx / (double)p->n + syy / (double)p->m - 2.0 * dot;
         c = 1.0 / mean;
     } else if (scale == OT_SCALE_MAX_COST) {
-        OT_CU(launch_max_cost(p->x, p->y, p->n, p->m, p->d, &ds->max_bits, p->s_int));
+        OT_CU(launch_max_cost(p->x, p->y, p->n, p->m, p->d, p->o, &ds->max_bits, p->s_int));
         p->launches += 1;
         rc = read_scalars(p);
         if (rc != OT_OK) return rc;

@@ -191,8 +191,94 @@ cudaError_t launch_coord_stats(const float *v, int64_t cnt, int d, double *part,
     return cudaGetLastError();
 }
 
+// d <= 3: max_j ||x'_i - y'_j||^2 = |x'_i|^2 + max_j (|y'_j|^2 - 2 x'_i . y'_j) on the
+// shifted coordinates (fp32, packed f32x2 FMAs, 3-input max): thread owns 8
+// rows, 256 columns per shared-memory chunk, stored as column pairs
+// [y0 y0' y1 y1' y2 y2' |y|^2 |y'|^2].
+template <int D>
+__global__ void __launch_bounds__(128) max_cost_lowd_kernel(const float *__restrict__ x,
+                                                            const float *__restrict__ y,
+                                                            int64_t n, int64_t m,
+                                                            const double *__restrict__ o,
+                                                            unsigned *out_bits) {
+    constexpr int R = 8, CH = 256;
+    __shared__ __align__(16) float4 sm[CH];
+    __shared__ float s_red[4];
+    const int tid = threadIdx.x;
+    float ov[3] = {0.f, 0.f, 0.f};
+    for (int q = 0; q < D; ++q) ov[q] = (float)o[q];
+    float2 xm[R][3];
+    float nx[R], best[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        const int64_t i = ((int64_t)blockIdx.x * R + k) * 128 + tid;
+        float v[3] = {0.f, 0.f, 0.f};
+        if (i < n)
+            for (int q = 0; q < D; ++q) v[q] = x[i * D + q] - ov[q];
+        nx[k] = v[0] * v[0] + v[1] * v[1] + v[2] * v[2];
+        for (int q = 0; q < 3; ++q) xm[k][q] = make_float2(-2.f * v[q], -2.f * v[q]);
+        best[k] = -INFINITY;
+    }
+    for (int64_t c0 = 0; c0 < m; c0 += CH) {
+        __syncthreads();
+        for (int u = tid; u < CH / 2; u += 128) {
+            float a[3] = {0.f, 0.f, 0.f}, b[3] = {0.f, 0.f, 0.f};
+            const int64_t j = c0 + 2 * u;
+            float na = -INFINITY, nb = -INFINITY;  // padding columns never win
+            if (j < m) {
+                for (int q = 0; q < D; ++q) a[q] = y[j * D + q] - ov[q];
+                na = a[0] * a[0] + a[1] * a[1] + a[2] * a[2];
+            }
+            if (j + 1 < m) {
+                for (int q = 0; q < D; ++q) b[q] = y[(j + 1) * D + q] - ov[q];
+                nb = b[0] * b[0] + b[1] * b[1] + b[2] * b[2];
+            }
+            sm[2 * u] = make_float4(a[0], b[0], a[1], b[1]);
+            sm[2 * u + 1] = make_float4(a[2], b[2], na, nb);
+        }
+        __syncthreads();
+        const int cn = (int)min((int64_t)CH, m - c0);
+        for (int q8 = 0; q8 < cn; q8 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = sm[q8 + u];
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                float2 t[4];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const float4 lo = v[2 * pp], hi = v[2 * pp + 1];
+                    float2 tt = __ffma2_rn(make_float2(lo.x, lo.y), xm[k][0], make_float2(hi.z, hi.w));
+                    if (D >= 2) tt = __ffma2_rn(make_float2(lo.z, lo.w), xm[k][1], tt);
+                    if (D >= 3) tt = __ffma2_rn(make_float2(hi.x, hi.y), xm[k][2], tt);
+                    t[pp] = tt;
+                }
+                best[k] = fmax3(best[k], fmax3(t[0].x, t[0].y, t[1].x), fmax3(t[1].y, t[2].x, t[2].y));
+                best[k] = fmax3(best[k], t[3].x, t[3].y);
+            }
+        }
+    }
+    float b = 0.0f;
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        const int64_t i = ((int64_t)blockIdx.x * R + k) * 128 + tid;
+        if (i < n) b = fmaxf(b, fmaxf(best[k] + nx[k], 0.0f));
+    }
+    for (int off = 16; off > 0; off >>= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, off));
+    if ((tid & 31) == 0) s_red[tid >> 5] = b;
+    __syncthreads();
+    if (tid == 0) atomicMax(out_bits, __float_as_uint(fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]))));
+}
+
 cudaError_t launch_max_cost(const float *x, const float *y, int64_t n, int64_t m, int d,
-                            unsigned *out_bits, cudaStream_t s) {
+                            const double *o, unsigned *out_bits, cudaStream_t s) {
+    if (d <= 3) {
+        const unsigned grid = (unsigned)((n + 8 * 128 - 1) / (8 * 128));
+        if (d == 1) max_cost_lowd_kernel<1><<<grid, 128, 0, s>>>(x, y, n, m, o, out_bits);
+        else if (d == 2) max_cost_lowd_kernel<2><<<grid, 128, 0, s>>>(x, y, n, m, o, out_bits);
+        else max_cost_lowd_kernel<3><<<grid, 128, 0, s>>>(x, y, n, m, o, out_bits);
+        return cudaGetLastError();
+    }
     const int64_t rows_per_block = (int64_t)kMaxThreads * kMaxRows;
     max_cost_kernel<<<(unsigned)((n + rows_per_block - 1) / rows_per_block), kMaxThreads, 0, s>>>(
         x, y, n, m, d, out_bits);

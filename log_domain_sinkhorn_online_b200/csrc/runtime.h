@@ -30,7 +30,7 @@ cudaError_t launch_coord_stats(const float *v, int64_t cnt, int d, double *part,
                                double *out, double *out2, int *flags,
                                unsigned long long *zero_count, cudaStream_t s);
 cudaError_t launch_max_cost(const float *x, const float *y, int64_t n, int64_t m, int d,
-                            unsigned *out_bits, cudaStream_t s);
+                            const double *o, unsigned *out_bits, cudaStream_t s);
 cudaError_t launch_set_params(Params *prm, double eps, double c, double tol, cudaStream_t s);
 cudaError_t launch_reset_state(State *st, cudaStream_t s);
 cudaError_t launch_tables(const float *p, const float *pot, int64_t cnt, int64_t cnt_pad, int d,
