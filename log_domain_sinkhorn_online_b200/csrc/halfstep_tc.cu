@@ -16,13 +16,14 @@
 // 1.8e-6). The row constant -c kappa |x'_i|^2 is added once per row, in
 // float64, by the shared tile finalizer.
 //
-// Block: 9 warps. Warp 8's elected lane is the producer: TMA loads of the row
+// Block: 17 warps. Warp 16's elected lane is the producer: TMA loads of the row
 // tile (once per work item) and of 128-column chunks of the column operand into
 // a 3-stage (2 for K > 192) shared-memory ring, 128B-swizzled K-major, and the
 // tcgen05.mma issue into one of two TMEM accumulators (128 lanes x 128 fp32
-// columns each). Warps 0-7 are the epilogue: warp w reads TMEM lanes
-// 32*(w%4)..+31 (its rows) and columns 64*(w/4)..+63 of each chunk, then runs the
-// lazily-rescaled max / ex2 / sum per row. Every wait on an mbarrier is bounded;
+// columns each). Warps 0-15 are the epilogue (four per SM sub-partition, to hide
+// the TMEM-load latency): warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and
+// columns 32*(w/4)..+31 of each chunk, then runs the lazily-rescaled max / ex2 /
+// sum per row; the four column quarters of a row merge in shared memory. Every wait on an mbarrier is bounded;
 // on timeout the block records State::wait_timeout, drains what it issued (again
 // bounded), frees its TMEM and returns. No TMA load uses cluster multicast.
 #include <cuda.h>
@@ -35,8 +36,10 @@ namespace tc {
 
 constexpr int M = 128;               // rows per tile (MMA M)
 constexpr int N = 128;               // columns per chunk (MMA N)
-constexpr int EPI_WARPS = 8;
-constexpr int THREADS = (EPI_WARPS + 1) * 32;
+constexpr int EPI_WARPS = 16;         // 4 per SM sub-partition
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int QCOLS = N / (EPI_WARPS / 4);  // columns of a chunk per epilogue warp
+constexpr int THREADS = (EPI_WARPS + 2) * 32;  // + TMA warp + MMA warp
 constexpr int SLAB = 64;             // bf16 per 128-byte swizzle row
 constexpr int SLAB_BYTES = M * 128;  // one slab of a 128-row operand tile (16 KB)
 constexpr uint32_t WAIT_LIMIT = 1u << 22;  // polls of one mbarrier before giving up
@@ -130,10 +133,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+
+// Warp-wide wait: lane 0 polls, the other lanes wait converged in the shuffle
+// (512 threads polling would compete with TMA and MMA for shared memory).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
 
 // Bounded wait that ignores the abort flag: used only to drain work this block
 // already issued before it frees its resources.
@@ -152,6 +162,23 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// tcgen05.wait::ld that also marks the loaded registers as written here, so the
+// compiler cannot read them before the wait
+__device__ __forceinline__ void tmem_wait_ld(float (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+                   "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]),
+                   "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]),
+                   "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]),
+                   "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]),
+                   "+f"(v[31])
+                 :
+                 : "memory");
+}
+
+constexpr int NBUF = 4;  // TMEM accumulators (4 x 128 fp32 columns = all 512)
+constexpr int TMA_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
+
 // Shared-memory plan (dynamic; base rounded up to 1024 B for the 128B swizzle).
 template <int KS>
 struct Smem {
@@ -159,11 +186,13 @@ struct Smem {
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = KS * SLAB_BYTES;
     static constexpr int BAR_OFF = B_OFF + STAGES * KS * SLAB_BYTES;
-    static constexpr int NBAR = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], afull
-    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem addr, abort, flag, 8 doubles
-    static constexpr int MERGE_OFF = MISC_OFF + 96;       // float2 [2][M]
-    static constexpr int BYTES = MERGE_OFF + 2 * M * 8;
-    static constexpr int ALLOC = BYTES + 1024;
+    // full[S], empty[S], tfull[NBUF], tempty[NBUF], afull, aempty, drain
+    static constexpr int NBAR = 2 * STAGES + 2 * NBUF + 3;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem addr, abort, flag, decide, 16 doubles
+    static constexpr int MERGE_OFF = MISC_OFF + 160;      // float2 [EPI_WARPS/4][M]
+    static constexpr int BYTES = MERGE_OFF + (EPI_WARPS / 4) * M * 8;
+    // at least 116 KB, so that one block holds an SM (it takes all 512 TMEM columns)
+    static constexpr int ALLOC = (BYTES + 1024) > 116 * 1024 ? BYTES + 1024 : 116 * 1024;
 };
 
 template <int KS>
@@ -180,8 +209,10 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *afull = tempty + 2;
+    uint64_t *tempty = tfull + NBUF;
+    uint64_t *afull = tempty + NBUF;
+    uint64_t *aempty = afull + 1;
+    uint64_t *drain = aempty + 1;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
     volatile int *s_abort = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
     int *s_flag = reinterpret_cast<int *>(sm + L::MISC_OFF + 8);
@@ -195,19 +226,21 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&tfull[0], 1);
-        mbar_init(&tfull[1], 1);
-        mbar_init(&tempty[0], EPI_WARPS);
-        mbar_init(&tempty[1], EPI_WARPS);
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], EPI_WARPS);
+        }
         mbar_init(afull, 1);
+        mbar_init(aempty, 1);
+        mbar_init(drain, 1);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 0) {  // two accumulators of N fp32 columns x 128 lanes
+    if (warp == 0) {  // all 512 TMEM columns: NBUF accumulators of N fp32 columns x 128 lanes
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(s_tmem)),
-                     "r"(2 * N));
+                     "r"(NBUF * N));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -216,43 +249,53 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     const uint32_t tmem = *s_tmem;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
 
-    if (warp == EPI_WARPS) {
-        // ------------------------------------------------ producer + MMA issue
+    if (warp == TMA_WARP) {
+        // -------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t g_load = 0, g_mma = 0, item_no = 0, item_start = 0;
-            int64_t col0 = 0;
-            bool ok = true, a_pending = false;
-            auto issue_load = [&](uint32_t gl) -> bool {
-                const int st = gl % STAGES;
-                if (gl >= (uint32_t)STAGES && !mbar_wait(&empty[st], ((gl / STAGES) - 1) & 1, s_abort))
-                    return false;
-                mbar_expect_tx(&full[st], KS * SLAB_BYTES);
-                uint8_t *dst = sB + st * KS * SLAB_BYTES;
-                const int y = (int)(col0 + (int64_t)(gl - item_start) * N);
-                for (int s = 0; s < KS; ++s) tma_load_2d(dst + s * SLAB_BYTES, &tmB, &full[st], s * SLAB, y);
-                return true;
-            };
+            uint32_t g = 0, item_no = 0, issued[STAGES] = {};
+            bool ok = true, a_out = false;
             for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++item_no) {
                 const int tile = (int)(item / A.splits), split = (int)(item % A.splits);
-                col0 = (int64_t)split * A.cols_per_split;
-                const int nch = (int)((min(col0 + A.cols_per_split, A.cols_pad) - col0) / N);
-                item_start = g_mma;
-                const uint32_t end = g_mma + nch;
-                // the row tile is overwritten only after every MMA reading it finished
-                if (g_mma > 0 && !mbar_wait(&tfull[(g_mma - 1) & 1], ((g_mma - 1) >> 1) & 1, s_abort)) {
-                    ok = false;
-                    break;
-                }
+                const int64_t c0 = (int64_t)split * A.cols_per_split;
+                const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
+                // the row tile is overwritten only after every MMA of the previous item
+                if (item_no > 0 && !(ok = mbar_wait(aempty, (item_no - 1) & 1, s_abort))) break;
                 mbar_expect_tx(afull, KS * SLAB_BYTES);
                 for (int s = 0; s < KS; ++s) tma_load_2d(sA + s * SLAB_BYTES, &tmA, afull, s * SLAB, tile * M);
-                a_pending = true;
-                while (ok && g_load < end && g_load < g_mma + STAGES) ok = issue_load(g_load++);
-                if (ok) ok = mbar_wait(afull, item_no & 1, s_abort);
-                if (ok) a_pending = false;
-                for (; ok && g_mma < end; ++g_mma) {
-                    const int st = g_mma % STAGES, b = g_mma & 1;
-                    if (!mbar_wait(&full[st], (g_mma / STAGES) & 1, s_abort)) { ok = false; break; }
-                    if (g_mma >= 2 && !mbar_wait(&tempty[b], ((g_mma >> 1) - 1) & 1, s_abort)) { ok = false; break; }
+                a_out = true;
+                for (int ch = 0; ch < nch && ok; ++ch, ++g) {
+                    const int st = g % STAGES;
+                    if (g >= (uint32_t)STAGES && !(ok = mbar_wait(&empty[st], ((g / STAGES) - 1) & 1, s_abort)))
+                        break;
+                    mbar_expect_tx(&full[st], KS * SLAB_BYTES);
+                    uint8_t *dst = sB + st * KS * SLAB_BYTES;
+                    for (int s = 0; s < KS; ++s)
+                        tma_load_2d(dst + s * SLAB_BYTES, &tmB, &full[st], s * SLAB, (int)(c0 + (int64_t)ch * N));
+                    ++issued[st];
+                }
+            }
+            if (!ok) {  // wait (bounded) for the loads this block put in flight
+                if (a_out) mbar_drain(afull, (item_no & 1) ^ 0);
+                for (int st = 0; st < STAGES; ++st)
+                    if (issued[st]) mbar_drain(&full[st], (issued[st] - 1) & 1);
+                atomicExch(&A.st->wait_timeout, 1);
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            uint32_t g = 0, item_no = 0;
+            bool ok = true, issued_any = false;
+            for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++item_no) {
+                const int split = (int)(item % A.splits);
+                const int64_t c0 = (int64_t)split * A.cols_per_split;
+                const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
+                if (!(ok = mbar_wait(afull, item_no & 1, s_abort))) break;
+                for (int ch = 0; ch < nch; ++ch, ++g) {
+                    const int st = g % STAGES, b = g % NBUF;
+                    if (!(ok = mbar_wait(&full[st], (g / STAGES) & 1, s_abort))) break;
+                    if (g >= (uint32_t)NBUF && !(ok = mbar_wait(&tempty[b], ((g / NBUF) - 1) & 1, s_abort)))
+                        break;
                     tc_fence_after();
                     const uint8_t *bst = sB + st * KS * SLAB_BYTES;
                     for (int k = 0; k < ksteps; ++k) {
@@ -261,25 +304,27 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                         mma_bf16(tmem + (uint32_t)(b * N), smem_desc(sA + slab * SLAB_BYTES) + adv,
                                  smem_desc(bst + slab * SLAB_BYTES) + adv, k > 0 ? 1u : 0u);
                     }
+                    issued_any = true;
                     mma_commit(&empty[st]);
                     mma_commit(&tfull[b]);
-                    if (g_load < end) ok = issue_load(g_load++);
                 }
+                if (ok) mma_commit(aempty);
             }
             if (!ok) {
-                // give up: wait (bounded) for what this block already put in flight
-                if (a_pending) mbar_drain(afull, item_no & 1);
-                for (uint32_t g = g_mma; g < g_load; ++g) mbar_drain(&full[g % STAGES], (g / STAGES) & 1);
-                if (g_mma > 0) mbar_drain(&tfull[(g_mma - 1) & 1], ((g_mma - 1) >> 1) & 1);
+                if (issued_any) {  // wait (bounded) until the issued MMAs are done
+                    mma_commit(drain);
+                    mbar_drain(drain, 0);
+                }
                 atomicExch(&A.st->wait_timeout, 1);
             }
         }
     } else {
         // -------------------------------------------------------- epilogue
-        const int q = warp & 3, h = warp >> 2;
+        const int q = warp & 3, h = warp >> 2;  // TMEM lane quarter, column quarter
         const int r = q * 32 + lane;  // row of the tile owned by this thread
-        const int etid = threadIdx.x;  // 0..255
-        uint32_t g_epi = 0;
+        const int etid = threadIdx.x;  // 0 .. EPI_THREADS-1
+        const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * QCOLS);
+        uint32_t g = 0;
         for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
             const int tile = (int)(item / A.splits), split = (int)(item % A.splits);
             const int64_t c0 = (int64_t)split * A.cols_per_split;
@@ -289,32 +334,35 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             float2 acc[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
-            for (int ch = 0; ch < nch; ++ch, ++g_epi) {
-                const int b = g_epi & 1;
-                // every lane polls; the warp reconverges before the warp-wide TMEM load
-                const bool ready = mbar_wait(&tfull[b], (g_epi >> 1) & 1, s_abort);
-                if (!__all_sync(0xffffffffu, ready)) break;
+            float va[32], vb[32];
+            // the item's first chunk: wait, load, release the accumulator
+            bool ok = mbar_wait_warp(&tfull[g % NBUF], (g / NBUF) & 1, s_abort);
+            if (ok) {
                 tc_fence_after();
-                float va[32], vb[32];
-                const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * N + h * 64);
-                tmem_ld32(ta, va);
-                tmem_ld32(ta + 32, vb);
-                tmem_wait_ld();
+                tmem_ld32(tlane + (uint32_t)((g % NBUF) * N), va);
+                tmem_wait_ld(va);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[b]);
+                if (lane == 0) mbar_arrive(&tempty[g % NBUF]);
+            }
+            for (int ch = 0; ch < nch && ok; ++ch, ++g) {
+                const bool more = ch + 1 < nch;
+                if (more) {  // start loading the next chunk before this chunk's exponentials
+                    const uint32_t gn = g + 1;
+                    ok = mbar_wait_warp(&tfull[gn % NBUF], (gn / NBUF) & 1, s_abort);
+                    if (ok) {
+                        tc_fence_after();
+                        tmem_ld32(tlane + (uint32_t)((gn % NBUF) * N), vb);
+                    }
+                }
                 // running maximum, refreshed lazily (terms stay <= 2^8)
-                float p[8];
+                float p[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 4; ++j)
                     p[j] = fmax3(fmax3(va[8 * j], va[8 * j + 1], va[8 * j + 2]),
                                  fmax3(va[8 * j + 3], va[8 * j + 4], va[8 * j + 5]),
                                  fmaxf(va[8 * j + 6], va[8 * j + 7]));
-                    p[4 + j] = fmax3(fmax3(vb[8 * j], vb[8 * j + 1], vb[8 * j + 2]),
-                                     fmax3(vb[8 * j + 3], vb[8 * j + 4], vb[8 * j + 5]),
-                                     fmaxf(vb[8 * j + 6], vb[8 * j + 7]));
-                }
-                const float cm = fmax3(fmax3(p[0], p[1], p[2]), fmax3(p[3], p[4], p[5]), fmaxf(p[6], p[7]));
+                const float cm = fmax3(p[0], p[1], fmaxf(p[2], p[3]));
                 if (cm > m + kLazyMax) {
                     const float sc = ex2_approx(m - cm);
 #pragma unroll
@@ -328,11 +376,6 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                     const float2 u0 = __fadd2_rn(make_float2(va[2 * j], va[2 * j + 1]), nm);
                     acc[j & 3] = __fadd2_rn(acc[j & 3], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
                 }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float2 u0 = __fadd2_rn(make_float2(vb[2 * j], vb[2 * j + 1]), nm);
-                    acc[j & 3] = __fadd2_rn(acc[j & 3], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
-                }
                 float cs = 0.0f;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -340,31 +383,43 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                     acc[u] = make_float2(0.f, 0.f);
                 }
                 tot += cs;
+                if (more && ok) {
+                    tmem_wait_ld(vb);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[(g + 1) % NBUF]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) va[i] = vb[i];
+                }
             }
-            // merge the two column halves of each row, then the column splits
+            // merge the column quarters of each row, then the column splits
             s_merge[h * M + r] = make_float2(m, tot);
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
             // one thread samples the abort flag, so every epilogue thread takes
             // the same path through the named barriers that follow
             if (etid == 0) *s_decide = *s_abort;
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
             const bool aborted = *s_decide != 0;
             if (!aborted && h == 0) {
-                const float2 o = s_merge[M + r];
-                const float M2 = fmaxf(m, o.x);
-                const float S2 = tot * ex2_approx(m - M2) + o.y * ex2_approx(o.x - M2);
+                float M2 = m;
+                for (int u = 1; u < EPI_WARPS / 4; ++u) M2 = fmaxf(M2, s_merge[u * M + r].x);
+                float S2 = tot * ex2_approx(m - M2);
+                for (int u = 1; u < EPI_WARPS / 4; ++u) {
+                    const float2 o = s_merge[u * M + r];
+                    S2 += o.y * ex2_approx(o.x - M2);
+                }
                 const int64_t row = (int64_t)tile * M + r;
                 if (row < A.rows) A.part[(int64_t)split * A.tiles * M + row] = make_float2(M2, S2);
             }
             if (aborted) break;
-            finish_tile<256, M, 1>(A, tile, etid, s_red, s_flag);
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            finish_tile<EPI_THREADS, M, 1>(A, tile, etid, s_red, s_flag);
+            asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * N));
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NBUF * N));
 }
 
 }  // namespace tc
