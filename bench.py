@@ -52,13 +52,21 @@ def _args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="w2", choices=["w1", "w2", "w3", "w4", "w5"])
+    ap.add_argument("--n", type=int, default=None, help="replica size of the workload (rows)")
+    ap.add_argument("--m", type=int, default=None, help="replica size of the workload (columns)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
 
-def _workload(name):
+def _workload(name, n=None, m=None):
+    """The named workload, or a same-recipe replica with n rows / m columns."""
     from log_domain_sinkhorn_online_b200 import workloads
-    return workloads.ALL[name]()
+    kw = {}
+    if n is not None:
+        kw["n"] = n
+    if m is not None:
+        kw["m"] = m
+    return workloads.ALL[name](**kw)
 
 
 class Clocks:
@@ -211,7 +219,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = _workload(args.workload)
+    w = _workload(args.workload, args.n, args.m)
     times, units = [], 0
     for it in range(args.warmup + args.steps):
         cb = _cpu_baseline(w, target_s=8.0)
@@ -233,7 +241,7 @@ def run_ours(args):
     import log_domain_sinkhorn_online_b200 as ot
     rank, world, dist = _dist_init(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = _workload(args.workload)
+    w = _workload(args.workload, args.n, args.m)
     step = Step(ot, w, dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
