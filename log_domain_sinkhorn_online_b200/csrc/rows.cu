@@ -12,10 +12,12 @@
 //   e2_ij = A_i + B_j + sum_q P_iq y'_jq,
 //   A_i = kappa (f_i - c |x'_i|^2), B_j = kappa (g_j - c |y'_j|^2), P_i = 2 c kappa x'_i,
 // all in float64 (FlashSinkhorn 2, section D.3: accurate evaluation is done in
-// FP64). Then e2 = k + r with k = rint(e2), |r| <= 1/2; T = 2^r (MUFU ex2 on
-// the float r, relative error ~2^-22) scaled by 2^k through the exponent
+// FP64). Then e2 = k + r with k the nearest integer, |r| <= 1/2; T = 2^r (MUFU
+// ex2 on the float r, relative error ~2^-22) scaled by 2^k through the exponent
 // field, with a two-step scaling into the subnormal range. A massless side
-// (potential -inf) gives e2 = -inf and T = 0.
+// (potential -inf) gives e2 = -inf and T = 0. The row passes keep their sums in
+// compensated float32 (and maxima/counts exactly), so each entry costs one
+// conversion and one ex2 on the XU pipe.
 #include "runtime.h"
 
 namespace ot {
@@ -23,8 +25,12 @@ namespace ot {
 __device__ __forceinline__ float exp2_split(double e2) {
     if (!(e2 > -152.0)) return 0.0f;          // below half the smallest subnormal
     if (e2 >= 128.0) return INFINITY;
-    const int k = __double2int_rn(e2);
-    const float p = ex2_approx((float)(e2 - (double)k));  // in [2^-1/2, 2^1/2]
+    // nearest integer k by adding 1.5 * 2^52 (ulp 1 there): k lands in the low
+    // mantissa bits and e2 - k is exact, so the only conversion left is r -> float
+    const double big = 6755399441055744.0;
+    const double t = e2 + big;
+    const int k = __double2loint(t);
+    const float p = ex2_approx((float)(e2 - (t - big)));  // in [2^-1/2, 2^1/2]
     if (k >= -125) return __int_as_float(__float_as_int(p) + (k << 23));
     return p * __int_as_float((k + 64 + 127) << 23) * 5.42101086242752217e-20f;  // * 2^-64
 }
@@ -75,62 +81,68 @@ __device__ __forceinline__ void load_row(const float *pts, const float *pot, int
 }
 
 // ------------------------------------------------------------ materializer
-// Block: 256 threads x 4 consecutive columns (1024 columns) x 16 rows of the
-// row list. Each thread keeps its 4 columns' float64 data in registers (d <= 3)
-// and streams 16 rows of float4 evict-first stores, coalesced per warp.
-constexpr int kMtThreads = 256, kMtRows = 16;
-
+// Block: 256 threads x 4 consecutive columns (1024 columns). A block keeps its
+// columns' float64 data in registers (d <= 3) and walks a range of up to 256
+// rows of the row list, staged 32 at a time through shared memory, four rows
+// in flight; each row is one coalesced float4 evict-first store per thread.
+constexpr int kMtThreads = 256, kMtStage = 32, kMtRowsPerBlock = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kMtThreads) materialize_kernel(MatArgs M) {
-    __shared__ double sA[kMtRows], sP[kMtRows][D > 0 ? D : kMaxD];
-    __shared__ int sValid[kMtRows];
+    __shared__ double sA[kMtStage], sP[kMtStage][D > 0 ? D : kMaxD];
+    __shared__ int sValid[kMtStage];
     const int tid = threadIdx.x;
-    const int64_t r0 = (int64_t)blockIdx.y * kMtRows;
     const int d = D > 0 ? D : M.d;
-    if (tid < kMtRows) {
-        const int64_t r = r0 + tid;
-        int ok = 0;
-        if (r < M.k) {
-            const int64_t i = M.row_idx[r];
-            if (i >= 0 && i < M.n) {
-                ok = 1;
-                load_row(M.x, M.f, i, d, M.o, M.prm->kappa, M.prm->c, &sA[tid], sP[tid]);
-            } else {
-                atomicExch(M.bad, 1);
-            }
-        }
-        sValid[tid] = ok;
-    }
-    __syncthreads();
     const int64_t j0 = ((int64_t)blockIdx.x * kMtThreads + tid) * 4;
-    if (j0 >= M.m) return;
-    const int ncol = (int)min((int64_t)4, M.m - j0);
+    const int ncol = j0 < M.m ? (int)min((int64_t)4, M.m - j0) : 0;
     constexpr int DS = (D > 0 ? D : 1) + 1;
     double cd[4][DS];
     if (D > 0) {
+#pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int q = 0; q < DS; ++q)
                 cd[u][q] = u < ncol ? M.dcol[(j0 + u) * DS + q] : -INFINITY;
     }
-    for (int rr = 0; rr < kMtRows; ++rr) {
-        if (!sValid[rr]) continue;
-        const int64_t r = r0 + rr;
-        float t[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (D > 0)
-                t[u] = u < ncol ? plan_entry<D>(sA[rr], sP[rr], cd[u], d) : 0.0f;
-            else
-                t[u] = u < ncol ? plan_entry<0>(sA[rr], sP[rr], M.dcol + (j0 + u) * (d + 1), d)
-                                : 0.0f;
+    const int64_t rb0 = (int64_t)blockIdx.y * kMtRowsPerBlock;
+    const int64_t rb1 = min(rb0 + kMtRowsPerBlock, M.k);
+    for (int64_t s0 = rb0; s0 < rb1; s0 += kMtStage) {
+        __syncthreads();
+        if (tid < kMtStage) {
+            const int64_t r = s0 + tid;
+            int ok = 0;
+            if (r < rb1) {
+                const int64_t i = M.row_idx[r];
+                if (i >= 0 && i < M.n) {
+                    ok = 1;
+                    load_row(M.x, M.f, i, d, M.o, M.prm->kappa, M.prm->c, &sA[tid], sP[tid]);
+                } else {
+                    atomicExch(M.bad, 1);
+                }
+            }
+            sValid[tid] = ok;
         }
-        float *dst = M.out + r * M.m + j0;
-        if (M.vec && ncol == 4) {
-            __stcs(reinterpret_cast<float4 *>(dst), make_float4(t[0], t[1], t[2], t[3]));
-        } else {
-            for (int u = 0; u < ncol; ++u) __stcs(dst + u, t[u]);
+        __syncthreads();
+        if (ncol == 0) continue;
+        const int nr = (int)min((int64_t)kMtStage, rb1 - s0);
+#pragma unroll 4
+        for (int rr = 0; rr < nr; ++rr) {
+            if (!sValid[rr]) continue;
+            float t[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (D > 0)
+                    t[u] = u < ncol ? plan_entry<D>(sA[rr], sP[rr], cd[u], d) : 0.0f;
+                else
+                    t[u] = u < ncol ? plan_entry<0>(sA[rr], sP[rr], M.dcol + (j0 + u) * (d + 1), d)
+                                    : 0.0f;
+            }
+            float *dst = M.out + (s0 + rr) * M.m + j0;
+            if (M.vec && ncol == 4) {
+                __stcs(reinterpret_cast<float4 *>(dst), make_float4(t[0], t[1], t[2], t[3]));
+            } else {
+                for (int u = 0; u < ncol; ++u) __stcs(dst + u, t[u]);
+            }
         }
     }
 }
@@ -162,9 +174,15 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
             sA[tid] = -INFINITY;
     }
     __syncthreads();
-    double acc[kRpRows];
+    // per row: max (OP_MAX), count (OP_COUNT) or a compensated float sum (OP_SUM)
+    float acc[kRpRows], comp[kRpRows];
+    int cnt[kRpRows];
 #pragma unroll
-    for (int r = 0; r < kRpRows; ++r) acc[r] = OP == OP_MAX ? -1.0 : 0.0;
+    for (int r = 0; r < kRpRows; ++r) {
+        acc[r] = OP == OP_MAX ? -1.0f : 0.0f;
+        comp[r] = 0.0f;
+        cnt[r] = 0;
+    }
     constexpr int DS = (D > 0 ? D : 1) + 1;
     for (int64_t j = tid; j < R.cols; j += kRpThreads) {
         double cd[DS];
@@ -177,14 +195,20 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
         for (int r = 0; r < kRpRows; ++r) {
             const float t = D > 0 ? plan_entry<D>(sA[r], sP[r], cd, d)
                                   : plan_entry<0>(sA[r], sP[r], col, d);
-            if (OP == OP_MAX) acc[r] = fmax(acc[r], (double)t);
-            if (OP == OP_COUNT) acc[r] += (t >= R.thr) ? 1.0 : 0.0;
-            if (OP == OP_SUM) acc[r] += (double)t;
+            if (OP == OP_MAX) acc[r] = fmaxf(acc[r], t);
+            if (OP == OP_COUNT) cnt[r] += (t >= R.thr) ? 1 : 0;
+            if (OP == OP_SUM) {  // Kahan: the error stays ~2^-24 of the sum
+                const float yv = t - comp[r];
+                const float u = acc[r] + yv;
+                comp[r] = (u - acc[r]) - yv;
+                acc[r] = u;
+            }
         }
     }
 #pragma unroll
     for (int r = 0; r < kRpRows; ++r) {
-        double v = acc[r];
+        double v = OP == OP_SUM ? (double)acc[r] - (double)comp[r]
+                 : OP == OP_COUNT ? (double)cnt[r] : (double)acc[r];
         for (int off = 16; off > 0; off >>= 1) {
             const double o2 = __shfl_xor_sync(0xffffffffu, v, off);
             v = OP == OP_MAX ? fmax(v, o2) : v + o2;
@@ -292,14 +316,14 @@ cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, co
 
 cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s) {
     const int64_t col_blocks = (M.m + kMtThreads * 4 - 1) / (kMtThreads * 4);
-    // at most 65535 row groups per launch: split long row lists
-    const int64_t max_rows = (int64_t)65535 * kMtRows;
+    // at most 65535 row ranges per launch: split long row lists
+    const int64_t max_rows = (int64_t)65535 * kMtRowsPerBlock;
     for (int64_t r = 0; r < M.k; r += max_rows) {
         MatArgs A = M;
         A.row_idx = M.row_idx + r;
         A.out = M.out + r * M.m;
         A.k = min(max_rows, M.k - r);
-        dim3 grid((unsigned)col_blocks, (unsigned)((A.k + kMtRows - 1) / kMtRows));
+        dim3 grid((unsigned)col_blocks, (unsigned)((A.k + kMtRowsPerBlock - 1) / kMtRowsPerBlock));
         switch (M.d) {
             case 1: materialize_kernel<1><<<grid, kMtThreads, 0, s>>>(A); break;
             case 2: materialize_kernel<2><<<grid, kMtThreads, 0, s>>>(A); break;
