@@ -309,7 +309,9 @@ def run_ours(args):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded point clouds; recipe in log_domain_sinkhorn_online_b200/workloads.py)",
                 "config": _config(w, world, info),
-                "roofline": {"bound": "alu", "kernel": "hs_lowd_kernel (fused f/g half-step)" if w.d <= 3
+                "roofline": {"bound": "alu", "kernel": ("hs_loop_kernel (device-resident f/g half-steps)"
+                                                        if float(w.n) * w.m <= 2.0 ** 28 else
+                                                        "hs_lowd_kernel (fused f/g half-step)") if w.d <= 3
                              else "hs_tc_kernel (fused f/g half-step, tcgen05 x.y)" if w.d >= 16
                              else "hs_generic_kernel (fused f/g half-step)",
                              "achieved": achieved, "peak": peak_tex2, "unit": "Tex2/s",

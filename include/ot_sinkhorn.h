@@ -95,6 +95,11 @@ typedef struct ot_options {
     int32_t tensor_cores;     /* 16 <= d <= 64: 1 (default) computes x.y on the tcgen05
                                  tensor cores (bf16 splits, fp32 accumulation); 0 uses
                                  the CUDA-core FMA kernel */
+    int32_t device_loop;      /* d <= 3: run the iterations inside one cooperative
+                                 kernel per chunk (no per-half-step launches): -1
+                                 (default) for problems up to 2^28 pairs, 0 never,
+                                 1 always */
+    int32_t reserved1;
 } ot_options;
 
 /* -------------------------------------------------------- solve report   */
@@ -130,7 +135,7 @@ OT_API const char *ot_last_error_string(void);
 
 /* Default options (warm_start 0, check_every 16, use_graphs 1,
  * iters_per_stage 20, scale_value 1, eps_init 0, eps_decay 0.7, timing 0,
- * col_splits 0, rows_per_thread 0, tensor_cores 1). */
+ * col_splits 0, rows_per_thread 0, tensor_cores 1, device_loop -1). */
 OT_API void ot_options_default(ot_options *opt);
 
 /* ------------------------------------------------- ot_sinkhorn_pointcloud

@@ -88,7 +88,7 @@ class Plan:
 def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None, warm_start=False,
              check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,
              timing=False, col_splits=0, rows_per_thread=0, tensor_cores=True,
-             stream=None) -> Plan:
+             device_loop=-1, stream=None) -> Plan:
     """Solves on the GPU; x [n,d], y [m,d], a [n], b [m] float32 CUDA tensors."""
     import torch
     x, y = _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y")
@@ -108,6 +108,7 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
     opt.col_splits = int(col_splits)
     opt.rows_per_thread = int(rows_per_thread)
     opt.tensor_cores = int(bool(tensor_cores))
+    opt.device_loop = int(device_loop)
     if isinstance(scale, str):
         sc = _SCALES[scale]
     else:

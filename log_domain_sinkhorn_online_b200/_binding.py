@@ -39,7 +39,8 @@ class OtOptions(ctypes.Structure):
                 ("scale_value", ctypes.c_double), ("eps_init", ctypes.c_double),
                 ("eps_decay", ctypes.c_double), ("timing", ctypes.c_int32),
                 ("col_splits", ctypes.c_int32), ("rows_per_thread", ctypes.c_int32),
-                ("tensor_cores", ctypes.c_int32)]
+                ("tensor_cores", ctypes.c_int32), ("device_loop", ctypes.c_int32),
+                ("reserved1", ctypes.c_int32)]
 
 
 class OtInfo(ctypes.Structure):

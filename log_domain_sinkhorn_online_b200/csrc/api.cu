@@ -109,6 +109,10 @@ struct ot_plan {
     int64_t *counts = nullptr;
     HostScalars *hs = nullptr;  // pinned
     int kp = 0;                 // tensor-core path: bf16 K extent of the operand tables
+    bool use_loop = false;      // device-resident iterations (loop.cu)
+    int loop_grid = 0;
+    unsigned *bar = nullptr;    // grid barrier: count, generation
+    double *blk_resid = nullptr;
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
     cudaStream_t s_int = nullptr;
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
@@ -253,6 +257,7 @@ HalfStep make_step(const ot_plan *p, int side, int parity) {
     A.cols_per_split = rows.cps;
     A.splits = rows.splits;
     A.tiles = rows.tiles;
+    A.tile_rows = rows.tile;
     A.dp = p->dp;
     A.side = side;
     A.part = p->part;
@@ -308,7 +313,39 @@ cudaError_t launch_iteration(const ot_plan *p, int parity) {
 // Runs `iters` iterations starting at global parity `parity0`, in chunks of
 // graph_len (replayed graphs when enabled). With `check`, the stop flag is
 // read after every chunk. Returns OT status.
+// Device-resident path: chunks of up to kLoopChunk iterations per cooperative launch.
+constexpr int kLoopChunk = 256;
+
+int run_loop(ot_plan *p, int parity0, int iters, bool check) {
+    LoopArgs L{};
+    L.f[0] = make_step(p, 0, 0);
+    L.f[1] = make_step(p, 0, 1);
+    L.g[0] = L.g[1] = make_step(p, 1, 0);
+    L.bar_count = p->bar;
+    L.bar_gen = p->bar + 1;
+    L.blk_resid = p->blk_resid;
+    int i = 0;
+    while (i < iters) {
+        const int len = std::min(kLoopChunk, iters - i);
+        L.iters = len;
+        L.parity0 = (parity0 + i) & 1;
+        OT_CU(cudaMemsetAsync(p->bar, 0, sizeof(unsigned), p->s_int));  // arrivals
+        OT_CU(mark(p));
+        OT_CU(launch_loop(p->d, L, p->loop_grid, p->s_int));
+        OT_CU(mark(p));
+        p->launches += 1;
+        i += len;
+        if (check || i < iters) {
+            int rc = read_state(p);
+            if (rc != OT_OK) return rc;
+            if (p->hs->st.stop || p->hs->st.wait_timeout) break;
+        }
+    }
+    return OT_OK;
+}
+
 int run_iterations(ot_plan *p, int parity0, int iters, bool check, bool use_graphs) {
+    if (p->use_loop) return run_loop(p, parity0, iters, check);
     int i = 0;
     while (i < iters) {
         const int len = std::min(p->graph_len, iters - i);
@@ -381,6 +418,7 @@ void ot_options_default(ot_options *opt) {
     opt->col_splits = 0;
     opt->rows_per_thread = 0;
     opt->tensor_cores = 1;
+    opt->device_loop = -1;
 }
 
 void ot_plan_destroy(ot_plan *plan) { plan_free(plan); }
@@ -411,11 +449,24 @@ int plan_setup(ot_plan *p, const ot_options &o) {
     p->sy.cnt = p->m;
     p->sx.pad = round_up(p->n, padq);
     p->sy.pad = round_up(p->m, padq);
-    int rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx, o.col_splits,
+    if (p->kind == 0 && o.device_loop != 0 &&
+        (o.device_loop == 1 || (double)p->n * (double)p->m <= (double)(1ll << 28))) {
+        const int bps = loop_blocks_per_sm(p->d);
+        if (bps > 0) {
+            p->use_loop = true;
+            p->loop_grid = bps * p->sm_count;
+            // both half-steps run 2 rows per thread inside the loop kernel
+            choose_splits(p->n, p->sy.pad, 2, kHsThreads * 2, p->loop_grid, p->sx, o.col_splits);
+            choose_splits(p->m, p->sx.pad, 2, kHsThreads * 2, p->loop_grid, p->sy, o.col_splits);
+        }
+    }
+    int rc = OT_OK;
+    if (!p->use_loop)
+        rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx, o.col_splits,
                           o.rows_per_thread);
     if (rc != OT_OK) return rc;
-    if ((rc = choose_shape(p->kind, p->dim, p->sm_count, p->m, p->sx.pad, p->sy, o.col_splits,
-                           o.rows_per_thread)) != OT_OK)
+    if (!p->use_loop && (rc = choose_shape(p->kind, p->dim, p->sm_count, p->m, p->sx.pad, p->sy,
+                                           o.col_splits, o.rows_per_thread)) != OT_OK)
         return rc;
     const int64_t part_cnt = std::max((int64_t)p->sx.splits * p->sx.tiles * p->sx.tile,
                                       (int64_t)p->sy.splits * p->sy.tiles * p->sy.tile);
@@ -441,6 +492,8 @@ int plan_setup(ot_plan *p, const ot_options &o) {
         p->part = cv.take<float2>(part_cnt);
         p->tile_cnt = cv.take<unsigned>(tiles);
         p->tile_resid = cv.take<double>(tiles);
+        p->bar = cv.take<unsigned>(2);
+        p->blk_resid = cv.take<double>(std::max(p->loop_grid, 1));
         if (pass == 0) OT_CU(cudaMalloc(&p->ws, cv.off));
     }
     if (p->kind == 2) {
@@ -452,6 +505,7 @@ int plan_setup(ot_plan *p, const ot_options &o) {
         if (e) return fail(OT_ERR_CUDA, "tensor map encoding failed (%d)", e);
     }
     OT_CU(cudaMemsetAsync(p->tile_cnt, 0, sizeof(unsigned) * tiles, p->s_int));
+    OT_CU(cudaMemsetAsync(p->bar, 0, sizeof(unsigned) * 2, p->s_int));
     OT_CU(cudaMemsetAsync(p->st, 0, sizeof(State), p->s_int));
     OT_CU(cudaMemsetAsync(p->ds, 0, sizeof(DevScalars), p->s_int));
     return OT_OK;

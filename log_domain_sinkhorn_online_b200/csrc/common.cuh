@@ -65,6 +65,7 @@ struct HalfStep {
     int64_t cols_per_split;    // multiple of kColPad (the last chunk of a split may be partial)
     int splits;                // column splits S
     int tiles;                 // row tiles
+    int tile_rows;             // rows per tile (partials are [splits][tiles*tile_rows])
     int dp;                    // row-table stride in floats
     int side;                  // 0: f-update (runs the stop test), 1: g-update
     float2 *part;              // [splits][tiles*tile] (running max, sum) partials

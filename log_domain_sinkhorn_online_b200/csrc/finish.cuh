@@ -13,6 +13,48 @@
 
 namespace ot {
 
+// New potential of one row from its merged (max M, sum S) over all columns:
+// writes pot_new[row] and the other half-step's column term, returns the
+// row's residual term |sum_j T_ij(old) - w_row|; *bad is set for a massful row
+// whose potential is not finite.
+__device__ __forceinline__ double finish_row(const HalfStep &A, int64_t row, float M, double S,
+                                             double eps, double kappa, double c, bool *bad) {
+    const float *xr = A.rowtab + row * (int64_t)A.dp;
+    double nrm = 0.0;
+    for (int q = 0; q < A.dp; ++q) nrm += (double)xr[q] * (double)xr[q];
+    const double wi = (double)A.w[row];
+    double pot = 0.0, term = 0.0;
+    if (wi == 0.0) {
+        pot = -INFINITY;  // massless row: empty row of the plan
+    } else if (!(S > 0.0)) {
+        pot = INFINITY;   // every column is massless: no finite potential
+        *bad = true;
+    } else {
+        const double L = (double)M + log2(S) - kappa * c * nrm;
+        pot = eps * log(wi) - L / kappa;
+        const double old = (double)__ldcg(A.pot_old + row);
+        term = fabs(exp2(kappa * old + L) - wi);
+    }
+    const float pf = (float)pot;
+    if (wi != 0.0 && !isfinite(pf)) *bad = true;
+    A.pot_new[row] = pf;
+    const double Gn = (wi == 0.0) ? -INFINITY : kappa * ((double)pf - c * nrm);
+    if (A.nxt_bf16) {
+        // three bf16 terms whose sum carries G to ~24 bits (-inf: first term only)
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(A.next_col) + row * A.nxt_a + A.nxt_b;
+        const __nv_bfloat16 g1 = __double2bfloat16(Gn);
+        const double r1 = isfinite(Gn) ? Gn - (double)__bfloat162float(g1) : 0.0;
+        const __nv_bfloat16 g2 = __double2bfloat16(r1);
+        const __nv_bfloat16 g3 = __double2bfloat16(r1 - (double)__bfloat162float(g2));
+        dst[0] = g1;
+        dst[1] = g2;
+        dst[2] = g3;
+    } else {
+        A.next_col[(row >> 1) * A.nxt_a + (row & 1) * A.nxt_l + A.nxt_b] = (float)Gn;
+    }
+    return term;
+}
+
 // Barrier among the THREADS threads that run finish_tile: the whole block
 // (BAR == 0) or a named barrier BAR (warp-specialised kernels).
 template <int THREADS, int BAR>
@@ -83,40 +125,7 @@ __device__ void finish_tile(const HalfStep &A, int tile, int tid, double *s_red,
     for (int k = 0; k < RPT; ++k) {
         const int64_t row = (int64_t)tile * TILE + k * THREADS + tid;
         if (k * THREADS + tid >= TILE || row >= A.rows) continue;
-        const float *xr = A.rowtab + row * (int64_t)A.dp;
-        double nrm = 0.0;
-        for (int q = 0; q < A.dp; ++q) nrm += (double)xr[q] * (double)xr[q];
-        const double wi = (double)A.w[row];
-        double pot = 0.0, term = 0.0;
-        if (wi == 0.0) {
-            pot = -INFINITY;  // massless row: empty row of the plan
-        } else if (!(S[k] > 0.0)) {
-            pot = INFINITY;   // every column is massless: no finite potential
-            bad = true;
-        } else {
-            const double L = (double)M[k] + log2(S[k]) - kappa * c * nrm;
-            pot = eps * log(wi) - L / kappa;
-            const double old = (double)A.pot_old[row];
-            term = fabs(exp2(kappa * old + L) - wi);
-        }
-        const float pf = (float)pot;
-        if (wi != 0.0 && !isfinite(pf)) bad = true;
-        A.pot_new[row] = pf;
-        const double Gn = (wi == 0.0) ? -INFINITY : kappa * ((double)pf - c * nrm);
-        if (A.nxt_bf16) {
-            // three bf16 terms whose sum carries G to ~24 bits (-inf: first term only)
-            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(A.next_col) + row * A.nxt_a + A.nxt_b;
-            const __nv_bfloat16 g1 = __double2bfloat16(Gn);
-            const double r1 = isfinite(Gn) ? Gn - (double)__bfloat162float(g1) : 0.0;
-            const __nv_bfloat16 g2 = __double2bfloat16(r1);
-            const __nv_bfloat16 g3 = __double2bfloat16(r1 - (double)__bfloat162float(g2));
-            dst[0] = g1;
-            dst[1] = g2;
-            dst[2] = g3;
-        } else {
-            A.next_col[(row >> 1) * A.nxt_a + (row & 1) * A.nxt_l + A.nxt_b] = (float)Gn;
-        }
-        rsum += term;
+        rsum += finish_row(A, row, M[k], S[k], eps, kappa, c, &bad);
     }
     if (bad) atomicExch(&A.st->nonfinite, 1);
     if (tid == 0) A.tile_cnt[tile] = 0;

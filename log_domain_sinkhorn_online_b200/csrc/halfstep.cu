@@ -24,6 +24,7 @@
 // The last tile to finish sums the residual partials in tile order (no float
 // atomics, so the result is deterministic) and runs the stop test.
 #include "finish.cuh"
+#include "lowd.cuh"
 
 namespace ot {
 
@@ -38,107 +39,16 @@ namespace ot {
 // splits to merge, on small problems).
 template <int D, int R>
 __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lowd_kernel(HalfStep A) {
-    constexpr int kHsRows = R;
-    constexpr int kHsTile = kHsThreads * R;
     __shared__ __align__(16) float4 sm[2][kHsChunk];
     __shared__ double s_red[kHsThreads / 32];
     __shared__ int s_flag;
     if (ld_volatile(&A.st->stop)) return;
-    const int tid = threadIdx.x;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
-    const float4 *rt4 = reinterpret_cast<const float4 *>(A.rowtab);
-
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int tile = (int)(item / A.splits);
         const int split = (int)(item % A.splits);
-
-        float2 xd[kHsRows][3];
-        float m[kHsRows], tot[kHsRows];
-        float2 nm[kHsRows], acc[kHsRows], acc2[kHsRows];
-#pragma unroll
-        for (int k = 0; k < kHsRows; ++k) {
-            const int64_t row = (int64_t)tile * kHsTile + k * kHsThreads + tid;
-            const float4 p = row < A.rows ? rt4[row] : make_float4(0.f, 0.f, 0.f, 0.f);
-            xd[k][0] = make_float2(p.x, p.x);
-            xd[k][1] = make_float2(p.y, p.y);
-            xd[k][2] = make_float2(p.z, p.z);
-            m[k] = kNegBig;
-            nm[k] = make_float2(-kNegBig, -kNegBig);
-            acc[k] = make_float2(0.f, 0.f);
-            acc2[k] = make_float2(0.f, 0.f);
-            tot[k] = 0.f;
-        }
-
-        const int64_t c0 = (int64_t)split * A.cols_per_split;
-        const int64_t span = min(c0 + A.cols_per_split, A.cols_pad) - c0;  // multiple of 8
-        const int nch = (int)((span + kHsChunk - 1) / kHsChunk);
-        const float4 *src = A.coltab + c0;
-        const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 p0 = tid < span ? src[tid] : zero4;
-        float4 p1 = tid + kHsThreads < span ? src[tid + kHsThreads] : zero4;
-
-#pragma unroll 1
-        for (int ch = 0; ch < nch; ++ch) {
-            float4 *buf = sm[ch & 1];
-            buf[tid] = p0;
-            buf[tid + kHsThreads] = p1;
-            __syncthreads();
-            const int64_t nb = (int64_t)(ch + 1) * kHsChunk;
-            if (ch + 1 < nch) {
-                p0 = nb + tid < span ? src[nb + tid] : zero4;
-                p1 = nb + kHsThreads + tid < span ? src[nb + kHsThreads + tid] : zero4;
-            }
-            const int ncols = (int)min((int64_t)kHsChunk, span - (int64_t)ch * kHsChunk);
-#pragma unroll 1
-            for (int q = 0; q < ncols; q += 8) {
-                float4 v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = buf[q + u];
-#pragma unroll
-                for (int k = 0; k < kHsRows; ++k) {
-                    float2 t[4];
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const float4 lo = v[2 * p], hi = v[2 * p + 1];
-                        float2 tt = __ffma2_rn(make_float2(lo.x, lo.y), xd[k][0],
-                                               make_float2(hi.z, hi.w));
-                        if (D >= 2) tt = __ffma2_rn(make_float2(lo.z, lo.w), xd[k][1], tt);
-                        if (D >= 3) tt = __ffma2_rn(make_float2(hi.x, hi.y), xd[k][2], tt);
-                        t[p] = tt;
-                    }
-                    const float cm = fmax3(fmax3(t[0].x, t[0].y, t[1].x), fmax3(t[1].y, t[2].x, t[2].y),
-                                           fmaxf(t[3].x, t[3].y));
-                    if (cm > m[k] + kLazyMax) {  // rare: refresh the running maximum
-                        const float sc = ex2_approx(m[k] - cm);
-                        acc[k] = __fmul2_rn(acc[k], make_float2(sc, sc));
-                        acc2[k] = __fmul2_rn(acc2[k], make_float2(sc, sc));
-                        tot[k] *= sc;
-                        m[k] = cm;
-                        nm[k] = make_float2(-cm, -cm);
-                    }
-                    const float2 u0 = __fadd2_rn(t[0], nm[k]), u1 = __fadd2_rn(t[1], nm[k]);
-                    const float2 u2 = __fadd2_rn(t[2], nm[k]), u3 = __fadd2_rn(t[3], nm[k]);
-                    acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
-                    acc2[k] = __fadd2_rn(acc2[k], make_float2(ex2_approx(u1.x), ex2_approx(u1.y)));
-                    acc[k] = __fadd2_rn(acc[k], make_float2(ex2_approx(u2.x), ex2_approx(u2.y)));
-                    acc2[k] = __fadd2_rn(acc2[k], make_float2(ex2_approx(u3.x), ex2_approx(u3.y)));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < kHsRows; ++k) {
-                tot[k] += (acc[k].x + acc[k].y) + (acc2[k].x + acc2[k].y);
-                acc[k] = make_float2(0.f, 0.f);
-                acc2[k] = make_float2(0.f, 0.f);
-            }
-        }
-
-        const int64_t stride = (int64_t)A.tiles * kHsTile;
-#pragma unroll
-        for (int k = 0; k < kHsRows; ++k) {
-            const int64_t row = (int64_t)tile * kHsTile + k * kHsThreads + tid;
-            if (row < A.rows) A.part[split * stride + row] = make_float2(m[k], tot[k]);
-        }
-        finish_tile<kHsThreads, kHsTile, 0>(A, tile, threadIdx.x, s_red, &s_flag);
+        lowd_item<D, R, false>(A, tile, split, sm);
+        finish_tile<kHsThreads, kHsThreads * R, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
     }
 }

@@ -14,6 +14,19 @@ int halfstep_blocks_per_sm(int kind, int dim, int rpt);
 cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,
                             cudaStream_t s);
 
+// loop.cu (device-resident iterations, d <= 3, 2 rows per thread)
+struct LoopArgs {
+    HalfStep f[2];          // f-update with the f buffers at parity 0 / 1
+    HalfStep g[2];          // g-update (same buffers; indexed like f)
+    int iters;              // iterations this launch may run
+    int parity0;            // parity of the f buffer holding the current state
+    unsigned *bar_count;    // grid barrier: arrivals
+    unsigned *bar_gen;      // grid barrier: generation
+    double *blk_resid;      // [grid] residual partial of each block
+};
+int loop_blocks_per_sm(int d);
+cudaError_t launch_loop(int d, const LoopArgs &L, int grid, cudaStream_t s);
+
 // halfstep_tc.cu (16 <= d <= 64: tensor-core path)
 int tc_ksteps(int d);
 int tc_slabs(int d);

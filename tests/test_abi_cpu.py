@@ -42,11 +42,11 @@ def test_version_and_defaults(B):
     o = B.ot_options_default()
     assert (o.warm_start, o.check_every, o.use_graphs, o.iters_per_stage) == (0, 16, 1, 20)
     assert (o.scale_value, o.eps_init, o.eps_decay) == (1.0, 0.0, 0.7)
-    assert (o.timing, o.col_splits, o.rows_per_thread, o.tensor_cores) == (0, 0, 0, 1)
+    assert (o.timing, o.col_splits, o.rows_per_thread, o.tensor_cores, o.device_loop) == (0, 0, 0, 1, -1)
 
 
 def test_struct_sizes_match_header_layout(B):
-    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 4 * 4
+    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4
     assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8
 
 

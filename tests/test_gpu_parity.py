@@ -234,3 +234,34 @@ def test_tensor_core_path_ragged_and_massless(ot, orc, n, m):
     f, g = _pots(plan)
     H.assert_potentials(f, f_ref, maxc, what="f")
     H.assert_potentials(g, g_ref, maxc, what="g")
+
+
+@pytest.mark.parametrize("loop", [0, 1])
+@pytest.mark.parametrize("d", [1, 3])
+def test_device_loop_and_launch_paths(ot, orc, loop, d):
+    """The same solve through per-half-step launches (loop=0) and through the
+    device-resident cooperative loop (loop=1): both against the oracle, with
+    the tol stop inside the loop (the count is checked like the launch path's)."""
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w2(n=1777, m=1501)
+    if d == 1:
+        w.x, w.y = w.x[:, :1].copy(), w.y[:, :1].copy()
+    plan, c, f_ref, g_ref, it_ref, r_ref = _solve_both(ot, orc, w, 300, tol=2e-3, device_loop=loop)
+    maxc = H.max_cost(w.x, w.y, c)
+    if plan.info.iterations != it_ref:
+        assert abs(plan.info.iterations - it_ref) <= 2
+        plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, it_ref, device_loop=loop)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+
+
+def test_device_loop_long_run_crosses_chunks(ot, orc):
+    """600 iterations: three cooperative launches of the loop kernel."""
+    w = _cloud(91, 900, 1100, 2, eps=0.03)
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 600, device_loop=1)
+    assert plan.info.iterations == 600
+    maxc = H.max_cost(w.x, w.y, c)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
