@@ -458,6 +458,12 @@ int plan_setup(ot_plan *p, const ot_options &o) {
             // both half-steps run 2 rows per thread inside the loop kernel
             choose_splits(p->n, p->sy.pad, 2, kHsThreads * 2, p->loop_grid, p->sx, o.col_splits);
             choose_splits(p->m, p->sx.pad, 2, kHsThreads * 2, p->loop_grid, p->sy, o.col_splits);
+            // no more blocks than there is work for: every block arrives at every barrier
+            const int64_t work = std::max({(int64_t)p->sx.tiles * p->sx.splits,
+                                           (int64_t)p->sy.tiles * p->sy.splits,
+                                           (std::max(p->n, p->m) + kHsThreads - 1) / kHsThreads,
+                                           (int64_t)1});
+            p->loop_grid = (int)std::min<int64_t>(p->loop_grid, work);
         }
     }
     int rc = OT_OK;

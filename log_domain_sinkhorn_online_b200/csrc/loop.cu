@@ -17,7 +17,7 @@
 // state before the update) without another barrier.
 //
 // All co-resident by construction (cooperative launch). The grid barrier waits
-// on a generation counter with a time limit (globaltimer): past it the kernel
+// on an arrival counter with a time limit (globaltimer): past it the kernel
 // records State::wait_timeout and every block leaves the loop. Data rewritten
 // inside the kernel (column tables, potentials, partials) is read with L1
 // bypassed.
@@ -43,22 +43,21 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
     return v;
 }
 
-// Grid-wide barrier for a cooperative launch. Returns false (uniformly per
-// block) if the wait gave up; then *err is set.
-__device__ bool grid_barrier(unsigned *count, unsigned *gen, int *err, volatile int *s_ok) {
+// Grid-wide barrier for a cooperative launch: a counter that only grows (the
+// host zeroes it before each launch). Barrier k of the launch is passed when
+// the counter reaches (k + 1) * gridDim.x; one release-add per block, acquire
+// polling by thread 0. Returns false (uniformly per block) if the wait gave up,
+// after setting *err.
+__device__ bool grid_barrier(unsigned *count, unsigned &k, int *err, volatile int *s_ok) {
     __syncthreads();
+    const unsigned target = (++k) * gridDim.x;
     if (threadIdx.x == 0) {
-        const unsigned g = ld_acquire_u32(gen);
-        __threadfence();
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
         int ok = 1;
-        if (atomicAdd(count, 1u) == gridDim.x - 1) {
-            atomicExch(count, 0u);
-            __threadfence();
-            atomicAdd(gen, 1u);
-        } else {
+        if (ld_acquire_u32(count) < target) {
             const uint64_t t0 = globaltimer();
-            while (ld_acquire_u32(gen) == g) {
-                __nanosleep(32);
+            while (ld_acquire_u32(count) < target) {
+                __nanosleep(20);
                 if (globaltimer() - t0 > kBarrierLimitNs) {
                     ok = 0;
                     atomicExch(err, 1);
@@ -66,7 +65,6 @@ __device__ bool grid_barrier(unsigned *count, unsigned *gen, int *err, volatile 
                 }
             }
         }
-        __threadfence();
         *s_ok = ok;
     }
     __syncthreads();
@@ -145,6 +143,7 @@ __global__ void __launch_bounds__(kHsThreads, 6) hs_loop_kernel(LoopArgs L) {
     int iter_done = ld_volatile(&st->iter_done);
     const double tol = L.f[0].prm->tol;
     bool bad = false;
+    unsigned nbar = 0;  // grid barriers passed in this launch
     for (int it = 0; it < L.iters; ++it) {
         // ------------------------------------------------------- f-update
         const HalfStep &F = L.f[par];
@@ -153,10 +152,10 @@ __global__ void __launch_bounds__(kHsThreads, 6) hs_loop_kernel(LoopArgs L) {
             __syncthreads();
             lowd_item<D, kLoopR, true>(F, (int)(item / F.splits), (int)(item % F.splits), sm);
         }
-        if (!grid_barrier(L.bar_count, L.bar_gen, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         const double br = merge_phase<kHsThreads>(F, s_red, &bad);
         if (threadIdx.x == 0) L.blk_resid[blockIdx.x] = br;
-        if (!grid_barrier(L.bar_count, L.bar_gen, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         const double R = grid_residual<kHsThreads>(L.blk_resid, s_red);
         if (blockIdx.x == 0 && threadIdx.x == 0) st->resid[0] = R;
         if (tol > 0.0 && iter_done >= 1 && R <= tol) {  // the same decision in every block
@@ -173,9 +172,9 @@ __global__ void __launch_bounds__(kHsThreads, 6) hs_loop_kernel(LoopArgs L) {
             __syncthreads();
             lowd_item<D, kLoopR, true>(G, (int)(item / G.splits), (int)(item % G.splits), sm);
         }
-        if (!grid_barrier(L.bar_count, L.bar_gen, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         merge_phase<kHsThreads>(G, s_red, &bad);
-        if (!grid_barrier(L.bar_count, L.bar_gen, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         ++iter_done;
         par ^= 1;
         if (blockIdx.x == 0 && threadIdx.x == 0) st->iter_done = iter_done;
