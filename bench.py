@@ -33,8 +33,10 @@ METRIC = "Sinkhorn pair-updates/s (n·m per half-step) and % of ex2/MUFU rooflin
 UNIT = "pair-updates/s"
 # MUFU ex2 peak: 148 SMs x 16 ex2 per clock per SM x 1.965 GHz (max SM clock)
 SMS, EX2_PER_CLK = 148, 16
-# DRAM traffic of one half-step launch from the committed ncu capture (bytes), or None
-HALFSTEP_TRAFFIC = None
+# DRAM bytes per half-step of the dominant kernel, from the committed ncu captures
+# (profiles/hs_loop_w2_8000.md: 874.5 KB per 512-half-step launch), keyed by
+# workload; None where no capture of the current kernel exists
+HALFSTEP_TRAFFIC = {"w2_gmm3d_8000": 874.5e3 / 512}
 
 
 def _peaks():
@@ -315,7 +317,8 @@ def run_ours(args):
                              else "hs_tc_kernel (fused f/g half-step, tcgen05 x.y)" if w.d >= 16
                              else "hs_generic_kernel (fused f/g half-step)",
                              "achieved": achieved, "peak": peak_tex2, "unit": "Tex2/s",
-                             "frac": achieved / peak_tex2, "traffic": HALFSTEP_TRAFFIC,
+                             "frac": achieved / peak_tex2,
+                             "traffic": HALFSTEP_TRAFFIC.get(w.name) if (args.n, args.m) == (None, None) else None,
                              "per_launch_us": per_launch_ms * 1e3,
                              "peak_note": f"148 SMs x 16 MUFU ex2/clk x {sm_max:.0f} MHz ({kind} sm_max)"},
                 "clocks": clk,
