@@ -119,13 +119,19 @@ def _dist_init(n_gpus):
     return rank, world, dist
 
 
-def _max_over_ranks(v, dist):
+def _max_over_ranks(v, dist, device="cuda"):
+    """The max of v over all ranks (the job's time is its slowest rank's)."""
     import torch
     if dist is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank, world, max_ms_per_step):
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (max_ms_per_step / 1e3)
 
 
 def _barrier(dist):
@@ -272,7 +278,7 @@ def run_ours(args):
     _barrier(dist)
     total_ms = _max_over_ranks(total_ms, dist)
     units = float(w.n) * float(w.m) * half_steps / args.steps  # pair-updates per step (this rank)
-    value = units * world / (total_ms / args.steps / 1e3)
+    value = weak_scaling_value(units, world, total_ms / args.steps)
 
     # ---- end to end through the public API: pinned host inputs in, results out
     host = [torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for v in (w.x, w.y, w.a, w.b)]

@@ -1,0 +1,128 @@
+"""The oracle's pins catch plausible mistakes: each test plants one mistake in a
+temporary copy of the oracle's C source (a flipped sign, a dropped factor, a max
+for a min, ...), builds it, and checks that the pin battery below fails on it
+while passing on the real oracle. Nothing here touches the real oracle's files.
+"""
+import importlib.util
+import math
+import os
+import shutil
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle")
+
+MUTANTS = {
+    "cost_sign_in_f_step": ("(g[j] - cost(x, y, i, j, d, c)) / eps", "(g[j] + cost(x, y, i, j, d, c)) / eps"),
+    "dropped_eps_on_log_weight": ("out = eps * log(a[i]) - eps * lse(v, m);", "out = log(a[i]) - eps * lse(v, m);"),
+    "plan_sign_of_g": ("exp((f[i] + g[j] - cost(x, y, i, j, d, c)) / eps)", "exp((f[i] - g[j] - cost(x, y, i, j, d, c)) / eps)"),
+    "plan_missing_eps": ("exp((f[i] + g[j] - cost(x, y, i, j, d, c)) / eps)", "exp((f[i] + g[j] - cost(x, y, i, j, d, c)))"),
+    "min_row_takes_max": ("if (rowmax[i] < thr) { thr = rowmax[i]; arg = i; }", "if (rowmax[i] > thr || thr == INFINITY) { thr = rowmax[i]; arg = i; }"),
+    "residual_wrong_sign": ("for (int64_t i = 0; i < n; ++i) r += fabs(rs[i] - a[i]);", "for (int64_t i = 0; i < n; ++i) r += fabs(rs[i] + a[i]);"),
+    "mean_scale_wrong_count": ("if (mode == 1) r /= ((double)n * (double)m);", "if (mode == 1) r /= ((double)n * (double)n);"),
+    "lse_no_shift_back": ("return mx + log(s);", "return log(s);"),
+    "g_step_uses_a_weight": ("out = eps * log(b[j]) - eps * lse(v, n);", "out = eps * log(b[0]) - eps * lse(v, n);"),
+}
+
+
+def _load_variant(tmp_path, name, old=None, new=None):
+    dst = tmp_path / f"oracle_{name}"
+    shutil.copytree(SRC, dst, ignore=shutil.ignore_patterns("_build", "__pycache__"))
+    if old is not None:
+        c = (dst / "sinkhorn_oracle.c").read_text()
+        assert old in c, f"mutation site for {name} not found"
+        (dst / "sinkhorn_oracle.c").write_text(c.replace(old, new, 1))
+    spec = importlib.util.spec_from_file_location(f"oracle_{name}", dst / "__init__.py",
+                                                  submodule_search_locations=[str(dst)])
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[spec.name] = mod
+    spec.loader.exec_module(mod)
+    mod.build(force=True)
+    return mod
+
+
+def _sqd(x, y):
+    xd, yd = np.asarray(x, np.float64), np.asarray(y, np.float64)
+    return ((xd[:, None, :] - yd[None]) ** 2).sum(-1)
+
+
+def _battery(orc):
+    """Returns the names of the pins that fail for this oracle build."""
+    failed = []
+    rng = np.random.default_rng(0)
+    x = rng.random((9, 2)).astype(np.float32)
+    y = rng.random((7, 2)).astype(np.float32)
+    a = rng.random(9) + 0.1
+    a /= a.sum()
+    b = rng.random(7) + 0.1
+    b /= b.sum()
+    g = rng.normal(0, 0.2, 7)
+    eps, c = 0.1, 1.3
+
+    def check(name, fn):
+        try:
+            if not fn():
+                failed.append(name)
+        except Exception:
+            failed.append(name)
+
+    def row_marginals():
+        f = orc.f_step(x, y, a, g, c, eps)
+        return np.allclose(orc.dense_plan(x, y, f, g, c, eps).sum(1), a, rtol=1e-12)
+
+    def col_marginals():
+        f = orc.f_step(x, y, a, g, c, eps)
+        g2 = orc.g_step(x, y, b, f, c, eps)
+        return np.allclose(orc.dense_plan(x, y, f, g2, c, eps).sum(0), b, rtol=1e-12)
+
+    def two_point():
+        x2 = np.array([[0.0], [1.0]], np.float32)
+        h = np.array([0.5, 0.5])
+        f, gg, _, _ = orc.sinkhorn(x2, x2, h, h, 1.0, 0.3, 5000, tol=1e-15)
+        p = 1.0 / (2.0 * (1.0 + math.exp(-1.0 / 0.3)))
+        return abs(orc.dense_plan(x2, x2, f, gg, 1.0, 0.3)[0, 0] - p) < 1e-9
+
+    def cross_ratio():
+        f = rng.normal(0, 0.2, 9)
+        T = orc.dense_plan(x, y, f, g, c, eps)
+        C = c * _sqd(x, y)
+        lhs = T[0, 0] * T[1, 1] / (T[0, 1] * T[1, 0])
+        return abs(lhs / math.exp((C[0, 1] + C[1, 0] - C[0, 0] - C[1, 1]) / eps) - 1) < 1e-10
+
+    def min_row_contract():
+        f, gg, _, _ = orc.sinkhorn(x, y, a, b, c, eps, 20)
+        T = orc.dense_plan(x, y, f, gg, c, eps)
+        o = orc.min_row(x, y, a, f, gg, c, eps)
+        return o["thr"] == T.max(1).min() and (o["counts"] >= 1).all()
+
+    def residual():
+        f, gg, _, _ = orc.sinkhorn(x, y, a, b, c, eps, 3)
+        T = orc.dense_plan(x, y, f, gg, c, eps)
+        r, q = orc.marginal_residual(x, y, a, b, f, gg, c, eps)
+        return abs(r - np.abs(T.sum(1) - a).sum()) < 1e-12 and abs(q - np.abs(T.sum(0) - b).sum()) < 1e-12
+
+    def mean_scale():
+        xd, yd = x.astype(np.float64), y.astype(np.float64)
+        mean = (xd ** 2).sum(1).mean() + (yd ** 2).sum(1).mean() - 2 * xd.mean(0) @ yd.mean(0)
+        return abs(1.0 / orc.inv_scale_cost(x, y, "mean") - mean) < 1e-12 * mean
+
+    for name, fn in [("row_marginals", row_marginals), ("col_marginals", col_marginals),
+                     ("two_point", two_point), ("cross_ratio", cross_ratio),
+                     ("min_row_contract", min_row_contract), ("residual", residual),
+                     ("mean_scale", mean_scale)]:
+        check(name, fn)
+    return failed
+
+
+def test_real_oracle_passes_the_battery(tmp_path):
+    assert _battery(_load_variant(tmp_path, "real")) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    failed = _battery(_load_variant(tmp_path, name, old, new))
+    assert failed, f"no pin caught the mutant {name}"
