@@ -57,6 +57,8 @@ def _args():
     ap.add_argument("--n", type=int, default=None, help="replica size of the workload (rows)")
     ap.add_argument("--m", type=int, default=None, help="replica size of the workload (columns)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-ms", type=int, default=200,
+                    help="nvidia-smi sampling period during the timed region")
     return ap.parse_args()
 
 
@@ -77,8 +79,8 @@ class Clocks:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index, self.proc, self.path = index, None, None
+    def __init__(self, index, period_ms=200):
+        self.index, self.proc, self.path, self.period = index, None, None, period_ms
 
     def start(self):
         import tempfile
@@ -86,7 +88,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", str(self.period)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
@@ -189,22 +191,27 @@ def _flush_l2(buf):
 
 
 def _cpu_baseline(w, target_s=10.0):
-    """The float64 oracle (as it stands) on a bounded row sample of the f-half-step."""
+    """The float64 oracle (as it stands) on a bounded sample of the f-half-step:
+    a row sample, repeated until about target_s seconds of CPU work."""
     import oracle
     oracle.build()
     c = 1.0  # the arithmetic per pair does not depend on the scale value
     g = np.zeros(w.m)
-    probe = min(w.n, 64)
+    probe = min(w.n, 256)
+    oracle.f_step(w.x, w.y, w.a, g, c, w.eps, rows=np.arange(probe))  # warm the thread pool
     t0 = time.perf_counter()
     oracle.f_step(w.x, w.y, w.a, g, c, w.eps, rows=np.arange(probe))
     rate = probe * w.m / max(time.perf_counter() - t0, 1e-6)
     rows = int(max(probe, min(w.n, rate * target_s / w.m)))
+    reps = max(1, int(round(target_s / max(rows * w.m / rate, 1e-6))))
     idx = np.linspace(0, w.n - 1, rows).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.f_step(w.x, w.y, w.a, g, c, w.eps, rows=idx)
+    for _ in range(reps):
+        oracle.f_step(w.x, w.y, w.a, g, c, w.eps, rows=idx)
     dt = time.perf_counter() - t0
-    return {"value": rows * w.m / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"one f-half-step on {rows} of {w.n} rows x all {w.m} columns "
+    return {"value": reps * rows * w.m / dt, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} f-half-step(s) on {rows} of {w.n} rows x all {w.m} columns "
                       f"(float64 C, OpenMP), {dt:.1f} s"}
 
 
@@ -258,7 +265,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # ---- device-resident timed region
-    clocks = Clocks(torch.cuda.current_device())
+    clocks = Clocks(torch.cuda.current_device(), args.clock_ms)
     _barrier(dist)
     clocks.start()
     total_ms, loop_ms, half_steps, launches, info = 0.0, 0.0, 0, 0, None

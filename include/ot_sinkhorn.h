@@ -227,7 +227,15 @@ OT_API int ot_marginal_residual_noalloc(const float *x, const float *y, const fl
                                         double inv_scale_cost, double *row_l1, double *col_l1,
                                         void *stream);
 
-/* Frees the plan's workspace (NULL is a no-op). Does not touch borrowed arrays. */
+/* Plans take their device workspace, pinned read-back buffer and internal
+ * stream from a per-device cache and return them there when destroyed, so
+ * repeated solves do not pay cudaMalloc/cudaFree (which synchronises the
+ * device) each time; the cache keeps at most 4 GiB of device memory per device.
+ * ot_trim_cache releases everything it holds (live plans are unaffected). */
+OT_API void ot_trim_cache(void);
+
+/* Returns the plan's workspace to the cache (NULL is a no-op). Does not touch
+ * borrowed arrays. Waits for the plan's internal stream. */
 OT_API void ot_plan_destroy(ot_plan *plan);
 
 #ifdef __cplusplus

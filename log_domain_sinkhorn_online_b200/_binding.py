@@ -29,7 +29,7 @@ OT_SCALE_NONE, OT_SCALE_MEAN, OT_SCALE_MAX_COST, OT_SCALE_VALUE = 0, 1, 2, 3
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sinkhorn_pointcloud",
             "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy",
-            "ot_marginal_residual_noalloc")
+            "ot_marginal_residual_noalloc", "ot_trim_cache")
 OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             L.ot_marginal_residual_noalloc.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D,
                                                        ctypes.POINTER(D), ctypes.POINTER(D), P]
             L.ot_marginal_residual_noalloc.restype = ctypes.c_int
+            L.ot_trim_cache.argtypes = []
+            L.ot_trim_cache.restype = None
             L.ot_plan_destroy.argtypes = [P]
             L.ot_plan_destroy.restype = None
             _lib = L
@@ -155,6 +157,10 @@ def ot_marginal_residual_noalloc(x, y, a, b, f, g, n, m, d, eps, inv_scale_cost,
     st = _check(lib().ot_marginal_residual_noalloc(x, y, a, b, f, g, n, m, d, eps, inv_scale_cost,
                                                    ctypes.byref(r), ctypes.byref(c), stream))
     return st, r.value, c.value
+
+
+def ot_trim_cache() -> None:
+    lib().ot_trim_cache()
 
 
 def ot_plan_destroy(plan) -> None:

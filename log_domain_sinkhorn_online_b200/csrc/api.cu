@@ -92,6 +92,7 @@ struct ot_plan {
     int64_t n_massless_rows = 0, n_massless_cols = 0;
     // workspace (one allocation, carved)
     char *ws = nullptr;
+    size_t ws_bytes = 0, ws_rows_bytes = 0;  // as obtained from the pool
     Params *prm = nullptr;
     State *st = nullptr;
     double *o = nullptr;
@@ -133,12 +134,14 @@ void plan_free(ot_plan *p) {
     for (auto &gx : p->graph)
         if (gx) cudaGraphExecDestroy(gx);
     for (auto ev : p->tev) cudaEventDestroy(ev);
-    if (p->ws) cudaFree(p->ws);
-    if (p->ws_rows) cudaFree(p->ws_rows);
-    if (p->hs) cudaFreeHost(p->hs);
+    // the workspaces and the stream go back to the pool once the plan's work is done
+    if (p->s_int) cudaStreamSynchronize(p->s_int);
+    pool_device_free(p->ws, p->ws_bytes);
+    pool_device_free(p->ws_rows, p->ws_rows_bytes);
+    pool_host_free(p->hs, sizeof(HostScalars));
     if (p->ev_in) cudaEventDestroy(p->ev_in);
     if (p->ev_out) cudaEventDestroy(p->ev_out);
-    if (p->s_int) cudaStreamDestroy(p->s_int);
+    pool_stream_release(p->s_int);
     delete p;
 }
 
@@ -500,7 +503,7 @@ int plan_setup(ot_plan *p, const ot_options &o) {
         p->tile_resid = cv.take<double>(tiles);
         p->bar = cv.take<unsigned>(2);
         p->blk_resid = cv.take<double>(std::max(p->loop_grid, 1));
-        if (pass == 0) OT_CU(cudaMalloc(&p->ws, cv.off));
+        if (pass == 0) OT_CU(pool_device_alloc(reinterpret_cast<void **>(&p->ws), cv.off, &p->ws_bytes));
     }
     if (p->kind == 2) {
         OT_CU(tc_setup(p->d));
@@ -629,10 +632,10 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     p->x = x; p->y = y; p->a = a; p->b = b; p->f = f; p->g = g;
     p->n = n; p->m = m; p->d = d;
     cudaStream_t us = (cudaStream_t)stream;
-    OT_CU(cudaStreamCreateWithFlags(&p->s_int, cudaStreamNonBlocking));
+    OT_CU(pool_stream(&p->s_int));
     OT_CU(cudaEventCreateWithFlags(&p->ev_in, cudaEventDisableTiming));
     OT_CU(cudaEventCreateWithFlags(&p->ev_out, cudaEventDisableTiming));
-    OT_CU(cudaMallocHost(&p->hs, sizeof(HostScalars)));
+    OT_CU(pool_host_alloc(reinterpret_cast<void **>(&p->hs), sizeof(HostScalars)));
     OT_CU(cudaEventRecord(p->ev_in, us));
     OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
     if ((rc = plan_setup(p, o)) != OT_OK) return rc;
@@ -761,7 +764,8 @@ int ensure_rows_ws(ot_plan *p) {
         p->rpart = cv.take<double>(rowpass_blocks(big));
         p->rowmax = cv.take<float>(p->n);
         p->counts = cv.take<int64_t>(p->n);
-        if (pass == 0) OT_CU(cudaMalloc(&p->ws_rows, cv.off));
+        if (pass == 0)
+            OT_CU(pool_device_alloc(reinterpret_cast<void **>(&p->ws_rows), cv.off, &p->ws_rows_bytes));
     }
     return OT_OK;
 }

@@ -9,6 +9,14 @@ namespace ot {
 // api.cu: sets the thread's last-error text and returns code
 int set_error(int code, const char *fmt, ...);
 
+// pool.cu: cached device workspaces, pinned host buffers and streams
+cudaError_t pool_device_alloc(void **ptr, size_t bytes, size_t *got);
+void pool_device_free(void *ptr, size_t bytes);
+cudaError_t pool_host_alloc(void **ptr, size_t bytes);
+void pool_host_free(void *ptr, size_t bytes);
+cudaError_t pool_stream(cudaStream_t *s);
+void pool_stream_release(cudaStream_t s);
+
 // halfstep.cu
 int halfstep_blocks_per_sm(int kind, int dim, int rpt);
 cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,

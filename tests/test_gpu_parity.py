@@ -265,3 +265,24 @@ def test_device_loop_long_run_crosses_chunks(ot, orc):
     f, g = _pots(plan)
     H.assert_potentials(f, f_ref, maxc, what="f")
     H.assert_potentials(g, g_ref, maxc, what="g")
+
+
+def test_resource_cache_reuse_and_trim(ot):
+    """Plans reuse cached workspaces (stale contents must not matter) and the
+    cache can be emptied; every solve gives the same bits."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    w = _cloud(55, 3000, 2500, 3, eps=0.02)
+    x, y, a, b = H.to_dev(w)
+    outs = []
+    for k in range(4):
+        if k == 2:
+            B.ot_trim_cache()
+        p = ot.sinkhorn(x, y, a, b, eps=w.eps, n_iters=30)
+        outs.append((p.f.clone(), p.g.clone()))
+        p.close()
+        # a different problem in between leaves other data in the cached buffers
+        q = ot.sinkhorn(y, x, b, a, eps=0.05, n_iters=3)
+        q.close()
+    for f, g in outs[1:]:
+        assert torch.equal(f, outs[0][0]) and torch.equal(g, outs[0][1])
