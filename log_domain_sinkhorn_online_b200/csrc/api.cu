@@ -159,13 +159,16 @@ struct Carver {
 };
 
 // Column splits for one half-step: rows -> tiles of `tile` rows; the column
-// table of `cols_pad` columns is cut into `splits` spans (multiples of
-// kColPad). Cost model in column-equivalents of one thread's work: every wave
-// of `cap` resident blocks costs rpt * (cps + 64 per-item overhead), and the
-// block that finishes a tile merges `splits` partials per row (~8 columns
-// each). Returns the estimate of the best split count, which it stores in sd.
+// table of `cols_pad` columns is cut into `splits` spans (multiples of `gran`).
+// Cost model in column-equivalents of one thread's work: resident blocks of one
+// SM share its ex2 pipe, so what counts is the most loaded SM, which runs
+// ceil(items / SMs) items of rpt * (cps + 64 per-item overhead) each (and no
+// fewer than `fill` items' worth: kernels that run several blocks per SM need
+// about 3 of them to keep the ex2 pipe busy); the block that
+// finishes a tile merges `splits` partials per row (~8 columns each). Returns
+// the estimate of the best split count, which it stores in sd.
 double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd,
-                     int force_s = 0, int gran = kColPad) {
+                     int force_s = 0, int gran = kColPad, int sms = 148, int fill = 3) {
     const int64_t tiles = (rows + tile - 1) / tile;
     double best = 1e300;
     int best_s = 1;
@@ -180,8 +183,10 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
             continue;
         }
         const int64_t items = tiles * s_eff;
+        const int64_t per_sm = std::max<int64_t>((items + sms - 1) / sms, fill);
         const int64_t waves = (items + cap - 1) / cap;
-        const double t = (double)waves * rpt * (double)(cps + 64) + 8.0 * rpt * (double)s_eff;
+        const double t = (double)std::max(per_sm, waves) * rpt * (double)(cps + 64) +
+                         8.0 * rpt * (double)s_eff;
         if (t < best * 0.995) {
             best = t;
             best_s = (int)s_eff;
@@ -202,13 +207,13 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
 int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Side &sd,
                  int force_s, int force_rpt) {
     if (kind == 2) {  // tensor cores: one 288-thread block per SM, 128-row tiles, 128-column chunks
-        choose_splits(rows, cols_pad, 1, 128, sms, sd, force_s, 128);
+        choose_splits(rows, cols_pad, 1, 128, sms, sd, force_s, 128, sms, 1);
         return OT_OK;
     }
     if (kind == 1) {
         const int bps = halfstep_blocks_per_sm(1, dim, kGnRows);
         if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
-        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd, force_s);
+        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd, force_s, kColPad, sms);
         return OT_OK;
     }
     double best = 1e300;
@@ -217,10 +222,11 @@ int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Sid
         const int bps = halfstep_blocks_per_sm(0, dim, rpt);
         if (bps <= 0) continue;
         Side tmp = sd;
-        // fewer rows per thread re-read the shared column data more often
-        const double eff = rpt == 2 ? 0.9 : 1.0;
+        // measured: 2 rows per thread run ~4% faster than 4 or 8 at n = 1e5..3e5
+        // (more resident warps hide the ex2 and shared-memory latency)
+        const double eff = rpt == 2 ? 1.04 : 1.0;
         const double t =
-            choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp, force_s) / eff;
+            choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp, force_s, kColPad, sms) / eff;
         if (t < best) {
             best = t;
             sd = tmp;
@@ -459,8 +465,10 @@ int plan_setup(ot_plan *p, const ot_options &o) {
             p->use_loop = true;
             p->loop_grid = bps * p->sm_count;
             // both half-steps run 2 rows per thread inside the loop kernel
-            choose_splits(p->n, p->sy.pad, 2, kHsThreads * 2, p->loop_grid, p->sx, o.col_splits);
-            choose_splits(p->m, p->sx.pad, 2, kHsThreads * 2, p->loop_grid, p->sy, o.col_splits);
+            choose_splits(p->n, p->sy.pad, 2, kHsThreads * 2, p->loop_grid, p->sx, o.col_splits,
+                          kColPad, p->sm_count);
+            choose_splits(p->m, p->sx.pad, 2, kHsThreads * 2, p->loop_grid, p->sy, o.col_splits,
+                          kColPad, p->sm_count);
             // no more blocks than there is work for: every block arrives at every barrier
             const int64_t work = std::max({(int64_t)p->sx.tiles * p->sx.splits,
                                            (int64_t)p->sy.tiles * p->sy.splits,
