@@ -158,15 +158,30 @@ struct Carver {
     }
 };
 
+// Time of the most loaded SM, in units of one item run at the SM's full ex2
+// rate. `items` equal items go to grid = min(items, cap) resident blocks, block
+// b taking items b, b + grid, ...; blocks land on SMs round-robin. The SM's
+// blocks share its ex2 pipe, which `fill` blocks keep busy: with k < fill
+// active blocks it runs at k / fill of its rate. So blocks that hold one item
+// more than the others finish in a slower tail.
+double sm_time(int64_t items, int64_t cap, int sms, int fill) {
+    const int64_t grid = std::min(items, cap);
+    const int64_t nb = (grid + sms - 1) / sms;         // blocks on the busiest SM
+    const int64_t hi = (items + grid - 1) / grid;      // most items of one block
+    const int64_t rem = items - (hi - 1) * grid;       // blocks holding hi items
+    const int64_t k_hi = std::min(nb, (rem + sms - 1) / sms);
+    double t = 0.0;
+    if (hi > 1) t += (double)(nb * (hi - 1)) * fill / (double)std::min<int64_t>(nb, fill);
+    t += (double)k_hi * fill / (double)std::min<int64_t>(k_hi, fill);
+    return t;
+}
+
 // Column splits for one half-step: rows -> tiles of `tile` rows; the column
 // table of `cols_pad` columns is cut into `splits` spans (multiples of `gran`).
-// Cost model in column-equivalents of one thread's work: resident blocks of one
-// SM share its ex2 pipe, so what counts is the most loaded SM, which runs
-// ceil(items / SMs) items of rpt * (cps + 64 per-item overhead) each (and no
-// fewer than `fill` items' worth: kernels that run several blocks per SM need
-// about 3 of them to keep the ex2 pipe busy); the block that
-// finishes a tile merges `splits` partials per row (~8 columns each). Returns
-// the estimate of the best split count, which it stores in sd.
+// Cost model in column-equivalents of one thread's work: the busiest SM's time
+// (sm_time) in items of rpt * (cps + 64 per-item overhead), plus the merge by
+// the block that finishes a tile of `splits` partials per row (~8 columns
+// each). Returns the estimate of the best split count, which it stores in sd.
 double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd,
                      int force_s = 0, int gran = kColPad, int sms = 148, int fill = 3) {
     const int64_t tiles = (rows + tile - 1) / tile;
@@ -183,9 +198,7 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
             continue;
         }
         const int64_t items = tiles * s_eff;
-        const int64_t per_sm = std::max<int64_t>((items + sms - 1) / sms, fill);
-        const int64_t waves = (items + cap - 1) / cap;
-        const double t = (double)std::max(per_sm, waves) * rpt * (double)(cps + 64) +
+        const double t = sm_time(items, cap, sms, fill) * rpt * (double)(cps + 64) +
                          8.0 * rpt * (double)s_eff;
         if (t < best * 0.995) {
             best = t;

@@ -117,11 +117,12 @@ __global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
                         t[u] = bf[(j + u) * ST + DP] + (s.x + s.y);
                     }
                     const float cm = fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3]));
-                    if (cm > m[k] + kLazyMax) {
-                        const float sc = ex2_approx(m[k] - cm);
+                    if (__any_sync(0xffffffffu, cm > m[k] + kLazyMax)) {
+                        const float mx = fmaxf(cm, m[k]);
+                        const float sc = ex2_approx(m[k] - mx);
                         acc[k] = __fmul2_rn(acc[k], make_float2(sc, sc));
                         tot[k] *= sc;
-                        m[k] = cm;
+                        m[k] = mx;
                     }
                     const float2 nm = make_float2(-m[k], -m[k]);
                     const float2 u0 = __fadd2_rn(make_float2(t[0], t[1]), nm);

@@ -363,13 +363,14 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                                  fmax3(va[8 * j + 3], va[8 * j + 4], va[8 * j + 5]),
                                  fmaxf(va[8 * j + 6], va[8 * j + 7]));
                 const float cm = fmax3(p[0], p[1], fmaxf(p[2], p[3]));
-                if (cm > m + kLazyMax) {
-                    const float sc = ex2_approx(m - cm);
+                if (__any_sync(0xffffffffu, cm > m + kLazyMax)) {
+                    const float mx = fmaxf(cm, m);
+                    const float sc = ex2_approx(m - mx);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) acc[u] = __fmul2_rn(acc[u], make_float2(sc, sc));
                     tot *= sc;
-                    m = cm;
-                    nm = make_float2(-cm, -cm);
+                    m = mx;
+                    nm = make_float2(-mx, -mx);
                 }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {

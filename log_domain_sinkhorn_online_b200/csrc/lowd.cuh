@@ -79,13 +79,14 @@ __device__ __forceinline__ void lowd_item(const HalfStep &A, int tile, int split
                 }
                 const float cm = fmax3(fmax3(t[0].x, t[0].y, t[1].x), fmax3(t[1].y, t[2].x, t[2].y),
                                        fmaxf(t[3].x, t[3].y));
-                if (cm > m[k] + kLazyMax) {  // rare: refresh the running maximum
-                    const float sc = ex2_approx(m[k] - cm);
+                if (__any_sync(0xffffffffu, cm > m[k] + kLazyMax)) {  // rare: refresh (warp vote)
+                    const float mx = fmaxf(cm, m[k]);
+                    const float sc = ex2_approx(m[k] - mx);
                     acc[k] = __fmul2_rn(acc[k], make_float2(sc, sc));
                     acc2[k] = __fmul2_rn(acc2[k], make_float2(sc, sc));
                     tot[k] *= sc;
-                    m[k] = cm;
-                    nm[k] = make_float2(-cm, -cm);
+                    m[k] = mx;
+                    nm[k] = make_float2(-mx, -mx);
                 }
                 const float2 u0 = __fadd2_rn(t[0], nm[k]), u1 = __fadd2_rn(t[1], nm[k]);
                 const float2 u2 = __fadd2_rn(t[2], nm[k]), u3 = __fadd2_rn(t[3], nm[k]);
