@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lo
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int tile = (int)(item / A.splits);
         const int split = (int)(item % A.splits);
-        lowd_item<D, R, false>(A, tile, split, sm);
+        lowd_item<D, R, false, true>(A, tile, split, sm);
         finish_tile<kHsThreads, kHsThreads * R, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
     }
@@ -160,8 +160,15 @@ static const void *lowd_fn(int dim) {
 
 // kind 0: low-d (dim = d in 1..3, rpt = rows per thread 2/4/8);
 // kind 1: generic (dim = DP in {8,16,32,64}, rpt ignored).
+// The kernel for a launch shape; nullptr for a shape that has no instantiation
+// (the tile size, hence the partials' layout, depends on rpt).
 static const void *halfstep_fn(int kind, int dim, int rpt) {
-    if (kind == 0) return rpt == 8 ? lowd_fn<8>(dim) : rpt == 4 ? lowd_fn<4>(dim) : lowd_fn<2>(dim);
+    if (kind == 0) {
+        if (rpt == 8) return lowd_fn<8>(dim);
+        if (rpt == 4) return lowd_fn<4>(dim);
+        if (rpt == 2) return lowd_fn<2>(dim);
+        return nullptr;
+    }
     if (dim == 8) return (const void *)hs_generic_kernel<8>;
     if (dim == 16) return (const void *)hs_generic_kernel<16>;
     if (dim == 32) return (const void *)hs_generic_kernel<32>;
@@ -171,7 +178,9 @@ static const void *halfstep_fn(int kind, int dim, int rpt) {
 int halfstep_blocks_per_sm(int kind, int dim, int rpt) {
     int nb = 0;
     const int threads = kind == 0 ? kHsThreads : kGnThreads;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, halfstep_fn(kind, dim, rpt), threads, 0) !=
+    const void *fn = halfstep_fn(kind, dim, rpt);
+    if (!fn) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, 0) !=
         cudaSuccess)
         return 0;
     return nb;
@@ -180,8 +189,10 @@ int halfstep_blocks_per_sm(int kind, int dim, int rpt) {
 cudaError_t launch_halfstep(int kind, int dim, int rpt, const HalfStep &A, int grid,
                             cudaStream_t s) {
     const int threads = kind == 0 ? kHsThreads : kGnThreads;
+    const void *fn = halfstep_fn(kind, dim, rpt);
+    if (!fn) return cudaErrorInvalidValue;
     void *args[] = {(void *)&A};
-    return cudaLaunchKernel(halfstep_fn(kind, dim, rpt), dim3(grid), dim3(threads), args, 0, s);
+    return cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, 0, s);
 }
 
 }  // namespace ot

@@ -129,11 +129,13 @@ __device__ double grid_residual(const double *blk, double *s_red) {
 
 }  // namespace
 
-// Rows per thread in the loop kernel (both half-steps): small problems.
+// Rows per thread in the loop kernel (both half-steps): small problems. At most
+// 4 blocks per SM: the problems it runs have a few hundred work items, and the
+// registers left free let the exponentials run ahead of the refresh vote.
 constexpr int kLoopR = 2;
 
 template <int D>
-__global__ void __launch_bounds__(kHsThreads, 6) hs_loop_kernel(LoopArgs L) {
+__global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
     __shared__ __align__(16) float4 sm[2][kHsChunk];
     __shared__ double s_red[kHsThreads / 32];
     __shared__ int s_ok;
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kHsThreads, 6) hs_loop_kernel(LoopArgs L) {
         const int64_t nf = (int64_t)F.tiles * F.splits;
         for (int64_t item = blockIdx.x; item < nf; item += gridDim.x) {
             __syncthreads();
-            lowd_item<D, kLoopR, true>(F, (int)(item / F.splits), (int)(item % F.splits), sm);
+            lowd_item<D, kLoopR, true, true>(F, (int)(item / F.splits), (int)(item % F.splits), sm);
         }
         if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         const double br = merge_phase<kHsThreads>(F, s_red, &bad);
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(kHsThreads, 6) hs_loop_kernel(LoopArgs L) {
         const int64_t ng = (int64_t)G.tiles * G.splits;
         for (int64_t item = blockIdx.x; item < ng; item += gridDim.x) {
             __syncthreads();
-            lowd_item<D, kLoopR, true>(G, (int)(item / G.splits), (int)(item % G.splits), sm);
+            lowd_item<D, kLoopR, true, true>(G, (int)(item / G.splits), (int)(item % G.splits), sm);
         }
         if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         merge_phase<kHsThreads>(G, s_red, &bad);
