@@ -7,7 +7,9 @@ residual at the returned potentials, the exact min_row threshold and per-row
 counts in row blocks of 1024, and the materialisation of every row in blocks of
 1024. Inputs are resident in HBM before the timed region; L2 is flushed before
 every step. The metric counts Sinkhorn pair-updates (n*m per half-step) per
-second; the row passes are inside the timed step but add no units.
+second; the row passes are inside the timed step but add no units. After the
+timed steps, the line's `large_n` object reports the d = 3 per-launch half-step
+at n = m = 1e5 against the same MUFU roofline (skip with --no-large-n).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload w2]
 
@@ -34,9 +36,8 @@ UNIT = "pair-updates/s"
 # MUFU ex2 peak: 148 SMs x 16 ex2 per clock per SM x 1.965 GHz (max SM clock)
 SMS, EX2_PER_CLK = 148, 16
 # DRAM bytes per half-step of the dominant kernel, from the committed ncu captures
-# (profiles/hs_loop_w2_8000.md: 874.5 KB per 512-half-step launch), keyed by
-# workload; None where no capture of the current kernel exists
-HALFSTEP_TRAFFIC = {"w2_gmm3d_8000": 874.5e3 / 512}
+# of the current kernel, keyed by workload; None where no such capture exists
+HALFSTEP_TRAFFIC = {"w2_gmm3d_8000": 870.1e3 / 512}  # profiles/hs_loop_w2_8000.md
 
 
 def _peaks():
@@ -57,6 +58,8 @@ def _args():
     ap.add_argument("--n", type=int, default=None, help="replica size of the workload (rows)")
     ap.add_argument("--m", type=int, default=None, help="replica size of the workload (columns)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-large-n", action="store_true",
+                    help="skip the d = 3 half-step measurement at n = m = 1e5")
     ap.add_argument("--clock-ms", type=int, default=200,
                     help="nvidia-smi sampling period during the timed region")
     return ap.parse_args()
@@ -251,6 +254,24 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _large_n(ot, dev, n=100_000, iters=5):
+    """The d = 3 per-launch half-step at n = m = 1e5 (spiral clouds, eps 1e-3,
+    max_cost scale): microseconds per half-step from CUDA events on the
+    library's stream, as a fraction of the MUFU ex2 rate."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w5(n=n)
+    x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
+    ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=1, device_loop=0).close()
+    p = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=iters, device_loop=0, timing=True)
+    info = p.info
+    p.close()
+    us = info.loop_ms * 1e3 / max(info.half_steps, 1)
+    return {"workload": f"spirals3d_{n} replica (n = m = {n}, d = 3, eps 1e-3, scale max_cost)",
+            "kernel": "hs_lowd_kernel (fused f/g half-step)", "half_steps": info.half_steps,
+            "per_launch_us": us, "achieved": float(n) * n / (us / 1e6) / 1e12, "unit": "Tex2/s"}
+
+
 def run_ours(args):
     import torch
     import log_domain_sinkhorn_online_b200 as ot
@@ -312,6 +333,7 @@ def run_ours(args):
         e2e_units += float(w.n) * float(w.m) * inf.half_steps
     e2e_ms = _max_over_ranks(e2e_ms, dist)
     e2e_value = e2e_units * world / (e2e_ms / 1e3)
+    large = _large_n(ot, dev) if w.d <= 3 and not args.no_large_n else None
 
     if rank == 0:
         peaks, kind = _peaks()
@@ -338,6 +360,10 @@ def run_ours(args):
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches}
+        if large is not None:
+            large["peak"] = peak_tex2
+            large["frac"] = large["achieved"] / peak_tex2
+            line["large_n"] = large
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = _cpu_baseline(w)
         print(json.dumps(line), flush=True)
