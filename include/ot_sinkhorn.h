@@ -143,7 +143,8 @@ OT_API void ot_options_default(ot_options *opt);
  *  x [n,d], y [m,d], a [n], b [m]: device, float32. Weights must be finite and
  *      >= 0 with positive sums; they are not renormalised. 1 <= d <= 64.
  *  eps > 0: entropic regularisation on the scaled cost (the final eps when
- *      annealing).
+ *      annealing). Held in float64 throughout, so the plan is the one of
+ *      exactly this eps.
  *  scale_cost: see ot_scale.
  *  n_iters >= 0: iteration cap (one iteration = f-update then g-update; the
  *      f-update comes first, from f = g = 0 unless opt->warm_start).
@@ -159,8 +160,8 @@ OT_API void ot_options_default(ot_options *opt);
  * Returns OT_OK, OT_WARN_MASSLESS_ROWS, or an error (then *plan_out = NULL and
  * f, g are unspecified). Synchronises `stream` (it reads scalars back). */
 OT_API int ot_sinkhorn_pointcloud(const float *x, const float *y, const float *a, const float *b,
-                           int64_t n, int64_t m, int32_t d, float eps, ot_scale scale_cost,
-                           int32_t n_iters, float tol, float *f, float *g, void *stream,
+                           int64_t n, int64_t m, int32_t d, double eps, ot_scale scale_cost,
+                           int32_t n_iters, double tol, float *f, float *g, void *stream,
                            const ot_options *opt, ot_plan **plan_out, ot_info *info);
 
 /* ---------------------------------------------------- ot_marginal_residual

@@ -73,8 +73,8 @@ def lib() -> ctypes.CDLL:
             L.ot_last_error_string.restype = ctypes.c_char_p
             L.ot_options_default.argtypes = [ctypes.POINTER(OtOptions)]
             L.ot_options_default.restype = None
-            L.ot_sinkhorn_pointcloud.argtypes = [P, P, P, P, I64, I64, I32, ctypes.c_float, ctypes.c_int,
-                                                 I32, ctypes.c_float, P, P, P,
+            L.ot_sinkhorn_pointcloud.argtypes = [P, P, P, P, I64, I64, I32, ctypes.c_double, ctypes.c_int,
+                                                 I32, ctypes.c_double, P, P, P,
                                                  ctypes.POINTER(OtOptions), ctypes.POINTER(P),
                                                  ctypes.POINTER(OtInfo)]
             L.ot_sinkhorn_pointcloud.restype = ctypes.c_int

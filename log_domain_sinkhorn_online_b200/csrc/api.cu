@@ -597,7 +597,7 @@ int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
 }
 
 int validate(const float *x, const float *y, const float *a, const float *b, int64_t n,
-             int64_t m, int32_t d, float eps, ot_scale scale, int32_t n_iters, float *f,
+             int64_t m, int32_t d, double eps, ot_scale scale, int32_t n_iters, float *f,
              float *g, const ot_options &o) {
     if (!x || !y || !a || !b || !f || !g) return fail(OT_ERR_INVALID_ARG, "null array pointer");
     if (n < 1 || m < 1) return fail(OT_ERR_INVALID_ARG, "n and m must be >= 1 (n=%lld m=%lld)",
@@ -607,7 +607,7 @@ int validate(const float *x, const float *y, const float *a, const float *b, int
                     (long long)m);
     if (d < 1 || d > kMaxD) return fail(d < 1 ? OT_ERR_INVALID_ARG : OT_ERR_UNSUPPORTED,
                                         "d=%d outside 1..%d", d, kMaxD);
-    if (!(eps > 0.0f) || !std::isfinite(eps)) return fail(OT_ERR_INVALID_ARG, "eps must be > 0 and finite");
+    if (!(eps > 0.0) || !std::isfinite(eps)) return fail(OT_ERR_INVALID_ARG, "eps must be > 0 and finite");
     if (scale < OT_SCALE_NONE || scale > OT_SCALE_VALUE) return fail(OT_ERR_INVALID_ARG, "bad scale_cost");
     if (scale == OT_SCALE_VALUE && !(o.scale_value > 0.0 && std::isfinite(o.scale_value)))
         return fail(OT_ERR_INVALID_ARG, "scale_value must be > 0 and finite");
@@ -629,8 +629,8 @@ int validate(const float *x, const float *y, const float *a, const float *b, int
 }  // namespace
 
 extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const float *a,
-                                      const float *b, int64_t n, int64_t m, int32_t d, float eps,
-                                      ot_scale scale_cost, int32_t n_iters, float tol, float *f,
+                                      const float *b, int64_t n, int64_t m, int32_t d, double eps,
+                                      ot_scale scale_cost, int32_t n_iters, double tol, float *f,
                                       float *g, void *stream, const ot_options *opt,
                                       ot_plan **plan_out, ot_info *info) {
     if (plan_out) *plan_out = nullptr;
@@ -673,12 +673,12 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     std::vector<double> stage_eps;
     if (o.eps_init > 0.0) {
         for (int k = 0;; ++k) {
-            const double ek = std::max((double)eps, o.eps_init * std::pow(o.eps_decay, (double)k));
+            const double ek = std::max(eps, o.eps_init * std::pow(o.eps_decay, (double)k));
             stage_eps.push_back(ek);
-            if (ek == (double)eps || k > 100000) break;
+            if (ek == eps || k > 100000) break;
         }
     } else {
-        stage_eps.push_back((double)eps);
+        stage_eps.push_back(eps);
     }
     float *fb[2] = {p->f, p->fspare};
     const int layout = p->kind == 0 ? 0 : 1;  // CUDA-core paths' column-table layout
@@ -687,7 +687,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     double resid = NAN;
     for (size_t si = 0; si < stage_eps.size(); ++si) {
         const bool last = si + 1 == stage_eps.size();
-        const double tol_s = (last && tol > 0.0f) ? (double)tol : 0.0;
+        const double tol_s = (last && tol > 0.0) ? tol : 0.0;
         const int iters = last ? n_iters : o.iters_per_stage;
         OT_CU(launch_set_params(p->prm, stage_eps[si], p->c, tol_s, p->s_int));
         OT_CU(launch_reset_state(p->st, p->s_int));

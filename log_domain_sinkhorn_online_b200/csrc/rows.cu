@@ -83,12 +83,15 @@ __device__ __forceinline__ void load_row(const float *pts, const float *pot, int
 // ------------------------------------------------------------ materializer
 // Block: 256 threads x 4 consecutive columns (1024 columns). A block keeps its
 // columns' float64 data in registers (d <= 3) and walks a range of up to 256
-// rows of the row list, staged 32 at a time through shared memory, four rows
-// in flight; each row is one coalesced float4 evict-first store per thread.
+// rows of the row list, staged 32 at a time through shared memory; each row is
+// one coalesced float4 evict-first store per thread. The kernel is bound by
+// the latency of each entry's float64 chain, so occupancy matters more than
+// rows in flight: 4 blocks per SM with 2 rows unrolled (measured at 4096 x 1e5,
+// d = 3: 2.63 TB/s written, against 2.29 at 3 blocks per SM, 4 rows).
 constexpr int kMtThreads = 256, kMtStage = 32, kMtRowsPerBlock = 256;
 
 template <int D>
-__global__ void __launch_bounds__(kMtThreads) materialize_kernel(MatArgs M) {
+__global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
     __shared__ double sA[kMtStage], sP[kMtStage][D > 0 ? D : kMaxD];
     __shared__ int sValid[kMtStage];
     const int tid = threadIdx.x;
@@ -125,9 +128,9 @@ __global__ void __launch_bounds__(kMtThreads) materialize_kernel(MatArgs M) {
         __syncthreads();
         if (ncol == 0) continue;
         const int nr = (int)min((int64_t)kMtStage, rb1 - s0);
-#pragma unroll 4
+#pragma unroll 2
         for (int rr = 0; rr < nr; ++rr) {
-            if (!sValid[rr]) continue;
+            const bool valid = sValid[rr] != 0;
             float t[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -138,6 +141,7 @@ __global__ void __launch_bounds__(kMtThreads) materialize_kernel(MatArgs M) {
                                     : 0.0f;
             }
             float *dst = M.out + (s0 + rr) * M.m + j0;
+            if (!valid) continue;
             if (M.vec && ncol == 4) {
                 __stcs(reinterpret_cast<float4 *>(dst), make_float4(t[0], t[1], t[2], t[3]));
             } else {
