@@ -37,19 +37,35 @@ namespace ot {
 // Rows: thread t of a tile owns rows t + 128 k, k < R (R = 2, 4 or 8; the tile
 // is 128 R rows: fewer rows per thread give more tiles, hence fewer column
 // splits to merge, on small problems).
+//
+// Work items are handed out dynamically: block b starts with item b, and each
+// item's first thread claims the next one (grid + a per-side atomic counter)
+// while the item runs. Blocks are not placed on SMs round-robin, so a static
+// stride left whole SMs idle at the end of a launch (ncu: SMs active 85 % of
+// the elapsed cycles at n = m = 1e5). The counter of one side is reset by
+// every launch of the other side before anything else (f- and g-launches
+// alternate, so its previous user has finished and its next user has not
+// started); reset_state clears both at the start of a stage.
 template <int D, int R>
 __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lowd_kernel(HalfStep A) {
     __shared__ __align__(16) float4 sm[2][kHsChunk];
     __shared__ double s_red[kHsThreads / 32];
     __shared__ int s_flag;
+    __shared__ long long s_next[2];
+    if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;
     if (ld_volatile(&A.st->stop)) return;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
-    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int64_t item = blockIdx.x;
+    for (int it = 0; item < n_items; ++it) {
+        // two slots: a slow thread still reading the previous claim is never overwritten
+        if (threadIdx.x == 0)
+            s_next[it & 1] = (long long)gridDim.x + (long long)atomicAdd(&A.st->work[A.side], 1u);
         const int tile = (int)(item / A.splits);
         const int split = (int)(item % A.splits);
         lowd_item<D, R, false, true>(A, tile, split, sm);
         finish_tile<kHsThreads, kHsThreads * R, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
+        item = s_next[it & 1];
     }
 }
 

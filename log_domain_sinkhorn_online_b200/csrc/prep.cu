@@ -134,6 +134,7 @@ __global__ void reset_state_kernel(State *st) {
     st->conv_iter = -1;
     st->resid[0] = st->resid[1] = -1.0;
     st->tiles_done[0] = st->tiles_done[1] = 0;
+    st->work[0] = st->work[1] = 0;
 }
 
 // ----------------------------------------------------------------- tables
