@@ -178,12 +178,22 @@ double sm_time(int64_t items, int64_t cap, int sms, int fill) {
 
 // Column splits for one half-step: rows -> tiles of `tile` rows; the column
 // table of `cols_pad` columns is cut into `splits` spans (multiples of `gran`).
-// Cost model in column-equivalents of one thread's work: the busiest SM's time
-// (sm_time) in items of rpt * (cps + 64 per-item overhead), plus the merge by
-// the block that finishes a tile of `splits` partials per row (~8 columns
-// each). Returns the estimate of the best split count, which it stores in sd.
+// Cost model in column-equivalents of one thread's work, an item being
+// rpt * (cps + 64 per-item overhead):
+//  - static assignment (loop and tensor-core kernels): the busiest SM's time
+//    (sm_time);
+//  - dynamic assignment (per-launch CUDA-core kernels, which claim items from a
+//    counter) with more items than resident blocks: the SMs stay balanced, so
+//    the work per SM (no less than `fill` items: fewer do not keep the ex2 pipe
+//    busy) plus a tail of about one item (fitted to measurements at n = m =
+//    1e5 and 3e5, d = 3); with one wave of items or less, sm_time again
+//    (measured at n = m = 8000: 13 splits 35.3 us, 20 splits 38.9 us);
+// plus the merge by the block that finishes a tile of `splits` partials per
+// row (~8 columns each). Returns the estimate of the best split count, which
+// it stores in sd.
 double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap, Side &sd,
-                     int force_s = 0, int gran = kColPad, int sms = 148, int fill = 3) {
+                     int force_s = 0, int gran = kColPad, int sms = 148, int fill = 3,
+                     bool dynamic = false) {
     const int64_t tiles = (rows + tile - 1) / tile;
     double best = 1e300;
     int best_s = 1;
@@ -198,8 +208,11 @@ double choose_splits(int64_t rows, int64_t cols_pad, int rpt, int tile, int cap,
             continue;
         }
         const int64_t items = tiles * s_eff;
-        const double t = sm_time(items, cap, sms, fill) * rpt * (double)(cps + 64) +
-                         8.0 * rpt * (double)s_eff;
+        const double item = (double)rpt * (double)(cps + 64);
+        const double per_sm = (dynamic && items > cap)
+                                  ? std::max((double)items / sms, (double)fill) + 1.2
+                                  : sm_time(items, cap, sms, fill);
+        const double t = per_sm * item + 8.0 * rpt * (double)s_eff;
         if (t < best * 0.995) {
             best = t;
             best_s = (int)s_eff;
@@ -226,7 +239,7 @@ int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Sid
     if (kind == 1) {
         const int bps = halfstep_blocks_per_sm(1, dim, kGnRows);
         if (bps <= 0) return fail(OT_ERR_CUDA, "half-step kernel cannot be made resident");
-        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd, force_s, kColPad, sms);
+        choose_splits(rows, cols_pad, kGnRows, kGnTile, bps * sms, sd, force_s, kColPad, sms, 3, true);
         return OT_OK;
     }
     double best = 1e300;
@@ -239,7 +252,8 @@ int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Sid
         // (more resident warps hide the ex2 and shared-memory latency)
         const double eff = rpt == 2 ? 1.04 : 1.0;
         const double t =
-            choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp, force_s, kColPad, sms) / eff;
+            choose_splits(rows, cols_pad, rpt, kHsThreads * rpt, bps * sms, tmp, force_s, kColPad, sms, 3,
+                          true) / eff;
         if (t < best) {
             best = t;
             sd = tmp;

@@ -56,7 +56,7 @@ struct State {
     int wait_timeout;   // a bounded wait in a tensor-core kernel gave up (error)
     double resid[2];    // last in-loop marginal residual of each side (0: rows, 1: cols)
     unsigned tiles_done[2];
-    unsigned work[2];   // work-item counters of the per-launch d <= 3 half-step (f, g side)
+    unsigned work[2];   // work-item counters of the per-launch CUDA-core half-steps (f, g side)
 };
 
 // Arguments of one half-step launch (the same kernel serves f and g: rows are

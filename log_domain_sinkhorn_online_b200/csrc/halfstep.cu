@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lo
 // floats, [Y_0 .. Y_{DP-1}, G, 0, 0, 0] (Y = 2 c kappa y', zero past d). Row
 // table: [rows][DP] floats x' (zero past d). Thread t owns rows t and t + 128
 // of the tile; the dot products run as packed f32x2 FMAs over coordinate pairs.
+// Work items are handed out dynamically, as in hs_lowd_kernel.
 template <int DP>
 __global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
     constexpr int ST = DP + 4;
@@ -81,11 +82,16 @@ __global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
     __shared__ __align__(16) float4 sm[2][CH4];
     __shared__ double s_red[kGnThreads / 32];
     __shared__ int s_flag;
+    __shared__ long long s_next[2];
+    if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;  // as in hs_lowd_kernel
     if (ld_volatile(&A.st->stop)) return;
     const int tid = threadIdx.x;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
 
-    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int64_t item = blockIdx.x;
+    for (int it = 0; item < n_items; ++it) {
+        if (tid == 0)
+            s_next[it & 1] = (long long)gridDim.x + (long long)atomicAdd(&A.st->work[A.side], 1u);
         const int tile = (int)(item / A.splits);
         const int split = (int)(item % A.splits);
 
@@ -163,6 +169,7 @@ __global__ void __launch_bounds__(kGnThreads, 2) hs_generic_kernel(HalfStep A) {
         }
         finish_tile<kGnThreads, kGnTile, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
+        item = s_next[it & 1];
     }
 }
 
