@@ -91,7 +91,9 @@ typedef struct ot_options {
                                  internal stream (ot_info.loop_ms); default 0 */
     int32_t col_splits;       /* tuning: column splits of the half-steps (0 = chosen
                                  from the problem size and the SM count) */
-    int32_t rows_per_thread;  /* tuning, d <= 3: 2, 4 or 8 rows per thread (0 = auto) */
+    int32_t rows_per_thread;  /* tuning, d <= 3: 1, 2, 4 or 8 rows per thread (0 =
+                                 auto); the device-resident loop runs 1 or 2 and
+                                 is not used when 4 or 8 is asked for */
     int32_t tensor_cores;     /* 16 <= d <= 64: 1 (default) computes x.y on the tcgen05
                                  tensor cores (bf16 splits, fp32 accumulation); 0 uses
                                  the CUDA-core FMA kernel */

@@ -112,6 +112,7 @@ struct ot_plan {
     int kp = 0;                 // tensor-core path: bf16 K extent of the operand tables
     bool use_loop = false;      // device-resident iterations (loop.cu)
     int loop_grid = 0;
+    int loop_rpt = 2;           // rows per thread of the loop kernel (1 or 2)
     unsigned *bar = nullptr;    // grid barrier: count, generation
     double *blk_resid = nullptr;
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
@@ -243,8 +244,8 @@ int choose_shape(int kind, int dim, int sms, int64_t rows, int64_t cols_pad, Sid
         return OT_OK;
     }
     double best = 1e300;
-    for (int rpt : {8, 4, 2}) {
-        if (force_rpt > 0 && rpt != force_rpt) continue;
+    for (int rpt : {8, 4, 2, 1}) {  // 1 only when asked for
+        if (force_rpt > 0 ? rpt != force_rpt : rpt == 1) continue;
         const int bps = halfstep_blocks_per_sm(0, dim, rpt);
         if (bps <= 0) continue;
         Side tmp = sd;
@@ -367,7 +368,7 @@ int run_loop(ot_plan *p, int parity0, int iters, bool check) {
         L.parity0 = (parity0 + i) & 1;
         OT_CU(cudaMemsetAsync(p->bar, 0, sizeof(unsigned), p->s_int));  // arrivals
         OT_CU(mark(p));
-        OT_CU(launch_loop(p->d, L, p->loop_grid, p->s_int));
+        OT_CU(launch_loop(p->d, p->loop_rpt, L, p->loop_grid, p->s_int));
         OT_CU(mark(p));
         p->launches += 1;
         i += len;
@@ -487,15 +488,29 @@ int plan_setup(ot_plan *p, const ot_options &o) {
     p->sy.pad = round_up(p->m, padq);
     if (p->kind == 0 && o.device_loop != 0 &&
         (o.device_loop == 1 || (double)p->n * (double)p->m <= (double)(1ll << 28))) {
-        const int bps = loop_blocks_per_sm(p->d);
-        if (bps > 0) {
-            p->use_loop = true;
-            p->loop_grid = bps * p->sm_count;
-            // both half-steps run 2 rows per thread inside the loop kernel
-            choose_splits(p->n, p->sy.pad, 2, kHsThreads * 2, p->loop_grid, p->sx, o.col_splits,
-                          kColPad, p->sm_count);
-            choose_splits(p->m, p->sx.pad, 2, kHsThreads * 2, p->loop_grid, p->sy, o.col_splits,
-                          kColPad, p->sm_count);
+        // rows per thread (1 or 2, both half-steps) with the smaller estimate;
+        // measured: 1 row runs ~6 % slower per pair, but balances better on some sizes
+        double best = 1e300;
+        for (int rpt : {2, 1}) {
+            if (o.rows_per_thread > 0 && rpt != o.rows_per_thread) continue;
+            const int bps = loop_blocks_per_sm(p->d, rpt);
+            if (bps <= 0) continue;
+            Side sx = p->sx, sy = p->sy;
+            const double t = (choose_splits(p->n, p->sy.pad, rpt, kHsThreads * rpt, bps * p->sm_count, sx,
+                                            o.col_splits, kColPad, p->sm_count) +
+                              choose_splits(p->m, p->sx.pad, rpt, kHsThreads * rpt, bps * p->sm_count, sy,
+                                            o.col_splits, kColPad, p->sm_count)) /
+                             (rpt == 1 ? 0.94 : 1.0);
+            if (t < best) {
+                best = t;
+                p->use_loop = true;
+                p->loop_rpt = rpt;
+                p->loop_grid = bps * p->sm_count;
+                p->sx = sx;
+                p->sy = sy;
+            }
+        }
+        if (p->use_loop) {
             // no more blocks than there is work for: every block arrives at every barrier
             const int64_t work = std::max({(int64_t)p->sx.tiles * p->sx.splits,
                                            (int64_t)p->sy.tiles * p->sy.splits,
@@ -630,9 +645,9 @@ int validate(const float *x, const float *y, const float *a, const float *b, int
         return fail(OT_ERR_INVALID_ARG, "n_iters == 0 needs warm_start (a plan at given f, g)");
     if (o.check_every < 1) return fail(OT_ERR_INVALID_ARG, "check_every must be >= 1");
     if (o.col_splits < 0) return fail(OT_ERR_INVALID_ARG, "col_splits must be >= 0");
-    if (o.rows_per_thread != 0 && o.rows_per_thread != 2 && o.rows_per_thread != 4 &&
-        o.rows_per_thread != 8)
-        return fail(OT_ERR_INVALID_ARG, "rows_per_thread must be 0, 2, 4 or 8");
+    if (o.rows_per_thread != 0 && o.rows_per_thread != 1 && o.rows_per_thread != 2 &&
+        o.rows_per_thread != 4 && o.rows_per_thread != 8)
+        return fail(OT_ERR_INVALID_ARG, "rows_per_thread must be 0, 1, 2, 4 or 8");
     if (o.eps_init > 0.0) {
         if (!(o.eps_decay > 0.0 && o.eps_decay < 1.0)) return fail(OT_ERR_INVALID_ARG, "eps_decay must be in (0,1)");
         if (o.iters_per_stage < 1) return fail(OT_ERR_INVALID_ARG, "iters_per_stage must be >= 1");

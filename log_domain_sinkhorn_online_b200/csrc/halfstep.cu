@@ -34,9 +34,10 @@ namespace ot {
 // with Y = 2 c kappa y' (zero past d) and G as above; padding columns have
 // Y = 0, G = -inf and add nothing. So column c's data starts at float4 c (c
 // even) and a chunk of 256 columns is 256 float4 (4 KB of shared memory).
-// Rows: thread t of a tile owns rows t + 128 k, k < R (R = 2, 4 or 8; the tile
-// is 128 R rows: fewer rows per thread give more tiles, hence fewer column
-// splits to merge, on small problems).
+// Rows: thread t of a tile owns rows t + 128 k, k < R (R = 1, 2, 4 or 8; the
+// tile is 128 R rows: fewer rows per thread give more tiles, hence fewer column
+// splits to merge, on small problems; R = 1 serves the f-update that follows a
+// 1-row device-resident loop, or a caller who asks for it).
 //
 // Work items are handed out dynamically: block b starts with item b, and each
 // item's first thread claims the next one (grid + a per-side atomic counter)
@@ -47,7 +48,7 @@ namespace ot {
 // alternate, so its previous user has finished and its next user has not
 // started); reset_state clears both at the start of a stage.
 template <int D, int R>
-__global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : 6) hs_lowd_kernel(HalfStep A) {
+__global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : R == 2 ? 6 : 8) hs_lowd_kernel(HalfStep A) {
     __shared__ __align__(16) float4 sm[2][kHsChunk];
     __shared__ double s_red[kHsThreads / 32];
     __shared__ int s_flag;
@@ -181,7 +182,7 @@ static const void *lowd_fn(int dim) {
     return (const void *)hs_lowd_kernel<3, R>;
 }
 
-// kind 0: low-d (dim = d in 1..3, rpt = rows per thread 2/4/8);
+// kind 0: low-d (dim = d in 1..3, rpt = rows per thread 1/2/4/8);
 // kind 1: generic (dim = DP in {8,16,32,64}, rpt ignored).
 // The kernel for a launch shape; nullptr for a shape that has no instantiation
 // (the tile size, hence the partials' layout, depends on rpt).
@@ -190,6 +191,7 @@ static const void *halfstep_fn(int kind, int dim, int rpt) {
         if (rpt == 8) return lowd_fn<8>(dim);
         if (rpt == 4) return lowd_fn<4>(dim);
         if (rpt == 2) return lowd_fn<2>(dim);
+        if (rpt == 1) return lowd_fn<1>(dim);
         return nullptr;
     }
     if (dim == 8) return (const void *)hs_generic_kernel<8>;

@@ -129,12 +129,12 @@ __device__ double grid_residual(const double *blk, double *s_red) {
 
 }  // namespace
 
-// Rows per thread in the loop kernel (both half-steps): small problems. At most
-// 4 blocks per SM: the problems it runs have a few hundred work items, and the
-// registers left free let the exponentials run ahead of the refresh vote.
-constexpr int kLoopR = 2;
-
-template <int D>
+// The loop kernel runs R = 1 or 2 rows per thread in both half-steps (the cost
+// model picks: 128-row tiles balance better across 148 SMs on some sizes, e.g.
+// 63 x 7 = 441 items at n = 8000, 2-row tiles on others). At most 4 blocks per
+// SM: the problems it runs have a few hundred work items, and the registers
+// left free let the exponentials run ahead of the refresh vote.
+template <int D, int R>
 __global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
     __shared__ __align__(16) float4 sm[2][kHsChunk];
     __shared__ double s_red[kHsThreads / 32];
@@ -152,15 +152,15 @@ __global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
         const int64_t nf = (int64_t)F.tiles * F.splits;
         for (int64_t item = blockIdx.x; item < nf; item += gridDim.x) {
             __syncthreads();
-            lowd_item<D, kLoopR, true, true>(F, (int)(item / F.splits), (int)(item % F.splits), sm);
+            lowd_item<D, R, true, true>(F, (int)(item / F.splits), (int)(item % F.splits), sm);
         }
         if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         const double br = merge_phase<kHsThreads>(F, s_red, &bad);
         if (threadIdx.x == 0) L.blk_resid[blockIdx.x] = br;
         if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
-        const double R = grid_residual<kHsThreads>(L.blk_resid, s_red);
-        if (blockIdx.x == 0 && threadIdx.x == 0) st->resid[0] = R;
-        if (tol > 0.0 && iter_done >= 1 && R <= tol) {  // the same decision in every block
+        const double resid = grid_residual<kHsThreads>(L.blk_resid, s_red);
+        if (blockIdx.x == 0 && threadIdx.x == 0) st->resid[0] = resid;
+        if (tol > 0.0 && iter_done >= 1 && resid <= tol) {  // the same decision in every block
             if (blockIdx.x == 0 && threadIdx.x == 0) {
                 st->stop = 1;
                 st->conv_iter = iter_done;
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
         const int64_t ng = (int64_t)G.tiles * G.splits;
         for (int64_t item = blockIdx.x; item < ng; item += gridDim.x) {
             __syncthreads();
-            lowd_item<D, kLoopR, true, true>(G, (int)(item / G.splits), (int)(item % G.splits), sm);
+            lowd_item<D, R, true, true>(G, (int)(item / G.splits), (int)(item % G.splits), sm);
         }
         if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
         merge_phase<kHsThreads>(G, s_red, &bad);
@@ -184,22 +184,32 @@ __global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
     if (bad) atomicExch(&st->nonfinite, 1);
 }
 
-static const void *loop_fn(int d) {
-    if (d == 1) return (const void *)hs_loop_kernel<1>;
-    if (d == 2) return (const void *)hs_loop_kernel<2>;
-    return (const void *)hs_loop_kernel<3>;
+template <int R>
+static const void *loop_fn_r(int d) {
+    if (d == 1) return (const void *)hs_loop_kernel<1, R>;
+    if (d == 2) return (const void *)hs_loop_kernel<2, R>;
+    return (const void *)hs_loop_kernel<3, R>;
 }
 
-int loop_blocks_per_sm(int d) {
+static const void *loop_fn(int d, int rpt) {
+    if (rpt == 1) return loop_fn_r<1>(d);
+    if (rpt == 2) return loop_fn_r<2>(d);
+    return nullptr;
+}
+
+int loop_blocks_per_sm(int d, int rpt) {
+    const void *fn = loop_fn(d, rpt);
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, loop_fn(d), kHsThreads, 0) != cudaSuccess)
+    if (!fn || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kHsThreads, 0) != cudaSuccess)
         return 0;
     return nb;
 }
 
-cudaError_t launch_loop(int d, const LoopArgs &L, int grid, cudaStream_t s) {
+cudaError_t launch_loop(int d, int rpt, const LoopArgs &L, int grid, cudaStream_t s) {
+    const void *fn = loop_fn(d, rpt);
+    if (!fn) return cudaErrorInvalidValue;
     void *args[] = {(void *)&L};
-    return cudaLaunchCooperativeKernel(loop_fn(d), dim3(grid), dim3(kHsThreads), args, 0, s);
+    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kHsThreads), args, 0, s);
 }
 
 }  // namespace ot

@@ -32,8 +32,8 @@ struct LoopArgs {
     unsigned *bar_gen;      // grid barrier: generation
     double *blk_resid;      // [grid] residual partial of each block
 };
-int loop_blocks_per_sm(int d);
-cudaError_t launch_loop(int d, const LoopArgs &L, int grid, cudaStream_t s);
+int loop_blocks_per_sm(int d, int rpt);
+cudaError_t launch_loop(int d, int rpt, const LoopArgs &L, int grid, cudaStream_t s);
 
 // halfstep_tc.cu (16 <= d <= 64: tensor-core path)
 int tc_ksteps(int d);

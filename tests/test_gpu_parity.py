@@ -256,6 +256,20 @@ def test_device_loop_and_launch_paths(ot, orc, loop, d):
     H.assert_potentials(g, g_ref, maxc, what="g")
 
 
+@pytest.mark.parametrize("loop,rpt", [(1, 1), (1, 2), (0, 1), (0, 2), (0, 4), (0, 8)])
+def test_rows_per_thread_shapes(ot, orc, loop, rpt):
+    """Every row layout of the d <= 3 kernels (tiles of 128 rpt rows) in both the
+    device-resident loop and the per-launch path, on a ragged problem (neither
+    side a multiple of a tile), against the oracle's trajectory."""
+    w = _cloud(17, 1313, 1207, 3, scale="mean", eps=0.02)
+    plan, c, f_ref, g_ref, _, _ = _solve_both(ot, orc, w, 40, device_loop=loop, rows_per_thread=rpt)
+    assert plan.info.kernel_launches < 40 if loop else plan.info.kernel_launches >= 80
+    maxc = H.max_cost(w.x, w.y, c)
+    f, g = _pots(plan)
+    H.assert_potentials(f, f_ref, maxc, what="f")
+    H.assert_potentials(g, g_ref, maxc, what="g")
+
+
 def test_device_loop_long_run_crosses_chunks(ot, orc):
     """600 iterations: three cooperative launches of the loop kernel."""
     w = _cloud(91, 900, 1100, 2, eps=0.03)
