@@ -65,6 +65,8 @@ def _load():
             lib.orc_dense_plan.argtypes = [P, P, P, P, I64, I64, I32, D, D, P]
             lib.orc_min_row.argtypes = [P, P, P, P, P, I64, I64, I32, D, D, I64, P, P, P, P]
             lib.orc_min_row.restype = I64
+            lib.orc_sparsify_csr.argtypes = [P, P, P, P, P, I64, I64, I32, D, D, D, P, P, P, I64]
+            lib.orc_sparsify_csr.restype = I64
             _lib = lib
     return _lib
 
@@ -212,6 +214,26 @@ def dense_plan(x, y, f, g, c, eps):
     T = np.empty((n, m))
     _load().orc_dense_plan(_ptr(x), _ptr(y), _ptr(f), _ptr(g), n, m, d, c, eps, _ptr(T))
     return T
+
+
+def sparsify_csr(x, y, a, f, g, c, eps, thr):
+    """The thresholded plan (T_ij >= thr, massful rows) in compressed-row form
+    (moscot PR #846, "Behavioural changes"). Returns (row_ptr, col_idx, vals)."""
+    x, y, n, m, d = _pts(x, y)
+    a, f, g = _f64(a), _f64(f), _f64(g)
+    row_ptr = np.zeros(n + 1, dtype=np.int64)
+    L = _load()
+    # first call with no room only sizes the result
+    nnz = L.orc_sparsify_csr(_ptr(x), _ptr(y), _ptr(a), _ptr(f), _ptr(g), n, m, d, c, eps, float(thr),
+                             _ptr(row_ptr), None, None, ctypes.c_int64(-1))
+    assert nnz == -1
+    total = int(row_ptr[n])
+    col_idx = np.empty(max(total, 1), dtype=np.int64)
+    vals = np.empty(max(total, 1), dtype=np.float64)
+    nnz = L.orc_sparsify_csr(_ptr(x), _ptr(y), _ptr(a), _ptr(f), _ptr(g), n, m, d, c, eps, float(thr),
+                             _ptr(row_ptr), _ptr(col_idx), _ptr(vals), ctypes.c_int64(total))
+    assert nnz == total
+    return row_ptr, col_idx[:total], vals[:total]
 
 
 def min_row(x, y, a, f, g, c, eps, block_rows=0):

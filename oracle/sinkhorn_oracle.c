@@ -342,3 +342,41 @@ int64_t orc_min_row(const float *x, const float *y, const double *a, const doubl
     if (nnz_out) *nnz_out = nnz;
     return massless;
 }
+
+/* ------------------------------------------------------------- sparsify --
+ * The sparse plan that thresholding produces (moscot PR #846, "Behavioural
+ * changes": entries with T_ij >= thr are kept, rows without mass keep nothing),
+ * in compressed-row form: row_ptr [n+1], and for row i the kept columns in
+ * increasing order in col_idx[row_ptr[i] .. row_ptr[i+1]) with their values in
+ * vals. A first pass counts every row, a second writes them. Returns nnz, or
+ * -1 (writing no entry) when nnz exceeds cap.                               */
+int64_t orc_sparsify_csr(const float *x, const float *y, const double *a, const double *f,
+                         const double *g, int64_t n, int64_t m, int d, double c, double eps,
+                         double thr, int64_t *row_ptr, int64_t *col_idx, double *vals,
+                         int64_t cap) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t cnt = 0;
+        if (a[i] != 0.0)
+            for (int64_t j = 0; j < m; ++j)
+                if (plan_entry(x, y, f, g, i, j, d, c, eps) >= thr) ++cnt;
+        row_ptr[i + 1] = cnt;
+    }
+    row_ptr[0] = 0;
+    for (int64_t i = 0; i < n; ++i) row_ptr[i + 1] += row_ptr[i];
+    if (row_ptr[n] > cap) return -1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        if (a[i] == 0.0) continue;
+        int64_t k = row_ptr[i];
+        for (int64_t j = 0; j < m; ++j) {
+            const double t = plan_entry(x, y, f, g, i, j, d, c, eps);
+            if (t >= thr) {
+                col_idx[k] = j;
+                vals[k] = t;
+                ++k;
+            }
+        }
+    }
+    return row_ptr[n];
+}

@@ -25,6 +25,8 @@ MUTANTS = {
     "mean_scale_wrong_count": ("if (mode == 1) r /= ((double)n * (double)m);", "if (mode == 1) r /= ((double)n * (double)n);"),
     "lse_no_shift_back": ("return mx + log(s);", "return log(s);"),
     "g_step_uses_a_weight": ("out = eps * log(b[j]) - eps * lse(v, n);", "out = eps * log(b[0]) - eps * lse(v, n);"),
+    "csr_strict_threshold": ("            if (t >= thr) {\n                col_idx[k] = j;", "            if (t > thr) {\n                col_idx[k] = j;"),
+    "csr_drops_the_column_order": ("                col_idx[k] = j;", "                col_idx[k] = m - 1 - j;"),
 }
 
 
@@ -104,6 +106,16 @@ def _battery(orc):
         r, q = orc.marginal_residual(x, y, a, b, f, gg, c, eps)
         return abs(r - np.abs(T.sum(1) - a).sum()) < 1e-12 and abs(q - np.abs(T.sum(0) - b).sum()) < 1e-12
 
+    def csr():
+        f, gg, _, _ = orc.sinkhorn(x, y, a, b, c, eps, 20)
+        T = orc.dense_plan(x, y, f, gg, c, eps)
+        thr = T.max(1).min()
+        row_ptr, col_idx, vals = orc.sparsify_csr(x, y, a, f, gg, c, eps, thr)
+        dense = np.zeros_like(T)
+        for i in range(len(a)):
+            dense[i, col_idx[row_ptr[i]:row_ptr[i + 1]]] = vals[row_ptr[i]:row_ptr[i + 1]]
+        return np.array_equal(dense != 0, T >= thr) and np.array_equal(dense[T >= thr], T[T >= thr])
+
     def mean_scale():
         xd, yd = x.astype(np.float64), y.astype(np.float64)
         mean = (xd ** 2).sum(1).mean() + (yd ** 2).sum(1).mean() - 2 * xd.mean(0) @ yd.mean(0)
@@ -111,7 +123,7 @@ def _battery(orc):
 
     for name, fn in [("row_marginals", row_marginals), ("col_marginals", col_marginals),
                      ("two_point", two_point), ("cross_ratio", cross_ratio),
-                     ("min_row_contract", min_row_contract), ("residual", residual),
+                     ("min_row_contract", min_row_contract), ("residual", residual), ("csr", csr),
                      ("mean_scale", mean_scale)]:
         check(name, fn)
     return failed

@@ -269,6 +269,50 @@ def test_min_row_contract(orc):
         assert T[o["argmin"]].max() == want and a[o["argmin"]] > 0
 
 
+@pytest.mark.parametrize("eps", [0.3, 0.1])
+def test_sparsify_two_point_keeps_the_diagonal(orc, eps):
+    # x = y = {0, 1}, uniform weights: the converged plan is [[p, q], [q, p]] with
+    # p = 1/(2(1+e^{-1/eps})) > q, so thr = p and thresholding keeps exactly the
+    # diagonal (moscot PR #846, "Behavioural changes").
+    x = np.array([[0.0], [1.0]], np.float32)
+    a = np.array([0.5, 0.5])
+    f, g, _, _ = orc.sinkhorn(x, x, a, a, 1.0, eps, 5000, tol=1e-15)
+    mr = orc.min_row(x, x, a, f, g, 1.0, eps)
+    p = 1.0 / (2.0 * (1.0 + math.exp(-1.0 / eps)))
+    assert mr["thr"] == pytest.approx(p, rel=1e-10)
+    row_ptr, col_idx, vals = orc.sparsify_csr(x, x, a, f, g, 1.0, eps, mr["thr"])
+    assert row_ptr.tolist() == [0, 1, 2] and col_idx.tolist() == [0, 1]
+    np.testing.assert_allclose(vals, [p, p], rtol=1e-10)
+
+
+def test_sparsify_csr_is_the_thresholded_plan(orc):
+    # The CSR lists, row by row in increasing column order, exactly the entries of
+    # the dense plan with T_ij >= thr in rows with mass; every massful row keeps
+    # at least its maximum; the per-row counts are min_row's.
+    x, y = _cloud(21, 40, 33, 3)
+    a = np.full(40, 1 / 37)
+    a[[0, 11, 39]] = 0.0
+    b = np.full(33, 1 / 33)
+    f, g, _, _ = orc.sinkhorn(x, y, a, b, 1.0, 0.02, 30)
+    T = orc.dense_plan(x, y, f, g, 1.0, 0.02)
+    mr = orc.min_row(x, y, a, f, g, 1.0, 0.02)
+    row_ptr, col_idx, vals = orc.sparsify_csr(x, y, a, f, g, 1.0, 0.02, mr["thr"])
+    assert row_ptr[0] == 0 and np.all(np.diff(row_ptr) >= 0) and row_ptr[-1] == len(col_idx) == mr["nnz"]
+    np.testing.assert_array_equal(np.diff(row_ptr), mr["counts"])
+    dense = np.zeros_like(T)
+    for i in range(40):
+        cols = col_idx[row_ptr[i]:row_ptr[i + 1]]
+        assert np.all(np.diff(cols) > 0)
+        dense[i, cols] = vals[row_ptr[i]:row_ptr[i + 1]]
+        if a[i] == 0.0:
+            assert len(cols) == 0
+        else:
+            assert int(np.argmax(T[i])) in cols.tolist()
+    mask = (T >= mr["thr"]) & (a[:, None] > 0)
+    np.testing.assert_array_equal(dense != 0, mask)
+    np.testing.assert_array_equal(dense[mask], T[mask])
+
+
 def test_min_row_all_massless(orc):
     x, y = _cloud(16, 5, 4, 2)
     o = orc.min_row(x, y, np.zeros(5), np.full(5, -np.inf), np.zeros(4), 1.0, 0.1)
