@@ -202,6 +202,29 @@ OT_API int ot_sparsify_min_row(const ot_plan *plan, int64_t block_rows, float *t
                         int64_t *row_counts, int64_t *nnz_out, int64_t *n_massless_out,
                         int64_t *argmin_out, void *stream);
 
+/* ---------------------------------------------------------- ot_sparsify_csr
+ * The plan thresholded at thr (moscot PR #846, "Behavioural changes": the
+ * entries T_ij >= thr are kept, rows with a_i == 0 keep nothing), written in
+ * compressed-row form for an [n, m] matrix: row i's kept columns, increasing,
+ * in col_idx[row_ptr[i] .. row_ptr[i+1]) and their values in vals. Values and
+ * comparisons come from the same float path as ot_materialize_rows and
+ * ot_sparsify_min_row: with thr = its thr_out, row_ptr differences are its
+ * row_counts and the total its nnz_out (use that to size col_idx / vals).
+ * The pages describe the threshold and the kept set; the compressed-row layout
+ * is this library's (the common sparse format; no page fixes one).
+ *  block_rows: rows per pass (> 0, or 0 = all); never changes a result.
+ *  row_ptr [n+1] int64, col_idx [capacity] int64, vals [capacity] float32:
+ *      device, caller-owned outputs.
+ *  nnz_out: host int64 or NULL: the number of kept entries (set also when it
+ *      exceeds capacity).
+ * Returns OT_ERR_OVERFLOW, with row_ptr written and col_idx / vals untouched,
+ * when the kept entries exceed capacity; OT_ERR_CUDA if the count and write
+ * passes ever disagreed (not expected: both call one entry function).
+ * Synchronises `stream`. */
+OT_API int ot_sparsify_csr(const ot_plan *plan, int64_t block_rows, float thr, int64_t *row_ptr,
+                           int64_t *col_idx, float *vals, int64_t capacity, int64_t *nnz_out,
+                           void *stream);
+
 /* ------------------------------------------- ot_marginal_residual_noalloc
  * The pages have no counterpart to this entry point: it exists for callers
  * that cannot allocate device memory when they need a residual -- a process

@@ -84,6 +84,31 @@ class Plan:
                                                       _stream(stream))
         return dict(thr=thr, counts=counts, nnz=nnz, n_massless=nm, argmin=arg, status=st)
 
+    def sparsify_csr(self, thr=None, block_rows=0, capacity=None, stream=None):
+        """The plan thresholded at thr (default: the min_row threshold) in
+        compressed-row form. Returns dict(row_ptr [n+1] int64, col_idx [nnz]
+        int64, vals [nnz] float32, nnz, thr); torch.sparse_csr_tensor(row_ptr,
+        col_idx, vals, (n, m)) turns it into a torch sparse matrix."""
+        import torch
+        dev = self.f.device
+        n = self.f.numel()
+        if thr is None:
+            mr = self.sparsify_min_row(block_rows=block_rows, stream=stream)
+            thr = mr["thr"]
+            if capacity is None:
+                capacity = mr["nnz"]
+        row_ptr = torch.empty(n + 1, dtype=torch.int64, device=dev)
+        if capacity is None:  # size it first: a call with no room only counts
+            _, capacity = B.ot_sparsify_csr(self._h, int(block_rows), float(thr), row_ptr.data_ptr(),
+                                            0, 0, 0, _stream(stream))
+        col_idx = torch.empty(max(int(capacity), 1), dtype=torch.int64, device=dev)
+        vals = torch.empty(max(int(capacity), 1), dtype=torch.float32, device=dev)
+        st, nnz = B.ot_sparsify_csr(self._h, int(block_rows), float(thr), row_ptr.data_ptr(),
+                                    col_idx.data_ptr(), vals.data_ptr(), int(capacity), _stream(stream))
+        if st == B.OT_ERR_OVERFLOW:
+            raise B.OTError(st, B.ot_last_error_string())
+        return dict(row_ptr=row_ptr, col_idx=col_idx[:nnz], vals=vals[:nnz], nnz=nnz, thr=thr)
+
 
 def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None, warm_start=False,
              check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,

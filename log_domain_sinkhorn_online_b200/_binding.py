@@ -29,7 +29,7 @@ OT_SCALE_NONE, OT_SCALE_MEAN, OT_SCALE_MAX_COST, OT_SCALE_VALUE = 0, 1, 2, 3
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sinkhorn_pointcloud",
             "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy",
-            "ot_marginal_residual_noalloc", "ot_trim_cache")
+            "ot_marginal_residual_noalloc", "ot_trim_cache", "ot_sparsify_csr")
 OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
                                               ctypes.POINTER(I64), ctypes.POINTER(I64),
                                               ctypes.POINTER(I64), P]
             L.ot_sparsify_min_row.restype = ctypes.c_int
+            L.ot_sparsify_csr.argtypes = [P, I64, ctypes.c_float, P, P, P, I64, ctypes.POINTER(I64), P]
+            L.ot_sparsify_csr.restype = ctypes.c_int
             L.ot_marginal_residual_noalloc.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D,
                                                        ctypes.POINTER(D), ctypes.POINTER(D), P]
             L.ot_marginal_residual_noalloc.restype = ctypes.c_int
@@ -139,6 +141,16 @@ def ot_marginal_residual(plan, stream):
 
 def ot_materialize_rows(plan, row_idx, k, out, stream) -> int:
     return _check(lib().ot_materialize_rows(plan, row_idx, k, out, stream))
+
+
+def ot_sparsify_csr(plan, block_rows, thr, row_ptr, col_idx, vals, capacity, stream):
+    """Returns (status, nnz); row_ptr / col_idx / vals: device pointers."""
+    nnz = ctypes.c_int64()
+    st = lib().ot_sparsify_csr(plan, block_rows, thr, row_ptr, col_idx or None, vals or None,
+                               capacity, ctypes.byref(nnz), stream)
+    if st != OT_ERR_OVERFLOW:
+        _check(st)
+    return st, nnz.value
 
 
 def ot_sparsify_min_row(plan, block_rows, row_counts, stream):

@@ -108,6 +108,7 @@ struct ot_plan {
     double *dcol = nullptr, *rpart = nullptr;
     float *rowmax = nullptr;
     int64_t *counts = nullptr;
+    int64_t *scan = nullptr;    // tile totals of the row_ptr scan
     HostScalars *hs = nullptr;  // pinned
     int kp = 0;                 // tensor-core path: bf16 K extent of the operand tables
     bool use_loop = false;      // device-resident iterations (loop.cu)
@@ -814,6 +815,7 @@ int ensure_rows_ws(ot_plan *p) {
         p->rpart = cv.take<double>(rowpass_blocks(big));
         p->rowmax = cv.take<float>(p->n);
         p->counts = cv.take<int64_t>(p->n);
+        p->scan = cv.take<int64_t>(scan_tmp_count(p->n));
         if (pass == 0)
             OT_CU(pool_device_alloc(reinterpret_cast<void **>(&p->ws_rows), cv.off, &p->ws_rows_bytes));
     }
@@ -896,6 +898,56 @@ extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, flo
         fail(OT_WARN_MASSLESS_ROWS, "%lld rows carry no mass", (long long)nm);
         return OT_WARN_MASSLESS_ROWS;
     }
+    return OT_OK;
+}
+
+extern "C" int ot_sparsify_csr(const ot_plan *cplan, int64_t block_rows, float thr, int64_t *row_ptr,
+                               int64_t *col_idx, float *vals, int64_t capacity, int64_t *nnz_out,
+                               void *stream) {
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if (block_rows < 0) return fail(OT_ERR_INVALID_ARG, "block_rows must be >= 0");
+    if (!row_ptr) return fail(OT_ERR_INVALID_ARG, "row_ptr must not be NULL");
+    if (capacity < 0) return fail(OT_ERR_INVALID_ARG, "capacity must be >= 0");
+    if (capacity > 0 && (!col_idx || !vals))
+        return fail(OT_ERR_INVALID_ARG, "col_idx and vals must not be NULL when capacity > 0");
+    if (std::isnan(thr)) return fail(OT_ERR_INVALID_ARG, "thr must not be NaN");
+    if (block_rows == 0 || block_rows > p->n) block_rows = p->n;
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    // pass 1: kept entries per row (the count pass of ot_sparsify_min_row)
+    RowPassArgs R{};
+    R.pts = p->x; R.pot = p->f; R.w = p->a; R.dcol = p->dcol; R.o = p->o; R.prm = p->prm;
+    R.cols = p->m; R.d = p->d; R.thr = thr; R.counts = p->counts;
+    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
+        R.row_begin = r0;
+        R.row_end = std::min(p->n, r0 + block_rows);
+        OT_CU(launch_rowpass(1, R, s));
+    }
+    // row pointers, and nnz = row_ptr[n]
+    OT_CU(launch_row_ptr_scan(p->counts, p->n, row_ptr, p->scan, s));
+    OT_CU(cudaMemcpyAsync(&p->ds->nnz, row_ptr + p->n, sizeof(int64_t), cudaMemcpyDeviceToDevice, s));
+    OT_CU(cudaMemsetAsync(&p->ds->bad, 0, sizeof(int), s));
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    const int64_t nnz = p->hs->s.nnz;
+    if (nnz_out) *nnz_out = nnz;
+    if (nnz > capacity)
+        return fail(OT_ERR_OVERFLOW, "%lld entries are kept, capacity is %lld", (long long)nnz,
+                    (long long)capacity);
+    // pass 2: the entries, in row order and increasing columns
+    CsrArgs C{};
+    C.pts = p->x; C.pot = p->f; C.w = p->a; C.dcol = p->dcol; C.o = p->o; C.prm = p->prm;
+    C.cols = p->m; C.d = p->d; C.thr = thr; C.row_ptr = row_ptr; C.col_idx = col_idx; C.vals = vals;
+    C.bad = &p->ds->bad;
+    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
+        C.row_begin = r0;
+        C.row_end = std::min(p->n, r0 + block_rows);
+        OT_CU(launch_csr_write(C, s));
+    }
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    if (p->hs->s.bad) return fail(OT_ERR_CUDA, "the count and write passes kept different entries");
     return OT_OK;
 }
 

@@ -243,6 +243,157 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
     }
 }
 
+// ----------------------------------------------------------- sparse plan
+// The kept entries (T_ij >= thr, rows with mass) of kRpRows rows per block in
+// compressed-row form. Thread t visits columns t, t + 256, ... in order; per
+// 256-column chunk and row, a warp ballot and the warps' counts in shared
+// memory give every kept entry its position, so each row's entries land in
+// increasing column order from row_ptr[i]. The entries come from the same
+// plan_entry() as the count pass that produced row_ptr; a row never writes
+// past its own segment, and a row whose kept entries do not fill it exactly
+// sets *bad (it cannot happen unless the two passes disagree).
+template <int D>
+__global__ void __launch_bounds__(kRpThreads) csr_write_kernel(CsrArgs C) {
+    constexpr int WARPS = kRpThreads / 32;
+    __shared__ double sA[kRpRows], sP[kRpRows][D > 0 ? D : kMaxD];
+    __shared__ int sCnt[kRpRows][WARPS];
+    __shared__ long long sPos[kRpRows], sEnd[kRpRows];
+    __shared__ int sLive[kRpRows];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t r0 = C.row_begin + (int64_t)blockIdx.x * kRpRows;
+    const int d = D > 0 ? D : C.d;
+    if (tid < kRpRows) {
+        const int64_t i = r0 + tid;
+        const int live = i < C.row_end && C.w[i] > 0.0f;
+        if (live) {
+            load_row(C.pts, C.pot, i, d, C.o, C.prm->kappa, C.prm->c, &sA[tid], sP[tid]);
+            sPos[tid] = C.row_ptr[i];
+            sEnd[tid] = C.row_ptr[i + 1];
+        } else {
+            sA[tid] = -INFINITY;
+            sPos[tid] = sEnd[tid] = 0;
+        }
+        sLive[tid] = live;
+    }
+    __syncthreads();
+    const unsigned below = (1u << lane) - 1u;
+    constexpr int DS = (D > 0 ? D : 1) + 1;
+    for (int64_t j0 = 0; j0 < C.cols; j0 += kRpThreads) {
+        const int64_t j = j0 + tid;
+        const bool colok = j < C.cols;
+        double cd[DS];
+        const double *col = C.dcol + (colok ? j : 0) * (d + 1);
+        if (D > 0) {
+#pragma unroll
+            for (int q = 0; q < DS; ++q) cd[q] = col[q];
+        }
+        float t[kRpRows];
+        unsigned bal[kRpRows];
+#pragma unroll
+        for (int r = 0; r < kRpRows; ++r) {
+            t[r] = D > 0 ? plan_entry<D>(sA[r], sP[r], cd, d) : plan_entry<0>(sA[r], sP[r], col, d);
+            const bool keep = colok && sLive[r] && t[r] >= C.thr;
+            bal[r] = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0) sCnt[r][warp] = __popc(bal[r]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < kRpRows; ++r) {
+            if (!((bal[r] >> lane) & 1u)) continue;
+            long long off = sPos[r] + __popc(bal[r] & below);
+            for (int w = 0; w < warp; ++w) off += sCnt[r][w];
+            if (off < sEnd[r]) {
+                C.col_idx[off] = j;
+                C.vals[off] = t[r];
+            } else {
+                atomicExch(C.bad, 1);
+            }
+        }
+        __syncthreads();
+        if (tid < kRpRows) {
+            int tot = 0;
+            for (int w = 0; w < WARPS; ++w) tot += sCnt[tid][w];
+            sPos[tid] += tot;
+        }
+        __syncthreads();
+    }
+    if (tid < kRpRows && sLive[tid] && sPos[tid] != sEnd[tid]) atomicExch(C.bad, 1);
+}
+
+// Exclusive scan of the row counts into row_ptr, in three launches: tiles of
+// kScanTile counts scanned in place (inclusive, at row_ptr[1..]) with the tile
+// totals on the side, the totals scanned by one block, the tile offsets added.
+constexpr int kScanThreads = 1024, kScanPer = 4, kScanTile = kScanThreads * kScanPer;
+
+__device__ long long block_incl_scan(long long v, long long *s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    if (lane == 31) s_warp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        long long w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long u = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += u;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const long long r = v + (warp > 0 ? s_warp[warp - 1] : 0);
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_tiles_kernel(const int64_t *counts, int64_t n,
+                                                                   int64_t *row_ptr, int64_t *sums) {
+    __shared__ long long s_warp[32];
+    const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanPer;
+    long long v[kScanPer], run = 0;
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) {
+        v[k] = base + k < n ? counts[base + k] : 0;
+        run += v[k];
+    }
+    const long long excl = block_incl_scan(run, s_warp) - run;
+    long long acc = excl;
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) {
+        acc += v[k];
+        if (base + k < n) row_ptr[base + k + 1] = acc;
+    }
+    if (threadIdx.x == blockDim.x - 1) sums[blockIdx.x] = acc;
+    if (blockIdx.x == 0 && threadIdx.x == 0) row_ptr[0] = 0;
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_sums_kernel(int64_t *sums, int64_t nb) {
+    __shared__ long long s_warp[32];
+    __shared__ long long s_tot;
+    long long carry = 0;
+    for (int64_t b0 = 0; b0 < nb; b0 += kScanThreads) {
+        const int64_t b = b0 + threadIdx.x;
+        const long long v = b < nb ? sums[b] : 0;
+        const long long incl = block_incl_scan(v, s_warp);
+        if (b < nb) sums[b] = carry + incl - v;  // exclusive: the offset of tile b
+        if (threadIdx.x == kScanThreads - 1) s_tot = incl;
+        __syncthreads();
+        carry += s_tot;
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_add_kernel(int64_t n, int64_t *row_ptr,
+                                                                 const int64_t *sums) {
+    if (blockIdx.x == 0) return;  // tile 0 has offset 0
+    const long long off = sums[blockIdx.x];
+    const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanPer;
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k)
+        if (base + k < n) row_ptr[base + k + 1] += off;
+}
+
 // ------------------------------------------------------------ reductions
 // min over massful rows of rowmax (smallest index on ties), number of massless
 // rows and (after the count pass) nnz. One block; fixed order per thread, then
@@ -371,6 +522,30 @@ cudaError_t launch_min_row_reduce(const float *rowmax, const float *w, int64_t n
 
 cudaError_t launch_sum_i64(const int64_t *v, int64_t cnt, int64_t *out, cudaStream_t s) {
     sum_kernel<int64_t><<<1, kRedThreads, 0, s>>>(v, cnt, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_csr_write(const CsrArgs &C, cudaStream_t s) {
+    const int64_t rows = C.row_end - C.row_begin;
+    if (rows <= 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + kRpRows - 1) / kRpRows);
+    switch (C.d) {
+        case 1: csr_write_kernel<1><<<grid, kRpThreads, 0, s>>>(C); break;
+        case 2: csr_write_kernel<2><<<grid, kRpThreads, 0, s>>>(C); break;
+        case 3: csr_write_kernel<3><<<grid, kRpThreads, 0, s>>>(C); break;
+        default: csr_write_kernel<0><<<grid, kRpThreads, 0, s>>>(C); break;
+    }
+    return cudaGetLastError();
+}
+
+int64_t scan_tmp_count(int64_t n) { return (n + kScanTile - 1) / kScanTile + 1; }
+
+cudaError_t launch_row_ptr_scan(const int64_t *counts, int64_t n, int64_t *row_ptr, int64_t *tmp,
+                                cudaStream_t s) {
+    const int64_t nb = std::max<int64_t>((n + kScanTile - 1) / kScanTile, 1);
+    scan_tiles_kernel<<<(unsigned)nb, kScanThreads, 0, s>>>(counts, n, row_ptr, tmp);
+    scan_sums_kernel<<<1, kScanThreads, 0, s>>>(tmp, nb);
+    scan_add_kernel<<<(unsigned)nb, kScanThreads, 0, s>>>(n, row_ptr, tmp);
     return cudaGetLastError();
 }
 

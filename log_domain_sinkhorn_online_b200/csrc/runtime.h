@@ -80,6 +80,24 @@ struct RowPassArgs {
     int64_t *counts;
     double *part;
 };
+struct CsrArgs {
+    const float *pts, *pot, *w;
+    const double *dcol, *o;
+    const Params *prm;
+    int64_t row_begin, row_end, cols;
+    int d;
+    float thr;
+    const int64_t *row_ptr;   // [n+1], exclusive prefix sum of the kept counts
+    int64_t *col_idx;
+    float *vals;
+    int *bad;                 // set if a row keeps a different number of entries
+};
+cudaError_t launch_csr_write(const CsrArgs &C, cudaStream_t s);
+// row_ptr[0] = 0, row_ptr[i+1] = counts[0] + ... + counts[i]; tmp holds
+// scan_tmp_count(n) int64
+int64_t scan_tmp_count(int64_t n);
+cudaError_t launch_row_ptr_scan(const int64_t *counts, int64_t n, int64_t *row_ptr, int64_t *tmp,
+                                cudaStream_t s);
 cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, const double *o,
                         const Params *prm, double *dcol, cudaStream_t s);
 cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s);

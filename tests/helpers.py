@@ -8,7 +8,10 @@ Tolerances (the readings are listed in the design doc):
  - marginal residual at the GPU's potentials: within 1e-5 (absolute; the
    residual of a unit-mass plan is at most 2);
  - min_row: thr within 1e-5 relative, the same argmin row, the same kept
-   (i, j) entries except those within 1e-5 relative of thr (counted).
+   (i, j) entries except those within 1e-5 relative of thr (counted);
+ - compressed-row sparsify: at the same thr, the same kept (i, j) except those
+   within 1e-5 relative of thr, columns increasing in each row, values as plan
+   entries.
 """
 from __future__ import annotations
 
@@ -72,3 +75,34 @@ def assert_min_row(got, ref, T_ref_rows=None, rows=None, tol=ROW_TOL):
     assert abs(got["thr"] - ref["thr"]) <= tol * ref["thr"], (got["thr"], ref["thr"])
     assert got["argmin"] == ref["argmin"]
     return 0
+
+
+def csr_rows(row_ptr, col_idx, vals):
+    """{row: (columns, values)} from compressed-row arrays (numpy)."""
+    out = {}
+    for i in range(len(row_ptr) - 1):
+        a, b = int(row_ptr[i]), int(row_ptr[i + 1])
+        out[i] = (np.asarray(col_idx[a:b]), np.asarray(vals[a:b], np.float64))
+    return out
+
+
+def assert_csr(got, ref, thr, tol=ROW_TOL):
+    """got/ref: (row_ptr, col_idx, vals) as numpy arrays, thresholded at thr.
+    The kept sets agree except entries within tol (relative) of thr; values of
+    entries kept by both agree as plan entries. Returns the tie-band count."""
+    g, r = csr_rows(*got), csr_rows(*ref)
+    assert len(g) == len(r)
+    band = 0
+    for i in r:
+        gc, gv = g[i]
+        rc, rv = r[i]
+        assert np.all(np.diff(gc) > 0), f"row {i}: columns not increasing"
+        common, gi, ri = np.intersect1d(gc, rc, return_indices=True)
+        if common.size:
+            assert_entries(gv[gi], rv[ri], tol)
+        only_g = np.setdiff1d(np.arange(len(gc)), gi)
+        only_r = np.setdiff1d(np.arange(len(rc)), ri)
+        for v in list(gv[only_g]) + list(rv[only_r]):
+            assert abs(v - thr) <= tol * thr, f"row {i}: entry {v:.6e} kept by one side only, thr {thr:.6e}"
+            band += 1
+    return band

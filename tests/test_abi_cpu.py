@@ -93,6 +93,7 @@ def test_row_calls_reject_null_plan(B):
     assert L.ot_materialize_rows(None, FAKE, 1, FAKE, None) == -1
     assert L.ot_marginal_residual(None, None, None, None) == -1
     assert L.ot_sparsify_min_row(None, 0, None, None, None, None, None, None) == -1
+    assert L.ot_sparsify_csr(None, 0, 0.5, FAKE, FAKE, FAKE, 1, None, None) == -1
     L.ot_plan_destroy(None)  # no-op
 
 

@@ -97,6 +97,22 @@ def test_w2_8000_full_path(ot, orc):
     rows = torch.arange(3 * 1024, 4 * 1024, device="cuda")
     T = plan.materialize_rows(rows).double().cpu().numpy()
     H.assert_entries(T[::16], orc.materialize_rows(w.x, w.y, f, g, c, w.eps, rows.cpu().numpy()[::16]))
+    # compressed-row sparsify in the same row blocks: min_row's counts, and on
+    # sampled rows the oracle's kept entries (outside the tie band) and values
+    csr = plan.sparsify_csr(block_rows=w.block_rows)
+    assert csr["thr"] == mr["thr"] and csr["nnz"] == mr["nnz"]
+    row_ptr = csr["row_ptr"].cpu().numpy()
+    np.testing.assert_array_equal(np.diff(row_ptr), mr["counts"].cpu().numpy())
+    col_idx, vals = csr["col_idx"].cpu().numpy(), csr["vals"].cpu().numpy()
+    pick = np.arange(0, w.n, 397)
+    Tref = orc.materialize_rows(w.x, w.y, f, g, c, w.eps, pick)
+    ref_ptr = np.concatenate([[0], np.cumsum((Tref >= csr["thr"]).sum(1))])
+    ref_cols = np.concatenate([np.nonzero(r >= csr["thr"])[0] for r in Tref])
+    ref_vals = np.concatenate([r[r >= csr["thr"]] for r in Tref])
+    got_ptr = np.concatenate([[0], np.cumsum([row_ptr[i + 1] - row_ptr[i] for i in pick])])
+    got_cols = np.concatenate([col_idx[row_ptr[i]:row_ptr[i + 1]] for i in pick])
+    got_vals = np.concatenate([vals[row_ptr[i]:row_ptr[i + 1]] for i in pick])
+    H.assert_csr((got_ptr, got_cols, got_vals), (ref_ptr, ref_cols, ref_vals), csr["thr"])
 
 
 def test_w3_tensor_core_full_size(ot, orc):

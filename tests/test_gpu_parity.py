@@ -182,6 +182,53 @@ def test_rows_and_residual_at_gpu_potentials(ot, orc):
         assert torch.equal(o["counts"], outs[0]["counts"])
 
 
+def _csr_case(ot):
+    w = _cloud(33, 517, 389, 2, scale="mean", eps=0.02)
+    w.a = w.a.copy()
+    w.a[[5, 100, 516]] = 0.0  # rows without mass keep nothing
+    x, y, a, b = H.to_dev(w)
+    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=40)
+    return w, plan
+
+
+def test_sparsify_csr_matches_oracle(ot, orc):
+    """Compressed-row sparsify at the GPU's potentials against the oracle's
+    thresholded plan at the same thr: the same kept entries outside the tie band,
+    values as plan entries, increasing columns; counts and nnz are min_row's."""
+    w, plan = _csr_case(ot)
+    mr = plan.sparsify_min_row()
+    csr = plan.sparsify_csr()
+    assert csr["thr"] == mr["thr"] and csr["nnz"] == mr["nnz"]
+    row_ptr = csr["row_ptr"].cpu().numpy()
+    np.testing.assert_array_equal(np.diff(row_ptr), mr["counts"].cpu().numpy())
+    assert all(row_ptr[i + 1] == row_ptr[i] for i in (5, 100, 516))
+    f, g = _pots(plan)
+    ref = orc.sparsify_csr(w.x, w.y, w.a, f, g, plan.info.inv_scale_cost, w.eps, csr["thr"])
+    band = H.assert_csr((row_ptr, csr["col_idx"].cpu().numpy(), csr["vals"].cpu().numpy()), ref,
+                        csr["thr"])
+    assert band <= max(2, csr["nnz"] // 1000)
+    plan.close()
+
+
+def test_sparsify_csr_block_rows_and_threshold(ot):
+    """block_rows never changes the output (bit for bit); a lower threshold keeps
+    a superset; a capacity below nnz is an overflow that reports nnz."""
+    import torch
+    w, plan = _csr_case(ot)
+    outs = [plan.sparsify_csr(block_rows=br) for br in (0, 1, 7, 64)]
+    for o in outs[1:]:
+        for k in ("row_ptr", "col_idx", "vals"):
+            assert torch.equal(o[k], outs[0][k])
+    lo = plan.sparsify_csr(thr=outs[0]["thr"] * 0.5)
+    assert lo["nnz"] >= outs[0]["nnz"]
+    assert plan.sparsify_csr(thr=float("inf"))["nnz"] == 0
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    with pytest.raises(B.OTError) as e:
+        plan.sparsify_csr(thr=outs[0]["thr"], capacity=outs[0]["nnz"] - 1)
+    assert e.value.status == B.OT_ERR_OVERFLOW
+    plan.close()
+
+
 def test_bad_row_index_is_reported(ot):
     import torch
     w = _cloud(3, 300, 200, 2)
