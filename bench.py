@@ -4,7 +4,8 @@ One step = the whole path on the 8000 x 8000, d = 3 Gaussian-mixture workload
 (scale "mean", eps 0.01): the solve to ||T1 - a||_1 <= 1e-3 (cap 2000, fused
 f/g half-steps with the in-loop residual), the float64-assembled marginal
 residual at the returned potentials, the exact min_row threshold and per-row
-counts in row blocks of 1024, and the materialisation of every row in blocks of
+counts in row blocks of 1024, the thresholded plan written in compressed-row
+form (the sparsify output), and the materialisation of every row in blocks of
 1024. Inputs are resident in HBM before the timed region; L2 is flushed before
 every step. The metric counts Sinkhorn pair-updates (n*m per half-step) per
 second; the row passes are inside the timed step but add no units. After the
@@ -168,6 +169,7 @@ class Step:
         self.rows = None if rows is None else torch.from_numpy(rows).to(dev)
         self.out = None if rows is None else torch.empty((min(self.block, len(rows)), w.m),
                                                          dtype=torch.float32, device=dev)
+        self.csr, self.nnz = None, 0
 
     def __call__(self, timing=False):
         w = self.w
@@ -179,6 +181,15 @@ class Step:
         mr = plan.sparsify_min_row(block_rows=w.block_rows, counts=self.counts)
         nb = -(-w.n // (w.block_rows or w.n))
         launches += 1 + 2 * nb + 2
+        # the sparse plan at that threshold, in compressed-row form
+        if self.csr is None or self.csr[1].numel() < mr["nnz"]:
+            import torch
+            cap = max(int(mr["nnz"] * 1.25), 1)
+            self.csr = (torch.empty(w.n + 1, dtype=torch.int64, device=self.dev),
+                        torch.empty(cap, dtype=torch.int64, device=self.dev),
+                        torch.empty(cap, dtype=torch.float32, device=self.dev))
+        self.nnz = plan.sparsify_csr(thr=mr["thr"], block_rows=w.block_rows, out=self.csr)["nnz"]
+        launches += 1 + 2 * nb + 3
         if self.rows is not None:
             for r0 in range(0, self.rows.numel(), self.block):
                 r = self.rows[r0:r0 + self.block]
@@ -312,8 +323,13 @@ def run_ours(args):
     host = [torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for v in (w.x, w.y, w.a, w.b)]
     outs = [torch.empty(w.n, dtype=torch.float32).pin_memory(), torch.empty(w.m, dtype=torch.float32).pin_memory(),
             torch.empty(w.n, dtype=torch.int64).pin_memory()]
+    # the sparse plan (row pointers, column indices, values) comes back too
+    csr_host = None if step.csr is None else [torch.empty(t.numel(), dtype=t.dtype).pin_memory()
+                                              for t in step.csr]
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = sum(t.numel() * t.element_size() for t in outs)
+    if csr_host is not None:
+        d2h += (w.n + 1) * 8 + step.nnz * (8 + 4)
     e2e_ms, e2e_units = 0.0, 0.0
     _barrier(dist)
     for _ in range(args.steps):
@@ -327,6 +343,10 @@ def run_ours(args):
         outs[0].copy_(step.f, non_blocking=True)
         outs[1].copy_(step.g, non_blocking=True)
         outs[2].copy_(step.counts, non_blocking=True)
+        if csr_host is not None:
+            csr_host[0].copy_(step.csr[0], non_blocking=True)
+            csr_host[1][:step.nnz].copy_(step.csr[1][:step.nnz], non_blocking=True)
+            csr_host[2][:step.nnz].copy_(step.csr[2][:step.nnz], non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms += e0.elapsed_time(e1)

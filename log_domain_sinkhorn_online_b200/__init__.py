@@ -84,25 +84,36 @@ class Plan:
                                                       _stream(stream))
         return dict(thr=thr, counts=counts, nnz=nnz, n_massless=nm, argmin=arg, status=st)
 
-    def sparsify_csr(self, thr=None, block_rows=0, capacity=None, stream=None):
+    def sparsify_csr(self, thr=None, block_rows=0, capacity=None, out=None, stream=None):
         """The plan thresholded at thr (default: the min_row threshold) in
         compressed-row form. Returns dict(row_ptr [n+1] int64, col_idx [nnz]
         int64, vals [nnz] float32, nnz, thr); torch.sparse_csr_tensor(row_ptr,
-        col_idx, vals, (n, m)) turns it into a torch sparse matrix."""
+        col_idx, vals, (n, m)) turns it into a torch sparse matrix. out: an
+        optional (row_ptr, col_idx, vals) of device tensors to write into (the
+        capacity is col_idx's length)."""
         import torch
         dev = self.f.device
         n = self.f.numel()
         if thr is None:
             mr = self.sparsify_min_row(block_rows=block_rows, stream=stream)
             thr = mr["thr"]
-            if capacity is None:
+            if capacity is None and out is None:
                 capacity = mr["nnz"]
-        row_ptr = torch.empty(n + 1, dtype=torch.int64, device=dev)
-        if capacity is None:  # size it first: a call with no room only counts
-            _, capacity = B.ot_sparsify_csr(self._h, int(block_rows), float(thr), row_ptr.data_ptr(),
-                                            0, 0, 0, _stream(stream))
-        col_idx = torch.empty(max(int(capacity), 1), dtype=torch.int64, device=dev)
-        vals = torch.empty(max(int(capacity), 1), dtype=torch.float32, device=dev)
+        if out is not None:
+            row_ptr, col_idx, vals = out
+            _dev(row_ptr, torch.int64, "row_ptr")
+            _dev(col_idx, torch.int64, "col_idx")
+            _dev(vals, torch.float32, "vals")
+            if row_ptr.numel() != n + 1 or vals.numel() < col_idx.numel():
+                raise ValueError("out: row_ptr needs n + 1 entries and vals as many as col_idx")
+            capacity = col_idx.numel()
+        else:
+            row_ptr = torch.empty(n + 1, dtype=torch.int64, device=dev)
+            if capacity is None:  # size it first: a call with no room only counts
+                _, capacity = B.ot_sparsify_csr(self._h, int(block_rows), float(thr),
+                                                row_ptr.data_ptr(), 0, 0, 0, _stream(stream))
+            col_idx = torch.empty(max(int(capacity), 1), dtype=torch.int64, device=dev)
+            vals = torch.empty(max(int(capacity), 1), dtype=torch.float32, device=dev)
         st, nnz = B.ot_sparsify_csr(self._h, int(block_rows), float(thr), row_ptr.data_ptr(),
                                     col_idx.data_ptr(), vals.data_ptr(), int(capacity), _stream(stream))
         if st == B.OT_ERR_OVERFLOW:
