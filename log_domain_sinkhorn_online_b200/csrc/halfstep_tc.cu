@@ -16,16 +16,19 @@
 // 1.8e-6). The row constant -c kappa |x'_i|^2 is added once per row, in
 // float64, by the shared tile finalizer.
 //
-// Block: 17 warps. Warp 16's elected lane is the producer: TMA loads of the row
-// tile (once per work item) and of 128-column chunks of the column operand into
-// a 3-stage (2 for K > 192) shared-memory ring, 128B-swizzled K-major, and the
-// tcgen05.mma issue into one of two TMEM accumulators (128 lanes x 128 fp32
-// columns each). Warps 0-15 are the epilogue (four per SM sub-partition, to hide
-// the TMEM-load latency): warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and
-// columns 32*(w/4)..+31 of each chunk, then runs the lazily-rescaled max / ex2 /
-// sum per row; the four column quarters of a row merge in shared memory. Every wait on an mbarrier is bounded;
-// on timeout the block records State::wait_timeout, drains what it issued (again
-// bounded), frees its TMEM and returns. No TMA load uses cluster multicast.
+// Block: 18 warps. Warp 16's elected lane issues the TMA loads of the row tile
+// (once per work item) and of 128-column chunks of the column operand into a
+// 3-stage (2 for K > 192) shared-memory ring, 128B-swizzled K-major; warp 17's
+// issues tcgen05.mma into one of four TMEM accumulators (128 lanes x 128 fp32
+// columns each). Warps 0-15 are the epilogue, four per accumulator: warp w
+// drains buffer w/4 (TMEM lanes 32*(w%4)..+31, its rows; all 128 columns of
+// every chunk in that buffer) with the lazily-rescaled max / ex2 / sum per row;
+// the four buffers' states of a row merge in shared memory at the end of a work
+// item. Each SM sub-partition holds one warp per buffer, a chunk apart in time,
+// so one warp's waits and loads overlap another's exponentials. Every wait on
+// an mbarrier is bounded; on timeout the block records State::wait_timeout,
+// drains what it issued (again bounded), frees its TMEM and returns. No TMA
+// load uses cluster multicast.
 #include <cuda.h>
 
 #include "finish.cuh"
@@ -38,7 +41,6 @@ constexpr int M = 128;               // rows per tile (MMA M)
 constexpr int N = 128;               // columns per chunk (MMA N)
 constexpr int EPI_WARPS = 16;         // 4 per SM sub-partition
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int QCOLS = N / (EPI_WARPS / 4);  // columns of a chunk per epilogue warp
 constexpr int THREADS = (EPI_WARPS + 2) * 32;  // + TMA warp + MMA warp
 constexpr int SLAB = 64;             // bf16 per 128-byte swizzle row
 constexpr int SLAB_BYTES = M * 128;  // one slab of a 128-row operand tile (16 KB)
@@ -108,7 +110,8 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");  // it reads shared memory: keep it after the barrier waits
 }
 
 // arrives once on `bar` when every MMA issued so far by this thread completes
@@ -178,6 +181,7 @@ __device__ __forceinline__ void tmem_wait_ld(float (&v)[32]) {
 
 constexpr int NBUF = 4;  // TMEM accumulators (4 x 128 fp32 columns = all 512)
 constexpr int TMA_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
+static_assert(EPI_WARPS == 4 * NBUF, "one group of four epilogue warps per accumulator buffer");
 
 // Shared-memory plan (dynamic; base rounded up to 1024 B for the 128B swizzle).
 template <int KS>
@@ -228,7 +232,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], EPI_WARPS);
+            mbar_init(&tempty[b], 4);  // the four warps (one per lane quarter) that drain buffer b
         }
         mbar_init(afull, 1);
         mbar_init(aempty, 1);
@@ -298,7 +302,12 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                         break;
                     tc_fence_after();
                     const uint8_t *bst = sB + st * KS * SLAB_BYTES;
-                    for (int k = 0; k < ksteps; ++k) {
+                    // fully unrolled over the template bound: with a loop over the runtime
+                    // count the issue of one tcgen05.mma took ~120 cycles (half the
+                    // tensor rate of a 128 x 128 x 16 MMA); unrolled it keeps up
+#pragma unroll
+                    for (int k = 0; k < 4 * KS; ++k) {
+                        if (k >= ksteps) break;
                         const int slab = k >> 2;
                         const uint64_t adv = (uint64_t)((k & 3) * 2);  // 32 bytes per K step of 16
                         mma_bf16(tmem + (uint32_t)(b * N), smem_desc(sA + slab * SLAB_BYTES) + adv,
@@ -320,11 +329,17 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
         }
     } else {
         // -------------------------------------------------------- epilogue
-        const int q = warp & 3, h = warp >> 2;  // TMEM lane quarter, column quarter
+        // Warp w drains accumulator buffer h = w / 4 for TMEM lanes 32 (w % 4)..+31:
+        // every chunk that the MMA warp put in buffer h (global chunk g with
+        // g % NBUF == h), all 128 columns, as four 32-column loads with the next
+        // one in flight. Each SM sub-partition thus holds one warp of each of the
+        // four buffers, a chunk apart in time, so one warp's waits and loads
+        // overlap another's exponentials.
+        const int q = warp & 3, h = warp >> 2;  // TMEM lane quarter, accumulator buffer
         const int r = q * 32 + lane;  // row of the tile owned by this thread
         const int etid = threadIdx.x;  // 0 .. EPI_THREADS-1
-        const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * QCOLS);
-        uint32_t g = 0;
+        const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * N);
+        uint32_t g = 0, uses = 0;  // chunks issued by the MMA warp so far; uses of buffer h
         for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
             const int tile = (int)(item / A.splits), split = (int)(item % A.splits);
             const int64_t c0 = (int64_t)split * A.cols_per_split;
@@ -335,65 +350,59 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
             for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
             float va[32], vb[32];
-            // the item's first chunk: wait, load, release the accumulator
-            bool ok = mbar_wait_warp(&tfull[g % NBUF], (g / NBUF) & 1, s_abort);
-            if (ok) {
+            bool ok = true;
+            for (int ch = (int)(((uint32_t)h + NBUF - g % NBUF) % NBUF); ch < nch && ok; ch += NBUF) {
+                ok = mbar_wait_warp(&tfull[h], uses & 1, s_abort);
+                if (!ok) break;
                 tc_fence_after();
-                tmem_ld32(tlane + (uint32_t)((g % NBUF) * N), va);
+                tmem_ld32(tlane, va);
                 tmem_wait_ld(va);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[g % NBUF]);
-            }
-            for (int ch = 0; ch < nch && ok; ++ch, ++g) {
-                const bool more = ch + 1 < nch;
-                if (more) {  // start loading the next chunk before this chunk's exponentials
-                    const uint32_t gn = g + 1;
-                    ok = mbar_wait_warp(&tfull[gn % NBUF], (gn / NBUF) & 1, s_abort);
-                    if (ok) {
-                        tc_fence_after();
-                        tmem_ld32(tlane + (uint32_t)((gn % NBUF) * N), vb);
+#pragma unroll 1
+                for (int sc = 0; sc < N / 32; ++sc) {
+                    const bool more = sc + 1 < N / 32;
+                    if (more) tmem_ld32(tlane + (uint32_t)((sc + 1) * 32), vb);
+                    // running maximum, refreshed lazily (terms stay <= 2^8)
+                    float p[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        p[j] = fmax3(fmax3(va[8 * j], va[8 * j + 1], va[8 * j + 2]),
+                                     fmax3(va[8 * j + 3], va[8 * j + 4], va[8 * j + 5]),
+                                     fmaxf(va[8 * j + 6], va[8 * j + 7]));
+                    const float cm = fmax3(p[0], p[1], fmaxf(p[2], p[3]));
+                    if (__any_sync(0xffffffffu, cm > m + kLazyMax)) {
+                        const float mx = fmaxf(cm, m);
+                        const float sc2 = ex2_approx(m - mx);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) acc[u] = __fmul2_rn(acc[u], make_float2(sc2, sc2));
+                        tot *= sc2;
+                        m = mx;
+                        nm = make_float2(-mx, -mx);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float2 u0 = __fadd2_rn(make_float2(va[2 * j], va[2 * j + 1]), nm);
+                        acc[j & 3] = __fadd2_rn(acc[j & 3], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
+                    }
+                    float cs = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        cs += acc[u].x + acc[u].y;
+                        acc[u] = make_float2(0.f, 0.f);
+                    }
+                    tot += cs;
+                    if (more) {
+                        tmem_wait_ld(vb);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) va[i] = vb[i];
                     }
                 }
-                // running maximum, refreshed lazily (terms stay <= 2^8)
-                float p[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    p[j] = fmax3(fmax3(va[8 * j], va[8 * j + 1], va[8 * j + 2]),
-                                 fmax3(va[8 * j + 3], va[8 * j + 4], va[8 * j + 5]),
-                                 fmaxf(va[8 * j + 6], va[8 * j + 7]));
-                const float cm = fmax3(p[0], p[1], fmaxf(p[2], p[3]));
-                if (__any_sync(0xffffffffu, cm > m + kLazyMax)) {
-                    const float mx = fmaxf(cm, m);
-                    const float sc = ex2_approx(m - mx);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) acc[u] = __fmul2_rn(acc[u], make_float2(sc, sc));
-                    tot *= sc;
-                    m = mx;
-                    nm = make_float2(-mx, -mx);
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float2 u0 = __fadd2_rn(make_float2(va[2 * j], va[2 * j + 1]), nm);
-                    acc[j & 3] = __fadd2_rn(acc[j & 3], make_float2(ex2_approx(u0.x), ex2_approx(u0.y)));
-                }
-                float cs = 0.0f;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    cs += acc[u].x + acc[u].y;
-                    acc[u] = make_float2(0.f, 0.f);
-                }
-                tot += cs;
-                if (more && ok) {
-                    tmem_wait_ld(vb);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[(g + 1) % NBUF]);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) va[i] = vb[i];
-                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[h]);
+                ++uses;
             }
-            // merge the column quarters of each row, then the column splits
+            g += (uint32_t)nch;
+            // merge the four buffers' partial states of each row, then the column splits
             s_merge[h * M + r] = make_float2(m, tot);
             asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
             // one thread samples the abort flag, so every epilogue thread takes
