@@ -22,10 +22,16 @@
 // issues tcgen05.mma into one of four TMEM accumulators (128 lanes x 128 fp32
 // columns each). Warps 0-15 are the epilogue, four per accumulator: warp w
 // drains buffer w/4 (TMEM lanes 32*(w%4)..+31, its rows; all 128 columns of
-// every chunk in that buffer) with the lazily-rescaled max / ex2 / sum per row;
+// chunks w/4, w/4 + 4, ... of each work item) with the lazily-rescaled max /
+// ex2 / sum per row, so the summation order depends on the item alone;
 // the four buffers' states of a row merge in shared memory at the end of a work
 // item. Each SM sub-partition holds one warp per buffer, a chunk apart in time,
-// so one warp's waits and loads overlap another's exponentials. Every wait on
+// so one warp's waits and loads overlap another's exponentials. Work items are
+// claimed dynamically by the producer (its first one is its block index, the
+// next ones come from the side's atomic counter) and handed to the MMA warp and
+// the epilogue through a four-slot ring in shared memory guarded by mbarriers
+// (a static stride left SMs idle 16 % of a launch: per-block times spread from
+// 672 to 874 us at 40000 x 50000, d = 50). Every wait on
 // an mbarrier is bounded; on timeout the block records State::wait_timeout,
 // drains what it issued (again bounded), frees its TMEM and returns. No TMA
 // load uses cluster multicast.
@@ -180,6 +186,7 @@ __device__ __forceinline__ void tmem_wait_ld(float (&v)[32]) {
 }
 
 constexpr int NBUF = 4;  // TMEM accumulators (4 x 128 fp32 columns = all 512)
+constexpr int RING = 4;  // work items published by the producer ahead of the MMA warp and the epilogue
 constexpr int TMA_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
 static_assert(EPI_WARPS == 4 * NBUF, "one group of four epilogue warps per accumulator buffer");
 
@@ -190,10 +197,12 @@ struct Smem {
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = KS * SLAB_BYTES;
     static constexpr int BAR_OFF = B_OFF + STAGES * KS * SLAB_BYTES;
-    // full[S], empty[S], tfull[NBUF], tempty[NBUF], afull, aempty, drain
-    static constexpr int NBAR = 2 * STAGES + 2 * NBUF + 3;
-    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem addr, abort, flag, decide, 16 doubles
-    static constexpr int MERGE_OFF = MISC_OFF + 160;      // float2 [EPI_WARPS/4][M]
+    // full[S], empty[S], tfull[NBUF], tempty[NBUF], afull, aempty, drain, ifull[RING], iempty[RING]
+    static constexpr int NBAR = 2 * STAGES + 2 * NBUF + 3 + 2 * RING;
+    // tmem addr, abort, flag, decide, 16 doubles, RING item slots, the epilogue's item
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int ITEMS_OFF = MISC_OFF + 144;
+    static constexpr int MERGE_OFF = MISC_OFF + 256;      // float2 [EPI_WARPS/4][M]
     static constexpr int BYTES = MERGE_OFF + (EPI_WARPS / 4) * M * 8;
     // at least 116 KB, so that one block holds an SM (it takes all 512 TMEM columns)
     static constexpr int ALLOC = (BYTES + 1024) > 116 * 1024 ? BYTES + 1024 : 116 * 1024;
@@ -206,6 +215,8 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     using L = Smem<KS>;
     constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
+    // the other side's work-item counter (as in the CUDA-core half-steps)
+    if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;
     if (ld_volatile(&A.st->stop)) return;
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *sA = sm + L::A_OFF;
@@ -217,6 +228,10 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     uint64_t *afull = tempty + NBUF;
     uint64_t *aempty = afull + 1;
     uint64_t *drain = aempty + 1;
+    uint64_t *ifull = drain + 1;
+    uint64_t *iempty = ifull + RING;
+    volatile long long *s_items = reinterpret_cast<volatile long long *>(sm + L::ITEMS_OFF);
+    volatile long long *s_item_epi = s_items + RING;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
     volatile int *s_abort = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
     int *s_flag = reinterpret_cast<int *>(sm + L::MISC_OFF + 8);
@@ -237,6 +252,10 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
         mbar_init(afull, 1);
         mbar_init(aempty, 1);
         mbar_init(drain, 1);
+        for (int q = 0; q < RING; ++q) {
+            mbar_init(&ifull[q], 1);   // the producer, after writing the slot
+            mbar_init(&iempty[q], 2);  // the MMA lane and the epilogue, after reading it
+        }
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -258,7 +277,17 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) {
             uint32_t g = 0, item_no = 0, issued[STAGES] = {};
             bool ok = true, a_out = false;
-            for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++item_no) {
+            int64_t item = blockIdx.x;
+            for (uint32_t iq = 0; ok; ++iq, ++item_no) {
+                // publish the item (or the end) to the MMA warp and the epilogue
+                const int slot = (int)(iq % RING);
+                if (iq >= (uint32_t)RING && !(ok = mbar_wait(&iempty[slot], ((iq / RING) - 1) & 1, s_abort)))
+                    break;
+                s_items[slot] = item < n_items ? item : -1;
+                mbar_arrive(&ifull[slot]);
+                if (item >= n_items) break;
+                // claim the next item now; its value is needed only after this item's loads
+                const int64_t next = (int64_t)gridDim.x + (int64_t)atomicAdd(&A.st->work[A.side], 1u);
                 const int tile = (int)(item / A.splits), split = (int)(item % A.splits);
                 const int64_t c0 = (int64_t)split * A.cols_per_split;
                 const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
@@ -277,6 +306,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                         tma_load_2d(dst + s * SLAB_BYTES, &tmB, &full[st], s * SLAB, (int)(c0 + (int64_t)ch * N));
                     ++issued[st];
                 }
+                item = next;
             }
             if (!ok) {  // wait (bounded) for the loads this block put in flight
                 if (a_out) mbar_drain(afull, (item_no & 1) ^ 0);
@@ -288,18 +318,25 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------ MMA issue
         if (lane == 0) {
-            uint32_t g = 0, item_no = 0;
+            uint32_t g = 0, item_no = 0, ub[NBUF] = {};  // ub: uses of each accumulator
             bool ok = true, issued_any = false;
-            for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++item_no) {
+            for (uint32_t iq = 0; ok; ++iq, ++item_no) {
+                const int slot = (int)(iq % RING);
+                if (!(ok = mbar_wait(&ifull[slot], (iq / RING) & 1, s_abort))) break;
+                const int64_t item = s_items[slot];
+                mbar_arrive(&iempty[slot]);
+                if (item < 0) break;
                 const int split = (int)(item % A.splits);
                 const int64_t c0 = (int64_t)split * A.cols_per_split;
                 const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
                 if (!(ok = mbar_wait(afull, item_no & 1, s_abort))) break;
                 for (int ch = 0; ch < nch; ++ch, ++g) {
-                    const int st = g % STAGES, b = g % NBUF;
+                    // accumulator by the chunk's index in its item, so that which epilogue
+                    // warps sum which columns does not depend on the schedule
+                    const int st = g % STAGES, b = ch % NBUF;
                     if (!(ok = mbar_wait(&full[st], (g / STAGES) & 1, s_abort))) break;
-                    if (g >= (uint32_t)NBUF && !(ok = mbar_wait(&tempty[b], ((g / NBUF) - 1) & 1, s_abort)))
-                        break;
+                    if (ub[b] > 0 && !(ok = mbar_wait(&tempty[b], (ub[b] - 1) & 1, s_abort))) break;
+                    ++ub[b];
                     tc_fence_after();
                     const uint8_t *bst = sB + st * KS * SLAB_BYTES;
                     // fully unrolled over the template bound: with a loop over the runtime
@@ -330,17 +367,30 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     } else {
         // -------------------------------------------------------- epilogue
         // Warp w drains accumulator buffer h = w / 4 for TMEM lanes 32 (w % 4)..+31:
-        // every chunk that the MMA warp put in buffer h (global chunk g with
-        // g % NBUF == h), all 128 columns, as four 32-column loads with the next
-        // one in flight. Each SM sub-partition thus holds one warp of each of the
+        // the chunks ch = h, h + 4, ... of every work item (the MMA warp puts chunk
+        // ch in buffer ch % 4), all 128 columns, as four 32-column loads with the
+        // next one in flight. Each SM sub-partition thus holds one warp of each of the
         // four buffers, a chunk apart in time, so one warp's waits and loads
         // overlap another's exponentials.
         const int q = warp & 3, h = warp >> 2;  // TMEM lane quarter, accumulator buffer
         const int r = q * 32 + lane;  // row of the tile owned by this thread
         const int etid = threadIdx.x;  // 0 .. EPI_THREADS-1
         const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * N);
-        uint32_t g = 0, uses = 0;  // chunks issued by the MMA warp so far; uses of buffer h
-        for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+        uint32_t uses = 0;  // uses of buffer h so far
+        for (uint32_t iq = 0;; ++iq) {
+            // thread 0 takes the next item from the producer and hands it to the others
+            if (etid == 0) {
+                const int slot = (int)(iq % RING);
+                long long it = -1;
+                if (mbar_wait(&ifull[slot], (iq / RING) & 1, s_abort)) {
+                    it = s_items[slot];
+                    mbar_arrive(&iempty[slot]);
+                }
+                *s_item_epi = it;
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
+            const int64_t item = *s_item_epi;
+            if (item < 0) break;
             const int tile = (int)(item / A.splits), split = (int)(item % A.splits);
             const int64_t c0 = (int64_t)split * A.cols_per_split;
             const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
@@ -351,7 +401,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
             float va[32], vb[32];
             bool ok = true;
-            for (int ch = (int)(((uint32_t)h + NBUF - g % NBUF) % NBUF); ch < nch && ok; ch += NBUF) {
+            for (int ch = h; ch < nch && ok; ch += NBUF) {
                 ok = mbar_wait_warp(&tfull[h], uses & 1, s_abort);
                 if (!ok) break;
                 tc_fence_after();
@@ -401,7 +451,6 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                 if (lane == 0) mbar_arrive(&tempty[h]);
                 ++uses;
             }
-            g += (uint32_t)nch;
             // merge the four buffers' partial states of each row, then the column splits
             s_merge[h * M + r] = make_float2(m, tot);
             asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
