@@ -229,6 +229,37 @@ def test_sparsify_csr_block_rows_and_threshold(ot):
     plan.close()
 
 
+@pytest.mark.parametrize("d,loop", [(3, 0), (8, 0), (24, 0)])
+def test_dynamic_work_items_are_deterministic(ot, d, loop):
+    """The per-launch kernels claim work items at run time; which block runs an
+    item must not change a result: two solves agree bit for bit."""
+    import torch
+    w = _cloud(57, 3001, 2777, d, scale="mean", eps=0.03)
+    x, y, a, b = H.to_dev(w)
+    outs = []
+    for _ in range(2):
+        plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=15, device_loop=loop)
+        outs.append((plan.f.clone(), plan.g.clone()))
+        plan.close()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_sparsify_csr_generic_d(ot, orc):
+    """The compressed-row sparsify on the generic-d entry path (d = 5)."""
+    w = _cloud(61, 301, 257, 5, scale="max_cost", eps=0.03)
+    x, y, a, b = H.to_dev(w)
+    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=25)
+    csr = plan.sparsify_csr(block_rows=64)
+    mr = plan.sparsify_min_row()
+    assert csr["nnz"] == mr["nnz"]
+    f, g = _pots(plan)
+    ref = orc.sparsify_csr(w.x, w.y, w.a, f, g, plan.info.inv_scale_cost, w.eps, csr["thr"])
+    band = H.assert_csr((csr["row_ptr"].cpu().numpy(), csr["col_idx"].cpu().numpy(),
+                         csr["vals"].cpu().numpy()), ref, csr["thr"])
+    assert band <= max(2, csr["nnz"] // 1000)
+    plan.close()
+
+
 def test_bad_row_index_is_reported(ot):
     import torch
     w = _cloud(3, 300, 200, 2)
