@@ -66,6 +66,8 @@ def _load():
             lib.orc_min_row.argtypes = [P, P, P, P, P, I64, I64, I32, D, D, I64, P, P, P, P]
             lib.orc_min_row.restype = I64
             lib.orc_sparsify_csr.argtypes = [P, P, P, P, P, I64, I64, I32, D, D, D, P, P, P, I64]
+            lib.orc_lr_rows.argtypes = [P, P, P, I64, I64, I32, P, I64, P]
+            lib.orc_lrc_rows.argtypes = [P, P, P, P, I64, I64, I32, D, D, D, P, I64, P]
             lib.orc_sparsify_csr.restype = I64
             _lib = lib
     return _lib
@@ -234,6 +236,34 @@ def sparsify_csr(x, y, a, f, g, c, eps, thr):
                              _ptr(row_ptr), _ptr(col_idx), _ptr(vals), ctypes.c_int64(total))
     assert nnz == total
     return row_ptr, col_idx[:total], vals[:total]
+
+
+def lr_rows(Q, R, g, rows):
+    """Rows of the low-rank coupling Q diag(1/g) R^T (moscot PR #846, "Fix")."""
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    R = np.ascontiguousarray(R, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    n, r = Q.shape
+    m = R.shape[0]
+    out = np.empty((len(rows), m), dtype=np.float64)
+    _load().orc_lr_rows(_ptr(Q), _ptr(R), _ptr(g), n, m, r, _ptr(rows), len(rows), _ptr(out))
+    return out
+
+
+def lrc_rows(cost1, cost2, f, g, bias, c, eps, rows):
+    """Entropic rows exp((f_i + g_j - c (cost1[i].cost2[j] + bias))/eps) on a
+    low-rank cost geometry (moscot PR #846, "Fix")."""
+    cost1 = np.ascontiguousarray(cost1, dtype=np.float32)
+    cost2 = np.ascontiguousarray(cost2, dtype=np.float32)
+    f, g = _f64(f), _f64(g)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    n, r = cost1.shape
+    m = cost2.shape[0]
+    out = np.empty((len(rows), m), dtype=np.float64)
+    _load().orc_lrc_rows(_ptr(cost1), _ptr(cost2), _ptr(f), _ptr(g), n, m, r, float(bias), float(c),
+                         float(eps), _ptr(rows), len(rows), _ptr(out))
+    return out
 
 
 def min_row(x, y, a, f, g, c, eps, block_rows=0):

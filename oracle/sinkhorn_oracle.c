@@ -343,6 +343,46 @@ int64_t orc_min_row(const float *x, const float *y, const double *a, const doubl
     return massless;
 }
 
+/* ------------------------------------------------------------ low rank --
+ * Rows of a low-rank coupling (moscot PR #846, "Fix": for low-rank outputs
+ * T[rows] = (Q diag(1/g) R^T)[rows], a matrix product, no geometry):
+ *     out[t*m + j] = sum_k Q[i,k] R[j,k] / g[k],   i = rows[t].
+ * Q [n,r], R [m,r], g [r] as given (float32, promoted to double).          */
+void orc_lr_rows(const float *Q, const float *R, const float *g, int64_t n, int64_t m, int r,
+                 const int64_t *rows, int64_t k, double *out) {
+    (void)n;
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < k; ++t) {
+        const int64_t i = rows[t];
+        for (int64_t j = 0; j < m; ++j) {
+            double s = 0.0;
+            for (int q = 0; q < r; ++q)
+                s += (double)Q[i * r + q] * (double)R[j * r + q] / (double)g[q];
+            out[t * m + j] = s;
+        }
+    }
+}
+
+/* Entropic rows on a low-rank cost geometry (same page: cost rows
+ * cost_1[rows] @ cost_2^T + bias), with the captured scale c and eps:
+ *     C_ij = c * (sum_k cost1[i,k] cost2[j,k] + bias),
+ *     out[t*m + j] = exp((f_i + g_j - C_ij) / eps),   i = rows[t].         */
+void orc_lrc_rows(const float *c1, const float *c2, const double *f, const double *g, int64_t n,
+                  int64_t m, int r, double bias, double c, double eps, const int64_t *rows,
+                  int64_t k, double *out) {
+    (void)n;
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < k; ++t) {
+        const int64_t i = rows[t];
+        for (int64_t j = 0; j < m; ++j) {
+            double dot = 0.0;
+            for (int q = 0; q < r; ++q) dot += (double)c1[i * r + q] * (double)c2[j * r + q];
+            const double C = c * (dot + bias);
+            out[t * m + j] = exp((f[i] + g[j] - C) / eps);
+        }
+    }
+}
+
 /* ------------------------------------------------------------- sparsify --
  * The sparse plan that thresholding produces (moscot PR #846, "Behavioural
  * changes": entries with T_ij >= thr are kept, rows without mass keep nothing),

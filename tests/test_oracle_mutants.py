@@ -27,6 +27,8 @@ MUTANTS = {
     "g_step_uses_a_weight": ("out = eps * log(b[j]) - eps * lse(v, n);", "out = eps * log(b[0]) - eps * lse(v, n);"),
     "csr_strict_threshold": ("            if (t >= thr) {\n                col_idx[k] = j;", "            if (t > thr) {\n                col_idx[k] = j;"),
     "csr_drops_the_column_order": ("                col_idx[k] = j;", "                col_idx[k] = m - 1 - j;"),
+    "lr_multiplies_by_g": ("(double)R[j * r + q] / (double)g[q];", "(double)R[j * r + q] * (double)g[q];"),
+    "lrc_drops_the_bias": ("const double C = c * (dot + bias);", "const double C = c * dot;"),
 }
 
 
@@ -116,6 +118,14 @@ def _battery(orc):
             dense[i, col_idx[row_ptr[i]:row_ptr[i + 1]]] = vals[row_ptr[i]:row_ptr[i + 1]]
         return np.array_equal(dense != 0, T >= thr) and np.array_equal(dense[T >= thr], T[T >= thr])
 
+    def lowrank():
+        g4 = np.array([0.2, 0.3, 0.5])
+        Q = np.outer(a, g4)
+        R = np.outer(b, g4)
+        ok = np.allclose(orc.lr_rows(Q, R, g4, np.arange(len(a))), np.outer(a, b), rtol=1e-6)
+        one = orc.lrc_rows(np.array([[2.0]]), np.array([[3.0]]), [0.4], [-0.1], 1.0, 0.5, 0.2, [0])
+        return ok and abs(one[0, 0] / math.exp((0.4 - 0.1 - 0.5 * 7.0) / 0.2) - 1) < 1e-12
+
     def mean_scale():
         xd, yd = x.astype(np.float64), y.astype(np.float64)
         mean = (xd ** 2).sum(1).mean() + (yd ** 2).sum(1).mean() - 2 * xd.mean(0) @ yd.mean(0)
@@ -124,6 +134,7 @@ def _battery(orc):
     for name, fn in [("row_marginals", row_marginals), ("col_marginals", col_marginals),
                      ("two_point", two_point), ("cross_ratio", cross_ratio),
                      ("min_row_contract", min_row_contract), ("residual", residual), ("csr", csr),
+                     ("lowrank", lowrank),
                      ("mean_scale", mean_scale)]:
         check(name, fn)
     return failed

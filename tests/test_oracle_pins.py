@@ -313,6 +313,57 @@ def test_sparsify_csr_is_the_thresholded_plan(orc):
     np.testing.assert_array_equal(dense[mask], T[mask])
 
 
+def test_lr_rows_separable_factors_give_the_product_coupling(orc):
+    # Q = a g^T, R = b g^T with sum(g) = 1: Q diag(1/g) R^T = a b^T sum(g) = a b^T
+    # (moscot PR #846, "Fix": low-rank rows are (Q diag(1/g) R^T)[rows]).
+    rng = np.random.default_rng(3)
+    a = rng.random(9); a /= a.sum()
+    b = rng.random(6); b /= b.sum()
+    g = rng.random(4) + 0.3; g /= g.sum()
+    T = orc.lr_rows(np.outer(a, g), np.outer(b, g), g, np.arange(9))
+    np.testing.assert_allclose(T, np.outer(a, b), rtol=1e-6)
+
+
+def test_lr_rows_marginal_and_rank(orc):
+    # If R^T 1 = g then T 1 = Q 1; T = Q diag(1/g) R^T has rank <= r; rows in any
+    # order and repeated come out as the same rows.
+    rng = np.random.default_rng(4)
+    n, m, r = 30, 25, 3
+    g = (rng.random(r) + 0.5).astype(np.float32)
+    R = rng.random((m, r)).astype(np.float64)
+    R = (R / R.sum(0) * g.astype(np.float64)).astype(np.float32)
+    Q = rng.random((n, r)).astype(np.float32)
+    T = orc.lr_rows(Q, R, g, np.arange(n))
+    want = Q.astype(np.float64).sum(1)
+    np.testing.assert_allclose(T.sum(1), want, rtol=2e-6)
+    sv = np.linalg.svd(T, compute_uv=False)
+    assert sv[r] <= 1e-12 * sv[0]
+    rows = np.array([7, 0, 7, 29])
+    np.testing.assert_array_equal(orc.lr_rows(Q, R, g, rows), T[rows])
+
+
+def test_lrc_rows_squared_euclidean_factorisation(orc):
+    # ||x - y||^2 = [|x|^2, 1, -2x] . [1, |y|^2, y]: the low-rank-cost rows with these
+    # factors are the point-cloud plan rows (moscot PR #846, "Fix", cost rows of an
+    # LRCGeometry); a bias b multiplies every entry by exp(-c b / eps).
+    x, y = _cloud(23, 12, 10, 3)
+    f = np.random.default_rng(5).normal(0, 0.1, 12)
+    g = np.random.default_rng(6).normal(0, 0.1, 10)
+    xd, yd = x.astype(np.float64), y.astype(np.float64)
+    c1 = np.concatenate([(xd ** 2).sum(1, keepdims=True), np.ones((12, 1)), -2 * xd], 1)
+    c2 = np.concatenate([np.ones((10, 1)), (yd ** 2).sum(1, keepdims=True), yd], 1)
+    rows = np.array([0, 5, 11])
+    eps, c = 0.1, 0.7
+    ref = orc.materialize_rows(x, y, f, g, c, eps, rows)
+    got = orc.lrc_rows(c1, c2, f, g, 0.0, c, eps, rows)
+    np.testing.assert_allclose(got, ref, rtol=1e-5)
+    biased = orc.lrc_rows(c1, c2, f, g, 0.25, c, eps, rows)
+    np.testing.assert_allclose(biased, got * np.exp(-c * 0.25 / eps), rtol=1e-12)
+    # one factor each, by hand: C = c (2 * 3 + bias)
+    one = orc.lrc_rows(np.array([[2.0]]), np.array([[3.0]]), [0.4], [-0.1], 1.0, 0.5, 0.2, [0])
+    assert one[0, 0] == pytest.approx(math.exp((0.4 - 0.1 - 0.5 * (6.0 + 1.0)) / 0.2), rel=1e-12)
+
+
 def test_min_row_all_massless(orc):
     x, y = _cloud(16, 5, 4, 2)
     o = orc.min_row(x, y, np.zeros(5), np.full(5, -np.inf), np.zeros(4), 1.0, 0.1)
