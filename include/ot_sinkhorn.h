@@ -186,6 +186,37 @@ OT_API int ot_marginal_residual(const ot_plan *plan, double *row_l1, double *col
 OT_API int ot_materialize_rows(const ot_plan *plan, const int64_t *row_idx, int64_t k, float *out,
                         void *stream);
 
+/* ------------------------------------------------ ot_materialize_rows_lowrank
+ * Rows of a low-rank coupling (moscot PR #846, section Fix: for low-rank
+ * outputs the rows are (Q diag(1/g) R^T)[rows], a matrix product that never
+ * touches a geometry):
+ *     out[t*m + j] = sum_k Q[i*r + k] * R[j*r + k] / g[k],   i = row_idx[t].
+ *  Q [n,r], R [m,r], g [r]: device float32, row-major (g > 0); 1 <= r <= 128.
+ *  row_idx [k]: device int64 in [0, n); out [k,m]: device float32, row-major.
+ * Accumulated in float32 in k order: relative error <= r * 2^-24 for the
+ * nonnegative factors of a low-rank coupling. No plan, no allocation beyond a
+ * cached flag. A row index out of range returns OT_ERR_INVALID_ARG (checked on
+ * the device; that row is not written). Synchronises `stream`. */
+OT_API int ot_materialize_rows_lowrank(const float *Q, const float *R, const float *g, int64_t n,
+                                       int64_t m, int32_t r, const int64_t *row_idx, int64_t k,
+                                       float *out, void *stream);
+
+/* ------------------------------------------------- ot_materialize_rows_lrcost
+ * Entropic rows on a low-rank cost geometry (moscot PR #846, section Fix: the
+ * cost rows of an LRCGeometry are cost_1[rows] @ cost_2^T + bias):
+ *     C_ij = inv_scale_cost * (sum_k cost1[i*r + k] * cost2[j*r + k] + bias),
+ *     out[t*m + j] = exp((f_i + g_j - C_ij) / eps),   i = row_idx[t],
+ * with the caller's resolved inv_scale_cost and eps (a subset never
+ * re-derives them). cost1 [n,r], cost2 [m,r], f [n], g [m]: device float32;
+ * 1 <= r <= 128. The dot products and the exponent are assembled in float64
+ * (as ot_materialize_rows), the value rounded to float32; f_i or g_j = -inf
+ * gives 0. row_idx / out and errors as ot_materialize_rows_lowrank.
+ * Synchronises `stream`. */
+OT_API int ot_materialize_rows_lrcost(const float *cost1, const float *cost2, const float *f,
+                                      const float *g, int64_t n, int64_t m, int32_t r, double bias,
+                                      double inv_scale_cost, double eps, const int64_t *row_idx,
+                                      int64_t k, float *out, void *stream);
+
 /* ------------------------------------------------------ ot_sparsify_min_row
  * The exact min_row threshold (moscot PR #846, "Behavioural changes"):
  *     thr = min over rows with a_i > 0 of max_j T_ij,

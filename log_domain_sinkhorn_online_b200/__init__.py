@@ -121,6 +121,50 @@ class Plan:
         return dict(row_ptr=row_ptr, col_idx=col_idx[:nnz], vals=vals[:nnz], nnz=nnz, thr=thr)
 
 
+def _rows_out(row_idx, m, out, dev):
+    import torch
+    row_idx = _dev(row_idx, torch.int64, "row_idx")
+    if out is None:
+        out = torch.empty((row_idx.numel(), m), dtype=torch.float32, device=dev)
+    _dev(out, torch.float32, "out")
+    if out.shape != (row_idx.numel(), m):
+        raise ValueError("out must be [k, m]")
+    return row_idx, out
+
+
+def lowrank_rows(Q, R, g, row_idx, out=None, stream=None):
+    """Rows (Q diag(1/g) R^T)[row_idx] of a low-rank coupling; Q [n, r], R [m, r],
+    g [r] float32 CUDA tensors. Returns out [k, m] float32."""
+    import torch
+    Q, R, g = _dev(Q, torch.float32, "Q"), _dev(R, torch.float32, "R"), _dev(g, torch.float32, "g")
+    n, r = Q.shape
+    m = R.shape[0]
+    if R.shape[1] != r or g.numel() != r:
+        raise ValueError("Q [n, r], R [m, r] and g [r] must share r")
+    row_idx, out = _rows_out(row_idx, m, out, Q.device)
+    B.ot_materialize_rows_lowrank(Q.data_ptr(), R.data_ptr(), g.data_ptr(), n, m, r, row_idx.data_ptr(),
+                                  row_idx.numel(), out.data_ptr(), _stream(stream))
+    return out
+
+
+def lrcost_rows(cost1, cost2, f, g, row_idx, eps, inv_scale_cost=1.0, bias=0.0, out=None, stream=None):
+    """Entropic rows exp((f_i + g_j - c (cost1[i].cost2[j] + bias)) / eps) on a
+    low-rank cost geometry; cost1 [n, r], cost2 [m, r], f [n], g [m] float32
+    CUDA tensors. Returns out [k, m] float32."""
+    import torch
+    c1, c2 = _dev(cost1, torch.float32, "cost1"), _dev(cost2, torch.float32, "cost2")
+    f, g = _dev(f, torch.float32, "f"), _dev(g, torch.float32, "g")
+    n, r = c1.shape
+    m = c2.shape[0]
+    if c2.shape[1] != r or f.numel() != n or g.numel() != m:
+        raise ValueError("cost1 [n, r], cost2 [m, r], f [n], g [m]")
+    row_idx, out = _rows_out(row_idx, m, out, c1.device)
+    B.ot_materialize_rows_lrcost(c1.data_ptr(), c2.data_ptr(), f.data_ptr(), g.data_ptr(), n, m, r,
+                                 float(bias), float(inv_scale_cost), float(eps), row_idx.data_ptr(),
+                                 row_idx.numel(), out.data_ptr(), _stream(stream))
+    return out
+
+
 def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None, warm_start=False,
              check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,
              timing=False, col_splits=0, rows_per_thread=0, tensor_cores=True,

@@ -29,7 +29,8 @@ OT_SCALE_NONE, OT_SCALE_MEAN, OT_SCALE_MAX_COST, OT_SCALE_VALUE = 0, 1, 2, 3
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sinkhorn_pointcloud",
             "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy",
-            "ot_marginal_residual_noalloc", "ot_trim_cache", "ot_sparsify_csr")
+            "ot_marginal_residual_noalloc", "ot_trim_cache", "ot_sparsify_csr",
+            "ot_materialize_rows_lowrank", "ot_materialize_rows_lrcost")
 OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
@@ -88,6 +89,10 @@ def lib() -> ctypes.CDLL:
             L.ot_sparsify_min_row.restype = ctypes.c_int
             L.ot_sparsify_csr.argtypes = [P, I64, ctypes.c_float, P, P, P, I64, ctypes.POINTER(I64), P]
             L.ot_sparsify_csr.restype = ctypes.c_int
+            L.ot_materialize_rows_lowrank.argtypes = [P, P, P, I64, I64, I32, P, I64, P, P]
+            L.ot_materialize_rows_lowrank.restype = ctypes.c_int
+            L.ot_materialize_rows_lrcost.argtypes = [P, P, P, P, I64, I64, I32, D, D, D, P, I64, P, P]
+            L.ot_materialize_rows_lrcost.restype = ctypes.c_int
             L.ot_marginal_residual_noalloc.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D,
                                                        ctypes.POINTER(D), ctypes.POINTER(D), P]
             L.ot_marginal_residual_noalloc.restype = ctypes.c_int
@@ -141,6 +146,16 @@ def ot_marginal_residual(plan, stream):
 
 def ot_materialize_rows(plan, row_idx, k, out, stream) -> int:
     return _check(lib().ot_materialize_rows(plan, row_idx, k, out, stream))
+
+
+def ot_materialize_rows_lowrank(Q, R, g, n, m, r, row_idx, k, out, stream):
+    return _check(lib().ot_materialize_rows_lowrank(Q, R, g, n, m, r, row_idx, k, out, stream))
+
+
+def ot_materialize_rows_lrcost(cost1, cost2, f, g, n, m, r, bias, inv_scale_cost, eps, row_idx, k,
+                               out, stream):
+    return _check(lib().ot_materialize_rows_lrcost(cost1, cost2, f, g, n, m, r, bias, inv_scale_cost,
+                                                   eps, row_idx, k, out, stream))
 
 
 def ot_sparsify_csr(plan, block_rows, thr, row_ptr, col_idx, vals, capacity, stream):

@@ -855,6 +855,70 @@ extern "C" int ot_materialize_rows(const ot_plan *cplan, const int64_t *row_idx,
     return OT_OK;
 }
 
+namespace {
+
+// The two low-rank row flavours: no plan, the factors are the output's own.
+int lowrank_rows(int mode, const float *fa, const float *fb, const float *g, const float *f,
+                 const float *gp, int64_t n, int64_t m, int32_t r, double bias, double c, double eps,
+                 const int64_t *row_idx, int64_t k, float *out, void *stream) {
+    if (n < 1 || m < 1) return fail(OT_ERR_INVALID_ARG, "n and m must be >= 1");
+    if (r < 1 || r > kLrMaxRank) return fail(OT_ERR_UNSUPPORTED, "rank r must be in [1, %d]", kLrMaxRank);
+    if (k < 0) return fail(OT_ERR_INVALID_ARG, "k must be >= 0");
+    if (!fa || !fb || (mode == 0 ? !g : (!f || !gp)))
+        return fail(OT_ERR_INVALID_ARG, "null factor or potential pointer");
+    if (mode == 1 && (!(eps > 0.0) || !std::isfinite(eps) || !std::isfinite(c) || !std::isfinite(bias)))
+        return fail(OT_ERR_INVALID_ARG, "eps must be > 0 and eps, inv_scale_cost, bias finite");
+    if (k == 0) return OT_OK;
+    if (!row_idx || !out) return fail(OT_ERR_INVALID_ARG, "null row_idx or out");
+    if (k > INT64_MAX / m) return fail(OT_ERR_OVERFLOW, "k*m overflows int64");
+    int dev = 0, sms = 0;
+    int rc = check_device(&dev, &sms);
+    if (rc != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    int *flag = nullptr, *hflag = nullptr;
+    size_t got = 0;
+    OT_CU(pool_device_alloc(reinterpret_cast<void **>(&flag), 256, &got));
+    if (pool_host_alloc(reinterpret_cast<void **>(&hflag), sizeof(int)) != cudaSuccess) {
+        pool_device_free(flag, got);
+        return fail(OT_ERR_OOM, "pinned host allocation failed");
+    }
+    LrArgs L{};
+    L.fa = fa; L.fb = fb; L.g = g; L.f = f; L.gp = gp;
+    L.n = n; L.m = m; L.k = k; L.r = r; L.row_idx = row_idx;
+    const double kappa = 1.4426950408889634 / eps;  // log2(e) / eps
+    L.bias = bias; L.kappa = kappa; L.kc = kappa * c;
+    L.out = out;
+    L.vec = (m % 4 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
+    L.bad = flag;
+    cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = launch_lowrank_rows(mode, L, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(hflag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    const int bad = e == cudaSuccess ? *hflag : 0;
+    pool_host_free(hflag, sizeof(int));
+    pool_device_free(flag, got);
+    if (e != cudaSuccess) return fail(OT_ERR_CUDA, "low-rank rows: %s", cudaGetErrorString(e));
+    if (bad) return fail(OT_ERR_INVALID_ARG, "a row index is outside [0, n)");
+    return OT_OK;
+}
+
+}  // namespace
+
+extern "C" int ot_materialize_rows_lowrank(const float *Q, const float *R, const float *g, int64_t n,
+                                           int64_t m, int32_t r, const int64_t *row_idx, int64_t k,
+                                           float *out, void *stream) {
+    return lowrank_rows(0, Q, R, g, nullptr, nullptr, n, m, r, 0.0, 1.0, 1.0, row_idx, k, out, stream);
+}
+
+extern "C" int ot_materialize_rows_lrcost(const float *cost1, const float *cost2, const float *f,
+                                          const float *g, int64_t n, int64_t m, int32_t r,
+                                          double bias, double inv_scale_cost, double eps,
+                                          const int64_t *row_idx, int64_t k, float *out,
+                                          void *stream) {
+    return lowrank_rows(1, cost1, cost2, nullptr, f, g, n, m, r, bias, inv_scale_cost, eps, row_idx, k,
+                        out, stream);
+}
+
 extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, float *thr_out,
                                    int64_t *row_counts, int64_t *nnz_out,
                                    int64_t *n_massless_out, int64_t *argmin_out, void *stream) {

@@ -80,6 +80,21 @@ struct RowPassArgs {
     int64_t *counts;
     double *part;
 };
+struct LrArgs {
+    const float *fa, *fb;       // row factors [n, r] and column factors [m, r]
+    const float *g;             // coupling: the middle diagonal [r]
+    const float *f, *gp;        // cost: potentials [n], [m]
+    int64_t n, m, k;
+    int r;
+    const int64_t *row_idx;
+    double bias, kc, kappa;     // cost: bias, kappa * inv_scale_cost, kappa = log2(e) / eps
+    float *out;
+    int vec;
+    int *bad;
+};
+constexpr int kLrMaxRank = 128;
+size_t lowrank_smem_bytes(int mode, int r);
+cudaError_t launch_lowrank_rows(int mode, const LrArgs &L, cudaStream_t s);
 struct CsrArgs {
     const float *pts, *pot, *w;
     const double *dcol, *o;

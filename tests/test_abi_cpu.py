@@ -97,6 +97,20 @@ def test_row_calls_reject_null_plan(B):
     L.ot_plan_destroy(None)  # no-op
 
 
+def test_lowrank_rows_validate_on_the_host(B):
+    L = B.lib()
+    # rank outside [1, 128] is unsupported, bad sizes / eps are invalid, k = 0 is a no-op
+    assert L.ot_materialize_rows_lowrank(FAKE, FAKE, FAKE, 4, 5, 0, FAKE, 1, FAKE, None) == -6
+    assert L.ot_materialize_rows_lowrank(FAKE, FAKE, FAKE, 4, 5, 129, FAKE, 1, FAKE, None) == -6
+    assert L.ot_materialize_rows_lowrank(FAKE, FAKE, FAKE, 0, 5, 3, FAKE, 1, FAKE, None) == -1
+    assert L.ot_materialize_rows_lowrank(None, FAKE, FAKE, 4, 5, 3, FAKE, 1, FAKE, None) == -1
+    assert L.ot_materialize_rows_lowrank(FAKE, FAKE, FAKE, 4, 5, 3, FAKE, 0, FAKE, None) == 0
+    assert L.ot_materialize_rows_lrcost(FAKE, FAKE, FAKE, FAKE, 4, 5, 3, 0.0, 1.0, 0.0, FAKE, 1, FAKE,
+                                        None) == -1
+    assert L.ot_materialize_rows_lrcost(FAKE, FAKE, None, FAKE, 4, 5, 3, 0.0, 1.0, 0.1, FAKE, 1, FAKE,
+                                        None) == -1
+
+
 def test_valid_call_without_gpu_fails_loudly(B):
     import torch
     if torch.cuda.is_available():

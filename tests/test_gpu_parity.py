@@ -260,6 +260,78 @@ def test_sparsify_csr_generic_d(ot, orc):
     plan.close()
 
 
+@pytest.mark.parametrize("r", [1, 7, 32, 128])
+def test_lowrank_coupling_rows_match_oracle(ot, orc, r):
+    """(Q diag(1/g) R^T)[rows] against the oracle: nonnegative factors, a ragged
+    column count, unsorted and repeated rows, rows past one launch tile."""
+    import torch
+    rng = np.random.default_rng(70 + r)
+    n, m = 203, 1031
+    Q = rng.random((n, r)).astype(np.float32)
+    R = rng.random((m, r)).astype(np.float32)
+    g = (rng.random(r) + 0.2).astype(np.float32)
+    rows = np.concatenate([rng.integers(0, n, 90), [0, n - 1, 5, 5]]).astype(np.int64)
+    got = ot.lowrank_rows(*(torch.from_numpy(v).cuda() for v in (Q, R, g, rows))).double().cpu().numpy()
+    H.assert_entries(got, orc.lr_rows(Q, R, g, rows))
+
+
+@pytest.mark.parametrize("r", [2, 16, 128])
+def test_lowrank_cost_rows_match_oracle(ot, orc, r):
+    """Entropic rows on a low-rank cost (signed factors, a bias, a massless row)
+    against the oracle, float64 exponent like the point-cloud rows."""
+    import torch
+    rng = np.random.default_rng(90 + r)
+    n, m = 150, 517
+    c1 = (rng.standard_normal((n, r)) / np.sqrt(r)).astype(np.float32)
+    c2 = (rng.standard_normal((m, r)) / np.sqrt(r)).astype(np.float32)
+    f = rng.normal(0, 0.05, n).astype(np.float32)
+    g = rng.normal(0, 0.05, m).astype(np.float32)
+    f[7] = -np.inf
+    rows = rng.integers(0, n, 70).astype(np.int64)
+    rows[3] = 7
+    eps, c, bias = 0.05, 0.8, 0.3
+    dev = [torch.from_numpy(v).cuda() for v in (c1, c2, f, g, rows)]
+    got = ot.lrcost_rows(*dev[:4], dev[4], eps=eps, inv_scale_cost=c, bias=bias).double().cpu().numpy()
+    ref = orc.lrc_rows(c1, c2, f, g, bias, c, eps, rows)
+    assert np.all(got[3] == 0.0)
+    H.assert_entries(got, ref)
+
+
+def test_lowrank_cost_rows_reproduce_point_cloud_rows(ot):
+    """Squared Euclidean as a low-rank cost, [|x|^2, 1, -2x] . [1, |y|^2, y]: the
+    low-rank-cost rows at a solved plan's potentials are that plan's rows."""
+    import torch
+    w = _cloud(71, 600, 450, 3, scale="mean", eps=0.05)
+    x, y, a, b = H.to_dev(w)
+    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=30)
+    xd, yd = w.x.astype(np.float64), w.y.astype(np.float64)
+    c1 = np.concatenate([(xd ** 2).sum(1, keepdims=True), np.ones((600, 1)), -2 * xd], 1).astype(np.float32)
+    c2 = np.concatenate([np.ones((450, 1)), (yd ** 2).sum(1, keepdims=True), yd], 1).astype(np.float32)
+    rows = torch.arange(0, 600, 7, device="cuda")
+    want = plan.materialize_rows(rows).double().cpu().numpy()
+    got = ot.lrcost_rows(torch.from_numpy(c1).cuda(), torch.from_numpy(c2).cuda(), plan.f, plan.g, rows,
+                         eps=w.eps, inv_scale_cost=plan.info.inv_scale_cost).double().cpu().numpy()
+    # the factors round |x|^2 and |y|^2 to float32: ~1e-7 of the cost, scaled by c / eps
+    H.assert_entries(got, want, tol=2e-5)
+    plan.close()
+
+
+def test_lowrank_rows_report_bad_rows_and_rank(ot):
+    import torch
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    Q = torch.rand(10, 4, device="cuda")
+    R = torch.rand(12, 4, device="cuda")
+    g = torch.rand(4, device="cuda") + 0.5
+    with pytest.raises(B.OTError) as e:
+        ot.lowrank_rows(Q, R, g, torch.tensor([0, 10], device="cuda"))
+    assert e.value.status == B.OT_ERR_INVALID_ARG
+    big = torch.rand(10, 129, device="cuda")
+    with pytest.raises(B.OTError) as e:
+        ot.lowrank_rows(big, torch.rand(12, 129, device="cuda"), torch.rand(129, device="cuda") + 0.5,
+                        torch.tensor([0], device="cuda"))
+    assert e.value.status == B.OT_ERR_UNSUPPORTED
+
+
 def test_bad_row_index_is_reported(ot):
     import torch
     w = _cloud(3, 300, 200, 2)
