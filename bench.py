@@ -59,6 +59,9 @@ def _args():
     ap.add_argument("--n", type=int, default=None, help="replica size of the workload (rows)")
     ap.add_argument("--m", type=int, default=None, help="replica size of the workload (columns)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lowrank", type=int, default=0, metavar="R",
+                    help="instead of the step: time the two low-rank row materializers at rank R "
+                         "(4096 rows x 100000 columns) and print their own JSON line")
     ap.add_argument("--no-large-n", action="store_true",
                     help="skip the d = 3 half-step measurement at n = m = 1e5")
     ap.add_argument("--clock-ms", type=int, default=200,
@@ -283,6 +286,42 @@ def _large_n(ot, dev, n=100_000, iters=5):
             "per_launch_us": us, "achieved": float(n) * n / (us / 1e6) / 1e12, "unit": "Tex2/s"}
 
 
+def run_lowrank(args, k=4096, m=100_000, n=20_000, reps=5):
+    """Write bandwidth of the low-rank row materializers (coupling rows and
+    entropic rows on a low-rank cost), k rows x m columns at rank args.lowrank,
+    seeded nonnegative factors; CUDA events over `reps` calls after a warm-up."""
+    import torch
+    import log_domain_sinkhorn_online_b200 as ot
+    dev = torch.device("cuda", 0)
+    r = args.lowrank
+    gen = torch.Generator(device=dev).manual_seed(7)
+    Q = torch.rand(n, r, device=dev, generator=gen)
+    R = torch.rand(m, r, device=dev, generator=gen)
+    g = torch.rand(r, device=dev, generator=gen) + 0.5
+    f = torch.rand(n, device=dev, generator=gen) * 0.01
+    gp = torch.rand(m, device=dev, generator=gen) * 0.01
+    rows = torch.randint(0, n, (k,), device=dev, generator=gen)
+    out = torch.empty((k, m), dtype=torch.float32, device=dev)
+    peaks, kind = _peaks()
+    line = {"metric": "low-rank row materializer write bandwidth", "unit": "GB/s", "rank": r,
+            "config": {"rows": k, "cols": m, "n": n, "factors": "seeded uniform [0, 1)"},
+            "peak_gbs": float(peaks["hbm_gbs"]), "peak_note": f"{kind} copy bandwidth"}
+    for name, call in (("coupling", lambda: ot.lowrank_rows(Q, R, g, rows, out=out)),
+                       ("cost", lambda: ot.lrcost_rows(Q, R, f, gp, rows, eps=0.05, bias=0.1, out=out))):
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        gbs = k * m * 4 / (ms / 1e3) / 1e9
+        line[name] = {"ms": ms, "gbs": gbs, "frac": gbs / float(peaks["hbm_gbs"])}
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
     import torch
     import log_domain_sinkhorn_online_b200 as ot
@@ -395,6 +434,8 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.lowrank:
+        run_lowrank(args)
     else:
         run_ours(args)
 

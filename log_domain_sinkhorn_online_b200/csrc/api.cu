@@ -12,6 +12,7 @@
 #include <cstring>
 #include <algorithm>
 #include <new>
+#include <atomic>
 #include <vector>
 
 #include "ot_sinkhorn.h"
@@ -423,14 +424,28 @@ int run_iterations(ot_plan *p, int parity0, int iters, bool check, bool use_grap
     return OT_OK;
 }
 
+// The current device must be sm_100; its SM count is cached per device (two
+// attribute queries the first time: a full property query costs milliseconds,
+// which every call would otherwise spend before its first launch).
 int check_device(int *dev, int *sms) {
+    static std::atomic<int> cached_sms[64];  // 0: not queried yet
     OT_CU(cudaGetDevice(dev));
-    cudaDeviceProp prop;
-    OT_CU(cudaGetDeviceProperties(&prop, *dev));
-    if (prop.major != 10)
-        return fail(OT_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a", *dev,
-                    prop.major, prop.minor);
-    *sms = prop.multiProcessorCount;
+    if (*dev >= 0 && *dev < 64) {
+        const int c = cached_sms[*dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *sms = c;
+            return OT_OK;
+        }
+    }
+    int major = 0, minor = 0, count = 0;
+    OT_CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev));
+    OT_CU(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev));
+    if (major != 10)
+        return fail(OT_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a", *dev, major,
+                    minor);
+    OT_CU(cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, *dev));
+    if (*dev >= 0 && *dev < 64) cached_sms[*dev].store(count, std::memory_order_relaxed);
+    *sms = count;
     return OT_OK;
 }
 

@@ -247,14 +247,15 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
 // Two more row flavours (moscot PR #846, "Fix"), both a small matrix product:
 //   MODE 0, low-rank coupling:  out[t, j] = sum_k Q[i,k] R[j,k] / g[k]
 //   MODE 1, low-rank cost:      out[t, j] = exp((f_i + g_j - c (cost1[i].cost2[j] + bias)) / eps)
-// with i = row_idx[t]. A block computes 64 rows x 128 columns; its 256 threads
-// are 8 row groups x 32 column groups and each owns 8 rows x 4 columns; both
-// factor blocks sit K-major in shared memory (rows read as broadcasts, columns
-// as one 16-byte load per thread and k). The coupling accumulates in float32
+// with i = row_idx[t]. A block owns 128 columns and up to 512 rows of the row
+// list: it stages its columns' factors once, then walks 64-row tiles; its 256
+// threads are 8 row groups x 32 column groups and each owns 8 rows x 4 columns
+// of a tile; both factor blocks sit K-major in shared memory (rows read as
+// broadcasts, columns as one 16-byte load per thread and k). The coupling accumulates in float32
 // (its factors are nonnegative: relative error <= r 2^-24); the cost
 // accumulates its dot products in float64 and assembles the exponent like the
 // point-cloud rows (exp2_split).
-constexpr int kLrRows = 64, kLrCols = 128, kLrThreads = 256;
+constexpr int kLrRows = 64, kLrCols = 128, kLrThreads = 256, kLrRowsPerBlock = 512;
 
 template <typename T, int MODE>
 __global__ void __launch_bounds__(kLrThreads) lowrank_rows_kernel(LrArgs L) {
@@ -262,76 +263,81 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_rows_kernel(LrArgs L) {
     T *sR = reinterpret_cast<T *>(lr_smem);    // [r][kLrRows]
     T *sC = sR + (size_t)L.r * kLrRows;         // [r][kLrCols]
     const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5;
-    const int64_t t0 = (int64_t)blockIdx.y * kLrRows;
     const int64_t j0 = (int64_t)blockIdx.x * kLrCols;
-    // row factors (a row list entry outside [0, n) is reported and yields no row)
-    for (int e = tid; e < L.r * kLrRows; e += kLrThreads) {
-        const int rr = e / L.r, q = e % L.r;  // consecutive threads: consecutive k of one row
-        const int64_t t = t0 + rr;
-        T v = (T)0;
-        if (t < L.k) {
-            const int64_t i = L.row_idx[t];
-            if (i >= 0 && i < L.n) {
-                v = (T)L.fa[i * L.r + q];
-                if (MODE == 0) v = v / (T)L.g[q];
-            } else if (q == 0) {
-                atomicExch(L.bad, 1);
-            }
-        }
-        sR[q * kLrRows + rr] = v;
-    }
+    // this block's columns, once
     for (int e = tid; e < L.r * kLrCols; e += kLrThreads) {
-        const int cc = e / L.r, q = e % L.r;
+        const int cc = e / L.r, q = e % L.r;  // consecutive threads: consecutive k of one column
         const int64_t j = j0 + cc;
         sC[q * kLrCols + cc] = j < L.m ? (T)L.fb[j * L.r + q] : (T)0;
     }
-    __syncthreads();
-    T acc[8][4];
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = (T)0;
-    for (int q = 0; q < L.r; ++q) {
-        T av[8], bv[4];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) av[a] = sR[q * kLrRows + rg * 8 + a];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) bv[b] = sC[q * kLrCols + cg * 4 + b];
+    const int64_t tb = (int64_t)blockIdx.y * kLrRowsPerBlock;
+    const int64_t te = min(tb + kLrRowsPerBlock, L.k);
+    const int64_t jb = j0 + cg * 4;
+    for (int64_t t0 = tb; t0 < te; t0 += kLrRows) {
+        __syncthreads();  // the previous tile's row factors are no longer read
+        // row factors (a row list entry outside [0, n) is reported and yields no row)
+        for (int e = tid; e < L.r * kLrRows; e += kLrThreads) {
+            const int rr = e / L.r, q = e % L.r;
+            const int64_t t = t0 + rr;
+            T v = (T)0;
+            if (t < te) {
+                const int64_t i = L.row_idx[t];
+                if (i >= 0 && i < L.n) {
+                    v = (T)L.fa[i * L.r + q];
+                    if (MODE == 0) v = v / (T)L.g[q];
+                } else if (q == 0) {
+                    atomicExch(L.bad, 1);
+                }
+            }
+            sR[q * kLrRows + rr] = v;
+        }
+        __syncthreads();
+        T acc[8][4];
 #pragma unroll
         for (int a = 0; a < 8; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
-    }
-    const int64_t jb = j0 + cg * 4;
+            for (int b = 0; b < 4; ++b) acc[a][b] = (T)0;
+        for (int q = 0; q < L.r; ++q) {
+            T av[8], bv[4];
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-        const int64_t t = t0 + rg * 8 + a;
-        if (t >= L.k) break;
-        const int64_t i = L.row_idx[t];
-        if (i < 0 || i >= L.n) continue;
-        float o[4];
-        double Ai = 0.0;
-        if (MODE == 1) {
-            const float fv = L.f[i];
-            Ai = fv == -INFINITY ? -1e15 : L.kappa * (double)fv;
+            for (int a = 0; a < 8; ++a) av[a] = sR[q * kLrRows + rg * 8 + a];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) bv[b] = sC[q * kLrCols + cg * 4 + b];
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
         }
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            if (MODE == 0) {
-                o[b] = (float)acc[a][b];
-            } else {
-                const int64_t j = jb + b < L.m ? jb + b : L.m - 1;
-                const float gv = L.gp[j];
-                const double Bj = gv == -INFINITY ? -1e15 : L.kappa * (double)gv;
-                const double e2 = Ai + Bj - L.kc * ((double)acc[a][b] + L.bias);
-                o[b] = exp2_split(fmin(fmax(e2, -1e15), 1e15));
+        for (int a = 0; a < 8; ++a) {
+            const int64_t t = t0 + rg * 8 + a;
+            if (t >= te) break;
+            const int64_t i = L.row_idx[t];
+            if (i < 0 || i >= L.n) continue;
+            float o[4];
+            double Ai = 0.0;
+            if (MODE == 1) {
+                const float fv = L.f[i];
+                Ai = fv == -INFINITY ? -1e15 : L.kappa * (double)fv;
             }
-        }
-        float *dst = L.out + t * L.m + jb;
-        if (L.vec && jb + 4 <= L.m) {
-            __stcs(reinterpret_cast<float4 *>(dst), make_float4(o[0], o[1], o[2], o[3]));
-        } else {
-            for (int b = 0; b < 4 && jb + b < L.m; ++b) __stcs(dst + b, o[b]);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                if (MODE == 0) {
+                    o[b] = (float)acc[a][b];
+                } else {
+                    const int64_t j = jb + b < L.m ? jb + b : L.m - 1;
+                    const float gv = L.gp[j];
+                    const double Bj = gv == -INFINITY ? -1e15 : L.kappa * (double)gv;
+                    const double e2 = Ai + Bj - L.kc * ((double)acc[a][b] + L.bias);
+                    o[b] = exp2_split(fmin(fmax(e2, -1e15), 1e15));
+                }
+            }
+            float *dst = L.out + t * L.m + jb;
+            if (L.vec && jb + 4 <= L.m) {
+                __stcs(reinterpret_cast<float4 *>(dst), make_float4(o[0], o[1], o[2], o[3]));
+            } else {
+                for (int b = 0; b < 4 && jb + b < L.m; ++b) __stcs(dst + b, o[b]);
+            }
         }
     }
 }
@@ -348,12 +354,13 @@ cudaError_t launch_lowrank_rows(int mode, const LrArgs &L, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t max_y = 65535;
-    for (int64_t r0 = 0; r0 < L.k; r0 += max_y * kLrRows) {
+    for (int64_t r0 = 0; r0 < L.k; r0 += max_y * kLrRowsPerBlock) {
         LrArgs A = L;
         A.row_idx = L.row_idx + r0;
         A.out = L.out + r0 * L.m;
-        A.k = std::min<int64_t>(max_y * kLrRows, L.k - r0);
-        dim3 grid((unsigned)((L.m + kLrCols - 1) / kLrCols), (unsigned)((A.k + kLrRows - 1) / kLrRows));
+        A.k = std::min<int64_t>(max_y * kLrRowsPerBlock, L.k - r0);
+        dim3 grid((unsigned)((L.m + kLrCols - 1) / kLrCols),
+                  (unsigned)((A.k + kLrRowsPerBlock - 1) / kLrRowsPerBlock));
         if (mode == 0) lowrank_rows_kernel<float, 0><<<grid, kLrThreads, smem, s>>>(A);
         else lowrank_rows_kernel<double, 1><<<grid, kLrThreads, smem, s>>>(A);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
