@@ -69,6 +69,18 @@ def _load():
             lib.orc_lr_rows.argtypes = [P, P, P, I64, I64, I32, P, I64, P]
             lib.orc_lrc_rows.argtypes = [P, P, P, P, I64, I64, I32, D, D, D, P, I64, P]
             lib.orc_sparsify_csr.restype = I64
+            lib.orc_morton_codes.argtypes = [P, I64, I32, P, P, P]
+            lib.orc_morton_order.argtypes = [P, I64, I32, P, P, P]
+            lib.orc_block_mask.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D, I64, D, I32,
+                                           P, P, P, P, P]
+            lib.orc_block_mask.restype = I64
+            lib.orc_sparse_f_step.argtypes = [P, P, P, P, I64, I64, I32, D, D, I64, P, P]
+            lib.orc_sparse_g_step.argtypes = [P, P, P, P, I64, I64, I32, D, D, I64, P, P]
+            lib.orc_sparse_row_residual.argtypes = [P, P, P, P, P, I64, I64, I32, D, D, I64, P]
+            lib.orc_sparse_row_residual.restype = D
+            lib.orc_sinkhorn_sparse.argtypes = [P, P, P, P, I64, I64, I32, D, D, I32, D, I64, D,
+                                                I32, D, P, P, P, P]
+            lib.orc_sinkhorn_sparse.restype = I32
             _lib = lib
     return _lib
 
@@ -280,3 +292,113 @@ def min_row(x, y, a, f, g, c, eps, block_rows=0):
                              _ptr(counts), ctypes.byref(nnz))
     return dict(thr=float(thr.value), argmin=int(arg.value), counts=counts,
                 nnz=int(nnz.value), n_massless=int(nm))
+
+
+# ------------------------------------------------------- block-sparse updates
+# "FlashSinkhorn 2: Block-Sparse Entropic Optimal Transport", sections 3, 3.2,
+# A.3, B.1 and B.3; the readings are spelled out in sinkhorn_oracle.c.
+
+def joint_box(x, y):
+    """(lo, hi) per coordinate over both clouds, float64."""
+    x, y, n, m, d = _pts(x, y)
+    both = np.concatenate([x, y]).astype(np.float64)
+    return both.min(0), both.max(0)
+
+
+def morton_codes(x, lo, hi):
+    """Morton codes (bits = 30/d per coordinate over the box [lo, hi])."""
+    x = _f32(x)
+    if x.ndim == 1:
+        x = x[:, None]
+    n, d = x.shape
+    lo, hi = _f64(lo), _f64(hi)
+    out = np.empty(n, dtype=np.uint64)
+    _load().orc_morton_codes(_ptr(x), n, d, _ptr(lo), _ptr(hi), _ptr(out))
+    return out
+
+
+def morton_order(x, lo, hi):
+    """perm with x[perm] in Morton order, ties by index (section 3)."""
+    x = _f32(x)
+    if x.ndim == 1:
+        x = x[:, None]
+    n, d = x.shape
+    lo, hi = _f64(lo), _f64(hi)
+    perm = np.empty(n, dtype=np.int64)
+    _load().orc_morton_order(_ptr(x), n, d, _ptr(lo), _ptr(hi), _ptr(perm))
+    return perm
+
+
+def block_mask(x, y, a, b, f, g, c, eps, B, delta, verify=True):
+    """Block-pair mask at (f, g) for points already in block order.
+
+    Returns dict(cand, adm: [NB, MB] bool, screen_margin, mass_margin: [NB, MB]
+    natural-log margins over the threshold, n_cand, n_adm).
+    """
+    x, y, n, m, d = _pts(x, y)
+    a, b, f, g = _f64(a), _f64(b), _f64(f), _f64(g)
+    NB, MB = -(-n // B), -(-m // B)
+    cand = np.empty((NB, MB), dtype=np.uint8)
+    adm = np.empty((NB, MB), dtype=np.uint8)
+    sm = np.empty((NB, MB))
+    mm = np.empty((NB, MB))
+    nc = ctypes.c_int64()
+    na = _load().orc_block_mask(_ptr(x), _ptr(y), _ptr(a), _ptr(b), _ptr(f), _ptr(g), n, m, d,
+                                float(c), float(eps), int(B), float(delta), int(bool(verify)),
+                                _ptr(cand), _ptr(adm), _ptr(sm), _ptr(mm), ctypes.byref(nc))
+    return dict(cand=cand.astype(bool), adm=adm.astype(bool), screen_margin=sm,
+                mass_margin=mm, n_cand=int(nc.value), n_adm=int(na))
+
+
+def sparse_f_step(x, y, a, g, c, eps, B, adm):
+    """f-update over the admitted tiles of each row block (all columns for a
+    block without one), points in block order."""
+    x, y, n, m, d = _pts(x, y)
+    a, g = _f64(a), _f64(g)
+    adm = np.ascontiguousarray(adm, dtype=np.uint8)
+    out = np.empty(n)
+    _load().orc_sparse_f_step(_ptr(x), _ptr(y), _ptr(a), _ptr(g), n, m, d, float(c), float(eps),
+                              int(B), _ptr(adm), _ptr(out))
+    return out
+
+
+def sparse_g_step(x, y, b, f, c, eps, B, adm):
+    """g-update over the admitted tiles of each column block (the mask read by columns)."""
+    x, y, n, m, d = _pts(x, y)
+    b, f = _f64(b), _f64(f)
+    adm = np.ascontiguousarray(adm, dtype=np.uint8)
+    out = np.empty(m)
+    _load().orc_sparse_g_step(_ptr(x), _ptr(y), _ptr(b), _ptr(f), n, m, d, float(c), float(eps),
+                              int(B), _ptr(adm), _ptr(out))
+    return out
+
+
+def sparse_row_residual(x, y, a, f, g, c, eps, B, adm):
+    """sum_i |sum over admitted j of T_ij - a_i| (the stop test of a sparse iteration)."""
+    x, y, n, m, d = _pts(x, y)
+    a, f, g = _f64(a), _f64(f), _f64(g)
+    adm = np.ascontiguousarray(adm, dtype=np.uint8)
+    return float(_load().orc_sparse_row_residual(_ptr(x), _ptr(y), _ptr(a), _ptr(f), _ptr(g), n,
+                                                 m, d, float(c), float(eps), int(B), _ptr(adm)))
+
+
+def sinkhorn_sparse(x, y, a, b, c, eps, n_iters, tol=0.0, B=128, delta=0.0, verify=True,
+                    dense_frac=0.5, f0=None, g0=None):
+    """Block-sparse fine iterations in Morton order, potentials in the caller's order.
+
+    Returns (f, g, iterations, residual, stats) with stats = (sparse
+    iterations, dense iterations, candidates, admitted tiles of the last mask).
+    """
+    x, y, n, m, d = _pts(x, y)
+    a, b = _f64(a), _f64(b)
+    f = np.zeros(n) if f0 is None else _f64(f0).copy()
+    g = np.zeros(m) if g0 is None else _f64(g0).copy()
+    r = ctypes.c_double(0.0)
+    st = np.zeros(4, dtype=np.int64)
+    it = _load().orc_sinkhorn_sparse(_ptr(x), _ptr(y), _ptr(a), _ptr(b), n, m, d, float(c),
+                                     float(eps), int(n_iters), float(tol), int(B), float(delta),
+                                     int(bool(verify)), float(dense_frac), _ptr(f), _ptr(g),
+                                     ctypes.byref(r), _ptr(st))
+    if it < 0:
+        raise ValueError("bad arguments (block size, sizes, or delta <= 0 with tol <= 0)")
+    return f, g, int(it), float(r.value), tuple(int(v) for v in st)

@@ -420,3 +420,362 @@ int64_t orc_sparsify_csr(const float *x, const float *y, const double *a, const 
     }
     return row_ptr[n];
 }
+
+/* ------------------------------------------------- block-sparse updates --
+ * "FlashSinkhorn 2: Block-Sparse Entropic Optimal Transport", sections 3,
+ * 3.2, A.3, B.1 and B.3: points in Morton order, blocks of B consecutive
+ * points, a block-pair screen from block potential maxima and bounding boxes,
+ * verification of the surviving pairs by their exact mass over the B x B
+ * point pairs, and half-steps that reduce only over the admitted tiles (a
+ * block with no admitted tile reduces over everything).
+ *
+ * Readings (the pages state the rules in words, not formulas):
+ *  - Morton code: every coordinate is quantised over the joint bounding box
+ *    of both clouds (lo_k = min, hi_k = max over all points) into 2^bits
+ *    cells, bits = 30/d (d = 1, 2, 3: 30, 15, 10):
+ *        q_k = floor((v_k - lo_k) * (2^bits / (hi_k - lo_k))), clamped to
+ *        [0, 2^bits - 1] (q_k = 0 when hi_k == lo_k);
+ *    bit t of q_k is bit t*d + (d-1-k) of the code (coordinate 0 the most
+ *    significant of each group); points are ordered by (code, index).
+ *  - Tile mass M_pq = sum over i in I_p, j in J_q of exp((f_i + g_j - C_ij)/eps).
+ *    Screen bound: C_ij >= c D_pq with D_pq the squared distance between the
+ *    two blocks' bounding boxes, f_i <= F_p = max over I_p, g_j <= G_q, so
+ *        M_pq <= U_pq = |I_p| |J_q| exp((F_p + G_q - c D_pq)/eps).
+ *  - Threshold (the mass-dependent rule of A.3): rho_pq = delta * min(amin_p,
+ *    bmin_q), amin_p the smallest nonzero a_i of block p. A tile is a
+ *    candidate when U_pq > rho_pq and admitted when it is a candidate and
+ *    (with verification) M_pq > rho_pq, so an omitted tile adds at most
+ *    delta a_i to row i and delta b_j to column j. delta defaults to
+ *    tol / (4 max(NB, MB)) (section 3.2): at most tol/4 of the mass is
+ *    omitted over all rows when the weights sum to one.
+ *  - A fine iteration builds the mask at the current (f, g) and runs the f-
+ *    and the g-update on it (the g-update reads it transposed). The stop test
+ *    takes the admitted plan's row residual at the state the mask was built
+ *    at and compares it with tol - MB delta sum(a), so that the full residual
+ *    (admitted plus omitted) is at most tol.
+ *  - An iteration whose candidate count exceeds dense_frac * NB * MB runs the
+ *    dense updates instead (sparse updates pay only when the admitted tiles
+ *    are well below all block pairs); its residual is then the full one.
+ */
+void orc_morton_codes(const float *x, int64_t n, int d, const double *lo, const double *hi,
+                      uint64_t *code) {
+    const int bits = 30 / d;
+    const double cells = (double)((int64_t)1 << bits);
+    for (int64_t i = 0; i < n; ++i) {
+        uint64_t cd = 0;
+        for (int k = 0; k < d; ++k) {
+            int64_t q = 0;
+            if (hi[k] > lo[k]) {
+                const double s = cells / (hi[k] - lo[k]);
+                const double t = floor(((double)x[i * d + k] - lo[k]) * s);
+                q = t < 0.0 ? 0 : t > cells - 1.0 ? (int64_t)cells - 1 : (int64_t)t;
+            }
+            for (int t = 0; t < bits; ++t)
+                if ((q >> t) & 1) cd |= (uint64_t)1 << (t * d + (d - 1 - k));
+        }
+        code[i] = cd;
+    }
+}
+
+typedef struct {
+    uint64_t code;
+    int64_t idx;
+} morton_key;
+
+static int morton_cmp(const void *p, const void *q) {
+    const morton_key *u = (const morton_key *)p, *v = (const morton_key *)q;
+    if (u->code != v->code) return u->code < v->code ? -1 : 1;
+    return u->idx < v->idx ? -1 : u->idx > v->idx ? 1 : 0;
+}
+
+/* perm[r] = index of the r-th point in Morton order */
+void orc_morton_order(const float *x, int64_t n, int d, const double *lo, const double *hi,
+                      int64_t *perm) {
+    uint64_t *code = (uint64_t *)malloc((size_t)(n > 0 ? n : 1) * sizeof(uint64_t));
+    morton_key *key = (morton_key *)malloc((size_t)(n > 0 ? n : 1) * sizeof(morton_key));
+    orc_morton_codes(x, n, d, lo, hi, code);
+    for (int64_t i = 0; i < n; ++i) {
+        key[i].code = code[i];
+        key[i].idx = i;
+    }
+    qsort(key, (size_t)n, sizeof(morton_key), morton_cmp);
+    for (int64_t r = 0; r < n; ++r) perm[r] = key[r].idx;
+    free(code);
+    free(key);
+}
+
+/* per block: potential maximum, smallest nonzero weight, bounding box */
+static void block_summary(const float *x, const double *w, const double *pot, int64_t cnt,
+                          int d, int64_t B, int64_t p, double *pmax, double *wmin, double *lo,
+                          double *hi) {
+    const int64_t i0 = p * B, i1 = (p + 1) * B < cnt ? (p + 1) * B : cnt;
+    *pmax = -INFINITY;
+    *wmin = INFINITY;
+    for (int k = 0; k < d; ++k) {
+        lo[k] = INFINITY;
+        hi[k] = -INFINITY;
+    }
+    for (int64_t i = i0; i < i1; ++i) {
+        if (pot[i] > *pmax) *pmax = pot[i];
+        if (w[i] > 0.0 && w[i] < *wmin) *wmin = w[i];
+        for (int k = 0; k < d; ++k) {
+            const double v = (double)x[i * d + k];
+            if (v < lo[k]) lo[k] = v;
+            if (v > hi[k]) hi[k] = v;
+        }
+    }
+}
+
+/* The block-pair mask at (f, g). x, y, a, b, f, g in Morton order. cand and
+ * adm: [NB * MB] bytes, 1 for a candidate / admitted tile. Optional outputs:
+ * screen_margin[pq] = ln U_pq - ln rho_pq and mass_margin[pq] = ln M_pq -
+ * ln rho_pq (NAN where not evaluated), n_cand. Returns the admitted count. */
+int64_t orc_block_mask(const float *x, const float *y, const double *a, const double *b,
+                       const double *f, const double *g, int64_t n, int64_t m, int d,
+                       double c, double eps, int64_t B, double delta, int verify,
+                       uint8_t *cand, uint8_t *adm, double *screen_margin, double *mass_margin,
+                       int64_t *n_cand) {
+    const int64_t NB = (n + B - 1) / B, MB = (m + B - 1) / B;
+    double *rs = (double *)malloc((size_t)NB * (2 + 2 * d) * sizeof(double));
+    double *cs = (double *)malloc((size_t)MB * (2 + 2 * d) * sizeof(double));
+    for (int64_t p = 0; p < NB; ++p) {
+        double *s = rs + p * (2 + 2 * d);
+        block_summary(x, a, f, n, d, B, p, s, s + 1, s + 2, s + 2 + d);
+    }
+    for (int64_t q = 0; q < MB; ++q) {
+        double *s = cs + q * (2 + 2 * d);
+        block_summary(y, b, g, m, d, B, q, s, s + 1, s + 2, s + 2 + d);
+    }
+    int64_t nc = 0, na = 0;
+    #pragma omp parallel for schedule(dynamic, 1) reduction(+ : nc, na)
+    for (int64_t p = 0; p < NB; ++p) {
+        const double *sp = rs + p * (2 + 2 * d);
+        const int64_t ni = ((p + 1) * B < n ? (p + 1) * B : n) - p * B;
+        double *v = (double *)malloc((size_t)(B * B) * sizeof(double));
+        for (int64_t q = 0; q < MB; ++q) {
+            const double *sq = cs + q * (2 + 2 * d);
+            const int64_t mj = ((q + 1) * B < m ? (q + 1) * B : m) - q * B;
+            const int64_t pq = p * MB + q;
+            cand[pq] = adm[pq] = 0;
+            if (screen_margin) screen_margin[pq] = -INFINITY;
+            if (mass_margin) mass_margin[pq] = NAN;
+            if (sp[0] == -INFINITY || sq[0] == -INFINITY) continue;  /* U_pq = 0 */
+            double D = 0.0;
+            for (int k = 0; k < d; ++k) {
+                double gap = 0.0;
+                if (sp[2 + k] - sq[2 + d + k] > gap) gap = sp[2 + k] - sq[2 + d + k];
+                if (sq[2 + k] - sp[2 + d + k] > gap) gap = sq[2 + k] - sp[2 + d + k];
+                D += gap * gap;
+            }
+            const double log_rho = log(delta) + log(sp[1] < sq[1] ? sp[1] : sq[1]);
+            const double log_u = log((double)ni * (double)mj) + (sp[0] + sq[0] - c * D) / eps;
+            if (screen_margin) screen_margin[pq] = log_u - log_rho;
+            if (!(log_u > log_rho)) continue;
+            cand[pq] = 1;
+            ++nc;
+            if (!verify) {
+                adm[pq] = 1;
+                ++na;
+                continue;
+            }
+            int64_t len = 0;
+            for (int64_t i = p * B; i < p * B + ni; ++i)
+                for (int64_t j = q * B; j < q * B + mj; ++j)
+                    v[len++] = (f[i] == -INFINITY || g[j] == -INFINITY)
+                                   ? -INFINITY
+                                   : (f[i] + g[j] - cost(x, y, i, j, d, c)) / eps;
+            const double log_m = lse(v, len);
+            if (mass_margin) mass_margin[pq] = log_m - log_rho;
+            if (log_m > log_rho) {
+                adm[pq] = 1;
+                ++na;
+            }
+        }
+        free(v);
+    }
+    free(rs);
+    free(cs);
+    if (n_cand) *n_cand = nc;
+    return na;
+}
+
+/* does block p (of the updated side) have an admitted tile? */
+static int block_has_tile(const uint8_t *adm, int64_t NB, int64_t MB, int64_t p, int rows_side) {
+    if (rows_side) {
+        for (int64_t q = 0; q < MB; ++q)
+            if (adm[p * MB + q]) return 1;
+    } else {
+        for (int64_t r = 0; r < NB; ++r)
+            if (adm[r * MB + p]) return 1;
+    }
+    return 0;
+}
+
+/* f-update on the mask (section 3.2): row i of block p reduces over the
+ * columns of the tiles q with adm[p][q]; over every column when block p has
+ * no admitted tile. x, y, a, g in Morton order.                            */
+void orc_sparse_f_step(const float *x, const float *y, const double *a, const double *g,
+                       int64_t n, int64_t m, int d, double c, double eps, int64_t B,
+                       const uint8_t *adm, double *f_out) {
+    const int64_t NB = (n + B - 1) / B, MB = (m + B - 1) / B;
+    #pragma omp parallel
+    {
+        double *v = (double *)malloc((size_t)(m > 0 ? m : 1) * sizeof(double));
+        #pragma omp for schedule(static)
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t p = i / B;
+            const int all = !block_has_tile(adm, NB, MB, p, 1);
+            if (a[i] == 0.0) {
+                f_out[i] = -INFINITY;
+                continue;
+            }
+            int64_t len = 0;
+            for (int64_t j = 0; j < m; ++j)
+                if (all || adm[p * MB + j / B]) v[len++] = (g[j] - cost(x, y, i, j, d, c)) / eps;
+            f_out[i] = eps * log(a[i]) - eps * lse(v, len);
+        }
+        free(v);
+    }
+}
+
+/* g-update on the same mask, read by columns. */
+void orc_sparse_g_step(const float *x, const float *y, const double *b, const double *f,
+                       int64_t n, int64_t m, int d, double c, double eps, int64_t B,
+                       const uint8_t *adm, double *g_out) {
+    const int64_t NB = (n + B - 1) / B, MB = (m + B - 1) / B;
+    #pragma omp parallel
+    {
+        double *v = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+        #pragma omp for schedule(static)
+        for (int64_t j = 0; j < m; ++j) {
+            const int64_t q = j / B;
+            const int all = !block_has_tile(adm, NB, MB, q, 0);
+            if (b[j] == 0.0) {
+                g_out[j] = -INFINITY;
+                continue;
+            }
+            int64_t len = 0;
+            for (int64_t i = 0; i < n; ++i)
+                if (all || adm[(i / B) * MB + q]) v[len++] = (f[i] - cost(x, y, i, j, d, c)) / eps;
+            g_out[j] = eps * log(b[j]) - eps * lse(v, len);
+        }
+        free(v);
+    }
+}
+
+/* row residual of the admitted plan, sum_i |sum_{admitted j} T_ij - a_i|
+ * (every column for a row block without an admitted tile).               */
+double orc_sparse_row_residual(const float *x, const float *y, const double *a, const double *f,
+                               const double *g, int64_t n, int64_t m, int d, double c,
+                               double eps, int64_t B, const uint8_t *adm) {
+    const int64_t NB = (n + B - 1) / B, MB = (m + B - 1) / B;
+    double *rs = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t p = i / B;
+        const int all = !block_has_tile(adm, NB, MB, p, 1);
+        double s = 0.0;
+        for (int64_t j = 0; j < m; ++j)
+            if (all || adm[p * MB + j / B]) s += plan_entry(x, y, f, g, i, j, d, c, eps);
+        rs[i] = fabs(s - a[i]);
+    }
+    double r = 0.0;
+    for (int64_t i = 0; i < n; ++i) r += rs[i];
+    free(rs);
+    return r;
+}
+
+/* Block-sparse solve (fine updates only; the readings above). Inputs and
+ * f, g (warm start in, result out) in the caller's order; the iterations run
+ * in Morton order. delta <= 0 takes tol / (4 max(NB, MB)) (then tol must be
+ * > 0). stats (optional, 4 entries): sparse iterations, dense iterations,
+ * candidates and admitted tiles of the last mask. Returns the iterations
+ * done, or -1 for bad arguments; *resid gets the stop test's residual of the
+ * returned state.                                                          */
+int orc_sinkhorn_sparse(const float *x, const float *y, const double *a, const double *b,
+                        int64_t n, int64_t m, int d, double c, double eps, int n_iters,
+                        double tol, int64_t B, double delta, int verify, double dense_frac,
+                        double *f, double *g, double *resid, int64_t *stats) {
+    if (B < 1 || n < 1 || m < 1) return -1;
+    const int64_t NB = (n + B - 1) / B, MB = (m + B - 1) / B;
+    if (delta <= 0.0) {
+        if (!(tol > 0.0)) return -1;
+        delta = tol / (4.0 * (double)(NB > MB ? NB : MB));
+    }
+    double lo[3], hi[3];
+    for (int k = 0; k < d; ++k) {
+        lo[k] = INFINITY;
+        hi[k] = -INFINITY;
+        for (int64_t i = 0; i < n; ++i) {
+            const double v = (double)x[i * d + k];
+            if (v < lo[k]) lo[k] = v;
+            if (v > hi[k]) hi[k] = v;
+        }
+        for (int64_t j = 0; j < m; ++j) {
+            const double v = (double)y[j * d + k];
+            if (v < lo[k]) lo[k] = v;
+            if (v > hi[k]) hi[k] = v;
+        }
+    }
+    int64_t *px = (int64_t *)malloc((size_t)n * sizeof(int64_t));
+    int64_t *py = (int64_t *)malloc((size_t)m * sizeof(int64_t));
+    orc_morton_order(x, n, d, lo, hi, px);
+    orc_morton_order(y, m, d, lo, hi, py);
+    float *xs = (float *)malloc((size_t)n * d * sizeof(float));
+    float *ys = (float *)malloc((size_t)m * d * sizeof(float));
+    double *as = (double *)malloc((size_t)n * sizeof(double));
+    double *bs = (double *)malloc((size_t)m * sizeof(double));
+    double *fs = (double *)malloc((size_t)n * sizeof(double));
+    double *gs = (double *)malloc((size_t)m * sizeof(double));
+    double asum = 0.0;
+    for (int64_t r = 0; r < n; ++r) {
+        for (int k = 0; k < d; ++k) xs[r * d + k] = x[px[r] * d + k];
+        as[r] = a[px[r]];
+        fs[r] = f[px[r]];
+        asum += as[r];
+    }
+    for (int64_t r = 0; r < m; ++r) {
+        for (int k = 0; k < d; ++k) ys[r * d + k] = y[py[r] * d + k];
+        bs[r] = b[py[r]];
+        gs[r] = g[py[r]];
+    }
+    const double tol_eff = tol - (double)MB * delta * asum;
+    uint8_t *cand = (uint8_t *)malloc((size_t)(NB * MB));
+    uint8_t *adm = (uint8_t *)malloc((size_t)(NB * MB));
+    int64_t n_sparse = 0, n_dense = 0, nc = 0, na = 0;
+    double r = NAN;
+    int it = 0;
+    for (;; ++it) {
+        na = orc_block_mask(xs, ys, as, bs, fs, gs, n, m, d, c, eps, B, delta, verify, cand, adm,
+                            NULL, NULL, &nc);
+        const int dense = (double)nc > dense_frac * (double)NB * (double)MB;
+        const int test = tol > 0.0 && it >= 1;
+        if (test || it == n_iters) {
+            r = dense ? row_residual(xs, ys, as, fs, gs, n, m, d, c, eps)
+                      : orc_sparse_row_residual(xs, ys, as, fs, gs, n, m, d, c, eps, B, adm);
+            if (test && r <= tol_eff) break;
+        }
+        if (it == n_iters) break;
+        if (dense) {
+            orc_f_step(xs, ys, as, gs, n, m, d, c, eps, NULL, 0, fs);
+            orc_g_step(xs, ys, bs, fs, n, m, d, c, eps, NULL, 0, gs);
+            ++n_dense;
+        } else {
+            orc_sparse_f_step(xs, ys, as, gs, n, m, d, c, eps, B, adm, fs);
+            orc_sparse_g_step(xs, ys, bs, fs, n, m, d, c, eps, B, adm, gs);
+            ++n_sparse;
+        }
+    }
+    for (int64_t r2 = 0; r2 < n; ++r2) f[px[r2]] = fs[r2];
+    for (int64_t r2 = 0; r2 < m; ++r2) g[py[r2]] = gs[r2];
+    if (resid) *resid = r;
+    if (stats) {
+        stats[0] = n_sparse;
+        stats[1] = n_dense;
+        stats[2] = nc;
+        stats[3] = na;
+    }
+    free(px); free(py); free(xs); free(ys); free(as); free(bs); free(fs); free(gs);
+    free(cand); free(adm);
+    return it;
+}

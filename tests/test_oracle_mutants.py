@@ -29,6 +29,12 @@ MUTANTS = {
     "csr_drops_the_column_order": ("                col_idx[k] = j;", "                col_idx[k] = m - 1 - j;"),
     "lr_multiplies_by_g": ("(double)R[j * r + q] / (double)g[q];", "(double)R[j * r + q] * (double)g[q];"),
     "lrc_drops_the_bias": ("const double C = c * (dot + bias);", "const double C = c * dot;"),
+    "morton_bit_order": ("cd |= (uint64_t)1 << (t * d + (d - 1 - k));", "cd |= (uint64_t)1 << (t * d + k);"),
+    "screen_drops_tile_size": ("log((double)ni * (double)mj) + (sp[0]", "(sp[0]"),
+    "screen_gap_one_sided": ("if (sq[2 + k] - sp[2 + d + k] > gap) gap = sq[2 + k] - sp[2 + d + k];", ""),
+    "threshold_takes_the_larger_weight": ("log(sp[1] < sq[1] ? sp[1] : sq[1])", "log(sp[1] > sq[1] ? sp[1] : sq[1])"),
+    "sparse_f_without_fallback": ("if (all || adm[p * MB + j / B]) v[len++]", "if (adm[p * MB + j / B]) v[len++]"),
+    "sparse_residual_counts_all_columns": ("if (all || adm[p * MB + j / B]) s +=", "s +="),
 }
 
 
@@ -131,7 +137,63 @@ def _battery(orc):
         mean = (xd ** 2).sum(1).mean() + (yd ** 2).sum(1).mean() - 2 * xd.mean(0) @ yd.mean(0)
         return abs(1.0 / orc.inv_scale_cost(x, y, "mean") - mean) < 1e-12 * mean
 
-    for name, fn in [("row_marginals", row_marginals), ("col_marginals", col_marginals),
+    def block_sparse():
+        # FlashSinkhorn 2, sections 3, 3.2, A.3: Z-order, screen, verification,
+        # omitted-mass bound and the masked updates' marginals
+        grid = np.array([(i / 3, j / 3) for i in range(4) for j in range(4)], np.float32)
+        perm = orc.morton_order(grid, np.zeros(2), np.ones(2))
+        z = [(0, 0), (0, 1), (1, 0), (1, 1), (0, 2), (0, 3), (1, 2), (1, 3),
+             (2, 0), (2, 1), (3, 0), (3, 1), (2, 2), (2, 3), (3, 2), (3, 3)]
+        if [(int(round(grid[k, 0] * 3)), int(round(grid[k, 1] * 3))) for k in perm] != z:
+            return False
+        r3 = np.random.default_rng(2)  # coincident points per block: the screen bound is exact
+        xt = np.repeat(r3.random((5, 3)), 4, axis=0).astype(np.float32)[:19]
+        yt = np.repeat(r3.random((4, 3)), 4, axis=0).astype(np.float32)
+        ft, gt = np.repeat(r3.normal(0, 0.05, 5), 4)[:19], np.repeat(r3.normal(0, 0.05, 4), 4)
+        at, bt = r3.random(19) + 0.1, r3.random(16) + 0.1
+        Tt = orc.dense_plan(xt, yt, ft, gt, 1.7, 0.05)
+        Mt = np.array([[Tt[p * 4:(p + 1) * 4, q * 4:(q + 1) * 4].sum() for q in range(4)] for p in range(5)])
+        rt = 1e-3 * np.minimum(np.array([at[p * 4:(p + 1) * 4].min() for p in range(5)])[:, None],
+                               np.array([bt[q * 4:(q + 1) * 4].min() for q in range(4)])[None, :])
+        ot = orc.block_mask(xt, yt, at, bt, ft, gt, 1.7, 0.05, 4, 1e-3)
+        if not np.allclose(ot["screen_margin"], np.log(Mt / rt), rtol=0, atol=1e-9):
+            return False
+        r2 = np.random.default_rng(5)
+        xs, ys = r2.random((120, 3)).astype(np.float32), r2.random((100, 3)).astype(np.float32)
+        lo, hi = orc.joint_box(xs, ys)
+        xs, ys = xs[orc.morton_order(xs, lo, hi)], ys[orc.morton_order(ys, lo, hi)]
+        aa, bb = r2.random(120) + 0.2, r2.random(100) + 0.2
+        aa, bb = aa / aa.sum(), bb / bb.sum()
+        e2, B, delta = 0.004, 8, 1e-3
+        f2, g2, _, _ = orc.sinkhorn(xs, ys, aa, bb, 1.0, e2, 15)
+        T = orc.dense_plan(xs, ys, f2, g2, 1.0, e2)
+        NB, MB = 15, 13
+        M = np.array([[T[p * B:(p + 1) * B, q * B:(q + 1) * B].sum() for q in range(MB)] for p in range(NB)])
+        amin = np.array([aa[p * B:(p + 1) * B].min() for p in range(NB)])
+        bmin = np.array([bb[q * B:(q + 1) * B].min() for q in range(MB)])
+        rho = delta * np.minimum(amin[:, None], bmin[None, :])
+        o = orc.block_mask(xs, ys, aa, bb, f2, g2, 1.0, e2, B, delta)
+        if not np.all(o["screen_margin"] >= np.log(M / rho) - 1e-9):
+            return False
+        if not np.array_equal(o["adm"], o["cand"] & (M > rho)):
+            return False
+        for p in range(NB):
+            for q in range(MB):
+                if not o["adm"][p, q]:
+                    t = T[p * B:(p + 1) * B, q * B:(q + 1) * B]
+                    if np.any(t.sum(1) > delta * aa[p * B:(p + 1) * B] * (1 + 1e-12)):
+                        return False
+        adm = o["adm"].copy()
+        adm[2, :] = False  # a row block that falls back to every column
+        fs = orc.sparse_f_step(xs, ys, aa, g2, 1.0, e2, B, adm)
+        rows = np.repeat(np.repeat(adm, B, axis=0), B, axis=1)[:120, :100]
+        rows[16:24, :] = True
+        T = orc.dense_plan(xs, ys, fs, g2, 1.0, e2)
+        if not np.allclose((T * rows).sum(1), aa, rtol=1e-12, atol=0):
+            return False
+        return abs(orc.sparse_row_residual(xs, ys, aa, fs, g2, 1.0, e2, B, adm)) < 1e-13
+
+    for name, fn in [("block_sparse", block_sparse), ("row_marginals", row_marginals), ("col_marginals", col_marginals),
                      ("two_point", two_point), ("cross_ratio", cross_ratio),
                      ("min_row_contract", min_row_contract), ("residual", residual), ("csr", csr),
                      ("lowrank", lowrank),
