@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define OT_ABI_VERSION 1
+#define OT_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define OT_API __attribute__((visibility("default")))
@@ -102,6 +102,29 @@ typedef struct ot_options {
                                  (default) for problems up to 2^28 pairs, 0 never,
                                  1 always */
     int32_t reserved1;
+    int32_t block_sparse;     /* d <= 3: 1 runs block-sparse fine iterations ("FlashSinkhorn 2:
+                                 Block-Sparse Entropic Optimal Transport", sections 3, 3.2,
+                                 A.3, B.3): the points are put in Morton order once; every
+                                 iteration screens all block pairs with the bound
+                                 |I||J| exp((F_I + G_J - c D_IJ)/eps) (block potential maxima,
+                                 squared bounding-box distance) against rho_IJ = delta *
+                                 min(smallest nonzero a_i of I, b_j of J), verifies the
+                                 candidates by their exact mass, and runs both half-steps over
+                                 the admitted tiles only (every tile for a block with none).
+                                 The stop test compares the admitted plan's row residual with
+                                 tol - MB delta sum(a), so that the full residual is <= tol.
+                                 f and g are returned in the caller's order. 0 (default):
+                                 dense iterations */
+    int32_t sparse_block;     /* block size B: 128 or 256 (0 = 128 when NB * MB <= 2^27,
+                                 else 256) */
+    int32_t sparse_verify;    /* 1 (default): candidate tiles are verified by their exact mass;
+                                 0: the box screen alone decides */
+    int32_t reserved2;
+    double sparse_delta;      /* delta of the tile threshold; 0 (default): tol / (4 max(NB,
+                                 MB)) (section 3.2), which needs tol > 0 */
+    double sparse_dense_frac; /* an iteration whose candidate tiles exceed this fraction of
+                                 all NB * MB block pairs runs the dense half-steps instead
+                                 (default 0.5) */
 } ot_options;
 
 /* -------------------------------------------------------- solve report   */
@@ -121,6 +144,13 @@ typedef struct ot_info {
     int64_t kernel_launches;   /* kernels this call launched (graph nodes included) */
     double loop_ms;            /* device time of the iteration loop, from CUDA events
                                   around each chunk (opt->timing), else 0 */
+    /* block-sparse mode only (zero otherwise) */
+    int64_t sparse_iterations; /* iterations run on a block mask */
+    int64_t dense_iterations;  /* iterations run dense (too many candidate tiles) */
+    int64_t tiles_candidate;   /* last mask: tiles that passed the box screen */
+    int64_t tiles_admitted;    /* last mask: tiles admitted after verification */
+    int64_t tiles_total;       /* NB * MB block pairs */
+    double omitted_bound;      /* bound on the row mass one mask omits: MB delta sum(a) */
 } ot_info;
 
 /* Opaque plan: the pages' "row materializer built once", which captures the

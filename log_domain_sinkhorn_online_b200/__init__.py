@@ -168,8 +168,18 @@ def lrcost_rows(cost1, cost2, f, g, row_idx, eps, inv_scale_cost=1.0, bias=0.0, 
 def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None, warm_start=False,
              check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,
              timing=False, col_splits=0, rows_per_thread=0, tensor_cores=True,
-             device_loop=-1, stream=None) -> Plan:
-    """Solves on the GPU; x [n,d], y [m,d], a [n], b [m] float32 CUDA tensors."""
+             device_loop=-1, block_sparse=False, sparse_block=0, sparse_verify=True,
+             sparse_delta=0.0, sparse_dense_frac=0.5, stream=None) -> Plan:
+    """Solves on the GPU; x [n,d], y [m,d], a [n], b [m] float32 CUDA tensors.
+
+    block_sparse (d <= 3): block-sparse fine iterations ("FlashSinkhorn 2",
+    sections 3.2, A.3, B.3): Morton-ordered blocks of sparse_block points, a
+    box screen and (sparse_verify) an exact-mass check of every block pair
+    against delta * min weight (sparse_delta, 0 = tol / (4 max(NB, MB))), the
+    half-steps over the admitted tiles only; an iteration whose candidates
+    exceed sparse_dense_frac of all pairs runs dense. f and g come back in the
+    caller's order.
+    """
     import torch
     x, y = _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y")
     a, b = _dev(a, torch.float32, "a"), _dev(b, torch.float32, "b")
@@ -189,6 +199,11 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
     opt.rows_per_thread = int(rows_per_thread)
     opt.tensor_cores = int(bool(tensor_cores))
     opt.device_loop = int(device_loop)
+    opt.block_sparse = int(bool(block_sparse))
+    opt.sparse_block = int(sparse_block)
+    opt.sparse_verify = int(bool(sparse_verify))
+    opt.sparse_delta = float(sparse_delta)
+    opt.sparse_dense_frac = float(sparse_dense_frac)
     if isinstance(scale, str):
         sc = _SCALES[scale]
     else:

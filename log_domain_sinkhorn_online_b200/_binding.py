@@ -41,7 +41,10 @@ class OtOptions(ctypes.Structure):
                 ("eps_decay", ctypes.c_double), ("timing", ctypes.c_int32),
                 ("col_splits", ctypes.c_int32), ("rows_per_thread", ctypes.c_int32),
                 ("tensor_cores", ctypes.c_int32), ("device_loop", ctypes.c_int32),
-                ("reserved1", ctypes.c_int32)]
+                ("reserved1", ctypes.c_int32), ("block_sparse", ctypes.c_int32),
+                ("sparse_block", ctypes.c_int32), ("sparse_verify", ctypes.c_int32),
+                ("reserved2", ctypes.c_int32), ("sparse_delta", ctypes.c_double),
+                ("sparse_dense_frac", ctypes.c_double)]
 
 
 class OtInfo(ctypes.Structure):
@@ -50,7 +53,10 @@ class OtInfo(ctypes.Structure):
                 ("residual", ctypes.c_double), ("inv_scale_cost", ctypes.c_double),
                 ("eps", ctypes.c_double), ("n_massless_rows", ctypes.c_int64),
                 ("n_massless_cols", ctypes.c_int64), ("half_steps", ctypes.c_int64),
-                ("kernel_launches", ctypes.c_int64), ("loop_ms", ctypes.c_double)]
+                ("kernel_launches", ctypes.c_int64), ("loop_ms", ctypes.c_double),
+                ("sparse_iterations", ctypes.c_int64), ("dense_iterations", ctypes.c_int64),
+                ("tiles_candidate", ctypes.c_int64), ("tiles_admitted", ctypes.c_int64),
+                ("tiles_total", ctypes.c_int64), ("omitted_bound", ctypes.c_double)]
 
 
 class OTError(RuntimeError):

@@ -8,6 +8,7 @@
 // scalars (the device stop flag, the in-loop residual, the iteration count).
 #include <cmath>
 #include <cstdarg>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
@@ -64,10 +65,18 @@ struct DevScalars {
     double wsum[4];               // sum a, -, sum b, -
 };
 
+// block-sparse mode: device counters of one iteration
+struct SparseCtr {
+    unsigned long long cand, adm;  // candidate and admitted tiles of the current mask
+    unsigned work, pad;            // verification: dynamic row-block counter
+    unsigned lohi[6];              // joint bounding box (order-preserving float bits)
+};
+
 // pinned host mirror for read-backs
 struct HostScalars {
     DevScalars s;
     State st;
+    SparseCtr sc, sc_prev;
     double o[kMaxD];
 };
 
@@ -117,6 +126,31 @@ struct ot_plan {
     int loop_rpt = 2;           // rows per thread of the loop kernel (1 or 2)
     unsigned *bar = nullptr;    // grid barrier: count, generation
     double *blk_resid = nullptr;
+    // arrays the iterations read: the caller's, or their Morton-ordered copies
+    // in block-sparse mode
+    const float *sx_pts = nullptr, *sy_pts = nullptr, *sa = nullptr, *sb = nullptr;
+    float *sf[2] = {nullptr, nullptr}, *sg = nullptr;
+    // block-sparse mode (ot_options.block_sparse)
+    bool sparse = false;
+    int sp_B = 0, sp_rpt = 1, sp_verify = 1;
+    int64_t sp_nb = 0, sp_mb = 0;
+    int sp_splits[2] = {1, 1}, sp_grid[2] = {1, 1}, sp_vgrid = 1;
+    double sp_delta = 0.0, sp_frac = 0.5, sp_bound = 0.0, asum = 0.0;
+    char *ws_sp = nullptr;
+    size_t ws_sp_bytes = 0;
+    int64_t *perm_x = nullptr, *perm_y = nullptr;
+    unsigned long long *keys = nullptr;
+    BlockSum *bsx = nullptr, *bsy = nullptr;
+    uint8_t *mask = nullptr, *mask_t = nullptr;
+    int64_t *cnt = nullptr, *cnt_t = nullptr, *ptr = nullptr, *ptr_t = nullptr, *sp_scan = nullptr;
+    int *lst = nullptr, *lst_t = nullptr;
+    float2 *sp_part = nullptr;
+    unsigned *sp_tcnt = nullptr;
+    double *sp_tres = nullptr;
+    SparseCtr *sc = nullptr;
+    int64_t sp_iters = 0, dn_iters = 0;
+    int64_t last_cand = 0, last_adm = 0;  // tiles of the last mask an iteration ran on
+    bool adm_pending = false;             // its admitted count is still on the device
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
     cudaStream_t s_int = nullptr;
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
@@ -141,6 +175,7 @@ void plan_free(ot_plan *p) {
     if (p->s_int) cudaStreamSynchronize(p->s_int);
     pool_device_free(p->ws, p->ws_bytes);
     pool_device_free(p->ws_rows, p->ws_rows_bytes);
+    pool_device_free(p->ws_sp, p->ws_sp_bytes);
     pool_host_free(p->hs, sizeof(HostScalars));
     if (p->ev_in) cudaEventDestroy(p->ev_in);
     if (p->ev_out) cudaEventDestroy(p->ev_out);
@@ -288,7 +323,7 @@ HalfStep make_step(const ot_plan *p, int side, int parity) {
     const bool f = side == 0;
     const Side &rows = f ? p->sx : p->sy;
     const Side &cols = f ? p->sy : p->sx;
-    float *fb[2] = {p->f, p->fspare};
+    float *const *fb = p->sf;
     A.coltab = reinterpret_cast<const float4 *>(cols.coltab);
     A.rowtab = rows.rowtab;
     A.rows = rows.cnt;
@@ -302,9 +337,9 @@ HalfStep make_step(const ot_plan *p, int side, int parity) {
     A.part = p->part;
     A.tile_cnt = p->tile_cnt;
     A.tile_resid = p->tile_resid;
-    A.w = f ? p->a : p->b;
-    A.pot_old = f ? fb[parity] : p->g;
-    A.pot_new = f ? fb[parity ^ 1] : p->g;
+    A.w = f ? p->sa : p->sb;
+    A.pot_old = f ? fb[parity] : p->sg;
+    A.pot_new = f ? fb[parity ^ 1] : p->sg;
     A.next_col = rows.coltab;  // this side's column table feeds the other half-step
     A.nxt_bf16 = 0;
     if (p->kind == 0) {
@@ -347,6 +382,243 @@ cudaError_t launch_iteration(const ot_plan *p, int parity) {
     cudaError_t e = launch_side(p, 0, parity);
     if (e != cudaSuccess) return e;
     return launch_side(p, 1, parity);
+}
+
+// ------------------------------------------------------- block-sparse mode
+// (csrc/sparse.cu has the kernels and the design)
+
+float float_from_order(unsigned o) {
+    const unsigned b = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
+    float v;
+    std::memcpy(&v, &b, sizeof v);
+    return v;
+}
+
+// Block size, launch shapes and workspace; the Morton order of both clouds and
+// the sorted copies of the points, weights and (warm start) potentials; the
+// blocks' static summaries. Runs after resolve_scale.
+int sparse_setup(ot_plan *p, const ot_options &o, double tol, bool warm) {
+    const int64_t n = p->n, m = p->m;
+    const int d = p->d;
+    int B = o.sparse_block;
+    if (B == 0) {
+        const int64_t nb = (n + 127) / 128, mb = (m + 127) / 128;
+        B = (double)nb * (double)mb <= (double)(1ll << 27) ? 128 : 256;
+    }
+    p->sp_B = B;
+    p->sp_rpt = B / kHsThreads;
+    const int64_t nb = (n + B - 1) / B, mb = (m + B - 1) / B;
+    p->sp_nb = nb;
+    p->sp_mb = mb;
+    if ((double)nb * (double)mb > (double)(1ll << 32))
+        return fail(OT_ERR_UNSUPPORTED, "block mask of %lld x %lld pairs is too large (use a larger block)",
+                    (long long)nb, (long long)mb);
+    if (nb > 65535ll * 32 || (mb + 63) / 64 > 65535)
+        return fail(OT_ERR_UNSUPPORTED, "too many blocks for the screen's grid");
+    p->sp_delta = o.sparse_delta > 0.0 ? o.sparse_delta : tol / (4.0 * (double)std::max(nb, mb));
+    p->sp_frac = o.sparse_dense_frac;
+    p->sp_verify = o.sparse_verify;
+    p->sp_bound = (double)mb * p->sp_delta * p->asum;
+    const int bps = sparse_blocks_per_sm(0, d, p->sp_rpt);
+    const int vbps = sparse_blocks_per_sm(1, d, p->sp_rpt);
+    if (bps <= 0 || vbps <= 0) return fail(OT_ERR_CUDA, "block-sparse kernels cannot be made resident");
+    const int64_t cap = (int64_t)bps * p->sm_count;
+    for (int side = 0; side < 2; ++side) {
+        const int64_t tiles = side == 0 ? nb : mb;
+        const int64_t sp = std::min<int64_t>(std::max<int64_t>((2 * cap + tiles - 1) / tiles, 1), 32);
+        p->sp_splits[side] = (int)sp;
+        p->sp_grid[side] = (int)std::min<int64_t>(tiles * sp, cap);
+    }
+    p->sp_vgrid = (int)std::min<int64_t>(nb, (int64_t)vbps * p->sm_count);
+    auto pow2 = [](int64_t v) {
+        int64_t r = 1;
+        while (r < v) r <<= 1;
+        return r;
+    };
+    const int64_t n2x = pow2(n), n2y = pow2(m);
+    const int64_t part = std::max((int64_t)p->sp_splits[0] * nb, (int64_t)p->sp_splits[1] * mb) * B;
+    float *xs = nullptr, *ys = nullptr, *as = nullptr, *bs = nullptr;
+    for (int pass = 0; pass < 2; ++pass) {
+        Carver cv{pass ? p->ws_sp : nullptr};
+        xs = cv.take<float>(n * d);
+        ys = cv.take<float>(m * d);
+        as = cv.take<float>(n);
+        bs = cv.take<float>(m);
+        p->sf[0] = cv.take<float>(n);
+        p->sf[1] = cv.take<float>(n);
+        p->sg = cv.take<float>(m);
+        p->perm_x = cv.take<int64_t>(n);
+        p->perm_y = cv.take<int64_t>(m);
+        p->keys = cv.take<unsigned long long>(std::max(n2x, n2y));
+        p->bsx = cv.take<BlockSum>(nb);
+        p->bsy = cv.take<BlockSum>(mb);
+        p->mask = cv.take<uint8_t>(nb * mb);
+        p->mask_t = cv.take<uint8_t>(nb * mb);
+        p->cnt = cv.take<int64_t>(nb);
+        p->cnt_t = cv.take<int64_t>(mb);
+        p->ptr = cv.take<int64_t>(nb + 1);
+        p->ptr_t = cv.take<int64_t>(mb + 1);
+        p->sp_scan = cv.take<int64_t>(scan_tmp_count(std::max(nb, mb)));
+        p->lst = cv.take<int>(nb * mb);
+        p->lst_t = cv.take<int>(nb * mb);
+        p->sp_part = cv.take<float2>(part);
+        p->sp_tcnt = cv.take<unsigned>(std::max(nb, mb));
+        p->sp_tres = cv.take<double>(std::max(nb, mb));
+        p->sc = cv.take<SparseCtr>(1);
+        if (pass == 0) OT_CU(pool_device_alloc(reinterpret_cast<void **>(&p->ws_sp), cv.off, &p->ws_sp_bytes));
+    }
+    cudaStream_t s = p->s_int;
+    OT_CU(cudaMemsetAsync(p->sp_tcnt, 0, sizeof(unsigned) * std::max(nb, mb), s));
+    OT_CU(cudaMemsetAsync(p->sc, 0, sizeof(SparseCtr), s));
+    OT_CU(cudaMemsetAsync(p->sc->lohi, 0xff, sizeof(unsigned) * 3, s));
+    OT_CU(launch_box(p->x, n, d, p->sc->lohi, s));
+    OT_CU(launch_box(p->y, m, d, p->sc->lohi, s));
+    OT_CU(cudaMemcpyAsync(&p->hs->sc, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, s));
+    OT_CU(cudaStreamSynchronize(s));
+    MortonArgs M{};
+    M.d = d;
+    M.bits = 30 / d;
+    const double cells = (double)(1ll << M.bits);
+    for (int k = 0; k < 3; ++k) {
+        if (k >= d) continue;
+        const double lo = (double)float_from_order(p->hs->sc.lohi[k]);
+        const double hi = (double)float_from_order(p->hs->sc.lohi[3 + k]);
+        M.lo[k] = lo;
+        M.s[k] = hi > lo ? cells / (hi - lo) : 0.0;
+    }
+    OT_CU(launch_morton_sort(p->x, n, n2x, M, p->keys, s));
+    OT_CU(launch_gather(p->keys, n, d, p->x, p->a, warm ? p->f : nullptr, p->perm_x, xs, as,
+                        p->sf[0], s));
+    OT_CU(launch_morton_sort(p->y, m, n2y, M, p->keys, s));
+    OT_CU(launch_gather(p->keys, m, d, p->y, p->b, warm ? p->g : nullptr, p->perm_y, ys, bs, p->sg, s));
+    if (!warm) {
+        OT_CU(cudaMemsetAsync(p->sf[0], 0, sizeof(float) * n, s));
+        OT_CU(cudaMemsetAsync(p->sg, 0, sizeof(float) * m, s));
+    }
+    OT_CU(launch_block_static(xs, as, n, d, B, p->bsx, s));
+    OT_CU(launch_block_static(ys, bs, m, d, B, p->bsy, s));
+    p->sx_pts = xs;
+    p->sy_pts = ys;
+    p->sa = as;
+    p->sb = bs;
+    return OT_OK;
+}
+
+HalfStep make_sparse_step(const ot_plan *p, int side, int parity) {
+    HalfStep A = make_step(p, side, parity);
+    const bool f = side == 0;
+    A.splits = p->sp_splits[side];
+    A.tiles = (int)(f ? p->sp_nb : p->sp_mb);
+    A.tile_rows = p->sp_B;
+    A.part = p->sp_part;
+    A.tile_cnt = p->sp_tcnt;
+    A.tile_resid = p->sp_tres;
+    A.sp_ptr = f ? p->ptr : p->ptr_t;
+    A.sp_idx = f ? p->lst : p->lst_t;
+    A.sp_coltiles = (int)(f ? p->sp_mb : p->sp_nb);
+    return A;
+}
+
+// One block-sparse iteration from the state at f-buffer parity `par`: the
+// mask at (f, g), then the f-update (f_only: the update that measures the
+// final residual) and the g-update on it. *stopped: the state had already
+// passed the stop test (nothing was launched after the screen).
+int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped) {
+    cudaStream_t s = p->s_int;
+    const int64_t nb = p->sp_nb, mb = p->sp_mb;
+    const int B = p->sp_B, d = p->d, rpt = p->sp_rpt;
+    *stopped = false;
+    OT_CU(cudaMemcpyAsync(&p->hs->sc_prev, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, s));
+    OT_CU(launch_block_max(p->sf[par], p->n, B, p->bsx, s));
+    OT_CU(launch_block_max(p->sg, p->m, B, p->bsy, s));
+    OT_CU(cudaMemsetAsync(p->cnt, 0, sizeof(int64_t) * nb, s));
+    OT_CU(cudaMemsetAsync(p->cnt_t, 0, sizeof(int64_t) * mb, s));
+    OT_CU(cudaMemsetAsync(p->sc, 0, offsetof(SparseCtr, lohi), s));
+    ScreenArgs S{};
+    S.rs = p->bsx;
+    S.cs = p->bsy;
+    S.nb = nb;
+    S.mb = mb;
+    S.d = d;
+    S.c = p->c;
+    S.eps = eps;
+    S.ln_delta = std::log(p->sp_delta);
+    S.mask = p->mask;
+    S.cnt = p->cnt;
+    S.cnt_t = p->cnt_t;
+    S.total = &p->sc->cand;
+    OT_CU(launch_screen(S, s));
+    OT_CU(cudaMemcpyAsync(&p->hs->sc, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, s));
+    OT_CU(cudaMemcpyAsync(&p->hs->st, p->st, sizeof(State), cudaMemcpyDeviceToHost, s));
+    OT_CU(cudaStreamSynchronize(s));
+    p->launches += 3;
+    if (p->adm_pending) {
+        p->last_cand = (int64_t)p->hs->sc_prev.cand;
+        p->last_adm = (int64_t)p->hs->sc_prev.adm;
+        p->adm_pending = false;
+    }
+    if (p->hs->st.stop) {
+        *stopped = true;
+        return OT_OK;
+    }
+    const bool dense = (double)p->hs->sc.cand > p->sp_frac * (double)nb * (double)mb;
+    p->last_cand = p->last_adm = (int64_t)p->hs->sc.cand;
+    if (dense) {
+        OT_CU(launch_side(p, 0, par));
+        if (!f_only) OT_CU(launch_side(p, 1, par));
+        p->launches += f_only ? 1 : 2;
+        if (!f_only) ++p->dn_iters;
+        return OT_OK;
+    }
+    if (p->sp_verify) {
+        VerifyArgs V{};
+        V.coltab = reinterpret_cast<const float4 *>(p->sy.coltab);
+        V.rowtab = p->sx.rowtab;
+        V.pot = p->sf[par];
+        V.prm = p->prm;
+        V.rs = p->bsx;
+        V.cs = p->bsy;
+        V.rows = p->n;
+        V.cols_pad = p->sy.pad;
+        V.nb = nb;
+        V.mb = mb;
+        V.l2_delta = std::log2(p->sp_delta);
+        V.mask = p->mask;
+        V.cnt = p->cnt;
+        V.cnt_t = p->cnt_t;
+        V.work = &p->sc->work;
+        V.total = &p->sc->adm;
+        OT_CU(launch_verify(d, rpt, V, p->sp_vgrid, s));
+        p->launches += 1;
+        p->adm_pending = true;
+    }
+    OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
+    OT_CU(launch_mask_list(p->mask, nb, mb, p->ptr, p->lst, s));
+    OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 0, par), p->sp_grid[0], s));
+    p->launches += 5;
+    if (!f_only) {
+        OT_CU(launch_transpose_bytes(p->mask, nb, mb, p->mask_t, s));
+        OT_CU(launch_row_ptr_scan(p->cnt_t, mb, p->ptr_t, p->sp_scan, s));
+        OT_CU(launch_mask_list(p->mask_t, mb, nb, p->ptr_t, p->lst_t, s));
+        OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 1, par), p->sp_grid[1], s));
+        p->launches += 6;
+        ++p->sp_iters;
+    }
+    return OT_OK;
+}
+
+// `iters` block-sparse iterations from global parity `parity0`; stops early
+// when the stop test has passed.
+int run_sparse(ot_plan *p, int parity0, int iters, double eps) {
+    for (int i = 0; i < iters; ++i) {
+        bool stopped = false;
+        OT_CU(mark(p));
+        int rc = sparse_iteration(p, (parity0 + i) & 1, false, eps, &stopped);
+        OT_CU(mark(p));
+        if (rc != OT_OK) return rc;
+        if (stopped) break;
+    }
+    return OT_OK;
 }
 
 // Runs `iters` iterations starting at global parity `parity0`, in chunks of
@@ -472,6 +744,11 @@ void ot_options_default(ot_options *opt) {
     opt->rows_per_thread = 0;
     opt->tensor_cores = 1;
     opt->device_loop = -1;
+    opt->block_sparse = 0;
+    opt->sparse_block = 0;
+    opt->sparse_verify = 1;
+    opt->sparse_delta = 0.0;
+    opt->sparse_dense_frac = 0.5;
 }
 
 void ot_plan_destroy(ot_plan *plan) { plan_free(plan); }
@@ -684,6 +961,19 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     if (opt) o = *opt;
     int rc = validate(x, y, a, b, n, m, d, eps, scale_cost, n_iters, f, g, o);
     if (rc != OT_OK) return rc;
+    const bool sparse = o.block_sparse != 0;
+    if (sparse) {
+        if (d > 3) return fail(OT_ERR_UNSUPPORTED, "block-sparse iterations need d <= 3");
+        if (o.sparse_block != 0 && o.sparse_block != 128 && o.sparse_block != 256)
+            return fail(OT_ERR_INVALID_ARG, "sparse_block must be 0, 128 or 256");
+        if (!(o.sparse_delta >= 0.0) || !std::isfinite(o.sparse_delta))
+            return fail(OT_ERR_INVALID_ARG, "sparse_delta must be >= 0 and finite");
+        if (o.sparse_delta == 0.0 && !(tol > 0.0))
+            return fail(OT_ERR_INVALID_ARG, "sparse_delta = 0 takes delta from tol, which must be > 0");
+        if (!(o.sparse_dense_frac >= 0.0 && o.sparse_dense_frac <= 1.0))
+            return fail(OT_ERR_INVALID_ARG, "sparse_dense_frac must be in [0, 1]");
+        o.device_loop = 0;  // the mask is rebuilt between every two iterations
+    }
     ot_plan *p = new (std::nothrow) ot_plan();
     if (!p) return fail(OT_ERR_OOM, "host allocation failed");
     struct Guard {
@@ -706,7 +996,13 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
     if ((rc = plan_setup(p, o)) != OT_OK) return rc;
     if ((rc = resolve_scale(p, scale_cost, o.scale_value)) != OT_OK) return rc;
-    if (!o.warm_start) {
+    p->sx_pts = x; p->sy_pts = y; p->sa = a; p->sb = b;
+    p->sf[0] = f; p->sf[1] = p->fspare; p->sg = g;
+    p->asum = p->hs->s.wsum[0];
+    p->sparse = sparse;
+    if (sparse) {
+        if ((rc = sparse_setup(p, o, tol, o.warm_start != 0)) != OT_OK) return rc;
+    } else if (!o.warm_start) {
         OT_CU(cudaMemsetAsync(f, 0, sizeof(float) * n, p->s_int));
         OT_CU(cudaMemsetAsync(g, 0, sizeof(float) * m, p->s_int));
     }
@@ -725,14 +1021,16 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     } else {
         stage_eps.push_back(eps);
     }
-    float *fb[2] = {p->f, p->fspare};
+    float *const *fb = p->sf;
     const int layout = p->kind == 0 ? 0 : 1;  // CUDA-core paths' column-table layout
     int t = 0, converged = 0;
     int64_t half_steps = 0;
     double resid = NAN;
     for (size_t si = 0; si < stage_eps.size(); ++si) {
         const bool last = si + 1 == stage_eps.size();
-        const double tol_s = (last && tol > 0.0) ? tol : 0.0;
+        // block-sparse: the admitted plan's residual must leave room for the
+        // mass the mask omits (at most sp_bound), so the full residual is <= tol
+        const double tol_s = (last && tol > 0.0) ? (sparse ? tol - p->sp_bound : tol) : 0.0;
         const int iters = last ? n_iters : o.iters_per_stage;
         OT_CU(launch_set_params(p->prm, stage_eps[si], p->c, tol_s, p->s_int));
         OT_CU(launch_reset_state(p->st, p->s_int));
@@ -742,13 +1040,15 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
             OT_CU(launch_tc_tables(y, g, m, p->sy.pad, d, p->dp, p->kp, p->o, p->prm,
                                    p->sy.rowtab, p->sy.arow, p->sy.bcol, p->s_int));
         } else {
-            OT_CU(launch_tables(x, fb[t & 1], n, p->sx.pad, d, p->dp, p->o, p->prm, p->sx.rowtab,
-                                p->sx.coltab, layout, p->s_int));
-            OT_CU(launch_tables(y, g, m, p->sy.pad, d, p->dp, p->o, p->prm, p->sy.rowtab,
-                                p->sy.coltab, layout, p->s_int));
+            OT_CU(launch_tables(p->sx_pts, fb[t & 1], n, p->sx.pad, d, p->dp, p->o, p->prm,
+                                p->sx.rowtab, p->sx.coltab, layout, p->s_int));
+            OT_CU(launch_tables(p->sy_pts, p->sg, m, p->sy.pad, d, p->dp, p->o, p->prm,
+                                p->sy.rowtab, p->sy.coltab, layout, p->s_int));
         }
         p->launches += 4;
-        if ((rc = run_iterations(p, t & 1, iters, tol_s > 0.0, o.use_graphs != 0)) != OT_OK) return rc;
+        rc = sparse ? run_sparse(p, t & 1, iters, stage_eps[si])
+                    : run_iterations(p, t & 1, iters, tol_s > 0.0, o.use_graphs != 0);
+        if (rc != OT_OK) return rc;
         if ((rc = read_state(p)) != OT_OK) return rc;
         const int done = p->hs->st.stop ? p->hs->st.conv_iter : iters;
         t += done;
@@ -760,9 +1060,14 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
             } else if (iters > 0) {
                 // one more f-update measures ||T1 - a||_1 of the final state
                 OT_CU(mark(p));
-                OT_CU(launch_side(p, 0, t & 1));
+                if (sparse) {
+                    bool stopped = false;
+                    if ((rc = sparse_iteration(p, t & 1, true, stage_eps[si], &stopped)) != OT_OK) return rc;
+                } else {
+                    OT_CU(launch_side(p, 0, t & 1));
+                    p->launches += 1;
+                }
                 OT_CU(mark(p));
-                p->launches += 1;
                 half_steps += 1;
                 if ((rc = read_state(p)) != OT_OK) return rc;
                 resid = p->hs->st.resid[0];
@@ -770,7 +1075,20 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
             }
         }
     }
-    if (t & 1) OT_CU(cudaMemcpyAsync(p->f, p->fspare, sizeof(float) * n, cudaMemcpyDeviceToDevice, p->s_int));
+    if (sparse && p->adm_pending) {
+        OT_CU(cudaMemcpyAsync(&p->hs->sc_prev, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, p->s_int));
+        OT_CU(cudaStreamSynchronize(p->s_int));
+        p->last_cand = (int64_t)p->hs->sc_prev.cand;
+        p->last_adm = (int64_t)p->hs->sc_prev.adm;
+        p->adm_pending = false;
+    }
+    if (sparse) {  // back to the caller's order
+        OT_CU(launch_scatter(p->sf[t & 1], p->perm_x, n, p->f, p->s_int));
+        OT_CU(launch_scatter(p->sg, p->perm_y, m, p->g, p->s_int));
+        p->launches += 2;
+    } else if (t & 1) {
+        OT_CU(cudaMemcpyAsync(p->f, p->fspare, sizeof(float) * n, cudaMemcpyDeviceToDevice, p->s_int));
+    }
     if ((rc = read_state(p)) != OT_OK) return rc;
     if (p->hs->st.wait_timeout)
         return fail(OT_ERR_CUDA, "a tensor-core pipeline wait timed out (results invalid)");
@@ -798,6 +1116,12 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         info->half_steps = half_steps;
         info->kernel_launches = p->launches;
         info->loop_ms = loop_ms;
+        info->sparse_iterations = p->sp_iters;
+        info->dense_iterations = p->dn_iters;
+        info->tiles_candidate = p->last_cand;
+        info->tiles_admitted = p->last_adm;
+        info->tiles_total = sparse ? p->sp_nb * p->sp_mb : 0;
+        info->omitted_bound = sparse ? p->sp_bound : 0.0;
     }
     if (plan_out) {
         *plan_out = p;

@@ -84,6 +84,12 @@ struct HalfStep {
                                //    terms at element i*nxt_a + nxt_b (tensor-core path)
     const Params *prm;
     State *st;
+    // block-sparse half-step only: the updated side's blocks list their column
+    // tiles in sp_idx[sp_ptr[t] .. sp_ptr[t+1]); an empty list means all
+    // sp_coltiles tiles
+    const int64_t *sp_ptr;
+    const int *sp_idx;
+    int sp_coltiles;
 };
 
 // ------------------------------------------------------ device helpers --

@@ -113,6 +113,61 @@ cudaError_t launch_csr_write(const CsrArgs &C, cudaStream_t s);
 int64_t scan_tmp_count(int64_t n);
 cudaError_t launch_row_ptr_scan(const int64_t *counts, int64_t n, int64_t *row_ptr, int64_t *tmp,
                                 cudaStream_t s);
+// sparse.cu (block-sparse fine updates, d <= 3)
+struct MortonArgs {
+    double lo[3];   // joint bounding box, lower corner
+    double s[3];    // 2^bits / (hi - lo), 0 for a flat coordinate
+    int bits;       // 30 / d
+    int d;
+};
+struct BlockSum {     // one block of B consecutive points (Morton order)
+    double lo[3], hi[3];  // bounding box (0 past d)
+    double pmax;          // largest potential (refreshed every iteration)
+    double lnw, l2w;      // ln and log2 of the smallest nonzero weight (+inf: none)
+    double lncnt;         // ln of the block's point count
+};
+struct ScreenArgs {
+    const BlockSum *rs, *cs;   // row (x) and column (y) blocks
+    int64_t nb, mb;
+    int d;
+    double c, eps, ln_delta;
+    uint8_t *mask;             // [nb][mb]: 1 for a candidate
+    int64_t *cnt, *cnt_t;      // candidates per row block / per column block (zeroed before)
+    unsigned long long *total; // candidates (zeroed before)
+};
+struct VerifyArgs {
+    const float4 *coltab;      // the column side's half-step table
+    const float *rowtab;       // x' rows, 4 floats each
+    const float *pot;          // f
+    const Params *prm;
+    const BlockSum *rs, *cs;
+    int64_t rows, cols_pad, nb, mb;
+    double l2_delta;
+    uint8_t *mask;             // candidates in, admitted tiles out
+    int64_t *cnt, *cnt_t;      // out: admitted per row block; in/out: per column block
+    unsigned *work;            // dynamic row-block counter (zeroed before)
+    unsigned long long *total; // admitted tiles (zeroed before)
+};
+int sparse_blocks_per_sm(int which, int d, int rpt);  // which: 0 half-step, 1 verification
+cudaError_t launch_box(const float *p, int64_t cnt, int d, unsigned *lohi, cudaStream_t s);
+cudaError_t launch_morton_sort(const float *p, int64_t cnt, int64_t n2, const MortonArgs &M,
+                               unsigned long long *keys, cudaStream_t s);
+cudaError_t launch_gather(const unsigned long long *keys, int64_t cnt, int d, const float *p,
+                          const float *w, const float *pot, int64_t *perm, float *ps, float *ws,
+                          float *pots, cudaStream_t s);
+cudaError_t launch_scatter(const float *in, const int64_t *perm, int64_t cnt, float *out,
+                           cudaStream_t s);
+cudaError_t launch_block_static(const float *ps, const float *ws, int64_t cnt, int d, int B,
+                                BlockSum *bs, cudaStream_t s);
+cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, BlockSum *bs, cudaStream_t s);
+cudaError_t launch_screen(const ScreenArgs &S, cudaStream_t s);
+cudaError_t launch_verify(int d, int rpt, const VerifyArgs &V, int grid, cudaStream_t s);
+cudaError_t launch_mask_list(const uint8_t *mask, int64_t rows, int64_t cols, const int64_t *ptr,
+                             int *list, cudaStream_t s);
+cudaError_t launch_transpose_bytes(const uint8_t *in, int64_t rows, int64_t cols, uint8_t *out,
+                                   cudaStream_t s);
+cudaError_t launch_halfstep_sparse(int d, int rpt, const HalfStep &A, int grid, cudaStream_t s);
+
 cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, const double *o,
                         const Params *prm, double *dcol, cudaStream_t s);
 cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s);

@@ -38,16 +38,18 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_version_and_defaults(B):
-    assert B.ot_version() == 1
+    assert B.ot_version() == 2
     o = B.ot_options_default()
     assert (o.warm_start, o.check_every, o.use_graphs, o.iters_per_stage) == (0, 16, 1, 20)
     assert (o.scale_value, o.eps_init, o.eps_decay) == (1.0, 0.0, 0.7)
     assert (o.timing, o.col_splits, o.rows_per_thread, o.tensor_cores, o.device_loop) == (0, 0, 0, 1, -1)
+    assert (o.block_sparse, o.sparse_block, o.sparse_verify, o.sparse_delta, o.sparse_dense_frac) == \
+        (0, 0, 1, 0.0, 0.5)
 
 
 def test_struct_sizes_match_header_layout(B):
-    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4
-    assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8
+    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4 + 4 * 4 + 2 * 8
+    assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8 + 5 * 8 + 8
 
 
 FAKE = 0x1000  # never dereferenced: validation fails first
@@ -86,6 +88,21 @@ def test_option_validation(B):
     assert _call(B, scale_cost=3, opt=o)[0] in (0, -3)  # 1.0 is valid: the call reaches the device
     o.scale_value = -2.0
     assert _call(B, scale_cost=3, opt=o)[0] == -1
+
+
+def test_block_sparse_options_are_validated(B):
+    def sp(**kw):
+        o = B.ot_options_default()
+        o.block_sparse = 1
+        for k, v in kw.items():
+            setattr(o, k, v)
+        return o
+    assert _call(B, d=5, tol=1e-2, opt=sp())[0] == -6          # d > 3 is not supported
+    assert _call(B, tol=1e-2, opt=sp(sparse_block=64))[0] == -1
+    assert _call(B, tol=0.0, opt=sp())[0] == -1                  # delta from tol needs tol > 0
+    assert _call(B, tol=0.0, opt=sp(sparse_delta=-1.0))[0] == -1
+    assert _call(B, tol=1e-2, opt=sp(sparse_dense_frac=1.5))[0] == -1
+    assert _call(B, tol=0.0, opt=sp(sparse_delta=1e-6))[0] in (0, -3)  # valid: reaches the device
 
 
 def test_row_calls_reject_null_plan(B):
