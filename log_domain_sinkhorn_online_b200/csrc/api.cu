@@ -148,7 +148,7 @@ struct ot_plan {
     unsigned *sp_tcnt = nullptr;
     double *sp_tres = nullptr;
     SparseCtr *sc = nullptr;
-    int64_t sp_iters = 0, dn_iters = 0;
+    std::vector<uint8_t> iter_sparse;     // per launched iteration: 1 sparse, 0 dense
     int64_t last_cand = 0, last_adm = 0;  // tiles of the last mask an iteration ran on
     bool adm_pending = false;             // its admitted count is still on the device
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
@@ -567,7 +567,7 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         OT_CU(launch_side(p, 0, par));
         if (!f_only) OT_CU(launch_side(p, 1, par));
         p->launches += f_only ? 1 : 2;
-        if (!f_only) ++p->dn_iters;
+        if (!f_only) p->iter_sparse.push_back(0);
         return OT_OK;
     }
     if (p->sp_verify) {
@@ -602,7 +602,7 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         OT_CU(launch_mask_list(p->mask_t, mb, nb, p->ptr_t, p->lst_t, s));
         OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 1, par), p->sp_grid[1], s));
         p->launches += 6;
-        ++p->sp_iters;
+        p->iter_sparse.push_back(1);
     }
     return OT_OK;
 }
@@ -1116,8 +1116,13 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         info->half_steps = half_steps;
         info->kernel_launches = p->launches;
         info->loop_ms = loop_ms;
-        info->sparse_iterations = p->sp_iters;
-        info->dense_iterations = p->dn_iters;
+        // iterations of the returned state (the one that met the stop test
+        // was launched but not completed)
+        int64_t sp_it = 0, dn_it = 0;
+        for (size_t k = 0; k < p->iter_sparse.size() && k < (size_t)t; ++k)
+            (p->iter_sparse[k] ? sp_it : dn_it) += 1;
+        info->sparse_iterations = sp_it;
+        info->dense_iterations = dn_it;
         info->tiles_candidate = p->last_cand;
         info->tiles_admitted = p->last_adm;
         info->tiles_total = sparse ? p->sp_nb * p->sp_mb : 0;

@@ -138,6 +138,7 @@ def test_sparse_stop_rule_certifies_the_full_residual(ot, orc):
 
 def test_full_mask_is_the_dense_solve(ot, orc):
     w = _clusters(22, 2600, 2100, 3)
+    w.eps = 0.05  # every tile then holds far more than 1e-300 of mass
     plan = _gpu(ot, w, 8, sparse_delta=1e-300, sparse_dense_frac=1.0)
     assert plan.info.tiles_admitted == plan.info.tiles_total
     f, g, _, _ = orc.sinkhorn(w.x, w.y, w.a, w.b, 1.0, w.eps, 8)
