@@ -62,6 +62,10 @@ def _args():
     ap.add_argument("--lowrank", type=int, default=0, metavar="R",
                     help="instead of the step: time the two low-rank row materializers at rank R "
                          "(4096 rows x 100000 columns) and print their own JSON line")
+    ap.add_argument("--sparse", type=int, default=0, metavar="N",
+                    help="instead of the step: block-sparse against dense fine iterations on the "
+                         "uniform-vs-64-clusters workload at n = m = N (its eps rule), from a "
+                         "state annealed by block-sparse iterations; prints its own JSON line")
     ap.add_argument("--no-large-n", action="store_true",
                     help="skip the d = 3 half-step measurement at n = m = 1e5")
     ap.add_argument("--clock-ms", type=int, default=200,
@@ -322,6 +326,61 @@ def run_lowrank(args, k=4096, m=100_000, n=20_000, reps=5):
     print(json.dumps(line), flush=True)
 
 
+def run_sparse(args, reps=10, dense_reps=2, tau=5e-3):
+    """Fine iterations at the target eps on the uniform-vs-64-clusters workload
+    (n = m = args.sparse, eps = (2 x mean nearest-neighbour spacing)^2): block-
+    sparse ("FlashSinkhorn 2", section 3.2; delta = tau / (4 max(NB, MB)),
+    tau = 5e-3) against dense, both from the same state. The state comes from an
+    untimed annealed block-sparse solve from 16 eps (x0.7 per stage, 20
+    iterations each). Times are the library's CUDA events around every
+    iteration (the sparse ones include the mask build and its host read-back)."""
+    import torch
+    import log_domain_sinkhorn_online_b200 as ot
+    from log_domain_sinkhorn_online_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    w = W.w4(n=args.sparse)
+    x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
+    nb = -(-w.n // 128)
+    delta = tau / (4.0 * max(nb, -(-w.m // 128)))
+    kw = dict(eps=w.eps, scale="none", block_sparse=True, sparse_delta=delta, sparse_block=128)
+    t0 = time.time()
+    warm = ot.sinkhorn(x, y, a, b, n_iters=20, eps_init=16.0 * w.eps, eps_decay=0.7,
+                       iters_per_stage=20, **kw)
+    torch.cuda.synchronize()
+    warm_s = time.time() - t0
+    f0, g0 = warm.f.clone(), warm.g.clone()
+    warm.close()
+    mufu = SMS * EX2_PER_CLK * 1.965e9
+    res = {}
+    for mode, k in (("sparse", reps), ("dense", dense_reps)):
+        extra = kw if mode == "sparse" else dict(eps=w.eps, scale="none")
+        plan = ot.sinkhorn(x, y, a, b, n_iters=k, f=f0.clone(), g=g0.clone(), warm_start=True,
+                           timing=True, **extra)
+        torch.cuda.synchronize()
+        info = plan.info
+        ms_it = info.loop_ms / max(info.iterations, 1)
+        res[mode] = {"ms_per_iteration": ms_it,
+                     "pair_updates_per_s": 2.0 * w.n * w.m / (ms_it / 1e3),
+                     "iterations": int(info.iterations), "residual": float(info.residual)}
+        if mode == "sparse":
+            res[mode].update(tiles_total=int(info.tiles_total), tiles_candidate=int(info.tiles_candidate),
+                             tiles_admitted=int(info.tiles_admitted),
+                             sparse_iterations=int(info.sparse_iterations),
+                             omitted_bound=float(info.omitted_bound))
+            full_row, full_col = plan.marginal_residual()
+            res[mode]["full_row_residual"] = float(full_row)
+        plan.close()
+    line = {"metric": "Sinkhorn pair-updates/s (n*m per half-step, dense equivalent)",
+            "unit": "pair-updates/s", "value": res["sparse"]["pair_updates_per_s"],
+            "dense_value": res["dense"]["pair_updates_per_s"],
+            "speedup_vs_dense": res["dense"]["ms_per_iteration"] / res["sparse"]["ms_per_iteration"],
+            "config": {"workload": f"uniform_vs_64clusters_{w.n}", "n": w.n, "m": w.m, "d": 3,
+                       "eps": w.eps, "scale": "none", "block": 128, "delta": delta, "tau": tau,
+                       "state": f"annealed block-sparse from 16 eps, {warm_s:.1f} s untimed"},
+            "sparse": res["sparse"], "dense": res["dense"], "mufu_peak_ex2_per_s": mufu}
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
     import torch
     import log_domain_sinkhorn_online_b200 as ot
@@ -436,6 +495,8 @@ def main():
         run_reference(args)
     elif args.lowrank:
         run_lowrank(args)
+    elif args.sparse:
+        run_sparse(args)
     else:
         run_ours(args)
 

@@ -575,6 +575,7 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         V.coltab = reinterpret_cast<const float4 *>(p->sy.coltab);
         V.rowtab = p->sx.rowtab;
         V.pot = p->sf[par];
+        V.pts = p->sx_pts;
         V.prm = p->prm;
         V.rs = p->bsx;
         V.cs = p->bsy;

@@ -139,6 +139,7 @@ struct VerifyArgs {
     const float4 *coltab;      // the column side's half-step table
     const float *rowtab;       // x' rows, 4 floats each
     const float *pot;          // f
+    const float *pts;          // the row side's points (Morton order), [rows][d]
     const Params *prm;
     const BlockSum *rs, *cs;
     int64_t rows, cols_pad, nb, mb;

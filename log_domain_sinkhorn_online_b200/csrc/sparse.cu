@@ -255,29 +255,49 @@ __global__ void __launch_bounds__(kScreenThreads) screen_kernel(ScreenArgs S) {
 
 // ------------------------------------------------------------ verification
 // One block per row block (claimed dynamically). The block lists the row's
-// candidates in windows of kVfWindow columns, then for each candidate tile q
-// streams its B columns and forms, per row i, the running (max m_i, sum s_i)
-// of 2^(t_ij) (t = G_j + x'_i.Y_j, as in the half-step). With the row term
-// b_i = kappa f_i - c kappa |x'_i|^2 (float64), the tile's mass is
-//     log2 M = log2 sum_i s_i 2^(b_i + m_i);
-// the tile stays admitted when log2 M > log2 delta + min(log2 amin_p,
-// log2 bmin_q); otherwise its byte is cleared and the counts are corrected.
+// candidates in windows of kVfWindow columns and tests each candidate tile q
+// against log2 rho = log2 delta + min(log2 amin_p, log2 bmin_q):
+//  1. a row-level bound, one warp per tile: with G_q the column block's
+//     largest potential and dist_i the distance from x_i to q's bounding box,
+//         M <= |J_q| sum_i 2^(kappa (f_i + G_q - c dist_i^2));
+//     a tile whose bound stays below rho by kVfMargin (base-2 units, far
+//     above the float32 rounding of the bound) is rejected here: its exact
+//     mass is below rho as well, so the admitted set is the same, at B
+//     exponentials per tile instead of B^2;
+//  2. the exact mass of the others, one block per tile: the tile's B columns
+//     are streamed and, per row i, the running (max m_i, sum s_i) of 2^(t_ij)
+//     (t = G_j + x'_i.Y_j, as in the half-step) is formed; with the row term
+//     b_i = kappa f_i - c kappa |x'_i|^2 (float64), log2 M = log2 sum_i s_i
+//     2^(b_i + m_i), and the tile stays admitted when log2 M > log2 rho.
+// A rejected tile's byte is cleared and the counts are corrected.
 constexpr int kVfWindow = 1024;
+constexpr float kVfMargin = 0.05f;
 
 template <int D, int R>
 __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(VerifyArgs V) {
     constexpr int kB = kHsThreads * R;
     __shared__ __align__(16) float4 buf[kB];
-    __shared__ int s_list[kVfWindow];
+    __shared__ int s_list[kVfWindow], s_exact[kVfWindow];
+    __shared__ float s_xr[kB][3], s_fr[kB];
     __shared__ int s_wcnt[kHsThreads / 32];
+    __shared__ int s_nexact;
     __shared__ float s_max[kHsThreads / 32], s_sum[kHsThreads / 32];
     __shared__ long long s_next;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float4 *rt4 = reinterpret_cast<const float4 *>(V.rowtab);
     const double kappa = V.prm->kappa, c = V.prm->c;
+    const float kf = (float)kappa, cf = (float)c;
 
     long long p = blockIdx.x;
     while (p < V.nb) {
+        // the block's points (caller's coordinates) and potentials for the row-level bound
+        for (int r = tid; r < kB; r += kHsThreads) {
+            const int64_t row = p * kB + r;
+            const bool in = row < V.rows;
+#pragma unroll
+            for (int k = 0; k < 3; ++k) s_xr[r][k] = (in && k < D) ? V.pts[row * D + k] : 0.f;
+            s_fr[r] = in ? V.pot[row] : -INFINITY;
+        }
         float2 xd[R][3];
         double base[R];
 #pragma unroll
@@ -318,10 +338,59 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
 #pragma unroll
             for (int u = 0; u < kPer; ++u)
                 if (flags[u]) s_list[pos++] = (int)(tid * kPer + u);
+            if (tid == 0) s_nexact = 0;
             __syncthreads();
 
-            for (int t = 0; t < total; ++t) {
+            // 1. row-level bound, one warp per candidate tile
+            for (int t = warp; t < total; t += kHsThreads / 32) {
                 const int64_t q = w0 + s_list[t];
+                const BlockSum &cq = V.cs[q];
+                float lo[3], hi[3];
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    lo[k] = (float)cq.lo[k];
+                    hi[k] = (float)cq.hi[k];
+                }
+                const float gq = (float)cq.pmax;
+                float u[kB / 32], mx = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < kB / 32; ++k) {
+                    const int r = lane + 32 * k;
+                    float dist = 0.f;
+#pragma unroll
+                    for (int e = 0; e < D; ++e) {
+                        const float gap = fmaxf(0.f, fmaxf(lo[e] - s_xr[r][e], s_xr[r][e] - hi[e]));
+                        dist = fmaf(gap, gap, dist);
+                    }
+                    u[k] = s_fr[r] == -INFINITY ? -INFINITY : kf * (s_fr[r] + gq - cf * dist);
+                    mx = fmaxf(mx, u[k]);
+                }
+                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                float sum = 0.f;
+                if (mx != -INFINITY) {
+#pragma unroll
+                    for (int k = 0; k < kB / 32; ++k)
+                        if (u[k] != -INFINITY) sum += ex2_approx(u[k] - mx);
+                }
+                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                if (lane == 0) {
+                    const double lb = mx == -INFINITY ? -INFINITY
+                                                      : (double)mx + log2((double)sum) + cq.lncnt * 1.4426950408889634;
+                    const double lrho = V.l2_delta + fmin(V.rs[p].l2w, cq.l2w);
+                    if (lb + kVfMargin <= lrho) {
+                        V.mask[p * V.mb + q] = 0;
+                        atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt_t + q), ~0ull);
+                    } else {
+                        s_exact[atomicAdd(&s_nexact, 1)] = s_list[t];
+                    }
+                }
+            }
+            __syncthreads();
+            const int n_exact = s_nexact;
+
+            // 2. exact mass, one block per remaining tile
+            for (int t = 0; t < n_exact; ++t) {
+                const int64_t q = w0 + s_exact[t];
                 for (int u = tid; u < kB; u += kHsThreads) {
                     const int64_t col = q * kB + u;
                     buf[u] = col < V.cols_pad ? V.coltab[col] : dead4(u);
