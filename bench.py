@@ -364,7 +364,7 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3):
                      "iterations": int(info.iterations), "residual": float(info.residual)}
         if mode == "sparse":
             res[mode].update(tiles_total=int(info.tiles_total), tiles_candidate=int(info.tiles_candidate),
-                             tiles_admitted=int(info.tiles_admitted),
+                             tiles_admitted=int(info.tiles_admitted), tiles_exact=int(info.tiles_exact),
                              sparse_iterations=int(info.sparse_iterations),
                              omitted_bound=float(info.omitted_bound))
             full_row, full_col = plan.marginal_residual()

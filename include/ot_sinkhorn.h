@@ -149,6 +149,8 @@ typedef struct ot_info {
     int64_t dense_iterations;  /* iterations run dense (too many candidate tiles) */
     int64_t tiles_candidate;   /* last mask: tiles that passed the box screen */
     int64_t tiles_admitted;    /* last mask: tiles admitted after verification */
+    int64_t tiles_exact;       /* last mask: candidates whose exact mass was evaluated (the
+                                  others fell below the threshold on a point-level bound) */
     int64_t tiles_total;       /* NB * MB block pairs */
     double omitted_bound;      /* bound on the row mass one mask omits: MB delta sum(a) */
 } ot_info;

@@ -55,7 +55,7 @@ class OtInfo(ctypes.Structure):
                 ("n_massless_cols", ctypes.c_int64), ("half_steps", ctypes.c_int64),
                 ("kernel_launches", ctypes.c_int64), ("loop_ms", ctypes.c_double),
                 ("sparse_iterations", ctypes.c_int64), ("dense_iterations", ctypes.c_int64),
-                ("tiles_candidate", ctypes.c_int64), ("tiles_admitted", ctypes.c_int64),
+                ("tiles_candidate", ctypes.c_int64), ("tiles_admitted", ctypes.c_int64), ("tiles_exact", ctypes.c_int64),
                 ("tiles_total", ctypes.c_int64), ("omitted_bound", ctypes.c_double)]
 
 

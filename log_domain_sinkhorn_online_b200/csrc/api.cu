@@ -68,6 +68,7 @@ struct DevScalars {
 // block-sparse mode: device counters of one iteration
 struct SparseCtr {
     unsigned long long cand, adm;  // candidate and admitted tiles of the current mask
+    unsigned long long exact;      // candidates whose exact mass was evaluated
     unsigned work, pad;            // verification: dynamic row-block counter
     unsigned lohi[6];              // joint bounding box (order-preserving float bits)
 };
@@ -149,7 +150,7 @@ struct ot_plan {
     double *sp_tres = nullptr;
     SparseCtr *sc = nullptr;
     std::vector<uint8_t> iter_sparse;     // per launched iteration: 1 sparse, 0 dense
-    int64_t last_cand = 0, last_adm = 0;  // tiles of the last mask an iteration ran on
+    int64_t last_cand = 0, last_adm = 0, last_exact = 0;  // tiles of the last mask an iteration ran on
     bool adm_pending = false;             // its admitted count is still on the device
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
     cudaStream_t s_int = nullptr;
@@ -555,6 +556,7 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
     if (p->adm_pending) {
         p->last_cand = (int64_t)p->hs->sc_prev.cand;
         p->last_adm = (int64_t)p->hs->sc_prev.adm;
+        p->last_exact = (int64_t)p->hs->sc_prev.exact;
         p->adm_pending = false;
     }
     if (p->hs->st.stop) {
@@ -563,6 +565,7 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
     }
     const bool dense = (double)p->hs->sc.cand > p->sp_frac * (double)nb * (double)mb;
     p->last_cand = p->last_adm = (int64_t)p->hs->sc.cand;
+    p->last_exact = 0;
     if (dense) {
         OT_CU(launch_side(p, 0, par));
         if (!f_only) OT_CU(launch_side(p, 1, par));
@@ -576,6 +579,7 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         V.rowtab = p->sx.rowtab;
         V.pot = p->sf[par];
         V.pts = p->sx_pts;
+        V.exact = &p->sc->exact;
         V.prm = p->prm;
         V.rs = p->bsx;
         V.cs = p->bsy;
@@ -1081,6 +1085,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         OT_CU(cudaStreamSynchronize(p->s_int));
         p->last_cand = (int64_t)p->hs->sc_prev.cand;
         p->last_adm = (int64_t)p->hs->sc_prev.adm;
+        p->last_exact = (int64_t)p->hs->sc_prev.exact;
         p->adm_pending = false;
     }
     if (sparse) {  // back to the caller's order
@@ -1126,6 +1131,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         info->dense_iterations = dn_it;
         info->tiles_candidate = p->last_cand;
         info->tiles_admitted = p->last_adm;
+        info->tiles_exact = p->last_exact;
         info->tiles_total = sparse ? p->sp_nb * p->sp_mb : 0;
         info->omitted_bound = sparse ? p->sp_bound : 0.0;
     }

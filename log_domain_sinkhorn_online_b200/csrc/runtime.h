@@ -148,6 +148,7 @@ struct VerifyArgs {
     int64_t *cnt, *cnt_t;      // out: admitted per row block; in/out: per column block
     unsigned *work;            // dynamic row-block counter (zeroed before)
     unsigned long long *total; // admitted tiles (zeroed before)
+    unsigned long long *exact; // tiles whose exact mass was evaluated (zeroed before)
 };
 int sparse_blocks_per_sm(int which, int d, int rpt);  // which: 0 half-step, 1 verification
 cudaError_t launch_box(const float *p, int64_t cnt, int d, unsigned *lohi, cudaStream_t s);

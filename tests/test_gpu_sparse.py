@@ -106,6 +106,8 @@ def test_sparse_trajectory_matches_the_oracle(ot, orc, d, B, verify, n, m):
     assert abs(info.tiles_candidate - cand) <= near_s, (info.tiles_candidate, cand, near_s)
     assert abs(info.tiles_admitted - adm) <= near_all, (info.tiles_admitted, adm, near_all)
     assert info.tiles_admitted < NB * MB  # the mask is not trivial here
+    if verify:  # every admitted tile had its exact mass evaluated
+        assert info.tiles_admitted <= info.tiles_exact <= info.tiles_candidate
     assert abs(info.residual - r) <= 1e-3 * max(r, 1e-3)
     plan.close()
 
