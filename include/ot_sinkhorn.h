@@ -153,6 +153,9 @@ typedef struct ot_info {
                                   others fell below the threshold on a point-level bound) */
     int64_t tiles_total;       /* NB * MB block pairs */
     double omitted_bound;      /* bound on the row mass one mask omits: MB delta sum(a) */
+    double verify_ms;          /* with opt->timing: device time of the tile verifications */
+    double sparse_hs_ms;       /* with opt->timing: device time of the block-sparse half-steps */
+    int64_t sparse_hs_launches;/* with opt->timing: block-sparse half-step launches timed */
 } ot_info;
 
 /* Opaque plan: the pages' "row materializer built once", which captures the

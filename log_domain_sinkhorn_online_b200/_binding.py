@@ -56,7 +56,9 @@ class OtInfo(ctypes.Structure):
                 ("kernel_launches", ctypes.c_int64), ("loop_ms", ctypes.c_double),
                 ("sparse_iterations", ctypes.c_int64), ("dense_iterations", ctypes.c_int64),
                 ("tiles_candidate", ctypes.c_int64), ("tiles_admitted", ctypes.c_int64), ("tiles_exact", ctypes.c_int64),
-                ("tiles_total", ctypes.c_int64), ("omitted_bound", ctypes.c_double)]
+                ("tiles_total", ctypes.c_int64), ("omitted_bound", ctypes.c_double),
+                ("verify_ms", ctypes.c_double), ("sparse_hs_ms", ctypes.c_double),
+                ("sparse_hs_launches", ctypes.c_int64)]
 
 
 class OTError(RuntimeError):

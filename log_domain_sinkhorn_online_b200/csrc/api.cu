@@ -163,6 +163,12 @@ struct ot_plan {
     bool timing = false;
     std::vector<cudaEvent_t> tev;
     size_t tev_used = 0;
+    // block-sparse mode with timing: events around the verification and the
+    // sparse half-step launches
+    struct Marks {
+        std::vector<cudaEvent_t> ev;
+        size_t used = 0;
+    } tm_verify, tm_hs;
 };
 
 namespace {
@@ -172,6 +178,8 @@ void plan_free(ot_plan *p) {
     for (auto &gx : p->graph)
         if (gx) cudaGraphExecDestroy(gx);
     for (auto ev : p->tev) cudaEventDestroy(ev);
+    for (auto ev : p->tm_verify.ev) cudaEventDestroy(ev);
+    for (auto ev : p->tm_hs.ev) cudaEventDestroy(ev);
     // the workspaces and the stream go back to the pool once the plan's work is done
     if (p->s_int) cudaStreamSynchronize(p->s_int);
     pool_device_free(p->ws, p->ws_bytes);
@@ -367,6 +375,29 @@ cudaError_t mark(ot_plan *p) {
         p->tev.push_back(ev);
     }
     return cudaEventRecord(p->tev[p->tev_used++], p->s_int);
+}
+
+// The same for one kind of kernel (pairs of events around its launches).
+cudaError_t mark_in(ot_plan *p, ot_plan::Marks &mk) {
+    if (!p->timing) return cudaSuccess;
+    if (mk.used == mk.ev.size()) {
+        cudaEvent_t ev;
+        cudaError_t e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) return e;
+        mk.ev.push_back(ev);
+    }
+    return cudaEventRecord(mk.ev[mk.used++], p->s_int);
+}
+
+int sum_marks(const ot_plan::Marks &mk, double *ms_out) {
+    double t = 0.0;
+    for (size_t e = 0; e + 1 < mk.used; e += 2) {
+        float ms = 0.0f;
+        OT_CU(cudaEventElapsedTime(&ms, mk.ev[e], mk.ev[e + 1]));
+        t += ms;
+    }
+    *ms_out = t;
+    return OT_OK;
 }
 
 // One half-step: side 0 updates f (rows x, columns y), side 1 updates g.
@@ -593,19 +624,25 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         V.cnt_t = p->cnt_t;
         V.work = &p->sc->work;
         V.total = &p->sc->adm;
+        OT_CU(mark_in(p, p->tm_verify));
         OT_CU(launch_verify(d, rpt, V, p->sp_vgrid, s));
+        OT_CU(mark_in(p, p->tm_verify));
         p->launches += 1;
         p->adm_pending = true;
     }
     OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
     OT_CU(launch_mask_list(p->mask, nb, mb, p->ptr, p->lst, s));
+    OT_CU(mark_in(p, p->tm_hs));
     OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 0, par), p->sp_grid[0], s));
+    OT_CU(mark_in(p, p->tm_hs));
     p->launches += 5;
     if (!f_only) {
         OT_CU(launch_transpose_bytes(p->mask, nb, mb, p->mask_t, s));
         OT_CU(launch_row_ptr_scan(p->cnt_t, mb, p->ptr_t, p->sp_scan, s));
         OT_CU(launch_mask_list(p->mask_t, mb, nb, p->ptr_t, p->lst_t, s));
+        OT_CU(mark_in(p, p->tm_hs));
         OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 1, par), p->sp_grid[1], s));
+        OT_CU(mark_in(p, p->tm_hs));
         p->launches += 6;
         p->iter_sparse.push_back(1);
     }
@@ -1134,6 +1171,9 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         info->tiles_exact = p->last_exact;
         info->tiles_total = sparse ? p->sp_nb * p->sp_mb : 0;
         info->omitted_bound = sparse ? p->sp_bound : 0.0;
+        if ((rc = sum_marks(p->tm_verify, &info->verify_ms)) != OT_OK) return rc;
+        if ((rc = sum_marks(p->tm_hs, &info->sparse_hs_ms)) != OT_OK) return rc;
+        info->sparse_hs_launches = (int64_t)(p->tm_hs.used / 2);
     }
     if (plan_out) {
         *plan_out = p;

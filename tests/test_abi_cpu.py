@@ -49,7 +49,7 @@ def test_version_and_defaults(B):
 
 def test_struct_sizes_match_header_layout(B):
     assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4 + 4 * 4 + 2 * 8
-    assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8 + 6 * 8 + 8
+    assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8 + 6 * 8 + 8 + 3 * 8
 
 
 FAKE = 0x1000  # never dereferenced: validation fails first
