@@ -145,7 +145,11 @@ struct VerifyArgs {
     int64_t rows, cols_pad, nb, mb;
     double l2_delta;
     uint8_t *mask;             // candidates in, admitted tiles out
-    int64_t *cnt, *cnt_t;      // out: admitted per row block; in/out: per column block
+    const int64_t *cptr;       // candidates of row block p: clist[cptr[p] .. cptr[p+1])
+    const int *clist;
+    int segs;                  // work items per row block
+    int64_t *cnt, *cnt_t;      // out: admitted per row block (zeroed before); in/out: per
+                               // column block
     unsigned *work;            // dynamic row-block counter (zeroed before)
     unsigned long long *total; // admitted tiles (zeroed before)
     unsigned long long *exact; // tiles whose exact mass was evaluated (zeroed before)

@@ -254,8 +254,10 @@ __global__ void __launch_bounds__(kScreenThreads) screen_kernel(ScreenArgs S) {
 }
 
 // ------------------------------------------------------------ verification
-// One block per row block (claimed dynamically). The block lists the row's
-// candidates in windows of kVfWindow columns and tests each candidate tile q
+// Work items (row block p, segment of its candidate list; V.segs segments per
+// row block, claimed dynamically, so a row block with many candidates does not
+// leave a tail). The candidates come as compressed rows (cptr, clist) in
+// column order, taken kVfWindow at a time. Each candidate tile q is tested
 // against log2 rho = log2 delta + min(log2 amin_p, log2 bmin_q):
 //  1. a row-level bound, one warp per tile: with G_q the column block's
 //     largest potential and dist_i the distance from x_i to q's bounding box,
@@ -282,7 +284,6 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
     __shared__ __align__(16) float4 buf[kB];
     __shared__ int s_list[kVfWindow], s_exact[kVfWindow];
     __shared__ float s_xr[kB][3], s_fr[kB];
-    __shared__ int s_wcnt[kHsThreads / 32];
     __shared__ int s_nexact;
     __shared__ float s_max[kHsThreads / 32], s_sum[kHsThreads / 32];
     __shared__ long long s_next;
@@ -291,8 +292,20 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
     const double kappa = V.prm->kappa, c = V.prm->c;
     const float kf = (float)kappa, cf = (float)c;
 
-    long long p = blockIdx.x;
-    while (p < V.nb) {
+    const long long n_items = V.nb * (long long)V.segs;
+    long long item = blockIdx.x;
+    while (item < n_items) {
+        const long long p = item / V.segs;
+        const int seg = (int)(item % V.segs);
+        const int64_t c0 = V.cptr[p], cp = V.cptr[p + 1] - c0;
+        const int64_t k0 = c0 + cp * seg / V.segs, k1 = c0 + cp * (seg + 1) / V.segs;
+        if (k0 == k1) {  // nothing to verify in this segment
+            if (tid == 0) s_next = (long long)gridDim.x + (long long)atomicAdd(V.work, 1u);
+            __syncthreads();
+            item = s_next;
+            __syncthreads();
+            continue;
+        }
         // the block's points (caller's coordinates) and potentials for the row-level bound
         for (int r = tid; r < kB; r += kHsThreads) {
             const int64_t row = p * kB + r;
@@ -314,39 +327,16 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
             base[k] = row < V.rows ? kappa * (double)V.pot[row] - c * kappa * nrm : -INFINITY;
         }
         int64_t kept = 0;
-        for (int64_t w0 = 0; w0 < V.mb; w0 += kVfWindow) {
-            // list this window's candidates in column order
-            constexpr int kPer = kVfWindow / kHsThreads;
-            int mine = 0;
-            uint8_t flags[kPer];
-#pragma unroll
-            for (int u = 0; u < kPer; ++u) {
-                const int64_t q = w0 + tid * kPer + u;
-                flags[u] = q < V.mb ? V.mask[p * V.mb + q] : 0;
-                mine += flags[u] != 0;
-            }
-            int incl = mine;
-            for (int off = 1; off < 32; off <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            if (lane == 31) s_wcnt[warp] = incl;
-            __syncthreads();
-            int woff = 0, total = 0;
-            for (int k = 0; k < kHsThreads / 32; ++k) {
-                if (k < warp) woff += s_wcnt[k];
-                total += s_wcnt[k];
-            }
-            int pos = woff + incl - mine;
-#pragma unroll
-            for (int u = 0; u < kPer; ++u)
-                if (flags[u]) s_list[pos++] = (int)(tid * kPer + u);
+        for (int64_t w0 = k0; w0 < k1; w0 += kVfWindow) {
+            // this window of the segment's candidate columns
+            const int total = (int)min((int64_t)kVfWindow, k1 - w0);
+            for (int t = tid; t < total; t += kHsThreads) s_list[t] = V.clist[w0 + t];
             if (tid == 0) s_nexact = 0;
             __syncthreads();
 
             // 1. row-level bound, one warp per candidate tile
             for (int t = warp; t < total; t += kHsThreads / 32) {
-                const int64_t q = w0 + s_list[t];
+                const int64_t q = s_list[t];
                 const BlockSum &cq = V.cs[q];
                 float lo[3], hi[3];
 #pragma unroll
@@ -394,7 +384,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
 
             // 2. exact mass, one block per remaining tile
             for (int t = 0; t < n_exact; ++t) {
-                const int64_t q = w0 + s_exact[t];
+                const int64_t q = s_exact[t];
                 for (int u = tid; u < kB; u += kHsThreads) {
                     const int64_t col = q * kB + u;
                     buf[u] = col < V.cols_pad ? V.coltab[col] : dead4(u);
@@ -453,15 +443,17 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
                     }
                 }
             }
-            __syncthreads();  // s_list and s_wcnt are rewritten by the next window
+            __syncthreads();  // s_list and s_exact are rewritten by the next window
         }
         if (tid == 0) {
-            V.cnt[p] = kept;
-            if (kept) atomicAdd(V.total, (unsigned long long)kept);
+            if (kept) {
+                atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt + p), (unsigned long long)kept);
+                atomicAdd(V.total, (unsigned long long)kept);
+            }
             s_next = (long long)gridDim.x + (long long)atomicAdd(V.work, 1u);
         }
         __syncthreads();
-        p = s_next;
+        item = s_next;
         __syncthreads();
     }
 }
