@@ -3,9 +3,10 @@
 Tolerances (the readings are listed in the design doc):
  - potentials: max |f - f_ref| and |g - g_ref| <= 1e-4 * max_ij C_ij (the cost
    as used, i.e. scaled), -inf at the same (massless) entries;
- - plan entries at the GPU's potentials: |T - T_ref| <= 1e-5 * T_ref where
+ - plan entries of a plan built at given potentials (the oracle's, rounded to
+   float32, or seeded ones; never the GPU's): |T - T_ref| <= 1e-5 * T_ref where
    T_ref >= 1e-30, and T <= 1e-30 where T_ref < 1e-30;
- - marginal residual at the GPU's potentials: within 1e-5 (absolute; the
+ - marginal residual at the same given potentials: within 1e-5 (absolute; the
    residual of a unit-mass plan is at most 2);
  - min_row: thr within 1e-5 relative, the same argmin row, the same kept
    (i, j) entries except those within 1e-5 relative of thr (counted);
@@ -86,10 +87,12 @@ def csr_rows(row_ptr, col_idx, vals):
     return out
 
 
-def assert_csr(got, ref, thr, tol=ROW_TOL):
+def assert_csr(got, ref, thr, tol=ROW_TOL, band_tol=None):
     """got/ref: (row_ptr, col_idx, vals) as numpy arrays, thresholded at thr.
-    The kept sets agree except entries within tol (relative) of thr; values of
-    entries kept by both agree as plan entries. Returns the tie-band count."""
+    The kept sets agree except entries within band_tol (relative, default tol) of
+    thr; values of entries kept by both agree as plan entries (tol). Returns the
+    tie-band count."""
+    band_tol = tol if band_tol is None else band_tol
     g, r = csr_rows(*got), csr_rows(*ref)
     assert len(g) == len(r)
     band = 0
@@ -103,6 +106,24 @@ def assert_csr(got, ref, thr, tol=ROW_TOL):
         only_g = np.setdiff1d(np.arange(len(gc)), gi)
         only_r = np.setdiff1d(np.arange(len(rc)), ri)
         for v in list(gv[only_g]) + list(rv[only_r]):
-            assert abs(v - thr) <= tol * thr, f"row {i}: entry {v:.6e} kept by one side only, thr {thr:.6e}"
+            assert abs(v - thr) <= band_tol * thr, f"row {i}: entry {v:.6e} kept by one side only, thr {thr:.6e}"
             band += 1
     return band
+
+
+def f32(v):
+    """float64 copy of v rounded to float32: the potentials both sides are given."""
+    return np.asarray(v, np.float64).astype(np.float32).astype(np.float64)
+
+
+def plan_at(ot, w, f, g, **kw):
+    """A GPU plan at given potentials (warm start, no iteration), so that rows,
+    residuals, min_row and sparsify are compared with the oracle at potentials
+    that come from the oracle or from a seeded generator, never from the GPU."""
+    import torch
+    x, y, a, b = to_dev(w)
+    ft = torch.from_numpy(np.asarray(f, np.float32).copy()).cuda()
+    gt = torch.from_numpy(np.asarray(g, np.float32).copy()).cuda()
+    kw.setdefault("eps", w.eps)
+    kw.setdefault("scale", w.scale)
+    return ot.sinkhorn(x, y, a, b, n_iters=0, f=ft, g=gt, warm_start=True, **kw)

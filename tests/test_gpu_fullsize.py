@@ -2,14 +2,19 @@
 
 A full oracle trajectory is out of reach beyond the 8000-point workload, so each
 test runs the GPU at the workload's real size and launch shape and checks:
- - teacher-forced steps: one GPU iteration from the GPU's own state, against the
-   oracle's f-update on sampled rows (from the same g) and g-update on sampled
-   columns (from the GPU's new f) -- the sampled checks of "FlashSinkhorn 2",
-   sections 3.1 and B.2, used as a verifier;
- - plan entries, residuals and min_row at the GPU's potentials, in full where the
-   oracle can afford it (8000 x 8000), on sampled rows otherwise;
+ - single steps from a seeded state: one GPU f-update from a g drawn by the test,
+   against the oracle's f-update on sampled rows from the same g, and the same for
+   the g-update with the clouds' roles exchanged -- the sampled checks of
+   "FlashSinkhorn 2", sections 3.1 and B.2, used as a verifier;
+ - plan entries, residuals and min_row of a plan built at potentials that come
+   from the oracle (in full where the oracle can afford it, 8000 x 8000) or, at
+   the larger sizes, at sampled rows whose potentials the oracle computed from a
+   seeded g;
+ - properties of the GPU's own full-size solve (finite potentials, the reported
+   residual against the GPU's float64 one);
  - the captured scale: exact for "mean" (closed form) and for "max_cost" (the
    farthest point of y from any x is a vertex of y's convex hull).
+No oracle input comes from the GPU.
 """
 import numpy as np
 import pytest
@@ -48,47 +53,68 @@ def _max_sqdist_hull(x, y):
     return best
 
 
-def _teacher_forced(ot, orc, w, x, y, a, b, f0, g0, c, maxc, seed, **kw):
-    """One GPU iteration from (f0, g0) vs the oracle on sampled rows/columns."""
+def _seeded_g(w, seed, spread):
+    """A potential on the columns drawn by the test (not a solution)."""
+    return np.random.default_rng(seed).normal(0.0, spread, w.m).astype(np.float32).astype(np.float64)
+
+
+def _single_steps(ot, orc, w, c, maxc, seed, **kw):
+    """One GPU f-update from a seeded g against the oracle's f-update on sampled
+    rows; then the same with the clouds exchanged (the g-update's arithmetic).
+    Returns the oracle's potentials at the sampled rows and the seeded g."""
     import torch
-    p = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=1, f=f0.clone(), g=g0.clone(),
-                    warm_start=True, **kw)
-    torch.cuda.synchronize()
-    assert p.info.inv_scale_cost == pytest.approx(c, rel=1e-6)
+    from dataclasses import replace
     rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(w.n, size=min(SAMPLE, w.n), replace=False))
-    cols = np.sort(rng.choice(w.m, size=min(SAMPLE, w.m), replace=False))
-    g0n = g0.double().cpu().numpy()
-    f1 = p.f.double().cpu().numpy()
-    g1 = p.g.double().cpu().numpy()
-    f_ref = orc.f_step(w.x, w.y, w.a, g0n, c, w.eps, rows=rows)
-    g_ref = orc.g_step(w.x, w.y, w.b, f1, c, w.eps, cols=cols)
-    ef = H.assert_potentials(f1[rows], f_ref, maxc, what="f (teacher-forced)")
-    eg = H.assert_potentials(g1[cols], g_ref, maxc, what="g (teacher-forced)")
-    p.close()
-    return ef, eg
+    out = []
+    for side, ws in (("f", w), ("g", replace(w, x=w.y, y=w.x, a=w.b, b=w.a))):
+        g0 = _seeded_g(ws, seed + (side == "g"), 0.02 * maxc)
+        x, y, a, b = H.to_dev(ws)
+        p = ot.sinkhorn(x, y, a, b, eps=ws.eps, scale=ws.scale, n_iters=1,
+                        f=torch.zeros(ws.n, dtype=torch.float32, device="cuda"),
+                        g=torch.from_numpy(g0.astype(np.float32)).cuda(), warm_start=True, **kw)
+        torch.cuda.synchronize()
+        assert p.info.inv_scale_cost == pytest.approx(c, rel=1e-6)
+        rows = np.sort(rng.choice(ws.n, size=min(SAMPLE, ws.n), replace=False))
+        f1 = p.f.double().cpu().numpy()
+        f_ref = orc.f_step(ws.x, ws.y, ws.a, g0, c, ws.eps, rows=rows)
+        H.assert_potentials(f1[rows], f_ref, maxc, what=f"{side} (one step from a seeded state)")
+        p.close()
+        out.append((rows, f_ref, g0))
+    return out[0]
+
+
+def _plan_at_sampled_rows(ot, w, rows, f_rows, g0, **kw):
+    """A plan whose sampled rows carry the oracle's potentials (0 elsewhere)."""
+    f = np.zeros(w.n)
+    f[rows] = f_rows
+    return H.plan_at(ot, w, H.f32(f), H.f32(g0), **kw), H.f32(f)
 
 
 def test_w2_8000_full_path(ot, orc):
-    """The benchmarked workload, in the bench's launch shape: solve to tol / cap,
-    then the full oracle residual, min_row and rows at the GPU's potentials."""
+    """The benchmarked workload, in the bench's launch shape: the GPU's solve to
+    tol / cap (its in-loop residual against its own float64 residual), single
+    steps from a seeded state, then the full oracle residual, min_row, rows and
+    sparse plan of a plan at the oracle's potentials after 30 iterations."""
     import torch
     from log_domain_sinkhorn_online_b200 import workloads
     w = workloads.w2()
     x, y, a, b = H.to_dev(w)
-    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=w.n_iters, tol=w.tol)
-    c = plan.info.inv_scale_cost
+    solved = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=w.n_iters, tol=w.tol)
+    c = solved.info.inv_scale_cost
     xd, yd = w.x.astype(np.float64), w.y.astype(np.float64)
     mean = (xd ** 2).sum(1).mean() + (yd ** 2).sum(1).mean() - 2 * xd.mean(0) @ yd.mean(0)
     assert c == pytest.approx(1.0 / mean, rel=1e-9)
+    # the in-loop residual (float32 LSE) agrees with the GPU's float64 one
+    assert solved.info.residual == pytest.approx(solved.marginal_residual()[0], rel=1e-3)
+    solved.close()
     maxc = H.max_cost(w.x, w.y, c)
-    _teacher_forced(ot, orc, w, x, y, a, b, plan.f, plan.g, c, maxc, seed=1)
-    f, g = plan.f.double().cpu().numpy(), plan.g.double().cpu().numpy()
+    _single_steps(ot, orc, w, c, maxc, seed=1)
+    f_o, g_o, _, _ = orc.sinkhorn(w.x, w.y, w.a, w.b, c, w.eps, 30)
+    f, g = H.f32(f_o), H.f32(g_o)
+    plan = H.plan_at(ot, w, f, g)
     r = plan.marginal_residual()
     r_ref = orc.marginal_residual(w.x, w.y, w.a, w.b, f, g, c, w.eps)
     assert abs(r[0] - r_ref[0]) <= H.RES_TOL and abs(r[1] - r_ref[1]) <= H.RES_TOL
-    # the in-loop residual (float32 LSE) agrees with the float64 one
-    assert plan.info.residual == pytest.approx(r_ref[0], rel=1e-3)
     mr = plan.sparsify_min_row(block_rows=w.block_rows)
     ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps, block_rows=w.block_rows)
     H.assert_min_row(mr, ref)
@@ -105,19 +131,23 @@ def test_w2_8000_full_path(ot, orc):
     np.testing.assert_array_equal(np.diff(row_ptr), mr["counts"].cpu().numpy())
     col_idx, vals = csr["col_idx"].cpu().numpy(), csr["vals"].cpu().numpy()
     pick = np.arange(0, w.n, 397)
+    thr_ref = ref["thr"]  # each side keeps what reaches its own min_row threshold
     Tref = orc.materialize_rows(w.x, w.y, f, g, c, w.eps, pick)
-    ref_ptr = np.concatenate([[0], np.cumsum((Tref >= csr["thr"]).sum(1))])
-    ref_cols = np.concatenate([np.nonzero(r >= csr["thr"])[0] for r in Tref])
-    ref_vals = np.concatenate([r[r >= csr["thr"]] for r in Tref])
+    ref_ptr = np.concatenate([[0], np.cumsum((Tref >= thr_ref).sum(1))])
+    ref_cols = np.concatenate([np.nonzero(r >= thr_ref)[0] for r in Tref])
+    ref_vals = np.concatenate([r[r >= thr_ref] for r in Tref])
     got_ptr = np.concatenate([[0], np.cumsum([row_ptr[i + 1] - row_ptr[i] for i in pick])])
     got_cols = np.concatenate([col_idx[row_ptr[i]:row_ptr[i + 1]] for i in pick])
     got_vals = np.concatenate([vals[row_ptr[i]:row_ptr[i + 1]] for i in pick])
-    H.assert_csr((got_ptr, got_cols, got_vals), (ref_ptr, ref_cols, ref_vals), csr["thr"])
+    H.assert_csr((got_ptr, got_cols, got_vals), (ref_ptr, ref_cols, ref_vals), thr_ref,
+                 band_tol=2 * H.ROW_TOL)
+    plan.close()
 
 
 def test_w3_tensor_core_full_size(ot, orc):
-    """40000 x 50000, d = 50 on the tcgen05 path: 500 iterations, then a
-    teacher-forced step and sampled rows at the GPU's potentials."""
+    """40000 x 50000, d = 50 on the tcgen05 path: the 500-iteration solve (finite),
+    single steps from a seeded state, and sampled rows of a plan whose sampled
+    rows carry the oracle's potentials."""
     import torch
     from log_domain_sinkhorn_online_b200 import workloads
     w = workloads.w3()
@@ -126,27 +156,33 @@ def test_w3_tensor_core_full_size(ot, orc):
     c = plan.info.inv_scale_cost
     f, g = plan.f.double().cpu().numpy(), plan.g.double().cpu().numpy()
     assert np.isfinite(f).all() and np.isfinite(g).all()
+    plan.close()
     maxc = H.max_cost(w.x, w.y, c)
-    _teacher_forced(ot, orc, w, x, y, a, b, plan.f, plan.g, c, maxc, seed=3)
-    rows = np.sort(np.random.default_rng(5).choice(w.n, 16, replace=False)).astype(np.int64)
-    T = plan.materialize_rows(torch.from_numpy(rows).cuda()).double().cpu().numpy()
-    H.assert_entries(T, orc.materialize_rows(w.x, w.y, f, g, c, w.eps, rows))
+    rows, f_rows, g0 = _single_steps(ot, orc, w, c, maxc, seed=3)
+    rows, f_rows = rows[:16], f_rows[:16]
+    p, fs = _plan_at_sampled_rows(ot, w, rows, f_rows, g0)
+    T = p.materialize_rows(torch.from_numpy(rows.astype(np.int64)).cuda()).double().cpu().numpy()
+    H.assert_entries(T, orc.materialize_rows(w.x, w.y, fs, H.f32(g0), c, w.eps, rows))
+    p.close()
 
 
 def test_w4_million_points_step(ot, orc):
     """10^6 x 10^6 uniform vs 64 clusters at the final eps: two GPU iterations
-    from zero, then a teacher-forced step (sampled rows and columns)."""
+    from zero (finite), then single steps from a seeded state (sampled rows, both
+    directions)."""
     from log_domain_sinkhorn_online_b200 import workloads
     w = workloads.w4()
     x, y, a, b = H.to_dev(w)
     plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=2)
+    assert np.isfinite(plan.f.cpu().numpy()).all()
+    plan.close()
     maxc = _max_sqdist_hull(w.x, w.y)
-    _teacher_forced(ot, orc, w, x, y, a, b, plan.f, plan.g, 1.0, maxc, seed=4)
+    _single_steps(ot, orc, w, 1.0, maxc, seed=4)
 
 
 def test_w5_two_million_points_step_and_rows(ot, orc):
-    """2*10^6 spirals, scale max_cost (checked exactly), eps 1e-3: a teacher-forced
-    step, then one 4096-row block of the 65,536 rows (32.8 GB) and sampled rows."""
+    """2*10^6 spirals, scale max_cost (checked exactly), eps 1e-3: single steps from
+    a seeded state, then one 4096-row block of the 65,536 rows (32.8 GB) and sampled rows."""
     import torch
     from log_domain_sinkhorn_online_b200 import workloads
     w = workloads.w5()
@@ -156,12 +192,18 @@ def test_w5_two_million_points_step_and_rows(ot, orc):
     c = plan.info.inv_scale_cost
     # the pass runs in float32 on shifted coordinates: ~1e-7 relative
     assert c == pytest.approx(1.0 / mx, rel=1e-6)
-    _teacher_forced(ot, orc, w, x, y, a, b, plan.f, plan.g, c, 1.0, seed=5)
-    f, g = plan.f.double().cpu().numpy(), plan.g.double().cpu().numpy()
+    plan.close()
+    _single_steps(ot, orc, w, c, 1.0, seed=5)
+    # one 4096-row block of the 65,536 rows; the sampled rows among them carry the
+    # oracle's potentials (f-update from a seeded g), the others 0
+    pick = np.arange(0, w.block_rows, 128)
+    g0 = _seeded_g(w, 6, 0.02)
+    f_rows = orc.f_step(w.x, w.y, w.a, g0, c, w.eps, rows=w.rows[pick])
+    p, fs = _plan_at_sampled_rows(ot, w, w.rows[pick], f_rows, g0)
     rows = torch.from_numpy(w.rows[:w.block_rows]).cuda()
     out = torch.empty((w.block_rows, w.m), dtype=torch.float32, device="cuda")
-    plan.materialize_rows(rows, out=out)
-    pick = np.arange(0, w.block_rows, 128)
+    p.materialize_rows(rows, out=out)
     T = out[torch.from_numpy(pick).cuda()].double().cpu().numpy()
     del out
-    H.assert_entries(T, orc.materialize_rows(w.x, w.y, f, g, c, w.eps, w.rows[pick]))
+    H.assert_entries(T, orc.materialize_rows(w.x, w.y, fs, H.f32(g0), c, w.eps, w.rows[pick]))
+    p.close()

@@ -90,6 +90,10 @@ def test_w1_full_workload(ot, orc):
     f, g = _pots(plan)
     H.assert_potentials(f, f_ref, maxc, what="f")
     H.assert_potentials(g, g_ref, maxc, what="g")
+    plan.close()
+    # rows, min_row and residual at the oracle's potentials (given to both sides)
+    f, g = H.f32(f_ref), H.f32(g_ref)
+    plan = H.plan_at(ot, w, f, g)
     T = plan.materialize_rows(torch.arange(w.n, device="cuda")).double().cpu().numpy()
     T_ref = orc.dense_plan(w.x, w.y, f, g, c, w.eps)
     H.assert_entries(T, T_ref)
@@ -133,6 +137,9 @@ def test_massless_rows_and_columns(ot, orc):
     f, g = _pots(plan)
     H.assert_potentials(f, f_ref, maxc, what="f")
     H.assert_potentials(g, g_ref, maxc, what="g")
+    plan.close()
+    f, g = H.f32(f_ref), H.f32(g_ref)
+    plan = H.plan_at(ot, w, f, g)
     mr = plan.sparsify_min_row(block_rows=333)
     ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)
     H.assert_min_row(mr, ref)
@@ -160,14 +167,17 @@ def test_no_graphs_same_result(ot, orc):
     assert torch.equal(p1.f, p2.f) and torch.equal(p1.g, p2.g)  # deterministic kernels
 
 
-def test_rows_and_residual_at_gpu_potentials(ot, orc):
+def test_rows_and_residual_at_given_potentials(ot, orc):
+    """Rows, residuals and min_row (several block sizes) of a plan at the
+    oracle's potentials after 60 iterations, against the oracle there."""
     import torch
     from log_domain_sinkhorn_online_b200 import workloads
     w = workloads.w2(n=3001, m=2777)
-    x, y, a, b = H.to_dev(w)
-    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=60)
-    f, g = _pots(plan)
-    c = plan.info.inv_scale_cost
+    c = orc.inv_scale_cost(w.x, w.y, w.scale)
+    f_ref, g_ref, _, _ = orc.sinkhorn(w.x, w.y, w.a, w.b, c, w.eps, 60)
+    f, g = H.f32(f_ref), H.f32(g_ref)
+    plan = H.plan_at(ot, w, f, g)
+    assert plan.info.inv_scale_cost == pytest.approx(c, rel=2e-7)
     rows = np.array([0, 1, 1023, 1024, 2047, 3000, 5, 5], dtype=np.int64)
     T = plan.materialize_rows(torch.from_numpy(rows).cuda()).double().cpu().numpy()
     H.assert_entries(T, orc.materialize_rows(w.x, w.y, f, g, c, w.eps, rows))
@@ -182,39 +192,44 @@ def test_rows_and_residual_at_gpu_potentials(ot, orc):
         assert torch.equal(o["counts"], outs[0]["counts"])
 
 
-def _csr_case(ot):
+def _csr_case(ot, orc):
+    """A plan at the oracle's potentials (40 iterations), with massless rows."""
     w = _cloud(33, 517, 389, 2, scale="mean", eps=0.02)
     w.a = w.a.copy()
     w.a[[5, 100, 516]] = 0.0  # rows without mass keep nothing
-    x, y, a, b = H.to_dev(w)
-    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=40)
-    return w, plan
+    c = orc.inv_scale_cost(w.x, w.y, w.scale)
+    f_ref, g_ref, _, _ = orc.sinkhorn(w.x, w.y, w.a, w.b, c, w.eps, 40)
+    f, g = H.f32(f_ref), H.f32(g_ref)
+    return w, H.plan_at(ot, w, f, g), f, g, c
 
 
 def test_sparsify_csr_matches_oracle(ot, orc):
-    """Compressed-row sparsify at the GPU's potentials against the oracle's
-    thresholded plan at the same thr: the same kept entries outside the tie band,
-    values as plan entries, increasing columns; counts and nnz are min_row's."""
-    w, plan = _csr_case(ot)
+    """Compressed-row sparsify against the oracle's thresholded plan, both at the
+    oracle's potentials and each at its own min_row threshold: the same kept
+    entries outside the tie band, values as plan entries, increasing columns;
+    counts and nnz are min_row's."""
+    w, plan, f, g, c = _csr_case(ot, orc)
     mr = plan.sparsify_min_row()
     csr = plan.sparsify_csr()
     assert csr["thr"] == mr["thr"] and csr["nnz"] == mr["nnz"]
     row_ptr = csr["row_ptr"].cpu().numpy()
     np.testing.assert_array_equal(np.diff(row_ptr), mr["counts"].cpu().numpy())
     assert all(row_ptr[i + 1] == row_ptr[i] for i in (5, 100, 516))
-    f, g = _pots(plan)
-    ref = orc.sparsify_csr(w.x, w.y, w.a, f, g, plan.info.inv_scale_cost, w.eps, csr["thr"])
+    thr_ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)["thr"]
+    assert abs(csr["thr"] - thr_ref) <= H.ROW_TOL * thr_ref
+    ref = orc.sparsify_csr(w.x, w.y, w.a, f, g, c, w.eps, thr_ref)
+    # each side thresholds at its own thr (within 1e-5 of the other): band 2e-5
     band = H.assert_csr((row_ptr, csr["col_idx"].cpu().numpy(), csr["vals"].cpu().numpy()), ref,
-                        csr["thr"])
+                        thr_ref, band_tol=2 * H.ROW_TOL)
     assert band <= max(2, csr["nnz"] // 1000)
     plan.close()
 
 
-def test_sparsify_csr_block_rows_and_threshold(ot):
+def test_sparsify_csr_block_rows_and_threshold(ot, orc):
     """block_rows never changes the output (bit for bit); a lower threshold keeps
     a superset; a capacity below nnz is an overflow that reports nnz."""
     import torch
-    w, plan = _csr_case(ot)
+    w, plan, _, _, _ = _csr_case(ot, orc)
     outs = [plan.sparsify_csr(block_rows=br) for br in (0, 1, 7, 64)]
     for o in outs[1:]:
         for k in ("row_ptr", "col_idx", "vals"):
@@ -247,15 +262,18 @@ def test_dynamic_work_items_are_deterministic(ot, d, loop):
 def test_sparsify_csr_generic_d(ot, orc):
     """The compressed-row sparsify on the generic-d entry path (d = 5)."""
     w = _cloud(61, 301, 257, 5, scale="max_cost", eps=0.03)
-    x, y, a, b = H.to_dev(w)
-    plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=25)
+    c = orc.inv_scale_cost(w.x, w.y, w.scale)
+    f_ref, g_ref, _, _ = orc.sinkhorn(w.x, w.y, w.a, w.b, c, w.eps, 25)
+    f, g = H.f32(f_ref), H.f32(g_ref)
+    plan = H.plan_at(ot, w, f, g)
     csr = plan.sparsify_csr(block_rows=64)
     mr = plan.sparsify_min_row()
     assert csr["nnz"] == mr["nnz"]
-    f, g = _pots(plan)
-    ref = orc.sparsify_csr(w.x, w.y, w.a, f, g, plan.info.inv_scale_cost, w.eps, csr["thr"])
+    thr_ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)["thr"]
+    assert abs(csr["thr"] - thr_ref) <= H.ROW_TOL * thr_ref
+    ref = orc.sparsify_csr(w.x, w.y, w.a, f, g, c, w.eps, thr_ref)
     band = H.assert_csr((csr["row_ptr"].cpu().numpy(), csr["col_idx"].cpu().numpy(),
-                         csr["vals"].cpu().numpy()), ref, csr["thr"])
+                         csr["vals"].cpu().numpy()), ref, thr_ref, band_tol=2 * H.ROW_TOL)
     assert band <= max(2, csr["nnz"] // 1000)
     plan.close()
 
