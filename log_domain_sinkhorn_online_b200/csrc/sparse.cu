@@ -281,11 +281,12 @@ constexpr float kVfMargin = 0.05f;
 template <int D, int R>
 __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(VerifyArgs V) {
     constexpr int kB = kHsThreads * R;
-    __shared__ __align__(16) float4 buf[kB];
+    __shared__ __align__(16) float4 sbuf[2][kHsChunk];
     __shared__ int s_list[kVfWindow], s_exact[kVfWindow];
     __shared__ float s_xr[kB][3], s_fr[kB];
     __shared__ int s_nexact;
-    __shared__ float s_max[kHsThreads / 32], s_sum[kHsThreads / 32];
+    __shared__ float s_max[kHsChunk / kB][kHsThreads / 32], s_sum[kHsChunk / kB][kHsThreads / 32];
+    __shared__ int s_kept;
     __shared__ long long s_next;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float4 *rt4 = reinterpret_cast<const float4 *>(V.rowtab);
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
             const double nrm = (double)x.x * x.x + (double)x.y * x.y + (double)x.z * x.z + (double)x.w * x.w;
             base[k] = row < V.rows ? kappa * (double)V.pot[row] - c * kappa * nrm : -INFINITY;
         }
-        int64_t kept = 0;
+        if (tid == 0) s_kept = 0;
         for (int64_t w0 = k0; w0 < k1; w0 += kVfWindow) {
             // this window of the segment's candidate columns
             const int total = (int)min((int64_t)kVfWindow, k1 - w0);
@@ -382,61 +383,91 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
             const int n_exact = s_nexact;
             if (tid == 0 && n_exact) atomicAdd(V.exact, (unsigned long long)n_exact);
 
-            // 2. exact mass, one block per remaining tile
-            for (int t = 0; t < n_exact; ++t) {
-                const int64_t q = s_exact[t];
-                for (int u = tid; u < kB; u += kHsThreads) {
-                    const int64_t col = q * kB + u;
-                    buf[u] = col < V.cols_pad ? V.coltab[col] : dead4(u);
-                }
+            // 2. exact mass of the remaining tiles, 256 / B tiles per step (one
+            // 256-column chunk), the next step's columns loaded while this one runs
+            constexpr int kTpc = kHsChunk / kB;
+            const int nsteps = (n_exact + kTpc - 1) / kTpc;
+            auto fetch = [&](int step, int u) -> float4 {
+                const int t = step * kTpc + u / kB;
+                if (t >= n_exact) return dead4(u);
+                const int64_t col = (int64_t)s_exact[t] * kB + (u % kB);
+                return col < V.cols_pad ? V.coltab[col] : dead4(u);
+            };
+            float4 p0 = make_float4(0.f, 0.f, 0.f, 0.f), p1 = p0;
+            if (nsteps > 0) {
+                p0 = fetch(0, tid);
+                p1 = fetch(0, tid + kHsThreads);
+            }
+            for (int step = 0; step < nsteps; ++step) {
+                float4 *buf = sbuf[step & 1];
+                buf[tid] = p0;
+                buf[tid + kHsThreads] = p1;
                 __syncthreads();
-                float m[R], tot[R];
-                float2 nm[R], acc[R], acc2[R];
-#pragma unroll
-                for (int k = 0; k < R; ++k) {
-                    m[k] = kNegBig;
-                    nm[k] = make_float2(-kNegBig, -kNegBig);
-                    acc[k] = acc2[k] = make_float2(0.f, 0.f);
-                    tot[k] = 0.f;
+                if (step + 1 < nsteps) {
+                    p0 = fetch(step + 1, tid);
+                    p1 = fetch(step + 1, tid + kHsThreads);
                 }
+                float wv[kTpc][R];
+                float tv[kTpc][R];
+#pragma unroll
+                for (int tt = 0; tt < kTpc; ++tt) {
+                    float m[R], tot[R];
+                    float2 nm[R], acc[R], acc2[R];
+#pragma unroll
+                    for (int k = 0; k < R; ++k) {
+                        m[k] = kNegBig;
+                        nm[k] = make_float2(-kNegBig, -kNegBig);
+                        acc[k] = acc2[k] = make_float2(0.f, 0.f);
+                        tot[k] = 0.f;
+                    }
+                    if (step * kTpc + tt < n_exact) {
 #pragma unroll 1
-                for (int j = 0; j < kB; j += 8) {
-                    float4 v[8];
+                        for (int j = 0; j < kB; j += 8) {
+                            float4 v[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) v[u] = buf[j + u];
-                    lowd_step8<D, R, true>(v, xd, m, nm, acc, acc2, tot);
-                }
-                float wv[R], wmax = -INFINITY;
+                            for (int u = 0; u < 8; ++u) v[u] = buf[tt * kB + j + u];
+                            lowd_step8<D, R, true>(v, xd, m, nm, acc, acc2, tot);
+                        }
+                    }
+                    float wmax = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < R; ++k) {
-                    tot[k] += (acc[k].x + acc[k].y) + (acc2[k].x + acc2[k].y);
-                    wv[k] = (tot[k] > 0.f && base[k] != -INFINITY) ? (float)(base[k] + (double)m[k])
-                                                                    : -INFINITY;
-                    wmax = fmaxf(wmax, wv[k]);
+                    for (int k = 0; k < R; ++k) {
+                        tot[k] += (acc[k].x + acc[k].y) + (acc2[k].x + acc2[k].y);
+                        tv[tt][k] = tot[k];
+                        wv[tt][k] = (tot[k] > 0.f && base[k] != -INFINITY)
+                                        ? (float)(base[k] + (double)m[k]) : -INFINITY;
+                        wmax = fmaxf(wmax, wv[tt][k]);
+                    }
+                    for (int off = 16; off > 0; off >>= 1)
+                        wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, off));
+                    if (lane == 0) s_max[tt][warp] = wmax;
                 }
-                for (int off = 16; off > 0; off >>= 1)
-                    wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, off));
-                if (lane == 0) s_max[warp] = wmax;
                 __syncthreads();
-                float W = s_max[0];
-                for (int k = 1; k < kHsThreads / 32; ++k) W = fmaxf(W, s_max[k]);
-                float sum = 0.f;
-                if (W != -INFINITY) {
+                float W[kTpc];
 #pragma unroll
-                    for (int k = 0; k < R; ++k)
-                        if (wv[k] != -INFINITY) sum += tot[k] * ex2_approx(wv[k] - W);
+                for (int tt = 0; tt < kTpc; ++tt) {
+                    W[tt] = s_max[tt][0];
+                    for (int k = 1; k < kHsThreads / 32; ++k) W[tt] = fmaxf(W[tt], s_max[tt][k]);
+                    float sum = 0.f;
+                    if (W[tt] != -INFINITY) {
+#pragma unroll
+                        for (int k = 0; k < R; ++k)
+                            if (wv[tt][k] != -INFINITY) sum += tv[tt][k] * ex2_approx(wv[tt][k] - W[tt]);
+                    }
+                    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                    if (lane == 0) s_sum[tt][warp] = sum;
                 }
-                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                if (lane == 0) s_sum[warp] = sum;
                 __syncthreads();
-                if (tid == 0) {
+                if (tid < kTpc && step * kTpc + tid < n_exact) {
+                    const int tt = tid;
+                    const int64_t q = s_exact[step * kTpc + tt];
                     float S = 0.f;
-                    for (int k = 0; k < kHsThreads / 32; ++k) S += s_sum[k];
-                    const double lm = (W == -INFINITY || !(S > 0.f)) ? -INFINITY
-                                                                      : (double)W + log2((double)S);
+                    for (int k = 0; k < kHsThreads / 32; ++k) S += s_sum[tt][k];
+                    const double lm = (W[tt] == -INFINITY || !(S > 0.f)) ? -INFINITY
+                                                                          : (double)W[tt] + log2((double)S);
                     const double lrho = V.l2_delta + fmin(V.rs[p].l2w, V.cs[q].l2w);
                     if (lm > lrho) {
-                        ++kept;
+                        atomicAdd(&s_kept, 1);
                     } else {
                         V.mask[p * V.mb + q] = 0;
                         atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt_t + q), ~0ull);
@@ -445,7 +476,9 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
             }
             __syncthreads();  // s_list and s_exact are rewritten by the next window
         }
+        __syncthreads();
         if (tid == 0) {
+            const int kept = s_kept;
             if (kept) {
                 atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt + p), (unsigned long long)kept);
                 atomicAdd(V.total, (unsigned long long)kept);
