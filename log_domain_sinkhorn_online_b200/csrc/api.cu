@@ -473,7 +473,8 @@ int sparse_setup(ot_plan *p, const ot_options &o, double tol, bool warm) {
         return r;
     };
     const int64_t n2x = pow2(n), n2y = pow2(m);
-    const int64_t part = std::max((int64_t)p->sp_splits[0] * nb, (int64_t)p->sp_splits[1] * mb) * B;
+    const int64_t part = std::max({(int64_t)p->sp_splits[0] * nb, (int64_t)kVerifySegs * nb,
+                                   (int64_t)p->sp_splits[1] * mb}) * B;
     float *xs = nullptr, *ys = nullptr, *as = nullptr, *bs = nullptr;
     for (int pass = 0; pass < 2; ++pass) {
         Carver cv{pass ? p->ws_sp : nullptr};
@@ -614,13 +615,11 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
         OT_CU(launch_mask_list(p->mask, nb, mb, p->ptr, p->lst, s));
         OT_CU(cudaMemsetAsync(p->cnt, 0, sizeof(int64_t) * nb, s));
-        p->launches += 4;
         VerifyArgs V{};
         V.coltab = reinterpret_cast<const float4 *>(p->sy.coltab);
         V.rowtab = p->sx.rowtab;
         V.pot = p->sf[par];
         V.pts = p->sx_pts;
-        V.exact = &p->sc->exact;
         V.prm = p->prm;
         V.rs = p->bsx;
         V.cs = p->bsy;
@@ -635,20 +634,31 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         V.segs = kVerifySegs;
         V.cnt = p->cnt;
         V.cnt_t = p->cnt_t;
-        V.work = &p->sc->work;
         V.total = &p->sc->adm;
+        V.exact = &p->sc->exact;
+        // the verification and the f-update over the admitted tiles in one launch
+        HalfStep A = make_sparse_step(p, 0, par);
+        A.splits = kVerifySegs;
         OT_CU(mark_in(p, p->tm_verify));
-        OT_CU(launch_verify(d, rpt, V, p->sp_vgrid, s));
+        OT_CU(launch_verify(d, rpt, A, V, p->sp_vgrid, s));
         OT_CU(mark_in(p, p->tm_verify));
-        p->launches += 1;
         p->adm_pending = true;
+        // row blocks left without an admitted tile: f-update over every column
+        OT_CU(cudaMemsetAsync(&p->st->work[0], 0, sizeof(unsigned), s));
+        HalfStep Af = make_sparse_step(p, 0, par);
+        Af.sp_ptr = nullptr;
+        Af.sp_idx = nullptr;
+        Af.sp_fallback = p->cnt;
+        OT_CU(launch_halfstep_sparse(d, rpt, Af, p->sp_grid[0], s));
+        p->launches += 6;
+    } else {
+        OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
+        OT_CU(launch_mask_list(p->mask, nb, mb, p->ptr, p->lst, s));
+        OT_CU(mark_in(p, p->tm_hs));
+        OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 0, par), p->sp_grid[0], s));
+        OT_CU(mark_in(p, p->tm_hs));
+        p->launches += 5;
     }
-    OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
-    OT_CU(launch_mask_list(p->mask, nb, mb, p->ptr, p->lst, s));
-    OT_CU(mark_in(p, p->tm_hs));
-    OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 0, par), p->sp_grid[0], s));
-    OT_CU(mark_in(p, p->tm_hs));
-    p->launches += 5;
     if (!f_only) {
         OT_CU(launch_transpose_bytes(p->mask, nb, mb, p->mask_t, s));
         OT_CU(launch_row_ptr_scan(p->cnt_t, mb, p->ptr_t, p->sp_scan, s));

@@ -90,6 +90,7 @@ struct HalfStep {
     const int64_t *sp_ptr;
     const int *sp_idx;
     int sp_coltiles;
+    const int64_t *sp_fallback;  // non-null: only blocks t with sp_fallback[t] == 0 are updated
 };
 
 // ------------------------------------------------------ device helpers --

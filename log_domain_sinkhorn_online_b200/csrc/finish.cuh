@@ -68,8 +68,11 @@ __device__ __forceinline__ void tile_sync() {
 // Merge the column splits of one row tile; run by the block that finishes a
 // tile last. Every one of the THREADS participating threads (tid < THREADS)
 // must call it.
+// skip_if_zero (block-sparse verification): when skip_if_zero[tile] == 0 the
+// tile is left to a later launch (its ticket is reset, nothing is written).
 template <int THREADS, int TILE, int BAR>
-__device__ void finish_tile(const HalfStep &A, int tile, int tid, double *s_red, int *s_flag) {
+__device__ void finish_tile(const HalfStep &A, int tile, int tid, double *s_red, int *s_flag,
+                            const int64_t *skip_if_zero = nullptr) {
     __threadfence();
     tile_sync<THREADS, BAR>();
     if (tid == 0) {
@@ -79,6 +82,11 @@ __device__ void finish_tile(const HalfStep &A, int tile, int tid, double *s_red,
     tile_sync<THREADS, BAR>();
     if (!*s_flag) return;
     __threadfence();
+    if (skip_if_zero && __ldcg(skip_if_zero + tile) == 0) {
+        tile_sync<THREADS, BAR>();  // every thread has read the count
+        if (tid == 0) A.tile_cnt[tile] = 0;
+        return;
+    }
 
     const double eps = A.prm->eps, kappa = A.prm->kappa, c = A.prm->c, tol = A.prm->tol;
     const int64_t stride = (int64_t)A.tiles * TILE;

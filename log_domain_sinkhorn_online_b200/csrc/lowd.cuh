@@ -188,8 +188,8 @@ __device__ __forceinline__ void sparse_item(const HalfStep &A, int tile, int spl
         tot[k] = 0.f;
     }
 
-    const int64_t lp0 = A.sp_ptr[tile];
-    const int64_t cnt_p = A.sp_ptr[tile + 1] - lp0;
+    const int64_t lp0 = A.sp_ptr ? A.sp_ptr[tile] : 0;
+    const int64_t cnt_p = A.sp_ptr ? A.sp_ptr[tile + 1] - lp0 : 0;  // no list: every tile
     const int64_t cnt = cnt_p > 0 ? cnt_p : (int64_t)A.sp_coltiles;
     const int64_t k0 = cnt * split / A.splits, k1 = cnt * (split + 1) / A.splits;
     const int nch = (int)((k1 - k0 + kTpc - 1) / kTpc);

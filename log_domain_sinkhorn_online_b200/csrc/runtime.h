@@ -150,7 +150,6 @@ struct VerifyArgs {
     int segs;                  // work items per row block
     int64_t *cnt, *cnt_t;      // out: admitted per row block (zeroed before); in/out: per
                                // column block
-    unsigned *work;            // dynamic row-block counter (zeroed before)
     unsigned long long *total; // admitted tiles (zeroed before)
     unsigned long long *exact; // tiles whose exact mass was evaluated (zeroed before)
 };
@@ -167,7 +166,9 @@ cudaError_t launch_block_static(const float *ps, const float *ws, int64_t cnt, i
                                 BlockSum *bs, cudaStream_t s);
 cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, BlockSum *bs, cudaStream_t s);
 cudaError_t launch_screen(const ScreenArgs &S, cudaStream_t s);
-cudaError_t launch_verify(int d, int rpt, const VerifyArgs &V, int grid, cudaStream_t s);
+// the verification fused with the f-update (A: the f half-step, V.segs splits)
+cudaError_t launch_verify(int d, int rpt, const HalfStep &A, const VerifyArgs &V, int grid,
+                          cudaStream_t s);
 cudaError_t launch_mask_list(const uint8_t *mask, int64_t rows, int64_t cols, const int64_t *ptr,
                              int *list, cudaStream_t s);
 cudaError_t launch_transpose_bytes(const uint8_t *in, int64_t rows, int64_t cols, uint8_t *out,

@@ -279,7 +279,7 @@ constexpr int kVfWindow = 1024;
 constexpr float kVfMargin = 0.05f;
 
 template <int D, int R>
-__global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(VerifyArgs V) {
+__global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(HalfStep A, VerifyArgs V) {
     constexpr int kB = kHsThreads * R;
     __shared__ __align__(16) float4 sbuf[2][kHsChunk];
     __shared__ int s_list[kVfWindow], s_exact[kVfWindow];
@@ -287,26 +287,27 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
     __shared__ int s_nexact;
     __shared__ float s_max[kHsChunk / kB][kHsThreads / 32], s_sum[kHsChunk / kB][kHsThreads / 32];
     __shared__ int s_kept;
-    __shared__ long long s_next;
+    __shared__ long long s_next[2];
+    __shared__ uint8_t s_keep[kVfWindow];
+    __shared__ int s_wcnt[kHsThreads / 32];
+    __shared__ double s_red[kHsThreads / 32];
+    __shared__ int s_flag;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float4 *rt4 = reinterpret_cast<const float4 *>(V.rowtab);
     const double kappa = V.prm->kappa, c = V.prm->c;
     const float kf = (float)kappa, cf = (float)c;
+    if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;  // as in hs_lowd_kernel
+    if (ld_volatile(&A.st->stop)) return;
 
     const long long n_items = V.nb * (long long)V.segs;
     long long item = blockIdx.x;
-    while (item < n_items) {
+    for (int it = 0; item < n_items; ++it) {
+        if (tid == 0)
+            s_next[it & 1] = (long long)gridDim.x + (long long)atomicAdd(&A.st->work[A.side], 1u);
         const long long p = item / V.segs;
         const int seg = (int)(item % V.segs);
         const int64_t c0 = V.cptr[p], cp = V.cptr[p + 1] - c0;
         const int64_t k0 = c0 + cp * seg / V.segs, k1 = c0 + cp * (seg + 1) / V.segs;
-        if (k0 == k1) {  // nothing to verify in this segment
-            if (tid == 0) s_next = (long long)gridDim.x + (long long)atomicAdd(V.work, 1u);
-            __syncthreads();
-            item = s_next;
-            __syncthreads();
-            continue;
-        }
         // the block's points (caller's coordinates) and potentials for the row-level bound
         for (int r = tid; r < kB; r += kHsThreads) {
             const int64_t row = p * kB + r;
@@ -327,12 +328,18 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
             const double nrm = (double)x.x * x.x + (double)x.y * x.y + (double)x.z * x.z + (double)x.w * x.w;
             base[k] = row < V.rows ? kappa * (double)V.pot[row] - c * kappa * nrm : -INFINITY;
         }
+        // this segment's share of the f-update: (running max, sum) over its admitted tiles
+        float mr[R], tr[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            mr[k] = kNegBig;
+            tr[k] = 0.f;
+        }
         if (tid == 0) s_kept = 0;
         for (int64_t w0 = k0; w0 < k1; w0 += kVfWindow) {
             // this window of the segment's candidate columns
             const int total = (int)min((int64_t)kVfWindow, k1 - w0);
             for (int t = tid; t < total; t += kHsThreads) s_list[t] = V.clist[w0 + t];
-            if (tid == 0) s_nexact = 0;
             __syncthreads();
 
             // 1. row-level bound, one warp per candidate tile
@@ -371,15 +378,35 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
                     const double lb = mx == -INFINITY ? -INFINITY
                                                       : (double)mx + log2((double)sum) + cq.lncnt * 1.4426950408889634;
                     const double lrho = V.l2_delta + fmin(V.rs[p].l2w, cq.l2w);
-                    if (lb + kVfMargin <= lrho) {
+                    const bool keep = lb + kVfMargin > lrho;
+                    s_keep[t] = keep;
+                    if (!keep) {
                         V.mask[p * V.mb + q] = 0;
                         atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt_t + q), ~0ull);
-                    } else {
-                        s_exact[atomicAdd(&s_nexact, 1)] = s_list[t];
                     }
                 }
             }
             __syncthreads();
+            {   // the survivors in list order (the f-update sums its tiles in a fixed order)
+                constexpr int kPer = kVfWindow / kHsThreads;
+                int mine = 0;
+#pragma unroll
+                for (int u = 0; u < kPer; ++u) mine += (tid * kPer + u < total) && s_keep[tid * kPer + u];
+                int incl = mine;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                if (lane == 31) s_wcnt[warp] = incl;
+                __syncthreads();
+                int pos = incl - mine;
+                for (int k = 0; k < warp; ++k) pos += s_wcnt[k];
+#pragma unroll
+                for (int u = 0; u < kPer; ++u)
+                    if ((tid * kPer + u < total) && s_keep[tid * kPer + u]) s_exact[pos++] = s_list[tid * kPer + u];
+                if (tid == kHsThreads - 1) s_nexact = pos;
+                __syncthreads();
+            }
             const int n_exact = s_nexact;
             if (tid == 0 && n_exact) atomicAdd(V.exact, (unsigned long long)n_exact);
 
@@ -408,7 +435,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
                     p1 = fetch(step + 1, tid + kHsThreads);
                 }
                 float wv[kTpc][R];
-                float tv[kTpc][R];
+                float tv[kTpc][R], mv[kTpc][R];
 #pragma unroll
                 for (int tt = 0; tt < kTpc; ++tt) {
                     float m[R], tot[R];
@@ -434,6 +461,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
                     for (int k = 0; k < R; ++k) {
                         tot[k] += (acc[k].x + acc[k].y) + (acc2[k].x + acc2[k].y);
                         tv[tt][k] = tot[k];
+                        mv[tt][k] = m[k];
                         wv[tt][k] = (tot[k] > 0.f && base[k] != -INFINITY)
                                         ? (float)(base[k] + (double)m[k]) : -INFINITY;
                         wmax = fmaxf(wmax, wv[tt][k]);
@@ -458,17 +486,28 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
                     if (lane == 0) s_sum[tt][warp] = sum;
                 }
                 __syncthreads();
-                if (tid < kTpc && step * kTpc + tid < n_exact) {
-                    const int tt = tid;
+#pragma unroll
+                for (int tt = 0; tt < kTpc; ++tt) {
+                    if (step * kTpc + tt >= n_exact) continue;
                     const int64_t q = s_exact[step * kTpc + tt];
                     float S = 0.f;
                     for (int k = 0; k < kHsThreads / 32; ++k) S += s_sum[tt][k];
                     const double lm = (W[tt] == -INFINITY || !(S > 0.f)) ? -INFINITY
                                                                           : (double)W[tt] + log2((double)S);
                     const double lrho = V.l2_delta + fmin(V.rs[p].l2w, V.cs[q].l2w);
-                    if (lm > lrho) {
-                        atomicAdd(&s_kept, 1);
-                    } else {
+                    if (lm > lrho) {  // admitted: the tile joins this segment's f-update
+#pragma unroll
+                        for (int k = 0; k < R; ++k) {
+                            if (!(tv[tt][k] > 0.f)) continue;
+                            if (mv[tt][k] > mr[k]) {
+                                tr[k] = tr[k] * ex2_approx(mr[k] - mv[tt][k]) + tv[tt][k];
+                                mr[k] = mv[tt][k];
+                            } else {
+                                tr[k] += tv[tt][k] * ex2_approx(mv[tt][k] - mr[k]);
+                            }
+                        }
+                        if (tid == 0) ++s_kept;
+                    } else if (tid == 0) {
                         V.mask[p * V.mb + q] = 0;
                         atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt_t + q), ~0ull);
                     }
@@ -483,11 +522,18 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) verify_kernel(Veri
                 atomicAdd(reinterpret_cast<unsigned long long *>(V.cnt + p), (unsigned long long)kept);
                 atomicAdd(V.total, (unsigned long long)kept);
             }
-            s_next = (long long)gridDim.x + (long long)atomicAdd(V.work, 1u);
         }
+        const int64_t stride = (int64_t)A.tiles * kB;
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t row = p * kB + k * kHsThreads + tid;
+            if (row < A.rows) A.part[seg * stride + row] = make_float2(mr[k], tr[k]);
+        }
+        // the last segment merges; a row block left with no admitted tile is
+        // skipped here and updated over every column by the fallback launch
+        finish_tile<kHsThreads, kB, 0>(A, (int)p, tid, s_red, &s_flag, V.cnt);
         __syncthreads();
-        item = s_next;
-        __syncthreads();
+        item = s_next[it & 1];
     }
 }
 
@@ -556,6 +602,11 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 4 : 8) hs_sparse_kernel(H
             s_next[it & 1] = (long long)gridDim.x + (long long)atomicAdd(&A.st->work[A.side], 1u);
         const int tile = (int)(item / A.splits);
         const int split = (int)(item % A.splits);
+        if (A.sp_fallback && __ldcg(A.sp_fallback + tile) != 0) {  // not a fallback block
+            __syncthreads();
+            item = s_next[it & 1];
+            continue;
+        }
         sparse_item<D, R>(A, tile, split, sm);
         finish_tile<kHsThreads, kHsThreads * R, 0>(A, tile, threadIdx.x, s_red, &s_flag);
         __syncthreads();
@@ -573,9 +624,9 @@ static const void *sparse_fn(int d) {
 
 template <int R>
 static const void *verify_fn(int d) {
-    if (d == 1) return (const void *)verify_kernel<1, R>;
-    if (d == 2) return (const void *)verify_kernel<2, R>;
-    return (const void *)verify_kernel<3, R>;
+    if (d == 1) return (const void *)hs_verify_kernel<1, R>;
+    if (d == 2) return (const void *)hs_verify_kernel<2, R>;
+    return (const void *)hs_verify_kernel<3, R>;
 }
 
 static const void *sparse_kernel_fn(int which, int d, int rpt) {
@@ -648,10 +699,11 @@ cudaError_t launch_screen(const ScreenArgs &S, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_verify(int d, int rpt, const VerifyArgs &V, int grid, cudaStream_t s) {
+cudaError_t launch_verify(int d, int rpt, const HalfStep &A, const VerifyArgs &V, int grid,
+                          cudaStream_t s) {
     const void *fn = sparse_kernel_fn(1, d, rpt);
     if (!fn) return cudaErrorInvalidValue;
-    void *args[] = {(void *)&V};
+    void *args[] = {(void *)&A, (void *)&V};
     return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(kHsThreads), args, 0, s);
 }
 
