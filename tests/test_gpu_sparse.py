@@ -208,3 +208,31 @@ def test_rows_after_a_sparse_solve_use_the_callers_order(ot, orc):
     big = T_ref > 1e-20
     assert np.all(rel[big] <= 2 * H.POT_TOL * H.max_cost(w.x, w.y, 1.0) / w.eps * 1.01)
     plan.close()
+
+
+def test_blocks_without_admitted_tiles_fall_back_to_every_column(ot, orc):
+    """Warm start in which the columns of one cluster carry no mass (g = -50):
+    the row blocks near that cluster keep no tile (their screen or verification
+    rejects everything), so their f-update runs over every column, while the other
+    row blocks stay sparse -- against the oracle's block-sparse solve."""
+    from log_domain_sinkhorn_online_b200.workloads import Workload
+    rng = np.random.default_rng(31)
+    n, m = 3000, 2600
+    x = rng.random((n, 3)).astype(np.float32)
+    y = np.concatenate([rng.random((m // 2, 3)) * 0.2, 0.8 + rng.random((m - m // 2, 3)) * 0.2])
+    y = y.astype(np.float32)
+    w = Workload("two_clusters", x, y, np.full(n, 1 / n, np.float32), np.full(m, 1 / m, np.float32),
+                 eps=1e-3, scale="none", n_iters=2)
+    f0 = np.zeros(n)
+    g0 = np.where(np.arange(m) < m // 2, 0.0, -50.0)
+    lo, hi = orc.joint_box(w.x, w.y)
+    px, py = orc.morton_order(w.x, lo, hi), orc.morton_order(w.y, lo, hi)
+    o = orc.block_mask(w.x[px], w.y[py], w.a[px].astype(np.float64), w.b[py].astype(np.float64),
+                       f0[px], g0[py], 1.0, w.eps, 128, 1e-6)
+    empty = ~o["adm"].any(1)
+    assert empty.any() and not empty.all()  # the case the test is about
+    plan = _gpu(ot, w, 2, f0=f0, g0=g0, sparse_delta=1e-6, sparse_dense_frac=1.0)
+    f, g, _, _, _ = orc.sinkhorn_sparse(w.x, w.y, w.a, w.b, 1.0, w.eps, 2, B=128, delta=1e-6,
+                                        dense_frac=1.0, f0=f0, g0=g0)
+    _compare(plan, f, g, w)
+    plan.close()
