@@ -10,7 +10,9 @@ form (the sparsify output), and the materialisation of every row in blocks of
 every step. The metric counts Sinkhorn pair-updates (n*m per half-step) per
 second; the row passes are inside the timed step but add no units. After the
 timed steps, the line's `large_n` object reports the d = 3 per-launch half-step
-at n = m = 1e5 against the same MUFU roofline (skip with --no-large-n).
+at n = m = 1e5 against the same MUFU roofline, and its `block_sparse` object the
+block-sparse fine iterations at n = m = 2^18 against dense ones (skip both with
+--no-large-n; `--sparse N` prints the full line at any size).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload w2]
 
@@ -326,7 +328,7 @@ def run_lowrank(args, k=4096, m=100_000, n=20_000, reps=5):
     print(json.dumps(line), flush=True)
 
 
-def run_sparse(args, reps=10, dense_reps=2, tau=5e-3):
+def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
     """Fine iterations at the target eps on the uniform-vs-64-clusters workload
     (n = m = args.sparse, eps = (2 x mean nearest-neighbour spacing)^2): block-
     sparse ("FlashSinkhorn 2", section 3.2; delta = tau / (4 max(NB, MB)),
@@ -338,7 +340,7 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3):
     import log_domain_sinkhorn_online_b200 as ot
     from log_domain_sinkhorn_online_b200 import workloads as W
     dev = torch.device("cuda", 0)
-    w = W.w4(n=args.sparse)
+    w = W.w4(n=args.sparse if emit else 262144)
     x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
     nb = -(-w.n // 128)
     delta = tau / (4.0 * max(nb, -(-w.m // 128)))
@@ -396,6 +398,8 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3):
                        "eps": w.eps, "scale": "none", "block": 128, "delta": delta, "tau": tau,
                        "state": f"annealed block-sparse from 16 eps, {warm_s:.1f} s untimed"},
             "sparse": res["sparse"], "dense": res["dense"], "mufu_peak_ex2_per_s": mufu}
+    if not emit:
+        return line
     print(json.dumps(line), flush=True)
 
 
@@ -470,6 +474,9 @@ def run_ours(args):
     e2e_ms = _max_over_ranks(e2e_ms, dist)
     e2e_value = e2e_units * world / (e2e_ms / 1e3)
     large = _large_n(ot, dev) if w.d <= 3 and not args.no_large_n else None
+    # the block-sparse fine iterations at n = m = 2^18 (a few seconds; --sparse N alone
+    # gives the same line at any size)
+    sparse_line = run_sparse(args, emit=False) if (not args.no_large_n and rank == 0) else None
 
     if rank == 0:
         peaks, kind = _peaks()
@@ -500,6 +507,17 @@ def run_ours(args):
             large["peak"] = peak_tex2
             large["frac"] = large["achieved"] / peak_tex2
             line["large_n"] = large
+        if sparse_line is not None:
+            sp = sparse_line["sparse"]
+            line["block_sparse"] = {
+                "workload": sparse_line["config"]["workload"], "eps": sparse_line["config"]["eps"],
+                "ms_per_fine_iteration": sp["ms_per_iteration"],
+                "dense_ms_per_iteration": sparse_line["dense"]["ms_per_iteration"],
+                "speedup_vs_dense": sparse_line["speedup_vs_dense"],
+                "pair_updates_per_s_dense_equivalent": sparse_line["value"],
+                "tiles_admitted": sp["tiles_admitted"], "tiles_total": sp["tiles_total"],
+                "residual_certified": sp["residual"], "residual_full": sp["full_row_residual"],
+                "hs_verify_frac": sp["verify_and_f"]["frac"], "hs_sparse_frac": sp["roofline"]["frac"]}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = _cpu_baseline(w)
         print(json.dumps(line), flush=True)

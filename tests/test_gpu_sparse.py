@@ -236,3 +236,27 @@ def test_blocks_without_admitted_tiles_fall_back_to_every_column(ot, orc):
                                         dense_frac=1.0, f0=f0, g0=g0)
     _compare(plan, f, g, w)
     plan.close()
+
+
+def test_annealed_block_sparse_solve_matches_the_oracle(ot, orc):
+    """eps-annealing with block-sparse iterations in every stage, against the
+    oracle's block-sparse solve run stage by stage with the same schedule."""
+    w = _clusters(41, 2500, 2300, 3)
+    eps_t, eps0, decay, per_stage = 1e-3, 8e-3, 0.5, 4
+    plan = _gpu(ot, w, 5, eps_init=eps0, eps_decay=decay, iters_per_stage=per_stage,
+                sparse_delta=1e-6, sparse_dense_frac=1.0)
+    f = np.zeros(w.n)
+    g = np.zeros(w.m)
+    k, stages = 0, 0
+    while True:
+        ek = max(eps_t, eps0 * decay ** k)
+        its = 5 if ek == eps_t else per_stage
+        f, g, _, _, _ = orc.sinkhorn_sparse(w.x, w.y, w.a, w.b, 1.0, ek, its, B=128, delta=1e-6,
+                                            dense_frac=1.0, f0=f, g0=g)
+        stages += 1
+        if ek == eps_t:
+            break
+        k += 1
+    assert plan.info.stages == stages == 4
+    _compare(plan, f, g, w)
+    plan.close()
