@@ -68,6 +68,10 @@ def _args():
                     help="instead of the step: block-sparse against dense fine iterations on the "
                          "uniform-vs-64-clusters workload at n = m = N (its eps rule), from a "
                          "state annealed by block-sparse iterations; prints its own JSON line")
+    ap.add_argument("--sparse-workload", default="w4", choices=["w4", "w5"],
+                    help="--sparse: uniform-vs-64-clusters (w4) or interleaved spirals (w5)")
+    ap.add_argument("--sparse-block", type=int, default=0, choices=[0, 128, 256],
+                    help="--sparse: block size B (0 = the library's choice)")
     ap.add_argument("--no-large-n", action="store_true",
                     help="skip the d = 3 half-step measurement at n = m = 1e5")
     ap.add_argument("--clock-ms", type=int, default=200,
@@ -340,11 +344,13 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
     import log_domain_sinkhorn_online_b200 as ot
     from log_domain_sinkhorn_online_b200 import workloads as W
     dev = torch.device("cuda", 0)
-    w = W.w4(n=args.sparse if emit else 262144)
+    gen = W.w5 if (emit and args.sparse_workload == "w5") else W.w4
+    w = gen(n=args.sparse if emit else 262144)
     x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
-    nb = -(-w.n // 128)
-    delta = tau / (4.0 * max(nb, -(-w.m // 128)))
-    kw = dict(eps=w.eps, scale="none", block_sparse=True, sparse_delta=delta, sparse_block=128)
+    blk = args.sparse_block if emit and args.sparse_block else (
+        128 if (-(-w.n // 128)) * (-(-w.m // 128)) <= (1 << 27) else 256)
+    delta = tau / (4.0 * max(-(-w.n // blk), -(-w.m // blk)))
+    kw = dict(eps=w.eps, scale=w.scale, block_sparse=True, sparse_delta=delta, sparse_block=blk)
     t0 = time.time()
     warm = ot.sinkhorn(x, y, a, b, n_iters=20, eps_init=16.0 * w.eps, eps_decay=0.7,
                        iters_per_stage=20, **kw)
@@ -355,7 +361,7 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
     mufu = SMS * EX2_PER_CLK * 1.965e9
     res = {}
     for mode, k in (("sparse", reps), ("dense", dense_reps)):
-        extra = kw if mode == "sparse" else dict(eps=w.eps, scale="none")
+        extra = kw if mode == "sparse" else dict(eps=w.eps, scale=w.scale)
         plan = ot.sinkhorn(x, y, a, b, n_iters=k, f=f0.clone(), g=g0.clone(), warm_start=True,
                            timing=True, **extra)
         torch.cuda.synchronize()
@@ -374,7 +380,7 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
             # the block-sparse half-step against the MUFU ex2 rate: one ex2 per
             # entry of every admitted tile (the last mask's count; the masks of
             # the timed iterations differ by a few tiles)
-            pairs = float(info.tiles_admitted) * 128 * 128 * info.sparse_hs_launches
+            pairs = float(info.tiles_admitted) * blk * blk * info.sparse_hs_launches
             hs_s = info.sparse_hs_ms / 1e3
             res[mode]["roofline"] = {
                 "bound": "alu", "kernel": "hs_sparse_kernel (block-sparse g half-step)",
@@ -383,7 +389,7 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
                 "per_launch_us": info.sparse_hs_ms * 1e3 / max(info.sparse_hs_launches, 1)}
             # the verification fused with the f-update (hs_verify_kernel): one ex2
             # per entry of every tile whose exact mass is evaluated
-            vx = float(info.tiles_exact) * 128 * 128 * (info.sparse_iterations + 1)
+            vx = float(info.tiles_exact) * blk * blk * (info.sparse_iterations + 1)
             res[mode]["verify_and_f"] = {"kernel": "hs_verify_kernel (tile verification + f-update)",
                                          "ms_per_iteration": info.verify_ms / (info.sparse_iterations + 1),
                                          "exact_tiles": int(info.tiles_exact),
@@ -394,8 +400,9 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
             "unit": "pair-updates/s", "value": res["sparse"]["pair_updates_per_s"],
             "dense_value": res["dense"]["pair_updates_per_s"],
             "speedup_vs_dense": res["dense"]["ms_per_iteration"] / res["sparse"]["ms_per_iteration"],
-            "config": {"workload": f"uniform_vs_64clusters_{w.n}", "n": w.n, "m": w.m, "d": 3,
-                       "eps": w.eps, "scale": "none", "block": 128, "delta": delta, "tau": tau,
+            "config": {"workload": f"{'spirals' if gen is W.w5 else 'uniform_vs_64clusters'}_{w.n}",
+                       "n": w.n, "m": w.m, "d": 3,
+                       "eps": w.eps, "scale": w.scale, "block": blk, "delta": delta, "tau": tau,
                        "state": f"annealed block-sparse from 16 eps, {warm_s:.1f} s untimed"},
             "sparse": res["sparse"], "dense": res["dense"], "mufu_peak_ex2_per_s": mufu}
     if not emit:
