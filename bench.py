@@ -68,6 +68,11 @@ def _args():
                     help="instead of the step: block-sparse against dense fine iterations on the "
                          "uniform-vs-64-clusters workload at n = m = N (its eps rule), from a "
                          "state annealed by block-sparse iterations; prints its own JSON line")
+    ap.add_argument("--configs", action="store_true",
+                    help="instead of the step: one JSON line per workload (w1..w5) with the GPU's "
+                         "time per half-step and pair-updates/s (measured; totals of the long "
+                         "configurations extrapolated and marked) and the oracle's rate on the "
+                         "host cores")
     ap.add_argument("--sparse-workload", default="w4", choices=["w4", "w5"],
                     help="--sparse: uniform-vs-64-clusters (w4) or interleaved spirals (w5)")
     ap.add_argument("--sparse-block", type=int, default=0, choices=[0, 128, 256],
@@ -332,6 +337,60 @@ def run_lowrank(args, k=4096, m=100_000, n=20_000, reps=5):
     print(json.dumps(line), flush=True)
 
 
+def run_configs(args):
+    """Per workload: the GPU solve as the configuration states it where that takes
+    seconds (w1, w2), else a short run of the same shape (w3: 20 of its 500
+    iterations; w4: 2 iterations at its final eps; w5: 2 of its 100 iterations)
+    whose time per half-step (CUDA events around the iteration loop) gives the
+    configuration's total by its half-step count (marked "extrapolated"); and the
+    oracle's pair-update rate on a bounded row sample on the host cores."""
+    import torch
+    import log_domain_sinkhorn_online_b200 as ot
+    from log_domain_sinkhorn_online_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    mufu = SMS * EX2_PER_CLK * 1.965e9
+    for name in ("w1", "w2", "w3", "w4", "w5"):
+        w = W.ALL[name]()
+        x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
+        if name in ("w1", "w2"):
+            iters, full_half_steps = w.n_iters, None
+        elif name == "w3":
+            iters, full_half_steps = 20, 2 * w.n_iters + 1
+        elif name == "w4":
+            stages = 1
+            while max(w.eps, w.anneal["eps_init"] * w.anneal["decay"] ** (stages - 1)) > w.eps:
+                stages += 1
+            iters, full_half_steps = 2, 2 * (stages * w.anneal["iters_per_stage"]) + 1
+        else:
+            iters, full_half_steps = 2, 2 * w.n_iters + 1
+        kw = dict(tol=w.tol) if name == "w2" else {}
+        plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=iters, timing=True, **kw)
+        torch.cuda.synchronize()
+        plan.close()  # warm: the timed call below reuses the cached workspace
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        plan = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=iters, timing=True, **kw)
+        e1.record()
+        torch.cuda.synchronize()
+        info = plan.info
+        plan.close()
+        per_hs_ms = info.loop_ms / max(info.half_steps, 1)
+        rate = float(w.n) * float(w.m) / (per_hs_ms / 1e3)
+        gpu = {"iterations": int(info.iterations), "half_steps": int(info.half_steps),
+               "call_ms": e0.elapsed_time(e1), "ms_per_half_step": per_hs_ms,
+               "pair_updates_per_s": rate, "frac_of_mufu": rate / mufu}
+        if full_half_steps:
+            gpu["total_s_extrapolated"] = per_hs_ms * full_half_steps / 1e3
+            gpu["total_half_steps"] = full_half_steps
+        cb = _cpu_baseline(w, target_s=5.0)
+        line = {"metric": METRIC, "unit": UNIT, "config": {"workload": w.name, "n": w.n, "m": w.m,
+                                                           "d": w.d, "eps": w.eps, "scale": w.scale},
+                "gpu": gpu, "oracle": {"pair_updates_per_s": cb["value"], "cores": cb["cores"],
+                                       "sample": cb["sample"],
+                                       "ms_per_half_step_extrapolated": float(w.n) * w.m / cb["value"] * 1e3}}
+        print(json.dumps(line), flush=True)
+
+
 def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
     """Fine iterations at the target eps on the uniform-vs-64-clusters workload
     (n = m = args.sparse, eps = (2 x mean nearest-neighbour spacing)^2): block-
@@ -540,6 +599,8 @@ def main():
         run_lowrank(args)
     elif args.sparse:
         run_sparse(args)
+    elif args.configs:
+        run_configs(args)
     else:
         run_ours(args)
 
