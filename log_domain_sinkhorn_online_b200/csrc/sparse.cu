@@ -11,13 +11,15 @@
 //     rho_IJ = delta * min(smallest nonzero a in I, smallest nonzero b in J)
 //     (screen_kernel, float64, one byte per pair);
 //  3. verifies the candidates by their exact mass over the B x B point pairs
-//     (verify_kernel, the half-step's own float32 exponentials, float64 row
-//     terms);
-//  4. lists the admitted tiles of every row block and, from the transposed
-//     mask, of every column block (mask_list_kernel, transpose_bytes_kernel);
-//  5. runs the f- and the g-update over the admitted tiles only
-//     (hs_sparse_kernel: the d <= 3 half-step with a gathered column stream);
-//     a block with no admitted tile reduces over every column.
+//     and, in the same pass, runs the f-update over the admitted ones
+//     (hs_verify_kernel: the half-step's own float32 exponentials, float64 row
+//     terms; a row block left without an admitted tile is updated over every
+//     column by a fallback hs_sparse_kernel launch);
+//  4. lists the admitted tiles of every column block from the transposed mask
+//     (transpose_bytes_kernel, mask_list_kernel);
+//  5. runs the g-update over the admitted tiles only (hs_sparse_kernel: the
+//     d <= 3 half-step with a gathered column stream); a block with no
+//     admitted tile reduces over every column.
 // The mask omits at most delta a_i per tile from row i (delta b_j from
 // column j), so with delta = tol / (4 max(NB, MB)) at most tol/4 of the mass.
 #include <float.h>
@@ -269,12 +271,15 @@ __global__ void __launch_bounds__(kScreenThreads) screen_kernel(ScreenArgs S) {
 //     of 3.67M candidates left for the exact test; a bound through the
 //     column side as well, or over 32-point sub-blocks of the column tile,
 //     left 7 % / 11 % fewer but cost more time than it saved);
-//  2. the exact mass of the others, one block per tile: the tile's B columns
-//     are streamed and, per row i, the running (max m_i, sum s_i) of 2^(t_ij)
-//     (t = G_j + x'_i.Y_j, as in the half-step) is formed; with the row term
-//     b_i = kappa f_i - c kappa |x'_i|^2 (float64), log2 M = log2 sum_i s_i
-//     2^(b_i + m_i), and the tile stays admitted when log2 M > log2 rho.
-// A rejected tile's byte is cleared and the counts are corrected.
+//  2. the exact mass of the others (taken in list order), 256 / B tiles per
+//     256-column step: per row i, the running (max m_i, sum s_i) of 2^(t_ij)
+//     (t = G_j + x'_i.Y_j, as in the half-step); with the row term b_i = kappa
+//     f_i - c kappa |x'_i|^2 (float64), log2 M = log2 sum_i s_i 2^(b_i + m_i),
+//     and the tile stays admitted when log2 M > log2 rho. An admitted tile's
+//     (m_i, s_i) joins the row's running sum: the segment's share of the
+//     f-update, written as a split partial and merged by finish_tile.
+// A rejected tile's byte is cleared and the counts are corrected. This kernel is
+// the f half-step of a block-sparse iteration (HalfStep A, side 0).
 constexpr int kVfWindow = 1024;
 constexpr float kVfMargin = 0.05f;
 
