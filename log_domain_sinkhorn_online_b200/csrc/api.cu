@@ -461,8 +461,13 @@ int sparse_setup(ot_plan *p, const ot_options &o, double tol, bool warm) {
     if (bps <= 0 || vbps <= 0) return fail(OT_ERR_CUDA, "block-sparse kernels cannot be made resident");
     const int64_t cap = (int64_t)bps * p->sm_count;
     for (int side = 0; side < 2; ++side) {
+        // side 1 (the g-update) with items of about 1/8 of a wave, so the launch's
+        // tail is short (measured: 3.57 -> 3.40 ms at n = m = 1e6, 0.77 -> 0.71 ms
+        // at 2^18 against 1/2 of a wave); side 0 only serves the fallback launch,
+        // whose items mostly return at once
         const int64_t tiles = side == 0 ? nb : mb;
-        const int64_t sp = std::min<int64_t>(std::max<int64_t>((2 * cap + tiles - 1) / tiles, 1), 32);
+        const int64_t per = side == 0 ? 2 : 8;
+        const int64_t sp = std::min<int64_t>(std::max<int64_t>((per * cap + tiles - 1) / tiles, 1), 32);
         p->sp_splits[side] = (int)sp;
         p->sp_grid[side] = (int)std::min<int64_t>(tiles * sp, cap);
     }
