@@ -495,12 +495,16 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
                 for (int tt = 0; tt < kTpc; ++tt) {
                     if (step * kTpc + tt >= n_exact) continue;
                     const int64_t q = s_exact[step * kTpc + tt];
-                    float S = 0.f;
-                    for (int k = 0; k < kHsThreads / 32; ++k) S += s_sum[tt][k];
-                    const double lm = (W[tt] == -INFINITY || !(S > 0.f)) ? -INFINITY
-                                                                          : (double)W[tt] + log2((double)S);
-                    const double lrho = V.l2_delta + fmin(V.rs[p].l2w, V.cs[q].l2w);
-                    if (lm > lrho) {  // admitted: the tile joins this segment's f-update
+                    // one lane per warp takes the decision (float64 log2), the warp shares it
+                    int adm = 0;
+                    if (lane == 0) {
+                        float S = 0.f;
+                        for (int k = 0; k < kHsThreads / 32; ++k) S += s_sum[tt][k];
+                        const double lm = (W[tt] == -INFINITY || !(S > 0.f))
+                                              ? -INFINITY : (double)W[tt] + log2((double)S);
+                        adm = lm > V.l2_delta + fmin(V.rs[p].l2w, V.cs[q].l2w);
+                    }
+                    if (__shfl_sync(0xffffffffu, adm, 0)) {  // admitted: the tile joins this segment's f-update
 #pragma unroll
                         for (int k = 0; k < R; ++k) {
                             if (!(tv[tt][k] > 0.f)) continue;
