@@ -207,3 +207,35 @@ def test_w5_two_million_points_step_and_rows(ot, orc):
     del out
     H.assert_entries(T, orc.materialize_rows(w.x, w.y, fs, H.f32(g0), c, w.eps, w.rows[pick]))
     p.close()
+
+
+def test_block_sparse_certificate_at_2_18(ot, orc):
+    """Block-sparse fine iterations on workload 4's clouds at n = m = 2^18 (its eps
+    rule), from a state annealed by block-sparse iterations: the stop test's
+    admitted-plan residual and the GPU's float64 residual over every pair differ by
+    at most the omitted-mass bound, the mask is far from full, and a rerun from the
+    same state is bit-identical."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w4(n=262144)
+    x, y, a, b = H.to_dev(w)
+    tau = 5e-3
+    delta = tau / (4 * 2048)
+    kw = dict(eps=w.eps, scale="none", block_sparse=True, sparse_delta=delta)
+    warm = ot.sinkhorn(x, y, a, b, n_iters=20, eps_init=16 * w.eps, eps_decay=0.7,
+                       iters_per_stage=20, **kw)
+    f0, g0 = warm.f.clone(), warm.g.clone()
+    warm.close()
+    runs = []
+    for _ in range(2):
+        p = ot.sinkhorn(x, y, a, b, n_iters=5, f=f0.clone(), g=g0.clone(), warm_start=True, **kw)
+        torch.cuda.synchronize()
+        runs.append((p.f.clone(), p.g.clone(), p.info.residual))
+        info = p.info
+        full_row, full_col = p.marginal_residual()
+        assert info.sparse_iterations == 5 and info.tiles_admitted < 0.1 * info.tiles_total
+        assert abs(full_row - info.residual) <= info.omitted_bound + 1e-5
+        assert info.omitted_bound <= tau / 4 * (1 + 1e-6)
+        p.close()
+    assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+    assert runs[0][2] == runs[1][2]
