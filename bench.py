@@ -40,7 +40,7 @@ UNIT = "pair-updates/s"
 SMS, EX2_PER_CLK = 148, 16
 # DRAM bytes per half-step of the dominant kernel, from the committed ncu captures
 # of the current kernel, keyed by workload; None where no such capture exists
-HALFSTEP_TRAFFIC = {"w2_gmm3d_8000": 874.5e3 / 512}  # profiles/hs_loop_w2_8000.md
+HALFSTEP_TRAFFIC = {"w2_gmm3d_8000": 775.7e3 / 512}  # profiles/hs_loop_w2_8000.md
 
 
 def _peaks():
