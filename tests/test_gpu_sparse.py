@@ -260,3 +260,24 @@ def test_annealed_block_sparse_solve_matches_the_oracle(ot, orc):
     assert plan.info.stages == stages == 4
     _compare(plan, f, g, w)
     plan.close()
+
+
+@pytest.mark.parametrize("scale,B,verify", [("mean", 128, True), ("max_cost", 256, False)])
+def test_scaled_costs_and_massless_columns(ot, orc, scale, B, verify):
+    """Block-sparse iterations on a scaled cost with massless rows and columns and
+    m much larger than n, against the oracle's block-sparse solve at the same c."""
+    w = _clusters(51, 1200, 4100, 3, massless=True)
+    w.b = w.b.copy()
+    w.b[[0, 77, 4099]] = 0.0
+    w.scale, w.eps = scale, 2e-3
+    c = orc.inv_scale_cost(w.x, w.y, scale)
+    plan = _gpu(ot, w, 6, sparse_block=B, sparse_verify=verify, sparse_delta=1e-6,
+                sparse_dense_frac=1.0)
+    assert plan.info.inv_scale_cost == pytest.approx(c, rel=2e-7)
+    f, g, _, _, st = orc.sinkhorn_sparse(w.x, w.y, w.a, w.b, c, w.eps, 6, B=B, delta=1e-6,
+                                         verify=verify, dense_frac=1.0)
+    maxc = H.max_cost(w.x, w.y, c)
+    H.assert_potentials(plan.f.double().cpu().numpy(), f, maxc, what="f")
+    H.assert_potentials(plan.g.double().cpu().numpy(), g, maxc, what="g")
+    assert plan.info.sparse_iterations == 6 and 0 < st[3] < plan.info.tiles_total
+    plan.close()
