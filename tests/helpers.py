@@ -1,6 +1,6 @@
 """Shared helpers for the GPU parity tests (comparison rules and device transfer).
 
-Tolerances (the readings are listed in the design doc):
+Tolerances:
  - potentials: max |f - f_ref| and |g - g_ref| <= 1e-4 * max_ij C_ij (the cost
    as used, i.e. scaled), -inf at the same (massless) entries;
  - plan entries of a plan built at given potentials (the oracle's, rounded to
