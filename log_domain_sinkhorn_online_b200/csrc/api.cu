@@ -69,7 +69,6 @@ struct DevScalars {
 struct SparseCtr {
     unsigned long long cand, adm;  // candidate and admitted tiles of the current mask
     unsigned long long exact;      // candidates whose exact mass was evaluated
-    unsigned work, pad;            // verification: dynamic row-block counter
     unsigned lohi[6];              // joint bounding box (order-preserving float bits)
 };
 
