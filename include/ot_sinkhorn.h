@@ -113,10 +113,11 @@ typedef struct ot_options {
                                  the admitted tiles only (every tile for a block with none).
                                  The stop test compares the admitted plan's row residual with
                                  tol - MB delta sum(a), so that the full residual is <= tol.
-                                 f and g are returned in the caller's order; the host reads
-                                 the candidate count once per iteration, so check_every,
-                                 use_graphs and device_loop do not apply. 0 (default):
-                                 dense iterations */
+                                 f and g are returned in the caller's order. The choice of
+                                 dense or sparse updates is made on the device each iteration;
+                                 the host reads the stop flag every check_every iterations;
+                                 use_graphs and device_loop do not apply. 0 (default): dense
+                                 iterations */
     int32_t sparse_block;     /* block size B: 128 or 256 (0 = 128 when NB * MB <= 2^27,
                                  else 256) */
     int32_t sparse_verify;    /* 1 (default): candidate tiles are verified by their exact mass;

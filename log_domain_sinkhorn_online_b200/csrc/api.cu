@@ -69,6 +69,8 @@ struct DevScalars {
 struct SparseCtr {
     unsigned long long cand, adm;  // candidate and admitted tiles of the current mask
     unsigned long long exact;      // candidates whose exact mass was evaluated
+    unsigned long long n_mode[2];  // iterations run sparse / dense (whole solve)
+    int mode[2];                   // this iteration's kind (kMode*), the last counted kind
     unsigned lohi[6];              // joint bounding box (order-preserving float bits)
 };
 
@@ -148,9 +150,7 @@ struct ot_plan {
     unsigned *sp_tcnt = nullptr;
     double *sp_tres = nullptr;
     SparseCtr *sc = nullptr;
-    std::vector<uint8_t> iter_sparse;     // per launched iteration: 1 sparse, 0 dense
     int64_t last_cand = 0, last_adm = 0, last_exact = 0;  // tiles of the last mask an iteration ran on
-    bool adm_pending = false;             // its admitted count is still on the device
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
     cudaStream_t s_int = nullptr;
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
@@ -563,20 +563,20 @@ HalfStep make_sparse_step(const ot_plan *p, int side, int parity) {
 
 // One block-sparse iteration from the state at f-buffer parity `par`: the
 // mask at (f, g), then the f-update (f_only: the update that measures the
-// final residual) and the g-update on it. *stopped: the state had already
-// passed the stop test (nothing was launched after the screen).
-int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped) {
+// final residual) and the g-update on it. Nothing is read back: a kernel after
+// the screen chooses dense or sparse updates on the device (the candidate count
+// against sparse_dense_frac of all block pairs), and the launches of both kinds
+// are gated on that choice; once the stop test has passed every launch returns
+// at once, so the host only reads the state every check_every iterations.
+int sparse_iteration(ot_plan *p, int par, bool f_only, double eps) {
     cudaStream_t s = p->s_int;
     const int64_t nb = p->sp_nb, mb = p->sp_mb;
     const int B = p->sp_B, d = p->d, rpt = p->sp_rpt;
-    *stopped = false;
-    OT_CU(cudaMemcpyAsync(&p->hs->sc_prev, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, s));
     OT_CU(launch_block_max(p->sf[par], p->n, B, p->bsx, s));
     OT_CU(launch_block_max(p->sg, p->m, B, p->bsy, s));
-    OT_CU(cudaMemsetAsync(p->cnt, 0, sizeof(int64_t) * nb, s));
-    OT_CU(cudaMemsetAsync(p->cnt_t, 0, sizeof(int64_t) * mb, s));
-    OT_CU(cudaMemsetAsync(p->sc, 0, offsetof(SparseCtr, lohi), s));
+    OT_CU(launch_sparse_prep(p->cnt, nb, p->cnt_t, mb, &p->sc->cand, 3, p->st, s));
     ScreenArgs S{};
+    S.st = p->st;
     S.rs = p->bsx;
     S.cs = p->bsy;
     S.nb = nb;
@@ -590,30 +590,18 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
     S.cnt_t = p->cnt_t;
     S.total = &p->sc->cand;
     OT_CU(launch_screen(S, s));
-    OT_CU(cudaMemcpyAsync(&p->hs->sc, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, s));
-    OT_CU(cudaMemcpyAsync(&p->hs->st, p->st, sizeof(State), cudaMemcpyDeviceToHost, s));
-    OT_CU(cudaStreamSynchronize(s));
-    p->launches += 3;
-    if (p->adm_pending) {
-        p->last_cand = (int64_t)p->hs->sc_prev.cand;
-        p->last_adm = (int64_t)p->hs->sc_prev.adm;
-        p->last_exact = (int64_t)p->hs->sc_prev.exact;
-        p->adm_pending = false;
-    }
-    if (p->hs->st.stop) {
-        *stopped = true;
-        return OT_OK;
-    }
-    const bool dense = (double)p->hs->sc.cand > p->sp_frac * (double)nb * (double)mb;
-    p->last_cand = p->last_adm = (int64_t)p->hs->sc.cand;
-    p->last_exact = 0;
-    if (dense) {
-        OT_CU(launch_side(p, 0, par));
-        if (!f_only) OT_CU(launch_side(p, 1, par));
-        p->launches += f_only ? 1 : 2;
-        if (!f_only) p->iter_sparse.push_back(0);
-        return OT_OK;
-    }
+    OT_CU(launch_decide(&p->sc->cand, p->sp_frac * (double)nb * (double)mb, p->st, p->sc->mode,
+                        p->sc->n_mode, f_only ? 0 : 1, s));
+    p->launches += 5;
+    auto gated = [&](HalfStep A, int val) {
+        A.gate = p->sc->mode;
+        A.gate_val = val;
+        return A;
+    };
+    // dense f-update (when the candidates are too many)
+    OT_CU(launch_halfstep(p->kind, p->dim, p->sx.rpt, gated(make_step(p, 0, par), kModeDense),
+                          p->sx.grid, s));
+    p->launches += 1;
     if (p->sp_verify) {
         // the candidates as compressed rows, then admitted counts from zero
         OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
@@ -641,15 +629,14 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         V.total = &p->sc->adm;
         V.exact = &p->sc->exact;
         // the verification and the f-update over the admitted tiles in one launch
-        HalfStep A = make_sparse_step(p, 0, par);
+        HalfStep A = gated(make_sparse_step(p, 0, par), kModeSparse);
         A.splits = kVerifySegs;
         OT_CU(mark_in(p, p->tm_verify));
         OT_CU(launch_verify(d, rpt, A, V, p->sp_vgrid, s));
         OT_CU(mark_in(p, p->tm_verify));
-        p->adm_pending = true;
         // row blocks left without an admitted tile: f-update over every column
         OT_CU(cudaMemsetAsync(&p->st->work[0], 0, sizeof(unsigned), s));
-        HalfStep Af = make_sparse_step(p, 0, par);
+        HalfStep Af = gated(make_sparse_step(p, 0, par), kModeSparse);
         Af.sp_ptr = nullptr;
         Af.sp_idx = nullptr;
         Af.sp_fallback = p->cnt;
@@ -659,7 +646,8 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         OT_CU(launch_row_ptr_scan(p->cnt, nb, p->ptr, p->sp_scan, s));
         OT_CU(launch_mask_list(p->mask, nb, mb, p->ptr, p->lst, s));
         OT_CU(mark_in(p, p->tm_hs));
-        OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 0, par), p->sp_grid[0], s));
+        OT_CU(launch_halfstep_sparse(d, rpt, gated(make_sparse_step(p, 0, par), kModeSparse),
+                                     p->sp_grid[0], s));
         OT_CU(mark_in(p, p->tm_hs));
         p->launches += 5;
     }
@@ -667,25 +655,29 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps, bool *stopped
         OT_CU(launch_transpose_bytes(p->mask, nb, mb, p->mask_t, s));
         OT_CU(launch_row_ptr_scan(p->cnt_t, mb, p->ptr_t, p->sp_scan, s));
         OT_CU(launch_mask_list(p->mask_t, mb, nb, p->ptr_t, p->lst_t, s));
+        OT_CU(launch_halfstep(p->kind, p->dim, p->sy.rpt, gated(make_step(p, 1, par), kModeDense),
+                              p->sy.grid, s));
         OT_CU(mark_in(p, p->tm_hs));
-        OT_CU(launch_halfstep_sparse(d, rpt, make_sparse_step(p, 1, par), p->sp_grid[1], s));
+        OT_CU(launch_halfstep_sparse(d, rpt, gated(make_sparse_step(p, 1, par), kModeSparse),
+                                     p->sp_grid[1], s));
         OT_CU(mark_in(p, p->tm_hs));
-        p->launches += 6;
-        p->iter_sparse.push_back(1);
+        p->launches += 7;
     }
     return OT_OK;
 }
 
-// `iters` block-sparse iterations from global parity `parity0`; stops early
-// when the stop test has passed.
-int run_sparse(ot_plan *p, int parity0, int iters, double eps) {
+// `iters` block-sparse iterations from global parity `parity0`; the state is
+// read every `check` iterations, and the loop ends once the stop test has passed.
+int run_sparse(ot_plan *p, int parity0, int iters, double eps, int check) {
     for (int i = 0; i < iters; ++i) {
-        bool stopped = false;
         OT_CU(mark(p));
-        int rc = sparse_iteration(p, (parity0 + i) & 1, false, eps, &stopped);
+        int rc = sparse_iteration(p, (parity0 + i) & 1, false, eps);
         OT_CU(mark(p));
         if (rc != OT_OK) return rc;
-        if (stopped) break;
+        if ((i + 1) % check == 0 && i + 1 < iters) {
+            if ((rc = read_state(p)) != OT_OK) return rc;
+            if (p->hs->st.stop) break;
+        }
     }
     return OT_OK;
 }
@@ -1115,7 +1107,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
                                 p->sy.rowtab, p->sy.coltab, layout, p->s_int));
         }
         p->launches += 4;
-        rc = sparse ? run_sparse(p, t & 1, iters, stage_eps[si])
+        rc = sparse ? run_sparse(p, t & 1, iters, stage_eps[si], tol_s > 0.0 ? o.check_every : iters)
                     : run_iterations(p, t & 1, iters, tol_s > 0.0, o.use_graphs != 0);
         if (rc != OT_OK) return rc;
         if ((rc = read_state(p)) != OT_OK) return rc;
@@ -1130,8 +1122,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
                 // one more f-update measures ||T1 - a||_1 of the final state
                 OT_CU(mark(p));
                 if (sparse) {
-                    bool stopped = false;
-                    if ((rc = sparse_iteration(p, t & 1, true, stage_eps[si], &stopped)) != OT_OK) return rc;
+                    if ((rc = sparse_iteration(p, t & 1, true, stage_eps[si])) != OT_OK) return rc;
                 } else {
                     OT_CU(launch_side(p, 0, t & 1));
                     p->launches += 1;
@@ -1144,13 +1135,22 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
             }
         }
     }
-    if (sparse && p->adm_pending) {
-        OT_CU(cudaMemcpyAsync(&p->hs->sc_prev, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, p->s_int));
+    int64_t sp_it = 0, dn_it = 0;
+    if (sparse) {
+        OT_CU(cudaMemcpyAsync(&p->hs->sc, p->sc, sizeof(SparseCtr), cudaMemcpyDeviceToHost, p->s_int));
         OT_CU(cudaStreamSynchronize(p->s_int));
-        p->last_cand = (int64_t)p->hs->sc_prev.cand;
-        p->last_adm = (int64_t)p->hs->sc_prev.adm;
-        p->last_exact = (int64_t)p->hs->sc_prev.exact;
-        p->adm_pending = false;
+        const SparseCtr &sc = p->hs->sc;
+        // the counters hold the last screened mask: of the last iteration that ran
+        const int kindm = sc.mode[0] == kModeStopped ? sc.mode[1] : sc.mode[0];
+        p->last_cand = (int64_t)sc.cand;
+        p->last_adm = (kindm == kModeDense || !p->sp_verify) ? (int64_t)sc.cand : (int64_t)sc.adm;
+        p->last_exact = kindm == kModeDense ? 0 : (int64_t)sc.exact;
+        // iterations of the returned state: the one whose f-update met the stop test
+        // was counted but not completed
+        sp_it = (int64_t)sc.n_mode[kModeSparse];
+        dn_it = (int64_t)sc.n_mode[kModeDense];
+        const int64_t excess = sp_it + dn_it - (int64_t)t;
+        if (excess > 0) (sc.mode[1] == kModeDense ? dn_it : sp_it) -= excess;
     }
     if (sparse) {  // back to the caller's order
         OT_CU(launch_scatter(p->sf[t & 1], p->perm_x, n, p->f, p->s_int));
@@ -1186,11 +1186,6 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         info->half_steps = half_steps;
         info->kernel_launches = p->launches;
         info->loop_ms = loop_ms;
-        // iterations of the returned state (the one that met the stop test
-        // was launched but not completed)
-        int64_t sp_it = 0, dn_it = 0;
-        for (size_t k = 0; k < p->iter_sparse.size() && k < (size_t)t; ++k)
-            (p->iter_sparse[k] ? sp_it : dn_it) += 1;
         info->sparse_iterations = sp_it;
         info->dense_iterations = dn_it;
         info->tiles_candidate = p->last_cand;

@@ -91,6 +91,8 @@ struct HalfStep {
     const int *sp_idx;
     int sp_coltiles;
     const int64_t *sp_fallback;  // non-null: only blocks t with sp_fallback[t] == 0 are updated
+    const int *gate;             // non-null: the launch does nothing unless *gate == gate_val
+    int gate_val;                //   (block-sparse iterations choose dense or sparse on the device)
 };
 
 // ------------------------------------------------------ device helpers --

@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 8 ? 3 : R == 4 ? 4 : R == 2 ?
     __shared__ long long s_next[2];
     if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;
     if (ld_volatile(&A.st->stop)) return;
+    if (A.gate && ld_volatile(A.gate) != A.gate_val) return;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
     int64_t item = blockIdx.x;
     for (int it = 0; item < n_items; ++it) {

@@ -126,7 +126,9 @@ struct BlockSum {     // one block of B consecutive points (Morton order)
     double lnw, l2w;      // ln and log2 of the smallest nonzero weight (+inf: none)
     double lncnt;         // ln of the block's point count
 };
+constexpr int kModeSparse = 0, kModeDense = 1, kModeStopped = 2;
 struct ScreenArgs {
+    const State *st;           // nothing is screened once the solve has stopped
     const BlockSum *rs, *cs;   // row (x) and column (y) blocks
     int64_t nb, mb;
     int d;
@@ -166,6 +168,11 @@ cudaError_t launch_block_static(const float *ps, const float *ws, int64_t cnt, i
                                 BlockSum *bs, cudaStream_t s);
 cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, BlockSum *bs, cudaStream_t s);
 cudaError_t launch_screen(const ScreenArgs &S, cudaStream_t s);
+cudaError_t launch_sparse_prep(int64_t *cnt, int64_t nb, int64_t *cnt_t, int64_t mb,
+                               unsigned long long *ctr, int nctr, const State *st, cudaStream_t s);
+// mode[0]: this iteration's kind, mode[1]: the last counted one; n_mode[kind] += count
+cudaError_t launch_decide(const unsigned long long *cand, double limit, const State *st, int *mode,
+                          unsigned long long *n_mode, int count, cudaStream_t s);
 // the verification fused with the f-update (A: the f half-step, V.segs splits)
 cudaError_t launch_verify(int d, int rpt, const HalfStep &A, const VerifyArgs &V, int grid,
                           cudaStream_t s);

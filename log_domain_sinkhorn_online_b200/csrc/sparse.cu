@@ -206,6 +206,7 @@ __global__ void block_max_kernel(const float *pot, int64_t cnt, int B, int64_t n
 constexpr int kScreenThreads = 256, kScreenRows = 32;
 
 __global__ void __launch_bounds__(kScreenThreads) screen_kernel(ScreenArgs S) {
+    if (ld_volatile(&S.st->stop)) return;  // a stopped solve keeps its last mask
     __shared__ BlockSum rs[kScreenRows];
     __shared__ unsigned long long s_tot[kScreenThreads / 32];
     const int tid = threadIdx.x;
@@ -252,6 +253,35 @@ __global__ void __launch_bounds__(kScreenThreads) screen_kernel(ScreenArgs S) {
         unsigned long long t = 0;
         for (int k = 0; k < kScreenThreads / 32; ++k) t += s_tot[k];
         if (t) atomicAdd(S.total, t);
+    }
+}
+
+// Start of a block-sparse iteration: zero the per-block counts and the tile
+// counters (nothing once the solve has stopped, so the last mask's counts stay).
+__global__ void sparse_prep_kernel(int64_t *cnt, int64_t nb, int64_t *cnt_t, int64_t mb,
+                                   unsigned long long *ctr, int nctr, const State *st) {
+    if (ld_volatile(&st->stop)) return;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb + mb + nctr;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nb) cnt[i] = 0;
+        else if (i < nb + mb) cnt_t[i - nb] = 0;
+        else ctr[i - nb - mb] = 0ull;
+    }
+}
+
+// After the screen: dense or sparse updates for this iteration (kModeSparse,
+// kModeDense; kModeStopped once the stop test has passed), counted per kind.
+__global__ void decide_kernel(const unsigned long long *cand, double limit, const State *st,
+                              int *mode, unsigned long long *n_mode, int count) {
+    if (ld_volatile(&st->stop)) {
+        *mode = kModeStopped;
+        return;
+    }
+    const int md = (double)*cand > limit ? kModeDense : kModeSparse;
+    *mode = md;
+    if (count) {
+        n_mode[md] += 1ull;
+        mode[1] = md;  // the kind of the last counted iteration
     }
 }
 
@@ -303,6 +333,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
     const float kf = (float)kappa, cf = (float)c;
     if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;  // as in hs_lowd_kernel
     if (ld_volatile(&A.st->stop)) return;
+    if (A.gate && ld_volatile(A.gate) != A.gate_val) return;
 
     const long long n_items = V.nb * (long long)V.segs;
     long long item = blockIdx.x;
@@ -604,6 +635,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 4 : 8) hs_sparse_kernel(H
     __shared__ long long s_next[2];
     if (blockIdx.x == 0 && threadIdx.x == 0) A.st->work[A.side ^ 1] = 0u;
     if (ld_volatile(&A.st->stop)) return;
+    if (A.gate && ld_volatile(A.gate) != A.gate_val) return;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
     int64_t item = blockIdx.x;
     for (int it = 0; item < n_items; ++it) {
@@ -697,6 +729,20 @@ cudaError_t launch_block_static(const float *ps, const float *ws, int64_t cnt, i
 cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, BlockSum *bs, cudaStream_t s) {
     const int64_t nblk = (cnt + B - 1) / B;
     block_max_kernel<<<(unsigned)((nblk * 32 + 255) / 256), 256, 0, s>>>(pot, cnt, B, nblk, bs);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_prep(int64_t *cnt, int64_t nb, int64_t *cnt_t, int64_t mb,
+                               unsigned long long *ctr, int nctr, const State *st, cudaStream_t s) {
+    const int64_t total = nb + mb + nctr;
+    const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 1184);
+    sparse_prep_kernel<<<std::max(grid, 1u), 256, 0, s>>>(cnt, nb, cnt_t, mb, ctr, nctr, st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decide(const unsigned long long *cand, double limit, const State *st, int *mode,
+                          unsigned long long *n_mode, int count, cudaStream_t s) {
+    decide_kernel<<<1, 1, 0, s>>>(cand, limit, st, mode, n_mode, count);
     return cudaGetLastError();
 }
 
