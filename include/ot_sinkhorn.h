@@ -192,6 +192,12 @@ OT_API void ot_options_default(ot_options *opt);
  *      must then be a warm start), e.g. to materialise rows of a known plan.
  *  tol: if > 0, stop after the first iteration whose ||T 1 - a||_1 <= tol;
  *      if <= 0, run exactly n_iters iterations. Missing tol is not an error.
+ *      With opt->block_sparse the test is on the admitted plan's residual
+ *      against tol - (the omitted-mass bound), so the full residual is <= tol.
+ *  Block-sparse mode (opt->block_sparse) needs d <= 3 (else OT_ERR_UNSUPPORTED),
+ *      sparse_block 0/128/256, sparse_delta >= 0 (0 needs tol > 0) and
+ *      sparse_dense_frac in [0, 1] (else OT_ERR_INVALID_ARG), and block counts
+ *      whose mask fits (NB * MB <= 2^32, NB <= 2^21; else OT_ERR_UNSUPPORTED).
  *  f [n], g [m]: device float32 outputs (and inputs for a warm start). A
  *      massless row/column gets -inf.
  *  plan_out: if non-NULL, receives a plan to pass to the calls below; free it
