@@ -572,8 +572,8 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps) {
     cudaStream_t s = p->s_int;
     const int64_t nb = p->sp_nb, mb = p->sp_mb;
     const int B = p->sp_B, d = p->d, rpt = p->sp_rpt;
-    OT_CU(launch_block_max(p->sf[par], p->n, B, p->bsx, s));
-    OT_CU(launch_block_max(p->sg, p->m, B, p->bsy, s));
+    OT_CU(launch_block_max(p->sf[par], p->n, B, kLog2e / eps, p->bsx, s));
+    OT_CU(launch_block_max(p->sg, p->m, B, kLog2e / eps, p->bsy, s));
     OT_CU(launch_sparse_prep(p->cnt, nb, p->cnt_t, mb, &p->sc->cand, 3, p->st, s));
     ScreenArgs S{};
     S.st = p->st;

@@ -123,6 +123,7 @@ struct MortonArgs {
 struct BlockSum {     // one block of B consecutive points (Morton order)
     double lo[3], hi[3];  // bounding box (0 past d)
     double pmax;          // largest potential (refreshed every iteration)
+    double l2gsum;        // log2 sum_j 2^(kappa pot_j) over the block (refreshed every iteration)
     double lnw, l2w;      // ln and log2 of the smallest nonzero weight (+inf: none)
     double lncnt;         // ln of the block's point count
 };
@@ -166,7 +167,8 @@ cudaError_t launch_scatter(const float *in, const int64_t *perm, int64_t cnt, fl
                            cudaStream_t s);
 cudaError_t launch_block_static(const float *ps, const float *ws, int64_t cnt, int d, int B,
                                 BlockSum *bs, cudaStream_t s);
-cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, BlockSum *bs, cudaStream_t s);
+cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, double kappa, BlockSum *bs,
+                             cudaStream_t s);
 cudaError_t launch_screen(const ScreenArgs &S, cudaStream_t s);
 cudaError_t launch_sparse_prep(int64_t *cnt, int64_t nb, int64_t *cnt_t, int64_t mb,
                                unsigned long long *ctr, int nctr, const State *st, cudaStream_t s);

@@ -186,8 +186,11 @@ __global__ void block_static_kernel(const float *ps, const float *ws, int64_t cn
     }
 }
 
-// One warp per block: the largest potential (-inf for a massless block).
-__global__ void block_max_kernel(const float *pot, int64_t cnt, int B, int64_t nblk, BlockSum *bs) {
+// One warp per block: the largest potential (-inf for a massless block) and
+// log2 sum_j 2^(kappa pot_j) (float64), the column factor of the verification's
+// point-level bound.
+__global__ void block_max_kernel(const float *pot, int64_t cnt, int B, int64_t nblk, double kappa,
+                                 BlockSum *bs) {
     const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (blk >= nblk) return;
@@ -195,7 +198,15 @@ __global__ void block_max_kernel(const float *pot, int64_t cnt, int B, int64_t n
     float mx = -INFINITY;
     for (int64_t i = i0 + lane; i < i1; i += 32) mx = fmaxf(mx, pot[i]);
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) bs[blk].pmax = (double)mx;
+    double sum = 0.0;
+    if (mx != -INFINITY)
+        for (int64_t i = i0 + lane; i < i1; i += 32)
+            if (pot[i] != -INFINITY) sum += exp2(kappa * ((double)pot[i] - (double)mx));
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) {
+        bs[blk].pmax = (double)mx;
+        bs[blk].l2gsum = mx == -INFINITY ? -INFINITY : kappa * (double)mx + log2(sum);
+    }
 }
 
 // ------------------------------------------------------------------ screen
@@ -291,14 +302,16 @@ __global__ void decide_kernel(const unsigned long long *cand, double limit, cons
 // leave a tail). The candidates come as compressed rows (cptr, clist) in
 // column order, taken kVfWindow at a time. Each candidate tile q is tested
 // against log2 rho = log2 delta + min(log2 amin_p, log2 bmin_q):
-//  1. a row-level bound, one warp per tile: with G_q the column block's
-//     largest potential and dist_i the distance from x_i to q's bounding box,
-//         M <= |J_q| sum_i 2^(kappa (f_i + G_q - c dist_i^2));
+//  1. a point-level bound, one warp per tile: with dist_i the distance from
+//     x_i to q's bounding box (so C_ij >= c dist_i^2 for every j of q),
+//         M <= sum_i 2^(kappa (f_i - c dist_i^2)) * sum_{j in q} 2^(kappa g_j),
+//     the column factor computed once per block and iteration (l2gsum);
 //     a tile whose bound stays below rho by kVfMargin (base-2 units, far
 //     above the float32 rounding of the bound) is rejected here: its exact
 //     mass is below rho as well, so the admitted set is the same, at B
-//     exponentials per tile instead of B^2 (measured at n = m = 1e6: 1.83M
-//     of 3.67M candidates left for the exact test; a bound through the
+//     exponentials per tile instead of B^2 (measured at n = m = 1e6: 1.76M
+//     of 3.67M candidates left for the exact test, 1.83M with |J| 2^(kappa
+//     max g) as the column factor; a bound through the
 //     column side as well, or over 32-point sub-blocks of the column tile,
 //     left 7 % / 11 % fewer but cost more time than it saved);
 //  2. the exact mass of the others (taken in list order), 256 / B tiles per
@@ -344,7 +357,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
         const int seg = (int)(item % V.segs);
         const int64_t c0 = V.cptr[p], cp = V.cptr[p + 1] - c0;
         const int64_t k0 = c0 + cp * seg / V.segs, k1 = c0 + cp * (seg + 1) / V.segs;
-        // the block's points (caller's coordinates) and potentials for the row-level bound
+        // the block's points (caller's coordinates) and potentials for the point-level bound
         for (int r = tid; r < kB; r += kHsThreads) {
             const int64_t row = p * kB + r;
             const bool in = row < V.rows;
@@ -378,7 +391,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
             for (int t = tid; t < total; t += kHsThreads) s_list[t] = V.clist[w0 + t];
             __syncthreads();
 
-            // 1. row-level bound, one warp per candidate tile
+            // 1. point-level bound, one warp per candidate tile
             for (int t = warp; t < total; t += kHsThreads / 32) {
                 const int64_t q = s_list[t];
                 const BlockSum &cq = V.cs[q];
@@ -388,7 +401,6 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
                     lo[k] = (float)cq.lo[k];
                     hi[k] = (float)cq.hi[k];
                 }
-                const float gq = (float)cq.pmax;
                 float u[kB / 32], mx = -INFINITY;
 #pragma unroll
                 for (int k = 0; k < kB / 32; ++k) {
@@ -399,7 +411,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
                         const float gap = fmaxf(0.f, fmaxf(lo[e] - s_xr[r][e], s_xr[r][e] - hi[e]));
                         dist = fmaf(gap, gap, dist);
                     }
-                    u[k] = s_fr[r] == -INFINITY ? -INFINITY : kf * (s_fr[r] + gq - cf * dist);
+                    u[k] = s_fr[r] == -INFINITY ? -INFINITY : kf * (s_fr[r] - cf * dist);
                     mx = fmaxf(mx, u[k]);
                 }
                 for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -411,8 +423,8 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
                 }
                 for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
                 if (lane == 0) {
-                    const double lb = mx == -INFINITY ? -INFINITY
-                                                      : (double)mx + log2((double)sum) + cq.lncnt * 1.4426950408889634;
+                    const double lb = (mx == -INFINITY || cq.l2gsum == -INFINITY)
+                                          ? -INFINITY : (double)mx + log2((double)sum) + cq.l2gsum;
                     const double lrho = V.l2_delta + fmin(V.rs[p].l2w, cq.l2w);
                     const bool keep = lb + kVfMargin > lrho;
                     s_keep[t] = keep;
@@ -726,9 +738,10 @@ cudaError_t launch_block_static(const float *ps, const float *ws, int64_t cnt, i
     return cudaGetLastError();
 }
 
-cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, BlockSum *bs, cudaStream_t s) {
+cudaError_t launch_block_max(const float *pot, int64_t cnt, int B, double kappa, BlockSum *bs,
+                             cudaStream_t s) {
     const int64_t nblk = (cnt + B - 1) / B;
-    block_max_kernel<<<(unsigned)((nblk * 32 + 255) / 256), 256, 0, s>>>(pot, cnt, B, nblk, bs);
+    block_max_kernel<<<(unsigned)((nblk * 32 + 255) / 256), 256, 0, s>>>(pot, cnt, B, nblk, kappa, bs);
     return cudaGetLastError();
 }
 
