@@ -188,7 +188,7 @@ __global__ void block_static_kernel(const float *ps, const float *ws, int64_t cn
 
 // One warp per block: the largest potential (-inf for a massless block) and
 // log2 sum_j 2^(kappa pot_j) (float64), the column factor of the verification's
-// point-level bound.
+// row-level bound.
 __global__ void block_max_kernel(const float *pot, int64_t cnt, int B, int64_t nblk, double kappa,
                                  BlockSum *bs) {
     const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -302,7 +302,7 @@ __global__ void decide_kernel(const unsigned long long *cand, double limit, cons
 // leave a tail). The candidates come as compressed rows (cptr, clist) in
 // column order, taken kVfWindow at a time. Each candidate tile q is tested
 // against log2 rho = log2 delta + min(log2 amin_p, log2 bmin_q):
-//  1. a point-level bound, one warp per tile: with dist_i the distance from
+//  1. a row-level bound, one warp per tile: with dist_i the distance from
 //     x_i to q's bounding box (so C_ij >= c dist_i^2 for every j of q),
 //         M <= sum_i 2^(kappa (f_i - c dist_i^2)) * sum_{j in q} 2^(kappa g_j),
 //     the column factor computed once per block and iteration (l2gsum);
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
         const int seg = (int)(item % V.segs);
         const int64_t c0 = V.cptr[p], cp = V.cptr[p + 1] - c0;
         const int64_t k0 = c0 + cp * seg / V.segs, k1 = c0 + cp * (seg + 1) / V.segs;
-        // the block's points (caller's coordinates) and potentials for the point-level bound
+        // the block's points (caller's coordinates) and potentials for the row-level bound
         for (int r = tid; r < kB; r += kHsThreads) {
             const int64_t row = p * kB + r;
             const bool in = row < V.rows;
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kHsThreads, R == 2 ? 5 : 8) hs_verify_kernel(H
             for (int t = tid; t < total; t += kHsThreads) s_list[t] = V.clist[w0 + t];
             __syncthreads();
 
-            // 1. point-level bound, one warp per candidate tile
+            // 1. row-level bound, one warp per candidate tile
             for (int t = warp; t < total; t += kHsThreads / 32) {
                 const int64_t q = s_list[t];
                 const BlockSum &cq = V.cs[q];
