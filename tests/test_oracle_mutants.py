@@ -35,6 +35,9 @@ MUTANTS = {
     "threshold_takes_the_larger_weight": ("log(sp[1] < sq[1] ? sp[1] : sq[1])", "log(sp[1] > sq[1] ? sp[1] : sq[1])"),
     "sparse_f_without_fallback": ("if (all || adm[p * MB + j / B]) v[len++]", "if (adm[p * MB + j / B]) v[len++]"),
     "sparse_residual_counts_all_columns": ("if (all || adm[p * MB + j / B]) s +=", "s +="),
+    "sparse_stop_ignores_the_omitted_mass": ("const double tol_eff = tol - (double)MB * delta * asum;",
+                                             "const double tol_eff = tol;"),
+    "sparse_g_step_without_fallback": ("if (all || adm[(i / B) * MB + q]) v[len++]", "if (adm[(i / B) * MB + q]) v[len++]"),
 }
 
 
@@ -191,7 +194,24 @@ def _battery(orc):
         T = orc.dense_plan(xs, ys, fs, g2, 1.0, e2)
         if not np.allclose((T * rows).sum(1), aa, rtol=1e-12, atol=0):
             return False
-        return abs(orc.sparse_row_residual(xs, ys, aa, fs, g2, 1.0, e2, B, adm)) < 1e-13
+        if abs(orc.sparse_row_residual(xs, ys, aa, fs, g2, 1.0, e2, B, adm)) >= 1e-13:
+            return False
+        # the g-update with a column block that falls back to every row
+        adm2 = o["adm"].copy()
+        adm2[:, 3] = False
+        gs = orc.sparse_g_step(xs, ys, bb, fs, 1.0, e2, B, adm2)
+        cols = np.repeat(np.repeat(adm2, B, axis=0), B, axis=1)[:120, :100]
+        cols[:, 24:32] = True
+        T = orc.dense_plan(xs, ys, fs, gs, 1.0, e2)
+        if not np.allclose((T * cols).sum(0), bb, rtol=1e-12, atol=0):
+            return False
+        # the certificate: the stop test leaves room for the omitted mass
+        ux, uy = r2.random((400, 3)).astype(np.float32), r2.random((380, 3)).astype(np.float32)
+        ua, ub = np.full(400, 1 / 400), np.full(380, 1 / 380)
+        tol = 1e-2
+        _, _, _, rr, _ = orc.sinkhorn_sparse(ux, uy, ua, ub, 1.0, 4e-3, 300, tol=tol, B=32, dense_frac=1.0)
+        omitted = 12 * (tol / (4 * 13)) * ua.sum()
+        return rr <= tol - omitted
 
     for name, fn in [("block_sparse", block_sparse), ("row_marginals", row_marginals), ("col_marginals", col_marginals),
                      ("two_point", two_point), ("cross_ratio", cross_ratio),
