@@ -1,27 +1,39 @@
 """Benchmark of the online log-domain Sinkhorn hot path on B200.
 
-One step = the whole path on the 8000 x 8000, d = 3 Gaussian-mixture workload
-(scale "mean", eps 0.01): the solve to ||T1 - a||_1 <= 1e-3 (cap 2000, fused
-f/g half-steps with the in-loop residual), the float64-assembled marginal
-residual at the returned potentials, the exact min_row threshold and per-row
-counts in row blocks of 1024, the thresholded plan written in compressed-row
-form (the sparsify output), and the materialisation of every row in blocks of
-1024. Inputs are resident in HBM before the timed region; L2 is flushed before
-every step. The metric counts Sinkhorn pair-updates (n*m per half-step) per
-second; the row passes are inside the timed step but add no units. After the
-timed steps, the line's `large_n` object reports the d = 3 per-launch half-step
-at n = m = 1e5 against the same MUFU roofline, and its `block_sparse` object the
-block-sparse fine iterations at n = m = 2^18 against dense ones (skip both with
---no-large-n; `--sparse N` prints the full line at any size).
+The bench line runs workload 5, the largest configuration that fits one GPU:
+n = m = 2e6 points in 3-D (two interleaved spirals), scale "max_cost",
+eps 1e-3, uniform weights. One step is one call of the public entry point
+ot_sinkhorn_pointcloud continuing the solve from the previous step's
+potentials (warm start): the per-point tables, one iteration (the f- and the
+g-half-step, fused streaming log-sum-exp over on-the-fly costs) and the f-update
+that measures ||T1 - a||_1 of the new state (the fused residual and stop test),
+i.e. 3 half-steps of n*m pair-updates each. The scale is resolved by the first
+(warm-up) call's all-pairs max_cost pass and passed as a value afterwards (the
+captured scale is never re-derived). Inputs are resident in HBM before the
+timed region; the column tables (32 MB) fit in L2, so L2 is flushed (512 MiB
+write) before every step. `value` = pair-updates per second of device time.
+`e2e` repeats the step through ot_sinkhorn_pointcloud_host, the C-ABI call
+that takes HOST arrays (pinned here): x, y, a, b, f, g copied in and f, g copied
+out inside the timed region.
 
-    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload w2]
+Side objects, timed once after the steps on the same problem: `scale_pass` (the
+max_cost pass), `rows` (the row kernels at the solved state: one 1024-row
+materializer block of 1024 x 2e6 entries, the float64-assembled marginal
+residual and the exact min_row threshold with counts, both over all 4e12
+entries) and `block_sparse` (block-sparse fine iterations against dense ones at
+n = m = 2^18); --no-side skips them.
 
-Under torchrun (N > 1) every rank solves its own replica (no collective on the
-data path); rank 0 prints the JSON line with the max-over-ranks time.
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload w5]
+
+Under torchrun (N > 1) the same problem is split by rows across the ranks
+(strong scaling): each rank updates its range of rows, NCCL all-gathers the
+potentials after every half-step and all-reduces the residual; rank 0 prints
+the JSON line with the max-over-ranks time.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -36,11 +48,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Sinkhorn pair-updates/s (n·m per half-step) and % of ex2/MUFU roofline"
 UNIT = "pair-updates/s"
-# MUFU ex2 peak: 148 SMs x 16 ex2 per clock per SM x 1.965 GHz (max SM clock)
+# MUFU ex2 peak: 148 SMs x 16 ex2 per clock per SM x the maximum SM clock
 SMS, EX2_PER_CLK = 148, 16
-# DRAM bytes per half-step of the dominant kernel, from the committed ncu captures
-# of the current kernel, keyed by workload; None where no such capture exists
-HALFSTEP_TRAFFIC = {"w2_gmm3d_8000": 775.7e3 / 512}  # profiles/hs_loop_w2_8000.md
 
 
 def _peaks():
@@ -57,9 +66,11 @@ def _args():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="w2", choices=["w1", "w2", "w3", "w4", "w5"])
+    ap.add_argument("--workload", default="w5", choices=["w1", "w2", "w3", "w4", "w5"])
     ap.add_argument("--n", type=int, default=None, help="replica size of the workload (rows)")
     ap.add_argument("--m", type=int, default=None, help="replica size of the workload (columns)")
+    ap.add_argument("--iters-per-step", type=int, default=1,
+                    help="Sinkhorn iterations per step (one call continuing the solve)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lowrank", type=int, default=0, metavar="R",
                     help="instead of the step: time the two low-rank row materializers at rank R "
@@ -77,8 +88,8 @@ def _args():
                     help="--sparse: uniform-vs-64-clusters (w4) or interleaved spirals (w5)")
     ap.add_argument("--sparse-block", type=int, default=0, choices=[0, 128, 256],
                     help="--sparse: block size B (0 = the library's choice)")
-    ap.add_argument("--no-large-n", action="store_true",
-                    help="skip the d = 3 half-step measurement at n = m = 1e5")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side measurements (scale pass, row kernels, block-sparse)")
     ap.add_argument("--clock-ms", type=int, default=200,
                     help="nvidia-smi sampling period during the timed region")
     return ap.parse_args()
@@ -163,59 +174,40 @@ def _barrier(dist):
         dist.barrier()
 
 
-def _solve_kwargs(w):
-    kw = dict(eps=w.eps, scale=w.scale, n_iters=w.n_iters, tol=w.tol)
-    if w.anneal:
-        kw.update(eps_init=w.anneal["eps_init"], eps_decay=w.anneal["decay"],
-                  iters_per_stage=w.anneal["iters_per_stage"])
-    return kw
-
-
 class Step:
-    """The whole hot path on one workload, device-resident buffers reused across steps."""
+    """One step: a call of ot_sinkhorn_pointcloud that continues the solve for
+    `iters` iterations from the current potentials (warm start), on device
+    buffers that stay resident. The first call resolves the cost scale (the
+    all-pairs pass of "max_cost", or the closed form of "mean"); later calls
+    pass that captured value, so the scale is never re-derived."""
 
-    def __init__(self, ot, w, dev):
+    def __init__(self, ot, w, dev, iters=1):
         import torch
-        self.ot, self.w, self.dev = ot, w, dev
+        self.ot, self.w, self.dev, self.iters = ot, w, dev, iters
         self.x, self.y, self.a, self.b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev)
                                           for v in (w.x, w.y, w.a, w.b))
-        self.f = torch.empty(w.n, dtype=torch.float32, device=dev)
-        self.g = torch.empty(w.m, dtype=torch.float32, device=dev)
-        self.counts = torch.empty(w.n, dtype=torch.int64, device=dev)
-        self.block = w.block_rows if w.block_rows else 1024
-        rows = w.rows if w.rows is not None else (np.arange(w.n, dtype=np.int64) if w.block_rows else None)
-        self.rows = None if rows is None else torch.from_numpy(rows).to(dev)
-        self.out = None if rows is None else torch.empty((min(self.block, len(rows)), w.m),
-                                                         dtype=torch.float32, device=dev)
-        self.csr, self.nnz = None, 0
+        self.f = torch.zeros(w.n, dtype=torch.float32, device=dev)
+        self.g = torch.zeros(w.m, dtype=torch.float32, device=dev)
+        self.scale = w.scale  # becomes the captured value after the first call
+        self.iterations = 0
+
+    def kwargs(self, timing=False):
+        return dict(eps=self.w.eps, scale=self.scale, n_iters=self.iters, warm_start=True,
+                    timing=timing)
+
+    def capture(self, info):
+        if isinstance(self.scale, str) and self.scale != "none":
+            # the float32 max (or mean) the library resolved, exactly: c = 1 / value
+            self.scale = float(np.float32(1.0 / info.inv_scale_cost)) if self.scale == "max_cost" \
+                else 1.0 / info.inv_scale_cost
+        self.iterations += int(info.iterations)
 
     def __call__(self, timing=False):
-        w = self.w
-        plan = self.ot.sinkhorn(self.x, self.y, self.a, self.b, f=self.f, g=self.g, timing=timing,
-                                **_solve_kwargs(w))
-        launches = plan.info.kernel_launches
-        plan.marginal_residual()
-        launches += 6
-        mr = plan.sparsify_min_row(block_rows=w.block_rows, counts=self.counts)
-        nb = -(-w.n // (w.block_rows or w.n))
-        launches += 1 + 2 * nb + 2
-        # the sparse plan at that threshold, in compressed-row form
-        if self.csr is None or self.csr[1].numel() < mr["nnz"]:
-            import torch
-            cap = max(int(mr["nnz"] * 1.25), 1)
-            self.csr = (torch.empty(w.n + 1, dtype=torch.int64, device=self.dev),
-                        torch.empty(cap, dtype=torch.int64, device=self.dev),
-                        torch.empty(cap, dtype=torch.float32, device=self.dev))
-        self.nnz = plan.sparsify_csr(thr=mr["thr"], block_rows=w.block_rows, out=self.csr)["nnz"]
-        launches += 1 + 2 * nb + 3
-        if self.rows is not None:
-            for r0 in range(0, self.rows.numel(), self.block):
-                r = self.rows[r0:r0 + self.block]
-                plan.materialize_rows(r, out=self.out[:r.numel()])
-                launches += 2
+        plan = self.ot.sinkhorn(self.x, self.y, self.a, self.b, f=self.f, g=self.g, **self.kwargs(timing))
         info = plan.info
         plan.close()
-        return info, mr, launches
+        self.capture(info)
+        return info
 
 
 def _flush_l2(buf):
@@ -247,58 +239,68 @@ def _cpu_baseline(w, target_s=10.0):
                       f"(float64 C, OpenMP), {dt:.1f} s"}
 
 
-def _config(w, world, info=None):
+def _config(w, world, iters_per_step):
+    """The workload as the bench line names it (the same for both arms)."""
     cfg = {"workload": w.name, "n": w.n, "m": w.m, "d": w.d, "eps": w.eps, "scale": w.scale,
-           "tol": w.tol, "cap": w.n_iters, "block_rows": w.block_rows,
+           "weights": "uniform" if float(w.a.min()) == float(w.a.max()) else "non-uniform",
+           "step": f"ot_sinkhorn_pointcloud continuing the solve: {iters_per_step} iteration(s) "
+                   f"+ the residual f-update",
+           "half_steps_per_step": 2 * iters_per_step + 1,
            "l2": "flushed (512 MiB write) before every step",
            "parallelism": "replicas" if world > 1 else "single-gpu"}
     if w.anneal:
         cfg["anneal"] = w.anneal
-    if info is not None:
-        cfg["iterations"] = int(info.iterations)
-        cfg["half_steps"] = int(info.half_steps)
-        cfg["col_splits"] = int(info.col_splits)
     return cfg
 
 
 def run_reference(args):
-    """The oracle, as it stands, on the host cores: bounded row samples of one half-step."""
+    """The oracle, as it stands, on the host cores: bounded row samples of one
+    f-half-step of the same workload, at the same metric."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = _workload(args.workload, args.n, args.m)
-    times, units = [], 0
+    times = []
     for it in range(args.warmup + args.steps):
         cb = _cpu_baseline(w, target_s=8.0)
         if it >= args.warmup:
             times.append(cb)
     value = statistics.mean(t["value"] for t in times)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": _config(w, 1),
+            "config": _config(w, 1, args.iters_per_step),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": times[0]["cores"], "kind": "oracle",
                              "sample": times[0]["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def _large_n(ot, dev, n=100_000, iters=5):
-    """The d = 3 per-launch half-step at n = m = 1e5 (spiral clouds, eps 1e-3,
-    max_cost scale): microseconds per half-step from CUDA events on the
-    library's stream, as a fraction of the MUFU ex2 rate."""
-    import torch
-    from log_domain_sinkhorn_online_b200 import workloads
-    w = workloads.w5(n=n)
-    x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
-    ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=1, device_loop=0).close()
-    p = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=iters, device_loop=0, timing=True)
-    info = p.info
-    p.close()
-    us = info.loop_ms * 1e3 / max(info.half_steps, 1)
-    return {"workload": f"spirals3d_{n} replica (n = m = {n}, d = 3, eps 1e-3, scale max_cost)",
-            "kernel": "hs_lowd_kernel (fused f/g half-step)", "half_steps": info.half_steps,
-            "per_launch_us": us, "achieved": float(n) * n / (us / 1e6) / 1e12, "unit": "Tex2/s"}
+# DRAM traffic per launch of the dominant kernel comes from ncu captures
+# recorded in profiles/dram_traffic.json, each with a digest of the kernel's
+# source files at capture time: a kernel changed since then reports null.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+
+
+def kernel_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload, kernel):
+    try:
+        with open(TRAFFIC_FILE) as fh:
+            rec = json.load(fh).get(f"{workload}/{kernel}")
+    except (OSError, ValueError):
+        return None, "no capture recorded"
+    if not rec:
+        return None, "no capture recorded for this workload and kernel"
+    if kernel_digest(rec["sources"]) != rec["digest"]:
+        return None, "kernel source changed since the capture"
+    return float(rec["bytes_per_launch"]), rec.get("note", "")
 
 
 def run_lowrank(args, k=4096, m=100_000, n=20_000, reps=5):
@@ -442,7 +444,7 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
             pairs = float(info.tiles_admitted) * blk * blk * info.sparse_hs_launches
             hs_s = info.sparse_hs_ms / 1e3
             res[mode]["roofline"] = {
-                "bound": "alu", "kernel": "hs_sparse_kernel (block-sparse g half-step)",
+                "bound": "mufu", "kernel": "hs_sparse_kernel (block-sparse g half-step)",
                 "achieved": pairs / hs_s / 1e12, "peak": mufu / 1e12, "unit": "Tex2/s",
                 "frac": pairs / hs_s / mufu, "traffic": None,
                 "per_launch_us": info.sparse_hs_ms * 1e3 / max(info.sparse_hs_launches, 1)}
@@ -469,16 +471,167 @@ def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
     print(json.dumps(line), flush=True)
 
 
+CSRC = "log_domain_sinkhorn_online_b200/csrc/"
+# the dominant kernel of a workload's step and the sources that define it
+KERNELS = {
+    "hs_loop_kernel": [CSRC + f for f in ("loop.cu", "lowd.cuh", "finish.cuh", "common.cuh")],
+    "hs_lowd_kernel": [CSRC + f for f in ("halfstep.cu", "lowd.cuh", "finish.cuh", "common.cuh")],
+    "hs_tc_kernel": [CSRC + f for f in ("halfstep_tc.cu", "finish.cuh", "common.cuh")],
+    "hs_generic_kernel": [CSRC + f for f in ("halfstep.cu", "finish.cuh", "common.cuh")],
+}
+
+
+def _dominant_kernel(w):
+    if w.d <= 3:
+        return "hs_loop_kernel" if float(w.n) * w.m <= 2.0 ** 28 else "hs_lowd_kernel"
+    return "hs_tc_kernel" if w.d >= 16 else "hs_generic_kernel"
+
+
+def _timed(fn, stream):
+    """Runs fn once between CUDA events on `stream`; returns (result, ms)."""
+    import torch
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    r = fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return r, e0.elapsed_time(e1)
+
+
+def _side(ot, step, w, stream, peak_ex2, hbm_gbs):
+    """Side measurements on the solved problem (each call timed once, warm)."""
+    import torch
+    out = {}
+    # a1: the all-pairs max_cost pass (a plan built with no iteration)
+    if w.scale == "max_cost":
+        kw = dict(eps=w.eps, n_iters=0, warm_start=True, f=step.f.clone(), g=step.g.clone())
+        ot.sinkhorn(step.x, step.y, step.a, step.b, scale="max_cost", **kw).close()
+        _, ms = _timed(lambda: ot.sinkhorn(step.x, step.y, step.a, step.b, scale="max_cost", **kw).close(),
+                       stream)
+        out["scale_pass"] = {"what": "plan set-up with the all-pairs max_cost pass (max_cost_lowd_kernel)",
+                             "ms": ms, "pairs_per_s": float(w.n) * w.m / (ms / 1e3)}
+    # a8-a10 at the solved state, through one plan
+    plan = ot.sinkhorn(step.x, step.y, step.a, step.b, eps=w.eps, scale=step.scale, n_iters=0,
+                       warm_start=True, f=step.f.clone(), g=step.g.clone())
+    k = 1024
+    rows = torch.from_numpy(np.ascontiguousarray(w.rows[:k] if w.rows is not None
+                                                 else np.arange(min(k, w.n), dtype=np.int64))).to(step.dev)
+    buf = torch.empty((rows.numel(), w.m), dtype=torch.float32, device=step.dev)
+    plan.materialize_rows(rows, out=buf)
+    _, ms = _timed(lambda: plan.materialize_rows(rows, out=buf), stream)
+    gbs = rows.numel() * w.m * 4 / (ms / 1e3) / 1e9
+    out["materialize"] = {"kernel": "materialize_kernel", "rows": int(rows.numel()), "cols": w.m, "ms": ms,
+                          "gb_per_s": gbs, "frac_of_hbm": gbs / hbm_gbs}
+    (r, c), ms = _timed(plan.marginal_residual, stream)
+    ent = 2.0 * w.n * w.m
+    out["marginal_residual"] = {"kernel": "rowpass_kernel (sum)", "ms": ms, "row_l1": r, "col_l1": c,
+                                "entries_per_s": ent / (ms / 1e3), "frac_of_mufu": ent / (ms / 1e3) / peak_ex2}
+    mr, ms = _timed(lambda: plan.sparsify_min_row(block_rows=w.block_rows or 0), stream)
+    out["min_row"] = {"kernel": "rowpass_kernel (max, count)", "ms": ms, "thr": mr["thr"], "nnz": mr["nnz"],
+                      "entries_per_s": ent / (ms / 1e3), "frac_of_mufu": ent / (ms / 1e3) / peak_ex2}
+    plan.close()
+    del buf
+    return out
+
+
+def run_sharded(args, rank, world, dist, w, dev):
+    """N > 1: the solve split by rows across the ranks (log_domain_sinkhorn_online_b200.sharded):
+    per step one iteration and the residual f-update, each half-step followed by an NCCL
+    all-gather of the updated potential ranges, the residual summed by an all-reduce.
+    Strong scaling: the whole problem's pair-updates over the slowest rank's time."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import sharded as S
+    x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
+    xr, yr = S.Ranges(w.n, world), S.Ranges(w.m, world)
+    scale = w.scale
+    if scale == "max_cost":
+        scale = S.max_cost_value(x, y, xr, rank)
+    backend = S.CudaShard(x, y, a, b, w.eps, scale, xr, yr, rank)
+    solver = S.ShardedSinkhorn(backend, xr, yr, rank, world, like=x)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    warmup = max(args.warmup, 3)
+    for _ in range(warmup):
+        solver.solve(args.iters_per_step)
+    torch.cuda.synchronize()
+    clocks = Clocks(torch.cuda.current_device(), args.clock_ms)
+    _barrier(dist)
+    clocks.start()
+    total_ms, resid = 0.0, None
+    for _ in range(args.steps):
+        _flush_l2(flush)
+        (_, resid), ms = _timed(lambda: solver.solve(args.iters_per_step), stream)
+        total_ms += ms
+    clk = clocks.stop()
+    _barrier(dist)
+    total_ms = _max_over_ranks(total_ms, dist)
+    half_steps = 2 * args.iters_per_step + 1
+    units = float(w.n) * float(w.m) * half_steps  # the whole problem's pair-updates per step
+    value = units / (total_ms / args.steps / 1e3)
+    # e2e: every rank's inputs and the potentials from and to pinned host memory
+    host = [t.cpu().pin_memory() for t in (x, y, a, b)]
+    fh = torch.zeros(w.n, dtype=torch.float32).pin_memory()
+    gh = torch.zeros(w.m, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_ms = 0.0
+
+    def e2e_step():
+        for dst, src in zip((x, y, a, b), host):
+            dst.copy_(src, non_blocking=True)
+        solver.f[solver.k][:w.n].copy_(fh, non_blocking=True)
+        solver.g[:w.m].copy_(gh, non_blocking=True)
+        solver.solve(args.iters_per_step)
+        f, g = solver.potentials()
+        fh.copy_(f, non_blocking=True)
+        gh.copy_(g, non_blocking=True)
+
+    _barrier(dist)
+    for _ in range(e2e_steps):
+        _flush_l2(flush)
+        _, ms = _timed(e2e_step, stream)
+        e2e_ms += ms
+    e2e_ms = _max_over_ranks(e2e_ms, dist)
+    backend.close()
+    if rank == 0:
+        peaks, kind = _peaks()
+        sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded point clouds; recipe in log_domain_sinkhorn_online_b200/workloads.py)",
+                "config": dict(_config(w, world, args.iters_per_step), parallelism=f"rows split over {world} GPUs"),
+                "clocks": clk,
+                "e2e": {"value": units * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                        "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host) + 4 * (w.n + w.m),
+                        "d2h_bytes_per_step": 4 * (w.n + w.m), "steps": e2e_steps,
+                        "call": "ot_shard_half_step per rank, NCCL all-gathers (pinned host arrays)"},
+                "gpu_launches": 2 * half_steps * args.steps,
+                "roofline": {"bound": "mufu", "kernel": _dominant_kernel(w) + " (fused f/g half-step, row range)",
+                             "achieved": units / world / (total_ms / args.steps / 1e3) / 1e12,
+                             "peak": SMS * EX2_PER_CLK * sm_max * 1e6 / 1e12, "unit": "Tex2/s per GPU",
+                             "frac": units / world / (total_ms / args.steps / 1e3) / (SMS * EX2_PER_CLK * sm_max * 1e6),
+                             "traffic": None, "traffic_note": "not captured for the split solve",
+                             "note": "per GPU, whole step time (collectives included)"},
+                "run": {"last_residual": resid}}
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+
+
 def run_ours(args):
     import torch
     import log_domain_sinkhorn_online_b200 as ot
+    from log_domain_sinkhorn_online_b200 import _binding as B
     rank, world, dist = _dist_init(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     w = _workload(args.workload, args.n, args.m)
-    step = Step(ot, w, dev)
+    if world > 1:
+        return run_sharded(args, rank, world, dist, w, dev)
+    step = Step(ot, w, dev, args.iters_per_step)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    for _ in range(max(args.warmup, 3)):
+    warmup = max(args.warmup, 3)
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
 
@@ -486,93 +639,74 @@ def run_ours(args):
     clocks = Clocks(torch.cuda.current_device(), args.clock_ms)
     _barrier(dist)
     clocks.start()
-    total_ms, loop_ms, half_steps, launches, info = 0.0, 0.0, 0, 0, None
+    total_ms, loop_ms, half_steps, launches = 0.0, 0.0, 0, 0
     for _ in range(args.steps):
         _flush_l2(flush)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        info, mr, nl = step(timing=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        total_ms += e0.elapsed_time(e1)
+        info, ms = _timed(lambda: step(timing=True), stream)
+        total_ms += ms
         loop_ms += info.loop_ms
         half_steps += info.half_steps
-        launches += nl
+        launches += info.kernel_launches
     clk = clocks.stop()
     _barrier(dist)
     total_ms = _max_over_ranks(total_ms, dist)
     units = float(w.n) * float(w.m) * half_steps / args.steps  # pair-updates per step (this rank)
     value = weak_scaling_value(units, world, total_ms / args.steps)
 
-    # ---- end to end through the public API: pinned host inputs in, results out
-    host = [torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for v in (w.x, w.y, w.a, w.b)]
-    outs = [torch.empty(w.n, dtype=torch.float32).pin_memory(), torch.empty(w.m, dtype=torch.float32).pin_memory(),
-            torch.empty(w.n, dtype=torch.int64).pin_memory()]
-    # the sparse plan (row pointers, column indices, values) comes back too
-    csr_host = None if step.csr is None else [torch.empty(t.numel(), dtype=t.dtype).pin_memory()
-                                              for t in step.csr]
+    # ---- end to end through the C-ABI call that takes host arrays (pinned)
+    host = [t.cpu().pin_memory() for t in (step.x, step.y, step.a, step.b, step.f, step.g)]
+    opt = B.ot_options_default()
+    opt.warm_start = 1
+    sc = B.OT_SCALE_VALUE if not isinstance(step.scale, str) else B.OT_SCALE_NONE
+    if sc == B.OT_SCALE_VALUE:
+        opt.scale_value = float(step.scale)
     h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = sum(t.numel() * t.element_size() for t in outs)
-    if csr_host is not None:
-        d2h += (w.n + 1) * 8 + step.nnz * (8 + 4)
+    d2h = (w.n + w.m) * 4
+    e2e_steps = max(1, min(args.steps, 5))
     e2e_ms, e2e_units = 0.0, 0.0
     _barrier(dist)
-    for _ in range(args.steps):
+    for _ in range(e2e_steps):
         _flush_l2(flush)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for dst, src in zip((step.x, step.y, step.a, step.b), host):
-            dst.copy_(src, non_blocking=True)
-        inf, _, _ = step()
-        outs[0].copy_(step.f, non_blocking=True)
-        outs[1].copy_(step.g, non_blocking=True)
-        outs[2].copy_(step.counts, non_blocking=True)
-        if csr_host is not None:
-            csr_host[0].copy_(step.csr[0], non_blocking=True)
-            csr_host[1][:step.nnz].copy_(step.csr[1][:step.nnz], non_blocking=True)
-            csr_host[2][:step.nnz].copy_(step.csr[2][:step.nnz], non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms += e0.elapsed_time(e1)
+        (_, _, inf), ms = _timed(lambda: B.ot_sinkhorn_pointcloud_host(
+            *(t.data_ptr() for t in host[:4]), w.n, w.m, w.d, float(w.eps), sc, args.iters_per_step, 0.0,
+            host[4].data_ptr(), host[5].data_ptr(), stream.cuda_stream, opt), stream)
+        e2e_ms += ms
         e2e_units += float(w.n) * float(w.m) * inf.half_steps
     e2e_ms = _max_over_ranks(e2e_ms, dist)
     e2e_value = e2e_units * world / (e2e_ms / 1e3)
-    large = _large_n(ot, dev) if w.d <= 3 and not args.no_large_n else None
-    # the block-sparse fine iterations at n = m = 2^18 (a few seconds; --sparse N alone
-    # gives the same line at any size)
-    sparse_line = run_sparse(args, emit=False) if (not args.no_large_n and rank == 0) else None
 
     if rank == 0:
         peaks, kind = _peaks()
         sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-        peak_tex2 = SMS * EX2_PER_CLK * sm_max * 1e6 / 1e12
+        peak_ex2 = SMS * EX2_PER_CLK * sm_max * 1e6
+        side = _side(ot, step, w, stream, peak_ex2, float(peaks["hbm_gbs"])) if not args.no_side else None
+        sparse_line = run_sparse(args, emit=False) if (not args.no_side and w.d <= 3) else None
         per_launch_ms = loop_ms / max(half_steps, 1)
-        achieved = float(w.n) * float(w.m) / (per_launch_ms / 1e3) / 1e12
+        achieved = float(w.n) * float(w.m) / (per_launch_ms / 1e3)
+        kname = _dominant_kernel(w)
+        traffic, tnote = _traffic(w.name if (args.n, args.m) == (None, None) else None, kname)
+        roof = {"bound": "mufu", "kernel": kname + " (fused f/g half-step)",
+                "achieved": achieved / 1e12, "peak": peak_ex2 / 1e12, "unit": "Tex2/s",
+                "frac": achieved / peak_ex2, "traffic": traffic, "traffic_note": tnote,
+                "per_launch_us": per_launch_ms * 1e3,
+                "peak_note": f"derived: 148 SMs x 16 MUFU ex2/clk x {sm_max:.0f} MHz ({kind} sm_max); "
+                             "one ex2 per pair-update"}
+        if clk.get("sm_mhz"):
+            roof["frac_at_sampled_clock"] = achieved / (SMS * EX2_PER_CLK * clk["sm_mhz"] * 1e6)
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "warmup": warmup, "ms_per_step": total_ms / args.steps,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded point clouds; recipe in log_domain_sinkhorn_online_b200/workloads.py)",
-                "config": _config(w, world, info),
-                "roofline": {"bound": "alu", "kernel": ("hs_loop_kernel (device-resident f/g half-steps)"
-                                                        if float(w.n) * w.m <= 2.0 ** 28 else
-                                                        "hs_lowd_kernel (fused f/g half-step)") if w.d <= 3
-                             else "hs_tc_kernel (fused f/g half-step, tcgen05 x.y)" if w.d >= 16
-                             else "hs_generic_kernel (fused f/g half-step)",
-                             "achieved": achieved, "peak": peak_tex2, "unit": "Tex2/s",
-                             "frac": achieved / peak_tex2,
-                             "traffic": HALFSTEP_TRAFFIC.get(w.name) if (args.n, args.m) == (None, None) else None,
-                             "per_launch_us": per_launch_ms * 1e3,
-                             "peak_note": f"148 SMs x 16 MUFU ex2/clk x {sm_max:.0f} MHz ({kind} sm_max)"},
-                "clocks": clk,
+                "config": _config(w, world, args.iters_per_step),
+                "roofline": roof, "clocks": clk,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h},
-                "gpu_launches": launches}
-        if large is not None:
-            large["peak"] = peak_tex2
-            large["frac"] = large["achieved"] / peak_tex2
-            line["large_n"] = large
+                        "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                        "call": "ot_sinkhorn_pointcloud_host (pinned host arrays)"},
+                "gpu_launches": launches,
+                "run": {"iterations_done": step.iterations, "half_steps_timed": half_steps,
+                        "last_residual": float(info.residual), "col_splits": int(info.col_splits)}}
+        if side:
+            line.update(side)
         if sparse_line is not None:
             sp = sparse_line["sparse"]
             line["block_sparse"] = {

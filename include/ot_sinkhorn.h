@@ -29,6 +29,8 @@
  *    non-OK status of the calling thread.
  *  - No CPU fallback exists: without a usable sm_100 device every call that
  *    computes returns OT_ERR_CUDA.
+ *  - Each call is wrapped in an NVTX range named after it (visible to Nsight
+ *    tools; a no-op without one).
  */
 #ifndef OT_SINKHORN_H
 #define OT_SINKHORN_H
@@ -39,7 +41,7 @@
 extern "C" {
 #endif
 
-#define OT_ABI_VERSION 2
+#define OT_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define OT_API __attribute__((visibility("default")))
@@ -128,6 +130,14 @@ typedef struct ot_options {
     double sparse_dense_frac; /* an iteration whose candidate tiles exceed this fraction of
                                  all NB * MB block pairs runs the dense half-steps instead
                                  (default 0.5) */
+    double *resid_history;    /* optional device float64 array [resid_history_len]: entry
+                                 k - 1 receives ||T 1 - a||_1 of the state after iteration k
+                                 (all stages counted), as measured in the loop by the next
+                                 f-update (FlashSinkhorn 2, section 3.1: the marginal residual
+                                 is the convergence measure). Entries no f-update measured
+                                 (the last iteration of each annealing stage but the final
+                                 one; iterations beyond the run) are NaN. NULL: none */
+    int64_t resid_history_len;/* entries of resid_history (0 = none) */
 } ot_options;
 
 /* -------------------------------------------------------- solve report   */
@@ -175,7 +185,9 @@ OT_API const char *ot_last_error_string(void);
 
 /* Default options (warm_start 0, check_every 16, use_graphs 1,
  * iters_per_stage 20, scale_value 1, eps_init 0, eps_decay 0.7, timing 0,
- * col_splits 0, rows_per_thread 0, tensor_cores 1, device_loop -1). */
+ * col_splits 0, rows_per_thread 0, tensor_cores 1, device_loop -1,
+ * block_sparse 0, sparse_block 0, sparse_verify 1, sparse_delta 0,
+ * sparse_dense_frac 0.5, resid_history NULL, resid_history_len 0). */
 OT_API void ot_options_default(ot_options *opt);
 
 /* ------------------------------------------------- ot_sinkhorn_pointcloud
@@ -209,6 +221,23 @@ OT_API int ot_sinkhorn_pointcloud(const float *x, const float *y, const float *a
                            int64_t n, int64_t m, int32_t d, double eps, ot_scale scale_cost,
                            int32_t n_iters, double tol, float *f, float *g, void *stream,
                            const ot_options *opt, ot_plan **plan_out, ot_info *info);
+
+/* ------------------------------------------------ ot_sinkhorn_pointcloud_host
+ * ot_sinkhorn_pointcloud for a caller that holds its arrays in HOST memory:
+ * x, y, a, b (and f, g with opt->warm_start) are copied to the device on
+ * `stream`, the problem is solved as above, and f, g are copied back into the
+ * caller's host arrays before the call returns. Host arrays may be pageable or
+ * pinned (pinned ones copy asynchronously and faster). The device copies come
+ * from the library's workspace cache; if plan_out is non-NULL the plan owns
+ * them (its row calls then take DEVICE row_idx / out arrays as usual) and
+ * ot_plan_destroy returns them, otherwise they are released before the call
+ * returns. Arguments, statuses and info are those of ot_sinkhorn_pointcloud.
+ * Synchronises `stream`. */
+OT_API int ot_sinkhorn_pointcloud_host(const float *x, const float *y, const float *a,
+                                       const float *b, int64_t n, int64_t m, int32_t d, double eps,
+                                       ot_scale scale_cost, int32_t n_iters, double tol, float *f,
+                                       float *g, void *stream, const ot_options *opt,
+                                       ot_plan **plan_out, ot_info *info);
 
 /* ---------------------------------------------------- ot_marginal_residual
  * row_l1 = sum_i |sum_j T_ij - a_i|, col_l1 = sum_j |sum_i T_ij - b_j| at the
@@ -327,6 +356,58 @@ OT_API int ot_marginal_residual_noalloc(const float *x, const float *y, const fl
                                         int64_t n, int64_t m, int32_t d, double eps,
                                         double inv_scale_cost, double *row_l1, double *col_l1,
                                         void *stream);
+
+/* ------------------------------------------------------------ sharded solve
+ * The solve split by rows across several GPUs ("FlashSinkhorn 2: Block-Sparse
+ * Entropic Optimal Transport", section 5: at 10^10 points one measure exceeds a
+ * single GPU, so the work is spread over several). Every rank holds x, y, a, b
+ * in full and updates one contiguous range of x's rows in the f-update and of
+ * y's rows in the g-update; between the half-steps the caller exchanges the
+ * updated ranges (an all-gather of the potential, e.g. NCCL over NVLink) and,
+ * for a stopping test, sums the ranks' residual partials (an all-reduce). The
+ * kernels are those of ot_sinkhorn_pointcloud; the half-step of a row tile
+ * depends only on that tile's rows and the other side's whole potential, so a
+ * tile-aligned split with the same opt->col_splits and opt->rows_per_thread
+ * gives the unsplit solve's potentials bit for bit. */
+
+/* ot_max_sqdist: *out = max over i in [x_lo, x_hi), j < m of ||x_i - y_j||^2,
+ * evaluated exactly as the OT_SCALE_MAX_COST pass does (float32 on coordinates
+ * shifted by the midpoint of the clouds' means), so the max over ranks of their
+ * ranges' values is the unsplit max_cost, and OT_SCALE_VALUE with that value
+ * resolves the same inv_scale_cost. x [n,d], y [m,d]: device float32; out:
+ * host float (0 for an empty range). Synchronises `stream`. */
+OT_API int ot_max_sqdist(const float *x, const float *y, int64_t n, int64_t m, int32_t d,
+                         int64_t x_lo, int64_t x_hi, float *out, void *stream);
+
+/* ot_shard_plan_create: a plan for the rows [x_lo, x_hi) of x and [y_lo, y_hi)
+ * of y (0 <= lo <= hi <= n or m; lo a multiple of 8; empty ranges allowed),
+ * with eps and the scale resolved as in ot_sinkhorn_pointcloud (pass the
+ * max_cost of all ranks as OT_SCALE_VALUE, see ot_max_sqdist). x, y, a, b are
+ * borrowed as by a solve. Honoured options: scale_value, col_splits,
+ * rows_per_thread, tensor_cores; block_sparse is OT_ERR_UNSUPPORTED. info (may
+ * be NULL) receives inv_scale_cost, eps, the massless counts and col_splits.
+ * The plan serves ot_shard_half_step only (row calls refuse it); free it with
+ * ot_plan_destroy. Synchronises `stream`. */
+OT_API int ot_shard_plan_create(const float *x, const float *y, const float *a, const float *b,
+                                int64_t n, int64_t m, int32_t d, double eps, ot_scale scale_cost,
+                                int64_t x_lo, int64_t x_hi, int64_t y_lo, int64_t y_hi, void *stream,
+                                const ot_options *opt, ot_plan **plan_out, ot_info *info);
+
+/* ot_shard_half_step: one half-step over the plan's rows of one side.
+ *  side 0 (f-update): other = g [m] (all of it), cur = f [n] before the update
+ *      (the rows of the range are read), out = f [n]: the range's rows are
+ *      written; out may equal cur.
+ *  side 1 (g-update): other = f [n], cur / out = g [m] likewise.
+ *  resid: host double or NULL: the range's part of ||T1 - a||_1 (side 0) or of
+ *      ||T^T 1 - b||_1 (side 1) at the state BEFORE the update (cur and other),
+ *      the terms the single-GPU solve sums for its stopping test; the sum over
+ *      ranks is the whole residual.
+ * Work is queued on `stream` after what is already there; the call returns at
+ * once unless resid is non-NULL or the range is non-empty (then it reads the
+ * plan's status back and synchronises). A potential that leaves the finite
+ * range returns OT_ERR_NONFINITE. */
+OT_API int ot_shard_half_step(ot_plan *plan, int32_t side, const float *other, const float *cur,
+                              float *out, double *resid, void *stream);
 
 /* Plans take their device workspace, pinned read-back buffer and internal
  * stream from a per-device cache and return them there when destroyed, so

@@ -169,7 +169,7 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
              check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,
              timing=False, col_splits=0, rows_per_thread=0, tensor_cores=True,
              device_loop=-1, block_sparse=False, sparse_block=0, sparse_verify=True,
-             sparse_delta=0.0, sparse_dense_frac=0.5, stream=None) -> Plan:
+             sparse_delta=0.0, sparse_dense_frac=0.5, resid_history=None, stream=None) -> Plan:
     """Solves on the GPU; x [n,d], y [m,d], a [n], b [m] float32 CUDA tensors.
 
     block_sparse (d <= 3): block-sparse fine iterations ("FlashSinkhorn 2",
@@ -179,6 +179,9 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
     half-steps over the admitted tiles only; an iteration whose candidates
     exceed sparse_dense_frac of all pairs runs dense. f and g come back in the
     caller's order.
+
+    resid_history: optional float64 CUDA tensor; entry k - 1 receives the
+    in-loop ||T1 - a||_1 after iteration k (NaN where none was measured).
     """
     import torch
     x, y = _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y")
@@ -204,6 +207,10 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
     opt.sparse_verify = int(bool(sparse_verify))
     opt.sparse_delta = float(sparse_delta)
     opt.sparse_dense_frac = float(sparse_dense_frac)
+    if resid_history is not None:
+        _dev(resid_history, torch.float64, "resid_history")
+        opt.resid_history = resid_history.data_ptr()
+        opt.resid_history_len = resid_history.numel()
     if isinstance(scale, str):
         sc = _SCALES[scale]
     else:

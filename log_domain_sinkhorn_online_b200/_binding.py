@@ -28,9 +28,11 @@ OT_SCALE_NONE, OT_SCALE_MEAN, OT_SCALE_MAX_COST, OT_SCALE_VALUE = 0, 1, 2, 3
 
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sinkhorn_pointcloud",
-            "ot_marginal_residual", "ot_materialize_rows", "ot_sparsify_min_row", "ot_plan_destroy",
-            "ot_marginal_residual_noalloc", "ot_trim_cache", "ot_sparsify_csr",
-            "ot_materialize_rows_lowrank", "ot_materialize_rows_lrcost")
+            "ot_sinkhorn_pointcloud_host", "ot_marginal_residual", "ot_materialize_rows",
+            "ot_sparsify_min_row", "ot_plan_destroy", "ot_marginal_residual_noalloc", "ot_trim_cache",
+            "ot_sparsify_csr", "ot_materialize_rows_lowrank", "ot_materialize_rows_lrcost",
+            "ot_testing_fail_device_allocs", "ot_testing_wait_fault", "ot_max_sqdist",
+            "ot_shard_plan_create", "ot_shard_half_step")
 OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
@@ -44,7 +46,8 @@ class OtOptions(ctypes.Structure):
                 ("reserved1", ctypes.c_int32), ("block_sparse", ctypes.c_int32),
                 ("sparse_block", ctypes.c_int32), ("sparse_verify", ctypes.c_int32),
                 ("reserved2", ctypes.c_int32), ("sparse_delta", ctypes.c_double),
-                ("sparse_dense_frac", ctypes.c_double)]
+                ("sparse_dense_frac", ctypes.c_double), ("resid_history", ctypes.c_void_p),
+                ("resid_history_len", ctypes.c_int64)]
 
 
 class OtInfo(ctypes.Structure):
@@ -87,6 +90,20 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.POINTER(OtOptions), ctypes.POINTER(P),
                                                  ctypes.POINTER(OtInfo)]
             L.ot_sinkhorn_pointcloud.restype = ctypes.c_int
+            L.ot_sinkhorn_pointcloud_host.argtypes = L.ot_sinkhorn_pointcloud.argtypes
+            L.ot_sinkhorn_pointcloud_host.restype = ctypes.c_int
+            L.ot_max_sqdist.argtypes = [P, P, I64, I64, I32, I64, I64, ctypes.POINTER(ctypes.c_float), P]
+            L.ot_max_sqdist.restype = ctypes.c_int
+            L.ot_shard_plan_create.argtypes = [P, P, P, P, I64, I64, I32, D, ctypes.c_int, I64, I64, I64, I64,
+                                               P, ctypes.POINTER(OtOptions), ctypes.POINTER(P),
+                                               ctypes.POINTER(OtInfo)]
+            L.ot_shard_plan_create.restype = ctypes.c_int
+            L.ot_shard_half_step.argtypes = [P, I32, P, P, P, ctypes.POINTER(D), P]
+            L.ot_shard_half_step.restype = ctypes.c_int
+            L.ot_testing_fail_device_allocs.argtypes = [ctypes.c_int]
+            L.ot_testing_fail_device_allocs.restype = None
+            L.ot_testing_wait_fault.argtypes = [ctypes.c_int]
+            L.ot_testing_wait_fault.restype = None
             L.ot_marginal_residual.argtypes = [P, ctypes.POINTER(D), ctypes.POINTER(D), P]
             L.ot_marginal_residual.restype = ctypes.c_int
             L.ot_materialize_rows.argtypes = [P, P, I64, P, P]
@@ -143,6 +160,56 @@ def ot_sinkhorn_pointcloud(x, y, a, b, n, m, d, eps, scale_cost, n_iters, tol, f
                                       ctypes.byref(info))
     _check(st)
     return st, (plan.value if want_plan else None), info
+
+
+def ot_sinkhorn_pointcloud_host(x, y, a, b, n, m, d, eps, scale_cost, n_iters, tol, f, g, stream,
+                                opt: OtOptions | None = None, want_plan: bool = False):
+    """As ot_sinkhorn_pointcloud with HOST pointers for x, y, a, b, f, g (the
+    library copies them in and f, g back). Returns (status, plan or None, OtInfo)."""
+    plan = ctypes.c_void_p()
+    info = OtInfo()
+    st = lib().ot_sinkhorn_pointcloud_host(x, y, a, b, n, m, d, eps, int(scale_cost), n_iters, tol, f, g,
+                                           stream, ctypes.byref(opt) if opt is not None else None,
+                                           ctypes.byref(plan) if want_plan else None,
+                                           ctypes.byref(info))
+    _check(st)
+    return st, (plan.value if want_plan else None), info
+
+
+def ot_max_sqdist(x, y, n, m, d, x_lo, x_hi, stream) -> float:
+    """max over i in [x_lo, x_hi), all j of ||x_i - y_j||^2 (the max_cost pass's value)."""
+    out = ctypes.c_float()
+    _check(lib().ot_max_sqdist(x, y, n, m, d, x_lo, x_hi, ctypes.byref(out), stream))
+    return out.value
+
+
+def ot_shard_plan_create(x, y, a, b, n, m, d, eps, scale_cost, x_lo, x_hi, y_lo, y_hi, stream,
+                         opt: OtOptions | None = None):
+    """Returns (plan handle, OtInfo) of a plan for the given row ranges."""
+    plan = ctypes.c_void_p()
+    info = OtInfo()
+    _check(lib().ot_shard_plan_create(x, y, a, b, n, m, d, eps, int(scale_cost), x_lo, x_hi, y_lo, y_hi,
+                                      stream, ctypes.byref(opt) if opt is not None else None,
+                                      ctypes.byref(plan), ctypes.byref(info)))
+    return plan.value, info
+
+
+def ot_shard_half_step(plan, side, other, cur, out, stream, want_resid=True):
+    """One half-step over the plan's rows; returns the range's residual part (or None)."""
+    r = ctypes.c_double()
+    _check(lib().ot_shard_half_step(plan, side, other, cur, out, ctypes.byref(r) if want_resid else None,
+                                    stream))
+    return r.value if want_resid else None
+
+
+def ot_testing_fail_device_allocs(after: int) -> None:
+    """Failure tests only: the device allocation after `after` more fails (see the testing header)."""
+    lib().ot_testing_fail_device_allocs(int(after))
+
+
+def ot_testing_wait_fault(mode: int) -> None:
+    """Failure tests only: make one bounded device wait give up (see the testing header)."""
+    lib().ot_testing_wait_fault(int(mode))
 
 
 def ot_marginal_residual(plan, stream):

@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "ot_sinkhorn.h"
+#include "ot_sinkhorn_testing.h"
 #include "runtime.h"
 
 using namespace ot;
@@ -24,6 +25,10 @@ using namespace ot;
 namespace {
 
 thread_local char g_err[512] = "no error";
+
+// failure tests (include/ot_sinkhorn_testing.h): which bounded device wait to
+// make give up, 0 = none
+std::atomic<int> g_wait_fault{0};
 
 }  // namespace
 
@@ -84,6 +89,7 @@ struct HostScalars {
 
 struct Side {          // one cloud's half of the problem
     int64_t cnt, pad;  // points, padded to kColPad
+    int64_t lo, rows;  // the rows this plan updates: [lo, lo + rows) (all of them unless sharded)
     float *rowtab;     // [pad][dp]
     float *coltab;     // layout per kind
     int tiles, splits, grid;
@@ -101,6 +107,7 @@ struct ot_plan {
     int64_t n = 0, m = 0;
     int d = 0, kind = 0, dim = 0, dp = 0;
     double eps = 0.0, c = 1.0;
+    double mean_sq = 0.0;  // mean over all pairs of ||x_i - y_j||^2 (closed form)
     int64_t n_massless_rows = 0, n_massless_cols = 0;
     // workspace (one allocation, carved)
     char *ws = nullptr;
@@ -140,6 +147,12 @@ struct ot_plan {
     double sp_delta = 0.0, sp_frac = 0.5, sp_bound = 0.0, asum = 0.0;
     char *ws_sp = nullptr;
     size_t ws_sp_bytes = 0;
+    // sharded plan (ot_shard_plan_create): the row ranges [lo, hi) of x and y it updates
+    bool shard = false;
+    int64_t range[2][2] = {{0, 0}, {0, 0}};
+    // ot_sinkhorn_pointcloud_host: the device copies of the caller's host arrays
+    char *ws_in = nullptr;
+    size_t ws_in_bytes = 0;
     int64_t *perm_x = nullptr, *perm_y = nullptr;
     unsigned long long *keys = nullptr;
     BlockSum *bsx = nullptr, *bsy = nullptr;
@@ -174,6 +187,11 @@ namespace {
 
 void plan_free(ot_plan *p) {
     if (!p) return;
+    // everything below belongs to the plan's device, which need not be the
+    // current one (a plan may be destroyed from any thread, under any device)
+    int prev = -1;
+    const bool swap = cudaGetDevice(&prev) == cudaSuccess && prev != p->device &&
+                      cudaSetDevice(p->device) == cudaSuccess;
     for (auto &gx : p->graph)
         if (gx) cudaGraphExecDestroy(gx);
     for (auto ev : p->tev) cudaEventDestroy(ev);
@@ -181,13 +199,15 @@ void plan_free(ot_plan *p) {
     for (auto ev : p->tm_hs.ev) cudaEventDestroy(ev);
     // the workspaces and the stream go back to the pool once the plan's work is done
     if (p->s_int) cudaStreamSynchronize(p->s_int);
-    pool_device_free(p->ws, p->ws_bytes);
-    pool_device_free(p->ws_rows, p->ws_rows_bytes);
-    pool_device_free(p->ws_sp, p->ws_sp_bytes);
+    pool_device_free(p->ws, p->ws_bytes, p->device);
+    pool_device_free(p->ws_rows, p->ws_rows_bytes, p->device);
+    pool_device_free(p->ws_sp, p->ws_sp_bytes, p->device);
+    pool_device_free(p->ws_in, p->ws_in_bytes, p->device);
     pool_host_free(p->hs, sizeof(HostScalars));
     if (p->ev_in) cudaEventDestroy(p->ev_in);
     if (p->ev_out) cudaEventDestroy(p->ev_out);
-    pool_stream_release(p->s_int);
+    pool_stream_release(p->s_int, p->device);
+    if (swap) cudaSetDevice(prev);
     delete p;
 }
 
@@ -333,8 +353,9 @@ HalfStep make_step(const ot_plan *p, int side, int parity) {
     const Side &cols = f ? p->sy : p->sx;
     float *const *fb = p->sf;
     A.coltab = reinterpret_cast<const float4 *>(cols.coltab);
-    A.rowtab = rows.rowtab;
-    A.rows = rows.cnt;
+    A.rowtab = rows.rowtab + rows.lo * p->dp;
+    A.rows = rows.rows;
+    A.row_off = rows.lo;
     A.cols_pad = cols.pad;
     A.cols_per_split = rows.cps;
     A.splits = rows.splits;
@@ -345,22 +366,29 @@ HalfStep make_step(const ot_plan *p, int side, int parity) {
     A.part = p->part;
     A.tile_cnt = p->tile_cnt;
     A.tile_resid = p->tile_resid;
-    A.w = f ? p->sa : p->sb;
-    A.pot_old = f ? fb[parity] : p->sg;
-    A.pot_new = f ? fb[parity ^ 1] : p->sg;
-    A.next_col = rows.coltab;  // this side's column table feeds the other half-step
+    A.w = (f ? p->sa : p->sb) + rows.lo;
+    A.pot_old = (f ? fb[parity] : p->sg) + rows.lo;
+    A.pot_new = (f ? fb[parity ^ 1] : p->sg) + rows.lo;
+    // this side's column table feeds the other half-step; row r of the update is
+    // point lo + r (lo is even: pairs of columns share a record in layout 0)
+    A.next_col = rows.coltab;
     A.nxt_bf16 = 0;
     if (p->kind == 0) {
         A.nxt_a = 8; A.nxt_l = 1; A.nxt_b = 6;
+        A.next_col += (rows.lo >> 1) * 8;
     } else if (p->kind == 1) {
         A.nxt_a = 2 * (p->dp + 4); A.nxt_l = p->dp + 4; A.nxt_b = p->dp;
+        A.next_col += rows.lo * (p->dp + 4);
     } else {
-        A.next_col = static_cast<float *>(rows.bcol);
+        A.next_col = static_cast<float *>(rows.bcol) + (rows.lo * p->kp) / 2;  // bf16 elements
         A.nxt_bf16 = 1;
         A.nxt_a = p->kp; A.nxt_l = 0; A.nxt_b = 3 * p->d;
     }
     A.prm = p->prm;
     A.st = p->st;
+    const bool fault = g_wait_fault.load() == 2;
+    A.wait_polls = fault ? (1u << 12) : (1u << 22);
+    A.withhold = fault ? 1 : 0;
     return A;
 }
 
@@ -696,6 +724,9 @@ int run_loop(ot_plan *p, int parity0, int iters, bool check) {
     L.bar_count = p->bar;
     L.bar_gen = p->bar + 1;
     L.blk_resid = p->blk_resid;
+    const bool fault = g_wait_fault.load() == 1;
+    L.wait_ns = fault ? 2000000ull : 10000000000ull;  // 2 ms under the failure test, else 10 s
+    L.withhold_block = fault ? 0 : -1;
     int i = 0;
     while (i < iters) {
         const int len = std::min(kLoopChunk, iters - i);
@@ -810,9 +841,16 @@ void ot_options_default(ot_options *opt) {
     opt->sparse_verify = 1;
     opt->sparse_delta = 0.0;
     opt->sparse_dense_frac = 0.5;
+    opt->resid_history = nullptr;
+    opt->resid_history_len = 0;
 }
 
-void ot_plan_destroy(ot_plan *plan) { plan_free(plan); }
+void ot_plan_destroy(ot_plan *plan) {
+    NvtxRange nvtx_range("ot_plan_destroy");
+    plan_free(plan);
+}
+
+void ot_testing_wait_fault(int mode) { g_wait_fault.store(mode == 1 || mode == 2 ? mode : 0); }
 
 }  // extern "C"
 
@@ -840,7 +878,11 @@ int plan_setup(ot_plan *p, const ot_options &o) {
     p->sy.cnt = p->m;
     p->sx.pad = round_up(p->n, padq);
     p->sy.pad = round_up(p->m, padq);
-    if (p->kind == 0 && o.device_loop != 0 &&
+    p->sx.lo = p->shard ? p->range[0][0] : 0;
+    p->sx.rows = p->shard ? p->range[0][1] - p->range[0][0] : p->n;
+    p->sy.lo = p->shard ? p->range[1][0] : 0;
+    p->sy.rows = p->shard ? p->range[1][1] - p->range[1][0] : p->m;
+    if (!p->shard && p->kind == 0 && o.device_loop != 0 &&
         (o.device_loop == 1 || (double)p->n * (double)p->m <= (double)(1ll << 28))) {
         // rows per thread (1 or 2, both half-steps) with the smaller estimate;
         // measured: 1 row runs ~6 % slower per pair, but balances better on some sizes
@@ -875,11 +917,11 @@ int plan_setup(ot_plan *p, const ot_options &o) {
     }
     int rc = OT_OK;
     if (!p->use_loop)
-        rc = choose_shape(p->kind, p->dim, p->sm_count, p->n, p->sy.pad, p->sx, o.col_splits,
-                          o.rows_per_thread);
+        rc = choose_shape(p->kind, p->dim, p->sm_count, std::max<int64_t>(p->sx.rows, 1), p->sy.pad, p->sx,
+                          o.col_splits, o.rows_per_thread);
     if (rc != OT_OK) return rc;
-    if (!p->use_loop && (rc = choose_shape(p->kind, p->dim, p->sm_count, p->m, p->sx.pad, p->sy,
-                                           o.col_splits, o.rows_per_thread)) != OT_OK)
+    if (!p->use_loop && (rc = choose_shape(p->kind, p->dim, p->sm_count, std::max<int64_t>(p->sy.rows, 1),
+                                           p->sx.pad, p->sy, o.col_splits, o.rows_per_thread)) != OT_OK)
         return rc;
     const int64_t part_cnt = std::max((int64_t)p->sx.splits * p->sx.tiles * p->sx.tile,
                                       (int64_t)p->sy.splits * p->sy.tiles * p->sy.tile);
@@ -924,26 +966,32 @@ int plan_setup(ot_plan *p, const ot_options &o) {
     return OT_OK;
 }
 
-// Input statistics, validation and the captured scale.
-int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
+// Input statistics, validation and the coordinate shift o (the midpoint of the
+// clouds' means, used by every table); fills p->hs->s with the sums.
+int coord_shift(ot_plan *p) {
     DevScalars *ds = p->ds;
     OT_CU(launch_coord_stats(p->x, p->n, p->d, p->part1, p->part2, ds->sums[0], ds->sums[1],
                              &ds->flags[0], nullptr, p->s_int));
     OT_CU(launch_coord_stats(p->y, p->m, p->d, p->part1, p->part2, ds->sums[2], ds->sums[3],
                              &ds->flags[1], nullptr, p->s_int));
-    OT_CU(launch_coord_stats(p->a, p->n, 1, p->part1, p->part2, &ds->wsum[0], &ds->wsum[1],
-                             &ds->flags[2], &ds->zeros[0], p->s_int));
-    OT_CU(launch_coord_stats(p->b, p->m, 1, p->part1, p->part2, &ds->wsum[2], &ds->wsum[3],
-                             &ds->flags[3], &ds->zeros[1], p->s_int));
-    p->launches += 8;
+    const bool weights = p->a && p->b;  // ot_max_sqdist has none
+    if (weights) {
+        OT_CU(launch_coord_stats(p->a, p->n, 1, p->part1, p->part2, &ds->wsum[0], &ds->wsum[1],
+                                 &ds->flags[2], &ds->zeros[0], p->s_int));
+        OT_CU(launch_coord_stats(p->b, p->m, 1, p->part1, p->part2, &ds->wsum[2], &ds->wsum[3],
+                                 &ds->flags[3], &ds->zeros[1], p->s_int));
+    }
+    p->launches += weights ? 8 : 4;
     int rc = read_scalars(p);
     if (rc != OT_OK) return rc;
     const DevScalars &h = p->hs->s;
     if ((h.flags[0] | h.flags[1]) & 1) return fail(OT_ERR_NONFINITE, "x or y holds a NaN or inf");
-    if ((h.flags[2] | h.flags[3]) & 1) return fail(OT_ERR_NONFINITE, "a or b holds a NaN or inf");
-    if ((h.flags[2] | h.flags[3]) & 2) return fail(OT_ERR_INVALID_ARG, "negative weight in a or b");
-    if (!(h.wsum[0] > 0.0) || !(h.wsum[2] > 0.0))
-        return fail(OT_ERR_INVALID_ARG, "a and b must have positive sums");
+    if (weights) {
+        if ((h.flags[2] | h.flags[3]) & 1) return fail(OT_ERR_NONFINITE, "a or b holds a NaN or inf");
+        if ((h.flags[2] | h.flags[3]) & 2) return fail(OT_ERR_INVALID_ARG, "negative weight in a or b");
+        if (!(h.wsum[0] > 0.0) || !(h.wsum[2] > 0.0))
+            return fail(OT_ERR_INVALID_ARG, "a and b must have positive sums");
+    }
     p->n_massless_rows = (int64_t)h.zeros[0];
     p->n_massless_cols = (int64_t)h.zeros[1];
     double dot = 0.0, sxx = 0.0, syy = 0.0;
@@ -956,10 +1004,21 @@ int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
     }
     for (int k = p->d; k < kMaxD; ++k) p->hs->o[k] = 0.0;
     OT_CU(cudaMemcpyAsync(p->o, p->hs->o, sizeof(double) * kMaxD, cudaMemcpyHostToDevice, p->s_int));
+    p->mean_sq = sxx / (double)p->n + syy / (double)p->m - 2.0 * dot;
+    // the stream must not leave before the pinned o[] has been copied
+    OT_CU(cudaStreamSynchronize(p->s_int));
+    return OT_OK;
+}
+
+// The captured scale (after coord_shift): 1, the closed-form mean, the
+// all-pairs max_cost pass, or the caller's value.
+int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
+    int rc = coord_shift(p);
+    if (rc != OT_OK) return rc;
+    DevScalars *ds = p->ds;
     double c = 1.0;
     if (scale == OT_SCALE_MEAN) {
-        const double mean = sxx / (double)p->n + syy / (double)p->m - 2.0 * dot;
-        c = 1.0 / mean;
+        c = 1.0 / p->mean_sq;
     } else if (scale == OT_SCALE_MAX_COST) {
         OT_CU(launch_max_cost(p->x, p->y, p->n, p->m, p->d, p->o, &ds->max_bits, p->s_int));
         p->launches += 1;
@@ -974,8 +1033,6 @@ int resolve_scale(ot_plan *p, ot_scale scale, double scale_value) {
     if (!std::isfinite(c) || !(c > 0.0))
         return fail(OT_ERR_INVALID_ARG, "cost scale is zero or not finite (all points equal?)");
     p->c = c;
-    // the stream must not leave before the pinned o[] has been copied
-    OT_CU(cudaStreamSynchronize(p->s_int));
     return OT_OK;
 }
 
@@ -998,6 +1055,8 @@ int validate(const float *x, const float *y, const float *a, const float *b, int
     if (n_iters == 0 && !o.warm_start)
         return fail(OT_ERR_INVALID_ARG, "n_iters == 0 needs warm_start (a plan at given f, g)");
     if (o.check_every < 1) return fail(OT_ERR_INVALID_ARG, "check_every must be >= 1");
+    if (o.resid_history_len < 0 || (o.resid_history_len > 0 && !o.resid_history))
+        return fail(OT_ERR_INVALID_ARG, "resid_history_len must be >= 0, with a non-NULL resid_history");
     if (o.col_splits < 0) return fail(OT_ERR_INVALID_ARG, "col_splits must be >= 0");
     if (o.rows_per_thread != 0 && o.rows_per_thread != 1 && o.rows_per_thread != 2 &&
         o.rows_per_thread != 4 && o.rows_per_thread != 8)
@@ -1016,6 +1075,7 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
                                       ot_scale scale_cost, int32_t n_iters, double tol, float *f,
                                       float *g, void *stream, const ot_options *opt,
                                       ot_plan **plan_out, ot_info *info) {
+    NvtxRange nvtx_range("ot_sinkhorn_pointcloud");
     if (plan_out) *plan_out = nullptr;
     ot_options o;
     ot_options_default(&o);
@@ -1067,6 +1127,9 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         OT_CU(cudaMemsetAsync(f, 0, sizeof(float) * n, p->s_int));
         OT_CU(cudaMemsetAsync(g, 0, sizeof(float) * m, p->s_int));
     }
+    if (o.resid_history_len > 0)  // every entry no f-update measures stays NaN
+        OT_CU(cudaMemsetAsync(o.resid_history, 0xff, sizeof(double) * (size_t)o.resid_history_len,
+                              p->s_int));
     p->graph_len = std::max(2, (o.check_every + 1) / 2 * 2);
     p->timing = o.timing != 0;
 
@@ -1093,7 +1156,8 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
         // mass the mask omits (at most sp_bound), so the full residual is <= tol
         const double tol_s = (last && tol > 0.0) ? (sparse ? tol - p->sp_bound : tol) : 0.0;
         const int iters = last ? n_iters : o.iters_per_stage;
-        OT_CU(launch_set_params(p->prm, stage_eps[si], p->c, tol_s, p->s_int));
+        OT_CU(launch_set_params(p->prm, stage_eps[si], p->c, tol_s, o.resid_history, (int64_t)t,
+                                o.resid_history_len, p->s_int));
         OT_CU(launch_reset_state(p->st, p->s_int));
         if (p->kind == 2) {
             OT_CU(launch_tc_tables(x, fb[t & 1], n, p->sx.pad, d, p->dp, p->kp, p->o, p->prm,
@@ -1111,6 +1175,9 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
                     : run_iterations(p, t & 1, iters, tol_s > 0.0, o.use_graphs != 0);
         if (rc != OT_OK) return rc;
         if ((rc = read_state(p)) != OT_OK) return rc;
+        if (p->hs->st.wait_timeout)
+            return fail(OT_ERR_CUDA, "a bounded device wait (grid barrier or tensor-core pipeline) "
+                                     "timed out; results invalid");
         const int done = p->hs->st.stop ? p->hs->st.conv_iter : iters;
         t += done;
         half_steps += 2 * (int64_t)done + (p->hs->st.stop ? 1 : 0);
@@ -1161,7 +1228,8 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     }
     if ((rc = read_state(p)) != OT_OK) return rc;
     if (p->hs->st.wait_timeout)
-        return fail(OT_ERR_CUDA, "a tensor-core pipeline wait timed out (results invalid)");
+        return fail(OT_ERR_CUDA, "a bounded device wait (grid barrier or tensor-core pipeline) "
+                                 "timed out; results invalid");
     if (p->hs->st.nonfinite)
         return fail(OT_ERR_NONFINITE, "a potential left the finite range (eps too small for float32?)");
     p->eps = stage_eps.back();
@@ -1208,10 +1276,272 @@ extern "C" int ot_sinkhorn_pointcloud(const float *x, const float *y, const floa
     return OT_OK;
 }
 
+extern "C" int ot_sinkhorn_pointcloud_host(const float *x, const float *y, const float *a,
+                                           const float *b, int64_t n, int64_t m, int32_t d,
+                                           double eps, ot_scale scale_cost, int32_t n_iters,
+                                           double tol, float *f, float *g, void *stream,
+                                           const ot_options *opt, ot_plan **plan_out,
+                                           ot_info *info) {
+    NvtxRange nvtx_range("ot_sinkhorn_pointcloud_host");
+    if (plan_out) *plan_out = nullptr;
+    if (!x || !y || !a || !b || !f || !g) return fail(OT_ERR_INVALID_ARG, "null array pointer");
+    if (n < 1 || m < 1 || n > INT32_MAX || m > INT32_MAX || d < 1 || d > kMaxD)
+        return fail(n > INT32_MAX || m > INT32_MAX ? OT_ERR_OVERFLOW
+                    : d > kMaxD                    ? OT_ERR_UNSUPPORTED
+                                                   : OT_ERR_INVALID_ARG,
+                    "bad sizes (n=%lld m=%lld d=%d)", (long long)n, (long long)m, d);
+    int dev = 0, sms = 0;
+    int rc = check_device(&dev, &sms);
+    if (rc != OT_OK) return rc;
+    const bool warm = opt && opt->warm_start;
+    cudaStream_t s = (cudaStream_t)stream;
+    // device copies of x, y, a, b, f, g in one pooled buffer
+    float *dx = nullptr, *dy = nullptr, *da = nullptr, *db = nullptr, *df = nullptr, *dg = nullptr;
+    char *buf = nullptr;
+    size_t got = 0;
+    for (int pass = 0; pass < 2; ++pass) {
+        Carver cv{pass ? buf : nullptr};
+        dx = cv.take<float>(n * d);
+        dy = cv.take<float>(m * d);
+        da = cv.take<float>(n);
+        db = cv.take<float>(m);
+        df = cv.take<float>(n);
+        dg = cv.take<float>(m);
+        if (pass == 0) OT_CU(pool_device_alloc(reinterpret_cast<void **>(&buf), cv.off, &got));
+    }
+    struct Release {
+        char *buf;
+        size_t got;
+        int dev;
+        cudaStream_t s;
+        ~Release() {
+            if (buf) {
+                cudaStreamSynchronize(s);  // no copy may still use it
+                pool_device_free(buf, got, dev);
+            }
+        }
+    } rel{buf, got, dev, s};
+    cudaError_t e = cudaSuccess;
+    const struct { void *dst; const void *src; size_t bytes; } in[] = {
+        {dx, x, sizeof(float) * (size_t)(n * d)}, {dy, y, sizeof(float) * (size_t)(m * d)},
+        {da, a, sizeof(float) * (size_t)n},       {db, b, sizeof(float) * (size_t)m},
+        {df, f, warm ? sizeof(float) * (size_t)n : 0}, {dg, g, warm ? sizeof(float) * (size_t)m : 0}};
+    for (const auto &c : in)
+        if (e == cudaSuccess && c.bytes) e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return fail(OT_ERR_CUDA, "host-to-device copy failed: %s", cudaGetErrorString(e));
+    ot_plan *plan = nullptr;
+    rc = ot_sinkhorn_pointcloud(dx, dy, da, db, n, m, d, eps, scale_cost, n_iters, tol, df, dg, stream,
+                                opt, &plan, info);
+    if (rc < 0) return rc;
+    e = cudaMemcpyAsync(f, df, sizeof(float) * (size_t)n, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(g, dg, sizeof(float) * (size_t)m, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        plan_free(plan);
+        return fail(OT_ERR_CUDA, "device-to-host copy failed: %s", cudaGetErrorString(e));
+    }
+    if (plan_out) {  // the plan keeps the device copies it reads
+        plan->ws_in = buf;
+        plan->ws_in_bytes = got;
+        rel.buf = nullptr;
+        *plan_out = plan;
+    } else {
+        plan_free(plan);
+    }
+    if (rc == OT_WARN_MASSLESS_ROWS) fail(OT_WARN_MASSLESS_ROWS, "some rows carry no mass");
+    return rc;
+}
+
+// ------------------------------------------------------------ sharded solve
+// The solve split by rows across ranks (FlashSinkhorn 2, section 5: problems
+// beyond one GPU's memory run on several): every rank holds both clouds in
+// full and updates a contiguous range of x's rows in the f-update and of y's in
+// the g-update; the caller exchanges the updated potential ranges between the
+// half-steps (an all-gather) and sums the residual partials (an all-reduce).
+
+extern "C" int ot_max_sqdist(const float *x, const float *y, int64_t n, int64_t m, int32_t d,
+                             int64_t x_lo, int64_t x_hi, float *out, void *stream) {
+    NvtxRange nvtx_range("ot_max_sqdist");
+    if (!x || !y || !out) return fail(OT_ERR_INVALID_ARG, "null pointer");
+    if (n < 1 || m < 1 || d < 1 || d > kMaxD)
+        return fail(d > kMaxD ? OT_ERR_UNSUPPORTED : OT_ERR_INVALID_ARG, "bad sizes");
+    if (n > INT32_MAX || m > INT32_MAX) return fail(OT_ERR_OVERFLOW, "n and m must be < 2^31");
+    if (x_lo < 0 || x_hi > n || x_lo > x_hi) return fail(OT_ERR_INVALID_ARG, "bad row range");
+    // a plan without iterations supplies the shift o (the same as every solve's)
+    // and the pass's scratch; its own scale resolution is skipped
+    ot_options o;
+    ot_options_default(&o);
+    o.device_loop = 0;
+    ot_plan *p = new (std::nothrow) ot_plan();
+    if (!p) return fail(OT_ERR_OOM, "host allocation failed");
+    struct Guard {
+        ot_plan *p;
+        ~Guard() { plan_free(p); }
+    } guard{p};
+    int rc = check_device(&p->device, &p->sm_count);
+    if (rc != OT_OK) return rc;
+    p->x = x; p->y = y; p->n = n; p->m = m; p->d = d;
+    p->shard = true;  // no half-step shapes are needed: an empty range
+    cudaStream_t us = (cudaStream_t)stream;
+    OT_CU(pool_stream(&p->s_int));
+    OT_CU(cudaEventCreateWithFlags(&p->ev_in, cudaEventDisableTiming));
+    OT_CU(cudaEventCreateWithFlags(&p->ev_out, cudaEventDisableTiming));
+    OT_CU(pool_host_alloc(reinterpret_cast<void **>(&p->hs), sizeof(HostScalars)));
+    OT_CU(cudaEventRecord(p->ev_in, us));
+    OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
+    if ((rc = plan_setup(p, o)) != OT_OK) return rc;
+    if ((rc = coord_shift(p)) != OT_OK) return rc;
+    unsigned bits = 0;
+    if (x_hi > x_lo) {
+        OT_CU(cudaMemsetAsync(&p->ds->max_bits, 0, sizeof(unsigned), p->s_int));
+        OT_CU(launch_max_cost(x + x_lo * d, y, x_hi - x_lo, m, d, p->o, &p->ds->max_bits, p->s_int));
+        if ((rc = read_scalars(p)) != OT_OK) return rc;
+        bits = p->hs->s.max_bits;
+    }
+    std::memcpy(out, &bits, sizeof bits);
+    OT_CU(cudaEventRecord(p->ev_out, p->s_int));
+    OT_CU(cudaStreamWaitEvent(us, p->ev_out, 0));
+    return OT_OK;
+}
+
+extern "C" int ot_shard_plan_create(const float *x, const float *y, const float *a, const float *b,
+                                    int64_t n, int64_t m, int32_t d, double eps, ot_scale scale_cost,
+                                    int64_t x_lo, int64_t x_hi, int64_t y_lo, int64_t y_hi,
+                                    void *stream, const ot_options *opt, ot_plan **plan_out,
+                                    ot_info *info) {
+    NvtxRange nvtx_range("ot_shard_plan_create");
+    if (!plan_out) return fail(OT_ERR_INVALID_ARG, "plan_out must not be NULL");
+    *plan_out = nullptr;
+    ot_options o;
+    ot_options_default(&o);
+    if (opt) o = *opt;
+    o.device_loop = 0;
+    o.warm_start = 1;
+    float dummy = 0.0f;
+    int rc = validate(x, y, a, b, n, m, d, eps, scale_cost, 1, &dummy, &dummy, o);
+    if (rc != OT_OK) return rc;
+    if (o.block_sparse) return fail(OT_ERR_UNSUPPORTED, "a sharded plan runs dense half-steps");
+    if (x_lo < 0 || x_hi > n || x_lo > x_hi || y_lo < 0 || y_hi > m || y_lo > y_hi)
+        return fail(OT_ERR_INVALID_ARG, "row ranges must satisfy 0 <= lo <= hi <= n (m)");
+    if ((x_lo | y_lo) & (kColPad - 1))
+        return fail(OT_ERR_INVALID_ARG, "x_lo and y_lo must be multiples of %d", kColPad);
+    ot_plan *p = new (std::nothrow) ot_plan();
+    if (!p) return fail(OT_ERR_OOM, "host allocation failed");
+    struct Guard {
+        ot_plan *p;
+        bool keep = false;
+        ~Guard() {
+            if (!keep) plan_free(p);
+        }
+    } guard{p};
+    rc = check_device(&p->device, &p->sm_count);
+    if (rc != OT_OK) return rc;
+    p->x = x; p->y = y; p->a = a; p->b = b;
+    p->n = n; p->m = m; p->d = d;
+    p->shard = true;
+    p->range[0][0] = x_lo; p->range[0][1] = x_hi;
+    p->range[1][0] = y_lo; p->range[1][1] = y_hi;
+    cudaStream_t us = (cudaStream_t)stream;
+    OT_CU(pool_stream(&p->s_int));
+    OT_CU(cudaEventCreateWithFlags(&p->ev_in, cudaEventDisableTiming));
+    OT_CU(cudaEventCreateWithFlags(&p->ev_out, cudaEventDisableTiming));
+    OT_CU(pool_host_alloc(reinterpret_cast<void **>(&p->hs), sizeof(HostScalars)));
+    OT_CU(cudaEventRecord(p->ev_in, us));
+    OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
+    if ((rc = plan_setup(p, o)) != OT_OK) return rc;
+    if ((rc = resolve_scale(p, scale_cost, o.scale_value)) != OT_OK) return rc;
+    p->sx_pts = x; p->sy_pts = y; p->sa = a; p->sb = b;
+    p->eps = eps;
+    // no tol: the caller decides when to stop from the summed residual
+    OT_CU(launch_set_params(p->prm, eps, p->c, 0.0, nullptr, 0, 0, p->s_int));
+    OT_CU(launch_reset_state(p->st, p->s_int));
+    // both clouds' row tables (the coordinates); each half-step rebuilds the other
+    // cloud's column terms from its potential (the weights stand in until then)
+    if (p->kind == 2) {
+        OT_CU(launch_tc_tables(x, a, n, p->sx.pad, d, p->dp, p->kp, p->o, p->prm, p->sx.rowtab, p->sx.arow,
+                               p->sx.bcol, p->s_int));
+        OT_CU(launch_tc_tables(y, b, m, p->sy.pad, d, p->dp, p->kp, p->o, p->prm, p->sy.rowtab, p->sy.arow,
+                               p->sy.bcol, p->s_int));
+    } else {
+        const int layout = p->kind == 0 ? 0 : 1;
+        OT_CU(launch_tables(x, a, n, p->sx.pad, d, p->dp, p->o, p->prm, p->sx.rowtab, p->sx.coltab, layout,
+                            p->s_int));
+        OT_CU(launch_tables(y, b, m, p->sy.pad, d, p->dp, p->o, p->prm, p->sy.rowtab, p->sy.coltab, layout,
+                            p->s_int));
+    }
+    OT_CU(cudaEventRecord(p->ev_out, p->s_int));
+    OT_CU(cudaStreamWaitEvent(us, p->ev_out, 0));
+    OT_CU(cudaStreamSynchronize(p->s_int));
+    if (info) {
+        std::memset(info, 0, sizeof *info);
+        info->col_splits = p->sx.splits;
+        info->inv_scale_cost = p->c;
+        info->eps = eps;
+        info->n_massless_rows = p->n_massless_rows;
+        info->n_massless_cols = p->n_massless_cols;
+    }
+    guard.keep = true;
+    *plan_out = p;
+    return OT_OK;
+}
+
+extern "C" int ot_shard_half_step(ot_plan *p, int32_t side, const float *other, const float *cur,
+                                  float *out, double *resid, void *stream) {
+    NvtxRange nvtx_range("ot_shard_half_step");
+    if (!p || !p->shard || !p->prm) return fail(OT_ERR_INVALID_ARG, "not a sharded plan");
+    if (side != 0 && side != 1) return fail(OT_ERR_INVALID_ARG, "side must be 0 (f) or 1 (g)");
+    if (!other || !cur || !out) return fail(OT_ERR_INVALID_ARG, "null potential pointer");
+    int dev = -1;
+    OT_CU(cudaGetDevice(&dev));
+    if (dev != p->device) return fail(OT_ERR_INVALID_ARG, "plan belongs to device %d, current is %d", p->device, dev);
+    cudaStream_t us = (cudaStream_t)stream;
+    OT_CU(cudaEventRecord(p->ev_in, us));
+    OT_CU(cudaStreamWaitEvent(p->s_int, p->ev_in, 0));
+    // the other cloud's column table from its whole potential (all ranks' rows)
+    const bool f = side == 0;
+    Side &cols = f ? p->sy : p->sx;
+    const float *cpts = f ? p->y : p->x;
+    if (p->kind == 2) {
+        OT_CU(launch_tc_tables(cpts, other, cols.cnt, cols.pad, p->d, p->dp, p->kp, p->o, p->prm,
+                               cols.rowtab, cols.arow, cols.bcol, p->s_int));
+    } else {
+        OT_CU(launch_tables(cpts, other, cols.cnt, cols.pad, p->d, p->dp, p->o, p->prm, cols.rowtab,
+                            cols.coltab, p->kind == 0 ? 0 : 1, p->s_int));
+    }
+    const Side &rows = f ? p->sx : p->sy;
+    if (rows.rows > 0) {
+        // the half-step over this plan's rows: old potential `cur`, new one into `out`
+        float *save[3] = {p->sf[0], p->sf[1], p->sg};
+        p->sf[0] = const_cast<float *>(cur);
+        p->sf[1] = out;
+        p->sg = out;  // g-update: pot_old and pot_new both come from sg
+        HalfStep A = make_step(p, side, 0);
+        if (!f) A.pot_old = cur + rows.lo;
+        p->sf[0] = save[0]; p->sf[1] = save[1]; p->sg = save[2];
+        cudaError_t e = p->kind == 2
+            ? launch_halfstep_tc(p->d, A, f ? &p->tm_arow_x : &p->tm_arow_y, f ? &p->tm_bcol_y : &p->tm_bcol_x,
+                                 rows.grid, p->s_int)
+            : launch_halfstep(p->kind, p->dim, rows.rpt, A, rows.grid, p->s_int);
+        if (e != cudaSuccess) return fail(OT_ERR_CUDA, "half-step launch failed: %s", cudaGetErrorString(e));
+    }
+    OT_CU(cudaEventRecord(p->ev_out, p->s_int));
+    OT_CU(cudaStreamWaitEvent(us, p->ev_out, 0));
+    if (resid || rows.rows > 0) {
+        int rc = read_state(p);
+        if (rc != OT_OK) return rc;
+        if (p->hs->st.wait_timeout)
+            return fail(OT_ERR_CUDA, "a bounded device wait timed out; results invalid");
+        if (p->hs->st.nonfinite) return fail(OT_ERR_NONFINITE, "a potential left the finite range");
+        if (resid) *resid = rows.rows > 0 ? p->hs->st.resid[side] : 0.0;
+    }
+    return OT_OK;
+}
+
 namespace {
 
 int plan_check(const ot_plan *p) {
     if (!p) return fail(OT_ERR_INVALID_ARG, "null plan");
+    if (p->shard) return fail(OT_ERR_INVALID_ARG, "a sharded plan serves ot_shard_half_step only");
     int dev = -1;
     OT_CU(cudaGetDevice(&dev));
     if (dev != p->device) return fail(OT_ERR_INVALID_ARG, "plan belongs to device %d, current is %d", p->device, dev);
@@ -1225,7 +1555,7 @@ int ensure_rows_ws(ot_plan *p) {
     for (int pass = 0; pass < 2; ++pass) {
         Carver cv{pass ? p->ws_rows : nullptr};
         p->dcol = cv.take<double>(big * (p->d + 1));
-        p->rpart = cv.take<double>(rowpass_blocks(big));
+        p->rpart = cv.take<double>(rowpass_blocks(big, p->d));
         p->rowmax = cv.take<float>(p->n);
         p->counts = cv.take<int64_t>(p->n);
         p->scan = cv.take<int64_t>(scan_tmp_count(p->n));
@@ -1245,6 +1575,7 @@ int sync_read(ot_plan *p, cudaStream_t s) {
 
 extern "C" int ot_materialize_rows(const ot_plan *cplan, const int64_t *row_idx, int64_t k,
                                    float *out, void *stream) {
+    NvtxRange nvtx_range("ot_materialize_rows");
     ot_plan *p = const_cast<ot_plan *>(cplan);
     int rc = plan_check(p);
     if (rc != OT_OK) return rc;
@@ -1292,7 +1623,7 @@ int lowrank_rows(int mode, const float *fa, const float *fb, const float *g, con
     size_t got = 0;
     OT_CU(pool_device_alloc(reinterpret_cast<void **>(&flag), 256, &got));
     if (pool_host_alloc(reinterpret_cast<void **>(&hflag), sizeof(int)) != cudaSuccess) {
-        pool_device_free(flag, got);
+        pool_device_free(flag, got, dev);
         return fail(OT_ERR_OOM, "pinned host allocation failed");
     }
     LrArgs L{};
@@ -1309,7 +1640,7 @@ int lowrank_rows(int mode, const float *fa, const float *fb, const float *g, con
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     const int bad = e == cudaSuccess ? *hflag : 0;
     pool_host_free(hflag, sizeof(int));
-    pool_device_free(flag, got);
+    pool_device_free(flag, got, dev);
     if (e != cudaSuccess) return fail(OT_ERR_CUDA, "low-rank rows: %s", cudaGetErrorString(e));
     if (bad) return fail(OT_ERR_INVALID_ARG, "a row index is outside [0, n)");
     return OT_OK;
@@ -1320,6 +1651,7 @@ int lowrank_rows(int mode, const float *fa, const float *fb, const float *g, con
 extern "C" int ot_materialize_rows_lowrank(const float *Q, const float *R, const float *g, int64_t n,
                                            int64_t m, int32_t r, const int64_t *row_idx, int64_t k,
                                            float *out, void *stream) {
+    NvtxRange nvtx_range("ot_materialize_rows_lowrank");
     return lowrank_rows(0, Q, R, g, nullptr, nullptr, n, m, r, 0.0, 1.0, 1.0, row_idx, k, out, stream);
 }
 
@@ -1328,6 +1660,7 @@ extern "C" int ot_materialize_rows_lrcost(const float *cost1, const float *cost2
                                           double bias, double inv_scale_cost, double eps,
                                           const int64_t *row_idx, int64_t k, float *out,
                                           void *stream) {
+    NvtxRange nvtx_range("ot_materialize_rows_lrcost");
     return lowrank_rows(1, cost1, cost2, nullptr, f, g, n, m, r, bias, inv_scale_cost, eps, row_idx, k,
                         out, stream);
 }
@@ -1335,6 +1668,7 @@ extern "C" int ot_materialize_rows_lrcost(const float *cost1, const float *cost2
 extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, float *thr_out,
                                    int64_t *row_counts, int64_t *nnz_out,
                                    int64_t *n_massless_out, int64_t *argmin_out, void *stream) {
+    NvtxRange nvtx_range("ot_sparsify_min_row");
     ot_plan *p = const_cast<ot_plan *>(cplan);
     int rc = plan_check(p);
     if (rc != OT_OK) return rc;
@@ -1381,6 +1715,7 @@ extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, flo
 extern "C" int ot_sparsify_csr(const ot_plan *cplan, int64_t block_rows, float thr, int64_t *row_ptr,
                                int64_t *col_idx, float *vals, int64_t capacity, int64_t *nnz_out,
                                void *stream) {
+    NvtxRange nvtx_range("ot_sparsify_csr");
     ot_plan *p = const_cast<ot_plan *>(cplan);
     int rc = plan_check(p);
     if (rc != OT_OK) return rc;
@@ -1430,6 +1765,7 @@ extern "C" int ot_sparsify_csr(const ot_plan *cplan, int64_t block_rows, float t
 
 extern "C" int ot_marginal_residual(const ot_plan *cplan, double *row_l1, double *col_l1,
                                     void *stream) {
+    NvtxRange nvtx_range("ot_marginal_residual");
     ot_plan *p = const_cast<ot_plan *>(cplan);
     int rc = plan_check(p);
     if (rc != OT_OK) return rc;
@@ -1441,12 +1777,12 @@ extern "C" int ot_marginal_residual(const ot_plan *cplan, double *row_l1, double
     OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
     R.pts = p->x; R.pot = p->f; R.w = p->a; R.cols = p->m; R.row_begin = 0; R.row_end = p->n;
     OT_CU(launch_rowpass(2, R, s));
-    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->n), &p->ds->r_sum[0], s));
+    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->n, p->d), &p->ds->r_sum[0], s));
     // columns: the same pass with the clouds' roles swapped
     OT_CU(launch_dcol(p->x, p->f, p->n, p->d, p->o, p->prm, p->dcol, s));
     R.pts = p->y; R.pot = p->g; R.w = p->b; R.cols = p->n; R.row_begin = 0; R.row_end = p->m;
     OT_CU(launch_rowpass(2, R, s));
-    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->m), &p->ds->r_sum[1], s));
+    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->m, p->d), &p->ds->r_sum[1], s));
     if ((rc = sync_read(p, s)) != OT_OK) return rc;
     if (row_l1) *row_l1 = p->hs->s.r_sum[0];
     if (col_l1) *col_l1 = p->hs->s.r_sum[1];

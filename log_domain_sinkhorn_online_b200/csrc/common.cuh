@@ -44,7 +44,21 @@ struct Params {
     double kappa;     // log2(e) / eps
     double c;         // inv_scale_cost
     double tol;       // stopping tolerance on ||T1 - a||_1 (<= 0: none)
+    double *hist;     // optional residual history: hist[hist_off + k - 1] = ||T1 - a||_1
+                      // after iteration k of this stage (k < hist_len - hist_off)
+    int64_t hist_off; // iterations of the earlier stages
+    int64_t hist_len;
 };
+
+// Records the in-loop row residual `v` of the state after iteration `k` of the
+// current stage in the optional history (one thread calls it).
+__device__ __forceinline__ void record_residual(const Params *prm, int k, double v) {
+    double *h = prm->hist;
+    if (h && k >= 1) {
+        const int64_t idx = prm->hist_off + (int64_t)k - 1;
+        if (idx < prm->hist_len) h[idx] = v;
+    }
+}
 
 // Solver state written by the kernels' last-finishing blocks.
 struct State {
@@ -53,7 +67,7 @@ struct State {
     int bad_index;      // a row index outside [0, n) was given to a row kernel
     int iter_done;      // completed iterations in the current stage
     int conv_iter;      // iteration count at which tol was met (-1: not yet)
-    int wait_timeout;   // a bounded wait in a tensor-core kernel gave up (error)
+    int wait_timeout;   // a bounded device wait (grid barrier, mbarrier) gave up (error)
     double resid[2];    // last in-loop marginal residual of each side (0: rows, 1: cols)
     unsigned tiles_done[2];
     unsigned work[2];   // work-item counters of the per-launch CUDA-core half-steps (f, g side)
@@ -64,7 +78,8 @@ struct State {
 struct HalfStep {
     const float4 *coltab;      // column table (layout depends on the kernel)
     const float *rowtab;       // row coordinates minus the shift, [rows_pad][dp]
-    int64_t rows;              // rows updated (n for the f side, m for g)
+    int64_t rows;              // rows updated (n for the f side, m for g; a shard's count)
+    int64_t row_off;           // index of the first updated row in its cloud (shards; 0 otherwise)
     int64_t cols_pad;          // padded column count (multiple of kColPad)
     int64_t cols_per_split;    // multiple of kColPad (the last chunk of a split may be partial)
     int splits;                // column splits S
@@ -93,6 +108,10 @@ struct HalfStep {
     const int64_t *sp_fallback;  // non-null: only blocks t with sp_fallback[t] == 0 are updated
     const int *gate;             // non-null: the launch does nothing unless *gate == gate_val
     int gate_val;                //   (block-sparse iterations choose dense or sparse on the device)
+    // tensor-core half-step only: polls of one mbarrier wait before it gives up,
+    // and (failure tests only) block 0's producer skipping its first column-chunk load
+    unsigned wait_polls;
+    int withhold;
 };
 
 // ------------------------------------------------------ device helpers --

@@ -162,6 +162,7 @@ __device__ void finish_tile(const HalfStep &A, int tile, int tid, double *s_red,
             st->resid[A.side] = v;
             st->tiles_done[A.side] = 0;
             if (A.side == 0) {
+                record_residual(A.prm, st->iter_done, v);
                 if (tol > 0.0 && st->iter_done >= 1 && v <= tol) {
                     st->stop = 1;
                     st->conv_iter = st->iter_done;

@@ -50,7 +50,6 @@ constexpr int EPI_THREADS = EPI_WARPS * 32;
 constexpr int THREADS = (EPI_WARPS + 2) * 32;  // + TMA warp + MMA warp
 constexpr int SLAB = 64;             // bf16 per 128-byte swizzle row
 constexpr int SLAB_BYTES = M * 128;  // one slab of a 128-row operand tile (16 KB)
-constexpr uint32_t WAIT_LIMIT = 1u << 22;  // polls of one mbarrier before giving up
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,10 +70,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 }
 
 // Bounded wait for the phase with parity `parity` to complete. Returns false
-// (and raises *abort) after WAIT_LIMIT polls or when another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// (and raises *abort) after `limit` polls (2^22 in production) or when another
+// role aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint32_t limit) {
     const uint32_t a = smem_u32(bar);
-    for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -148,17 +149,18 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 
 // Warp-wide wait: lane 0 polls, the other lanes wait converged in the shuffle
 // (512 threads polling would compete with TMA and MMA for shared memory).
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                               uint32_t limit) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // Bounded wait that ignores the abort flag: used only to drain work this block
 // already issued before it frees its resources.
-__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, uint32_t limit) {
     const uint32_t a = smem_u32(bar);
-    for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -271,6 +273,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const int64_t n_items = (int64_t)A.tiles * A.splits;
+    const uint32_t lim = A.wait_polls;
 
     if (warp == TMA_WARP) {
         // -------------------------------------------------- TMA producer
@@ -281,7 +284,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             for (uint32_t iq = 0; ok; ++iq, ++item_no) {
                 // publish the item (or the end) to the MMA warp and the epilogue
                 const int slot = (int)(iq % RING);
-                if (iq >= (uint32_t)RING && !(ok = mbar_wait(&iempty[slot], ((iq / RING) - 1) & 1, s_abort)))
+                if (iq >= (uint32_t)RING && !(ok = mbar_wait(&iempty[slot], ((iq / RING) - 1) & 1, s_abort, lim)))
                     break;
                 s_items[slot] = item < n_items ? item : -1;
                 mbar_arrive(&ifull[slot]);
@@ -292,14 +295,18 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                 const int64_t c0 = (int64_t)split * A.cols_per_split;
                 const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
                 // the row tile is overwritten only after every MMA of the previous item
-                if (item_no > 0 && !(ok = mbar_wait(aempty, (item_no - 1) & 1, s_abort))) break;
+                if (item_no > 0 && !(ok = mbar_wait(aempty, (item_no - 1) & 1, s_abort, lim))) break;
                 mbar_expect_tx(afull, KS * SLAB_BYTES);
-                for (int s = 0; s < KS; ++s) tma_load_2d(sA + s * SLAB_BYTES, &tmA, afull, s * SLAB, tile * M);
+                for (int s = 0; s < KS; ++s)
+                    tma_load_2d(sA + s * SLAB_BYTES, &tmA, afull, s * SLAB, (int)(tile * M + A.row_off));
                 a_out = true;
                 for (int ch = 0; ch < nch && ok; ++ch, ++g) {
                     const int st = g % STAGES;
-                    if (g >= (uint32_t)STAGES && !(ok = mbar_wait(&empty[st], ((g / STAGES) - 1) & 1, s_abort)))
+                    if (g >= (uint32_t)STAGES && !(ok = mbar_wait(&empty[st], ((g / STAGES) - 1) & 1, s_abort, lim)))
                         break;
+                    // failure tests only: block 0 leaves its first chunk unloaded, so the
+                    // MMA warp's wait on it gives up
+                    if (g == 0 && A.withhold && blockIdx.x == 0) continue;
                     mbar_expect_tx(&full[st], KS * SLAB_BYTES);
                     uint8_t *dst = sB + st * KS * SLAB_BYTES;
                     for (int s = 0; s < KS; ++s)
@@ -309,9 +316,9 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
                 item = next;
             }
             if (!ok) {  // wait (bounded) for the loads this block put in flight
-                if (a_out) mbar_drain(afull, (item_no & 1) ^ 0);
+                if (a_out) mbar_drain(afull, (item_no & 1) ^ 0, lim);
                 for (int st = 0; st < STAGES; ++st)
-                    if (issued[st]) mbar_drain(&full[st], (issued[st] - 1) & 1);
+                    if (issued[st]) mbar_drain(&full[st], (issued[st] - 1) & 1, lim);
                 atomicExch(&A.st->wait_timeout, 1);
             }
         }
@@ -322,20 +329,20 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             bool ok = true, issued_any = false;
             for (uint32_t iq = 0; ok; ++iq, ++item_no) {
                 const int slot = (int)(iq % RING);
-                if (!(ok = mbar_wait(&ifull[slot], (iq / RING) & 1, s_abort))) break;
+                if (!(ok = mbar_wait(&ifull[slot], (iq / RING) & 1, s_abort, lim))) break;
                 const int64_t item = s_items[slot];
                 mbar_arrive(&iempty[slot]);
                 if (item < 0) break;
                 const int split = (int)(item % A.splits);
                 const int64_t c0 = (int64_t)split * A.cols_per_split;
                 const int nch = (int)((min(c0 + A.cols_per_split, A.cols_pad) - c0) / N);
-                if (!(ok = mbar_wait(afull, item_no & 1, s_abort))) break;
+                if (!(ok = mbar_wait(afull, item_no & 1, s_abort, lim))) break;
                 for (int ch = 0; ch < nch; ++ch, ++g) {
                     // accumulator by the chunk's index in its item, so that which epilogue
                     // warps sum which columns does not depend on the schedule
                     const int st = g % STAGES, b = ch % NBUF;
-                    if (!(ok = mbar_wait(&full[st], (g / STAGES) & 1, s_abort))) break;
-                    if (ub[b] > 0 && !(ok = mbar_wait(&tempty[b], (ub[b] - 1) & 1, s_abort))) break;
+                    if (!(ok = mbar_wait(&full[st], (g / STAGES) & 1, s_abort, lim))) break;
+                    if (ub[b] > 0 && !(ok = mbar_wait(&tempty[b], (ub[b] - 1) & 1, s_abort, lim))) break;
                     ++ub[b];
                     tc_fence_after();
                     const uint8_t *bst = sB + st * KS * SLAB_BYTES;
@@ -359,7 +366,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             if (!ok) {
                 if (issued_any) {  // wait (bounded) until the issued MMAs are done
                     mma_commit(drain);
-                    mbar_drain(drain, 0);
+                    mbar_drain(drain, 0, lim);
                 }
                 atomicExch(&A.st->wait_timeout, 1);
             }
@@ -382,7 +389,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             if (etid == 0) {
                 const int slot = (int)(iq % RING);
                 long long it = -1;
-                if (mbar_wait(&ifull[slot], (iq / RING) & 1, s_abort)) {
+                if (mbar_wait(&ifull[slot], (iq / RING) & 1, s_abort, lim)) {
                     it = s_items[slot];
                     mbar_arrive(&iempty[slot]);
                 }
@@ -402,7 +409,7 @@ hs_tc_kernel(HalfStep A, const __grid_constant__ CUtensorMap tmA,
             float va[32], vb[32];
             bool ok = true;
             for (int ch = h; ch < nch && ok; ch += NBUF) {
-                ok = mbar_wait_warp(&tfull[h], uses & 1, s_abort);
+                ok = mbar_wait_warp(&tfull[h], uses & 1, s_abort, lim);
                 if (!ok) break;
                 tc_fence_after();
                 tmem_ld32(tlane, va);

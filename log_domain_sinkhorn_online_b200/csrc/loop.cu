@@ -17,8 +17,9 @@
 // state before the update) without another barrier.
 //
 // All co-resident by construction (cooperative launch). The grid barrier waits
-// on an arrival counter with a time limit (globaltimer): past it the kernel
-// records State::wait_timeout and every block leaves the loop. Data rewritten
+// on an arrival counter with a time limit (globaltimer; 10 s, set by the
+// host): past it the kernel records State::wait_timeout and every block leaves
+// the loop. Data rewritten
 // inside the kernel (column tables, potentials, partials) is read with L1
 // bypassed.
 #include "finish.cuh"
@@ -28,8 +29,6 @@
 namespace ot {
 
 namespace {
-
-constexpr uint64_t kBarrierLimitNs = 10ull * 1000 * 1000 * 1000;  // 10 s
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -48,7 +47,8 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
 // the counter reaches (k + 1) * gridDim.x; one release-add per block, acquire
 // polling by thread 0. Returns false (uniformly per block) if the wait gave up,
 // after setting *err.
-__device__ bool grid_barrier(unsigned *count, unsigned &k, int *err, volatile int *s_ok) {
+__device__ bool grid_barrier(unsigned *count, unsigned &k, int *err, volatile int *s_ok,
+                             uint64_t limit_ns) {
     __syncthreads();
     const unsigned target = (++k) * gridDim.x;
     if (threadIdx.x == 0) {
@@ -58,7 +58,7 @@ __device__ bool grid_barrier(unsigned *count, unsigned &k, int *err, volatile in
             const uint64_t t0 = globaltimer();
             while (ld_acquire_u32(count) < target) {
                 __nanosleep(20);
-                if (globaltimer() - t0 > kBarrierLimitNs) {
+                if (globaltimer() - t0 > limit_ns) {
                     ok = 0;
                     atomicExch(err, 1);
                     break;
@@ -154,12 +154,16 @@ __global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
             __syncthreads();
             lowd_item<D, R, true, true>(F, (int)(item / F.splits), (int)(item % F.splits), sm);
         }
-        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
+        if (nbar == 0 && (int)blockIdx.x == L.withhold_block) return;  // failure tests only
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok, L.wait_ns)) break;
         const double br = merge_phase<kHsThreads>(F, s_red, &bad);
         if (threadIdx.x == 0) L.blk_resid[blockIdx.x] = br;
-        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok, L.wait_ns)) break;
         const double resid = grid_residual<kHsThreads>(L.blk_resid, s_red);
-        if (blockIdx.x == 0 && threadIdx.x == 0) st->resid[0] = resid;
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            st->resid[0] = resid;
+            record_residual(F.prm, iter_done, resid);
+        }
         if (tol > 0.0 && iter_done >= 1 && resid <= tol) {  // the same decision in every block
             if (blockIdx.x == 0 && threadIdx.x == 0) {
                 st->stop = 1;
@@ -174,9 +178,9 @@ __global__ void __launch_bounds__(kHsThreads, 4) hs_loop_kernel(LoopArgs L) {
             __syncthreads();
             lowd_item<D, R, true, true>(G, (int)(item / G.splits), (int)(item % G.splits), sm);
         }
-        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok, L.wait_ns)) break;
         merge_phase<kHsThreads>(G, s_red, &bad);
-        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok)) break;
+        if (!grid_barrier(L.bar_count, nbar, &st->wait_timeout, &s_ok, L.wait_ns)) break;
         ++iter_done;
         par ^= 1;
         if (blockIdx.x == 0 && threadIdx.x == 0) st->iter_done = iter_done;

@@ -146,6 +146,7 @@ extern "C" int ot_marginal_residual_noalloc(const float *x, const float *y, cons
                                             double inv_scale_cost, double *row_l1,
                                             double *col_l1, void *stream) {
     using namespace ot;
+    NvtxRange nvtx_range("ot_marginal_residual_noalloc");
     if (!x || !y || !a || !b || !f || !g) return set_error(OT_ERR_INVALID_ARG, "null array pointer");
     if (n < 1 || m < 1) return set_error(OT_ERR_INVALID_ARG, "n and m must be >= 1");
     if (n > OT_NOALLOC_MAX_POINTS || m > OT_NOALLOC_MAX_POINTS)

@@ -7,12 +7,16 @@
 // synchronises the device), page pinning and stream creation every time. Freed
 // resources go back to this cache (up to kKeepBytes of device memory per
 // device) and a later plan of the same or a slightly smaller size reuses them.
-// ot_trim_cache() releases everything the cache holds.
+// ot_trim_cache() releases everything the cache holds. A resource goes back
+// under the device it was made on (the caller names it), whichever device is
+// current when it is returned.
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <vector>
 
 #include "ot_sinkhorn.h"
+#include "ot_sinkhorn_testing.h"
 #include "runtime.h"
 
 namespace ot {
@@ -52,7 +56,18 @@ void *take(std::multimap<size_t, void *> &m, size_t bytes, size_t *got) {
 
 }  // namespace
 
+// Allocation-failure injection for the host-side failure tests (see
+// ot_testing_fail_device_allocs): allocations left before one fails, -1 = off.
+std::atomic<int> g_fail_countdown{-1};
+
 cudaError_t pool_device_alloc(void **ptr, size_t bytes, size_t *got) {
+    int left = g_fail_countdown.load();
+    while (left >= 0 && !g_fail_countdown.compare_exchange_weak(left, left - 1)) {
+    }
+    if (left == 0) {
+        *ptr = nullptr;
+        return cudaErrorMemoryAllocation;
+    }
     const int d = current_device();
     if (d >= 0) {
         Pool &P = pool();
@@ -67,10 +82,9 @@ cudaError_t pool_device_alloc(void **ptr, size_t bytes, size_t *got) {
     return cudaMalloc(ptr, bytes);
 }
 
-void pool_device_free(void *ptr, size_t bytes) {
+void pool_device_free(void *ptr, size_t bytes, int d) {
     if (!ptr) return;
-    const int d = current_device();
-    if (d >= 0) {
+    if (d >= 0 && d < kDevices) {
         Pool &P = pool();
         std::lock_guard<std::mutex> lk(P.mu);
         if (P.dev_bytes[d] + bytes <= kKeepBytes) {
@@ -120,10 +134,9 @@ cudaError_t pool_stream(cudaStream_t *s) {
     return cudaStreamCreateWithFlags(s, cudaStreamNonBlocking);
 }
 
-void pool_stream_release(cudaStream_t s) {
+void pool_stream_release(cudaStream_t s, int d) {
     if (!s) return;
-    const int d = current_device();
-    if (d >= 0) {
+    if (d >= 0 && d < kDevices) {
         Pool &P = pool();
         std::lock_guard<std::mutex> lk(P.mu);
         if (P.streams[d].size() < 16) {
@@ -156,4 +169,11 @@ extern "C" void ot_trim_cache(void) {
     cudaSetDevice(prev);
     for (auto &kv : P.host) cudaFreeHost(kv.second);
     P.host.clear();
+}
+
+// Test hook (include/ot_sinkhorn_testing.h): the device-workspace allocation
+// after `after` more successful ones fails as cudaMalloc does when memory runs
+// out; a negative value switches the injection off.
+extern "C" void ot_testing_fail_device_allocs(int after) {
+    ot::g_fail_countdown.store(after < 0 ? -1 : after);
 }

@@ -120,11 +120,15 @@ __global__ void __launch_bounds__(kMaxThreads) max_cost_kernel(const float *__re
 }
 
 // ----------------------------------------------------------------- params
-__global__ void set_params_kernel(Params *prm, double eps, double c, double tol) {
+__global__ void set_params_kernel(Params *prm, double eps, double c, double tol, double *hist,
+                                  int64_t hist_off, int64_t hist_len) {
     prm->eps = eps;
     prm->kappa = kLog2e / eps;
     prm->c = c;
     prm->tol = tol;
+    prm->hist = hist;
+    prm->hist_off = hist_off;
+    prm->hist_len = hist_len;
 }
 
 __global__ void reset_state_kernel(State *st) {
@@ -286,8 +290,9 @@ cudaError_t launch_max_cost(const float *x, const float *y, int64_t n, int64_t m
     return cudaGetLastError();
 }
 
-cudaError_t launch_set_params(Params *prm, double eps, double c, double tol, cudaStream_t s) {
-    set_params_kernel<<<1, 1, 0, s>>>(prm, eps, c, tol);
+cudaError_t launch_set_params(Params *prm, double eps, double c, double tol, double *hist,
+                              int64_t hist_off, int64_t hist_len, cudaStream_t s) {
+    set_params_kernel<<<1, 1, 0, s>>>(prm, eps, c, tol, hist, hist_off, hist_len);
     return cudaGetLastError();
 }
 

@@ -12,41 +12,53 @@
 //   e2_ij = A_i + B_j + sum_q P_iq y'_jq,
 //   A_i = kappa (f_i - c |x'_i|^2), B_j = kappa (g_j - c |y'_j|^2), P_i = 2 c kappa x'_i,
 // all in float64 (FlashSinkhorn 2, section D.3: accurate evaluation is done in
-// FP64). Then e2 = k + r with k the nearest integer, |r| <= 1/2; T = 2^r (MUFU
-// ex2 on the float r, relative error ~2^-22) scaled by 2^k through the exponent
-// field, with a two-step scaling into the subnormal range. A massless side
-// (potential -inf) gives e2 = -inf and T = 0. The row passes keep their sums in
-// compensated float32 (and maxima/counts exactly), so each entry costs one
-// conversion and one ex2 on the XU pipe.
+// FP64). The sum is formed on t = kShift + e2 rather than on e2: kShift = 1.5 *
+// 2^29 + 190 keeps t in [2^29, 2^30), where a float64 step is 2^-23, so every
+// operation rounds e2 to a multiple of 2^-23 (at most 2^-24 off, ~2e-7 relative
+// in T after the five operations) and the low 32 bits of t are the integer
+// (190 + e2) * 2^23 -- the range reduction is then two integer operations: the
+// fraction of e2 goes into the mantissa of a float in [1, 2), whose MUFU ex2
+// (relative error ~2^-22) is scaled by 2^floor(e2) through the exponent field.
+// e2 is clamped to [-189, 64] first (two float64 min/max): below, T rounds to 0
+// (a massless side, potential -inf, lands there); at 64 and above T is +inf
+// (the float result of an entry of 2^64 or more). The scaled value is formed
+// 2^64 too large and multiplied by 2^-64 at the end, so entries below 2^-126
+// round correctly into the subnormal range. Per entry: d + 1 float64 FMAs/adds,
+// two float64 min/max, two integer operations, one ex2 and one float multiply.
+// The row passes accumulate each row's terms 8 at a time in float32 and those
+// partial sums in float64 (maxima and counts exactly).
 #include "runtime.h"
 
 namespace ot {
 
-__device__ __forceinline__ float exp2_split(double e2) {
-    if (!(e2 > -152.0)) return 0.0f;          // below half the smallest subnormal
-    if (e2 >= 128.0) return INFINITY;
-    // nearest integer k by adding 1.5 * 2^52 (ulp 1 there): k lands in the low
-    // mantissa bits and e2 - k is exact, so the only conversion left is r -> float
-    const double big = 6755399441055744.0;
-    const double t = e2 + big;
-    const int k = __double2loint(t);
-    const float p = ex2_approx((float)(e2 - (t - big)));  // in [2^-1/2, 2^1/2]
-    if (k >= -125) return __int_as_float(__float_as_int(p) + (k << 23));
-    return p * __int_as_float((k + 64 + 127) << 23) * 5.42101086242752217e-20f;  // * 2^-64
+constexpr double kShift = 805306368.0 + 190.0;  // 1.5 * 2^29 + 190
+constexpr double kShiftLo = kShift - 189.0;     // e2 >= -189
+constexpr double kShiftHi = kShift + 64.0;      // e2 <= 64
+
+// T = 2^e2 from t = kShift + e2 (see above).
+__device__ __forceinline__ float exp2_shifted(double t) {
+    t = fmin(fmax(t, kShiftLo), kShiftHi);
+    const unsigned q = (unsigned)__double2loint(t);          // (190 + e2) * 2^23
+    const unsigned mant = (q & 0x7FFFFFu) | 0x3F800000u;      // 1 + frac(e2), in [1, 2)
+    const float p = ex2_approx(__uint_as_float(mant));         // 2^(1 + frac(e2)), in [2, 4]
+    // exponent field + floor(e2) + 63: q - mant = (floor(e2) + 63) * 2^23
+    const float v = __uint_as_float(__float_as_uint(p) + q - mant);
+    return v * 5.42101086242752217e-20f;                       // * 2^-64
 }
 
-// the one float path for a plan entry: row data (A, P[d]), column data (y'[d], B)
+// the one float path for a plan entry: row data (A' = A + kShift, P[d]),
+// column data (y'[d], B)
 template <int D>
-__device__ __forceinline__ float plan_entry(double A, const double *P, const double *col, int d) {
+__device__ __forceinline__ float plan_entry(double Ash, const double *P, const double *col, int d) {
     const int dd = D > 0 ? D : d;
-    double s = A + col[dd];
+    double t = Ash + col[dd];
 #pragma unroll
     for (int q = 0; q < (D > 0 ? D : 1); ++q) {
-        if (D > 0) s = fma(P[q], col[q], s);
+        if (D > 0) t = fma(P[q], col[q], t);
     }
     if (D == 0)
-        for (int q = 0; q < dd; ++q) s = fma(P[q], col[q], s);
-    return exp2_split(s);
+        for (int q = 0; q < dd; ++q) t = fma(P[q], col[q], t);
+    return exp2_shifted(t);
 }
 
 // Column table in float64: dcol[j*(d+1) + q] = y'_jq (q < d), dcol[j*(d+1) + d] = B_j.
@@ -66,7 +78,7 @@ __global__ void build_dcol_kernel(const float *__restrict__ p, const float *__re
     dcol[j * (d + 1) + d] = (pv == -INFINITY) ? -INFINITY : kappa * ((double)pv - c * nrm);
 }
 
-// Row data of one row into shared memory: A and P (d values).
+// Row data of one row: A' = A + kShift and P (d values).
 __device__ __forceinline__ void load_row(const float *pts, const float *pot, int64_t i, int d,
                                          const double *o, double kappa, double c, double *A,
                                          double *P) {
@@ -77,7 +89,7 @@ __device__ __forceinline__ void load_row(const float *pts, const float *pot, int
         nrm += v * v;
     }
     const float pv = pot[i];
-    *A = (pv == -INFINITY) ? -INFINITY : kappa * ((double)pv - c * nrm);
+    *A = (pv == -INFINITY) ? -INFINITY : kappa * ((double)pv - c * nrm) + kShift;
 }
 
 // ------------------------------------------------------------ materializer
@@ -152,25 +164,151 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
 }
 
 // ------------------------------------------------------- row-complete passes
-// A block owns 8 rows and visits every column, so each row's reduction stays
-// in one block and is done in a fixed order (deterministic):
+// A pass visits every entry of a range of rows and reduces each row:
 //   OP_MAX:   rowmax[i] = max_j T_ij                       (min_row, pass A)
 //   OP_COUNT: counts[i] = #{j : T_ij >= thr} if w_i > 0    (min_row, pass B)
 //   OP_SUM:   part[block] = sum over its rows of |sum_j T_ij - w_i|  (residual)
 // "Rows" may be either cloud: the column residual runs the same pass with the
 // roles of (x, f, a) and (y, g, b) swapped, since T is symmetric in them.
+//
+// d <= 3: a block of 8 warps owns 64 rows, 8 per warp, whose float64 data sit
+// in registers; the columns' float64 records (y'[d], B) stream through shared
+// memory 256 at a time (the next chunk prefetched into registers), so a column
+// is read from L2 once per 64 rows and from shared memory once per 8 entries.
+// Lane l takes columns l, l + 32, ... of each chunk for all 8 rows of its warp,
+// so every row's reduction stays in one warp, in a fixed lane order
+// (deterministic). Sums: the 8 terms of a row in one chunk add up in float32,
+// those partial sums in float64.
 enum { OP_MAX = 0, OP_COUNT = 1, OP_SUM = 2 };
-constexpr int kRpThreads = 256, kRpRows = 8;
-
+constexpr int kRpThreads = 256, kRpWarps = kRpThreads / 32, kRpR = 8, kRpChunk = 256;
+constexpr int kRpRows = kRpWarps * kRpR;  // rows per block, d <= 3
+constexpr int kRgRows = 8;                // rows per block, generic d
 
 template <int D, int OP>
-__global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
-    __shared__ double sA[kRpRows], sP[kRpRows][D > 0 ? D : kMaxD];
-    __shared__ double sRed[kRpThreads / 32][kRpRows];
+__global__ void __launch_bounds__(kRpThreads, 2) rowpass_kernel(RowPassArgs R) {
+    constexpr int DS = D + 1;                 // doubles per column record
+    constexpr int DP = D == 1 ? 2 : 4;        // padded stride in shared memory
+    constexpr int PER = (kRpChunk * DS + kRpThreads - 1) / kRpThreads;  // prefetched doubles
+    __shared__ __align__(16) double sc[kRpChunk * DP];
+    __shared__ double sRed[kRpWarps][kRpR];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rw = R.row_begin + (int64_t)blockIdx.x * kRpRows + (int64_t)warp * kRpR;
+    double Ash[kRpR], P[kRpR][D];
+#pragma unroll
+    for (int r = 0; r < kRpR; ++r) {
+        if (rw + r < R.row_end) {
+            load_row(R.pts, R.pot, rw + r, D, R.o, R.prm->kappa, R.prm->c, &Ash[r], P[r]);
+        } else {
+            Ash[r] = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < D; ++q) P[r][q] = 0.0;
+        }
+    }
+    float mx[kRpR];
+    int cnt[kRpR];
+    double sum[kRpR];
+#pragma unroll
+    for (int r = 0; r < kRpR; ++r) {
+        mx[r] = -1.0f;
+        cnt[r] = 0;
+        sum[r] = 0.0;
+    }
+    // chunk c's records are elements [c * 256 * DS, (c + 1) * 256 * DS) of dcol;
+    // thread t holds elements t, t + 256, ... of the next one
+    const int64_t total = R.cols * DS;
+    double pre[PER];
+    auto fetch = [&](int64_t c0) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t e = c0 * DS + tid + (int64_t)k * kRpThreads;
+            pre[k] = (tid + k * kRpThreads < kRpChunk * DS && e < total) ? __ldg(R.dcol + e)
+                     : ((tid + k * kRpThreads) % DS == D ? -INFINITY : 0.0);
+        }
+    };
+    fetch(0);
+    for (int64_t c0 = 0; c0 < R.cols; c0 += kRpChunk) {
+        __syncthreads();  // the previous chunk is no longer read
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int e = tid + k * kRpThreads;
+            if (e < kRpChunk * DS) sc[(e / DS) * DP + (e % DS)] = pre[k];
+        }
+        __syncthreads();
+        if (c0 + kRpChunk < R.cols) fetch(c0 + kRpChunk);
+        float part[kRpR];
+#pragma unroll
+        for (int r = 0; r < kRpR; ++r) part[r] = 0.0f;
+#pragma unroll 2
+        for (int s = 0; s < kRpChunk / 32; ++s) {
+            const int cc = s * 32 + lane;
+            double col[DP];
+            if (DP == 2) {
+                const double2 v = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
+                col[0] = v.x;
+                col[1] = v.y;
+            } else {
+                const double2 v0 = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
+                const double2 v1 = *reinterpret_cast<const double2 *>(&sc[cc * DP + 2]);
+                col[0] = v0.x;
+                col[1] = v0.y;
+                col[2] = v1.x;
+                col[3] = v1.y;
+            }
+            const bool live = c0 + cc < R.cols;
+#pragma unroll
+            for (int r = 0; r < kRpR; ++r) {
+                const float t = plan_entry<D>(Ash[r], P[r], col, D);
+                if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
+                if (OP == OP_COUNT) cnt[r] += (live && t >= R.thr) ? 1 : 0;
+                if (OP == OP_SUM) part[r] += t;
+            }
+        }
+        if (OP == OP_SUM) {
+#pragma unroll
+            for (int r = 0; r < kRpR; ++r) sum[r] += (double)part[r];
+        }
+    }
+    // per-row reductions across the warp (fixed order), then per block
+#pragma unroll
+    for (int r = 0; r < kRpR; ++r) {
+        double v = OP == OP_SUM ? sum[r] : OP == OP_COUNT ? (double)cnt[r] : (double)mx[r];
+        for (int off = 16; off > 0; off >>= 1) {
+            const double o2 = __shfl_xor_sync(0xffffffffu, v, off);
+            v = OP == OP_MAX ? fmax(v, o2) : v + o2;
+        }
+        if (lane == 0) {
+            const int64_t i = rw + r;
+            double res = 0.0;
+            if (i < R.row_end) {
+                const float wi = R.w[i];
+                if (OP == OP_MAX) R.rowmax[i] = (float)v;
+                if (OP == OP_COUNT) R.counts[i] = wi > 0.0f ? (int64_t)v : 0;
+                if (OP == OP_SUM) res = fabs(v - (double)wi);
+            }
+            sRed[warp][r] = res;
+        }
+    }
+    if (OP == OP_SUM) {
+        __syncthreads();
+        if (tid == 0) {
+            double t = 0.0;
+            for (int w = 0; w < kRpWarps; ++w)
+                for (int r = 0; r < kRpR; ++r) t += sRed[w][r];
+            R.part[blockIdx.x] = t;
+        }
+    }
+}
+
+// Generic d (> 3): a block owns 8 rows (float64 data in shared memory) and its
+// 256 threads visit every column, each entry read from the global column table.
+template <int OP>
+__global__ void __launch_bounds__(kRpThreads) rowpass_generic_kernel(RowPassArgs R) {
+    __shared__ double sA[kRgRows], sP[kRgRows][kMaxD];
+    __shared__ double sRed[kRpThreads / 32][kRgRows];
     const int tid = threadIdx.x;
-    const int64_t r0 = R.row_begin + (int64_t)blockIdx.x * kRpRows;
-    const int d = D > 0 ? D : R.d;
-    if (tid < kRpRows) {
+    const int64_t r0 = R.row_begin + (int64_t)blockIdx.x * kRgRows;
+    const int d = R.d;
+    if (tid < kRgRows) {
         const int64_t i = r0 + tid;
         if (i < R.row_end)
             load_row(R.pts, R.pot, i, d, R.o, R.prm->kappa, R.prm->c, &sA[tid], sP[tid]);
@@ -178,41 +316,37 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
             sA[tid] = -INFINITY;
     }
     __syncthreads();
-    // per row: max (OP_MAX), count (OP_COUNT) or a compensated float sum (OP_SUM)
-    float acc[kRpRows], comp[kRpRows];
-    int cnt[kRpRows];
+    float mx[kRgRows];
+    int cnt[kRgRows];
+    double sum[kRgRows];
 #pragma unroll
-    for (int r = 0; r < kRpRows; ++r) {
-        acc[r] = OP == OP_MAX ? -1.0f : 0.0f;
-        comp[r] = 0.0f;
+    for (int r = 0; r < kRgRows; ++r) {
+        mx[r] = -1.0f;
         cnt[r] = 0;
+        sum[r] = 0.0;
     }
-    constexpr int DS = (D > 0 ? D : 1) + 1;
-    for (int64_t j = tid; j < R.cols; j += kRpThreads) {
-        double cd[DS];
-        const double *col = R.dcol + j * (d + 1);
-        if (D > 0) {
+    for (int64_t j0 = 0; j0 < R.cols; j0 += (int64_t)kRpThreads * 8) {
+        float part[kRgRows];
 #pragma unroll
-            for (int q = 0; q < DS; ++q) cd[q] = col[q];
-        }
+        for (int r = 0; r < kRgRows; ++r) part[r] = 0.0f;
+        for (int64_t j = j0 + tid; j < min(R.cols, j0 + (int64_t)kRpThreads * 8); j += kRpThreads) {
+            const double *col = R.dcol + j * (d + 1);
 #pragma unroll
-        for (int r = 0; r < kRpRows; ++r) {
-            const float t = D > 0 ? plan_entry<D>(sA[r], sP[r], cd, d)
-                                  : plan_entry<0>(sA[r], sP[r], col, d);
-            if (OP == OP_MAX) acc[r] = fmaxf(acc[r], t);
-            if (OP == OP_COUNT) cnt[r] += (t >= R.thr) ? 1 : 0;
-            if (OP == OP_SUM) {  // Kahan: the error stays ~2^-24 of the sum
-                const float yv = t - comp[r];
-                const float u = acc[r] + yv;
-                comp[r] = (u - acc[r]) - yv;
-                acc[r] = u;
+            for (int r = 0; r < kRgRows; ++r) {
+                const float t = plan_entry<0>(sA[r], sP[r], col, d);
+                if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
+                if (OP == OP_COUNT) cnt[r] += (t >= R.thr) ? 1 : 0;
+                if (OP == OP_SUM) part[r] += t;
             }
         }
+        if (OP == OP_SUM) {
+#pragma unroll
+            for (int r = 0; r < kRgRows; ++r) sum[r] += (double)part[r];
+        }
     }
 #pragma unroll
-    for (int r = 0; r < kRpRows; ++r) {
-        double v = OP == OP_SUM ? (double)acc[r] - (double)comp[r]
-                 : OP == OP_COUNT ? (double)cnt[r] : (double)acc[r];
+    for (int r = 0; r < kRgRows; ++r) {
+        double v = OP == OP_SUM ? sum[r] : OP == OP_COUNT ? (double)cnt[r] : (double)mx[r];
         for (int off = 16; off > 0; off >>= 1) {
             const double o2 = __shfl_xor_sync(0xffffffffu, v, off);
             v = OP == OP_MAX ? fmax(v, o2) : v + o2;
@@ -220,7 +354,7 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
         if ((tid & 31) == 0) sRed[tid >> 5][r] = v;
     }
     __syncthreads();
-    if (tid < kRpRows) {
+    if (tid < kRgRows) {
         double v = sRed[0][tid];
         for (int w = 1; w < kRpThreads / 32; ++w) v = OP == OP_MAX ? fmax(v, sRed[w][tid]) : v + sRed[w][tid];
         const int64_t i = r0 + tid;
@@ -237,7 +371,7 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
         __syncthreads();
         if (tid == 0) {
             double t = 0.0;
-            for (int r = 0; r < kRpRows; ++r) t += sRed[0][r];
+            for (int r = 0; r < kRgRows; ++r) t += sRed[0][r];
             R.part[blockIdx.x] = t;
         }
     }
@@ -254,7 +388,7 @@ __global__ void __launch_bounds__(kRpThreads) rowpass_kernel(RowPassArgs R) {
 // broadcasts, columns as one 16-byte load per thread and k). The coupling accumulates in float32
 // (its factors are nonnegative: relative error <= r 2^-24); the cost
 // accumulates its dot products in float64 and assembles the exponent like the
-// point-cloud rows (exp2_split).
+// point-cloud rows (exp2_shifted).
 constexpr int kLrRows = 64, kLrCols = 128, kLrThreads = 256, kLrRowsPerBlock = 512;
 
 template <typename T, int MODE>
@@ -328,8 +462,7 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_rows_kernel(LrArgs L) {
                     const int64_t j = jb + b < L.m ? jb + b : L.m - 1;
                     const float gv = L.gp[j];
                     const double Bj = gv == -INFINITY ? -1e15 : L.kappa * (double)gv;
-                    const double e2 = Ai + Bj - L.kc * ((double)acc[a][b] + L.bias);
-                    o[b] = exp2_split(fmin(fmax(e2, -1e15), 1e15));
+                    o[b] = exp2_shifted(fma(-L.kc, (double)acc[a][b] + L.bias, (Ai + kShift) + Bj));
                 }
             }
             float *dst = L.out + t * L.m + jb;
@@ -377,17 +510,19 @@ cudaError_t launch_lowrank_rows(int mode, const LrArgs &L, cudaStream_t s) {
 // plan_entry() as the count pass that produced row_ptr; a row never writes
 // past its own segment, and a row whose kept entries do not fill it exactly
 // sets *bad (it cannot happen unless the two passes disagree).
+constexpr int kCsrRows = 8;  // rows per block of the compressed-row write
+
 template <int D>
 __global__ void __launch_bounds__(kRpThreads) csr_write_kernel(CsrArgs C) {
     constexpr int WARPS = kRpThreads / 32;
-    __shared__ double sA[kRpRows], sP[kRpRows][D > 0 ? D : kMaxD];
-    __shared__ int sCnt[kRpRows][WARPS];
-    __shared__ long long sPos[kRpRows], sEnd[kRpRows];
-    __shared__ int sLive[kRpRows];
+    __shared__ double sA[kCsrRows], sP[kCsrRows][D > 0 ? D : kMaxD];
+    __shared__ int sCnt[kCsrRows][WARPS];
+    __shared__ long long sPos[kCsrRows], sEnd[kCsrRows];
+    __shared__ int sLive[kCsrRows];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t r0 = C.row_begin + (int64_t)blockIdx.x * kRpRows;
+    const int64_t r0 = C.row_begin + (int64_t)blockIdx.x * kCsrRows;
     const int d = D > 0 ? D : C.d;
-    if (tid < kRpRows) {
+    if (tid < kCsrRows) {
         const int64_t i = r0 + tid;
         const int live = i < C.row_end && C.w[i] > 0.0f;
         if (live) {
@@ -412,10 +547,10 @@ __global__ void __launch_bounds__(kRpThreads) csr_write_kernel(CsrArgs C) {
 #pragma unroll
             for (int q = 0; q < DS; ++q) cd[q] = col[q];
         }
-        float t[kRpRows];
-        unsigned bal[kRpRows];
+        float t[kCsrRows];
+        unsigned bal[kCsrRows];
 #pragma unroll
-        for (int r = 0; r < kRpRows; ++r) {
+        for (int r = 0; r < kCsrRows; ++r) {
             t[r] = D > 0 ? plan_entry<D>(sA[r], sP[r], cd, d) : plan_entry<0>(sA[r], sP[r], col, d);
             const bool keep = colok && sLive[r] && t[r] >= C.thr;
             bal[r] = __ballot_sync(0xffffffffu, keep);
@@ -423,7 +558,7 @@ __global__ void __launch_bounds__(kRpThreads) csr_write_kernel(CsrArgs C) {
         }
         __syncthreads();
 #pragma unroll
-        for (int r = 0; r < kRpRows; ++r) {
+        for (int r = 0; r < kCsrRows; ++r) {
             if (!((bal[r] >> lane) & 1u)) continue;
             long long off = sPos[r] + __popc(bal[r] & below);
             for (int w = 0; w < warp; ++w) off += sCnt[r][w];
@@ -435,14 +570,14 @@ __global__ void __launch_bounds__(kRpThreads) csr_write_kernel(CsrArgs C) {
             }
         }
         __syncthreads();
-        if (tid < kRpRows) {
+        if (tid < kCsrRows) {
             int tot = 0;
             for (int w = 0; w < WARPS; ++w) tot += sCnt[tid][w];
             sPos[tid] += tot;
         }
         __syncthreads();
     }
-    if (tid < kRpRows && sLive[tid] && sPos[tid] != sEnd[tid]) atomicExch(C.bad, 1);
+    if (tid < kCsrRows && sLive[tid] && sPos[tid] != sEnd[tid]) atomicExch(C.bad, 1);
 }
 
 // Exclusive scan of the row counts into row_ptr, in three launches: tiles of
@@ -617,12 +752,13 @@ cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s) {
 }
 
 template <int OP>
-static void rowpass_dispatch(const RowPassArgs &R, unsigned grid, cudaStream_t s) {
+static void rowpass_dispatch(const RowPassArgs &R, int64_t rows, cudaStream_t s) {
+    const unsigned grid = (unsigned)rowpass_blocks(rows, R.d);
     switch (R.d) {
         case 1: rowpass_kernel<1, OP><<<grid, kRpThreads, 0, s>>>(R); break;
         case 2: rowpass_kernel<2, OP><<<grid, kRpThreads, 0, s>>>(R); break;
         case 3: rowpass_kernel<3, OP><<<grid, kRpThreads, 0, s>>>(R); break;
-        default: rowpass_kernel<0, OP><<<grid, kRpThreads, 0, s>>>(R); break;
+        default: rowpass_generic_kernel<OP><<<grid, kRpThreads, 0, s>>>(R); break;
     }
 }
 
@@ -630,14 +766,16 @@ static void rowpass_dispatch(const RowPassArgs &R, unsigned grid, cudaStream_t s
 cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s) {
     const int64_t rows = R.row_end - R.row_begin;
     if (rows <= 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((rows + kRpRows - 1) / kRpRows);
-    if (op == OP_MAX) rowpass_dispatch<OP_MAX>(R, grid, s);
-    else if (op == OP_COUNT) rowpass_dispatch<OP_COUNT>(R, grid, s);
-    else rowpass_dispatch<OP_SUM>(R, grid, s);
+    if (op == OP_MAX) rowpass_dispatch<OP_MAX>(R, rows, s);
+    else if (op == OP_COUNT) rowpass_dispatch<OP_COUNT>(R, rows, s);
+    else rowpass_dispatch<OP_SUM>(R, rows, s);
     return cudaGetLastError();
 }
 
-int64_t rowpass_blocks(int64_t rows) { return (rows + kRpRows - 1) / kRpRows; }
+int64_t rowpass_blocks(int64_t rows, int d) {
+    const int per = d <= 3 ? kRpRows : kRgRows;
+    return (rows + per - 1) / per;
+}
 
 cudaError_t launch_min_row_reduce(const float *rowmax, const float *w, int64_t n, float *thr,
                                   int64_t *argmin, int64_t *n_massless, cudaStream_t s) {
@@ -653,7 +791,7 @@ cudaError_t launch_sum_i64(const int64_t *v, int64_t cnt, int64_t *out, cudaStre
 cudaError_t launch_csr_write(const CsrArgs &C, cudaStream_t s) {
     const int64_t rows = C.row_end - C.row_begin;
     if (rows <= 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((rows + kRpRows - 1) / kRpRows);
+    const unsigned grid = (unsigned)((rows + kCsrRows - 1) / kCsrRows);
     switch (C.d) {
         case 1: csr_write_kernel<1><<<grid, kRpThreads, 0, s>>>(C); break;
         case 2: csr_write_kernel<2><<<grid, kRpThreads, 0, s>>>(C); break;

@@ -1,21 +1,34 @@
 // runtime.h -- host-side declarations of the kernel launchers (internal).
 #pragma once
 #include <cuda.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 
 namespace ot {
 
+// An NVTX range around one C-ABI call, so profilers show each call of the
+// library by name (NVTX v3 is header-only: without a tool attached the push
+// and pop cost a branch).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
 // api.cu: sets the thread's last-error text and returns code
 int set_error(int code, const char *fmt, ...);
 
-// pool.cu: cached device workspaces, pinned host buffers and streams
+// pool.cu: cached device workspaces, pinned host buffers and streams (an
+// allocation is made on the current device; a release names the device the
+// resource belongs to)
 cudaError_t pool_device_alloc(void **ptr, size_t bytes, size_t *got);
-void pool_device_free(void *ptr, size_t bytes);
+void pool_device_free(void *ptr, size_t bytes, int device);
 cudaError_t pool_host_alloc(void **ptr, size_t bytes);
 void pool_host_free(void *ptr, size_t bytes);
 cudaError_t pool_stream(cudaStream_t *s);
-void pool_stream_release(cudaStream_t s);
+void pool_stream_release(cudaStream_t s, int device);
 
 // halfstep.cu
 int halfstep_blocks_per_sm(int kind, int dim, int rpt);
@@ -31,6 +44,9 @@ struct LoopArgs {
     unsigned *bar_count;    // grid barrier: arrivals
     unsigned *bar_gen;      // grid barrier: generation
     double *blk_resid;      // [grid] residual partial of each block
+    unsigned long long wait_ns;  // grid-barrier time limit
+    int withhold_block;     // failure tests only: this block returns before its first
+                            // barrier arrival (-1: none)
 };
 int loop_blocks_per_sm(int d, int rpt);
 cudaError_t launch_loop(int d, int rpt, const LoopArgs &L, int grid, cudaStream_t s);
@@ -52,7 +68,8 @@ cudaError_t launch_coord_stats(const float *v, int64_t cnt, int d, double *part,
                                unsigned long long *zero_count, cudaStream_t s);
 cudaError_t launch_max_cost(const float *x, const float *y, int64_t n, int64_t m, int d,
                             const double *o, unsigned *out_bits, cudaStream_t s);
-cudaError_t launch_set_params(Params *prm, double eps, double c, double tol, cudaStream_t s);
+cudaError_t launch_set_params(Params *prm, double eps, double c, double tol, double *hist,
+                              int64_t hist_off, int64_t hist_len, cudaStream_t s);
 cudaError_t launch_reset_state(State *st, cudaStream_t s);
 cudaError_t launch_tables(const float *p, const float *pot, int64_t cnt, int64_t cnt_pad, int d,
                           int dp, const double *o, const Params *prm, float *rowtab,
@@ -188,7 +205,8 @@ cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, co
                         const Params *prm, double *dcol, cudaStream_t s);
 cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s);
 cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s);
-int64_t rowpass_blocks(int64_t rows);
+// residual partials one pass over `rows` rows writes (blocks of the pass)
+int64_t rowpass_blocks(int64_t rows, int d);
 cudaError_t launch_min_row_reduce(const float *rowmax, const float *w, int64_t n, float *thr,
                                   int64_t *argmin, int64_t *n_massless, cudaStream_t s);
 cudaError_t launch_sum_i64(const int64_t *v, int64_t cnt, int64_t *out, cudaStream_t s);

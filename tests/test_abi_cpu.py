@@ -8,7 +8,8 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "ot_sinkhorn.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,7 +21,7 @@ def B():
 
 
 def _declared():
-    txt = open(HEADER).read()
+    txt = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"^OT_API [^(]*?\b(ot_\w+)\(", txt, re.M)))
 
 
@@ -38,7 +39,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_version_and_defaults(B):
-    assert B.ot_version() == 2
+    assert B.ot_version() == 3
     o = B.ot_options_default()
     assert (o.warm_start, o.check_every, o.use_graphs, o.iters_per_stage) == (0, 16, 1, 20)
     assert (o.scale_value, o.eps_init, o.eps_decay) == (1.0, 0.0, 0.7)
@@ -48,7 +49,7 @@ def test_version_and_defaults(B):
 
 
 def test_struct_sizes_match_header_layout(B):
-    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4 + 4 * 4 + 2 * 8
+    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4 + 4 * 4 + 2 * 8 + 2 * 8
     assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8 + 6 * 8 + 8 + 3 * 8
 
 
@@ -134,3 +135,23 @@ def test_valid_call_without_gpu_fails_loudly(B):
         pytest.skip("a GPU is present")
     st, plan = _call(B)
     assert st == -3 and plan is None
+
+
+def test_residual_history_needs_an_array(B):
+    o = B.ot_options_default()
+    o.resid_history_len = 5  # no array
+    assert _call(B, opt=o)[0] == B.OT_ERR_INVALID_ARG
+    o.resid_history_len = -1
+    assert _call(B, opt=o)[0] == B.OT_ERR_INVALID_ARG
+
+
+def test_host_entry_point_validates_before_touching_memory(B):
+    L = B.lib()
+    for n, d, code in ((0, 3, B.OT_ERR_INVALID_ARG), (4, 0, B.OT_ERR_INVALID_ARG),
+                       (4, 65, B.OT_ERR_UNSUPPORTED), (1 << 31, 3, B.OT_ERR_OVERFLOW)):
+        st = L.ot_sinkhorn_pointcloud_host(FAKE, FAKE, FAKE, FAKE, n, 4, d, 0.1, 0, 1, 0.0, FAKE, FAKE,
+                                           None, None, None, None)
+        assert st == code, (n, d, st)
+    st = L.ot_sinkhorn_pointcloud_host(None, FAKE, FAKE, FAKE, 4, 4, 3, 0.1, 0, 1, 0.0, FAKE, FAKE,
+                                       None, None, None, None)
+    assert st == B.OT_ERR_INVALID_ARG

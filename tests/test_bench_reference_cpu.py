@@ -28,7 +28,7 @@ def test_reference_arm_prints_one_contract_line():
                 "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in line, key
     assert line["impl"] == "reference" and line["higher_is_better"] is True
-    assert line["config"]["workload"] == "w2_gmm3d_8000"
+    assert line["config"]["workload"] == "w5_spirals_2e6"
     assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["value"] == line["value"] and line["e2e"]["unit"] == line["unit"]
