@@ -88,6 +88,10 @@ def _args():
                     help="--sparse: uniform-vs-64-clusters (w4) or interleaved spirals (w5)")
     ap.add_argument("--sparse-block", type=int, default=0, choices=[0, 128, 256],
                     help="--sparse: block size B (0 = the library's choice)")
+    ap.add_argument("--rows", action="store_true",
+                    help="instead of the step: the row kernels (a 1024-row materializer block, the "
+                         "marginal residual, min_row) at the state after 5 iterations of the workload "
+                         "(or its --n/--m replica); prints its own JSON line")
     ap.add_argument("--no-side", action="store_true",
                     help="skip the side measurements (scale pass, row kernels, block-sparse)")
     ap.add_argument("--clock-ms", type=int, default=200,
@@ -725,10 +729,29 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_rows(args):
+    """The row kernels alone on a solved state of the workload."""
+    import torch
+    import log_domain_sinkhorn_online_b200 as ot
+    dev = torch.device("cuda", 0)
+    w = _workload(args.workload, args.n, args.m)
+    step = Step(ot, w, dev, iters=5)
+    step()
+    peaks, kind = _peaks()
+    peak_ex2 = SMS * EX2_PER_CLK * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    side = _side(ot, step, w, torch.cuda.current_stream(), peak_ex2, float(peaks["hbm_gbs"]))
+    side.pop("scale_pass", None)
+    print(json.dumps({"metric": "row kernels", "config": {"workload": w.name, "n": w.n, "m": w.m, "d": w.d},
+                      "peak_ex2_per_s": peak_ex2, "hbm_gbs": float(peaks["hbm_gbs"]), "peaks": kind,
+                      **side}), flush=True)
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.rows:
+        run_rows(args)
     elif args.lowrank:
         run_lowrank(args)
     elif args.sparse:

@@ -138,6 +138,13 @@ typedef struct ot_options {
                                  (the last iteration of each annealing stage but the final
                                  one; iterations beyond the run) are NaN. NULL: none */
     int64_t resid_history_len;/* entries of resid_history (0 = none) */
+    uint8_t *sparse_mask_out; /* block-sparse mode, optional device array [NB * MB] (NB, MB: the
+                                 blocks of x and y in Morton order; NB * MB <= sparse_mask_len,
+                                 else OT_ERR_INVALID_ARG): receives the block mask of the first
+                                 fine update of the solve, the one built at the starting
+                                 potentials -- 1 for an admitted tile (a candidate, in an
+                                 iteration that ran dense), row-major by x block. NULL: none */
+    int64_t sparse_mask_len;  /* bytes available at sparse_mask_out */
 } ot_options;
 
 /* -------------------------------------------------------- solve report   */
@@ -187,7 +194,8 @@ OT_API const char *ot_last_error_string(void);
  * iters_per_stage 20, scale_value 1, eps_init 0, eps_decay 0.7, timing 0,
  * col_splits 0, rows_per_thread 0, tensor_cores 1, device_loop -1,
  * block_sparse 0, sparse_block 0, sparse_verify 1, sparse_delta 0,
- * sparse_dense_frac 0.5, resid_history NULL, resid_history_len 0). */
+ * sparse_dense_frac 0.5, resid_history NULL, resid_history_len 0,
+ * sparse_mask_out NULL, sparse_mask_len 0). */
 OT_API void ot_options_default(ot_options *opt);
 
 /* ------------------------------------------------- ot_sinkhorn_pointcloud
@@ -253,7 +261,9 @@ OT_API int ot_marginal_residual(const ot_plan *plan, double *row_l1, double *col
  * Fix: entropic rows exp((f_i + g_j - C_ij)/eps) with the captured scale and
  * eps; O(k*m) memory). row_idx [k]: device int64, each in [0, n) (repeats
  * allowed); out [k,m]: device float32, row-major. The exponent is assembled
- * in float64; the value is rounded to float32. A row index out of range makes
+ * in float64; the value is rounded to float32, with entries of 2^128 or more
+ * returned as +inf and entries below 2^-126 (1.2e-38, the smallest normal
+ * float) as 0 (the same holds for every row call). A row index out of range makes
  * the call return OT_ERR_INVALID_ARG (checked on the device, no fault); the
  * rows with valid indices are still written. Synchronises `stream`. */
 OT_API int ot_materialize_rows(const ot_plan *plan, const int64_t *row_idx, int64_t k, float *out,
@@ -296,7 +306,8 @@ OT_API int ot_materialize_rows_lrcost(const float *cost1, const float *cost2, co
  * with every T_ij computed by the same float path as ot_materialize_rows, so
  * that keeping T_ij >= thr leaves every massful row non-empty. Massless rows
  * (a_i == 0) keep nothing and take no part. block_rows (> 0, or 0 = all rows)
- * only sets how many rows one launch covers; it never changes a result.
+ * only sets how many rows one launch covers (raised to a few waves of the GPU
+ * when smaller); it never changes a result.
  *  thr_out: host float (+inf if every row is massless).
  *  row_counts: device int64 [n] or NULL: kept entries per row.
  *  nnz_out, n_massless_out, argmin_out: host int64 or NULL (argmin_out: the
@@ -346,7 +357,8 @@ OT_API int ot_sparsify_csr(const ot_plan *plan, int64_t block_rows, float thr, i
  * n or m above OT_NOALLOC_MAX_POINTS returns OT_ERR_UNSUPPORTED with a message.
  * The first call on a device looks up the scratch's device address (once per
  * device, with that device current); make that first call before any stream
- * capture. All calls on a device share the scratch and each call overwrites
+ * capture. The address is kept for the life of the process, so the device must
+ * not be reset (cudaDeviceReset) after that first call. All calls on a device share the scratch and each call overwrites
  * every slot it reads, so nothing carries over from the previous call; but
  * calls whose GPU work overlaps (e.g. from two host threads on two streams)
  * race on it. Synchronises `stream`. Calls no allocating routine.           */

@@ -169,7 +169,8 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
              check_every=16, use_graphs=True, eps_init=0.0, eps_decay=0.7, iters_per_stage=20,
              timing=False, col_splits=0, rows_per_thread=0, tensor_cores=True,
              device_loop=-1, block_sparse=False, sparse_block=0, sparse_verify=True,
-             sparse_delta=0.0, sparse_dense_frac=0.5, resid_history=None, stream=None) -> Plan:
+             sparse_delta=0.0, sparse_dense_frac=0.5, resid_history=None, sparse_mask_out=None,
+             stream=None) -> Plan:
     """Solves on the GPU; x [n,d], y [m,d], a [n], b [m] float32 CUDA tensors.
 
     block_sparse (d <= 3): block-sparse fine iterations ("FlashSinkhorn 2",
@@ -182,6 +183,8 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
 
     resid_history: optional float64 CUDA tensor; entry k - 1 receives the
     in-loop ||T1 - a||_1 after iteration k (NaN where none was measured).
+    sparse_mask_out: optional uint8 CUDA tensor of at least NB * MB bytes; the
+    block mask of the first fine update (at the starting potentials).
     """
     import torch
     x, y = _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y")
@@ -207,6 +210,10 @@ def sinkhorn(x, y, a, b, eps, scale="none", n_iters=100, tol=0.0, f=None, g=None
     opt.sparse_verify = int(bool(sparse_verify))
     opt.sparse_delta = float(sparse_delta)
     opt.sparse_dense_frac = float(sparse_dense_frac)
+    if sparse_mask_out is not None:
+        _dev(sparse_mask_out, torch.uint8, "sparse_mask_out")
+        opt.sparse_mask_out = sparse_mask_out.data_ptr()
+        opt.sparse_mask_len = sparse_mask_out.numel()
     if resid_history is not None:
         _dev(resid_history, torch.float64, "resid_history")
         opt.resid_history = resid_history.data_ptr()

@@ -47,7 +47,8 @@ class OtOptions(ctypes.Structure):
                 ("sparse_block", ctypes.c_int32), ("sparse_verify", ctypes.c_int32),
                 ("reserved2", ctypes.c_int32), ("sparse_delta", ctypes.c_double),
                 ("sparse_dense_frac", ctypes.c_double), ("resid_history", ctypes.c_void_p),
-                ("resid_history_len", ctypes.c_int64)]
+                ("resid_history_len", ctypes.c_int64), ("sparse_mask_out", ctypes.c_void_p),
+                ("sparse_mask_len", ctypes.c_int64)]
 
 
 class OtInfo(ctypes.Structure):

@@ -164,6 +164,7 @@ struct ot_plan {
     double *sp_tres = nullptr;
     SparseCtr *sc = nullptr;
     int64_t last_cand = 0, last_adm = 0, last_exact = 0;  // tiles of the last mask an iteration ran on
+    uint8_t *mask_out = nullptr;  // where the first mask goes (ot_options.sparse_mask_out), until then
     CUtensorMap tm_arow_x, tm_bcol_y, tm_arow_y, tm_bcol_x;
     cudaStream_t s_int = nullptr;
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
@@ -479,6 +480,12 @@ int sparse_setup(ot_plan *p, const ot_options &o, double tol, bool warm) {
                     (long long)nb, (long long)mb);
     if (nb > 65535ll * 32 || (mb + 63) / 64 > 65535)
         return fail(OT_ERR_UNSUPPORTED, "too many blocks for the screen's grid");
+    if (o.sparse_mask_out) {
+        if (o.sparse_mask_len < nb * mb)
+            return fail(OT_ERR_INVALID_ARG, "sparse_mask_len %lld < %lld block pairs",
+                        (long long)o.sparse_mask_len, (long long)(nb * mb));
+        p->mask_out = o.sparse_mask_out;
+    }
     p->sp_delta = o.sparse_delta > 0.0 ? o.sparse_delta : tol / (4.0 * (double)std::max(nb, mb));
     p->sp_frac = o.sparse_dense_frac;
     p->sp_verify = o.sparse_verify;
@@ -679,6 +686,10 @@ int sparse_iteration(ot_plan *p, int par, bool f_only, double eps) {
         OT_CU(mark_in(p, p->tm_hs));
         p->launches += 5;
     }
+    if (p->mask_out) {  // the solve's first mask (at the starting potentials), on request
+        OT_CU(cudaMemcpyAsync(p->mask_out, p->mask, (size_t)(nb * mb), cudaMemcpyDeviceToDevice, s));
+        p->mask_out = nullptr;
+    }
     if (!f_only) {
         OT_CU(launch_transpose_bytes(p->mask, nb, mb, p->mask_t, s));
         OT_CU(launch_row_ptr_scan(p->cnt_t, mb, p->ptr_t, p->sp_scan, s));
@@ -843,6 +854,8 @@ void ot_options_default(ot_options *opt) {
     opt->sparse_dense_frac = 0.5;
     opt->resid_history = nullptr;
     opt->resid_history_len = 0;
+    opt->sparse_mask_out = nullptr;
+    opt->sparse_mask_len = 0;
 }
 
 void ot_plan_destroy(ot_plan *plan) {
@@ -1057,6 +1070,8 @@ int validate(const float *x, const float *y, const float *a, const float *b, int
     if (o.check_every < 1) return fail(OT_ERR_INVALID_ARG, "check_every must be >= 1");
     if (o.resid_history_len < 0 || (o.resid_history_len > 0 && !o.resid_history))
         return fail(OT_ERR_INVALID_ARG, "resid_history_len must be >= 0, with a non-NULL resid_history");
+    if (o.sparse_mask_out && !o.block_sparse)
+        return fail(OT_ERR_INVALID_ARG, "sparse_mask_out needs block_sparse");
     if (o.col_splits < 0) return fail(OT_ERR_INVALID_ARG, "col_splits must be >= 0");
     if (o.rows_per_thread != 0 && o.rows_per_thread != 1 && o.rows_per_thread != 2 &&
         o.rows_per_thread != 4 && o.rows_per_thread != 8)
@@ -1565,6 +1580,16 @@ int ensure_rows_ws(ot_plan *p) {
     return OT_OK;
 }
 
+// Rows one launch of a row pass covers: the caller's block (0 = all rows), but
+// never fewer than four waves of the row-pass blocks on every SM -- a block of
+// rows changes no result (every row is reduced within one thread block), so a
+// small block would only leave SMs idle.
+int64_t launch_rows(const ot_plan *p, int64_t block_rows) {
+    const int64_t min_rows = rowpass_rows_per_block(p->d) * 2 * 4 * std::max(p->sm_count, 1);
+    if (block_rows == 0 || block_rows > p->n) return p->n;
+    return std::min(p->n, std::max(block_rows, min_rows));
+}
+
 int sync_read(ot_plan *p, cudaStream_t s) {
     OT_CU(cudaMemcpyAsync(&p->hs->s, p->ds, sizeof(DevScalars), cudaMemcpyDeviceToHost, s));
     OT_CU(cudaStreamSynchronize(s));
@@ -1673,7 +1698,7 @@ extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, flo
     int rc = plan_check(p);
     if (rc != OT_OK) return rc;
     if (block_rows < 0) return fail(OT_ERR_INVALID_ARG, "block_rows must be >= 0");
-    if (block_rows == 0 || block_rows > p->n) block_rows = p->n;
+    block_rows = launch_rows(p, block_rows);
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
     OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
@@ -1725,7 +1750,7 @@ extern "C" int ot_sparsify_csr(const ot_plan *cplan, int64_t block_rows, float t
     if (capacity > 0 && (!col_idx || !vals))
         return fail(OT_ERR_INVALID_ARG, "col_idx and vals must not be NULL when capacity > 0");
     if (std::isnan(thr)) return fail(OT_ERR_INVALID_ARG, "thr must not be NaN");
-    if (block_rows == 0 || block_rows > p->n) block_rows = p->n;
+    block_rows = launch_rows(p, block_rows);
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
     OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));

@@ -13,37 +13,36 @@
 //   A_i = kappa (f_i - c |x'_i|^2), B_j = kappa (g_j - c |y'_j|^2), P_i = 2 c kappa x'_i,
 // all in float64 (FlashSinkhorn 2, section D.3: accurate evaluation is done in
 // FP64). The sum is formed on t = kShift + e2 rather than on e2: kShift = 1.5 *
-// 2^29 + 190 keeps t in [2^29, 2^30), where a float64 step is 2^-23, so every
+// 2^29 + 126 keeps t in [2^29, 2^30), where a float64 step is 2^-23, so every
 // operation rounds e2 to a multiple of 2^-23 (at most 2^-24 off, ~2e-7 relative
 // in T after the five operations) and the low 32 bits of t are the integer
-// (190 + e2) * 2^23 -- the range reduction is then two integer operations: the
+// (126 + e2) * 2^23 -- the range reduction is then two integer operations: the
 // fraction of e2 goes into the mantissa of a float in [1, 2), whose MUFU ex2
 // (relative error ~2^-22) is scaled by 2^floor(e2) through the exponent field.
-// e2 is clamped to [-189, 64] first (two float64 min/max): below, T rounds to 0
-// (a massless side, potential -inf, lands there); at 64 and above T is +inf
-// (the float result of an entry of 2^64 or more). The scaled value is formed
-// 2^64 too large and multiplied by 2^-64 at the end, so entries below 2^-126
-// round correctly into the subnormal range. Per entry: d + 1 float64 FMAs/adds,
-// two float64 min/max, two integer operations, one ex2 and one float multiply.
-// The row passes accumulate each row's terms 8 at a time in float32 and those
-// partial sums in float64 (maxima and counts exactly).
+// e2 is clamped to [-200, 128] first (two float64 min/max; a massless side,
+// potential -inf, lands on the floor): from 128 on T is +inf (the exponent field
+// saturates exactly there), and below -126 T is returned as 0 (entries under
+// 2^-126 = 1.2e-38, the smallest normal float, are flushed). Per entry: d + 1
+// float64 FMAs/adds, two float64 min/max, three integer operations and a select,
+// one ex2. The row passes accumulate each row's terms 8 at a time in float32
+// and those partial sums in float64 (maxima and counts exactly).
 #include "runtime.h"
 
 namespace ot {
 
-constexpr double kShift = 805306368.0 + 190.0;  // 1.5 * 2^29 + 190
-constexpr double kShiftLo = kShift - 189.0;     // e2 >= -189
-constexpr double kShiftHi = kShift + 64.0;      // e2 <= 64
+constexpr double kShift = 805306368.0 + 126.0;  // 1.5 * 2^29 + 126
+constexpr double kShiftLo = kShift - 200.0;     // e2 >= -200 (then flushed to 0)
+constexpr double kShiftHi = kShift + 128.0;     // e2 <= 128 (+inf)
 
 // T = 2^e2 from t = kShift + e2 (see above).
 __device__ __forceinline__ float exp2_shifted(double t) {
     t = fmin(fmax(t, kShiftLo), kShiftHi);
-    const unsigned q = (unsigned)__double2loint(t);          // (190 + e2) * 2^23
+    const unsigned q = (unsigned)__double2loint(t);          // (126 + e2) * 2^23 (mod 2^32)
     const unsigned mant = (q & 0x7FFFFFu) | 0x3F800000u;      // 1 + frac(e2), in [1, 2)
     const float p = ex2_approx(__uint_as_float(mant));         // 2^(1 + frac(e2)), in [2, 4]
-    // exponent field + floor(e2) + 63: q - mant = (floor(e2) + 63) * 2^23
+    // exponent field + floor(e2) - 1: q - mant = (floor(e2) - 1) * 2^23
     const float v = __uint_as_float(__float_as_uint(p) + q - mant);
-    return v * 5.42101086242752217e-20f;                       // * 2^-64
+    return (int)q < 0 ? 0.0f : v;                               // e2 < -126
 }
 
 // the one float path for a plan entry: row data (A' = A + kShift, P[d]),
@@ -772,8 +771,10 @@ cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+int64_t rowpass_rows_per_block(int d) { return d <= 3 ? kRpRows : kRgRows; }
+
 int64_t rowpass_blocks(int64_t rows, int d) {
-    const int per = d <= 3 ? kRpRows : kRgRows;
+    const int64_t per = rowpass_rows_per_block(d);
     return (rows + per - 1) / per;
 }
 

@@ -207,6 +207,7 @@ cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s);
 cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s);
 // residual partials one pass over `rows` rows writes (blocks of the pass)
 int64_t rowpass_blocks(int64_t rows, int d);
+int64_t rowpass_rows_per_block(int d);
 cudaError_t launch_min_row_reduce(const float *rowmax, const float *w, int64_t n, float *thr,
                                   int64_t *argmin, int64_t *n_massless, cudaStream_t s);
 cudaError_t launch_sum_i64(const int64_t *v, int64_t cnt, int64_t *out, cudaStream_t s);

@@ -68,7 +68,7 @@ def assert_entries(T, T_ref, tol=ROW_TOL):
     return worst
 
 
-def assert_min_row(got, ref, T_ref_rows=None, rows=None, tol=ROW_TOL):
+def assert_min_row(got, ref, tol=ROW_TOL):
     assert got["n_massless"] == ref["n_massless"]
     if ref["argmin"] < 0:
         assert got["argmin"] == -1 and np.isinf(got["thr"])

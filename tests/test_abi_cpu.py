@@ -49,7 +49,7 @@ def test_version_and_defaults(B):
 
 
 def test_struct_sizes_match_header_layout(B):
-    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4 + 4 * 4 + 2 * 8 + 2 * 8
+    assert ctypes.sizeof(B.OtOptions) == 4 * 4 + 3 * 8 + 6 * 4 + 4 * 4 + 2 * 8 + 4 * 8
     assert ctypes.sizeof(B.OtInfo) == 4 * 4 + 3 * 8 + 4 * 8 + 8 + 6 * 8 + 8 + 3 * 8
 
 
@@ -142,6 +142,10 @@ def test_residual_history_needs_an_array(B):
     o.resid_history_len = 5  # no array
     assert _call(B, opt=o)[0] == B.OT_ERR_INVALID_ARG
     o.resid_history_len = -1
+    assert _call(B, opt=o)[0] == B.OT_ERR_INVALID_ARG
+    o = B.ot_options_default()
+    o.sparse_mask_out = FAKE  # a mask needs block-sparse iterations
+    o.sparse_mask_len = 100
     assert _call(B, opt=o)[0] == B.OT_ERR_INVALID_ARG
 
 

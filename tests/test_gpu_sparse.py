@@ -281,3 +281,41 @@ def test_scaled_costs_and_massless_columns(ot, orc, scale, B, verify):
     H.assert_potentials(plan.g.double().cpu().numpy(), g, maxc, what="g")
     assert plan.info.sparse_iterations == 6 and 0 < st[3] < plan.info.tiles_total
     plan.close()
+
+
+@pytest.mark.parametrize("d,B,verify,n,m", [
+    (3, 128, True, 5000, 4100), (3, 256, True, 5000, 4100), (2, 128, True, 3000, 3333),
+    (1, 128, True, 2000, 1500), (3, 128, False, 4000, 3000),
+])
+def test_first_mask_matches_the_oracle_tile_by_tile(ot, orc, d, B, verify, n, m):
+    """The block mask built at given potentials (the oracle's after 6 block-sparse
+    iterations, rounded to float32) against the oracle's mask at the same
+    potentials, tile by tile: every tile whose oracle margin lies outside BAND of
+    the threshold (the screen's, and the exact mass's where it was evaluated)
+    takes the same decision ("FlashSinkhorn 2", sections 3.2 and A.3)."""
+    import torch
+    w = _clusters(20 + d, n, m, d)
+    delta = 1e-6
+    f6, g6, _, _, _ = orc.sinkhorn_sparse(w.x, w.y, w.a, w.b, 1.0, w.eps, 6, B=B, delta=delta,
+                                          verify=verify, dense_frac=1.0)
+    f0, g0 = H.f32(f6), H.f32(g6)
+    NB, MB = -(-n // B), -(-m // B)
+    mask = torch.full((NB * MB,), 7, dtype=torch.uint8, device="cuda")
+    plan = _gpu(ot, w, 1, f0=f0, g0=g0, sparse_block=B, sparse_verify=verify, sparse_delta=delta,
+                sparse_dense_frac=1.0, sparse_mask_out=mask)
+    plan.close()
+    got = mask.cpu().numpy().reshape(NB, MB)
+    assert set(np.unique(got)) <= {0, 1}
+    lo, hi = orc.joint_box(w.x, w.y)
+    px, py = orc.morton_order(w.x, lo, hi), orc.morton_order(w.y, lo, hi)
+    o = orc.block_mask(w.x[px], w.y[py], w.a[px].astype(np.float64), w.b[py].astype(np.float64),
+                       f0[px], g0[py], 1.0, w.eps, B, delta, verify)
+    ref = o["adm"] if verify else o["cand"]
+    sm, mm = o["screen_margin"], o["mass_margin"]
+    clear = np.abs(sm) > BAND
+    if verify:
+        clear &= ~np.isfinite(mm) | (np.abs(mm) > BAND)
+    assert clear.mean() > 0.9, clear.mean()
+    bad = np.argwhere(clear & (got.astype(bool) != ref))
+    assert bad.size == 0, (bad[:5], int(got.sum()), int(ref.sum()))
+    assert 0 < int(ref.sum()) < NB * MB  # neither empty nor full

@@ -47,10 +47,13 @@ def test_noalloc_residual_matches_plan_residual_twice_in_a_row():
         pytest.skip("needs a GPU")
     import log_domain_sinkhorn_online_b200 as pkg
     from log_domain_sinkhorn_online_b200 import _binding as B
-    # two calls in a row on different problems: the second must not see the
-    # first one's leftovers in the shared scratch
+    # calls in a row on different problems: none may see the previous one's
+    # leftovers in the shared scratch; the fourth fills the scratch exactly
+    # (OT_NOALLOC_MAX_POINTS rows: every partial slot, the results right after),
+    # the fifth runs the generic kernel at the largest d
     for w in (_problem(1, 3001, 2777, 3, "mean"), _problem(2, 1500, 4100, 2, "none"),
-              _problem(3, 700, 650, 17, "max_cost")):
+              _problem(3, 700, 650, 17, "max_cost"), _problem(4, B.OT_NOALLOC_MAX_POINTS, 64, 3, "mean"),
+              _problem(5, 900, 800, 64, "none")):
         st, got, want = _via_plan_and_noalloc(pkg, B, w)
         assert st == 0
         assert abs(got[0] - want[0]) <= H.RES_TOL, (got, want)
