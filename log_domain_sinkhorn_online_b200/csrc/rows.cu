@@ -19,30 +19,32 @@
 // (126 + e2) * 2^23 -- the range reduction is then two integer operations: the
 // fraction of e2 goes into the mantissa of a float in [1, 2), whose MUFU ex2
 // (relative error ~2^-22) is scaled by 2^floor(e2) through the exponent field.
-// e2 is clamped to [-200, 128] first (two float64 min/max; a massless side,
-// potential -inf, lands on the floor): from 128 on T is +inf (the exponent field
-// saturates exactly there), and below -126 T is returned as 0 (entries under
-// 2^-126 = 1.2e-38, the smallest normal float, are flushed). Per entry: d + 1
-// float64 FMAs/adds, two float64 min/max, three integer operations and a select,
-// one ex2. The row passes accumulate each row's terms 8 at a time in float32
-// and those partial sums in float64 (maxima and counts exactly).
+// The range takes two float64 compares and an integer min: for e2 in
+// [-126, 386) t lies in [kBase, kBase + 512) (kBase = 1.5 * 2^29), where the low
+// word is exact; the integer min caps it at e2 = 128, where the exponent field
+// saturates to +inf exactly; below -126 T is returned as 0 (entries under
+// 2^-126 = 1.2e-38, the smallest normal float, are flushed; a massless side,
+// potential -inf, lands there) and from 386 on as +inf. Per entry: d + 1 float64
+// FMAs/adds, two float64 compares, three integer operations, two selects, one
+// ex2. The row passes accumulate each row's terms 8 at a time in float32 and
+// those partial sums in float64 (maxima and counts exactly).
 #include "runtime.h"
 
 namespace ot {
 
 constexpr double kShift = 805306368.0 + 126.0;  // 1.5 * 2^29 + 126
-constexpr double kShiftLo = kShift - 200.0;     // e2 >= -200 (then flushed to 0)
-constexpr double kShiftHi = kShift + 128.0;     // e2 <= 128 (+inf)
+constexpr double kShiftLo = kShift - 126.0;     // e2 >= -126 (else 0)
+constexpr double kShiftHi = kShift + 386.0;     // e2 < 386 (else +inf)
 
 // T = 2^e2 from t = kShift + e2 (see above).
 __device__ __forceinline__ float exp2_shifted(double t) {
-    t = fmin(fmax(t, kShiftLo), kShiftHi);
-    const unsigned q = (unsigned)__double2loint(t);          // (126 + e2) * 2^23 (mod 2^32)
-    const unsigned mant = (q & 0x7FFFFFu) | 0x3F800000u;      // 1 + frac(e2), in [1, 2)
-    const float p = ex2_approx(__uint_as_float(mant));         // 2^(1 + frac(e2)), in [2, 4]
+    const unsigned q = min((unsigned)__double2loint(t), 254u << 23);  // (126 + e2) * 2^23, capped
+    const unsigned mant = (q & 0x7FFFFFu) | 0x3F800000u;              // 1 + frac(e2), in [1, 2)
+    const float p = ex2_approx(__uint_as_float(mant));                 // 2^(1 + frac(e2)), in [2, 4]
     // exponent field + floor(e2) - 1: q - mant = (floor(e2) - 1) * 2^23
     const float v = __uint_as_float(__float_as_uint(p) + q - mant);
-    return (int)q < 0 ? 0.0f : v;                               // e2 < -126
+    const float r = t >= kShiftLo ? v : 0.0f;
+    return t < kShiftHi ? r : INFINITY;
 }
 
 // the one float path for a plan entry: row data (A' = A + kShift, P[d]),
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
         for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int q = 0; q < DS; ++q)
-                cd[u][q] = u < ncol ? M.dcol[(j0 + u) * DS + q] : -INFINITY;
+                cd[u][q] = u < ncol ? M.dcol[(j0 + u) * DS + q] : (q == DS - 1 ? -INFINITY : 0.0);
     }
     const int64_t rb0 = (int64_t)blockIdx.y * kMtRowsPerBlock;
     const int64_t rb1 = min(rb0 + kMtRowsPerBlock, M.k);
@@ -139,21 +141,22 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
         __syncthreads();
         if (ncol == 0) continue;
         const int nr = (int)min((int64_t)kMtStage, rb1 - s0);
+        const bool full = M.vec && ncol == 4;
+        float *dst = M.out + s0 * M.m + j0;
 #pragma unroll 2
-        for (int rr = 0; rr < nr; ++rr) {
-            const bool valid = sValid[rr] != 0;
+        for (int rr = 0; rr < nr; ++rr, dst += M.m) {
+            if (!sValid[rr]) continue;  // the same for every thread of the block
             float t[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
+                // a column past m carries B = -inf and gives 0, never stored
                 if (D > 0)
-                    t[u] = u < ncol ? plan_entry<D>(sA[rr], sP[rr], cd[u], d) : 0.0f;
+                    t[u] = plan_entry<D>(sA[rr], sP[rr], cd[u], d);
                 else
                     t[u] = u < ncol ? plan_entry<0>(sA[rr], sP[rr], M.dcol + (j0 + u) * (d + 1), d)
                                     : 0.0f;
             }
-            float *dst = M.out + (s0 + rr) * M.m + j0;
-            if (!valid) continue;
-            if (M.vec && ncol == 4) {
+            if (full) {
                 __stcs(reinterpret_cast<float4 *>(dst), make_float4(t[0], t[1], t[2], t[3]));
             } else {
                 for (int u = 0; u < ncol; ++u) __stcs(dst + u, t[u]);
@@ -170,21 +173,25 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
 // "Rows" may be either cloud: the column residual runs the same pass with the
 // roles of (x, f, a) and (y, g, b) swapped, since T is symmetric in them.
 //
-// d <= 3: a block of 8 warps owns 64 rows, 8 per warp, whose float64 data sit
+// d <= 3: a block of 8 warps owns 32 rows, 4 per warp, whose float64 data sit
 // in registers; the columns' float64 records (y'[d], B) stream through shared
 // memory 256 at a time (the next chunk prefetched into registers), so a column
-// is read from L2 once per 64 rows and from shared memory once per 8 entries.
+// is read from L2 once per 32 rows and from shared memory once per 4 entries.
+// 3 blocks per SM (85 registers): the entry is a chain of dependent float64
+// operations, and more resident warps hide it better than more rows per warp
+// (measured at n = m = 1e5: 4 rows x 3 blocks 32 % of the MUFU rate for the
+// residual pass, 8 rows x 2 blocks 30 %).
 // Lane l takes columns l, l + 32, ... of each chunk for all 8 rows of its warp,
 // so every row's reduction stays in one warp, in a fixed lane order
 // (deterministic). Sums: the 8 terms of a row in one chunk add up in float32,
 // those partial sums in float64.
 enum { OP_MAX = 0, OP_COUNT = 1, OP_SUM = 2 };
-constexpr int kRpThreads = 256, kRpWarps = kRpThreads / 32, kRpR = 8, kRpChunk = 256;
-constexpr int kRpRows = kRpWarps * kRpR;  // rows per block, d <= 3
+constexpr int kRpThreads = 256, kRpWarps = kRpThreads / 32, kRpR = 4, kRpChunk = 256;
+constexpr int kRpRows = kRpWarps * kRpR;  // rows per block, d <= 3 (32)
 constexpr int kRgRows = 8;                // rows per block, generic d
 
 template <int D, int OP>
-__global__ void __launch_bounds__(kRpThreads, 2) rowpass_kernel(RowPassArgs R) {
+__global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
     constexpr int DS = D + 1;                 // doubles per column record
     constexpr int DP = D == 1 ? 2 : 4;        // padded stride in shared memory
     constexpr int PER = (kRpChunk * DS + kRpThreads - 1) / kRpThreads;  // prefetched doubles
