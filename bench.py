@@ -17,10 +17,10 @@ that takes HOST arrays (pinned here): x, y, a, b, f, g copied in and f, g copied
 out inside the timed region.
 
 Side objects, timed once after the steps on the same problem: `scale_pass` (the
-max_cost pass), `rows` (the row kernels at the solved state: one 1024-row
-materializer block of 1024 x 2e6 entries, the float64-assembled marginal
-residual and the exact min_row threshold with counts, both over all 4e12
-entries) and `block_sparse` (block-sparse fine iterations against dense ones at
+max_cost pass), `rows` (the row kernels at the solved state: one 4096-row
+materializer block of the workload's 65,536 rows, 4096 x 2e6 entries = 32.8 GB,
+the float64-assembled marginal residual and the exact min_row threshold with
+counts, both over all 4e12 entries) and `block_sparse` (block-sparse fine iterations against dense ones at
 n = m = 2^18); --no-side skips them.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload w5]
@@ -89,7 +89,7 @@ def _args():
     ap.add_argument("--sparse-block", type=int, default=0, choices=[0, 128, 256],
                     help="--sparse: block size B (0 = the library's choice)")
     ap.add_argument("--rows", action="store_true",
-                    help="instead of the step: the row kernels (a 1024-row materializer block, the "
+                    help="instead of the step: the row kernels (one materializer block of the workload, the "
                          "marginal residual, min_row) at the state after 5 iterations of the workload "
                          "(or its --n/--m replica); prints its own JSON line")
     ap.add_argument("--no-side", action="store_true",
@@ -518,7 +518,7 @@ def _side(ot, step, w, stream, peak_ex2, hbm_gbs):
     # a8-a10 at the solved state, through one plan
     plan = ot.sinkhorn(step.x, step.y, step.a, step.b, eps=w.eps, scale=step.scale, n_iters=0,
                        warm_start=True, f=step.f.clone(), g=step.g.clone())
-    k = 1024
+    k = w.block_rows or 1024  # one block of the workload's row materialization
     rows = torch.from_numpy(np.ascontiguousarray(w.rows[:k] if w.rows is not None
                                                  else np.arange(min(k, w.n), dtype=np.int64))).to(step.dev)
     buf = torch.empty((rows.numel(), w.m), dtype=torch.float32, device=step.dev)
@@ -730,7 +730,8 @@ def run_ours(args):
 
 
 def run_rows(args):
-    """The row kernels alone on a solved state of the workload."""
+    """The row kernels alone on a solved state of the workload (one materializer
+    block of the workload's block size)."""
     import torch
     import log_domain_sinkhorn_online_b200 as ot
     dev = torch.device("cuda", 0)
