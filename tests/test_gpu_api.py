@@ -151,3 +151,25 @@ def test_plan_destroyed_from_another_thread(ot):
         np.testing.assert_array_equal(q.f.cpu().numpy(), fr)
         q.close()
     torch.cuda.synchronize()
+
+
+def test_residual_history_with_tol_and_block_sparse(ot):
+    import torch
+    w = _w(2000, 1800)
+    x, y, a, b = H.to_dev(w)
+    # a tolerance met inside the run: the history stops at the returned state
+    hist = torch.empty(400, dtype=torch.float64, device="cuda")
+    p = ot.sinkhorn(x, y, a, b, eps=0.05, scale=w.scale, n_iters=400, tol=1e-4, resid_history=hist)
+    h = hist.cpu().numpy()
+    k = p.info.iterations
+    assert p.info.converged == 1 and 1 <= k < 400
+    assert h[k - 1] == p.info.residual and h[k - 1] <= 1e-4 and h[k - 2] > 1e-4
+    assert np.isnan(h[k + 1:]).all()
+    p.close()
+    # block-sparse iterations record the admitted plan's residual after every iteration
+    hist = torch.empty(6, dtype=torch.float64, device="cuda")
+    p = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=6, block_sparse=True, sparse_delta=1e-7,
+                    sparse_dense_frac=1.0, resid_history=hist)
+    h = hist.cpu().numpy()
+    assert np.isfinite(h).all() and h[5] == p.info.residual
+    p.close()

@@ -142,3 +142,27 @@ def test_shard_plan_argument_checks(ot):
     with pytest.raises(B.OTError):
         B.ot_shard_half_step(plan, 2, x.data_ptr(), a.data_ptr(), a.data_ptr(), s)
     B.ot_plan_destroy(plan)
+
+
+def test_split_with_empty_ranges_and_massless_rows(ot):
+    """Four ranks on 1500 x 1300 points with 1024-row ranges: two ranks own no rows;
+    a few massless rows and columns (-inf potentials) pass through unchanged."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w2(n=1500, m=1300)
+    a = w.a.copy()
+    b = w.b.copy()
+    a[::97] = 0.0
+    b[5::131] = 0.0
+    a = (a / a.sum()).astype(np.float32)
+    b = (b / b.sum()).astype(np.float32)
+    x, y = (torch.from_numpy(np.ascontiguousarray(v)).cuda() for v in (w.x, w.y))
+    at, bt = torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()
+    opts = dict(col_splits=3, rows_per_thread=2)
+    p = ot.sinkhorn(x, y, at, bt, eps=w.eps, scale=w.scale, n_iters=7, device_loop=0, **opts)
+    fr, gr = p.f.cpu().numpy(), p.g.cpu().numpy()
+    p.close()
+    f, g, _, _ = _emulated_split(ot, x, y, at, bt, w.eps, w.scale, 4, 7, 1024, **opts)
+    assert np.isneginf(f[::97]).all() and np.isneginf(g[5::131]).all()
+    np.testing.assert_array_equal(f, fr)
+    np.testing.assert_array_equal(g, gr)
