@@ -3,9 +3,9 @@
 Every row call (materializer, residual, min_row, sparsify) evaluates
 T_ij = exp((f_i + g_j - C_ij)/eps) through one device function (moscot PR #846,
 "Behavioural changes": one float path for threshold and values). Its range
-reduction keeps the base-2 exponent e2 on a float64 grid of 2^-23 and clamps it
-to [-200, 128]; these tests pin what that means for a caller, against exp()
-evaluated in float64 on the host:
+reduction keeps the base-2 exponent e2 on a float64 grid of 2^-23, returns 0
+below e2 = -126 and saturates to +inf from e2 = 128 on; these tests pin what that
+means for a caller, against exp() evaluated in float64 on the host:
  - normal results (2^-126 <= T < 2^128) within 1e-6 relative (the bar of the
    parity tests is 1e-5);
  - T = 0 below 2^-126 (entries under the smallest normal float are flushed) and
