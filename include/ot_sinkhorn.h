@@ -41,7 +41,7 @@
 extern "C" {
 #endif
 
-#define OT_ABI_VERSION 3
+#define OT_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define OT_API __attribute__((visibility("default")))
@@ -420,6 +420,39 @@ OT_API int ot_shard_plan_create(const float *x, const float *y, const float *a, 
  * range returns OT_ERR_NONFINITE. */
 OT_API int ot_shard_half_step(ot_plan *plan, int32_t side, const float *other, const float *cur,
                               float *out, double *resid, void *stream);
+
+/* Row calls over a range of rows, for the same split (section 5 of FlashSinkhorn
+ * 2 again): the rows of the plan are independent, so each rank reduces its own
+ * and one all-reduce combines them. They take a plan of ot_sinkhorn_pointcloud
+ * (on every rank, with the gathered potentials: n_iters = 0 with warm_start),
+ * use the same kernels and float path as the whole-plan calls, and with the
+ * full range give exactly their values. A range outside the plan returns
+ * OT_ERR_INVALID_ARG; block_rows as in ot_sparsify_min_row. All synchronise
+ * `stream`.
+ *
+ * ot_marginal_residual_range: *row_part = sum over i in [row_lo, row_hi) of
+ *     |sum_j T_ij - a_i|, *col_part = sum over j in [col_lo, col_hi) of
+ *     |sum_i T_ij - b_j| (host doubles, NULL ok); the sums over ranks of the
+ *     parts are ot_marginal_residual's two values, in another summation order.
+ * ot_min_row_range: pass A of ot_sparsify_min_row over rows [row_lo, row_hi)
+ *     (moscot PR #846, "Behavioural changes"): *thr_out = min over the range's
+ *     rows with a_i > 0 of max_j T_ij (+inf if none), *argmin_out = the global
+ *     index of the row attaining it (smallest on ties, -1 if none),
+ *     *n_massless_out = massless rows in the range. The min over ranks of
+ *     thr_out is ot_sparsify_min_row's thr (and the smallest argmin among the
+ *     ranks attaining it its argmin).
+ * ot_kept_counts_range: pass B at a given thr (not NaN): row_counts (device
+ *     int64 [row_hi - row_lo], NULL ok) = #{j : T_ij >= thr} per row of the
+ *     range, 0 for a massless row; *nnz_out = their sum. */
+OT_API int ot_marginal_residual_range(const ot_plan *plan, int64_t row_lo, int64_t row_hi,
+                                      int64_t col_lo, int64_t col_hi, double *row_part,
+                                      double *col_part, void *stream);
+OT_API int ot_min_row_range(const ot_plan *plan, int64_t row_lo, int64_t row_hi, int64_t block_rows,
+                            float *thr_out, int64_t *argmin_out, int64_t *n_massless_out,
+                            void *stream);
+OT_API int ot_kept_counts_range(const ot_plan *plan, int64_t row_lo, int64_t row_hi,
+                                int64_t block_rows, float thr, int64_t *row_counts, int64_t *nnz_out,
+                                void *stream);
 
 /* Plans take their device workspace, pinned read-back buffer and internal
  * stream from a per-device cache and return them there when destroyed, so

@@ -32,7 +32,8 @@ EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sink
             "ot_sparsify_min_row", "ot_plan_destroy", "ot_marginal_residual_noalloc", "ot_trim_cache",
             "ot_sparsify_csr", "ot_materialize_rows_lowrank", "ot_materialize_rows_lrcost",
             "ot_testing_fail_device_allocs", "ot_testing_wait_fault", "ot_max_sqdist",
-            "ot_shard_plan_create", "ot_shard_half_step")
+            "ot_shard_plan_create", "ot_shard_half_step", "ot_marginal_residual_range",
+            "ot_min_row_range", "ot_kept_counts_range")
 OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
@@ -122,6 +123,14 @@ def lib() -> ctypes.CDLL:
             L.ot_marginal_residual_noalloc.argtypes = [P, P, P, P, P, P, I64, I64, I32, D, D,
                                                        ctypes.POINTER(D), ctypes.POINTER(D), P]
             L.ot_marginal_residual_noalloc.restype = ctypes.c_int
+            L.ot_marginal_residual_range.argtypes = [P, I64, I64, I64, I64, ctypes.POINTER(D),
+                                                     ctypes.POINTER(D), P]
+            L.ot_marginal_residual_range.restype = ctypes.c_int
+            L.ot_min_row_range.argtypes = [P, I64, I64, I64, ctypes.POINTER(ctypes.c_float),
+                                           ctypes.POINTER(I64), ctypes.POINTER(I64), P]
+            L.ot_min_row_range.restype = ctypes.c_int
+            L.ot_kept_counts_range.argtypes = [P, I64, I64, I64, ctypes.c_float, P, ctypes.POINTER(I64), P]
+            L.ot_kept_counts_range.restype = ctypes.c_int
             L.ot_trim_cache.argtypes = []
             L.ot_trim_cache.restype = None
             L.ot_plan_destroy.argtypes = [P]
@@ -252,6 +261,31 @@ def ot_sparsify_min_row(plan, block_rows, row_counts, stream):
                                           ctypes.byref(nnz), ctypes.byref(nm), ctypes.byref(arg),
                                           stream))
     return st, thr.value, nnz.value, nm.value, arg.value
+
+
+def ot_marginal_residual_range(plan, row_lo, row_hi, col_lo, col_hi, stream):
+    """Returns (row_part, col_part) over rows [row_lo, row_hi) and columns [col_lo, col_hi)."""
+    r, c = ctypes.c_double(), ctypes.c_double()
+    _check(lib().ot_marginal_residual_range(plan, row_lo, row_hi, col_lo, col_hi, ctypes.byref(r),
+                                            ctypes.byref(c), stream))
+    return r.value, c.value
+
+
+def ot_min_row_range(plan, row_lo, row_hi, block_rows, stream):
+    """Returns (thr, argmin, n_massless) of rows [row_lo, row_hi)."""
+    thr = ctypes.c_float()
+    arg, nm = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ot_min_row_range(plan, row_lo, row_hi, block_rows, ctypes.byref(thr), ctypes.byref(arg),
+                                  ctypes.byref(nm), stream))
+    return thr.value, arg.value, nm.value
+
+
+def ot_kept_counts_range(plan, row_lo, row_hi, block_rows, thr, row_counts, stream):
+    """Returns nnz of rows [row_lo, row_hi) at thr; row_counts: device int64 [row_hi - row_lo] or 0."""
+    nnz = ctypes.c_int64()
+    _check(lib().ot_kept_counts_range(plan, row_lo, row_hi, block_rows, thr, row_counts or None,
+                                      ctypes.byref(nnz), stream))
+    return nnz.value
 
 
 def ot_marginal_residual_noalloc(x, y, a, b, f, g, n, m, d, eps, inv_scale_cost, stream):

@@ -1596,6 +1596,79 @@ int sync_read(ot_plan *p, cudaStream_t s) {
     return OT_OK;
 }
 
+RowPassArgs row_args(const ot_plan *p) {
+    RowPassArgs R{};
+    R.pts = p->x; R.pot = p->f; R.w = p->a; R.dcol = p->dcol; R.o = p->o; R.prm = p->prm;
+    R.cols = p->m; R.d = p->d; R.rowmax = p->rowmax; R.counts = p->counts; R.part = p->rpart;
+    return R;
+}
+
+// min_row pass A over rows [lo, hi): max_j T_ij of every row, then the
+// minimum over the massful ones (thr, its smallest global row index, -1 if
+// none) and the number of massless rows. The column table must be current.
+int min_row_pass(ot_plan *p, int64_t lo, int64_t hi, int64_t block_rows, cudaStream_t s,
+                 float *thr, int64_t *argmin, int64_t *n_massless) {
+    RowPassArgs R = row_args(p);
+    for (int64_t r0 = lo; r0 < hi; r0 += block_rows) {
+        R.row_begin = r0;
+        R.row_end = std::min(hi, r0 + block_rows);
+        OT_CU(launch_rowpass(0, R, s));
+    }
+    OT_CU(launch_min_row_reduce(p->rowmax + lo, p->a + lo, hi - lo, &p->ds->thr, &p->ds->argmin,
+                                &p->ds->n_massless, s));
+    int rc = sync_read(p, s);
+    if (rc != OT_OK) return rc;
+    *thr = p->hs->s.thr;
+    *argmin = p->hs->s.argmin >= 0 ? p->hs->s.argmin + lo : -1;
+    *n_massless = p->hs->s.n_massless;
+    return OT_OK;
+}
+
+// min_row pass B over rows [lo, hi): counts[i] = #{j : T_ij >= thr} (0 for a
+// massless row), indexed by the global row, and their sum.
+int count_pass(ot_plan *p, int64_t lo, int64_t hi, int64_t block_rows, float thr, int64_t *counts,
+               cudaStream_t s, int64_t *nnz) {
+    RowPassArgs R = row_args(p);
+    R.thr = thr;
+    R.counts = counts;
+    for (int64_t r0 = lo; r0 < hi; r0 += block_rows) {
+        R.row_begin = r0;
+        R.row_end = std::min(hi, r0 + block_rows);
+        OT_CU(launch_rowpass(1, R, s));
+    }
+    OT_CU(launch_sum_i64(counts + lo, hi - lo, &p->ds->nnz, s));
+    int rc = sync_read(p, s);
+    if (rc != OT_OK) return rc;
+    *nnz = p->hs->s.nnz;
+    return OT_OK;
+}
+
+// One side of the marginal residual over rows [lo, hi) of that side:
+// sum_i |sum_j T_ij - w_i| (side 0: rows of x against a; side 1: rows of y
+// against b, the pass with the clouds' roles swapped). Rebuilds the column
+// table of the other side; the result lands in p->ds->r_sum[side].
+int residual_pass(ot_plan *p, int side, int64_t lo, int64_t hi, cudaStream_t s) {
+    RowPassArgs R = row_args(p);
+    if (side == 0) {
+        OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    } else {
+        OT_CU(launch_dcol(p->x, p->f, p->n, p->d, p->o, p->prm, p->dcol, s));
+        R.pts = p->y; R.pot = p->g; R.w = p->b; R.cols = p->n;
+    }
+    R.row_begin = lo;
+    R.row_end = hi;
+    OT_CU(launch_rowpass(2, R, s));
+    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(hi - lo, p->d), &p->ds->r_sum[side], s));
+    return OT_OK;
+}
+
+int range_check(int64_t lo, int64_t hi, int64_t count, const char *what) {
+    if (lo < 0 || hi < lo || hi > count)
+        return fail(OT_ERR_INVALID_ARG, "%s range [%lld, %lld) is not inside [0, %lld)", what,
+                    (long long)lo, (long long)hi, (long long)count);
+    return OT_OK;
+}
+
 }  // namespace
 
 extern "C" int ot_materialize_rows(const ot_plan *cplan, const int64_t *row_idx, int64_t k,
@@ -1702,38 +1775,66 @@ extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, flo
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
     OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
-    RowPassArgs R{};
-    R.pts = p->x; R.pot = p->f; R.w = p->a; R.dcol = p->dcol; R.o = p->o; R.prm = p->prm;
-    R.cols = p->m; R.d = p->d; R.rowmax = p->rowmax;
-    R.counts = row_counts ? row_counts : p->counts;
-    // pass A: max_j T_ij of every row, block by block
-    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
-        R.row_begin = r0;
-        R.row_end = std::min(p->n, r0 + block_rows);
-        OT_CU(launch_rowpass(0, R, s));
-    }
-    OT_CU(launch_min_row_reduce(p->rowmax, p->a, p->n, &p->ds->thr, &p->ds->argmin,
-                                &p->ds->n_massless, s));
-    if ((rc = sync_read(p, s)) != OT_OK) return rc;
-    const float thr = p->hs->s.thr;
-    const int64_t argmin = p->hs->s.argmin, nm = p->hs->s.n_massless;
-    // pass B: entries kept per row (T_ij >= thr, same float path)
-    R.thr = thr;
-    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
-        R.row_begin = r0;
-        R.row_end = std::min(p->n, r0 + block_rows);
-        OT_CU(launch_rowpass(1, R, s));
-    }
-    OT_CU(launch_sum_i64(R.counts, p->n, &p->ds->nnz, s));
-    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    float thr = 0.0f;
+    int64_t argmin = -1, nm = 0, nnz = 0;
+    if ((rc = min_row_pass(p, 0, p->n, block_rows, s, &thr, &argmin, &nm)) != OT_OK) return rc;
+    rc = count_pass(p, 0, p->n, block_rows, thr, row_counts ? row_counts : p->counts, s, &nnz);
+    if (rc != OT_OK) return rc;
     if (thr_out) *thr_out = thr;
-    if (nnz_out) *nnz_out = p->hs->s.nnz;
+    if (nnz_out) *nnz_out = nnz;
     if (n_massless_out) *n_massless_out = nm;
     if (argmin_out) *argmin_out = argmin;
     if (nm > 0) {
         fail(OT_WARN_MASSLESS_ROWS, "%lld rows carry no mass", (long long)nm);
         return OT_WARN_MASSLESS_ROWS;
     }
+    return OT_OK;
+}
+
+extern "C" int ot_min_row_range(const ot_plan *cplan, int64_t row_lo, int64_t row_hi,
+                                int64_t block_rows, float *thr_out, int64_t *argmin_out,
+                                int64_t *n_massless_out, void *stream) {
+    NvtxRange nvtx_range("ot_min_row_range");
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if ((rc = range_check(row_lo, row_hi, p->n, "row")) != OT_OK) return rc;
+    if (block_rows < 0) return fail(OT_ERR_INVALID_ARG, "block_rows must be >= 0");
+    block_rows = launch_rows(p, block_rows);
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    float thr = 0.0f;
+    int64_t argmin = -1, nm = 0;
+    if ((rc = min_row_pass(p, row_lo, row_hi, block_rows, s, &thr, &argmin, &nm)) != OT_OK) return rc;
+    if (thr_out) *thr_out = thr;
+    if (argmin_out) *argmin_out = argmin;
+    if (n_massless_out) *n_massless_out = nm;
+    return OT_OK;
+}
+
+extern "C" int ot_kept_counts_range(const ot_plan *cplan, int64_t row_lo, int64_t row_hi,
+                                    int64_t block_rows, float thr, int64_t *row_counts,
+                                    int64_t *nnz_out, void *stream) {
+    NvtxRange nvtx_range("ot_kept_counts_range");
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if ((rc = range_check(row_lo, row_hi, p->n, "row")) != OT_OK) return rc;
+    if (block_rows < 0) return fail(OT_ERR_INVALID_ARG, "block_rows must be >= 0");
+    if (std::isnan(thr)) return fail(OT_ERR_INVALID_ARG, "thr must not be NaN");
+    block_rows = launch_rows(p, block_rows);
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    int64_t nnz = 0;
+    if ((rc = count_pass(p, row_lo, row_hi, block_rows, thr, p->counts, s, &nnz)) != OT_OK) return rc;
+    if (row_counts && row_hi > row_lo) {
+        OT_CU(cudaMemcpyAsync(row_counts, p->counts + row_lo, (size_t)(row_hi - row_lo) * sizeof(int64_t),
+                              cudaMemcpyDeviceToDevice, s));
+        OT_CU(cudaStreamSynchronize(s));
+    }
+    if (nnz_out) *nnz_out = nnz;
     return OT_OK;
 }
 
@@ -1796,20 +1897,29 @@ extern "C" int ot_marginal_residual(const ot_plan *cplan, double *row_l1, double
     if (rc != OT_OK) return rc;
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
-    RowPassArgs R{};
-    R.o = p->o; R.prm = p->prm; R.d = p->d; R.dcol = p->dcol; R.part = p->rpart;
-    // rows: sum_j T_ij against a_i
-    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
-    R.pts = p->x; R.pot = p->f; R.w = p->a; R.cols = p->m; R.row_begin = 0; R.row_end = p->n;
-    OT_CU(launch_rowpass(2, R, s));
-    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->n, p->d), &p->ds->r_sum[0], s));
-    // columns: the same pass with the clouds' roles swapped
-    OT_CU(launch_dcol(p->x, p->f, p->n, p->d, p->o, p->prm, p->dcol, s));
-    R.pts = p->y; R.pot = p->g; R.w = p->b; R.cols = p->n; R.row_begin = 0; R.row_end = p->m;
-    OT_CU(launch_rowpass(2, R, s));
-    OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(p->m, p->d), &p->ds->r_sum[1], s));
+    if ((rc = residual_pass(p, 0, 0, p->n, s)) != OT_OK) return rc;
+    if ((rc = residual_pass(p, 1, 0, p->m, s)) != OT_OK) return rc;
     if ((rc = sync_read(p, s)) != OT_OK) return rc;
     if (row_l1) *row_l1 = p->hs->s.r_sum[0];
     if (col_l1) *col_l1 = p->hs->s.r_sum[1];
+    return OT_OK;
+}
+
+extern "C" int ot_marginal_residual_range(const ot_plan *cplan, int64_t row_lo, int64_t row_hi,
+                                          int64_t col_lo, int64_t col_hi, double *row_part,
+                                          double *col_part, void *stream) {
+    NvtxRange nvtx_range("ot_marginal_residual_range");
+    ot_plan *p = const_cast<ot_plan *>(cplan);
+    int rc = plan_check(p);
+    if (rc != OT_OK) return rc;
+    if ((rc = range_check(row_lo, row_hi, p->n, "row")) != OT_OK) return rc;
+    if ((rc = range_check(col_lo, col_hi, p->m, "column")) != OT_OK) return rc;
+    if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((rc = residual_pass(p, 0, row_lo, row_hi, s)) != OT_OK) return rc;
+    if ((rc = residual_pass(p, 1, col_lo, col_hi, s)) != OT_OK) return rc;
+    if ((rc = sync_read(p, s)) != OT_OK) return rc;
+    if (row_part) *row_part = p->hs->s.r_sum[0];
+    if (col_part) *col_part = p->hs->s.r_sum[1];
     return OT_OK;
 }

@@ -18,6 +18,12 @@ steps in the same order. The half-steps run in the library's kernels; this
 module only orders the calls and the collectives (torch.distributed: NCCL for
 CUDA tensors, gloo for the CPU tests, whose ranks use the float64 oracle's
 half-step as a stand-in backend).
+
+The row calls split the same way (ShardedRows): each rank reduces its own
+rows of the plan at the gathered potentials -- the marginal residual's parts
+(one all-reduce, sum), the min_row threshold's candidates (all-reduce, min),
+then the kept counts at that threshold (all-reduce, sum) -- and materializes
+its own share of a row list, which needs no exchange at all.
 """
 from __future__ import annotations
 
@@ -169,3 +175,93 @@ class ShardedSinkhorn:
 
     def potentials(self):
         return self.f[self.k][:self.xr.count], self.g[:self.yr.count]
+
+
+class CudaRows:
+    """The library's row calls over one rank's rows: a plan of
+    ot_sinkhorn_pointcloud at the given (gathered) potentials, no iteration.
+    scale: the resolved value the solve used (a string re-resolves it, which
+    for "max_cost" is a full pass over all pairs)."""
+
+    def __init__(self, x, y, a, b, f, g, eps, scale, stream=None):
+        import torch
+        from . import _binding as B
+        from . import sinkhorn
+        self.B = B
+        self.stream = (torch.cuda.current_stream() if stream is None else stream)
+        self.plan = sinkhorn(x, y, a, b, eps=eps, scale=scale, n_iters=0, warm_start=True,
+                             f=f.clone(), g=g.clone(), stream=self.stream)
+        self.n = x.shape[0]
+
+    def residual(self, row_lo, row_hi, col_lo, col_hi):
+        return self.B.ot_marginal_residual_range(self.plan.handle, row_lo, row_hi, col_lo, col_hi,
+                                                 self.stream.cuda_stream)
+
+    def row_max(self, lo, hi, block_rows):
+        return self.B.ot_min_row_range(self.plan.handle, lo, hi, block_rows, self.stream.cuda_stream)
+
+    def row_count(self, lo, hi, thr, block_rows):
+        import torch
+        counts = torch.empty(max(hi - lo, 0), dtype=torch.int64, device=self.plan.f.device)
+        nnz = self.B.ot_kept_counts_range(self.plan.handle, lo, hi, block_rows, float(thr),
+                                          counts.data_ptr() if hi > lo else 0, self.stream.cuda_stream)
+        return counts, nnz
+
+    def materialize(self, row_idx, out=None):
+        return self.plan.materialize_rows(row_idx, out=out, stream=self.stream)
+
+    def close(self):
+        self.plan.close()
+
+
+def share(count: int, rank: int, world: int):
+    """Positions [lo, hi) of a list of `count` items that rank `rank` takes
+    (contiguous, sizes differing by at most one)."""
+    lo = count * rank // world
+    return lo, count * (rank + 1) // world
+
+
+class ShardedRows:
+    """Row calls with the rows split across the ranks of `group` (the same
+    Ranges as the solve). backend: residual(row_lo, row_hi, col_lo, col_hi) ->
+    (row_part, col_part); row_max(lo, hi, block_rows) -> (thr, argmin,
+    n_massless); row_count(lo, hi, thr, block_rows) -> (counts of the range,
+    nnz). device: where the collectives' buffers live (CUDA for NCCL)."""
+
+    _NONE = 1 << 62
+
+    def __init__(self, backend, xr: Ranges, yr: Ranges, rank, world, group=None, device=None):
+        self.backend, self.xr, self.yr = backend, xr, yr
+        self.rank, self.world, self.group, self.device = rank, world, group, device
+
+    def _reduce(self, vals, dtype, op):
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor(vals, dtype=dtype, device=self.device)
+        if self.world > 1:
+            dist.all_reduce(t, op=op, group=self.group)
+        return t.tolist()
+
+    def marginal_residual(self):
+        """(||T1 - a||_1, ||T^T 1 - b||_1): this rank's rows of x and of y."""
+        import torch
+        import torch.distributed as dist
+        r, c = self.backend.residual(self.xr.lo(self.rank), self.xr.hi(self.rank),
+                                     self.yr.lo(self.rank), self.yr.hi(self.rank))
+        return tuple(self._reduce([r, c], torch.float64, dist.ReduceOp.SUM))
+
+    def min_row(self, block_rows=0):
+        """The min_row threshold of the whole plan (thr, argmin, n_massless,
+        nnz) and this rank's kept counts (rows [xr.lo(rank), xr.hi(rank)))."""
+        import torch
+        import torch.distributed as dist
+        lo, hi = self.xr.lo(self.rank), self.xr.hi(self.rank)
+        thr_l, arg_l, nm_l = self.backend.row_max(lo, hi, block_rows)
+        thr = self._reduce([thr_l], torch.float64, dist.ReduceOp.MIN)[0]
+        cand = arg_l if (arg_l >= 0 and thr_l == thr) else self._NONE
+        arg = self._reduce([cand], torch.int64, dist.ReduceOp.MIN)[0]
+        nm = self._reduce([nm_l], torch.int64, dist.ReduceOp.SUM)[0]
+        counts, nnz_l = self.backend.row_count(lo, hi, thr, block_rows)
+        nnz = self._reduce([nnz_l], torch.int64, dist.ReduceOp.SUM)[0]
+        return dict(thr=thr, argmin=-1 if arg == self._NONE else arg, n_massless=nm, nnz=nnz,
+                    counts=counts)

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_version_and_defaults(B):
-    assert B.ot_version() == 3
+    assert B.ot_version() == 4
     o = B.ot_options_default()
     assert (o.warm_start, o.check_every, o.use_graphs, o.iters_per_stage) == (0, 16, 1, 20)
     assert (o.scale_value, o.eps_init, o.eps_decay) == (1.0, 0.0, 0.7)
@@ -112,6 +112,9 @@ def test_row_calls_reject_null_plan(B):
     assert L.ot_marginal_residual(None, None, None, None) == -1
     assert L.ot_sparsify_min_row(None, 0, None, None, None, None, None, None) == -1
     assert L.ot_sparsify_csr(None, 0, 0.5, FAKE, FAKE, FAKE, 1, None, None) == -1
+    assert L.ot_marginal_residual_range(None, 0, 1, 0, 1, None, None, None) == -1
+    assert L.ot_min_row_range(None, 0, 1, 0, None, None, None, None) == -1
+    assert L.ot_kept_counts_range(None, 0, 1, 0, 0.5, None, None, None) == -1
     L.ot_plan_destroy(None)  # no-op
 
 

@@ -11,6 +11,12 @@ in-loop residual (another summation order), ot_max_sqdist over the ranges must
 give the unsplit max_cost exactly, and the driver of the split solve
 (log_domain_sinkhorn_online_b200.sharded) must give the same result at world
 size 1.
+
+The row calls over ranges (ot_marginal_residual_range, ot_min_row_range,
+ot_kept_counts_range) combined over the ranks of a split as the all-reduces
+combine them must give the whole-plan calls' values: thr, argmin, the massless
+count, the counts and nnz exactly, the residual to 1e-12 (another summation
+order).
 """
 import numpy as np
 import pytest
@@ -166,3 +172,100 @@ def test_split_with_empty_ranges_and_massless_rows(ot):
     assert np.isneginf(f[::97]).all() and np.isneginf(g[5::131]).all()
     np.testing.assert_array_equal(f, fr)
     np.testing.assert_array_equal(g, gr)
+
+
+def _massless_problem(d, n, m, seed):
+    import torch
+    rng = np.random.default_rng(seed)
+    x = rng.random((n, d), dtype=np.float32)
+    y = rng.random((m, d), dtype=np.float32)
+    a = rng.random(n).astype(np.float32) + 0.1
+    a[::53] = 0.0
+    a = (a / a.sum()).astype(np.float32)
+    b = np.full(m, 1.0 / m, dtype=np.float32)
+    return tuple(torch.from_numpy(v).cuda() for v in (x, y, a, b))
+
+
+@pytest.mark.parametrize("d,world,block_rows", [(3, 2, 0), (3, 3, 64), (2, 4, 0), (5, 3, 0)])
+def test_range_row_calls_combine_to_the_whole_plan(ot, d, world, block_rows):
+    import torch
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    from log_domain_sinkhorn_online_b200 import sharded as S
+    n, m = 2100, 1700
+    x, y, a, b = _massless_problem(d, n, m, 40 + d)
+    p = ot.sinkhorn(x, y, a, b, eps=0.02, scale="mean", n_iters=5)
+    whole = p.sparsify_min_row(block_rows=block_rows)
+    rw, cw = p.marginal_residual()
+    s = torch.cuda.current_stream().cuda_stream
+    xr, yr = S.Ranges(n, world, 256), S.Ranges(m, world, 256)
+    thr, arg, nm, nnz, rr, cc = np.inf, -1, 0, 0, 0.0, 0.0
+    cands = []
+    counts = torch.full((n,), -1, dtype=torch.int64, device="cuda")
+    for r in range(world):
+        lo, hi = xr.lo(r), xr.hi(r)
+        t, ar, k = B.ot_min_row_range(p.handle, lo, hi, block_rows, s)
+        cands.append((t, ar))
+        thr, nm = min(thr, t), nm + k
+        part_r, part_c = B.ot_marginal_residual_range(p.handle, lo, hi, yr.lo(r), yr.hi(r), s)
+        rr, cc = rr + part_r, cc + part_c
+    arg = min((ar for t, ar in cands if t == thr and ar >= 0), default=-1)
+    for r in range(world):
+        lo, hi = xr.lo(r), xr.hi(r)
+        nnz += B.ot_kept_counts_range(p.handle, lo, hi, block_rows, thr,
+                                      counts[lo:].data_ptr() if hi > lo else 0, s)
+    assert whole["n_massless"] == nm == len(range(0, n, 53))
+    assert thr == whole["thr"] and arg == whole["argmin"] and nnz == whole["nnz"]
+    assert torch.equal(counts, whole["counts"])
+    assert rr == pytest.approx(rw, rel=1e-12) and cc == pytest.approx(cw, rel=1e-12)
+    p.close()
+
+
+def test_sharded_rows_driver_at_world_size_one(ot):
+    import torch
+    from log_domain_sinkhorn_online_b200 import sharded as S
+    n, m = 3000, 2500
+    x, y, a, b = _massless_problem(3, n, m, 7)
+    p = ot.sinkhorn(x, y, a, b, eps=0.01, scale="max_cost", n_iters=8)
+    whole = p.sparsify_min_row()
+    rw, cw = p.marginal_residual()
+    rows = torch.arange(0, n, 7, device="cuda")
+    T = p.materialize_rows(rows)
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    vmax = B.ot_max_sqdist(x.data_ptr(), y.data_ptr(), n, m, 3, 0, n, torch.cuda.current_stream().cuda_stream)
+    back = S.CudaRows(x, y, a, b, p.f, p.g, 0.01, vmax)
+    # the max_cost value passed as a value resolves the same inv_scale_cost
+    assert back.plan.info.inv_scale_cost == p.info.inv_scale_cost
+    sr = S.ShardedRows(back, S.Ranges(n, 1), S.Ranges(m, 1), 0, 1, device=x.device)
+    mr = sr.min_row()
+    assert (mr["thr"], mr["argmin"], mr["n_massless"], mr["nnz"]) == \
+        (whole["thr"], whole["argmin"], whole["n_massless"], whole["nnz"])
+    assert torch.equal(mr["counts"], whole["counts"])
+    assert sr.marginal_residual() == pytest.approx((rw, cw), rel=1e-12)
+    lo, hi = S.share(rows.numel(), 0, 1)
+    assert torch.equal(back.materialize(rows[lo:hi]), T)
+    back.close()
+    p.close()
+
+
+def test_range_calls_check_their_ranges(ot):
+    import torch
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    x, y, a, b = _massless_problem(3, 300, 200, 3)
+    p = ot.sinkhorn(x, y, a, b, eps=0.05, n_iters=2)
+    s = torch.cuda.current_stream().cuda_stream
+    for lo, hi in ((-1, 10), (20, 10), (0, 301)):
+        for call in (lambda: B.ot_min_row_range(p.handle, lo, hi, 0, s),
+                     lambda: B.ot_kept_counts_range(p.handle, lo, hi, 0, 0.5, 0, s),
+                     lambda: B.ot_marginal_residual_range(p.handle, lo, hi, 0, 200, s)):
+            with pytest.raises(B.OTError) as e:
+                call()
+            assert e.value.status == B.OT_ERR_INVALID_ARG
+    with pytest.raises(B.OTError):
+        B.ot_marginal_residual_range(p.handle, 0, 300, 0, 201, s)
+    with pytest.raises(B.OTError):
+        B.ot_kept_counts_range(p.handle, 0, 300, 0, float("nan"), 0, s)
+    # empty ranges: nothing to reduce
+    assert B.ot_min_row_range(p.handle, 5, 5, 0, s) == (float("inf"), -1, 0)
+    assert B.ot_kept_counts_range(p.handle, 5, 5, 0, 0.5, 0, s) == 0
+    assert B.ot_marginal_residual_range(p.handle, 5, 5, 7, 7, s) == (0.0, 0.0)
+    p.close()

@@ -81,12 +81,81 @@ def _rank(rank, world, port, q, n_iters, tol):
         dist.destroy_process_group()
 
 
-def _run(world, n_iters, tol):
+class OracleRows:
+    """The oracle's row reductions over a range of rows (float64), the stand-in
+    for the library's range calls: min_row and kept counts on the sub-cloud of
+    the range's rows, the residual's parts from the oracle's row and column sums."""
+
+    def __init__(self, w, c, f, g):
+        import oracle
+        self.orc, self.w, self.c, self.f, self.g = oracle, w, c, f, g
+
+    def residual(self, row_lo, row_hi, col_lo, col_hi):
+        w = self.w
+        _, _, rs, cs = self.orc.marginal_residual(w.x, w.y, w.a, w.b, self.f, self.g, self.c, w.eps,
+                                                  return_sums=True)
+        a, b = w.a.astype(np.float64), w.b.astype(np.float64)
+        return (float(np.abs(rs[row_lo:row_hi] - a[row_lo:row_hi]).sum()),
+                float(np.abs(cs[col_lo:col_hi] - b[col_lo:col_hi]).sum()))
+
+    def row_max(self, lo, hi, block_rows):
+        if hi <= lo:
+            return float("inf"), -1, 0
+        w = self.w
+        r = self.orc.min_row(w.x[lo:hi], w.y, w.a[lo:hi], self.f[lo:hi], self.g, self.c, w.eps)
+        return r["thr"], (r["argmin"] + lo if r["argmin"] >= 0 else -1), r["n_massless"]
+
+    def row_count(self, lo, hi, thr, block_rows):
+        if hi <= lo:
+            return np.zeros(0, dtype=np.int64), 0
+        w = self.w
+        row_ptr, _, _ = self.orc.sparsify_csr(w.x[lo:hi], w.y, w.a[lo:hi], self.f[lo:hi], self.g,
+                                              self.c, w.eps, thr)
+        return np.diff(row_ptr), int(row_ptr[-1])
+
+
+def _rows_problem():
+    """workload 2's recipe on 301 x 245 points with a few massless rows, at the
+    oracle's potentials after 6 iterations."""
+    import oracle
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w2(n=301, m=245)
+    a = w.a.copy()
+    a[[0, 77, 300]] = 0.0
+    w.a = (a / a.sum()).astype(np.float32)
+    c = oracle.inv_scale_cost(w.x, w.y, w.scale)
+    f, g, _, _ = oracle.sinkhorn(w.x, w.y, w.a, w.b, c, w.eps, 6)
+    return w, c, f, g
+
+
+def _rows_rank(rank, world, port, q, align):
+    import sys
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from log_domain_sinkhorn_online_b200 import sharded as S
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), OMP_NUM_THREADS="1")
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        w, c, f, g = _rows_problem()
+        xr, yr = S.Ranges(w.n, world, align=align), S.Ranges(w.m, world, align=align)
+        rows = S.ShardedRows(OracleRows(w, c, f, g), xr, yr, rank, world)
+        resid = rows.marginal_residual()
+        mr = rows.min_row()
+        q.put((rank, resid, mr["thr"], mr["argmin"], mr["n_massless"], mr["nnz"],
+               np.asarray(mr["counts"]).copy(), (xr.lo(rank), xr.hi(rank))))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, n_iters, tol, target=None, args=None):
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, q, n_iters, tol)) for r in range(world)]
+    target = target or _rank
+    args = (n_iters, tol) if args is None else args
+    procs = [ctx.Process(target=target, args=(r, world, port, q) + args) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted((q.get(timeout=300) for _ in procs), key=lambda r: r[0])
@@ -137,3 +206,23 @@ def test_ranges_cover_the_points_once():
         assert covered == list(range(count))
         assert all(lo % align == 0 for lo, hi in spans) and r.padded >= count
         assert r.shard % align == 0
+
+
+@pytest.mark.parametrize("world,align", [(2, 64), (3, 8), (4, 128)])
+def test_split_row_calls_equal_the_whole_plan(orc, world, align):
+    """min_row (thr, argmin, massless rows, counts, nnz) and the marginal
+    residual with the rows split across gloo ranks equal the oracle's whole-plan
+    values; (4, 128) leaves one rank without x rows and two without y rows."""
+    w, c, f, g = _rows_problem()
+    ref = orc.min_row(w.x, w.y, w.a, f, g, c, w.eps)
+    r_ref = orc.marginal_residual(w.x, w.y, w.a, w.b, f, g, c, w.eps)
+    assert ref["n_massless"] == 3
+    res = _run(world, 0, 0.0, target=_rows_rank, args=(align,))
+    counts = np.zeros(w.n, dtype=np.int64)
+    for rank, resid, thr, arg, nm, nnz, cnt, (lo, hi) in res:
+        assert thr == ref["thr"] and arg == ref["argmin"]
+        assert nm == ref["n_massless"] and nnz == ref["nnz"]
+        assert resid[0] == pytest.approx(r_ref[0], rel=1e-12)
+        assert resid[1] == pytest.approx(r_ref[1], rel=1e-12)
+        counts[lo:hi] = cnt
+    np.testing.assert_array_equal(counts, ref["counts"])
