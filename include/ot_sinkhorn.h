@@ -253,7 +253,13 @@ OT_API int ot_sinkhorn_pointcloud_host(const float *x, const float *y, const flo
  * evaluated at the returned potentials; section D.3: the exponent is built in
  * float64 from the coordinates). Each T_ij: float64 exponent, float32 exp.
  * Deterministic (fixed reduction order). row_l1/col_l1: host pointers, either
- * may be NULL. Synchronises `stream`. */
+ * may be NULL. Synchronises `stream`.
+ * Tile screen (d <= 3; also in the min_row and count passes): rows and columns
+ * are visited in Morton order, and a tile of 32 rows x 256 columns whose bound
+ * kappa (max f + max g) - kappa c dist(boxes)^2 on the base-2 exponent is below
+ * -127 is skipped -- each of its entries is below 2^-126, where the entry is
+ * exactly 0 -- so the results are those of visiting every entry (sums up to
+ * summation order); ot_row_pass_stats reports how much was evaluated. */
 OT_API int ot_marginal_residual(const ot_plan *plan, double *row_l1, double *col_l1, void *stream);
 
 /* ------------------------------------------------------ ot_materialize_rows
@@ -444,6 +450,13 @@ OT_API int ot_shard_half_step(ot_plan *plan, int32_t side, const float *other, c
  * ot_kept_counts_range: pass B at a given thr (not NaN): row_counts (device
  *     int64 [row_hi - row_lo], NULL ok) = #{j : T_ij >= thr} per row of the
  *     range, 0 for a massless row; *nnz_out = their sum. */
+/* ot_row_pass_stats: the tile screen's work in the plan's last row call
+ * (ot_marginal_residual[_range], ot_sparsify_min_row, ot_min_row_range,
+ * ot_kept_counts_range, the count pass of ot_sparsify_csr): tiles of 32 rows x
+ * 256 columns evaluated, and those a visit of every entry evaluates (their
+ * ratio is the share of the plan's entries the call computed). 0 and 0 for
+ * d > 3 (no screen). Host outputs, NULL ok; no device work. */
+OT_API int ot_row_pass_stats(const ot_plan *plan, int64_t *chunks_visited, int64_t *chunks_total);
 OT_API int ot_marginal_residual_range(const ot_plan *plan, int64_t row_lo, int64_t row_hi,
                                       int64_t col_lo, int64_t col_hi, double *row_part,
                                       double *col_part, void *stream);

@@ -64,6 +64,10 @@ class Plan:
         _, r, c = B.ot_marginal_residual(self._h, _stream(stream))
         return r, c
 
+    def row_pass_stats(self):
+        """(tiles evaluated, tiles of a full visit) in the last row call (d <= 3)."""
+        return B.ot_row_pass_stats(self._h)
+
     def materialize_rows(self, row_idx, out=None, stream=None):
         import torch
         row_idx = _dev(row_idx, torch.int64, "row_idx")

@@ -33,7 +33,7 @@ EXPORTED = ("ot_version", "ot_last_error_string", "ot_options_default", "ot_sink
             "ot_sparsify_csr", "ot_materialize_rows_lowrank", "ot_materialize_rows_lrcost",
             "ot_testing_fail_device_allocs", "ot_testing_wait_fault", "ot_max_sqdist",
             "ot_shard_plan_create", "ot_shard_half_step", "ot_marginal_residual_range",
-            "ot_min_row_range", "ot_kept_counts_range")
+            "ot_min_row_range", "ot_kept_counts_range", "ot_row_pass_stats")
 OT_NOALLOC_MAX_POINTS = 1 << 20
 
 
@@ -131,6 +131,8 @@ def lib() -> ctypes.CDLL:
             L.ot_min_row_range.restype = ctypes.c_int
             L.ot_kept_counts_range.argtypes = [P, I64, I64, I64, ctypes.c_float, P, ctypes.POINTER(I64), P]
             L.ot_kept_counts_range.restype = ctypes.c_int
+            L.ot_row_pass_stats.argtypes = [P, ctypes.POINTER(I64), ctypes.POINTER(I64)]
+            L.ot_row_pass_stats.restype = ctypes.c_int
             L.ot_trim_cache.argtypes = []
             L.ot_trim_cache.restype = None
             L.ot_plan_destroy.argtypes = [P]
@@ -286,6 +288,13 @@ def ot_kept_counts_range(plan, row_lo, row_hi, block_rows, thr, row_counts, stre
     _check(lib().ot_kept_counts_range(plan, row_lo, row_hi, block_rows, thr, row_counts or None,
                                       ctypes.byref(nnz), stream))
     return nnz.value
+
+
+def ot_row_pass_stats(plan):
+    """Returns (tiles evaluated, tiles of a full visit) of the plan's last row call."""
+    v, t = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ot_row_pass_stats(plan, ctypes.byref(v), ctypes.byref(t)))
+    return v.value, t.value
 
 
 def ot_marginal_residual_noalloc(x, y, a, b, f, g, n, m, d, eps, inv_scale_cost, stream):

@@ -68,6 +68,7 @@ struct DevScalars {
     double r_sum[2];
     double sums[4][kMaxD];        // sum x, sum x^2, sum y, sum y^2 (per coordinate)
     double wsum[4];               // sum a, -, sum b, -
+    unsigned long long visited;   // row passes: column chunks evaluated since the call began
 };
 
 // block-sparse mode: device counters of one iteration
@@ -128,6 +129,17 @@ struct ot_plan {
     float *rowmax = nullptr;
     int64_t *counts = nullptr;
     int64_t *scan = nullptr;    // tile totals of the row_ptr scan
+    // tile screen of the row passes (d <= 3): Morton orders of the clouds
+    int64_t *mperm[2] = {nullptr, nullptr};  // x, y in Morton order (computed once)
+    int64_t *rperm = nullptr;                // Morton order of a range of rows (per call)
+    unsigned long long *rkeys = nullptr;     // sort keys
+    double *csum = nullptr;                  // chunk summaries of the column table
+    unsigned *rlohi = nullptr;               // a cloud's box (order-preserving bits)
+    bool mperm_ready[2] = {false, false};
+    int64_t screen_total = 0;                // row passes: chunks a full visit would evaluate
+    int64_t screen_visited = 0;              // and those the last row call evaluated
+    bool mort_ready[2] = {false, false};
+    MortonArgs mort[2]{};
     HostScalars *hs = nullptr;  // pinned
     int kp = 0;                 // tensor-core path: bf16 K extent of the operand tables
     bool use_loop = false;      // device-resident iterations (loop.cu)
@@ -447,6 +459,12 @@ cudaError_t launch_iteration(const ot_plan *p, int parity) {
 // ------------------------------------------------------- block-sparse mode
 // (csrc/sparse.cu has the kernels and the design)
 
+int64_t next_pow2(int64_t v) {
+    int64_t r = 1;
+    while (r < v) r <<= 1;
+    return r;
+}
+
 float float_from_order(unsigned o) {
     const unsigned b = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
     float v;
@@ -506,12 +524,7 @@ int sparse_setup(ot_plan *p, const ot_options &o, double tol, bool warm) {
         p->sp_grid[side] = (int)std::min<int64_t>(tiles * sp, cap);
     }
     p->sp_vgrid = (int)std::min<int64_t>(nb * kVerifySegs, (int64_t)vbps * p->sm_count);
-    auto pow2 = [](int64_t v) {
-        int64_t r = 1;
-        while (r < v) r <<= 1;
-        return r;
-    };
-    const int64_t n2x = pow2(n), n2y = pow2(m);
+    const int64_t n2x = next_pow2(n), n2y = next_pow2(m);
     const int64_t part = std::max({(int64_t)p->sp_splits[0] * nb, (int64_t)kVerifySegs * nb,
                                    (int64_t)p->sp_splits[1] * mb}) * B;
     float *xs = nullptr, *ys = nullptr, *as = nullptr, *bs = nullptr;
@@ -1574,6 +1587,14 @@ int ensure_rows_ws(ot_plan *p) {
         p->rowmax = cv.take<float>(p->n);
         p->counts = cv.take<int64_t>(p->n);
         p->scan = cv.take<int64_t>(scan_tmp_count(p->n));
+        if (p->d <= 3) {
+            p->mperm[0] = cv.take<int64_t>(p->n);
+            p->mperm[1] = cv.take<int64_t>(p->m);
+            p->rperm = cv.take<int64_t>(big);
+            p->rkeys = cv.take<unsigned long long>(next_pow2(big));
+            p->csum = cv.take<double>(7 * chunk_count(big));
+            p->rlohi = cv.take<unsigned>(6);
+        }
         if (pass == 0)
             OT_CU(pool_device_alloc(reinterpret_cast<void **>(&p->ws_rows), cv.off, &p->ws_rows_bytes));
     }
@@ -1593,6 +1614,7 @@ int64_t launch_rows(const ot_plan *p, int64_t block_rows) {
 int sync_read(ot_plan *p, cudaStream_t s) {
     OT_CU(cudaMemcpyAsync(&p->hs->s, p->ds, sizeof(DevScalars), cudaMemcpyDeviceToHost, s));
     OT_CU(cudaStreamSynchronize(s));
+    p->screen_visited = (int64_t)p->hs->s.visited;
     return OT_OK;
 }
 
@@ -1600,19 +1622,105 @@ RowPassArgs row_args(const ot_plan *p) {
     RowPassArgs R{};
     R.pts = p->x; R.pot = p->f; R.w = p->a; R.dcol = p->dcol; R.o = p->o; R.prm = p->prm;
     R.cols = p->m; R.d = p->d; R.rowmax = p->rowmax; R.counts = p->counts; R.part = p->rpart;
+    R.visited = p->d <= 3 ? &p->ds->visited : nullptr;
     return R;
 }
 
+// Start of a row call: zero its chunk statistics.
+int screen_reset(ot_plan *p, cudaStream_t s) {
+    OT_CU(cudaMemsetAsync(&p->ds->visited, 0, sizeof(unsigned long long), s));
+    p->screen_total = 0;
+    return OT_OK;
+}
+
+// Chunks a full visit of positions [p0, p1) against `cols` columns evaluates.
+void screen_count(ot_plan *p, int64_t p0, int64_t p1, int64_t cols) {
+    if (p->d <= 3 && p1 > p0) p->screen_total += rowpass_blocks(p1 - p0, p->d) * chunk_count(cols);
+}
+
+// Morton order (30-bit codes over the cloud's own bounding box, the point
+// index breaking ties) of points [lo, hi) of cloud `cl` (0: x, 1: y) into perm
+// (indices of the cloud).
+int morton_order(ot_plan *p, int cl, int64_t lo, int64_t hi, int64_t *perm, cudaStream_t s) {
+    const float *pts = cl ? p->y : p->x;
+    const int64_t cnt = cl ? p->m : p->n;
+    const int d = p->d;
+    if (!p->mort_ready[cl]) {
+        OT_CU(cudaMemsetAsync(p->rlohi, 0xff, 3 * sizeof(unsigned), s));
+        OT_CU(cudaMemsetAsync(p->rlohi + 3, 0, 3 * sizeof(unsigned), s));
+        OT_CU(launch_box(pts, cnt, d, p->rlohi, s));
+        unsigned h[6];
+        OT_CU(cudaMemcpyAsync(h, p->rlohi, sizeof h, cudaMemcpyDeviceToHost, s));
+        OT_CU(cudaStreamSynchronize(s));
+        MortonArgs &M = p->mort[cl];
+        M = MortonArgs{};
+        M.d = d;
+        M.bits = 30 / d;
+        const double cells = (double)(1ll << M.bits);
+        for (int k = 0; k < d; ++k) {
+            const double blo = (double)float_from_order(h[k]), bhi = (double)float_from_order(h[3 + k]);
+            M.lo[k] = blo;
+            M.s[k] = bhi > blo ? cells / (bhi - blo) : 0.0;
+        }
+        p->mort_ready[cl] = true;
+    }
+    const int64_t k = hi - lo;
+    if (k <= 0) return OT_OK;
+    OT_CU(launch_morton_sort(pts + lo * d, k, next_pow2(k), p->mort[cl], p->rkeys, s));
+    OT_CU(launch_perm_from_keys(p->rkeys, k, lo, perm, s));
+    return OT_OK;
+}
+
+// The rows a pass visits and the column table it reads. For d <= 3 the
+// columns (the other cloud) are put in Morton order with their chunk
+// summaries, and rows [lo, hi) of the pass's cloud (`side` 0: x, 1: y) are
+// visited in Morton order, positions [0, hi - lo); `screen` lets the kernel
+// skip the chunks whose entries all vanish. Otherwise the columns keep their
+// order and positions are the rows themselves.
+struct PassRows {
+    const int64_t *rperm = nullptr;
+    const double *csum = nullptr;
+    int64_t p0 = 0, p1 = 0;
+};
+
+int pass_setup(ot_plan *p, int side, int64_t lo, int64_t hi, bool screen, cudaStream_t s, PassRows &pr) {
+    const float *cpts = side ? p->x : p->y, *cpot = side ? p->f : p->g;
+    const int64_t ccnt = side ? p->n : p->m, rcnt = side ? p->m : p->n;
+    if (p->d > 3) {
+        OT_CU(launch_dcol(cpts, cpot, ccnt, p->d, p->o, p->prm, p->dcol, s));
+        pr = PassRows{nullptr, nullptr, lo, hi};
+        return OT_OK;
+    }
+    int rc = OT_OK;
+    for (int cl = 0; cl < 2; ++cl) {
+        if (p->mperm_ready[cl]) continue;
+        if ((rc = morton_order(p, cl, 0, cl ? p->m : p->n, p->mperm[cl], s)) != OT_OK) return rc;
+        p->mperm_ready[cl] = true;
+    }
+    OT_CU(launch_dcol(cpts, cpot, ccnt, p->d, p->o, p->prm, p->dcol, s, p->mperm[side ^ 1]));
+    OT_CU(launch_chunk_summary(p->dcol, ccnt, p->d, p->prm, p->csum, s));
+    const int64_t *rperm = p->mperm[side];
+    if (lo != 0 || hi != rcnt) {
+        if ((rc = morton_order(p, side, lo, hi, p->rperm, s)) != OT_OK) return rc;
+        rperm = p->rperm;
+    }
+    pr = PassRows{rperm, screen ? p->csum : nullptr, 0, hi - lo};
+    return OT_OK;
+}
+
 // min_row pass A over rows [lo, hi): max_j T_ij of every row, then the
-// minimum over the massful ones (thr, its smallest global row index, -1 if
-// none) and the number of massless rows. The column table must be current.
-int min_row_pass(ot_plan *p, int64_t lo, int64_t hi, int64_t block_rows, cudaStream_t s,
-                 float *thr, int64_t *argmin, int64_t *n_massless) {
+// minimum over the massful ones (thr, its smallest row index, -1 if none) and
+// the number of massless rows. pr from pass_setup(side 0, lo, hi).
+int min_row_pass(ot_plan *p, int64_t lo, int64_t hi, const PassRows &pr, int64_t block_rows,
+                 cudaStream_t s, float *thr, int64_t *argmin, int64_t *n_massless) {
     RowPassArgs R = row_args(p);
-    for (int64_t r0 = lo; r0 < hi; r0 += block_rows) {
+    R.rperm = pr.rperm;
+    R.csum = pr.csum;
+    for (int64_t r0 = pr.p0; r0 < pr.p1; r0 += block_rows) {
         R.row_begin = r0;
-        R.row_end = std::min(hi, r0 + block_rows);
+        R.row_end = std::min(pr.p1, r0 + block_rows);
         OT_CU(launch_rowpass(0, R, s));
+        screen_count(p, R.row_begin, R.row_end, R.cols);
     }
     OT_CU(launch_min_row_reduce(p->rowmax + lo, p->a + lo, hi - lo, &p->ds->thr, &p->ds->argmin,
                                 &p->ds->n_massless, s));
@@ -1625,16 +1733,20 @@ int min_row_pass(ot_plan *p, int64_t lo, int64_t hi, int64_t block_rows, cudaStr
 }
 
 // min_row pass B over rows [lo, hi): counts[i] = #{j : T_ij >= thr} (0 for a
-// massless row), indexed by the global row, and their sum.
-int count_pass(ot_plan *p, int64_t lo, int64_t hi, int64_t block_rows, float thr, int64_t *counts,
-               cudaStream_t s, int64_t *nnz) {
+// massless row), indexed by the row, and their sum. The tile screen applies
+// only at thr > 0 (below, the vanishing entries count too).
+int count_pass(ot_plan *p, int64_t lo, int64_t hi, const PassRows &pr, int64_t block_rows,
+               float thr, int64_t *counts, cudaStream_t s, int64_t *nnz) {
     RowPassArgs R = row_args(p);
     R.thr = thr;
     R.counts = counts;
-    for (int64_t r0 = lo; r0 < hi; r0 += block_rows) {
+    R.rperm = pr.rperm;
+    R.csum = thr > 0.0f ? pr.csum : nullptr;
+    for (int64_t r0 = pr.p0; r0 < pr.p1; r0 += block_rows) {
         R.row_begin = r0;
-        R.row_end = std::min(hi, r0 + block_rows);
+        R.row_end = std::min(pr.p1, r0 + block_rows);
         OT_CU(launch_rowpass(1, R, s));
+        screen_count(p, R.row_begin, R.row_end, R.cols);
     }
     OT_CU(launch_sum_i64(counts + lo, hi - lo, &p->ds->nnz, s));
     int rc = sync_read(p, s);
@@ -1648,16 +1760,19 @@ int count_pass(ot_plan *p, int64_t lo, int64_t hi, int64_t block_rows, float thr
 // against b, the pass with the clouds' roles swapped). Rebuilds the column
 // table of the other side; the result lands in p->ds->r_sum[side].
 int residual_pass(ot_plan *p, int side, int64_t lo, int64_t hi, cudaStream_t s) {
+    PassRows pr;
+    int rc = pass_setup(p, side, lo, hi, true, s, pr);
+    if (rc != OT_OK) return rc;
     RowPassArgs R = row_args(p);
-    if (side == 0) {
-        OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
-    } else {
-        OT_CU(launch_dcol(p->x, p->f, p->n, p->d, p->o, p->prm, p->dcol, s));
+    if (side == 1) {
         R.pts = p->y; R.pot = p->g; R.w = p->b; R.cols = p->n;
     }
-    R.row_begin = lo;
-    R.row_end = hi;
+    R.rperm = pr.rperm;
+    R.csum = pr.csum;
+    R.row_begin = pr.p0;
+    R.row_end = pr.p1;
     OT_CU(launch_rowpass(2, R, s));
+    screen_count(p, R.row_begin, R.row_end, R.cols);
     OT_CU(launch_sum_f64(p->rpart, rowpass_blocks(hi - lo, p->d), &p->ds->r_sum[side], s));
     return OT_OK;
 }
@@ -1774,11 +1889,13 @@ extern "C" int ot_sparsify_min_row(const ot_plan *cplan, int64_t block_rows, flo
     block_rows = launch_rows(p, block_rows);
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
-    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    if ((rc = screen_reset(p, s)) != OT_OK) return rc;
+    PassRows pr;
+    if ((rc = pass_setup(p, 0, 0, p->n, true, s, pr)) != OT_OK) return rc;
     float thr = 0.0f;
     int64_t argmin = -1, nm = 0, nnz = 0;
-    if ((rc = min_row_pass(p, 0, p->n, block_rows, s, &thr, &argmin, &nm)) != OT_OK) return rc;
-    rc = count_pass(p, 0, p->n, block_rows, thr, row_counts ? row_counts : p->counts, s, &nnz);
+    if ((rc = min_row_pass(p, 0, p->n, pr, block_rows, s, &thr, &argmin, &nm)) != OT_OK) return rc;
+    rc = count_pass(p, 0, p->n, pr, block_rows, thr, row_counts ? row_counts : p->counts, s, &nnz);
     if (rc != OT_OK) return rc;
     if (thr_out) *thr_out = thr;
     if (nnz_out) *nnz_out = nnz;
@@ -1803,10 +1920,12 @@ extern "C" int ot_min_row_range(const ot_plan *cplan, int64_t row_lo, int64_t ro
     block_rows = launch_rows(p, block_rows);
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
-    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    if ((rc = screen_reset(p, s)) != OT_OK) return rc;
+    PassRows pr;
+    if ((rc = pass_setup(p, 0, row_lo, row_hi, true, s, pr)) != OT_OK) return rc;
     float thr = 0.0f;
     int64_t argmin = -1, nm = 0;
-    if ((rc = min_row_pass(p, row_lo, row_hi, block_rows, s, &thr, &argmin, &nm)) != OT_OK) return rc;
+    if ((rc = min_row_pass(p, row_lo, row_hi, pr, block_rows, s, &thr, &argmin, &nm)) != OT_OK) return rc;
     if (thr_out) *thr_out = thr;
     if (argmin_out) *argmin_out = argmin;
     if (n_massless_out) *n_massless_out = nm;
@@ -1826,9 +1945,11 @@ extern "C" int ot_kept_counts_range(const ot_plan *cplan, int64_t row_lo, int64_
     block_rows = launch_rows(p, block_rows);
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
-    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    if ((rc = screen_reset(p, s)) != OT_OK) return rc;
+    PassRows pr;
+    if ((rc = pass_setup(p, 0, row_lo, row_hi, true, s, pr)) != OT_OK) return rc;
     int64_t nnz = 0;
-    if ((rc = count_pass(p, row_lo, row_hi, block_rows, thr, p->counts, s, &nnz)) != OT_OK) return rc;
+    if ((rc = count_pass(p, row_lo, row_hi, pr, block_rows, thr, p->counts, s, &nnz)) != OT_OK) return rc;
     if (row_counts && row_hi > row_lo) {
         OT_CU(cudaMemcpyAsync(row_counts, p->counts + row_lo, (size_t)(row_hi - row_lo) * sizeof(int64_t),
                               cudaMemcpyDeviceToDevice, s));
@@ -1854,16 +1975,14 @@ extern "C" int ot_sparsify_csr(const ot_plan *cplan, int64_t block_rows, float t
     block_rows = launch_rows(p, block_rows);
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
-    OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
+    if ((rc = screen_reset(p, s)) != OT_OK) return rc;
     // pass 1: kept entries per row (the count pass of ot_sparsify_min_row)
-    RowPassArgs R{};
-    R.pts = p->x; R.pot = p->f; R.w = p->a; R.dcol = p->dcol; R.o = p->o; R.prm = p->prm;
-    R.cols = p->m; R.d = p->d; R.thr = thr; R.counts = p->counts;
-    for (int64_t r0 = 0; r0 < p->n; r0 += block_rows) {
-        R.row_begin = r0;
-        R.row_end = std::min(p->n, r0 + block_rows);
-        OT_CU(launch_rowpass(1, R, s));
-    }
+    PassRows pr;
+    if ((rc = pass_setup(p, 0, 0, p->n, true, s, pr)) != OT_OK) return rc;
+    int64_t counted = 0;
+    if ((rc = count_pass(p, 0, p->n, pr, block_rows, thr, p->counts, s, &counted)) != OT_OK) return rc;
+    // the write pass reads the columns in their own order
+    if (p->d <= 3) OT_CU(launch_dcol(p->y, p->g, p->m, p->d, p->o, p->prm, p->dcol, s));
     // row pointers, and nnz = row_ptr[n]
     OT_CU(launch_row_ptr_scan(p->counts, p->n, row_ptr, p->scan, s));
     OT_CU(cudaMemcpyAsync(&p->ds->nnz, row_ptr + p->n, sizeof(int64_t), cudaMemcpyDeviceToDevice, s));
@@ -1897,11 +2016,19 @@ extern "C" int ot_marginal_residual(const ot_plan *cplan, double *row_l1, double
     if (rc != OT_OK) return rc;
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
+    if ((rc = screen_reset(p, s)) != OT_OK) return rc;
     if ((rc = residual_pass(p, 0, 0, p->n, s)) != OT_OK) return rc;
     if ((rc = residual_pass(p, 1, 0, p->m, s)) != OT_OK) return rc;
     if ((rc = sync_read(p, s)) != OT_OK) return rc;
     if (row_l1) *row_l1 = p->hs->s.r_sum[0];
     if (col_l1) *col_l1 = p->hs->s.r_sum[1];
+    return OT_OK;
+}
+
+extern "C" int ot_row_pass_stats(const ot_plan *plan, int64_t *chunks_visited, int64_t *chunks_total) {
+    if (!plan) return fail(OT_ERR_INVALID_ARG, "null plan");
+    if (chunks_visited) *chunks_visited = plan->d <= 3 ? plan->screen_visited : 0;
+    if (chunks_total) *chunks_total = plan->d <= 3 ? plan->screen_total : 0;
     return OT_OK;
 }
 
@@ -1916,6 +2043,7 @@ extern "C" int ot_marginal_residual_range(const ot_plan *cplan, int64_t row_lo, 
     if ((rc = range_check(col_lo, col_hi, p->m, "column")) != OT_OK) return rc;
     if ((rc = ensure_rows_ws(p)) != OT_OK) return rc;
     cudaStream_t s = (cudaStream_t)stream;
+    if ((rc = screen_reset(p, s)) != OT_OK) return rc;
     if ((rc = residual_pass(p, 0, row_lo, row_hi, s)) != OT_OK) return rc;
     if ((rc = residual_pass(p, 1, col_lo, col_hi, s)) != OT_OK) return rc;
     if ((rc = sync_read(p, s)) != OT_OK) return rc;

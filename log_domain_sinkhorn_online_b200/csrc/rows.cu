@@ -62,21 +62,74 @@ __device__ __forceinline__ float plan_entry(double Ash, const double *P, const d
     return exp2_shifted(t);
 }
 
-// Column table in float64: dcol[j*(d+1) + q] = y'_jq (q < d), dcol[j*(d+1) + d] = B_j.
+// Column table in float64: dcol[j*(d+1) + q] = y'_jq (q < d), dcol[j*(d+1) + d] = B_j,
+// for the column perm[j] (perm NULL: column j).
 __global__ void build_dcol_kernel(const float *__restrict__ p, const float *__restrict__ pot,
                                   int64_t cnt, int d, const double *__restrict__ o,
-                                  const Params *__restrict__ prm, double *dcol) {
+                                  const Params *__restrict__ prm, const int64_t *__restrict__ perm,
+                                  double *dcol) {
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= cnt) return;
+    const int64_t src = perm ? perm[j] : j;
     const double kappa = prm->kappa, c = prm->c;
     double nrm = 0.0;
     for (int q = 0; q < d; ++q) {
-        const double v = (double)p[j * d + q] - o[q];
+        const double v = (double)p[src * d + q] - o[q];
         dcol[j * (d + 1) + q] = v;
         nrm += v * v;
     }
-    const float pv = pot[j];
+    const float pv = pot[src];
     dcol[j * (d + 1) + d] = (pv == -INFINITY) ? -INFINITY : kappa * ((double)pv - c * nrm);
+}
+
+// Summary of each chunk of kRpChunk consecutive columns of the column table
+// (d <= 3), for the tile screen of the row passes: csum[7c .. 7c+2] and
+// [7c+3 .. 7c+5] the chunk's box in y' (0 past d), csum[7c+6] = max over its
+// columns of kappa g_j = B_j + kappa c |y'_j|^2 (-inf if every column is
+// massless). One warp per chunk.
+constexpr int kRpChunkC = 256;
+__global__ void chunk_summary_kernel(const double *__restrict__ dcol, int64_t cnt, int d,
+                                     const Params *__restrict__ prm, double *csum) {
+    const int64_t chunk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunks = (cnt + kRpChunkC - 1) / kRpChunkC;
+    if (chunk >= nchunks) return;
+    const double kc = prm->kappa * prm->c;
+    double lo[3] = {INFINITY, INFINITY, INFINITY}, hi[3] = {-INFINITY, -INFINITY, -INFINITY};
+    double gmax = -INFINITY;
+    const int64_t j1 = min(cnt, (chunk + 1) * kRpChunkC);
+    for (int64_t j = chunk * kRpChunkC + lane; j < j1; j += 32) {
+        double nrm = 0.0;
+        for (int q = 0; q < d; ++q) {
+            const double v = dcol[j * (d + 1) + q];
+            lo[q] = fmin(lo[q], v);
+            hi[q] = fmax(hi[q], v);
+            nrm += v * v;
+        }
+        const double B = dcol[j * (d + 1) + d];
+        if (B != -INFINITY) gmax = fmax(gmax, B + kc * nrm);
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+        for (int q = 0; q < 3; ++q) {
+            lo[q] = fmin(lo[q], __shfl_xor_sync(0xffffffffu, lo[q], off));
+            hi[q] = fmax(hi[q], __shfl_xor_sync(0xffffffffu, hi[q], off));
+        }
+        gmax = fmax(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
+    }
+    if (lane == 0) {
+        for (int q = 0; q < 3; ++q) {
+            csum[chunk * 7 + q] = q < d ? lo[q] : 0.0;
+            csum[chunk * 7 + 3 + q] = q < d ? hi[q] : 0.0;
+        }
+        csum[chunk * 7 + 6] = gmax;
+    }
+}
+
+// perm[r] = off + the point index in the r-th sorted Morton key
+__global__ void perm_from_keys_kernel(const unsigned long long *keys, int64_t cnt, int64_t off,
+                                      int64_t *perm) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r < cnt) perm[r] = off + (int64_t)(keys[r] & 0xffffffffull);
 }
 
 // Row data of one row: A' = A + kShift and P (d values).
@@ -181,15 +234,30 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
 // operations, and more resident warps hide it better than more rows per warp
 // (measured at n = m = 1e5: 4 rows x 3 blocks 32 % of the MUFU rate for the
 // residual pass, 8 rows x 2 blocks 30 %).
-// Lane l takes columns l, l + 32, ... of each chunk for all 8 rows of its warp,
+// Lane l takes columns l, l + 32, ... of each chunk for all 4 rows of its warp,
 // so every row's reduction stays in one warp, in a fixed lane order
 // (deterministic). Sums: the 8 terms of a row in one chunk add up in float32,
-// those partial sums in float64.
+// those partial sums in float64. With R.rperm the pass's positions are taken
+// through that permutation (results still land at the row's own index); the
+// column order is whatever the column table holds.
 enum { OP_MAX = 0, OP_COUNT = 1, OP_SUM = 2 };
-constexpr int kRpThreads = 256, kRpWarps = kRpThreads / 32, kRpR = 4, kRpChunk = 256;
+constexpr int kRpThreads = 256, kRpWarps = kRpThreads / 32, kRpR = 4, kRpChunk = kRpChunkC;
 constexpr int kRpRows = kRpWarps * kRpR;  // rows per block, d <= 3 (32)
 constexpr int kRgRows = 8;                // rows per block, generic d
+constexpr int kRpWin = 8192;              // chunks screened at a time (one bit each)
 
+// Tile screen (d <= 3, R.csum set). The pass's rows come in Morton order
+// (R.rperm), so a block's 32 rows are close together, and so are the columns
+// of a chunk (the column table is in Morton order too). For rows I and the
+// columns J of a chunk,
+//   e2_ij = kappa (f_i + g_j) - kappa c |x'_i - y'_j|^2
+//        <= kappa max_I f + kappa max_J g - kappa c dist(box(x'_I), box(y'_J))^2,
+// and a chunk whose bound is below -127 is skipped: every entry of it is below
+// 2^-126, where the entry function returns exactly 0 (the margin of one unit of
+// e2 is far above the float64 rounding of the bound and of the entry), so row
+// sums, maxima and counts at a threshold above 0 are the same as with every
+// chunk visited. The block bounds its rows first (lane 0 of each warp, then one
+// thread), then every thread screens kRpWin chunks at a time into a bit mask.
 template <int D, int OP>
 __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
     constexpr int DS = D + 1;                 // doubles per column record
@@ -197,17 +265,46 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
     constexpr int PER = (kRpChunk * DS + kRpThreads - 1) / kRpThreads;  // prefetched doubles
     __shared__ __align__(16) double sc[kRpChunk * DP];
     __shared__ double sRed[kRpWarps][kRpR];
+    __shared__ double sBox[kRpWarps + 1][7];  // per warp, then the block: lo[3], hi[3], kappa max f
+    __shared__ unsigned sLive[kRpWin / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t rw = R.row_begin + (int64_t)blockIdx.x * kRpRows + (int64_t)warp * kRpR;
+    const int64_t rw = R.row_begin + (int64_t)blockIdx.x * kRpRows + (int64_t)warp * kRpR;  // positions
     double Ash[kRpR], P[kRpR][D];
 #pragma unroll
     for (int r = 0; r < kRpR; ++r) {
         if (rw + r < R.row_end) {
-            load_row(R.pts, R.pot, rw + r, D, R.o, R.prm->kappa, R.prm->c, &Ash[r], P[r]);
+            const int64_t i = R.rperm ? R.rperm[rw + r] : rw + r;
+            load_row(R.pts, R.pot, i, D, R.o, R.prm->kappa, R.prm->c, &Ash[r], P[r]);
         } else {
             Ash[r] = -INFINITY;
 #pragma unroll
             for (int q = 0; q < D; ++q) P[r][q] = 0.0;
+        }
+    }
+    if (R.csum) {
+        if (lane == 0) {
+            double b[7] = {INFINITY, INFINITY, INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            for (int r = 0; r < kRpR; ++r) {
+                if (rw + r >= R.row_end) break;
+                const int64_t i = R.rperm ? R.rperm[rw + r] : rw + r;
+                for (int q = 0; q < D; ++q) {
+                    const double v = (double)R.pts[i * D + q] - R.o[q];
+                    b[q] = fmin(b[q], v);
+                    b[3 + q] = fmax(b[3 + q], v);
+                }
+                const float pv = R.pot[i];
+                if (pv != -INFINITY) b[6] = fmax(b[6], R.prm->kappa * (double)pv);
+            }
+            for (int q = 0; q < 7; ++q) sBox[warp][q] = b[q];
+        }
+        __syncthreads();
+        if (tid == 0) {
+            for (int q = 0; q < 7; ++q) {
+                double v = sBox[0][q];
+                for (int w = 1; w < kRpWarps; ++w)
+                    v = (q < 3) ? fmin(v, sBox[w][q]) : fmax(v, sBox[w][q]);
+                sBox[kRpWarps][q] = v;
+            }
         }
     }
     float mx[kRpR];
@@ -215,7 +312,7 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
     double sum[kRpR];
 #pragma unroll
     for (int r = 0; r < kRpR; ++r) {
-        mx[r] = -1.0f;
+        mx[r] = 0.0f;  // entries are >= 0, and a row has at least one
         cnt[r] = 0;
         sum[r] = 0.0;
     }
@@ -231,49 +328,87 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
                      : ((tid + k * kRpThreads) % DS == D ? -INFINITY : 0.0);
         }
     };
-    fetch(0);
-    for (int64_t c0 = 0; c0 < R.cols; c0 += kRpChunk) {
-        __syncthreads();  // the previous chunk is no longer read
+    const int64_t nchunks = (R.cols + kRpChunk - 1) / kRpChunk;
+    const double kc = R.prm->kappa * R.prm->c;
+    unsigned nvis = 0;  // chunks evaluated (the same in every thread)
+    for (int64_t w0 = 0; w0 < nchunks; w0 += kRpWin) {
+        const int nw = (int)min((int64_t)kRpWin, nchunks - w0);
+        __syncthreads();  // the previous window's mask and chunk are no longer read
+        for (int k = tid; k < ((nw + 31) & ~31); k += kRpThreads) {
+            bool live = k < nw;
+            if (live && R.csum) {
+                const double *cs = R.csum + (w0 + k) * 7;
+                const double *bb = sBox[kRpWarps];
+                double d2 = 0.0;
 #pragma unroll
-        for (int k = 0; k < PER; ++k) {
-            const int e = tid + k * kRpThreads;
-            if (e < kRpChunk * DS) sc[(e / DS) * DP + (e % DS)] = pre[k];
+                for (int q = 0; q < D; ++q) {
+                    const double gap = fmax(0.0, fmax(cs[q] - bb[3 + q], bb[q] - cs[3 + q]));
+                    d2 = fma(gap, gap, d2);
+                }
+                live = bb[6] + cs[6] - kc * d2 >= -127.0;
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, live);
+            if (lane == 0) sLive[k >> 5] = bal;
         }
         __syncthreads();
-        if (c0 + kRpChunk < R.cols) fetch(c0 + kRpChunk);
-        float part[kRpR];
+        auto next_live = [&](int k) {  // first chunk >= k of the window that is visited, or nw
+            while (k < nw) {
+                const unsigned word = sLive[k >> 5] >> (k & 31);
+                if (word) return k + __ffs(word) - 1;
+                k = (k | 31) + 1;
+            }
+            return nw;
+        };
+        int k = next_live(0);
+        if (k < nw) fetch((w0 + k) * kRpChunk);
+        while (k < nw) {
+            const int64_t c0 = (w0 + k) * kRpChunk;
+            ++nvis;
+            __syncthreads();  // the previous chunk is no longer read
 #pragma unroll
-        for (int r = 0; r < kRpR; ++r) part[r] = 0.0f;
+            for (int u = 0; u < PER; ++u) {
+                const int e = tid + u * kRpThreads;
+                if (e < kRpChunk * DS) sc[(e / DS) * DP + (e % DS)] = pre[u];
+            }
+            __syncthreads();
+            const int kn = next_live(k + 1);
+            if (kn < nw) fetch((w0 + kn) * kRpChunk);
+            float part[kRpR];
+#pragma unroll
+            for (int r = 0; r < kRpR; ++r) part[r] = 0.0f;
 #pragma unroll 2
-        for (int s = 0; s < kRpChunk / 32; ++s) {
-            const int cc = s * 32 + lane;
-            double col[DP];
-            if (DP == 2) {
-                const double2 v = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
-                col[0] = v.x;
-                col[1] = v.y;
-            } else {
-                const double2 v0 = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
-                const double2 v1 = *reinterpret_cast<const double2 *>(&sc[cc * DP + 2]);
-                col[0] = v0.x;
-                col[1] = v0.y;
-                col[2] = v1.x;
-                col[3] = v1.y;
-            }
-            const bool live = c0 + cc < R.cols;
+            for (int s2 = 0; s2 < kRpChunk / 32; ++s2) {
+                const int cc = s2 * 32 + lane;
+                double col[DP];
+                if (DP == 2) {
+                    const double2 v = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
+                    col[0] = v.x;
+                    col[1] = v.y;
+                } else {
+                    const double2 v0 = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
+                    const double2 v1 = *reinterpret_cast<const double2 *>(&sc[cc * DP + 2]);
+                    col[0] = v0.x;
+                    col[1] = v0.y;
+                    col[2] = v1.x;
+                    col[3] = v1.y;
+                }
+                const bool live = c0 + cc < R.cols;
 #pragma unroll
-            for (int r = 0; r < kRpR; ++r) {
-                const float t = plan_entry<D>(Ash[r], P[r], col, D);
-                if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
-                if (OP == OP_COUNT) cnt[r] += (live && t >= R.thr) ? 1 : 0;
-                if (OP == OP_SUM) part[r] += t;
+                for (int r = 0; r < kRpR; ++r) {
+                    const float t = plan_entry<D>(Ash[r], P[r], col, D);
+                    if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
+                    if (OP == OP_COUNT) cnt[r] += (live && t >= R.thr) ? 1 : 0;
+                    if (OP == OP_SUM) part[r] += t;
+                }
             }
-        }
-        if (OP == OP_SUM) {
+            if (OP == OP_SUM) {
 #pragma unroll
-            for (int r = 0; r < kRpR; ++r) sum[r] += (double)part[r];
+                for (int r = 0; r < kRpR; ++r) sum[r] += (double)part[r];
+            }
+            k = kn;
         }
     }
+    if (tid == 0 && R.visited) atomicAdd(R.visited, (unsigned long long)nvis);
     // per-row reductions across the warp (fixed order), then per block
 #pragma unroll
     for (int r = 0; r < kRpR; ++r) {
@@ -283,9 +418,10 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
             v = OP == OP_MAX ? fmax(v, o2) : v + o2;
         }
         if (lane == 0) {
-            const int64_t i = rw + r;
+            const int64_t pos = rw + r;
             double res = 0.0;
-            if (i < R.row_end) {
+            if (pos < R.row_end) {
+                const int64_t i = R.rperm ? R.rperm[pos] : pos;
                 const float wi = R.w[i];
                 if (OP == OP_MAX) R.rowmax[i] = (float)v;
                 if (OP == OP_COUNT) R.counts[i] = wi > 0.0f ? (int64_t)v : 0;
@@ -729,9 +865,26 @@ __global__ void __launch_bounds__(kRedThreads) sum_kernel(const T *v, int64_t cn
 
 // ----------------------------------------------------------------- launchers
 cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, const double *o,
-                        const Params *prm, double *dcol, cudaStream_t s) {
+                        const Params *prm, double *dcol, cudaStream_t s, const int64_t *perm) {
     if (cnt <= 0) return cudaSuccess;
-    build_dcol_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, s>>>(p, pot, cnt, d, o, prm, dcol);
+    build_dcol_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, s>>>(p, pot, cnt, d, o, prm, perm, dcol);
+    return cudaGetLastError();
+}
+
+int64_t chunk_count(int64_t cols) { return (cols + kRpChunkC - 1) / kRpChunkC; }
+
+cudaError_t launch_chunk_summary(const double *dcol, int64_t cnt, int d, const Params *prm,
+                                 double *csum, cudaStream_t s) {
+    const int64_t warps = chunk_count(cnt);
+    if (warps <= 0) return cudaSuccess;
+    chunk_summary_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(dcol, cnt, d, prm, csum);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_perm_from_keys(const unsigned long long *keys, int64_t cnt, int64_t off,
+                                  int64_t *perm, cudaStream_t s) {
+    if (cnt <= 0) return cudaSuccess;
+    perm_from_keys_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, s>>>(keys, cnt, off, perm);
     return cudaGetLastError();
 }
 

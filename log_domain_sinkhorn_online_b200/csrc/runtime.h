@@ -90,12 +90,15 @@ struct RowPassArgs {
     const float *pts, *pot, *w;
     const double *dcol, *o;
     const Params *prm;
-    int64_t row_begin, row_end, cols;
+    int64_t row_begin, row_end, cols;  // positions [row_begin, row_end) of the pass
     int d;
     float thr;
     float *rowmax;
     int64_t *counts;
     double *part;
+    const int64_t *rperm;  // position -> row (NULL: the identity)
+    const double *csum;    // chunk summaries of the column table for the tile screen (NULL: none)
+    unsigned long long *visited;  // += chunks the pass evaluated (NULL: not counted)
 };
 struct LrArgs {
     const float *fa, *fb;       // row factors [n, r] and column factors [m, r]
@@ -202,7 +205,13 @@ cudaError_t launch_transpose_bytes(const uint8_t *in, int64_t rows, int64_t cols
 cudaError_t launch_halfstep_sparse(int d, int rpt, const HalfStep &A, int grid, cudaStream_t s);
 
 cudaError_t launch_dcol(const float *p, const float *pot, int64_t cnt, int d, const double *o,
-                        const Params *prm, double *dcol, cudaStream_t s);
+                        const Params *prm, double *dcol, cudaStream_t s, const int64_t *perm = nullptr);
+// chunks of the row passes' column table (256 columns each) and their summaries
+int64_t chunk_count(int64_t cols);
+cudaError_t launch_chunk_summary(const double *dcol, int64_t cnt, int d, const Params *prm,
+                                 double *csum, cudaStream_t s);
+cudaError_t launch_perm_from_keys(const unsigned long long *keys, int64_t cnt, int64_t off,
+                                  int64_t *perm, cudaStream_t s);
 cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s);
 cudaError_t launch_rowpass(int op, const RowPassArgs &R, cudaStream_t s);
 // residual partials one pass over `rows` rows writes (blocks of the pass)

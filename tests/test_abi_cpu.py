@@ -115,6 +115,7 @@ def test_row_calls_reject_null_plan(B):
     assert L.ot_marginal_residual_range(None, 0, 1, 0, 1, None, None, None) == -1
     assert L.ot_min_row_range(None, 0, 1, 0, None, None, None, None) == -1
     assert L.ot_kept_counts_range(None, 0, 1, 0, 0.5, None, None, None) == -1
+    assert L.ot_row_pass_stats(None, None, None) == -1
     L.ot_plan_destroy(None)  # no-op
 
 
