@@ -515,7 +515,15 @@ def _side(ot, step, w, stream, peak_ex2, hbm_gbs):
                        stream)
         out["scale_pass"] = {"what": "plan set-up with the all-pairs max_cost pass (max_cost_lowd_kernel)",
                              "ms": ms, "pairs_per_s": float(w.n) * w.m / (ms / 1e3)}
-    # a8-a10 at the solved state, through one plan
+    # a8-a10 at the solved state, through one plan; the row kernels are loaded first on a
+    # small problem of the same d (their first launch would otherwise load the module)
+    xs, ys = step.x[:256].contiguous(), step.y[:256].contiguous()
+    ws = torch.full((256,), 1.0 / 256, device=step.dev)
+    small = ot.sinkhorn(xs, ys, ws, ws, eps=w.eps, scale=step.scale, n_iters=2)
+    small.materialize_rows(torch.arange(8, device=step.dev))
+    small.marginal_residual()
+    small.sparsify_min_row()
+    small.close()
     plan = ot.sinkhorn(step.x, step.y, step.a, step.b, eps=w.eps, scale=step.scale, n_iters=0,
                        warm_start=True, f=step.f.clone(), g=step.g.clone())
     k = w.block_rows or 1024  # one block of the workload's row materialization
