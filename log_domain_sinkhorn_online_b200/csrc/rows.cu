@@ -26,8 +26,13 @@
 // 2^-126 = 1.2e-38, the smallest normal float, are flushed; a massless side,
 // potential -inf, lands there) and from 386 on as +inf. Per entry: d + 1 float64
 // FMAs/adds, two float64 compares, three integer operations, two selects, one
-// ex2. The row passes accumulate each row's terms 8 at a time in float32 and
-// those partial sums in float64 (maxima and counts exactly).
+// ex2. Where a tile bound proves e2 < 128 for all its entries, the row passes
+// use exp2_shifted_capped: one integer compare of the high word replaces both
+// float64 compares, the cap and a select, with the same value bit for bit.
+// The row passes accumulate each row's terms 8 at a time in float32 and those
+// partial sums in float64 (maxima and counts exactly).
+#include <type_traits>
+
 #include "runtime.h"
 
 namespace ot {
@@ -47,6 +52,19 @@ __device__ __forceinline__ float exp2_shifted(double t) {
     return t < kShiftHi ? r : INFINITY;
 }
 
+// The same for an e2 known to lie below 128 (a tile whose bound says so): the
+// high word of t is that of kShift - 126 exactly when e2 >= -126 (t in
+// [2^29 * 1.5, 2^29 * 1.5 + 512)), which takes the place of both range tests
+// and of the cap; the value is bit for bit that of exp2_shifted.
+constexpr unsigned kBaseHi = 0x41C80000u;  // high word of 1.5 * 2^29
+__device__ __forceinline__ float exp2_shifted_capped(double t) {
+    const unsigned lo = (unsigned)__double2loint(t);
+    const unsigned mant = (lo & 0x7FFFFFu) | 0x3F800000u;
+    const float p = ex2_approx(__uint_as_float(mant));
+    const float v = __uint_as_float(__float_as_uint(p) + lo - mant);
+    return (unsigned)__double2hiint(t) == kBaseHi ? v : 0.0f;
+}
+
 // the one float path for a plan entry: row data (A' = A + kShift, P[d]),
 // column data (y'[d], B)
 template <int D>
@@ -60,6 +78,15 @@ __device__ __forceinline__ float plan_entry(double Ash, const double *P, const d
     if (D == 0)
         for (int q = 0; q < dd; ++q) t = fma(P[q], col[q], t);
     return exp2_shifted(t);
+}
+
+// plan_entry for an entry known to lie below 2^128 (d <= 3)
+template <int D>
+__device__ __forceinline__ float plan_entry_capped(double Ash, const double *P, const double *col) {
+    double t = Ash + col[D];
+#pragma unroll
+    for (int q = 0; q < D; ++q) t = fma(P[q], col[q], t);
+    return exp2_shifted_capped(t);
 }
 
 // Column table in float64: dcol[j*(d+1) + q] = y'_jq (q < d), dcol[j*(d+1) + d] = B_j,
@@ -266,7 +293,7 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
     __shared__ __align__(16) double sc[kRpChunk * DP];
     __shared__ double sRed[kRpWarps][kRpR];
     __shared__ double sBox[kRpWarps + 1][7];  // per warp, then the block: lo[3], hi[3], kappa max f
-    __shared__ unsigned sLive[kRpWin / 32];
+    __shared__ unsigned sLive[kRpWin / 32], sSafe[kRpWin / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t rw = R.row_begin + (int64_t)blockIdx.x * kRpRows + (int64_t)warp * kRpR;  // positions
     double Ash[kRpR], P[kRpR][D];
@@ -335,7 +362,7 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
         const int nw = (int)min((int64_t)kRpWin, nchunks - w0);
         __syncthreads();  // the previous window's mask and chunk are no longer read
         for (int k = tid; k < ((nw + 31) & ~31); k += kRpThreads) {
-            bool live = k < nw;
+            bool live = k < nw, safe = false;
             if (live && R.csum) {
                 const double *cs = R.csum + (w0 + k) * 7;
                 const double *bb = sBox[kRpWarps];
@@ -345,10 +372,16 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
                     const double gap = fmax(0.0, fmax(cs[q] - bb[3 + q], bb[q] - cs[3 + q]));
                     d2 = fma(gap, gap, d2);
                 }
-                live = bb[6] + cs[6] - kc * d2 >= -127.0;
+                const double bound = bb[6] + cs[6] - kc * d2;
+                live = bound >= -127.0;
+                safe = bound < 127.0;  // no entry reaches 2^128: the capped entry applies
             }
             const unsigned bal = __ballot_sync(0xffffffffu, live);
-            if (lane == 0) sLive[k >> 5] = bal;
+            const unsigned bsafe = __ballot_sync(0xffffffffu, safe);
+            if (lane == 0) {
+                sLive[k >> 5] = bal;
+                sSafe[k >> 5] = bsafe;
+            }
         }
         __syncthreads();
         auto next_live = [&](int k) {  // first chunk >= k of the window that is visited, or nw
@@ -373,38 +406,47 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
             __syncthreads();
             const int kn = next_live(k + 1);
             if (kn < nw) fetch((w0 + kn) * kRpChunk);
-            float part[kRpR];
+            // the chunk's entries; CAPPED: the tile bound keeps them below 2^128
+            auto run_chunk = [&](auto capped) {
+                constexpr bool CAPPED = decltype(capped)::value;
+                float part[kRpR];
 #pragma unroll
-            for (int r = 0; r < kRpR; ++r) part[r] = 0.0f;
+                for (int r = 0; r < kRpR; ++r) part[r] = 0.0f;
 #pragma unroll 2
-            for (int s2 = 0; s2 < kRpChunk / 32; ++s2) {
-                const int cc = s2 * 32 + lane;
-                double col[DP];
-                if (DP == 2) {
-                    const double2 v = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
-                    col[0] = v.x;
-                    col[1] = v.y;
-                } else {
-                    const double2 v0 = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
-                    const double2 v1 = *reinterpret_cast<const double2 *>(&sc[cc * DP + 2]);
-                    col[0] = v0.x;
-                    col[1] = v0.y;
-                    col[2] = v1.x;
-                    col[3] = v1.y;
-                }
-                const bool live = c0 + cc < R.cols;
+                for (int s2 = 0; s2 < kRpChunk / 32; ++s2) {
+                    const int cc = s2 * 32 + lane;
+                    double col[DP];
+                    if (DP == 2) {
+                        const double2 v = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
+                        col[0] = v.x;
+                        col[1] = v.y;
+                    } else {
+                        const double2 v0 = *reinterpret_cast<const double2 *>(&sc[cc * DP]);
+                        const double2 v1 = *reinterpret_cast<const double2 *>(&sc[cc * DP + 2]);
+                        col[0] = v0.x;
+                        col[1] = v0.y;
+                        col[2] = v1.x;
+                        col[3] = v1.y;
+                    }
+                    const bool live = c0 + cc < R.cols;
 #pragma unroll
-                for (int r = 0; r < kRpR; ++r) {
-                    const float t = plan_entry<D>(Ash[r], P[r], col, D);
-                    if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
-                    if (OP == OP_COUNT) cnt[r] += (live && t >= R.thr) ? 1 : 0;
-                    if (OP == OP_SUM) part[r] += t;
+                    for (int r = 0; r < kRpR; ++r) {
+                        const float t = CAPPED ? plan_entry_capped<D>(Ash[r], P[r], col)
+                                               : plan_entry<D>(Ash[r], P[r], col, D);
+                        if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
+                        if (OP == OP_COUNT) cnt[r] += (live && t >= R.thr) ? 1 : 0;
+                        if (OP == OP_SUM) part[r] += t;
+                    }
                 }
-            }
-            if (OP == OP_SUM) {
+                if (OP == OP_SUM) {
 #pragma unroll
-                for (int r = 0; r < kRpR; ++r) sum[r] += (double)part[r];
-            }
+                    for (int r = 0; r < kRpR; ++r) sum[r] += (double)part[r];
+                }
+            };
+            if ((sSafe[k >> 5] >> (k & 31)) & 1u)
+                run_chunk(std::true_type{});
+            else
+                run_chunk(std::false_type{});
             k = kn;
         }
     }
