@@ -122,3 +122,25 @@ def test_screened_range_rows_equal_the_materialized_plan(ot):
     r, _ = B.ot_marginal_residual_range(p.handle, lo, hi, 0, 0, s)
     assert abs(r - (T.double().sum(1) - a[lo:hi].double()).abs().sum().item()) <= 1e-6
     p.close()
+
+
+def test_screen_over_several_windows_of_chunks(ot):
+    """More than 8192 chunks of 256 columns (m = 2.2e6): the pass screens them a
+    window at a time; rows 100, so the materialized plan is the reference."""
+    import torch
+    n, m = 100, 2_200_000
+    x, y, a, b = _problem(3, n, m, 91)
+    p = ot.sinkhorn(x, y, a, b, eps=3e-4, scale="max_cost", n_iters=3)
+    T = p.materialize_rows(torch.arange(n, device="cuda"))
+    massful = a > 0
+    rowmax = T.max(1).values
+    thr_ref = rowmax[massful].min()
+    mr = p.sparsify_min_row()
+    visited, total = p.row_pass_stats()
+    assert 0 < visited < total
+    assert mr["thr"] == float(thr_ref)
+    counts_ref = torch.where(massful, (T >= thr_ref).sum(1), torch.zeros_like(mr["counts"]))
+    assert torch.equal(mr["counts"], counts_ref)
+    r, _ = p.marginal_residual()
+    assert abs(r - (T.double().sum(1) - a.double()).abs().sum().item()) <= 1e-6
+    p.close()
