@@ -31,6 +31,9 @@
  *    computes returns OT_ERR_CUDA.
  *  - Each call is wrapped in an NVTX range named after it (visible to Nsight
  *    tools; a no-op without one).
+ *  - A plan keeps scratch and state between calls (workspaces, the Morton
+ *    orders of the row passes, the last row call's statistics): calls on one
+ *    plan must not overlap; different plans may be used from different threads.
  */
 #ifndef OT_SINKHORN_H
 #define OT_SINKHORN_H
