@@ -315,8 +315,8 @@ OT_API int ot_materialize_rows_lrcost(const float *cost1, const float *cost2, co
  * with every T_ij computed by the same float path as ot_materialize_rows, so
  * that keeping T_ij >= thr leaves every massful row non-empty. Massless rows
  * (a_i == 0) keep nothing and take no part. block_rows (> 0, or 0 = all rows)
- * only sets how many rows one launch covers (raised to a few waves of the GPU
- * when smaller); it never changes a result.
+ * only sets how many rows one launch covers (raised to sixteen waves of the
+ * GPU when smaller); it never changes a result.
  *  thr_out: host float (+inf if every row is massless).
  *  row_counts: device int64 [n] or NULL: kept entries per row.
  *  nnz_out, n_massless_out, argmin_out: host int64 or NULL (argmin_out: the
