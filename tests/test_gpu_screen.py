@@ -144,3 +144,35 @@ def test_screen_over_several_windows_of_chunks(ot):
     r, _ = p.marginal_residual()
     assert abs(r - (T.double().sum(1) - a.double()).abs().sum().item()) <= 1e-6
     p.close()
+
+
+def test_screen_at_workload_5_full_size(ot):
+    """Workload 5 at n = m = 2e6, in the launch shape the bench times, after 5
+    iterations: min_row's thr, argmin and counts against sampled materialized rows
+    (exactly: the argmin row's maximum is thr, every sampled massful row keeps
+    its count of entries >= thr), and the residual's part of single-row ranges
+    against the rows' float64 sums."""
+    import torch
+    from log_domain_sinkhorn_online_b200 import _binding as B
+    from log_domain_sinkhorn_online_b200 import workloads
+    w = workloads.w5()
+    x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).cuda() for v in (w.x, w.y, w.a, w.b))
+    p = ot.sinkhorn(x, y, a, b, eps=w.eps, scale=w.scale, n_iters=5)
+    mr = p.sparsify_min_row(block_rows=w.block_rows)
+    visited, total = p.row_pass_stats()
+    assert 0 < visited < 0.6 * total                      # the screen skips most tiles here
+    arg = mr["argmin"]
+    rows = np.unique(np.concatenate([[arg], np.linspace(0, w.n - 1, 63).astype(np.int64)]))
+    rt = torch.from_numpy(rows).cuda()
+    T = p.materialize_rows(rt)
+    rowmax = T.max(1).values
+    k = int(np.nonzero(rows == arg)[0][0])
+    assert float(rowmax[k]) == mr["thr"]
+    assert bool((rowmax >= mr["thr"]).all())
+    assert torch.equal((T >= mr["thr"]).sum(1), mr["counts"][rt])
+    s = torch.cuda.current_stream().cuda_stream
+    sums = T.double().sum(1).cpu().numpy()
+    for t, i in enumerate(rows[:16]):
+        part, _ = B.ot_marginal_residual_range(p.handle, int(i), int(i) + 1, 0, 0, s)
+        assert abs(part - abs(sums[t] - float(w.a[i]))) <= 1e-6 * float(w.a[i])
+    p.close()
