@@ -84,6 +84,11 @@ def _args():
                          "time per half-step and pair-updates/s (measured; totals of the long "
                          "configurations extrapolated and marked) and the oracle's rate on the "
                          "host cores")
+    ap.add_argument("--full-run", default=None, choices=["w3", "w4", "w5"],
+                    help="instead of the step: the configuration end to end as it is stated (its "
+                         "iterations or anneal, then the residual, min_row and, for w5, every block "
+                         "of its 65,536 rows), each part timed with CUDA events; prints its own "
+                         "JSON line")
     ap.add_argument("--sparse-workload", default="w4", choices=["w4", "w5"],
                     help="--sparse: uniform-vs-64-clusters (w4) or interleaved spirals (w5)")
     ap.add_argument("--sparse-block", type=int, default=0, choices=[0, 128, 256],
@@ -395,6 +400,62 @@ def run_configs(args):
                                        "sample": cb["sample"],
                                        "ms_per_half_step_extrapolated": float(w.n) * w.m / cb["value"] * 1e3}}
         print(json.dumps(line), flush=True)
+
+
+def run_full(args):
+    """One configuration end to end (measured, nothing extrapolated): the solve as the
+    configuration states it (w3: 500 iterations; w4: the anneal from eps 1.0 by 0.7
+    per stage of 20 iterations down to its eps; w5: 100 iterations with the max_cost
+    scale), then at the solved state the marginal residual, min_row with the
+    workload's row blocks and, where it lists rows (w5), their materialization block
+    by block into one reused buffer."""
+    import torch
+    import log_domain_sinkhorn_online_b200 as ot
+    dev = torch.device("cuda", 0)
+    w = _workload(args.full_run)
+    x, y, a, b = (torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (w.x, w.y, w.a, w.b))
+    kw = dict(eps=w.eps, scale=w.scale, n_iters=w.n_iters, timing=True)
+    if w.anneal:
+        kw.update(n_iters=w.anneal["iters_per_stage"], eps_init=w.anneal["eps_init"],
+                  eps_decay=w.anneal["decay"], iters_per_stage=w.anneal["iters_per_stage"])
+    stream = torch.cuda.current_stream()
+    clocks = Clocks(torch.cuda.current_device(), args.clock_ms)
+    clocks.start()
+    plan, solve_ms = _timed(lambda: ot.sinkhorn(x, y, a, b, **kw), stream)
+    info = plan.info
+    (r, c), res_ms = _timed(plan.marginal_residual, stream)
+    mr, mr_ms = _timed(lambda: plan.sparsify_min_row(block_rows=w.block_rows or 0), stream)
+    visited, total = plan.row_pass_stats()
+    out = {"metric": "configuration end to end", "config": {"workload": w.name, "n": w.n, "m": w.m, "d": w.d,
+                                                            "eps": w.eps, "scale": w.scale},
+           "solve": {"ms": solve_ms, "iterations": int(info.iterations), "stages": int(info.stages),
+                     "half_steps": int(info.half_steps), "loop_ms": info.loop_ms,
+                     "pair_updates_per_s": float(w.n) * w.m * info.half_steps / (info.loop_ms / 1e3),
+                     "final_residual": info.residual},
+           "marginal_residual": {"ms": res_ms, "row_l1": r, "col_l1": c},
+           "min_row": {"ms": mr_ms, "thr": mr["thr"], "nnz": mr["nnz"], "evaluated_share": visited / total
+                       if total else 1.0}}
+    total_ms = solve_ms + res_ms + mr_ms
+    if w.rows is not None:
+        k = w.block_rows or 4096
+        buf = torch.empty((k, w.m), dtype=torch.float32, device=dev)
+        rows = torch.from_numpy(np.ascontiguousarray(w.rows)).to(dev)
+        plan.materialize_rows(rows[:k], out=buf)  # load the kernel once, untimed
+
+        def blocks():
+            for s0 in range(0, rows.numel(), k):
+                r_ = rows[s0:s0 + k]
+                plan.materialize_rows(r_, out=buf[:r_.numel()])
+        _, rows_ms = _timed(blocks, stream)
+        out["materialize"] = {"rows": int(rows.numel()), "block_rows": k, "ms": rows_ms,
+                              "gb_written": rows.numel() * w.m * 4 / 1e9,
+                              "gb_per_s": rows.numel() * w.m * 4 / (rows_ms / 1e3) / 1e9}
+        total_ms += rows_ms
+        del buf
+    out["clocks"] = clocks.stop()
+    out["total_s"] = total_ms / 1e3
+    plan.close()
+    print(json.dumps(out), flush=True)
 
 
 def run_sparse(args, reps=10, dense_reps=2, tau=5e-3, emit=True):
@@ -769,6 +830,8 @@ def main():
         run_reference(args)
     elif args.rows:
         run_rows(args)
+    elif args.full_run:
+        run_full(args)
     elif args.lowrank:
         run_lowrank(args)
     elif args.sparse:
