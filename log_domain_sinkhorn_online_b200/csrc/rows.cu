@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
 enum { OP_MAX = 0, OP_COUNT = 1, OP_SUM = 2 };
 constexpr int kRpThreads = 256, kRpWarps = kRpThreads / 32, kRpR = 4, kRpChunk = kRpChunkC;
 constexpr int kRpRows = kRpWarps * kRpR;  // rows per block, d <= 3 (32)
-constexpr int kRgRows = 8;                // rows per block, generic d
+constexpr int kRgRows = 64;               // rows per block, d > 3
 constexpr int kRpWin = 8192;              // chunks screened at a time (one bit each)
 
 // Tile screen (d <= 3, R.csum set). The pass's rows come in Morton order
@@ -483,79 +483,120 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
     }
 }
 
-// Generic d (> 3): a block owns 8 rows (float64 data in shared memory) and its
-// 256 threads visit every column, each entry read from the global column table.
+// d > 3: register-tiled float64 dot products. A block owns 64 rows (A' = A +
+// kShift in sA, P transposed in sPt[q][r]) and streams the columns 64 at a
+// time (y' transposed into sYt[q][.], swizzled, B into sB[c]; dynamic shared
+// memory); thread t takes rows 4 (t / 16) + {0..3} and columns 4 (t % 16) +
+// {0..3} of the chunk and forms t = A' + B + sum_q P_q y'_q in the order of
+// plan_entry (so the same value bit for bit), then the entry and its
+// reduction: per (q, thread) two 16-byte loads of P (shared by the 16 threads
+// of the rows) and two of y' for 16 float64 FMAs. A row is reduced over the 16
+// threads of its half warp in a fixed order.
+constexpr int kWdCols = 64;
+
+int64_t wide_smem_bytes(int d) { return (int64_t)(d * (kRgRows + kWdCols) + kRgRows * 2 + kWdCols) * 8; }
+
 template <int OP>
-__global__ void __launch_bounds__(kRpThreads) rowpass_generic_kernel(RowPassArgs R) {
-    __shared__ double sA[kRgRows], sP[kRgRows][kMaxD];
-    __shared__ double sRed[kRpThreads / 32][kRgRows];
-    const int tid = threadIdx.x;
-    const int64_t r0 = R.row_begin + (int64_t)blockIdx.x * kRgRows;
+__global__ void __launch_bounds__(kRpThreads, 3) rowpass_wide_kernel(RowPassArgs R) {
+    extern __shared__ __align__(16) double wsm[];
     const int d = R.d;
+    double *sPt = wsm;                    // [d][64]
+    double *sYt = sPt + d * kRgRows;      // [d][64]
+    double *sA = sYt + d * kWdCols;       // [64]
+    double *sB = sA + kRgRows;            // [64]
+    double *sRed = sB + kWdCols;          // [64]
+    const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
+    const int64_t r0 = R.row_begin + (int64_t)blockIdx.x * kRgRows;
     if (tid < kRgRows) {
         const int64_t i = r0 + tid;
-        if (i < R.row_end)
-            load_row(R.pts, R.pot, i, d, R.o, R.prm->kappa, R.prm->c, &sA[tid], sP[tid]);
-        else
-            sA[tid] = -INFINITY;
+        double P[kMaxD];
+        double A = -INFINITY;
+        if (i < R.row_end) {
+            load_row(R.pts, R.pot, i, d, R.o, R.prm->kappa, R.prm->c, &A, P);
+        } else {
+            for (int q = 0; q < d; ++q) P[q] = 0.0;
+        }
+        sA[tid] = A;
+        for (int q = 0; q < d; ++q) sPt[q * kRgRows + tid] = P[q];
     }
-    __syncthreads();
-    float mx[kRgRows];
-    int cnt[kRgRows];
-    double sum[kRgRows];
-#pragma unroll
-    for (int r = 0; r < kRgRows; ++r) {
-        mx[r] = -1.0f;
-        cnt[r] = 0;
-        sum[r] = 0.0;
-    }
-    for (int64_t j0 = 0; j0 < R.cols; j0 += (int64_t)kRpThreads * 8) {
-        float part[kRgRows];
-#pragma unroll
-        for (int r = 0; r < kRgRows; ++r) part[r] = 0.0f;
-        for (int64_t j = j0 + tid; j < min(R.cols, j0 + (int64_t)kRpThreads * 8); j += kRpThreads) {
-            const double *col = R.dcol + j * (d + 1);
-#pragma unroll
-            for (int r = 0; r < kRgRows; ++r) {
-                const float t = plan_entry<0>(sA[r], sP[r], col, d);
-                if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
-                if (OP == OP_COUNT) cnt[r] += (t >= R.thr) ? 1 : 0;
-                if (OP == OP_SUM) part[r] += t;
+    float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // entries are >= 0, and a row has at least one
+    int cnt[4] = {0, 0, 0, 0};
+    double sum[4] = {0.0, 0.0, 0.0, 0.0};
+    const int DS = d + 1;
+    for (int64_t c0 = 0; c0 < R.cols; c0 += kWdCols) {
+        __syncthreads();  // the previous chunk is no longer read (and the rows are staged)
+        // warp w stages columns w, w + 8, ..., its lanes the column's record (coalesced);
+        // y'_q of column c sits at sYt[q][c ^ 4 (q % 16)] (a swizzle that keeps a
+        // thread's four columns together and spreads the lanes' stores over the banks)
+        for (int c = tid >> 5; c < kWdCols; c += kRpThreads / 32) {
+            const int64_t j = c0 + c;
+            for (int q = tid & 31; q < DS; q += 32) {
+                const double v = j < R.cols ? R.dcol[j * DS + q] : (q == d ? -INFINITY : 0.0);
+                if (q < d)
+                    sYt[q * kWdCols + (c ^ ((q & 15) << 2))] = v;
+                else
+                    sB[c] = v;
             }
         }
-        if (OP == OP_SUM) {
+        __syncthreads();
+        double acc[4][4];
 #pragma unroll
-            for (int r = 0; r < kRgRows; ++r) sum[r] += (double)part[r];
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[r][c] = sA[4 * rg + r] + sB[4 * cg + c];
+#pragma unroll 2
+        for (int q = 0; q < d; ++q) {
+            const double *pq = &sPt[q * kRgRows + 4 * rg];
+            const double2 p0 = *reinterpret_cast<const double2 *>(pq);
+            const double2 p1 = *reinterpret_cast<const double2 *>(pq + 2);
+            const double *yq = &sYt[q * kWdCols + ((4 * cg) ^ ((q & 15) << 2))];
+            const double2 y0 = *reinterpret_cast<const double2 *>(yq);
+            const double2 y1 = *reinterpret_cast<const double2 *>(yq + 2);
+            const double pr[4] = {p0.x, p0.y, p1.x, p1.y}, yc[4] = {y0.x, y0.y, y1.x, y1.y};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = fma(pr[r], yc[c], acc[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            float part = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float t = exp2_shifted(acc[r][c]);
+                if (OP == OP_MAX) mx[r] = fmaxf(mx[r], t);
+                if (OP == OP_COUNT) cnt[r] += (c0 + 4 * cg + c < R.cols && t >= R.thr) ? 1 : 0;
+                if (OP == OP_SUM) part += t;
+            }
+            if (OP == OP_SUM) sum[r] += (double)part;
         }
     }
+    // each row over the 16 threads of its half warp, in a fixed order
 #pragma unroll
-    for (int r = 0; r < kRgRows; ++r) {
+    for (int r = 0; r < 4; ++r) {
         double v = OP == OP_SUM ? sum[r] : OP == OP_COUNT ? (double)cnt[r] : (double)mx[r];
-        for (int off = 16; off > 0; off >>= 1) {
+        for (int off = 8; off > 0; off >>= 1) {
             const double o2 = __shfl_xor_sync(0xffffffffu, v, off);
             v = OP == OP_MAX ? fmax(v, o2) : v + o2;
         }
-        if ((tid & 31) == 0) sRed[tid >> 5][r] = v;
-    }
-    __syncthreads();
-    if (tid < kRgRows) {
-        double v = sRed[0][tid];
-        for (int w = 1; w < kRpThreads / 32; ++w) v = OP == OP_MAX ? fmax(v, sRed[w][tid]) : v + sRed[w][tid];
-        const int64_t i = r0 + tid;
-        if (i < R.row_end) {
-            const float wi = R.w[i];
-            if (OP == OP_MAX) R.rowmax[i] = (float)v;
-            if (OP == OP_COUNT) R.counts[i] = wi > 0.0f ? (int64_t)v : 0;
-            if (OP == OP_SUM) sRed[0][tid] = fabs(v - (double)wi);
-        } else if (OP == OP_SUM) {
-            sRed[0][tid] = 0.0;
+        if (cg == 0) {
+            const int rr = 4 * rg + r;
+            const int64_t i = r0 + rr;
+            double res = 0.0;
+            if (i < R.row_end) {
+                const float wi = R.w[i];
+                if (OP == OP_MAX) R.rowmax[i] = (float)v;
+                if (OP == OP_COUNT) R.counts[i] = wi > 0.0f ? (int64_t)v : 0;
+                if (OP == OP_SUM) res = fabs(v - (double)wi);
+            }
+            sRed[rr] = res;
         }
     }
     if (OP == OP_SUM) {
         __syncthreads();
         if (tid == 0) {
             double t = 0.0;
-            for (int r = 0; r < kRgRows; ++r) t += sRed[0][r];
+            for (int r = 0; r < kRgRows; ++r) t += sRed[r];
             R.part[blockIdx.x] = t;
         }
     }
@@ -959,7 +1000,15 @@ static void rowpass_dispatch(const RowPassArgs &R, int64_t rows, cudaStream_t s)
         case 1: rowpass_kernel<1, OP><<<grid, kRpThreads, 0, s>>>(R); break;
         case 2: rowpass_kernel<2, OP><<<grid, kRpThreads, 0, s>>>(R); break;
         case 3: rowpass_kernel<3, OP><<<grid, kRpThreads, 0, s>>>(R); break;
-        default: rowpass_generic_kernel<OP><<<grid, kRpThreads, 0, s>>>(R); break;
+        default: {
+            // up to 50 KB of shared memory at d = 64: the opt-in is per device, so every
+            // launch sets it (a host-side call)
+            if (cudaFuncSetAttribute(rowpass_wide_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)wide_smem_bytes(kMaxD)) != cudaSuccess)
+                return;  // the caller's cudaGetLastError reports it
+            rowpass_wide_kernel<OP><<<grid, kRpThreads, (size_t)wide_smem_bytes(R.d), s>>>(R);
+            break;
+        }
     }
 }
 
