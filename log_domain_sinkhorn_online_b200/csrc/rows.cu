@@ -245,6 +245,99 @@ __global__ void __launch_bounds__(kMtThreads, 4) materialize_kernel(MatArgs M) {
     }
 }
 
+// Materializer for d > 3: the float64 exponent's dot product as a register-
+// tiled product, as in rowpass_wide_kernel (its comment has the layout): a
+// block takes 64 entries of the row list and a range of kMwChunks chunks of 64
+// columns; each thread forms a 4 x 4 tile of entries in the order of
+// plan_entry (the same values bit for bit) and stores 4 consecutive columns of
+// each of its rows (one float4 streaming store when the row is aligned).
+constexpr int kMwRows = 64, kMwCols = 64, kMwChunks = 16;
+
+int64_t matwide_smem_bytes(int d) { return (int64_t)(d * (kMwRows + kMwCols) + kMwRows * 3 + kMwCols) * 8; }
+
+__global__ void __launch_bounds__(256, 3) materialize_wide_kernel(MatArgs M) {
+    extern __shared__ __align__(16) double msm[];
+    const int d = M.d;
+    double *sPt = msm;                    // [d][64]
+    double *sYt = sPt + d * kMwRows;      // [d][64]
+    double *sA = sYt + d * kMwCols;       // [64]
+    double *sB = sA + kMwRows;            // [64]
+    int64_t *sRow = reinterpret_cast<int64_t *>(sB + kMwCols);  // [64] output row, -1: skip
+    const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
+    const int64_t t0 = (int64_t)blockIdx.y * kMwRows;
+    if (tid < kMwRows) {
+        const int64_t t = t0 + tid;
+        double P[kMaxD];
+        double A = -INFINITY;
+        int64_t out_row = -1;
+        if (t < M.k) {
+            const int64_t i = M.row_idx[t];
+            if (i >= 0 && i < M.n) {
+                load_row(M.x, M.f, i, d, M.o, M.prm->kappa, M.prm->c, &A, P);
+                out_row = t;
+            } else {
+                atomicExch(M.bad, 1);
+            }
+        }
+        if (out_row < 0)
+            for (int q = 0; q < d; ++q) P[q] = 0.0;
+        sA[tid] = A;
+        sRow[tid] = out_row;
+        for (int q = 0; q < d; ++q) sPt[q * kMwRows + tid] = P[q];
+    }
+    const int DS = d + 1;
+    const int64_t cbeg = (int64_t)blockIdx.x * kMwChunks * kMwCols;
+    const int64_t cend = min(M.m, cbeg + (int64_t)kMwChunks * kMwCols);
+    for (int64_t c0 = cbeg; c0 < cend; c0 += kMwCols) {
+        __syncthreads();  // the previous chunk is no longer read (and the rows are staged)
+        for (int c = tid >> 5; c < kMwCols; c += 8) {
+            const int64_t j = c0 + c;
+            for (int q = tid & 31; q < DS; q += 32) {
+                const double v = j < M.m ? M.dcol[j * DS + q] : (q == d ? -INFINITY : 0.0);
+                if (q < d)
+                    sYt[q * kMwCols + (c ^ ((q & 15) << 2))] = v;
+                else
+                    sB[c] = v;
+            }
+        }
+        __syncthreads();
+        double acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[r][c] = sA[4 * rg + r] + sB[4 * cg + c];
+#pragma unroll 2
+        for (int q = 0; q < d; ++q) {
+            const double *pq = &sPt[q * kMwRows + 4 * rg];
+            const double2 p0 = *reinterpret_cast<const double2 *>(pq);
+            const double2 p1 = *reinterpret_cast<const double2 *>(pq + 2);
+            const double *yq = &sYt[q * kMwCols + ((4 * cg) ^ ((q & 15) << 2))];
+            const double2 y0 = *reinterpret_cast<const double2 *>(yq);
+            const double2 y1 = *reinterpret_cast<const double2 *>(yq + 2);
+            const double pr[4] = {p0.x, p0.y, p1.x, p1.y}, yc[4] = {y0.x, y0.y, y1.x, y1.y};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = fma(pr[r], yc[c], acc[r][c]);
+        }
+        const int64_t j0 = c0 + 4 * cg;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int64_t orow = sRow[4 * rg + r];
+            if (orow < 0 || j0 >= M.m) continue;
+            float t[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) t[c] = exp2_shifted(acc[r][c]);
+            float *dst = M.out + orow * M.m + j0;
+            if (M.vec && j0 + 4 <= M.m) {
+                __stcs(reinterpret_cast<float4 *>(dst), make_float4(t[0], t[1], t[2], t[3]));
+            } else {
+                for (int c = 0; c < 4 && j0 + c < M.m; ++c) __stcs(dst + c, t[c]);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------- row-complete passes
 // A pass visits every entry of a range of rows and reduces each row:
 //   OP_MAX:   rowmax[i] = max_j T_ij                       (min_row, pass A)
@@ -974,7 +1067,7 @@ cudaError_t launch_perm_from_keys(const unsigned long long *keys, int64_t cnt, i
 cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s) {
     const int64_t col_blocks = (M.m + kMtThreads * 4 - 1) / (kMtThreads * 4);
     // at most 65535 row ranges per launch: split long row lists
-    const int64_t max_rows = (int64_t)65535 * kMtRowsPerBlock;
+    const int64_t max_rows = (int64_t)65535 * (M.d > 3 ? kMwRows : kMtRowsPerBlock);
     for (int64_t r = 0; r < M.k; r += max_rows) {
         MatArgs A = M;
         A.row_idx = M.row_idx + r;
@@ -985,7 +1078,17 @@ cudaError_t launch_materialize(const MatArgs &M, cudaStream_t s) {
             case 1: materialize_kernel<1><<<grid, kMtThreads, 0, s>>>(A); break;
             case 2: materialize_kernel<2><<<grid, kMtThreads, 0, s>>>(A); break;
             case 3: materialize_kernel<3><<<grid, kMtThreads, 0, s>>>(A); break;
-            default: materialize_kernel<0><<<grid, kMtThreads, 0, s>>>(A); break;
+            default: {
+                // d > 3: 64 list entries x 16 chunks of 64 columns per block (up to 66 KB of
+                // shared memory at d = 64: the opt-in is per device, so every launch sets it)
+                if (cudaFuncSetAttribute(materialize_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)matwide_smem_bytes(kMaxD)) != cudaSuccess)
+                    return cudaGetLastError();
+                const int64_t wcols = (M.m + (int64_t)kMwChunks * kMwCols - 1) / ((int64_t)kMwChunks * kMwCols);
+                dim3 wgrid((unsigned)wcols, (unsigned)((A.k + kMwRows - 1) / kMwRows));
+                materialize_wide_kernel<<<wgrid, 256, (size_t)matwide_smem_bytes(M.d), s>>>(A);
+                break;
+            }
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -176,3 +176,36 @@ def test_screen_at_workload_5_full_size(ot):
         part, _ = B.ot_marginal_residual_range(p.handle, int(i), int(i) + 1, 0, 0, s)
         assert abs(part - abs(sums[t] - float(w.a[i]))) <= 1e-6 * float(w.a[i])
     p.close()
+
+
+@pytest.mark.parametrize("d", [5, 17, 50, 64])
+def test_wide_passes_equal_the_materialized_plan(ot, d):
+    """d > 3: the register-tiled row passes and the register-tiled materializer form
+    every entry in the same order, so min_row's thr, argmin and counts equal those of
+    the materialized rows bit for bit (ragged sizes: rows and columns not multiples
+    of the 64-row / 64-column tiles)."""
+    import torch
+    rng = np.random.default_rng(100 + d)
+    n, m = 333, 1201
+    x = torch.from_numpy(rng.random((n, d), dtype=np.float32)).cuda()
+    y = torch.from_numpy((rng.random((m, d)) * 1.2).astype(np.float32)).cuda()
+    a = rng.random(n).astype(np.float32) + 0.2
+    a[::41] = 0.0
+    a = torch.from_numpy((a / a.sum()).astype(np.float32)).cuda()
+    b = torch.full((m,), 1.0 / m, device="cuda")
+    p = ot.sinkhorn(x, y, a, b, eps=0.05, scale="mean", n_iters=6)
+    T = p.materialize_rows(torch.arange(n, device="cuda"))
+    Tsub = p.materialize_rows(torch.tensor([n - 1, 0, 200, 200], device="cuda"))
+    assert torch.equal(Tsub, T[[n - 1, 0, 200, 200]])      # row lists in any order, repeats
+    massful = a > 0
+    rowmax = T.max(1).values
+    thr = rowmax[massful].min()
+    mr = p.sparsify_min_row(block_rows=100)
+    assert mr["thr"] == float(thr)
+    assert mr["argmin"] == int(torch.nonzero(massful & (rowmax == thr))[0])
+    assert torch.equal(mr["counts"], torch.where(massful, (T >= thr).sum(1), torch.zeros_like(mr["counts"])))
+    r, c = p.marginal_residual()
+    Td = T.double()
+    assert abs(r - (Td.sum(1) - a.double()).abs().sum().item()) <= 1e-6
+    assert abs(c - (Td.sum(0) - b.double()).abs().sum().item()) <= 1e-6
+    p.close()
