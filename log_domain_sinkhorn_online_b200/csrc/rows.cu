@@ -579,25 +579,29 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_kernel(RowPassArgs R) {
 // d > 3: register-tiled float64 dot products. A block owns 64 rows (A' = A +
 // kShift in sA, P transposed in sPt[q][r]) and streams the columns 64 at a
 // time (y' transposed into sYt[q][.], swizzled, B into sB[c]; dynamic shared
-// memory); thread t takes rows 4 (t / 16) + {0..3} and columns 4 (t % 16) +
-// {0..3} of the chunk and forms t = A' + B + sum_q P_q y'_q in the order of
-// plan_entry (so the same value bit for bit), then the entry and its
-// reduction: per (q, thread) two 16-byte loads of P (shared by the 16 threads
-// of the rows) and two of y' for 16 float64 FMAs. A row is reduced over the 16
-// threads of its half warp in a fixed order.
+// memory, two chunk buffers: the next chunk's records are copied straight to
+// shared memory with cp.async while the current one is computed); thread t
+// takes rows 4 (t / 16) + {0..3} and columns 4 (t % 16) + {0..3} of the chunk
+// and forms t = A' + B + sum_q P_q y'_q in the order of plan_entry (so the
+// same value bit for bit), then the entry and its reduction: per (q, thread)
+// two 16-byte loads of P (shared by the 16 threads of the rows) and two of y'
+// for 16 float64 FMAs. A row is reduced over the 16 threads of its half warp in
+// a fixed order. 2 blocks per SM (120 registers; measured at workload 3: the
+// residual 47 -> 40 ms and min_row 52 -> 41 ms against a single chunk buffer
+// at 3 blocks per SM).
 constexpr int kWdCols = 64;
 
-int64_t wide_smem_bytes(int d) { return (int64_t)(d * (kRgRows + kWdCols) + kRgRows * 2 + kWdCols) * 8; }
+int64_t wide_smem_bytes(int d) { return (int64_t)(d * (kRgRows + 2 * kWdCols) + kRgRows * 2 + 2 * kWdCols) * 8; }
 
 template <int OP>
-__global__ void __launch_bounds__(kRpThreads, 3) rowpass_wide_kernel(RowPassArgs R) {
+__global__ void __launch_bounds__(kRpThreads, 2) rowpass_wide_kernel(RowPassArgs R) {
     extern __shared__ __align__(16) double wsm[];
     const int d = R.d;
     double *sPt = wsm;                    // [d][64]
-    double *sYt = sPt + d * kRgRows;      // [d][64]
-    double *sA = sYt + d * kWdCols;       // [64]
-    double *sB = sA + kRgRows;            // [64]
-    double *sRed = sB + kWdCols;          // [64]
+    double *sYt2 = sPt + d * kRgRows;     // [2][d][64]
+    double *sA = sYt2 + 2 * d * kWdCols;  // [64]
+    double *sB2 = sA + kRgRows;           // [2][64]
+    double *sRed = sB2 + 2 * kWdCols;     // [64]
     const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
     const int64_t r0 = R.row_begin + (int64_t)blockIdx.x * kRgRows;
     if (tid < kRgRows) {
@@ -612,32 +616,39 @@ __global__ void __launch_bounds__(kRpThreads, 3) rowpass_wide_kernel(RowPassArgs
         sA[tid] = A;
         for (int q = 0; q < d; ++q) sPt[q * kRgRows + tid] = P[q];
     }
-    float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // entries are >= 0, and a row has at least one
+    float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     int cnt[4] = {0, 0, 0, 0};
     double sum[4] = {0.0, 0.0, 0.0, 0.0};
     const int DS = d + 1;
-    for (int64_t c0 = 0; c0 < R.cols; c0 += kWdCols) {
-        __syncthreads();  // the previous chunk is no longer read (and the rows are staged)
-        // warp w stages columns w, w + 8, ..., its lanes the column's record (coalesced);
-        // y'_q of column c sits at sYt[q][c ^ 4 (q % 16)] (a swizzle that keeps a
-        // thread's four columns together and spreads the lanes' stores over the banks)
+    auto stage = [&](int64_t c0, int buf) {
+        double *sYt = sYt2 + buf * d * kWdCols, *sB = sB2 + buf * kWdCols;
         for (int c = tid >> 5; c < kWdCols; c += kRpThreads / 32) {
             const int64_t j = c0 + c;
             for (int q = tid & 31; q < DS; q += 32) {
-                const double v = j < R.cols ? R.dcol[j * DS + q] : (q == d ? -INFINITY : 0.0);
-                if (q < d)
-                    sYt[q * kWdCols + (c ^ ((q & 15) << 2))] = v;
-                else
-                    sB[c] = v;
+                double *dst = q < d ? &sYt[q * kWdCols + (c ^ ((q & 15) << 2))] : &sB[c];
+                if (j < R.cols) {
+                    const unsigned sa = (unsigned)__cvta_generic_to_shared(dst);
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(R.dcol + j * DS + q) : "memory");
+                } else {
+                    *dst = q == d ? -INFINITY : 0.0;
+                }
             }
         }
-        __syncthreads();
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    stage(0, 0);
+    int buf = 0;
+    for (int64_t c0 = 0; c0 < R.cols; c0 += kWdCols, buf ^= 1) {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();  // chunk c0 is staged, and the other buffer is no longer read
+        if (c0 + kWdCols < R.cols) stage(c0 + kWdCols, buf ^ 1);
+        const double *sYt = sYt2 + buf * d * kWdCols, *sB = sB2 + buf * kWdCols;
         double acc[4][4];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[r][c] = sA[4 * rg + r] + sB[4 * cg + c];
-#pragma unroll 2
+#pragma unroll 4
         for (int q = 0; q < d; ++q) {
             const double *pq = &sPt[q * kRgRows + 4 * rg];
             const double2 p0 = *reinterpret_cast<const double2 *>(pq);
